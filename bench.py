@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA layer on B200.
+
+One step = one chunkwise forward (gate cumsum, intra-chunk A, UT transform,
+state scan, intra-chunk output, final state) over the prefill workload
+(B=2, H=16, T=4096, d_k=d_v=128, bf16 q/k/v, fp32 state, chunk 64), inputs
+resident in HBM.  Two input sets of ~200 MB each (larger than the 126 MB L2)
+alternate between steps, so no step starts with its inputs in L2.  The decode
+step (256 sequences x 32 heads, 64 consecutive tokens) is timed in the same
+run and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own copy of the
+workload with its own seed (weak scaling, no data-path collective); the time is
+the max over ranks.  --impl reference times the fp64 CPU oracle on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA chunk-fwd tokens/s & TFLOP/s (% roofline); decode-step state GB/s on 1 B200"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- work model
+def bytes_per_token_head(dk, dv, elem):
+    """Algorithmic HBM bytes per (token, head): q, k, v in, o out (elem bytes
+    each), log alpha (fp32 per key channel) and beta (fp32) in."""
+    return elem * (2 * dk + 2 * dv) + 4 * dk + 4
+
+
+def flops_per_token_head(dk, dv, C=64):
+    """Algorithmic FLOPs per (token, head) of the chunk forward, triangles at
+    half: A and P ((C-1) and (C+1) pairs of d_k), U-like 2C d_v, the four
+    state products 6 d_k d_v, the UT transform C^2/3."""
+    return (2 * (C - 1) + (C + 1)) * dk + 2 * C * dv + 6 * dk * dv + C * C / 3.0
+
+
+def chunk_work(B, T, H, dk, dv, elem=2, state_in=True, state_out=True):
+    th = B * T * H
+    nbytes = th * bytes_per_token_head(dk, dv, elem)
+    nbytes += (int(state_in) + int(state_out)) * B * H * dk * dv * 4
+    return nbytes, th * flops_per_token_head(dk, dv)
+
+
+def decode_state_bytes(N, H, dk, dv):
+    return 2 * N * H * dk * dv * 4
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (the timing rule)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device=None):
+    if world > 1:
+        if device is not None and device.type == "cuda":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
+    FIELDS = ("index,timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(getattr(self, "out", ""))) if len(r) >= 10]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
+        power = [num(r[4]) for r in rows if num(r[4]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].strip().lower() == "active"})
+        # "under load": samples at or above the median power draw
+        load = sm
+        if power and len(power) == len(sm):
+            cut = statistics.median(power)
+            load = [s for s, p in zip(sm, power) if p >= cut] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: p[k] for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_133_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, or None
+    when the kernel sources changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel_key)
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def event_pairs(n):
+    return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import gated_delta_rule_133_b200 as kda
+    from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    init_dist(world, "nccl")
+    w = WORKLOADS["prefill"]
+    stream = torch.cuda.current_stream(device)
+
+    nsets = 2
+    sets = [make_inputs(w, device, seed=w.seed + 1000 * rank + i) for i in range(nsets)]
+    outs = [(torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.bfloat16, device=device),
+             torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)) for _ in range(nsets)]
+    nbytes, nflops = chunk_work(w.B, w.T, w.H, w.dk, w.dv)
+    set_bytes = sum(t.numel() * t.element_size() for t in sets[0].values() if t is not None)
+
+    def step(i):
+        d, (o, s) = sets[i % nsets], outs[i % nsets]
+        kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], d["initial_state"],
+                          o=o, final_state=s, stream=stream)
+
+    sampler = ClockSampler(device.index)
+    with sampler:
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize(device)
+        kda.kda_check()
+        ev = event_pairs(args.steps)
+        barrier(world, device)
+        torch.cuda.synchronize(device)
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(world, device)
+        kda.kda_check()
+        elapsed = reduce_max(t_start.elapsed_time(t_end) / 1e3, world, device)
+        launch_s = statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3
+
+        # ---- decode: 64 consecutive steps over 256 x 32 fp32 states
+        dec = run_decode(kda, device, stream, world, rank, max(1, args.warmup))
+
+        # ---- end to end through the public API from pinned host buffers
+        e2e = run_e2e(kda, sets[0], w, device, stream, world, steps=max(1, min(args.steps, 5)))
+
+    clocks = sampler.summary()
+    tokens = w.B * w.T * world
+    value = tokens * args.steps / elapsed
+    pk, pk_kind = peaks()
+    achieved = nbytes / launch_s / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"prefill: B={w.B} H={w.H} T={w.T} d_k={w.dk} d_v={w.dv} chunk={w.chunk}, "
+                               "bf16 q/k/v, fp32 state, random fp32 initial state",
+                   "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {nsets} input sets of {set_bytes / 1e6:.0f} MB alternate"},
+        "tflops": nflops * world * args.steps / elapsed / 1e12,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic("chunk_fwd_prefill"),
+                     "peak_kind": f"{pk_kind} copy bandwidth",
+                     "bytes_per_launch": nbytes, "launch_ms": launch_s * 1e3,
+                     "tensor_frac": nflops / launch_s / 1e12 / pk["bf16_tflops"]},
+        "decode": dec,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    return line, rank
+
+
+def run_decode(kda, device, stream, world, rank, warmup):
+    from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
+    w = WORKLOADS["decode"]
+    x = make_inputs(w, device, seed=w.seed + 1000 * rank)
+    state = x["initial_state"].clone()
+    o = torch.empty(w.B, w.H, w.dv, dtype=torch.bfloat16, device=device)
+
+    def one(s):
+        kda.kda_recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["beta"][s], x["log_alpha"][s], state,
+                               o=o, stream=stream)
+
+    for s in range(warmup):
+        one(s % w.T)
+    torch.cuda.synchronize(device)
+    state.copy_(x["initial_state"])
+    ev = event_pairs(w.T)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    for s in range(w.T):
+        ev[s][0].record(stream)
+        one(s)
+        ev[s][1].record(stream)
+    torch.cuda.synchronize(device)
+    per = [a.elapsed_time(b) / 1e3 for a, b in ev]
+    total = reduce_max(ev[0][0].elapsed_time(ev[-1][1]) / 1e3, world, device)
+    nbytes = decode_state_bytes(w.B, w.H, w.dk, w.dv)
+    pk, kind = peaks()
+    gbs = nbytes * world * w.T / total / 1e9
+    per_launch = nbytes / statistics.mean(per) / 1e9
+    return {"workload": f"decode: {w.B} sequences x H={w.H}, d_k=d_v={w.dk}, fp32 state "
+                        f"({w.B * w.H * w.dk * w.dv * 4 / 2**20:.0f} MiB), {w.T} consecutive steps",
+            "value": gbs, "unit": "GB/s (state read + write)", "us_per_step": total / w.T * 1e6,
+            "roofline": {"bound": "hbm", "achieved": per_launch, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": per_launch / pk["hbm_gbs"], "traffic": recorded_traffic("decode_step"),
+                         "peak_kind": f"{kind} copy bandwidth"},
+            "gpu_launches": w.T}
+
+
+def run_e2e(kda, d, w, device, stream, world, steps):
+    """Same metric through the public API with pinned host buffers: every step
+    copies its inputs host->device and reads o and the final state back."""
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in d.items()}
+    dev = {k: (None if v is None else torch.empty_like(v, device=device)) for k, v in d.items()}
+    o_h = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.bfloat16).pin_memory()
+    s_h = torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
+
+    def one():
+        for k, v in host.items():
+            if v is not None:
+                dev[k].copy_(v, non_blocking=True)
+        o, s = kda.kda_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_alpha"],
+                                 dev["initial_state"], stream=stream)
+        o_h.copy_(o, non_blocking=True)
+        s_h.copy_(s, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    t = reduce_max(a.elapsed_time(b) / 1e3, world, device)
+    return {"value": w.B * w.T * world * steps / t, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_sample(heads_max=16):
+    """Times the fp64 oracle on the prefill workload (all tokens of both
+    sequences for up to `heads_max` heads; all 16 by default, about 1 s on 8
+    cores).  Returns the equivalent whole-workload tokens/s, the threads used
+    and the sample description."""
+    import numpy as np
+    import oracle
+    from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
+    w = WORKLOADS["prefill"]
+    d = make_inputs(w, "cpu")
+    cores = os.cpu_count() or 1
+    heads = max(1, min(heads_max, w.H))
+    f = lambda x: x[:, :, :heads].to(torch.float64).numpy().reshape(w.B * w.T, heads, *x.shape[3:])
+    q, k, v, la = f(d["q"]), f(d["k"]), f(d["v"]), f(d["log_alpha"])
+    beta = d["beta"][:, :, :heads].to(torch.float64).numpy().reshape(w.B * w.T, heads)
+    s0 = d["initial_state"][:, :heads].to(torch.float64).numpy()
+    cu = np.array([0, w.T, 2 * w.T])
+    t0 = time.perf_counter()
+    oracle.recurrence(q, k, v, beta, la, cu, s0, nthreads=cores)
+    dt = time.perf_counter() - t0
+    full_time = dt * w.H / heads
+    return {"value": w.B * w.T / full_time, "unit": "tokens/s", "cores": min(cores, w.B * heads),
+            "kind": "oracle",
+            "sample": f"prefill workload, {heads} of {w.H} heads x both sequences x all {w.T} tokens "
+                      f"({dt:.1f} s), scaled to all heads"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    vals = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        info = oracle_sample()
+        if i >= args.warmup:
+            vals.append(info["value"])
+    value = statistics.mean(vals) if vals else info["value"]
+    from gated_delta_rule_133_b200.inputs import WORKLOADS
+    w = WORKLOADS["prefill"]
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": w.B * w.T / value * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"prefill: B={w.B} H={w.H} T={w.T} d_k={w.dk} d_v={w.dv} (fp64 CPU oracle)"},
+            "cpu_baseline": {**info, "value": value},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    line, rank = run_ours(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample()
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

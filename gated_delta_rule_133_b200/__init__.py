@@ -1,0 +1,133 @@
+"""KDA / gated-DeltaNet linear-attention layer for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/kda.h`` (``libkda.so``).  These
+functions only marshal arguments (check devices, dtypes and shapes, allocate
+outputs with PyTorch, pass pointers and the current CUDA stream); every step of
+the computation runs in the library's CUDA kernels.  There is no CPU path.
+
+    o, S_T = kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state)
+    o, S_N = kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state)
+    o      = kda_recurrent_step(q, k, v, beta, log_alpha, state)   # state updated in place
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+from ._lib import KdaError
+
+__all__ = ["kda_chunk_fwd", "kda_varlen_fwd", "kda_recurrent_step", "kda_check", "KdaError"]
+
+_DTYPES = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check(t, name, shape, dtype, device):
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final_state=None,
+                  output_final_state=True, chunk=64, stream=None):
+    """Chunkwise forward over equal-length sequences.
+
+    q, k [B, T, H, dk] and v [B, T, H, dv] (bf16 or fp32); beta [B, T, H] and
+    log_alpha [B, T, H, dk] fp32; initial_state [B, H, dk, dv] fp32 or None.
+    Returns (o [B, T, H, dv], final_state [B, H, dk, dv] or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for t, n, s, d in ((q, "q", (B, T, H, dk), dt), (k, "k", (B, T, H, dk), dt),
+                       (v, "v", (B, T, H, dv), dt), (beta, "beta", (B, T, H), torch.float32),
+                       (log_alpha, "log_alpha", (B, T, H, dk), torch.float32)):
+        _check(t, n, s, d, dev)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=dt, device=dev)
+    _check(o, "o", (B, T, H, dv), dt, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _check(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
+    _lib.call("kda_chunk_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
+              _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk,
+              _DTYPES[dt], _stream(stream))
+    return o, final_state
+
+
+def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, o=None,
+                   final_state=None, output_final_state=True, chunk=64, stream=None):
+    """Chunkwise forward over N packed variable-length sequences.
+
+    q, k [T, H, dk], v [T, H, dv]; beta [T, H]; log_alpha [T, H, dk];
+    cu_seqlens [N + 1] int32 on the device; initial_state [N, H, dk, dv] or None.
+    Returns (o [T, H, dv], final_state [N, H, dk, dv] or None)."""
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.shape[0] - 1
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for t, n, s, d in ((q, "q", (T, H, dk), dt), (k, "k", (T, H, dk), dt), (v, "v", (T, H, dv), dt),
+                       (beta, "beta", (T, H), torch.float32),
+                       (log_alpha, "log_alpha", (T, H, dk), torch.float32),
+                       (cu_seqlens, "cu_seqlens", (N + 1,), torch.int32)):
+        _check(t, n, s, d, dev)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (N, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=dt, device=dev)
+    _check(o, "o", (T, H, dv), dt, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _check(final_state, "final_state", (N, H, dk, dv), torch.float32, dev)
+    _lib.call("kda_varlen_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
+              _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(o), _ptr(final_state), T, H, dk, dv,
+              chunk, _DTYPES[dt], _stream(stream))
+    return o, final_state
+
+
+def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, stream=None):
+    """One decode step: q, k [N, H, dk], v [N, H, dv], beta [N, H],
+    log_alpha [N, H, dk]; state [N, H, dk, dv] fp32 is updated in place.
+    Returns o [N, H, dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for t, n, s, d in ((q, "q", (N, H, dk), dt), (k, "k", (N, H, dk), dt), (v, "v", (N, H, dv), dt),
+                       (beta, "beta", (N, H), torch.float32),
+                       (log_alpha, "log_alpha", (N, H, dk), torch.float32),
+                       (state, "state", (N, H, dk, dv), torch.float32)):
+        _check(t, n, s, d, dev)
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=dt, device=dev)
+    _check(o, "o", (N, H, dv), dt, dev)
+    _lib.call("kda_recurrent_step", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
+              _ptr(state), _ptr(o), N, H, dk, dv, _DTYPES[dt], _stream(stream))
+    return o
+
+
+def kda_check(stream=None):
+    """Synchronise the stream and raise if a kernel reported a device-side timeout."""
+    _lib.call("kda_check", _stream(stream))

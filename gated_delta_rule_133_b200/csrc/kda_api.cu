@@ -1,0 +1,122 @@
+// C ABI of the KDA library: argument validation, path selection, status codes.
+// Declarations and the contract of every entry point are in include/kda.h.
+#include <cuda_runtime.h>
+
+#include "kda_chunk.cuh"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_d(int d) { return d == 64 || d == 128; }
+
+kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+// Shared checks of the forward entry points.
+kda_status check_fwd(const void* q, const void* k, const void* v, const float* beta,
+                     const float* log_alpha, const float* s0, const void* o, const float* sT,
+                     long long tokens, int H, int dk, int dv, int chunk, kda_dtype dtype)
+{
+    if (H <= 0 || dk <= 0 || dv <= 0 || tokens < 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (tokens > 0) {
+        if (!q || !k || !v || !beta || !log_alpha || !o) return KDA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) ||
+            !aligned16(log_alpha) || !aligned16(o))
+            return KDA_ERR_INVALID_ARG;
+    }
+    if ((s0 && !aligned16(s0)) || (sT && !aligned16(sT))) return KDA_ERR_INVALID_ARG;
+    if (chunk != 64 || !supported_d(dk) || !supported_d(dv)) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+// Writes final = initial (or zeros) for sequences that have no tokens at all.
+kda_status copy_state(const float* s0, float* sT, size_t elems, cudaStream_t s)
+{
+    if (!sT || elems == 0) return KDA_OK;
+    if (s0 == sT) return KDA_OK;
+    if (s0) return from_cuda(cudaMemcpyAsync(sT, s0, elems * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    return from_cuda(cudaMemsetAsync(sT, 0, elems * sizeof(float), s));
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
+                         const float* log_alpha, const float* initial_state, void* o,
+                         float* final_state, int B, int T, int H, int dk, int dv, int chunk,
+                         kda_dtype dtype, void* stream)
+{
+    if (B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    const long long tokens = (long long)B * T;
+    kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, tokens, H,
+                              dk, dv, chunk, dtype);
+    if (st != KDA_OK) return st;
+    if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tokens == 0) return copy_state(initial_state, final_state, (size_t)B * H * dk * dv, s);
+    return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, initial_state, o, final_state,
+                                         nullptr, B, T, H, dk, dv, dtype, s));
+}
+
+kda_status kda_varlen_fwd(const void* q, const void* k, const void* v, const float* beta,
+                          const float* log_alpha, const int32_t* cu_seqlens, int N,
+                          const float* initial_state, void* o, float* final_state, int T, int H,
+                          int dk, int dv, int chunk, kda_dtype dtype, void* stream)
+{
+    if (N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, T, H, dk,
+                              dv, chunk, dtype);
+    if (st != KDA_OK) return st;
+    if (N == 0) return T == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
+    if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) return copy_state(initial_state, final_state, (size_t)N * H * dk * dv, s);
+    return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, initial_state, o, final_state,
+                                         cu_seqlens, N, T, H, dk, dv, dtype, s));
+}
+
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* beta,
+                              const float* log_alpha, float* state, void* o, int N, int H, int dk,
+                              int dv, kda_dtype dtype, void* stream)
+{
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (N == 0) return KDA_OK;
+    if (!q || !k || !v || !beta || !log_alpha || !state || !o) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) ||
+        !aligned16(log_alpha) || !aligned16(state) || !aligned16(o))
+        return KDA_ERR_INVALID_ARG;
+    if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_UNSUPPORTED;
+    return from_cuda(kda::decode_step(q, k, v, beta, log_alpha, state, o, (long long)N * H, dk,
+                                      dv, dtype, static_cast<cudaStream_t>(stream)));
+}
+
+kda_status kda_check(void* stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+    unsigned word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, kda::g_status, sizeof(word)) != cudaSuccess) return KDA_ERR_CUDA;
+    if (word && cudaMemcpyToSymbol(kda::g_status, &zero, sizeof(zero)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (word & kda::KDA_DEV_ERR_TIMEOUT) return KDA_ERR_TIMEOUT;
+    return KDA_OK;
+}
+
+const char* kda_status_string(kda_status status)
+{
+    switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: size or type not implemented";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a device-side bounded wait ran out";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+int kda_version(void) { return 100; }
+
+}  // extern "C"

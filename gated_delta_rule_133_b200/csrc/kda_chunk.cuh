@@ -1,0 +1,20 @@
+// Internal launchers of the KDA CUDA library (not part of the C ABI).
+#pragma once
+
+#include "kda_common.cuh"
+
+namespace kda {
+
+// Decode step over NH = N * H independent (sequence, head) states.
+cudaError_t decode_step(const void* q, const void* k, const void* v, const float* beta,
+                        const float* log_alpha, float* state, void* o, long long NH, int dk,
+                        int dv, kda_dtype dtype, cudaStream_t stream);
+
+// Chunkwise forward on CUDA cores (fp32 arithmetic).  cu == nullptr: nseq
+// sequences of T tokens each; otherwise nseq packed sequences given by cu.
+cudaError_t chunk_fwd_simt(const void* q, const void* k, const void* v, const float* beta,
+                           const float* log_alpha, const float* s0, void* o, float* sT,
+                           const int32_t* cu, int nseq, int T, int H, int dk, int dv,
+                           kda_dtype dtype, cudaStream_t stream);
+
+}  // namespace kda

@@ -1,0 +1,316 @@
+// Chunkwise-parallel KDA forward on CUDA cores, fp32 arithmetic throughout.
+//
+// This is the precise path (fp32 q/k/v, where tensor-core operand rounding
+// would exceed a 1e-4 relative budget) and the path for shapes the
+// tensor-core kernel does not take.  It follows the chunk recurrence of "Hybrid
+// Linear Attention Architecture: Making LLM Training and Inference More
+// Efficient", section IV (also "... Technical Deep Dive ...", section 4, and
+// "Linear Attention Architecture Deep Dive", section 5):
+//
+//   per chunk of C = 64 tokens, G = inclusive cumulative sum of log alpha
+//   (accumulated in log space, fp32), gamma = exp(G_last);
+//   A[r,s] = beta_r sum_c k_rc k_sc exp(G_rc - G_sc)   (s < r)   intra-chunk
+//   T      = (I + A)^-1                                  UT transform
+//   V'     = T diag(beta) (V - (exp(G) * K) S)          = U - W S  (WY form,
+//                                                        applied factored)
+//   O      = (exp(G) * Q) S + Tril_incl(P) V',   P[r,s] = sum_c q_rc k_sc exp(G_rc - G_sc)
+//   S     <- Diag(gamma) S + (exp(G_last - G) * K)^T V'
+//
+// Relative decays exp(G_r - G_s) are factored around the chunk's middle row m
+// ("segmenting intra-chunk cumulative gates"): E = exp(G - G_m) on the row
+// side and F = exp(G_m - G) on the column side, so every factor is bounded
+// by the decay of 32 tokens instead of a whole chunk.  Then
+// exp(G) = exp(G_m) E and exp(G_last - G) = exp(G_last - G_m) F, and the
+// per-channel factors exp(G_m), exp(G_last - G_m) are folded into the state.
+//
+// One CTA (256 threads) per (sequence, head, 32-column slice of d_v); the
+// columns of S evolve independently because the transition acts on the d_k
+// side only.  The CTA walks its chunks in order; everything lives in shared
+// memory.
+#include "kda_chunk.cuh"
+
+namespace kda {
+
+namespace simt {
+
+constexpr int C = 64;       // chunk length
+constexpr int NV = 32;      // value columns per CTA
+constexpr int NT = 256;     // threads per CTA
+
+// acc[i][j] += sum_kk A[(m0 + i*MS) * a_m + kk * a_k] * B[kk * b_k + (n0 + j*NS) * b_n]
+template <int TM, int TN>
+__device__ __forceinline__ void mma_tile(float (&acc)[TM][TN], const float* A, int a_m, int a_k,
+                                         const float* B, int b_k, int b_n, int K, int m0, int MS,
+                                         int n0, int NS)
+{
+#pragma unroll 4
+    for (int kk = 0; kk < K; ++kk) {
+        float a[TM], b[TN];
+#pragma unroll
+        for (int i = 0; i < TM; ++i) a[i] = A[(m0 + i * MS) * a_m + kk * a_k];
+#pragma unroll
+        for (int j = 0; j < TN; ++j) b[j] = B[kk * b_k + (n0 + j * NS) * b_n];
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+}
+
+template <int DK>
+struct Smem {
+    static constexpr int LDK = DK + 1;   // padded row pitch of the [C][DK] tiles
+    static constexpr int LDC = C + 1;    // padded pitch of the [C][C] tiles
+    float qm[C * LDK];    // q * E
+    float km[C * LDK];    // k * E
+    float kf[C * LDK];    // cumulative gate G, then k * F
+    float A[C * LDC];
+    float P[C * LDC];
+    float T[C * LDC];
+    float S[DK * NV];     // state slice, fp32, carried across chunks
+    float Sm[DK * NV];    // exp(G_m) * S for the current chunk
+    float V[C * NV];      // values, then Y = beta (V - X)
+    float Vp[C * NV];     // V' = T Y
+    float gm[DK];         // exp(G_m)
+    float gam[DK];        // exp(G_last)
+    float glm[DK];        // exp(G_last - G_m)
+    float beta[C];
+};
+
+// Rank-r sequence in longest-first order (ties: lower index first).  N is small.
+__device__ int seq_by_rank(const int32_t* cu, int N, int rank, int* s_out)
+{
+    if (threadIdx.x == 0) *s_out = rank;
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        const int li = cu[i + 1] - cu[i];
+        int rk = 0;
+        for (int j = 0; j < N; ++j) {
+            const int lj = cu[j + 1] - cu[j];
+            rk += (lj > li) || (lj == li && j < i);
+        }
+        if (rk == rank) *s_out = i;
+    }
+    __syncthreads();
+    const int n = *s_out;
+    __syncthreads();
+    return n;
+}
+
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(NT)
+chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                      const TIn* __restrict__ v, const float* __restrict__ beta,
+                      const float* __restrict__ log_alpha, const float* s0, TIn* __restrict__ o,
+                      float* sT, const int32_t* __restrict__ cu, int nseq, int T, int H, int DV)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    Smem<DK>& sm = *reinterpret_cast<Smem<DK>*>(smem_raw);
+    constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC;
+    __shared__ int s_tmp;
+
+    const int nslice = DV / NV;
+    const int slice = blockIdx.x % nslice;
+    const int h = (blockIdx.x / nslice) % H;
+    const int rank = blockIdx.x / (nslice * H);
+    int n, tok0, len;
+    if (cu) {
+        n = seq_by_rank(cu, nseq, rank, &s_tmp);
+        tok0 = cu[n];
+        len = cu[n + 1] - tok0;
+    } else {
+        n = rank;
+        tok0 = n * T;
+        len = T;
+    }
+    const int col0 = slice * NV;
+    const int tid = threadIdx.x;
+
+    // initial state slice
+    for (int e = tid; e < DK * NV; e += NT) {
+        const int c = e / NV, j = e % NV;
+        sm.S[e] = s0 ? s0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
+    }
+
+    for (int t0 = 0; t0 < len; t0 += C) {
+        const int L = min(C, len - t0);
+        __syncthreads();
+        // ---- load the chunk (rows >= L are zero: no key, no value, no decay)
+        for (int e = tid; e < C * DK; e += NT) {
+            const int r = e / DK, c = e % DK;
+            float qv = 0.f, kv = 0.f, gv = 0.f;
+            if (r < L) {
+                const size_t off = ((size_t)(tok0 + t0 + r) * H + h) * DK + c;
+                qv = Elem<TIn>::load(q + off);
+                kv = Elem<TIn>::load(k + off);
+                gv = log_alpha[off];
+            }
+            sm.qm[r * LDK + c] = qv;
+            sm.km[r * LDK + c] = kv;
+            sm.kf[r * LDK + c] = gv;
+        }
+        for (int e = tid; e < C * NV; e += NT) {
+            const int r = e / NV, j = e % NV;
+            sm.V[e] = r < L ? Elem<TIn>::load(v + ((size_t)(tok0 + t0 + r) * H + h) * DV + col0 + j) : 0.f;
+        }
+        if (tid < C) sm.beta[tid] = tid < L ? beta[(size_t)(tok0 + t0 + tid) * H + h] : 0.f;
+        __syncthreads();
+
+        // ---- gate cumsum per channel (fp32, log space) and the factor split
+        if (tid < DK) {
+            const int c = tid;
+            float acc = 0.f;
+            for (int r = 0; r < C; ++r) { acc += sm.kf[r * LDK + c]; sm.kf[r * LDK + c] = acc; }
+            const float Gm = sm.kf[(C / 2 - 1) * LDK + c];
+            const float Gl = acc;
+            sm.gm[c] = expf(Gm);
+            sm.gam[c] = expf(Gl);
+            sm.glm[c] = expf(Gl - Gm);
+            for (int r = 0; r < C; ++r) {
+                const float G = sm.kf[r * LDK + c];
+                const float Er = expf(fminf(G - Gm, 80.f));
+                const float Fr = expf(fminf(Gm - G, 80.f));
+                sm.qm[r * LDK + c] *= Er;
+                const float kk = sm.km[r * LDK + c];
+                sm.km[r * LDK + c] = kk * Er;
+                sm.kf[r * LDK + c] = kk * Fr;
+            }
+        }
+        __syncthreads();
+
+        // ---- P = (q E)(k F)^T (lower incl.), A = beta (k E)(k F)^T (strictly lower)
+        {
+            const int tn = tid % 16, tm = tid / 16;
+            float p[4][4] = {}, a[4][4] = {};
+            mma_tile<4, 4>(p, sm.qm, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
+            mma_tile<4, 4>(a, sm.km, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int r = tm + 16 * i, s = tn + 16 * j;
+                    sm.P[r * LDC + s] = s <= r ? p[i][j] : 0.f;
+                    sm.A[r * LDC + s] = s < r ? sm.beta[r] * a[i][j] : 0.f;
+                }
+            // Sm = exp(G_m) * S  (state rows scaled per key channel)
+            for (int e = tid; e < DK * NV; e += NT) sm.Sm[e] = sm.gm[e / NV] * sm.S[e];
+        }
+        __syncthreads();
+
+        // ---- UT transform T = (I + A)^-1 by forward substitution: column j of T
+        // depends only on column j of earlier rows; 4 lanes share one column.
+        {
+            const int j = tid >> 2, p = tid & 3;
+            for (int r = 0; r < C; ++r) {
+                float acc = 0.f;
+                if (r > j)
+                    for (int s = j + p; s < r; s += 4) acc = fmaf(sm.A[r * LDC + s], sm.T[s * LDC + j], acc);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                if (p == 0) sm.T[r * LDC + j] = (r == j ? 1.f : 0.f) - (r > j ? acc : 0.f);
+                __syncwarp();
+            }
+        }
+        // ---- X = (k E) Sm ; Y = beta (V - X)   (into sm.V)
+        {
+            const int tn = tid % 16, tm = tid / 16;
+            float x[4][2] = {};
+            mma_tile<4, 2>(x, sm.km, LDK, 1, sm.Sm, NV, 1, DK, tm, 16, tn, 16);
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int r = tm + 16 * i, cc = tn + 16 * j;
+                    sm.V[r * NV + cc] = sm.beta[r] * (sm.V[r * NV + cc] - x[i][j]);
+                }
+        }
+        __syncthreads();
+        // ---- V' = T Y
+        {
+            const int tn = tid % 16, tm = tid / 16;
+            float y[4][2] = {};
+            mma_tile<4, 2>(y, sm.T, LDC, 1, sm.V, NV, 1, C, tm, 16, tn, 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) sm.Vp[(tm + 16 * i) * NV + tn + 16 * j] = y[i][j];
+        }
+        __syncthreads();
+        // ---- O = (q E) Sm + P V'  -> output rows < L
+        {
+            const int tn = tid % 16, tm = tid / 16;
+            float ov[4][2] = {};
+            mma_tile<4, 2>(ov, sm.qm, LDK, 1, sm.Sm, NV, 1, DK, tm, 16, tn, 16);
+            mma_tile<4, 2>(ov, sm.P, LDC, 1, sm.Vp, NV, 1, C, tm, 16, tn, 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = tm + 16 * i;
+                if (r < L)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+                        Elem<TIn>::store(o + ((size_t)(tok0 + t0 + r) * H + h) * DV + col0 + tn + 16 * j,
+                                         ov[i][j]);
+            }
+        }
+        // ---- S <- gamma S + exp(G_last - G_m) (k F)^T V'
+        {
+            constexpr int TM = DK / 16;
+            const int tn = tid % 16, tm = tid / 16;
+            float ds[TM][2] = {};
+            mma_tile<TM, 2>(ds, sm.kf, 1, LDK, sm.Vp, NV, 1, C, tm, 16, tn, 16);
+#pragma unroll
+            for (int i = 0; i < TM; ++i) {
+                const int c = tm + 16 * i;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int e = c * NV + tn + 16 * j;
+                    sm.S[e] = fmaf(sm.gam[c], sm.S[e], sm.glm[c] * ds[i][j]);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (sT)
+        for (int e = tid; e < DK * NV; e += NT) {
+            const int c = e / NV, j = e % NV;
+            sT[(((size_t)n * H + h) * DK + c) * DV + col0 + j] = sm.S[e];
+        }
+}
+
+template <typename TIn, int DK>
+cudaError_t launch(const void* q, const void* k, const void* v, const float* beta,
+                   const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
+                   int nseq, int T, int H, int dv, cudaStream_t stream)
+{
+    const size_t smem = sizeof(Smem<DK>);
+    auto kern = chunk_fwd_simt_kernel<TIn, DK>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const long long blocks = (long long)nseq * H * (dv / NV);
+    if (blocks == 0) return cudaSuccess;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    kern<<<(unsigned)blocks, NT, smem, stream>>>(
+        static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), beta,
+        log_alpha, s0, static_cast<TIn*>(o), sT, cu, nseq, T, H, dv);
+    return cudaGetLastError();
+}
+
+}  // namespace simt
+
+cudaError_t chunk_fwd_simt(const void* q, const void* k, const void* v, const float* beta,
+                           const float* log_alpha, const float* s0, void* o, float* sT,
+                           const int32_t* cu, int nseq, int T, int H, int dk, int dv,
+                           kda_dtype dtype, cudaStream_t stream)
+{
+    if (dtype == KDA_BF16) {
+        if (dk == 128) return simt::launch<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, stream);
+        if (dk == 64) return simt::launch<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, stream);
+    } else {
+        if (dk == 128) return simt::launch<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, stream);
+        if (dk == 64) return simt::launch<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

@@ -1,0 +1,37 @@
+// Shared device helpers of the KDA CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// Per-device status word (the library is one translation unit, so this is its
+// only definition).  Kernels set bits here when a bounded wait gives up;
+// kda_check() reads and clears it.
+enum : unsigned { KDA_DEV_ERR_TIMEOUT = 1u };
+__device__ unsigned g_status = 0;
+
+__device__ __forceinline__ void flag_timeout() { atomicOr(&g_status, KDA_DEV_ERR_TIMEOUT); }
+
+// Element access for the two supported q/k/v/o element types.
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float load(const float* p) { return *p; }
+    static __device__ __forceinline__ void store(float* p, float x) { *p = x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+};
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+}  // namespace kda

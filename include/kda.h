@@ -1,0 +1,137 @@
+/*
+ * kda.h -- C ABI of the KDA / gated-DeltaNet layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer keeps, per (sequence, head), a d_k x d_v fp32 state S and for each
+ * token t applies
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = S_t^T q_t,                 alpha_t = exp(log_alpha_t)  (per channel)
+ *
+ * ("Hybrid Linear Attention Architecture: Making LLM Training and Inference
+ * More Efficient", section 3.3: decay per channel first, then the delta
+ * rule's erase and write; the output is read after the write as in the
+ * inference loop of "Demystifying Hybrid LLM Architectures", section 2.3.)
+ * No query scaling is applied.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller; the library
+ *    allocates no device memory and keeps no pointer after the call returns.
+ *  - Layouts are dense, row-major, token-major ("[B, T, H, d]": d fastest).
+ *  - q, k, v and o have the element type `dtype` (KDA_BF16 or KDA_F32);
+ *    beta, log_alpha and all states are always fp32.  log_alpha must be <= 0
+ *    (alpha in (0, 1]); it is not checked on the device.
+ *  - Every pointer must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *    asynchronous on that stream and never synchronise.
+ *  - Argument errors are reported synchronously (nothing is launched).  A
+ *    launch failure returns KDA_ERR_CUDA.  Device-side failures (a bounded
+ *    wait that ran out) are recorded in a per-device status word and reported
+ *    by kda_check().
+ *  - Supported: d_k, d_v in {64, 128}, chunk == 64.  Other sizes return
+ *    KDA_ERR_UNSUPPORTED.  No C++ exception crosses this interface.
+ *  - Numerical domain: inside one 64-token chunk the per-channel decay is
+ *    factored around the chunk's middle token; that requires the decay of any
+ *    32 consecutive tokens of one channel to stay below about 80 nats
+ *    (average alpha above ~0.08).  Stronger gates lose accuracy in the
+ *    intra-chunk terms (results stay finite).
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size          */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (d, chunk, dtype)  */
+    KDA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed         */
+    KDA_ERR_TIMEOUT = 4       /* a device-side bounded wait ran out           */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/*
+ * Chunkwise-parallel forward over B equal-length sequences (training and
+ * prefill).  The chunk recurrence is the one given in "Hybrid Linear Attention
+ * Architecture: Making LLM Training and Inference More Efficient", section IV,
+ * "... Technical Deep Dive ...", section 4 and "Linear Attention Architecture
+ * Deep Dive", section 5 (state carried between chunks, WY residual
+ * correction U - W S, lower-triangular intra-chunk term).
+ *
+ *   q, k        [B, T, H, dk]  dtype
+ *   v           [B, T, H, dv]  dtype
+ *   beta        [B, T, H]      fp32, write strength in (0, 1)
+ *   log_alpha   [B, T, H, dk]  fp32, per-channel log forget gate (<= 0)
+ *   initial_state [B, H, dk, dv] fp32, or NULL for zeros (read only)
+ *   o           [B, T, H, dv]  dtype, written
+ *   final_state [B, H, dk, dv] fp32, or NULL if not wanted; written.  It may
+ *               alias initial_state (in-place state update).
+ *   B >= 0, T >= 0 (B*T == 0 is a no-op that still writes final_state from
+ *   initial_state), H >= 1, chunk must be 64.
+ */
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
+                         const float* beta, const float* log_alpha,
+                         const float* initial_state, void* o, float* final_state,
+                         int B, int T, int H, int dk, int dv, int chunk,
+                         kda_dtype dtype, void* stream);
+
+/*
+ * Same computation over N variable-length sequences packed along one token
+ * axis (B = 1).  The state restarts (from initial_state[n] or zero) at every
+ * sequence boundary; the last chunk of each sequence may be shorter than 64.
+ *
+ *   q, k [T, H, dk], v [T, H, dv], beta [T, H], log_alpha [T, H, dk], o [T, H, dv]
+ *   cu_seqlens  [N + 1] int32, DEVICE pointer, cu_seqlens[0] = 0,
+ *               non-decreasing, cu_seqlens[N] = T (not checked on the device;
+ *               a violation is undefined behaviour).
+ *   initial_state / final_state [N, H, dk, dv] fp32 or NULL.
+ *   N <= 65535.  Work is ordered longest sequence first.
+ */
+kda_status kda_varlen_fwd(const void* q, const void* k, const void* v,
+                          const float* beta, const float* log_alpha,
+                          const int32_t* cu_seqlens, int N,
+                          const float* initial_state, void* o, float* final_state,
+                          int T, int H, int dk, int dv, int chunk,
+                          kda_dtype dtype, void* stream);
+
+/*
+ * One decode step of the recurrence for N independent sequences (one new
+ * token each), updating the state in place: the recurrent form of "Hybrid
+ * Linear Attention Architecture: Making LLM Training and Inference More
+ * Efficient", section 3.3, one state update and one state read per token
+ * (its section I).  Memory bound: every state is read once and written once.
+ *
+ *   q, k [N, H, dk], v [N, H, dv]  dtype
+ *   beta [N, H], log_alpha [N, H, dk]  fp32
+ *   state [N, H, dk, dv] fp32, read and overwritten in place
+ *   o [N, H, dv] dtype, written
+ */
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
+                              const float* beta, const float* log_alpha,
+                              float* state, void* o,
+                              int N, int H, int dk, int dv,
+                              kda_dtype dtype, void* stream);
+
+/*
+ * Synchronises `stream` and reports (then clears) the current device's
+ * status word: KDA_ERR_TIMEOUT if a device-side bounded wait ran out since the
+ * last check, KDA_ERR_CUDA if the stream reports an error, else KDA_OK.
+ */
+kda_status kda_check(void* stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char* kda_status_string(kda_status status);
+
+/* Interface version: major * 10000 + minor * 100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -1,0 +1,86 @@
+"""The C ABI loads, exports every declared symbol and validates arguments on
+the host (no GPU needed: only calls that fail validation are made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_133_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert {"kda_chunk_fwd", "kda_varlen_fwd", "kda_recurrent_step"} <= set(names)
+    lib = _lib.load()
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, n
+
+
+def test_status_strings_and_version():
+    for st in range(5):
+        assert _lib.status_string(st).startswith("KDA_")
+    assert "UNKNOWN" in _lib.status_string(99)
+    assert _lib.load().kda_version() >= 100
+
+
+P = 256  # a 16-byte aligned fake address: never dereferenced, validation fails first
+
+
+@pytest.mark.parametrize("args,want", [
+    # negative sizes
+    ((P, P, P, P, P, None, P, None, -1, 8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, None, P, None, 1, -8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, None, P, None, 1, 8, 0, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
+    # null or misaligned tensors
+    ((None, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P + 4, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, P + 8, P, None, 1, 8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
+    # bad dtype code
+    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 7, None), _lib.KDA_ERR_INVALID_ARG),
+    # unsupported sizes
+    ((P, P, P, P, P, None, P, None, 1, 8, 2, 96, 128, 64, 1, None), _lib.KDA_ERR_UNSUPPORTED),
+    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 256, 64, 1, None), _lib.KDA_ERR_UNSUPPORTED),
+    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 32, 1, None), _lib.KDA_ERR_UNSUPPORTED),
+])
+def test_chunk_fwd_validation(args, want):
+    assert _lib.load().kda_chunk_fwd(*args) == want
+
+
+def test_varlen_validation():
+    f = _lib.load().kda_varlen_fwd
+    base = [P, P, P, P, P, P, 4, None, P, None, 100, 2, 128, 128, 64, 1, None]
+    assert f(*base[:6], -1, *base[7:]) == _lib.KDA_ERR_INVALID_ARG          # N < 0
+    assert f(*base[:6], 70000, *base[7:]) == _lib.KDA_ERR_INVALID_ARG       # N too large
+    assert f(*base[:5], None, *base[6:]) == _lib.KDA_ERR_INVALID_ARG        # no cu_seqlens
+    assert f(*base[:5], P + 2, *base[6:]) == _lib.KDA_ERR_INVALID_ARG       # misaligned int32
+    assert f(*base[:12], 80, *base[13:]) == _lib.KDA_ERR_UNSUPPORTED         # d_k = 80
+    assert f(*base[:6], 0, *base[7:]) == _lib.KDA_ERR_INVALID_ARG           # N = 0 with tokens
+
+
+def test_recurrent_step_validation():
+    f = _lib.load().kda_recurrent_step
+    assert f(P, P, P, P, P, P, P, -1, 2, 128, 128, 1, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f(P, P, P, P, P, None, P, 3, 2, 128, 128, 1, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f(P, P, P, P, P, P, P + 4, 3, 2, 128, 128, 1, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f(P, P, P, P, P, P, P, 3, 2, 128, 32, 1, None) == _lib.KDA_ERR_UNSUPPORTED
+    assert f(None, None, None, None, None, None, None, 0, 2, 128, 128, 1, None) == _lib.KDA_OK
+
+
+def test_python_binding_rejects_bad_tensors():
+    import torch
+    import gated_delta_rule_133_b200 as kda
+    q = torch.zeros(1, 8, 2, 128)
+    with pytest.raises(ValueError):
+        kda.kda_chunk_fwd(q, q, q, torch.zeros(1, 8, 2), torch.zeros(1, 8, 2, 64))
+    with pytest.raises(ValueError):
+        kda.kda_chunk_fwd(q, q, q.to(torch.float64), torch.zeros(1, 8, 2), q)
