@@ -40,10 +40,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ----------------------------------------------------------------------------- work model
-def bytes_per_token_head(dk, dv, elem):
-    """Algorithmic HBM bytes per (token, head): q, k, v in, o out (elem bytes
-    each), log alpha (fp32 per key channel) and beta (fp32) in."""
-    return elem * (2 * dk + 2 * dv) + 4 * dk + 4
+def bytes_per_token_head(dk, dv, elem, o_elem=4):
+    """Algorithmic HBM bytes per (token, head): q, k, v in (elem bytes each),
+    o out (o_elem bytes), log alpha (fp32 per key channel) and beta (fp32) in."""
+    return elem * (2 * dk + dv) + o_elem * dv + 4 * dk + 4
 
 
 def flops_per_token_head(dk, dv, C=64):
@@ -53,9 +53,9 @@ def flops_per_token_head(dk, dv, C=64):
     return (2 * (C - 1) + (C + 1)) * dk + 2 * C * dv + 6 * dk * dv + C * C / 3.0
 
 
-def chunk_work(B, T, H, dk, dv, elem=2, state_in=True, state_out=True):
+def chunk_work(B, T, H, dk, dv, elem=2, o_elem=4, state_in=True, state_out=True):
     th = B * T * H
-    nbytes = th * bytes_per_token_head(dk, dv, elem)
+    nbytes = th * bytes_per_token_head(dk, dv, elem, o_elem)
     nbytes += (int(state_in) + int(state_out)) * B * H * dk * dv * 4
     return nbytes, th * flops_per_token_head(dk, dv)
 
@@ -199,7 +199,7 @@ def run_ours(args, world, rank, local):
 
     nsets = 2
     sets = [make_inputs(w, device, seed=w.seed + 1000 * rank + i) for i in range(nsets)]
-    outs = [(torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.bfloat16, device=device),
+    outs = [(torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32, device=device),
              torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)) for _ in range(nsets)]
     nbytes, nflops = chunk_work(w.B, w.T, w.H, w.dk, w.dv)
     set_bytes = sum(t.numel() * t.element_size() for t in sets[0].values() if t is not None)
@@ -249,7 +249,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": f"prefill: B={w.B} H={w.H} T={w.T} d_k={w.dk} d_v={w.dv} chunk={w.chunk}, "
-                               "bf16 q/k/v, fp32 state, random fp32 initial state",
+                               "bf16 q/k/v, fp32 state and fp32 output, random fp32 initial state",
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {nsets} input sets of {set_bytes / 1e6:.0f} MB alternate"},
         "tflops": nflops * world * args.steps / elapsed / 1e12,
@@ -271,7 +271,7 @@ def run_decode(kda, device, stream, world, rank, warmup):
     w = WORKLOADS["decode"]
     x = make_inputs(w, device, seed=w.seed + 1000 * rank)
     state = x["initial_state"].clone()
-    o = torch.empty(w.B, w.H, w.dv, dtype=torch.bfloat16, device=device)
+    o = torch.empty(w.B, w.H, w.dv, dtype=torch.float32, device=device)
 
     def one(s):
         kda.kda_recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["beta"][s], x["log_alpha"][s], state,
@@ -309,7 +309,7 @@ def run_e2e(kda, d, w, device, stream, world, steps):
     copies its inputs host->device and reads o and the final state back."""
     host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in d.items()}
     dev = {k: (None if v is None else torch.empty_like(v, device=device)) for k, v in d.items()}
-    o_h = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.bfloat16).pin_memory()
+    o_h = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32).pin_memory()
     s_h = torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
     d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()

@@ -8,6 +8,8 @@ the computation runs in the library's CUDA kernels.  There is no CPU path.
     o, S_T = kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state)
     o, S_N = kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state)
     o      = kda_recurrent_step(q, k, v, beta, log_alpha, state)   # state updated in place
+
+The output o is fp32 by default (``o_dtype=torch.bfloat16`` rounds it to bf16).
 """
 from __future__ import annotations
 
@@ -43,12 +45,13 @@ def _check(t, name, shape, dtype, device):
 
 
 def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final_state=None,
-                  output_final_state=True, chunk=64, stream=None):
+                  output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None):
     """Chunkwise forward over equal-length sequences.
 
     q, k [B, T, H, dk] and v [B, T, H, dv] (bf16 or fp32); beta [B, T, H] and
     log_alpha [B, T, H, dk] fp32; initial_state [B, H, dk, dv] fp32 or None.
-    Returns (o [B, T, H, dv], final_state [B, H, dk, dv] or None)."""
+    Returns (o [B, T, H, dv] in o_dtype (or o's dtype when o is given),
+    final_state [B, H, dk, dv] or None)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev, dt = q.device, q.dtype
@@ -61,20 +64,23 @@ def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final
     if initial_state is not None:
         _check(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
     if o is None:
-        o = torch.empty(B, T, H, dv, dtype=dt, device=dev)
-    _check(o, "o", (B, T, H, dv), dt, dev)
+        o = torch.empty(B, T, H, dv, dtype=o_dtype, device=dev)
+    _check(o, "o", (B, T, H, dv), o.dtype, dev)
+    if o.dtype not in _DTYPES:
+        raise ValueError(f"unsupported output dtype {o.dtype}")
     if final_state is None and output_final_state:
         final_state = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
     if final_state is not None:
         _check(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
     _lib.call("kda_chunk_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
               _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk,
-              _DTYPES[dt], _stream(stream))
+              _DTYPES[dt], _DTYPES[o.dtype], _stream(stream))
     return o, final_state
 
 
 def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, o=None,
-                   final_state=None, output_final_state=True, chunk=64, stream=None):
+                   final_state=None, output_final_state=True, o_dtype=torch.float32, chunk=64,
+                   stream=None):
     """Chunkwise forward over N packed variable-length sequences.
 
     q, k [T, H, dk], v [T, H, dv]; beta [T, H]; log_alpha [T, H, dk];
@@ -94,19 +100,22 @@ def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, 
     if initial_state is not None:
         _check(initial_state, "initial_state", (N, H, dk, dv), torch.float32, dev)
     if o is None:
-        o = torch.empty(T, H, dv, dtype=dt, device=dev)
-    _check(o, "o", (T, H, dv), dt, dev)
+        o = torch.empty(T, H, dv, dtype=o_dtype, device=dev)
+    _check(o, "o", (T, H, dv), o.dtype, dev)
+    if o.dtype not in _DTYPES:
+        raise ValueError(f"unsupported output dtype {o.dtype}")
     if final_state is None and output_final_state:
         final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
     if final_state is not None:
         _check(final_state, "final_state", (N, H, dk, dv), torch.float32, dev)
     _lib.call("kda_varlen_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
               _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(o), _ptr(final_state), T, H, dk, dv,
-              chunk, _DTYPES[dt], _stream(stream))
+              chunk, _DTYPES[dt], _DTYPES[o.dtype], _stream(stream))
     return o, final_state
 
 
-def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, stream=None):
+def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, o_dtype=torch.float32,
+                       stream=None):
     """One decode step: q, k [N, H, dk], v [N, H, dv], beta [N, H],
     log_alpha [N, H, dk]; state [N, H, dk, dv] fp32 is updated in place.
     Returns o [N, H, dv]."""
@@ -121,10 +130,12 @@ def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, stream=None):
                        (state, "state", (N, H, dk, dv), torch.float32)):
         _check(t, n, s, d, dev)
     if o is None:
-        o = torch.empty(N, H, dv, dtype=dt, device=dev)
-    _check(o, "o", (N, H, dv), dt, dev)
+        o = torch.empty(N, H, dv, dtype=o_dtype, device=dev)
+    _check(o, "o", (N, H, dv), o.dtype, dev)
+    if o.dtype not in _DTYPES:
+        raise ValueError(f"unsupported output dtype {o.dtype}")
     _lib.call("kda_recurrent_step", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
-              _ptr(state), _ptr(o), N, H, dk, dv, _DTYPES[dt], _stream(stream))
+              _ptr(state), _ptr(o), N, H, dk, dv, _DTYPES[dt], _DTYPES[o.dtype], _stream(stream))
     return o
 
 

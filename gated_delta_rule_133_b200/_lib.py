@@ -19,9 +19,9 @@ KDA_F32, KDA_BF16 = 0, 1
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 SIGNATURES = {
-    "kda_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
-    "kda_varlen_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
-    "kda_recurrent_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "kda_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_varlen_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_recurrent_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "kda_check": (_I, [_P]),
     "kda_status_string": (ctypes.c_char_p, [_I]),
     "kda_version": (_I, []),

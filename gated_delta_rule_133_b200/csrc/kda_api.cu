@@ -1,6 +1,7 @@
 // C ABI of the KDA library: argument validation, path selection, status codes.
 // Declarations and the contract of every entry point are in include/kda.h.
 #include <cuda_runtime.h>
+#include <stdlib.h>
 
 #include "kda_chunk.cuh"
 
@@ -10,15 +11,46 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool supported_d(int d) { return d == 64 || d == 128; }
 
+bool valid_dtype(kda_dtype t) { return t == KDA_F32 || t == KDA_BF16; }
+
 kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+// KDA_FORCE_SIMT=1 routes bf16 inputs to the CUDA-core kernel (used by tests
+// that compare the two kernels); KDA_TIMEOUT_CYCLES bounds every device-side
+// wait of the tensor-core kernel (default 2^31 SM cycles, about one second).
+bool force_simt()
+{
+    const char* e = getenv("KDA_FORCE_SIMT");
+    return e && e[0] == '1';
+}
+
+long long timeout_cycles()
+{
+    const char* e = getenv("KDA_TIMEOUT_CYCLES");
+    long long v = e ? atoll(e) : 0;
+    return v > 0 ? v : (1LL << 31);
+}
+
+kda_status run_chunk(const void* q, const void* k, const void* v, const float* beta,
+                     const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
+                     int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype dtype,
+                     kda_dtype o_dtype, cudaStream_t s)
+{
+    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && !force_simt())
+        return from_cuda(kda::chunk_fwd_tc(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk,
+                                           dv, o_dtype, timeout_cycles(), s));
+    return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, dtype,
+                                         o_dtype, s));
+}
 
 // Shared checks of the forward entry points.
 kda_status check_fwd(const void* q, const void* k, const void* v, const float* beta,
                      const float* log_alpha, const float* s0, const void* o, const float* sT,
-                     long long tokens, int H, int dk, int dv, int chunk, kda_dtype dtype)
+                     long long tokens, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                     kda_dtype o_dtype)
 {
     if (H <= 0 || dk <= 0 || dv <= 0 || tokens < 0) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype) || !valid_dtype(o_dtype)) return KDA_ERR_INVALID_ARG;
     if (tokens > 0) {
         if (!q || !k || !v || !beta || !log_alpha || !o) return KDA_ERR_INVALID_ARG;
         if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) ||
@@ -46,43 +78,44 @@ extern "C" {
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
                          const float* log_alpha, const float* initial_state, void* o,
                          float* final_state, int B, int T, int H, int dk, int dv, int chunk,
-                         kda_dtype dtype, void* stream)
+                         kda_dtype dtype, kda_dtype o_dtype, void* stream)
 {
     if (B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
     const long long tokens = (long long)B * T;
     kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, tokens, H,
-                              dk, dv, chunk, dtype);
+                              dk, dv, chunk, dtype, o_dtype);
     if (st != KDA_OK) return st;
     if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (tokens == 0) return copy_state(initial_state, final_state, (size_t)B * H * dk * dv, s);
-    return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, initial_state, o, final_state,
-                                         nullptr, B, T, H, dk, dv, dtype, s));
+    return run_chunk(q, k, v, beta, log_alpha, initial_state, o, final_state, nullptr, B, T, tokens, H, dk,
+                     dv, dtype, o_dtype, s);
 }
 
 kda_status kda_varlen_fwd(const void* q, const void* k, const void* v, const float* beta,
                           const float* log_alpha, const int32_t* cu_seqlens, int N,
                           const float* initial_state, void* o, float* final_state, int T, int H,
-                          int dk, int dv, int chunk, kda_dtype dtype, void* stream)
+                          int dk, int dv, int chunk, kda_dtype dtype, kda_dtype o_dtype,
+                          void* stream)
 {
     if (N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
     kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, T, H, dk,
-                              dv, chunk, dtype);
+                              dv, chunk, dtype, o_dtype);
     if (st != KDA_OK) return st;
     if (N == 0) return T == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
     if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0) return copy_state(initial_state, final_state, (size_t)N * H * dk * dv, s);
-    return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, initial_state, o, final_state,
-                                         cu_seqlens, N, T, H, dk, dv, dtype, s));
+    return run_chunk(q, k, v, beta, log_alpha, initial_state, o, final_state, cu_seqlens, N, T, T, H, dk,
+                     dv, dtype, o_dtype, s);
 }
 
 kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* beta,
                               const float* log_alpha, float* state, void* o, int N, int H, int dk,
-                              int dv, kda_dtype dtype, void* stream)
+                              int dv, kda_dtype dtype, kda_dtype o_dtype, void* stream)
 {
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype) || !valid_dtype(o_dtype)) return KDA_ERR_INVALID_ARG;
     if (N == 0) return KDA_OK;
     if (!q || !k || !v || !beta || !log_alpha || !state || !o) return KDA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) ||
@@ -90,7 +123,7 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
         return KDA_ERR_INVALID_ARG;
     if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_UNSUPPORTED;
     return from_cuda(kda::decode_step(q, k, v, beta, log_alpha, state, o, (long long)N * H, dk,
-                                      dv, dtype, static_cast<cudaStream_t>(stream)));
+                                      dv, dtype, o_dtype, static_cast<cudaStream_t>(stream)));
 }
 
 kda_status kda_check(void* stream)

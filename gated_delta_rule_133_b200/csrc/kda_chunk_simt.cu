@@ -97,11 +97,11 @@ __device__ int seq_by_rank(const int32_t* cu, int N, int rank, int* s_out)
     return n;
 }
 
-template <typename TIn, int DK>
+template <typename TIn, typename TOut, int DK>
 __global__ void __launch_bounds__(NT)
 chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                       const TIn* __restrict__ v, const float* __restrict__ beta,
-                      const float* __restrict__ log_alpha, const float* s0, TIn* __restrict__ o,
+                      const float* __restrict__ log_alpha, const float* s0, TOut* __restrict__ o,
                       float* sT, const int32_t* __restrict__ cu, int nseq, int T, int H, int DV)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -249,7 +249,7 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                 if (r < L)
 #pragma unroll
                     for (int j = 0; j < 2; ++j)
-                        Elem<TIn>::store(o + ((size_t)(tok0 + t0 + r) * H + h) * DV + col0 + tn + 16 * j,
+                        Elem<TOut>::store(o + ((size_t)(tok0 + t0 + r) * H + h) * DV + col0 + tn + 16 * j,
                                          ov[i][j]);
             }
         }
@@ -278,13 +278,13 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
         }
 }
 
-template <typename TIn, int DK>
+template <typename TIn, typename TOut, int DK>
 cudaError_t launch(const void* q, const void* k, const void* v, const float* beta,
                    const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
                    int nseq, int T, int H, int dv, cudaStream_t stream)
 {
     const size_t smem = sizeof(Smem<DK>);
-    auto kern = chunk_fwd_simt_kernel<TIn, DK>;
+    auto kern = chunk_fwd_simt_kernel<TIn, TOut, DK>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     const long long blocks = (long long)nseq * H * (dv / NV);
@@ -292,8 +292,18 @@ cudaError_t launch(const void* q, const void* k, const void* v, const float* bet
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     kern<<<(unsigned)blocks, NT, smem, stream>>>(
         static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), beta,
-        log_alpha, s0, static_cast<TIn*>(o), sT, cu, nseq, T, H, dv);
+        log_alpha, s0, static_cast<TOut*>(o), sT, cu, nseq, T, H, dv);
     return cudaGetLastError();
+}
+
+template <typename TIn, typename TOut>
+cudaError_t launch_dk(const void* q, const void* k, const void* v, const float* beta,
+                      const float* log_alpha, const float* s0, void* o, float* sT,
+                      const int32_t* cu, int nseq, int T, int H, int dk, int dv, cudaStream_t s)
+{
+    if (dk == 128) return launch<TIn, TOut, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, s);
+    if (dk == 64) return launch<TIn, TOut, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, s);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace simt
@@ -301,16 +311,16 @@ cudaError_t launch(const void* q, const void* k, const void* v, const float* bet
 cudaError_t chunk_fwd_simt(const void* q, const void* k, const void* v, const float* beta,
                            const float* log_alpha, const float* s0, void* o, float* sT,
                            const int32_t* cu, int nseq, int T, int H, int dk, int dv,
-                           kda_dtype dtype, cudaStream_t stream)
+                           kda_dtype dtype, kda_dtype o_dtype, cudaStream_t s)
 {
-    if (dtype == KDA_BF16) {
-        if (dk == 128) return simt::launch<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, stream);
-        if (dk == 64) return simt::launch<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, stream);
-    } else {
-        if (dk == 128) return simt::launch<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, stream);
-        if (dk == 64) return simt::launch<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, stream);
-    }
-    return cudaErrorInvalidValue;
+    using bf = __nv_bfloat16;
+    if (dtype == KDA_BF16 && o_dtype == KDA_BF16)
+        return simt::launch_dk<bf, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, s);
+    if (dtype == KDA_BF16 && o_dtype == KDA_F32)
+        return simt::launch_dk<bf, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, s);
+    if (dtype == KDA_F32 && o_dtype == KDA_BF16)
+        return simt::launch_dk<float, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, s);
+    return simt::launch_dk<float, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, s);
 }
 
 }  // namespace kda

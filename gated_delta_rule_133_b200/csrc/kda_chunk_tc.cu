@@ -1,0 +1,611 @@
+// Chunkwise-parallel KDA forward on the sm_100a tensor cores (bf16 q/k/v,
+// fp32 gates, state, operands and accumulation; tcgen05 kind::tf32).
+//
+// Same chunk algebra as the CUDA-core path ("Hybrid Linear Attention
+// Architecture: Making LLM Training and Inference More Efficient", section IV;
+// "... Technical Deep Dive ...", section 4; "Linear Attention Architecture Deep
+// Dive", section 5), arranged so that every chunk-local and state product is a
+// 128-row tcgen05.mma with its fp32 accumulator in TMEM:
+//
+//   per chunk, G = cumsum(log alpha) (fp32), m = middle row,
+//   E = exp(G - G_m), F = exp(G_m - G)                 (bounded by 32 tokens)
+//   A1 = [q E ; k E]   (128 x d_k)     B1 = k F  (64 x d_k)
+//   [P ; A~] = A1 B1^T                 -> P (lower incl.), A = beta A~ (strictly lower)
+//   X = A1 (diag(exp(G_m)) S)          -> rows 0..63: (exp(G) q) S, rows 64..127: (exp(G) k) S
+//   Y = diag(beta) (V - (exp(G) k) S)  (so that V' = T Y = U - W S)
+//   T = (I + A)^-1                     (UT transform, blocked substitution, fp32)
+//   Z = diag(exp(G_last - G_m)) B1^T T = (exp(G_last - G) k)^T T   (d_k x 64)
+//   PT = P T
+//   dS = Z Y ;  O = (exp(G) q) S + PT Y ;  S <- diag(exp(G_last)) S + dS
+//
+// Operands are tf32 (10-bit mantissa): the layer's outputs are heavy-tailed
+// (max |o| is about 10 x RMS) and a 2e-2 max/RMS budget leaves ~2^-11 relative
+// precision for the largest outputs, which bf16 operands (2^-9) do not meet.
+// The state S stays in fp32 registers (one key channel per thread).  q, k and
+// log alpha tiles arrive by TMA (no multicast).
+//
+// One CTA of 128 threads (one warpgroup: thread i owns TMEM lane i) per
+// (sequence, head, 64 value columns).  The CTA walks its chunks in order;
+// shared-memory regions are reused as each operand dies (see Plan).
+#include "kda_chunk.cuh"
+#include "kda_sm100.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace kda {
+namespace tc {
+
+using namespace sm100;
+
+constexpr int C = 64;      // chunk length
+constexpr int NV = 64;     // value columns per CTA
+constexpr int NT = 128;    // threads per CTA
+constexpr int LDA = 65;    // fp32 pitch of the inversion scratch
+
+struct Params {
+    const __nv_bfloat16* v;
+    const float* beta;
+    const float* s0;
+    void* o;
+    float* sT;
+    const int32_t* cu;
+    int nseq, T, H, DV;
+    long long timeout_cycles;
+};
+
+// Shared-memory plan (byte offsets from a 1024-aligned base).  Every operand
+// tile is fp32 in the K-major 128-byte-swizzled layout.
+//   R1: A1 [128][d_k] until MMAs PA and X complete; then P [64][64] (0),
+//       T^T [64][64] (16 KB), the fp32 inversion scratch A (32 KB) and X (~48 KB);
+//       PT [64][64] reuses P's place once MMA PT completes.
+//   R2: B1 [64][d_k] until MMA Z completes; then Z [128][64].
+//   R3: the state operand [64][d_k] until MMA X completes; then Y [64][64].
+//   STG: TMA staging of q, k (bf16) and log alpha (fp32) for the next chunk.
+struct Plan {
+    static constexpr int R1 = 0;
+    static constexpr int P = R1, TOP = R1 + 16384, AS = R1 + 32768, XS = AS + C * LDA * 4;
+    static constexpr int R2 = 65536;
+    static constexpr int R3 = 98304;
+    static constexpr int STG = 131072;
+    static constexpr int VEC = STG + 65536;        // gm[128] gam[128] glm[128] beta[64]
+    static constexpr int BAR = VEC + (3 * 128 + 64) * 4;
+    static constexpr int END = BAR + 64;
+    static constexpr int BYTES = END + 1024;       // + alignment slack
+};
+static_assert(Plan::XS + 32 * 33 * 4 <= Plan::R2, "inversion scratch overflows R1");
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p)
+{
+    const uint32_t a = smem_u32(p);
+    return p + (((a + 1023u) & ~1023u) - a);
+}
+
+// Rank-r sequence in longest-first order (ties: lower index first).
+__device__ int seq_by_rank(const int32_t* cu, int N, int rank, int* slot)
+{
+    if (threadIdx.x == 0) *slot = rank;
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        const int li = cu[i + 1] - cu[i];
+        int rk = 0;
+        for (int j = 0; j < N; ++j) {
+            const int lj = cu[j + 1] - cu[j];
+            rk += (lj > li) || (lj == li && j < i);
+        }
+        if (rk == rank) *slot = i;
+    }
+    __syncthreads();
+    const int n = *slot;
+    __syncthreads();
+    return n;
+}
+
+// T[s][j], stored transposed in the K-major operand tile (row j, column s).
+__device__ __forceinline__ float& Tat(unsigned char* Top, int s, int j) { return swf(Top, j, s, C); }
+
+// T = (I + A)^-1 for the strictly lower 64 x 64 A in `As` (fp32, pitch 65),
+// written into the operand tile Top (zeros above the diagonal).  Diagonal
+// 16 x 16 blocks by forward substitution (one warp per block, one lane per
+// column), then T10 = -T11 A10 T00, T32 = -T33 A32 T22, and the lower-left
+// 32 x 32 block -T_BB A_BA T_AA.
+__device__ __forceinline__ void invert_unit_lower(const float* As, unsigned char* Top, float* X)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < C * C / 4; e += NT) reinterpret_cast<float4*>(Top)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+    {
+        const int j = lane & 15, b0 = 16 * warp;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int s = 0; s < r; ++s) acc = fmaf(As[(b0 + r) * LDA + b0 + s], x[s], acc);
+            x[r] = (r == j) ? 1.f : (r < j ? 0.f : -acc);
+        }
+        if (lane < 16) {
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tat(Top, b0 + r, b0 + j) = x[r];
+        }
+    }
+    __syncthreads();
+    {
+        const int blk = tid >> 6, i = (tid & 63) >> 2, j0 = (tid & 3) * 4;
+        const int rb = blk ? 48 : 16, cb = blk ? 32 : 0;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+            const float a = As[(rb + i) * LDA + cb + k];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] = fmaf(a, Tat(Top, cb + k, cb + j0 + q), acc[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) X[(blk * 16 + i) * 33 + j0 + q] = acc[q];
+        __syncthreads();
+        float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+            const float a = Tat(Top, rb + i, rb + k);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) t[q] = fmaf(a, X[(blk * 16 + k) * 33 + j0 + q], t[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) Tat(Top, rb + i, cb + j0 + q) = -t[q];
+    }
+    __syncthreads();
+    {
+        const int i = tid >> 2, j0 = (tid & 3) * 8;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+            const float a = As[(32 + i) * LDA + k];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = fmaf(a, Tat(Top, k, j0 + q), acc[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) X[i * 33 + j0 + q] = acc[q];
+        __syncthreads();
+        float t[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+            const float a = Tat(Top, 32 + i, 32 + k);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) t[q] = fmaf(a, X[k * 33 + j0 + q], t[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) Tat(Top, 32 + i, j0 + q) = -t[q];
+    }
+    __syncthreads();
+    // operand rounding to tf32, once the full-precision solve is done
+    for (int e = tid; e < C * C / 4; e += NT) {
+        float4* p4 = reinterpret_cast<float4*>(Top) + e;
+        float4 v = *p4;
+        *p4 = make_float4(tf32r(v.x), tf32r(v.y), tf32r(v.z), tf32r(v.w));
+    }
+}
+
+// K-major fp32 SW128 operand descriptor for MMA k-step kk (K = 8 per step):
+// 4 steps per 128-byte atom column, atom columns `atom_stride` bytes apart.
+__device__ __forceinline__ uint64_t kdesc(const unsigned char* tile, int kk, int atom_stride)
+{
+    return sdesc_sw128(smem_u32(tile) + (kk >> 2) * atom_stride + (kk & 3) * 32, 16, 1024);
+}
+
+// All threads poll; a CTA-wide vote turns any timeout into a common exit.
+#define KDA_WAIT_OR_EXIT(bar, parity)                                                  \
+    do {                                                                               \
+        const bool ok_ = mbar_wait((bar), (parity), abort_flag, p.timeout_cycles);    \
+        if (__syncthreads_or(!ok_)) goto finish;                                       \
+    } while (0)
+
+template <typename TO, int DK>
+__global__ void __launch_bounds__(NT, 1)
+chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                    const __grid_constant__ CUtensorMap tmg, const Params p)
+{
+    using PL = Plan;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = align1024(smem_raw);
+    unsigned char* A1 = sm + PL::R1;
+    unsigned char* Pb = sm + PL::P;
+    unsigned char* PTb = sm + PL::P;
+    unsigned char* Top = sm + PL::TOP;
+    float* As = reinterpret_cast<float*>(sm + PL::AS);
+    float* Xs = reinterpret_cast<float*>(sm + PL::XS);
+    unsigned char* B1 = sm + PL::R2;
+    unsigned char* Zb = sm + PL::R2;
+    unsigned char* Smb = sm + PL::R3;
+    unsigned char* Yb = sm + PL::R3;
+    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(sm + PL::STG);
+    const __nv_bfloat16* ks = qs + C * DK;
+    const float* gs = reinterpret_cast<const float*>(ks + C * DK);
+    float* gm_s = reinterpret_cast<float*>(sm + PL::VEC);
+    float* gam_s = gm_s + 128;
+    float* glm_s = gam_s + 128;
+    float* beta_s = glm_s + 128;
+    uint64_t* mb_tma = reinterpret_cast<uint64_t*>(sm + PL::BAR);
+    uint64_t* mb_mma = mb_tma + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mb_tma + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* misc_slot = reinterpret_cast<int*>(tmem_slot + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int nslice = p.DV / NV;
+    const int slice = blockIdx.x % nslice;
+    const int h = (blockIdx.x / nslice) % p.H;
+    const int rank = blockIdx.x / (nslice * p.H);
+    const int H = p.H, DV = p.DV;
+    int n, tok0, len;
+    if (p.cu) {
+        n = seq_by_rank(p.cu, p.nseq, rank, misc_slot);
+        tok0 = p.cu[n];
+        len = p.cu[n + 1] - tok0;
+    } else {
+        n = rank;
+        tok0 = n * p.T;
+        len = p.T;
+    }
+    const int col0 = slice * NV;
+    const int nchunks = (len + C - 1) / C;
+
+    if (tid == 0) {
+        mbar_init(mb_tma, 1);
+        mbar_init(mb_mma, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async();
+        prefetch_tmap(&tmq);
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmg);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t t_PA = tmem, t_O = tmem + 64, t_Z = tmem + 128, t_PT = tmem + 192, t_dS = tmem + 256;
+
+    // fp32 state: thread c < DK owns row c of this 64-column slice
+    float S[NV];
+    {
+        const bool own = tid < DK;
+        const float* src = (p.s0 && own) ? p.s0 + (((size_t)n * H + h) * DK + tid) * DV + col0 : nullptr;
+#pragma unroll
+        for (int j = 0; j < NV; j += 4) {
+            float4 v4 = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
+        }
+    }
+
+    uint32_t mma_phase = 0;
+    int tma_pending = 0, tma_parity = 0, mma_pending = 0;
+    constexpr uint32_t kStageBytes = (uint32_t)C * DK * (2 + 2 + 4);
+    constexpr uint32_t kI = idesc_tf32(128, 64, 0, 0);
+    constexpr uint32_t kI_AMN = idesc_tf32(128, 64, 1, 0);
+    constexpr int kA1 = 128 * 128;   // atom-column strides (bytes) of the 128-row and 64-row tiles
+    constexpr int kR64 = 64 * 128;
+
+    if (tid == 0 && nchunks > 0) {
+        mbar_expect_tx(mb_tma, kStageBytes);
+        tma_load_3d((void*)qs, &tmq, mb_tma, 0, h, tok0);
+        tma_load_3d((void*)ks, &tmk, mb_tma, 0, h, tok0);
+        tma_load_3d((void*)gs, &tmg, mb_tma, 0, h, tok0);
+    }
+    tma_pending = nchunks > 0;
+    float beta_next = 0.f;
+    if (tid < C && tid < len) beta_next = p.beta[(size_t)(tok0 + tid) * H + h];
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int L = min(C, len - c * C);
+        const int tokc = tok0 + c * C;
+
+        // values of this chunk for Y (thread 64 + s owns chunk row s), and beta
+        uint4 vraw[8];
+        {
+            const int s = tid - C;
+            const bool live = tid >= C && s < L;
+            const uint4* src = live ? reinterpret_cast<const uint4*>(p.v + ((size_t)(tokc + s) * H + h) * DV + col0)
+                                    : nullptr;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) vraw[u] = live ? __ldg(src + u) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (tid < C) beta_s[tid] = beta_next;
+
+        tma_parity = c & 1;
+        KDA_WAIT_OR_EXIT(mb_tma, (uint32_t)(c & 1));
+        tma_pending = 0;
+        if (tid < C) beta_next = (c + 1 < nchunks && C + tid < len - c * C)
+                                     ? p.beta[(size_t)(tokc + C + tid) * H + h] : 0.f;
+
+        // ---- gate cumsum in log space (fp32), operands A1, B1 and the state operand
+        if (tid < DK) {
+            float G[C];
+#pragma unroll
+            for (int r = 0; r < C; ++r) G[r] = (r < L) ? gs[r * DK + tid] : 0.f;
+#pragma unroll
+            for (int r = 1; r < C; ++r) G[r] += G[r - 1];
+            const float Gm = G[C / 2 - 1], Gl = G[C - 1];
+            const float egm = expf(Gm);
+            gm_s[tid] = egm;
+            gam_s[tid] = expf(Gl);
+            glm_s[tid] = expf(Gl - Gm);
+#pragma unroll
+            for (int r = 0; r < C; ++r) {
+                const float e = __expf(fminf(G[r] - Gm, 80.f));
+                const float f = __expf(fminf(Gm - G[r], 80.f));
+                const bool live = r < L;
+                const float qv = live ? __bfloat162float(qs[r * DK + tid]) : 0.f;
+                const float kv = live ? __bfloat162float(ks[r * DK + tid]) : 0.f;
+                swf(A1, r, tid, 128) = tf32r(qv * e);
+                swf(A1, C + r, tid, 128) = tf32r(kv * e);
+                swf(B1, r, tid, C) = tf32r(kv * f);
+            }
+#pragma unroll
+            for (int j = 0; j < NV; ++j) swf(Smb, j, tid, NV) = tf32r(egm * S[j]);
+        }
+        fence_proxy_async();
+        __syncthreads();
+
+        if (tid == 0) {
+            if (c + 1 < nchunks) {  // staging is free again: fetch the next chunk
+                mbar_expect_tx(mb_tma, kStageBytes);
+                tma_load_3d((void*)qs, &tmq, mb_tma, 0, h, tokc + C);
+                tma_load_3d((void*)ks, &tmk, mb_tma, 0, h, tokc + C);
+                tma_load_3d((void*)gs, &tmg, mb_tma, 0, h, tokc + C);
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < DK / 8; ++kk)   // [P ; A~] = A1 B1^T
+                umma_tf32(t_PA, kdesc(A1, kk, kA1), kdesc(B1, kk, kR64), kI, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < DK / 8; ++kk)   // X = A1 (diag(exp(G_m)) S)
+                umma_tf32(t_O, kdesc(A1, kk, kA1), kdesc(Smb, kk, kR64), kI, kk > 0);
+            umma_commit(mb_mma);
+        }
+        tma_pending = c + 1 < nchunks;
+        tma_parity = (c + 1) & 1;
+        mma_pending = 1;
+        KDA_WAIT_OR_EXIT(mb_mma, mma_phase & 1);
+        ++mma_phase;
+        mma_pending = 0;
+        tc_fence_after();
+
+        // ---- P (lanes 0..63), A (lanes 64..127), Y (lanes 64..127 of X)
+        {
+            float acc[64];
+            tmem_ld64(t_PA + lane_off, acc);
+            tmem_wait_ld();
+            if (tid < C) {
+                const int r = tid;
+#pragma unroll
+                for (int s = 0; s < C; ++s) acc[s] = s <= r ? acc[s] : 0.f;
+                st_row_swf<16>(Pb, r, 0, C, acc);
+            } else {
+                const int r = tid - C;
+                const float b = beta_s[r];
+#pragma unroll
+                for (int s = 0; s < C; ++s) As[r * LDA + s] = s < r ? b * acc[s] : 0.f;
+            }
+            tmem_ld64(t_O + lane_off, acc);
+            tmem_wait_ld();
+            if (tid >= C) {
+                const int s = tid - C;
+                const float b = beta_s[s];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vraw[u]);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const float2 f2 = __bfloat1622float2(v2[w]);
+                        const int j = u * 8 + w * 2;
+                        swf(Yb, j, s, NV) = tf32r(b * (f2.x - acc[j]));
+                        swf(Yb, j + 1, s, NV) = tf32r(b * (f2.y - acc[j + 1]));
+                    }
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- UT transform into the T^T operand tile
+        invert_unit_lower(As, Top, Xs);
+        fence_proxy_async();
+        __syncthreads();
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C / 8; ++kk)    // Z' = B1^T T   (B1 read MN-major)
+                umma_tf32(t_Z, sdesc_sw128(smem_u32(B1) + kk * 1024, kR64, 1024), kdesc(Top, kk, kR64), kI_AMN,
+                          kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < C / 8; ++kk)    // PT = P T  (rows 64..127 unused)
+                umma_tf32(t_PT, kdesc(Pb, kk, kR64), kdesc(Top, kk, kR64), kI, kk > 0);
+            umma_commit(mb_mma);
+        }
+        mma_pending = 1;
+        KDA_WAIT_OR_EXIT(mb_mma, mma_phase & 1);
+        ++mma_phase;
+        mma_pending = 0;
+        tc_fence_after();
+
+        {
+            float acc[64];
+            tmem_ld64(t_Z + lane_off, acc);    // Z = diag(exp(G_last - G_m)) Z'  (row = key channel)
+            tmem_wait_ld();
+            {
+                const float sc = tid < DK ? glm_s[tid] : 0.f;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) acc[j] *= sc;
+                st_row_swf<16>(Zb, tid, 0, 128, acc);
+            }
+            tmem_ld64(t_PT + lane_off, acc);
+            tmem_wait_ld();
+            if (tid < C) st_row_swf<16>(PTb, tid, 0, C, acc);
+        }
+        tc_fence_before();
+        fence_proxy_async();
+        __syncthreads();
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C / 8; ++kk)    // dS = Z Y
+                umma_tf32(t_dS, kdesc(Zb, kk, kA1), kdesc(Yb, kk, kR64), kI, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < C / 8; ++kk)    // O += PT Y  (rows 0..63 of X)
+                umma_tf32(t_O, kdesc(PTb, kk, kR64), kdesc(Yb, kk, kR64), kI, 1);
+            umma_commit(mb_mma);
+        }
+        mma_pending = 1;
+        KDA_WAIT_OR_EXIT(mb_mma, mma_phase & 1);
+        ++mma_phase;
+        mma_pending = 0;
+        tc_fence_after();
+
+        {
+            float acc[64];
+            tmem_ld64(t_dS + lane_off, acc);
+            tmem_wait_ld();
+            if (tid < DK) {
+                const float gm = gam_s[tid];
+#pragma unroll
+                for (int j = 0; j < NV; ++j) S[j] = fmaf(gm, S[j], acc[j]);
+            }
+            tmem_ld64(t_O + lane_off, acc);
+            tmem_wait_ld();
+            if (tid < L) {
+                const size_t off = ((size_t)(tokc + tid) * H + h) * DV + col0;
+                if constexpr (sizeof(TO) == 4) {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + off);
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
+                        dst[u] = make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        dst[u] = make_uint4(pack_bf16(acc[8 * u], acc[8 * u + 1]), pack_bf16(acc[8 * u + 2], acc[8 * u + 3]),
+                                            pack_bf16(acc[8 * u + 4], acc[8 * u + 5]), pack_bf16(acc[8 * u + 6], acc[8 * u + 7]));
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    if (p.sT && tid < DK) {
+        float* dst = p.sT + (((size_t)n * H + h) * DK + tid) * DV + col0;
+#pragma unroll
+        for (int j = 0; j < NV; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+
+finish:
+    // After a timeout, give the copies and the MMAs still in flight a bounded
+    // chance to land before the TMEM is released and the CTA exits.
+    if (*abort_flag) {
+        volatile int never = 0;
+        if (tma_pending) (void)mbar_wait(mb_tma, (uint32_t)tma_parity, &never, p.timeout_cycles);
+        if (mma_pending) (void)mbar_wait(mb_mma, mma_phase & 1, &never, p.timeout_cycles);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+#undef KDA_WAIT_OR_EXIT
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// [tokens, H, DK] (bf16 or fp32), box = 64 tokens x 1 head x DK channels, no
+// swizzle; rows past the end of the tensor are filled with zeros.
+static bool make_tmap(CUtensorMap* m, const void* base, long long tokens, int H, int DK, bool fp32)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t es = fp32 ? 4 : 2;
+    const cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)H, (cuuint64_t)tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)DK * es, (cuuint64_t)H * DK * es};
+    const cuuint32_t box[3] = {(cuuint32_t)DK, 1, (cuuint32_t)C};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename TO, int DK>
+static cudaError_t launch(const void* q, const void* k, const float* log_alpha, const Params& prm,
+                          long long tokens, cudaStream_t stream)
+{
+    CUtensorMap tq, tk, tg;
+    if (!make_tmap(&tq, q, tokens, prm.H, DK, false) || !make_tmap(&tk, k, tokens, prm.H, DK, false) ||
+        !make_tmap(&tg, log_alpha, tokens, prm.H, DK, true))
+        return cudaErrorInvalidValue;
+    auto kern = chunk_fwd_tc_kernel<TO, DK>;
+    const int smem = Plan::BYTES;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    const long long blocks = (long long)prm.nseq * prm.H * (prm.DV / NV);
+    if (blocks == 0) return cudaSuccess;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    kern<<<(unsigned)blocks, NT, smem, stream>>>(tq, tk, tg, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+
+bool chunk_fwd_tc_supported(int dk, int dv, kda_dtype dtype)
+{
+    return dtype == KDA_BF16 && (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
+}
+
+cudaError_t chunk_fwd_tc(const void* q, const void* k, const void* v, const float* beta,
+                         const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
+                         int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
+                         long long timeout_cycles, cudaStream_t stream)
+{
+    tc::Params prm;
+    prm.v = static_cast<const __nv_bfloat16*>(v);
+    prm.beta = beta;
+    prm.s0 = s0;
+    prm.o = o;
+    prm.sT = sT;
+    prm.cu = cu;
+    prm.nseq = nseq;
+    prm.T = T;
+    prm.H = H;
+    prm.DV = dv;
+    prm.timeout_cycles = timeout_cycles;
+    if (o_dtype == KDA_F32) {
+        if (dk == 128) return tc::launch<float, 128>(q, k, log_alpha, prm, tokens, stream);
+        if (dk == 64) return tc::launch<float, 64>(q, k, log_alpha, prm, tokens, stream);
+    } else {
+        if (dk == 128) return tc::launch<__nv_bfloat16, 128>(q, k, log_alpha, prm, tokens, stream);
+        if (dk == 64) return tc::launch<__nv_bfloat16, 64>(q, k, log_alpha, prm, tokens, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

@@ -17,11 +17,11 @@
 
 namespace kda {
 
-template <typename T, int DK, int DV>
+template <typename T, typename TO, int DK, int DV>
 __global__ void __launch_bounds__(256)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ log_alpha,
-                   float* __restrict__ state, T* __restrict__ o)
+                   float* __restrict__ state, TO* __restrict__ o)
 {
     constexpr int COLS = 64;
     constexpr int SPLIT = DV / COLS;
@@ -100,43 +100,44 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
         const float kq = s_kq;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            Elem<T>::store(o + (size_t)head * DV + col0 + 4 * cg + j, fmaf(d[j], kq, Y[j]));
+            Elem<TO>::store(o + (size_t)head * DV + col0 + 4 * cg + j, fmaf(d[j], kq, Y[j]));
     }
 }
 
-template <typename T, int DK, int DV>
+template <typename T, typename TO, int DK, int DV>
 static cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* beta,
                                  const float* log_alpha, float* state, void* o, long long NH,
                                  cudaStream_t stream)
 {
     const long long blocks = NH * (DV / 64);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    decode_step_kernel<T, DK, DV><<<(unsigned)blocks, 256, 0, stream>>>(
+    decode_step_kernel<T, TO, DK, DV><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), beta,
-        log_alpha, state, static_cast<T*>(o));
+        log_alpha, state, static_cast<TO*>(o));
     return cudaGetLastError();
+}
+
+template <typename T, typename TO>
+static cudaError_t decode_dims(const void* q, const void* k, const void* v, const float* beta,
+                               const float* log_alpha, float* state, void* o, long long NH, int dk,
+                               int dv, cudaStream_t s)
+{
+    if (dk == 128 && dv == 128) return launch_decode<T, TO, 128, 128>(q, k, v, beta, log_alpha, state, o, NH, s);
+    if (dk == 128 && dv == 64) return launch_decode<T, TO, 128, 64>(q, k, v, beta, log_alpha, state, o, NH, s);
+    if (dk == 64 && dv == 128) return launch_decode<T, TO, 64, 128>(q, k, v, beta, log_alpha, state, o, NH, s);
+    if (dk == 64 && dv == 64) return launch_decode<T, TO, 64, 64>(q, k, v, beta, log_alpha, state, o, NH, s);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t decode_step(const void* q, const void* k, const void* v, const float* beta,
                         const float* log_alpha, float* state, void* o, long long NH, int dk,
-                        int dv, kda_dtype dtype, cudaStream_t stream)
+                        int dv, kda_dtype dtype, kda_dtype o_dtype, cudaStream_t s)
 {
-#define KDA_DECODE_CASE(TT, DK_, DV_)                                                         \
-    if (dk == DK_ && dv == DV_)                                                               \
-        return launch_decode<TT, DK_, DV_>(q, k, v, beta, log_alpha, state, o, NH, stream);
-    if (dtype == KDA_BF16) {
-        KDA_DECODE_CASE(__nv_bfloat16, 128, 128)
-        KDA_DECODE_CASE(__nv_bfloat16, 128, 64)
-        KDA_DECODE_CASE(__nv_bfloat16, 64, 128)
-        KDA_DECODE_CASE(__nv_bfloat16, 64, 64)
-    } else {
-        KDA_DECODE_CASE(float, 128, 128)
-        KDA_DECODE_CASE(float, 128, 64)
-        KDA_DECODE_CASE(float, 64, 128)
-        KDA_DECODE_CASE(float, 64, 64)
-    }
-#undef KDA_DECODE_CASE
-    return cudaErrorInvalidValue;
+    using bf = __nv_bfloat16;
+    if (dtype == KDA_BF16 && o_dtype == KDA_BF16) return decode_dims<bf, bf>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, s);
+    if (dtype == KDA_BF16 && o_dtype == KDA_F32) return decode_dims<bf, float>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, s);
+    if (dtype == KDA_F32 && o_dtype == KDA_BF16) return decode_dims<float, bf>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, s);
+    return decode_dims<float, float>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, s);
 }
 
 }  // namespace kda

@@ -18,7 +18,9 @@
  *  - Every tensor pointer is a DEVICE pointer owned by the caller; the library
  *    allocates no device memory and keeps no pointer after the call returns.
  *  - Layouts are dense, row-major, token-major ("[B, T, H, d]": d fastest).
- *  - q, k, v and o have the element type `dtype` (KDA_BF16 or KDA_F32);
+ *  - q, k and v have the element type `dtype` (KDA_BF16 or KDA_F32); the
+ *    output o has the element type `o_dtype` (either, independently; KDA_F32
+ *    keeps the fp32 accumulation, KDA_BF16 rounds it to nearest even);
  *    beta, log_alpha and all states are always fp32.  log_alpha must be <= 0
  *    (alpha in (0, 1]); it is not checked on the device.
  *  - Every pointer must be 16-byte aligned.
@@ -68,7 +70,7 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
  *   beta        [B, T, H]      fp32, write strength in (0, 1)
  *   log_alpha   [B, T, H, dk]  fp32, per-channel log forget gate (<= 0)
  *   initial_state [B, H, dk, dv] fp32, or NULL for zeros (read only)
- *   o           [B, T, H, dv]  dtype, written
+ *   o           [B, T, H, dv]  o_dtype, written
  *   final_state [B, H, dk, dv] fp32, or NULL if not wanted; written.  It may
  *               alias initial_state (in-place state update).
  *   B >= 0, T >= 0 (B*T == 0 is a no-op that still writes final_state from
@@ -78,14 +80,15 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          const float* beta, const float* log_alpha,
                          const float* initial_state, void* o, float* final_state,
                          int B, int T, int H, int dk, int dv, int chunk,
-                         kda_dtype dtype, void* stream);
+                         kda_dtype dtype, kda_dtype o_dtype, void* stream);
 
 /*
  * Same computation over N variable-length sequences packed along one token
  * axis (B = 1).  The state restarts (from initial_state[n] or zero) at every
  * sequence boundary; the last chunk of each sequence may be shorter than 64.
  *
- *   q, k [T, H, dk], v [T, H, dv], beta [T, H], log_alpha [T, H, dk], o [T, H, dv]
+ *   q, k [T, H, dk], v [T, H, dv] (dtype), beta [T, H], log_alpha [T, H, dk],
+ *   o [T, H, dv] (o_dtype)
  *   cu_seqlens  [N + 1] int32, DEVICE pointer, cu_seqlens[0] = 0,
  *               non-decreasing, cu_seqlens[N] = T (not checked on the device;
  *               a violation is undefined behaviour).
@@ -97,7 +100,7 @@ kda_status kda_varlen_fwd(const void* q, const void* k, const void* v,
                           const int32_t* cu_seqlens, int N,
                           const float* initial_state, void* o, float* final_state,
                           int T, int H, int dk, int dv, int chunk,
-                          kda_dtype dtype, void* stream);
+                          kda_dtype dtype, kda_dtype o_dtype, void* stream);
 
 /*
  * One decode step of the recurrence for N independent sequences (one new
@@ -109,13 +112,13 @@ kda_status kda_varlen_fwd(const void* q, const void* k, const void* v,
  *   q, k [N, H, dk], v [N, H, dv]  dtype
  *   beta [N, H], log_alpha [N, H, dk]  fp32
  *   state [N, H, dk, dv] fp32, read and overwritten in place
- *   o [N, H, dv] dtype, written
+ *   o [N, H, dv] o_dtype, written
  */
 kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
                               const float* beta, const float* log_alpha,
                               float* state, void* o,
                               int N, int H, int dk, int dv,
-                              kda_dtype dtype, void* stream);
+                              kda_dtype dtype, kda_dtype o_dtype, void* stream);
 
 /*
  * Synchronises `stream` and reports (then clears) the current device's

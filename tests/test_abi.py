@@ -38,19 +38,20 @@ P = 256  # a 16-byte aligned fake address: never dereferenced, validation fails 
 
 @pytest.mark.parametrize("args,want", [
     # negative sizes
-    ((P, P, P, P, P, None, P, None, -1, 8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
-    ((P, P, P, P, P, None, P, None, 1, -8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
-    ((P, P, P, P, P, None, P, None, 1, 8, 0, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, None, P, None, -1, 8, 2, 128, 128, 64, 1, 0, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, None, P, None, 1, -8, 2, 128, 128, 64, 1, 0, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, None, P, None, 1, 8, 0, 128, 128, 64, 1, 0, None), _lib.KDA_ERR_INVALID_ARG),
     # null or misaligned tensors
-    ((None, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
-    ((P + 4, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
-    ((P, P, P, P, P, P + 8, P, None, 1, 8, 2, 128, 128, 64, 1, None), _lib.KDA_ERR_INVALID_ARG),
+    ((None, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 1, 0, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P + 4, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 1, 0, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, P + 8, P, None, 1, 8, 2, 128, 128, 64, 1, 0, None), _lib.KDA_ERR_INVALID_ARG),
     # bad dtype code
-    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 7, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 7, 0, None), _lib.KDA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 1, 5, None), _lib.KDA_ERR_INVALID_ARG),
     # unsupported sizes
-    ((P, P, P, P, P, None, P, None, 1, 8, 2, 96, 128, 64, 1, None), _lib.KDA_ERR_UNSUPPORTED),
-    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 256, 64, 1, None), _lib.KDA_ERR_UNSUPPORTED),
-    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 32, 1, None), _lib.KDA_ERR_UNSUPPORTED),
+    ((P, P, P, P, P, None, P, None, 1, 8, 2, 96, 128, 64, 1, 0, None), _lib.KDA_ERR_UNSUPPORTED),
+    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 256, 64, 1, 0, None), _lib.KDA_ERR_UNSUPPORTED),
+    ((P, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 32, 1, 0, None), _lib.KDA_ERR_UNSUPPORTED),
 ])
 def test_chunk_fwd_validation(args, want):
     assert _lib.load().kda_chunk_fwd(*args) == want
@@ -58,7 +59,7 @@ def test_chunk_fwd_validation(args, want):
 
 def test_varlen_validation():
     f = _lib.load().kda_varlen_fwd
-    base = [P, P, P, P, P, P, 4, None, P, None, 100, 2, 128, 128, 64, 1, None]
+    base = [P, P, P, P, P, P, 4, None, P, None, 100, 2, 128, 128, 64, 1, 0, None]
     assert f(*base[:6], -1, *base[7:]) == _lib.KDA_ERR_INVALID_ARG          # N < 0
     assert f(*base[:6], 70000, *base[7:]) == _lib.KDA_ERR_INVALID_ARG       # N too large
     assert f(*base[:5], None, *base[6:]) == _lib.KDA_ERR_INVALID_ARG        # no cu_seqlens
@@ -69,11 +70,12 @@ def test_varlen_validation():
 
 def test_recurrent_step_validation():
     f = _lib.load().kda_recurrent_step
-    assert f(P, P, P, P, P, P, P, -1, 2, 128, 128, 1, None) == _lib.KDA_ERR_INVALID_ARG
-    assert f(P, P, P, P, P, None, P, 3, 2, 128, 128, 1, None) == _lib.KDA_ERR_INVALID_ARG
-    assert f(P, P, P, P, P, P, P + 4, 3, 2, 128, 128, 1, None) == _lib.KDA_ERR_INVALID_ARG
-    assert f(P, P, P, P, P, P, P, 3, 2, 128, 32, 1, None) == _lib.KDA_ERR_UNSUPPORTED
-    assert f(None, None, None, None, None, None, None, 0, 2, 128, 128, 1, None) == _lib.KDA_OK
+    assert f(P, P, P, P, P, P, P, -1, 2, 128, 128, 1, 0, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f(P, P, P, P, P, None, P, 3, 2, 128, 128, 1, 0, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f(P, P, P, P, P, P, P + 4, 3, 2, 128, 128, 1, 0, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f(P, P, P, P, P, P, P, 3, 2, 128, 32, 1, 0, None) == _lib.KDA_ERR_UNSUPPORTED
+    assert f(P, P, P, P, P, P, P, 3, 2, 128, 128, 1, 9, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f(None, None, None, None, None, None, None, 0, 2, 128, 128, 1, 0, None) == _lib.KDA_OK
 
 
 def test_python_binding_rejects_bad_tensors():

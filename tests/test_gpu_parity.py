@@ -176,3 +176,47 @@ def test_decode_steps_equal_chunk_forward():
     torch.cuda.synchronize()
     assert norm_max_err(f64(o_dec), f64(o_chk)) <= 1e-4
     assert norm_max_err(f64(state), f64(s_chk)) <= 1e-4
+
+
+def test_bf16_output_is_the_rounded_fp32_output():
+    """o_dtype=bf16 stores exactly the fp32 result rounded to nearest even."""
+    w = Workload("case", "dense", 2, 150, 3, 128, 128, "bf16", -3.0, 0.02, seed=25)
+    d = _to(make_inputs(w, "cpu"), DEV)
+    args = (d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], d["initial_state"])
+    o32, s32 = kda.kda_chunk_fwd(*args)
+    o16, s16 = kda.kda_chunk_fwd(*args, o_dtype=torch.bfloat16)
+    lens = [70, 0, 130]
+    v = _to(_varlen_case(lens, 2, 128, "bf16", 26), DEV)
+    vargs = (v["q"], v["k"], v["v"], v["beta"], v["log_alpha"], v["cu_seqlens"], v["initial_state"])
+    vo32, _ = kda.kda_varlen_fwd(*vargs)
+    vo16, _ = kda.kda_varlen_fwd(*vargs, o_dtype=torch.bfloat16)
+    x = _to(make_inputs(Workload("dec", "decode", 4, 1, 2, 128, 128, "bf16", -3.0, 0.02, seed=27), "cpu"), DEV)
+    st_a, st_b = x["initial_state"].clone(), x["initial_state"].clone()
+    dargs = tuple(x[n][0] for n in ("q", "k", "v", "beta", "log_alpha"))
+    do32 = kda.kda_recurrent_step(*dargs, st_a)
+    do16 = kda.kda_recurrent_step(*dargs, st_b, o_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert o16.dtype == torch.bfloat16 and torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(s16, s32)
+    assert torch.equal(vo16, vo32.to(torch.bfloat16))
+    assert torch.equal(do16, do32.to(torch.bfloat16)) and torch.equal(st_a, st_b)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_tensor_core_and_cuda_core_kernels_agree(monkeypatch, d):
+    """bf16 inputs go to the tcgen05 kernel; KDA_FORCE_SIMT=1 sends them to the
+    CUDA-core kernel.  Both meet the bar against the oracle and agree closely."""
+    w = Workload("case", "dense", 2, 333, 2, d, d, "bf16", -1.0, 0.05, seed=28)
+    d_cpu = make_inputs(w, "cpu")
+    g = _to(d_cpu, DEV)
+    args = (g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"])
+    o_tc, s_tc = kda.kda_chunk_fwd(*args)
+    monkeypatch.setenv("KDA_FORCE_SIMT", "1")
+    o_cc, s_cc = kda.kda_chunk_fwd(*args)
+    torch.cuda.synchronize()
+    o_ref, s_ref = _dense_oracle(d_cpu, 2, 333)
+    flat = lambda t: f64(t).reshape(2 * 333, 2, d)
+    assert norm_max_err(flat(o_tc), o_ref) <= TOL_BF16
+    assert norm_max_err(flat(o_cc), o_ref) <= 1e-4
+    assert norm_max_err(f64(s_tc), s_ref) <= TOL_BF16
+    assert norm_max_err(f64(s_cc), s_ref) <= 1e-4
