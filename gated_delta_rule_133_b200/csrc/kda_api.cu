@@ -8,6 +8,7 @@
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool supported_d(int d) { return d == 64 || d == 128; }
 
@@ -53,7 +54,7 @@ kda_status check_fwd(const void* q, const void* k, const void* v, const float* b
     if (!valid_dtype(dtype) || !valid_dtype(o_dtype)) return KDA_ERR_INVALID_ARG;
     if (tokens > 0) {
         if (!q || !k || !v || !beta || !log_alpha || !o) return KDA_ERR_INVALID_ARG;
-        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) ||
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(beta) ||
             !aligned16(log_alpha) || !aligned16(o))
             return KDA_ERR_INVALID_ARG;
     }
@@ -118,7 +119,7 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
     if (!valid_dtype(dtype) || !valid_dtype(o_dtype)) return KDA_ERR_INVALID_ARG;
     if (N == 0) return KDA_OK;
     if (!q || !k || !v || !beta || !log_alpha || !state || !o) return KDA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) ||
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(beta) ||
         !aligned16(log_alpha) || !aligned16(state) || !aligned16(o))
         return KDA_ERR_INVALID_ARG;
     if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_UNSUPPORTED;

@@ -58,7 +58,8 @@ struct Params {
 //   R1: A1 [128][d_k] until MMAs PA and X complete; then P [64][64] (0),
 //       T^T [64][64] (16 KB), the fp32 inversion scratch A (32 KB) and X (~48 KB);
 //       PT [64][64] reuses P's place once MMA PT completes.
-//   R2: B1 [64][d_k] until MMA Z completes; then Z [128][64].
+//   R2: B1 [64][d_k] until MMA PA completes; then its transpose B1^T [128][64]
+//       until MMA Z completes; then Z [128][64].
 //   R3: the state operand [64][d_k] until MMA X completes; then Y [64][64].
 //   STG: TMA staging of q, k (bf16) and log alpha (fp32) for the next chunk.
 struct Plan {
@@ -213,6 +214,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     float* As = reinterpret_cast<float*>(sm + PL::AS);
     float* Xs = reinterpret_cast<float*>(sm + PL::XS);
     unsigned char* B1 = sm + PL::R2;
+    unsigned char* KBt = sm + PL::R2;
     unsigned char* Zb = sm + PL::R2;
     unsigned char* Smb = sm + PL::R3;
     unsigned char* Yb = sm + PL::R3;
@@ -285,7 +287,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     int tma_pending = 0, tma_parity = 0, mma_pending = 0;
     constexpr uint32_t kStageBytes = (uint32_t)C * DK * (2 + 2 + 4);
     constexpr uint32_t kI = idesc_tf32(128, 64, 0, 0);
-    constexpr uint32_t kI_AMN = idesc_tf32(128, 64, 1, 0);
     constexpr int kA1 = 128 * 128;   // atom-column strides (bytes) of the 128-row and 64-row tiles
     constexpr int kR64 = 64 * 128;
 
@@ -408,6 +409,15 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                 }
             }
         }
+        // ---- B1 is no longer needed as [s][c]: rewrite it in place as the
+        // K-major operand B1^T [c][s] (thread = key channel = row)
+        {
+            float kb[C];
+#pragma unroll
+            for (int s2 = 0; s2 < C; ++s2) kb[s2] = tid < DK ? swf(B1, s2, tid, C) : 0.f;
+            __syncthreads();
+            st_row_swf<16>(KBt, tid, 0, 128, kb);
+        }
         __syncthreads();
 
         // ---- UT transform into the T^T operand tile
@@ -418,9 +428,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)    // Z' = B1^T T   (B1 read MN-major)
-                umma_tf32(t_Z, sdesc_sw128(smem_u32(B1) + kk * 1024, kR64, 1024), kdesc(Top, kk, kR64), kI_AMN,
-                          kk > 0);
+            for (int kk = 0; kk < C / 8; ++kk)    // Z' = B1^T T
+                umma_tf32(t_Z, kdesc(KBt, kk, kA1), kdesc(Top, kk, kR64), kI, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk)    // PT = P T  (rows 64..127 unused)
                 umma_tf32(t_PT, kdesc(Pb, kk, kR64), kdesc(Top, kk, kR64), kI, kk > 0);

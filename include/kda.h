@@ -23,7 +23,8 @@
  *    keeps the fp32 accumulation, KDA_BF16 rounds it to nearest even);
  *    beta, log_alpha and all states are always fp32.  log_alpha must be <= 0
  *    (alpha in (0, 1]); it is not checked on the device.
- *  - Every pointer must be 16-byte aligned.
+ *  - Every tensor pointer must be 16-byte aligned, except beta and
+ *    cu_seqlens (4-byte aligned).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
  *    asynchronous on that stream and never synchronise.
  *  - Argument errors are reported synchronously (nothing is launched).  A

@@ -73,6 +73,7 @@ def test_recurrent_step_validation():
     assert f(P, P, P, P, P, P, P, -1, 2, 128, 128, 1, 0, None) == _lib.KDA_ERR_INVALID_ARG
     assert f(P, P, P, P, P, None, P, 3, 2, 128, 128, 1, 0, None) == _lib.KDA_ERR_INVALID_ARG
     assert f(P, P, P, P, P, P, P + 4, 3, 2, 128, 128, 1, 0, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f(P, P, P, P + 2, P, P, P, 3, 2, 128, 128, 1, 0, None) == _lib.KDA_ERR_INVALID_ARG  # beta: 4-byte
     assert f(P, P, P, P, P, P, P, 3, 2, 128, 32, 1, 0, None) == _lib.KDA_ERR_UNSUPPORTED
     assert f(P, P, P, P, P, P, P, 3, 2, 128, 128, 1, 9, None) == _lib.KDA_ERR_INVALID_ARG
     assert f(None, None, None, None, None, None, None, 0, 2, 128, 128, 1, 0, None) == _lib.KDA_OK
