@@ -39,8 +39,8 @@ using namespace sm100;
 
 constexpr int C = 64;      // chunk length
 constexpr int NV = 64;     // value columns per CTA
-constexpr int NT = 128;    // threads per CTA
-constexpr int LDA = 65;    // fp32 pitch of the inversion scratch
+constexpr int NT = 256;    // threads per CTA: two warpgroups
+constexpr int LDA = 65;    // fp32 pitch of the UT-transform scratch
 
 struct Params {
     const __nv_bfloat16* v;
@@ -53,27 +53,33 @@ struct Params {
     long long timeout_cycles;
 };
 
-// Shared-memory plan (byte offsets from a 1024-aligned base).  Every operand
-// tile is fp32 in the K-major 128-byte-swizzled layout.
-//   R1: A1 [128][d_k] until MMAs PA and X complete; then P [64][64] (0),
-//       T^T [64][64] (16 KB), the fp32 inversion scratch A (32 KB) and X (~48 KB);
-//       PT [64][64] reuses P's place once MMA PT completes.
-//   R2: B1 [64][d_k] until MMA PA completes; then its transpose B1^T [128][64]
-//       until MMA Z completes; then Z [128][64].
-//   R3: the state operand [64][d_k] until MMA X completes; then Y [64][64].
-//   STG: TMA staging of q, k (bf16) and log alpha (fp32) for the next chunk.
+// Shared-memory plan (byte offsets from a 1024-aligned base).  Operand tiles
+// are fp32 in the K-major 128-byte-swizzled layout, rounded to tf32.
+//   R1: A1 [128][d_k] until MMA [PA|X] completes; then P [64][64] (0),
+//       T^T [64][64] (16 KB) and the fp32 UT scratch (A below the diagonal,
+//       T transposed on and above it; 32 KB) plus a 32 x 33 product scratch;
+//       PT [64][64] takes P's place once MMA PT completes.
+//   R2: the 128-row B operand of MMA [PA|X]: rows 0..63 = B1 = k F, rows
+//       64..127 = the state operand (diag(exp(G_m)) S)^T, [128][d_k].  Then
+//       B1^T [128][64] (first 32 KB) until MMA Z completes, then Z there;
+//       Y [64][64] at +32 KB.
+//   STG: TMA staging of q, k (bf16) and log alpha (fp32); the gate cumsum G
+//       overwrites log alpha in place.
+//   VEC: per-chunk channel vectors, double-buffered (the next chunk's are
+//       computed while this chunk's last MMAs run).
 struct Plan {
     static constexpr int R1 = 0;
     static constexpr int P = R1, TOP = R1 + 16384, AS = R1 + 32768, XS = AS + C * LDA * 4;
     static constexpr int R2 = 65536;
-    static constexpr int R3 = 98304;
+    static constexpr int KBT = R2, Y = R2 + 32768;
     static constexpr int STG = 131072;
-    static constexpr int VEC = STG + 65536;        // gm[128] gam[128] glm[128] beta[64]
-    static constexpr int BAR = VEC + (3 * 128 + 64) * 4;
-    static constexpr int END = BAR + 64;
-    static constexpr int BYTES = END + 1024;       // + alignment slack
+    static constexpr int VEC = STG + 65536;         // 2 x {gml gm gam glm htot [128], beta[64]}
+    static constexpr int VECN = 5 * 128 + 64;       // floats per buffer
+    static constexpr int BAR = VEC + 2 * VECN * 4;
+    static constexpr int END = BAR + 128;
+    static constexpr int BYTES = END + 1024;        // + alignment slack
 };
-static_assert(Plan::XS + 32 * 33 * 4 <= Plan::R2, "inversion scratch overflows R1");
+static_assert(Plan::XS + 32 * 33 * 4 <= Plan::R2, "UT scratch overflows R1");
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* p)
 {
@@ -101,88 +107,96 @@ __device__ int seq_by_rank(const int32_t* cu, int N, int rank, int* slot)
     return n;
 }
 
-// T[s][j], stored transposed in the K-major operand tile (row j, column s).
-__device__ __forceinline__ float& Tat(unsigned char* Top, int s, int j) { return swf(Top, j, s, C); }
-
-// T = (I + A)^-1 for the strictly lower 64 x 64 A in `As` (fp32, pitch 65),
-// written into the operand tile Top (zeros above the diagonal).  Diagonal
-// 16 x 16 blocks by forward substitution (one warp per block, one lane per
-// column), then T10 = -T11 A10 T00, T32 = -T33 A32 T22, and the lower-left
-// 32 x 32 block -T_BB A_BA T_AA.
-__device__ __forceinline__ void invert_unit_lower(const float* As, unsigned char* Top, float* X)
+// 1/x for normal x by Newton-Raphson on the FMA pipe (keeps the exponent
+// unit free for exp): seed from the exponent bits (relative error < 5.1 %),
+// two iterations (< 1e-5, below tf32 resolution).
+__device__ __forceinline__ float rcp_nr(float x)
 {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int e = tid; e < C * C / 4; e += NT) reinterpret_cast<float4*>(Top)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    __syncthreads();
-    {
-        const int j = lane & 15, b0 = 16 * warp;
+    float y = __int_as_float(0x7EF311C3 - __float_as_int(x));
+    y = y * fmaf(-x, y, 2.f);
+    y = y * fmaf(-x, y, 2.f);
+    return y;
+}
+
+// T[k][j] of the unit lower-triangular T, kept transposed in the upper
+// triangle (diagonal included) of the UT scratch.
+__device__ __forceinline__ float Tget(const float* As, int k, int j) { return k >= j ? As[j * LDA + k] : 0.f; }
+
+// UT transform.  On entry As[r*LDA + s] (s < r) holds the strictly lower A;
+// on return As[j*LDA + s] (s >= j) holds T[s][j], T = (I + A)^-1, with A left
+// intact below the diagonal.  Diagonal 16x16 blocks by column-sweep forward
+// substitution (one lane per column), then T10 = -T11 A10 T00,
+// T32 = -T33 A32 T22 and the lower-left 32x32 block -T_BB A_BA T_AA.
+__device__ __forceinline__ void ut_transform(float* As, float* X)
+{
+    const int tid = threadIdx.x;
+    if (tid < 64) {
+        const int b0 = 16 * (tid >> 4), j = tid & 15;
         float x[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = 0.f;
+        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int s = 0; s < r; ++s) acc = fmaf(As[(b0 + r) * LDA + b0 + s], x[s], acc);
-            x[r] = (r == j) ? 1.f : (r < j ? 0.f : -acc);
-        }
-        if (lane < 16) {
+        for (int s = 0; s < 15; ++s) {
+            const float xs = x[s];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) Tat(Top, b0 + r, b0 + j) = x[r];
+            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-As[(b0 + r) * LDA + b0 + s], xs, x[r]);
         }
+#pragma unroll
+        for (int r = 0; r < 16; ++r)
+            if (r >= j) As[(b0 + j) * LDA + b0 + r] = x[r];
     }
     __syncthreads();
     {
-        const int blk = tid >> 6, i = (tid & 63) >> 2, j0 = (tid & 3) * 4;
+        const int blk = tid >> 7, i = (tid & 127) >> 3, j0 = (tid & 7) * 2;
         const int rb = blk ? 48 : 16, cb = blk ? 32 : 0;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int k = 0; k < 16; ++k) {
-            const float a = As[(rb + i) * LDA + cb + k];
+        float a0 = 0.f, a1 = 0.f, b0_ = 0.f, b1 = 0.f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) acc[q] = fmaf(a, Tat(Top, cb + k, cb + j0 + q), acc[q]);
+        for (int k = 0; k < 16; k += 2) {
+            const float u0 = As[(rb + i) * LDA + cb + k], u1 = As[(rb + i) * LDA + cb + k + 1];
+            a0 = fmaf(u0, Tget(As, cb + k, cb + j0), a0);
+            a1 = fmaf(u0, Tget(As, cb + k, cb + j0 + 1), a1);
+            b0_ = fmaf(u1, Tget(As, cb + k + 1, cb + j0), b0_);
+            b1 = fmaf(u1, Tget(As, cb + k + 1, cb + j0 + 1), b1);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) X[(blk * 16 + i) * 33 + j0 + q] = acc[q];
+        X[(blk * 16 + i) * 33 + j0] = a0 + b0_;
+        X[(blk * 16 + i) * 33 + j0 + 1] = a1 + b1;
         __syncthreads();
-        float t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int k = 0; k < 16; ++k) {
-            const float a = Tat(Top, rb + i, rb + k);
+        float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) t[q] = fmaf(a, X[(blk * 16 + k) * 33 + j0 + q], t[q]);
+        for (int k = 0; k < 16; k += 2) {
+            const float w0 = Tget(As, rb + i, rb + k), w1 = Tget(As, rb + i, rb + k + 1);
+            t0 = fmaf(w0, X[(blk * 16 + k) * 33 + j0], t0);
+            t1 = fmaf(w0, X[(blk * 16 + k) * 33 + j0 + 1], t1);
+            t2 = fmaf(w1, X[(blk * 16 + k + 1) * 33 + j0], t2);
+            t3 = fmaf(w1, X[(blk * 16 + k + 1) * 33 + j0 + 1], t3);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) Tat(Top, rb + i, cb + j0 + q) = -t[q];
+        As[(cb + j0) * LDA + rb + i] = -(t0 + t2);
+        As[(cb + j0 + 1) * LDA + rb + i] = -(t1 + t3);
     }
     __syncthreads();
     {
-        const int i = tid >> 2, j0 = (tid & 3) * 8;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+        const int i = tid >> 3, j0 = (tid & 7) * 4;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
         for (int k = 0; k < 32; ++k) {
             const float a = As[(32 + i) * LDA + k];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) acc[q] = fmaf(a, Tat(Top, k, j0 + q), acc[q]);
+            for (int q = 0; q < 4; ++q) acc[k & 1][q] = fmaf(a, Tget(As, k, j0 + q), acc[k & 1][q]);
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) X[i * 33 + j0 + q] = acc[q];
+        for (int q = 0; q < 4; ++q) X[i * 33 + j0 + q] = acc[0][q] + acc[1][q];
         __syncthreads();
-        float t[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int k = 0; k < 32; ++k) {
-            const float a = Tat(Top, 32 + i, 32 + k);
+        float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-            for (int q = 0; q < 8; ++q) t[q] = fmaf(a, X[k * 33 + j0 + q], t[q]);
+        for (int k = 0; k < 32; ++k) {
+            const float w = Tget(As, 32 + i, 32 + k);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) t[k & 1][q] = fmaf(w, X[k * 33 + j0 + q], t[k & 1][q]);
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) Tat(Top, 32 + i, j0 + q) = -t[q];
+        for (int q = 0; q < 4; ++q) As[(j0 + q) * LDA + 32 + i] = -(t[0][q] + t[1][q]);
     }
     __syncthreads();
-    // operand rounding to tf32, once the full-precision solve is done
-    for (int e = tid; e < C * C / 4; e += NT) {
-        float4* p4 = reinterpret_cast<float4*>(Top) + e;
-        float4 v = *p4;
-        *p4 = make_float4(tf32r(v.x), tf32r(v.y), tf32r(v.z), tf32r(v.w));
-    }
 }
 
 // K-major fp32 SW128 operand descriptor for MMA k-step kk (K = 8 per step):
@@ -192,11 +206,33 @@ __device__ __forceinline__ uint64_t kdesc(const unsigned char* tile, int kk, int
     return sdesc_sw128(smem_u32(tile) + (kk >> 2) * atom_stride + (kk & 3) * 32, 16, 1024);
 }
 
-// All threads poll; a CTA-wide vote turns any timeout into a common exit.
-#define KDA_WAIT_OR_EXIT(bar, parity)                                                  \
-    do {                                                                               \
-        const bool ok_ = mbar_wait((bar), (parity), abort_flag, p.timeout_cycles);    \
-        if (__syncthreads_or(!ok_)) goto finish;                                       \
+__device__ __forceinline__ float4 bf16x4(const __nv_bfloat16* p)
+{
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ float4 tf32r4(float a, float b, float c, float d)
+{
+    return make_float4(tf32r(a), tf32r(b), tf32r(c), tf32r(d));
+}
+
+// Phase markers: empty in the library build.  A profiling build may define
+// them to accumulate clock64() deltas per chunk stage.
+#ifndef KDA_PHASE
+#define KDA_PHASE_DECL
+#define KDA_PHASE(i) ((void)0)
+#define KDA_PHASE_FLUSH
+#endif
+
+// Every thread polls; a CTA-wide vote turns any timeout into a common exit.
+#define KDA_WAIT_OR_EXIT(bar, bit, parity)                                               \
+    do {                                                                                 \
+        const bool ok_ = mbar_wait((bar), (uint32_t)(parity), abort_flag, p.timeout_cycles); \
+        if (__syncthreads_or(!ok_)) goto finish;                                         \
+        pend &= ~(bit);                                                                  \
     } while (0)
 
 template <typename TO, int DK>
@@ -206,6 +242,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 {
     using PL = Plan;
     extern __shared__ unsigned char smem_raw[];
+    KDA_PHASE_DECL
     unsigned char* sm = align1024(smem_raw);
     unsigned char* A1 = sm + PL::R1;
     unsigned char* Pb = sm + PL::P;
@@ -213,25 +250,26 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     unsigned char* Top = sm + PL::TOP;
     float* As = reinterpret_cast<float*>(sm + PL::AS);
     float* Xs = reinterpret_cast<float*>(sm + PL::XS);
-    unsigned char* B1 = sm + PL::R2;
-    unsigned char* KBt = sm + PL::R2;
-    unsigned char* Zb = sm + PL::R2;
-    unsigned char* Smb = sm + PL::R3;
-    unsigned char* Yb = sm + PL::R3;
+    unsigned char* Bx = sm + PL::R2;            // [B1 ; state operand], 128 rows
+    unsigned char* KBt = sm + PL::KBT;
+    unsigned char* Zb = sm + PL::KBT;
+    unsigned char* Yb = sm + PL::Y;
     const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(sm + PL::STG);
     const __nv_bfloat16* ks = qs + C * DK;
-    const float* gs = reinterpret_cast<const float*>(ks + C * DK);
-    float* gm_s = reinterpret_cast<float*>(sm + PL::VEC);
-    float* gam_s = gm_s + 128;
-    float* glm_s = gam_s + 128;
-    float* beta_s = glm_s + 128;
-    uint64_t* mb_tma = reinterpret_cast<uint64_t*>(sm + PL::BAR);
-    uint64_t* mb_mma = mb_tma + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mb_tma + 2);
+    float* gs = reinterpret_cast<float*>(sm + PL::STG + 2 * C * DK * 2);
+    float* vec0 = reinterpret_cast<float*>(sm + PL::VEC);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::BAR);
+    uint64_t* mb_tma = bars + 0;
+    uint64_t* mb_px = bars + 1;
+    uint64_t* mb_z = bars + 2;
+    uint64_t* mb_zy = bars + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* misc_slot = reinterpret_cast<int*>(tmem_slot + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int lt = tid & 127;          // TMEM lane owned by this thread
+    const int wg = tid >> 7;           // warpgroup: which 32-column half it loads
     const int nslice = p.DV / NV;
     const int slice = blockIdx.x % nslice;
     const int h = (blockIdx.x / nslice) % p.H;
@@ -251,8 +289,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     const int nchunks = (len + C - 1) / C;
 
     if (tid == 0) {
-        mbar_init(mb_tma, 1);
-        mbar_init(mb_mma, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
@@ -268,27 +305,70 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t t_PA = tmem, t_O = tmem + 64, t_Z = tmem + 128, t_PT = tmem + 192, t_dS = tmem + 256;
+    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32) << 16;
+    const uint32_t half_off = (uint32_t)wg * 32;
+    // TMEM columns: [PA | X] 0..127 (O accumulates onto X), Z 128, PT 192, dS 256
+    const uint32_t t_PA = tmem, t_X = tmem + 64, t_Z = tmem + 128, t_PT = tmem + 192, t_dS = tmem + 256;
 
-    // fp32 state: thread c < DK owns row c of this 64-column slice
-    float S[NV];
+    // fp32 state: thread (key channel lt < DK, half wg) owns S[lt][32 wg .. 32 wg + 32)
+    float S[32];
     {
-        const bool own = tid < DK;
-        const float* src = (p.s0 && own) ? p.s0 + (((size_t)n * H + h) * DK + tid) * DV + col0 : nullptr;
+        const bool own = lt < DK;
+        const float* src = (p.s0 && own) ? p.s0 + (((size_t)n * H + h) * DK + lt) * DV + col0 + 32 * wg : nullptr;
 #pragma unroll
-        for (int j = 0; j < NV; j += 4) {
-            float4 v4 = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < 32; j += 4) {
+            const float4 v4 = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
             S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
         }
     }
 
-    uint32_t mma_phase = 0;
-    int tma_pending = 0, tma_parity = 0, mma_pending = 0;
+    unsigned pend = 0;                 // bit i: a completion of bars[i] is outstanding
+    int tma_par = 0;                   // phase parity of the outstanding TMA load
+    int c = 0;
     constexpr uint32_t kStageBytes = (uint32_t)C * DK * (2 + 2 + 4);
-    constexpr uint32_t kI = idesc_tf32(128, 64, 0, 0);
-    constexpr int kA1 = 128 * 128;   // atom-column strides (bytes) of the 128-row and 64-row tiles
+    constexpr uint32_t kI64 = idesc_tf32(128, 64, 0, 0);
+    constexpr uint32_t kI128 = idesc_tf32(128, 128, 0, 0);
+    constexpr int kR128 = 128 * 128;  // atom-column strides (bytes) of 128-row and 64-row tiles
     constexpr int kR64 = 64 * 128;
+    constexpr int NG = DK / 4;        // 4-channel groups per row
+    constexpr int RPP = NT / NG;      // rows per pass of the operand build (8 or 16)
+
+    // gate cumsum of the chunk in the staging buffer (in place), channel
+    // vectors into buffer vb; beta of the chunk (prefetched value) alongside
+    auto cumsum = [&](int Lc, int vb, float beta_v) {
+        float* gml_s = vec0 + vb * PL::VECN;
+        float* gm_s = gml_s + 128;
+        float* gam_s = gm_s + 128;
+        float* glm_s = gam_s + 128;
+        float* htot_s = glm_s + 128;
+        float* beta_s = htot_s + 128;
+        float G[32];
+        if (lt < DK) {
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) {
+                const int row = 32 * wg + rr;
+                G[rr] = row < Lc ? gs[row * DK + lt] : 0.f;
+            }
+#pragma unroll
+            for (int rr = 1; rr < 32; ++rr) G[rr] += G[rr - 1];
+            if (wg == 0) htot_s[lt] = G[31];
+        }
+        if (tid < C) beta_s[tid] = beta_v;
+        __syncthreads();
+        if (lt < DK) {
+            const float off = wg ? htot_s[lt] : 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) gs[(32 * wg + rr) * DK + lt] = G[rr] + off;
+            if (wg == 0) {
+                gml_s[lt] = G[31];
+                gm_s[lt] = expf(G[31]);
+            } else {
+                const float Gl = G[31] + off;
+                gam_s[lt] = expf(Gl);
+                glm_s[lt] = expf(Gl - off);
+            }
+        }
+    };
 
     if (tid == 0 && nchunks > 0) {
         mbar_expect_tx(mb_tma, kStageBytes);
@@ -296,60 +376,71 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tma_load_3d((void*)ks, &tmk, mb_tma, 0, h, tok0);
         tma_load_3d((void*)gs, &tmg, mb_tma, 0, h, tok0);
     }
-    tma_pending = nchunks > 0;
+    if (nchunks > 0) pend |= 1u;
+    tma_par = 0;
     float beta_next = 0.f;
     if (tid < C && tid < len) beta_next = p.beta[(size_t)(tok0 + tid) * H + h];
+    if (nchunks > 0) {
+        KDA_WAIT_OR_EXIT(mb_tma, 1u, 0);
+        cumsum(min(C, len), 0, beta_next);
+        if (tid < C) beta_next = (C + tid < len) ? p.beta[(size_t)(tok0 + C + tid) * H + h] : 0.f;
+        __syncthreads();
+    }
 
-    for (int c = 0; c < nchunks; ++c) {
+    for (c = 0; c < nchunks; ++c) {
         const int L = min(C, len - c * C);
         const int tokc = tok0 + c * C;
+        const float* gml_s = vec0 + (c & 1) * PL::VECN;
+        const float* gm_s = gml_s + 128;
+        const float* gam_s = gm_s + 128;
+        const float* glm_s = gam_s + 128;
+        const float* beta_s = gml_s + 5 * 128;
+        KDA_PHASE(0);
 
-        // values of this chunk for Y (thread 64 + s owns chunk row s), and beta
-        uint4 vraw[8];
+        // values for Y: thread (chunk row s = lt - 64, half wg) owns v[s][32 wg .. + 32)
+        uint4 vraw[4];
         {
-            const int s = tid - C;
-            const bool live = tid >= C && s < L;
-            const uint4* src = live ? reinterpret_cast<const uint4*>(p.v + ((size_t)(tokc + s) * H + h) * DV + col0)
-                                    : nullptr;
+            const int s = lt - C;
+            const bool live = lt >= C && s < L;
+            const uint4* src =
+                live ? reinterpret_cast<const uint4*>(p.v + ((size_t)(tokc + s) * H + h) * DV + col0 + 32 * wg) : nullptr;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) vraw[u] = live ? __ldg(src + u) : make_uint4(0u, 0u, 0u, 0u);
+            for (int u = 0; u < 4; ++u) vraw[u] = live ? __ldg(src + u) : make_uint4(0u, 0u, 0u, 0u);
         }
-        if (tid < C) beta_s[tid] = beta_next;
 
-        tma_parity = c & 1;
-        KDA_WAIT_OR_EXIT(mb_tma, (uint32_t)(c & 1));
-        tma_pending = 0;
-        if (tid < C) beta_next = (c + 1 < nchunks && C + tid < len - c * C)
-                                     ? p.beta[(size_t)(tokc + C + tid) * H + h] : 0.f;
-
-        // ---- gate cumsum in log space (fp32), operands A1, B1 and the state operand
-        if (tid < DK) {
-            float G[C];
+        // ---- operands: A1 = [q E; k E] (R1); B rows 0..63 = k F, rows 64..127 = state (R2)
+        {
+            const int r0 = tid / NG, c0 = (tid % NG) * 4;
+            const float4 m4 = *reinterpret_cast<const float4*>(gml_s + c0);
+            const uint32_t oq = swf_off(r0, c0, 128), ok = swf_off(C + r0, c0, 128), ob = swf_off(r0, c0, 128);
 #pragma unroll
-            for (int r = 0; r < C; ++r) G[r] = (r < L) ? gs[r * DK + tid] : 0.f;
-#pragma unroll
-            for (int r = 1; r < C; ++r) G[r] += G[r - 1];
-            const float Gm = G[C / 2 - 1], Gl = G[C - 1];
-            const float egm = expf(Gm);
-            gm_s[tid] = egm;
-            gam_s[tid] = expf(Gl);
-            glm_s[tid] = expf(Gl - Gm);
-#pragma unroll
-            for (int r = 0; r < C; ++r) {
-                const float e = __expf(fminf(G[r] - Gm, 80.f));
-                const float f = __expf(fminf(Gm - G[r], 80.f));
-                const bool live = r < L;
-                const float qv = live ? __bfloat162float(qs[r * DK + tid]) : 0.f;
-                const float kv = live ? __bfloat162float(ks[r * DK + tid]) : 0.f;
-                swf(A1, r, tid, 128) = tf32r(qv * e);
-                swf(A1, C + r, tid, 128) = tf32r(kv * e);
-                swf(B1, r, tid, C) = tf32r(kv * f);
+            for (int i = 0; i < C / RPP; ++i) {
+                const int r = r0 + RPP * i;
+                const float4 g4 = *reinterpret_cast<const float4*>(gs + r * DK + c0);
+                float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = q4;
+                if (r < L) {
+                    q4 = bf16x4(qs + r * DK + c0);
+                    k4 = bf16x4(ks + r * DK + c0);
+                }
+                const float e0 = __expf(fminf(fmaxf(g4.x - m4.x, -80.f), 80.f));
+                const float e1 = __expf(fminf(fmaxf(g4.y - m4.y, -80.f), 80.f));
+                const float e2 = __expf(fminf(fmaxf(g4.z - m4.z, -80.f), 80.f));
+                const float e3 = __expf(fminf(fmaxf(g4.w - m4.w, -80.f), 80.f));
+                const uint32_t step = (uint32_t)(RPP * 128 * i);
+                *reinterpret_cast<float4*>(A1 + oq + step) = tf32r4(q4.x * e0, q4.y * e1, q4.z * e2, q4.w * e3);
+                *reinterpret_cast<float4*>(A1 + ok + step) = tf32r4(k4.x * e0, k4.y * e1, k4.z * e2, k4.w * e3);
+                *reinterpret_cast<float4*>(Bx + ob + step) =
+                    tf32r4(k4.x * rcp_nr(e0), k4.y * rcp_nr(e1), k4.z * rcp_nr(e2), k4.w * rcp_nr(e3));
             }
+        }
+        if (lt < DK) {
+            const float sc = gm_s[lt];
 #pragma unroll
-            for (int j = 0; j < NV; ++j) swf(Smb, j, tid, NV) = tf32r(egm * S[j]);
+            for (int jj = 0; jj < 32; ++jj) swf(Bx, C + 32 * wg + jj, lt, 128) = tf32r(sc * S[jj]);
         }
         fence_proxy_async();
         __syncthreads();
+        KDA_PHASE(1);
 
         if (tid == 0) {
             if (c + 1 < nchunks) {  // staging is free again: fetch the next chunk
@@ -360,143 +451,156 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < DK / 8; ++kk)   // [P ; A~] = A1 B1^T
-                umma_tf32(t_PA, kdesc(A1, kk, kA1), kdesc(B1, kk, kR64), kI, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < DK / 8; ++kk)   // X = A1 (diag(exp(G_m)) S)
-                umma_tf32(t_O, kdesc(A1, kk, kA1), kdesc(Smb, kk, kR64), kI, kk > 0);
-            umma_commit(mb_mma);
+            for (int kk = 0; kk < DK / 8; ++kk)   // [P ; A~ | X] = A1 [B1 ; state]^T
+                umma_tf32(t_PA, kdesc(A1, kk, kR128), kdesc(Bx, kk, kR128), kI128, kk > 0);
+            umma_commit(mb_px);
         }
-        tma_pending = c + 1 < nchunks;
-        tma_parity = (c + 1) & 1;
-        mma_pending = 1;
-        KDA_WAIT_OR_EXIT(mb_mma, mma_phase & 1);
-        ++mma_phase;
-        mma_pending = 0;
+        if (c + 1 < nchunks) {
+            pend |= 1u;
+            tma_par = (c + 1) & 1;
+        }
+        pend |= 2u;
+        KDA_WAIT_OR_EXIT(mb_px, 2u, c & 1);
         tc_fence_after();
+        KDA_PHASE(2);
 
-        // ---- P (lanes 0..63), A (lanes 64..127), Y (lanes 64..127 of X)
+        // ---- P (lanes 0..63, lower incl.) and A = beta A~ (lanes 64..127, strictly lower)
         {
-            float acc[64];
-            tmem_ld64(t_PA + lane_off, acc);
+            float pa[32];
+            tmem_ld32(t_PA + lane_off + half_off, pa);
             tmem_wait_ld();
-            if (tid < C) {
-                const int r = tid;
+            if (lt < C) {
+                const int r = lt;
 #pragma unroll
-                for (int s = 0; s < C; ++s) acc[s] = s <= r ? acc[s] : 0.f;
-                st_row_swf<16>(Pb, r, 0, C, acc);
+                for (int s2 = 0; s2 < 32; ++s2) pa[s2] = (32 * wg + s2 <= r) ? pa[s2] : 0.f;
+                st_row_swf<8>(Pb, r, 32 * wg, C, pa);
             } else {
-                const int r = tid - C;
+                const int r = lt - C;
                 const float b = beta_s[r];
 #pragma unroll
-                for (int s = 0; s < C; ++s) As[r * LDA + s] = s < r ? b * acc[s] : 0.f;
-            }
-            tmem_ld64(t_O + lane_off, acc);
-            tmem_wait_ld();
-            if (tid >= C) {
-                const int s = tid - C;
-                const float b = beta_s[s];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vraw[u]);
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const float2 f2 = __bfloat1622float2(v2[w]);
-                        const int j = u * 8 + w * 2;
-                        swf(Yb, j, s, NV) = tf32r(b * (f2.x - acc[j]));
-                        swf(Yb, j + 1, s, NV) = tf32r(b * (f2.y - acc[j + 1]));
-                    }
-                }
+                for (int s2 = 0; s2 < 32; ++s2) As[r * LDA + 32 * wg + s2] = (32 * wg + s2 < r) ? b * pa[s2] : 0.f;
             }
         }
-        // ---- B1 is no longer needed as [s][c]: rewrite it in place as the
-        // K-major operand B1^T [c][s] (thread = key channel = row)
+        // ---- B1 -> B1^T [c][s] (first 32 KB of R2), read fully before any write
         {
-            float kb[C];
+            float kb[32];
 #pragma unroll
-            for (int s2 = 0; s2 < C; ++s2) kb[s2] = tid < DK ? swf(B1, s2, tid, C) : 0.f;
+            for (int s2 = 0; s2 < 32; ++s2) kb[s2] = lt < DK ? swf(Bx, 32 * wg + s2, lt, 128) : 0.f;
             __syncthreads();
-            st_row_swf<16>(KBt, tid, 0, 128, kb);
+            st_row_swf<8>(KBt, lt, 32 * wg, 128, kb);
         }
-        __syncthreads();
+        KDA_PHASE(3);
 
-        // ---- UT transform into the T^T operand tile
-        invert_unit_lower(As, Top, Xs);
+        // ---- UT transform, then T^T into the operand tile (row j, column s)
+        ut_transform(As, Xs);
+        {
+            const int j = tid >> 2, c4 = (tid & 3) * 16;
+            float x[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) x[u] = (c4 + u >= j) ? As[j * LDA + c4 + u] : 0.f;
+            st_row_swf<4>(Top, j, c4, C, x);
+        }
         fence_proxy_async();
         __syncthreads();
+        KDA_PHASE(4);
 
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk)    // Z' = B1^T T
-                umma_tf32(t_Z, kdesc(KBt, kk, kA1), kdesc(Top, kk, kR64), kI, kk > 0);
+                umma_tf32(t_Z, kdesc(KBt, kk, kR128), kdesc(Top, kk, kR64), kI64, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk)    // PT = P T  (rows 64..127 unused)
-                umma_tf32(t_PT, kdesc(Pb, kk, kR64), kdesc(Top, kk, kR64), kI, kk > 0);
-            umma_commit(mb_mma);
+                umma_tf32(t_PT, kdesc(Pb, kk, kR64), kdesc(Top, kk, kR64), kI64, kk > 0);
+            umma_commit(mb_z);
         }
-        mma_pending = 1;
-        KDA_WAIT_OR_EXIT(mb_mma, mma_phase & 1);
-        ++mma_phase;
-        mma_pending = 0;
-        tc_fence_after();
-
+        pend |= 4u;
+        // ---- while Z and PT run: Y = beta (V - (exp(G) k) S) from rows 64..127 of X
         {
-            float acc[64];
-            tmem_ld64(t_Z + lane_off, acc);    // Z = diag(exp(G_last - G_m)) Z'  (row = key channel)
+            float acc[32];
+            tmem_ld32(t_X + lane_off + half_off, acc);
             tmem_wait_ld();
-            {
-                const float sc = tid < DK ? glm_s[tid] : 0.f;
+            if (lt >= C) {
+                const int s2 = lt - C;
+                const float b = beta_s[s2];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) acc[j] *= sc;
-                st_row_swf<16>(Zb, tid, 0, 128, acc);
+                for (int u = 0; u < 4; ++u) {
+                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vraw[u]);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const float2 f2 = __bfloat1622float2(v2[w]);
+                        const int jj = u * 8 + w * 2;
+                        swf(Yb, 32 * wg + jj, s2, NV) = tf32r(b * (f2.x - acc[jj]));
+                        swf(Yb, 32 * wg + jj + 1, s2, NV) = tf32r(b * (f2.y - acc[jj + 1]));
+                    }
+                }
             }
-            tmem_ld64(t_PT + lane_off, acc);
+        }
+        KDA_PHASE(5);
+        KDA_WAIT_OR_EXIT(mb_z, 4u, c & 1);
+        tc_fence_after();
+        KDA_PHASE(6);
+        {
+            float acc[32];
+            tmem_ld32(t_Z + lane_off + half_off, acc);   // Z = diag(exp(G_last - G_m)) Z'
             tmem_wait_ld();
-            if (tid < C) st_row_swf<16>(PTb, tid, 0, C, acc);
+            const float sc = lt < DK ? glm_s[lt] : 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] *= sc;
+            st_row_swf<8>(Zb, lt, 32 * wg, 128, acc);
+            tmem_ld32(t_PT + lane_off + half_off, acc);
+            tmem_wait_ld();
+            if (lt < C) st_row_swf<8>(PTb, lt, 32 * wg, C, acc);
         }
         tc_fence_before();
         fence_proxy_async();
         __syncthreads();
+        KDA_PHASE(7);
 
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk)    // dS = Z Y
-                umma_tf32(t_dS, kdesc(Zb, kk, kA1), kdesc(Yb, kk, kR64), kI, kk > 0);
+                umma_tf32(t_dS, kdesc(Zb, kk, kR128), kdesc(Yb, kk, kR64), kI64, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk)    // O += PT Y  (rows 0..63 of X)
-                umma_tf32(t_O, kdesc(PTb, kk, kR64), kdesc(Yb, kk, kR64), kI, 1);
-            umma_commit(mb_mma);
+                umma_tf32(t_X, kdesc(PTb, kk, kR64), kdesc(Yb, kk, kR64), kI64, 1);
+            umma_commit(mb_zy);
         }
-        mma_pending = 1;
-        KDA_WAIT_OR_EXIT(mb_mma, mma_phase & 1);
-        ++mma_phase;
-        mma_pending = 0;
+        pend |= 8u;
+        // ---- while dS and O run: the next chunk's gate cumsum and vectors
+        if (c + 1 < nchunks) {
+            KDA_WAIT_OR_EXIT(mb_tma, 1u, (c + 1) & 1);
+            cumsum(min(C, len - (c + 1) * C), (c + 1) & 1, beta_next);
+            if (tid < C) beta_next = (c + 2 < nchunks && 2 * C + tid < len - c * C)
+                                         ? p.beta[(size_t)(tokc + 2 * C + tid) * H + h] : 0.f;
+        }
+        KDA_PHASE(8);
+        KDA_WAIT_OR_EXIT(mb_zy, 8u, c & 1);
         tc_fence_after();
-
+        KDA_PHASE(9);
         {
-            float acc[64];
-            tmem_ld64(t_dS + lane_off, acc);
+            float acc[32];
+            tmem_ld32(t_dS + lane_off + half_off, acc);
             tmem_wait_ld();
-            if (tid < DK) {
-                const float gm = gam_s[tid];
+            if (lt < DK) {
+                const float gm = gam_s[lt];
 #pragma unroll
-                for (int j = 0; j < NV; ++j) S[j] = fmaf(gm, S[j], acc[j]);
+                for (int j = 0; j < 32; ++j) S[j] = fmaf(gm, S[j], acc[j]);
             }
-            tmem_ld64(t_O + lane_off, acc);
+            tmem_ld32(t_X + lane_off + half_off, acc);
             tmem_wait_ld();
-            if (tid < L) {
-                const size_t off = ((size_t)(tokc + tid) * H + h) * DV + col0;
+            if (lt < L) {
+                const size_t off = ((size_t)(tokc + lt) * H + h) * DV + col0 + 32 * wg;
                 if constexpr (sizeof(TO) == 4) {
                     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + off);
 #pragma unroll
-                    for (int u = 0; u < 16; ++u)
+                    for (int u = 0; u < 8; ++u)
                         dst[u] = make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
                 } else {
                     uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
+                    for (int u = 0; u < 4; ++u)
                         dst[u] = make_uint4(pack_bf16(acc[8 * u], acc[8 * u + 1]), pack_bf16(acc[8 * u + 2], acc[8 * u + 3]),
                                             pack_bf16(acc[8 * u + 4], acc[8 * u + 5]), pack_bf16(acc[8 * u + 6], acc[8 * u + 7]));
                 }
@@ -504,22 +608,27 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         }
         tc_fence_before();
         __syncthreads();
+        KDA_PHASE(10);
     }
 
-    if (p.sT && tid < DK) {
-        float* dst = p.sT + (((size_t)n * H + h) * DK + tid) * DV + col0;
+    if (p.sT && lt < DK) {
+        float* dst = p.sT + (((size_t)n * H + h) * DK + lt) * DV + col0 + 32 * wg;
 #pragma unroll
-        for (int j = 0; j < NV; j += 4)
+        for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
 
 finish:
-    // After a timeout, give the copies and the MMAs still in flight a bounded
-    // chance to land before the TMEM is released and the CTA exits.
+    KDA_PHASE_FLUSH
+    // After a timeout, give the copy and the MMAs still in flight a bounded
+    // chance to land before the TMEM is released and the CTA exits.  Each
+    // outstanding MMA barrier completes the phase of the running chunk; the
+    // TMA barrier the phase of the chunk whose load is in flight.
     if (*abort_flag) {
         volatile int never = 0;
-        if (tma_pending) (void)mbar_wait(mb_tma, (uint32_t)tma_parity, &never, p.timeout_cycles);
-        if (mma_pending) (void)mbar_wait(mb_mma, mma_phase & 1, &never, p.timeout_cycles);
+        for (int i = 0; i < 4; ++i)
+            if (pend & (1u << i))
+                (void)mbar_wait(bars + i, i == 0 ? (uint32_t)tma_par : (uint32_t)(c & 1), &never, p.timeout_cycles);
     }
     tc_fence_before();
     __syncthreads();
