@@ -39,7 +39,7 @@ using namespace sm100;
 
 constexpr int C = 64;      // chunk length
 constexpr int NV = 64;     // value columns per CTA
-constexpr int NT = 256;    // threads per CTA: two warpgroups
+constexpr int NT = 512;    // threads per CTA: four warpgroups
 constexpr int LDA = 65;    // fp32 pitch of the UT-transform scratch
 
 struct Params {
@@ -55,26 +55,32 @@ struct Params {
 
 // Shared-memory plan (byte offsets from a 1024-aligned base).  Operand tiles
 // are fp32 in the K-major 128-byte-swizzled layout, rounded to tf32.
-//   R1: A1 [128][d_k] until MMA [PA|X] completes; then P [64][64] (0),
-//       T^T [64][64] (16 KB) and the fp32 UT scratch (A below the diagonal,
-//       T transposed on and above it; 32 KB) plus a 32 x 33 product scratch;
-//       PT [64][64] takes P's place once MMA PT completes.
+//   R1: A1 [128][d_k] until MMA [PA|X] completes; then T^T [64][64] (16 KB)
+//       and the fp32 UT scratch (A below the diagonal, T transposed on and
+//       above it; 32 KB) plus a 32 x 33 product scratch.
 //   R2: the 128-row B operand of MMA [PA|X]: rows 0..63 = B1 = k F, rows
-//       64..127 = the state operand (diag(exp(G_m)) S)^T, [128][d_k].  Then
-//       B1^T [128][64] (first 32 KB) until MMA Z completes, then Z there;
+//       64..127 = the state operand (diag(exp(G_m)) S)^T, [128][d_k]; then
 //       Y [64][64] at +32 KB.
 //   STG: TMA staging of q, k (bf16) and log alpha (fp32); the gate cumsum G
 //       overwrites log alpha in place.
 //   VEC: per-chunk channel vectors, double-buffered (the next chunk's are
 //       computed while this chunk's last MMAs run).
+// TMEM (fp32 columns, lane = row): [PA | X] 0..127 (P is masked in place and
+//   is the A operand of MMA PT; O accumulates onto X), Z' 128..191, PT
+//   192..255 (both A operands of the last MMAs), state 256..319 and B1^T
+//   320..383 (lane = key channel).  The state column block holds
+//   S / exp(G_last - G_m) of the chunk before; it is replaced by the chunk's
+//   state operand diag(exp(G_m)) S, onto which MMA Z' Y accumulates, leaving
+//   S_next / exp(G_last - G_m) (the scale of Z = diag(exp(G_last - G_m)) Z'
+//   is thus applied one chunk later, and to the final state).
 struct Plan {
     static constexpr int R1 = 0;
-    static constexpr int P = R1, TOP = R1 + 16384, AS = R1 + 32768, XS = AS + C * LDA * 4;
+    static constexpr int TOP = R1 + 16384, AS = R1 + 32768, XS = AS + C * LDA * 4;
     static constexpr int R2 = 65536;
-    static constexpr int KBT = R2, Y = R2 + 32768;
+    static constexpr int Y = R2 + 32768;
     static constexpr int STG = 131072;
-    static constexpr int VEC = STG + 65536;         // 2 x {gml gm gam glm htot [128], beta[64]}
-    static constexpr int VECN = 5 * 128 + 64;       // floats per buffer
+    static constexpr int VEC = STG + 65536;         // 2 x {gml gm (unused) glm [128], qtot [4][128], beta [64]}
+    static constexpr int VECN = 8 * 128 + 64;       // floats per buffer
     static constexpr int BAR = VEC + 2 * VECN * 4;
     static constexpr int END = BAR + 128;
     static constexpr int BYTES = END + 1024;        // + alignment slack
@@ -122,11 +128,13 @@ __device__ __forceinline__ float rcp_nr(float x)
 // triangle (diagonal included) of the UT scratch.
 __device__ __forceinline__ float Tget(const float* As, int k, int j) { return k >= j ? As[j * LDA + k] : 0.f; }
 
-// UT transform.  On entry As[r*LDA + s] (s < r) holds the strictly lower A;
-// on return As[j*LDA + s] (s >= j) holds T[s][j], T = (I + A)^-1, with A left
-// intact below the diagonal.  Diagonal 16x16 blocks by column-sweep forward
-// substitution (one lane per column), then T10 = -T11 A10 T00,
-// T32 = -T33 A32 T22 and the lower-left 32x32 block -T_BB A_BA T_AA.
+// UT transform, run by the first 128 threads (named barrier 1; the other
+// warps are free meanwhile).  On entry As[r*LDA + s] (s < r) holds the
+// strictly lower A; on return As[j*LDA + s] (s >= j) holds T[s][j],
+// T = (I + A)^-1, with A left intact below the diagonal.  Diagonal 16x16
+// blocks by column-sweep forward substitution (one lane per column), then
+// T10 = -T11 A10 T00, T32 = -T33 A32 T22 (2x2 register tiles) and the
+// lower-left 32x32 block -T_BB A_BA T_AA (2x4 register tiles).
 __device__ __forceinline__ void ut_transform(float* As, float* X)
 {
     const int tid = threadIdx.x;
@@ -145,58 +153,71 @@ __device__ __forceinline__ void ut_transform(float* As, float* X)
         for (int r = 0; r < 16; ++r)
             if (r >= j) As[(b0 + j) * LDA + b0 + r] = x[r];
     }
-    __syncthreads();
+    bar_sync(1, 128);
     {
-        const int blk = tid >> 7, i = (tid & 127) >> 3, j0 = (tid & 7) * 2;
+        const int blk = tid >> 6, tile = tid & 63, i0 = (tile >> 3) * 2, j0 = (tile & 7) * 2;
         const int rb = blk ? 48 : 16, cb = blk ? 32 : 0;
-        float a0 = 0.f, a1 = 0.f, b0_ = 0.f, b1 = 0.f;
+        float a[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-        for (int k = 0; k < 16; k += 2) {
-            const float u0 = As[(rb + i) * LDA + cb + k], u1 = As[(rb + i) * LDA + cb + k + 1];
-            a0 = fmaf(u0, Tget(As, cb + k, cb + j0), a0);
-            a1 = fmaf(u0, Tget(As, cb + k, cb + j0 + 1), a1);
-            b0_ = fmaf(u1, Tget(As, cb + k + 1, cb + j0), b0_);
-            b1 = fmaf(u1, Tget(As, cb + k + 1, cb + j0 + 1), b1);
+        for (int k = 0; k < 16; ++k) {
+            const float u0 = As[(rb + i0) * LDA + cb + k], u1 = As[(rb + i0 + 1) * LDA + cb + k];
+            const float t0 = Tget(As, cb + k, cb + j0), t1 = Tget(As, cb + k, cb + j0 + 1);
+            a[0][0] = fmaf(u0, t0, a[0][0]); a[0][1] = fmaf(u0, t1, a[0][1]);
+            a[1][0] = fmaf(u1, t0, a[1][0]); a[1][1] = fmaf(u1, t1, a[1][1]);
         }
-        X[(blk * 16 + i) * 33 + j0] = a0 + b0_;
-        X[(blk * 16 + i) * 33 + j0 + 1] = a1 + b1;
-        __syncthreads();
-        float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
 #pragma unroll
-        for (int k = 0; k < 16; k += 2) {
-            const float w0 = Tget(As, rb + i, rb + k), w1 = Tget(As, rb + i, rb + k + 1);
-            t0 = fmaf(w0, X[(blk * 16 + k) * 33 + j0], t0);
-            t1 = fmaf(w0, X[(blk * 16 + k) * 33 + j0 + 1], t1);
-            t2 = fmaf(w1, X[(blk * 16 + k + 1) * 33 + j0], t2);
-            t3 = fmaf(w1, X[(blk * 16 + k + 1) * 33 + j0 + 1], t3);
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < 2; ++v) X[(blk * 16 + i0 + u) * 33 + j0 + v] = a[u][v];
+        bar_sync(1, 128);
+        float t[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float w0 = Tget(As, rb + i0, rb + k), w1 = Tget(As, rb + i0 + 1, rb + k);
+            const float x0 = X[(blk * 16 + k) * 33 + j0], x1 = X[(blk * 16 + k) * 33 + j0 + 1];
+            t[0][0] = fmaf(w0, x0, t[0][0]); t[0][1] = fmaf(w0, x1, t[0][1]);
+            t[1][0] = fmaf(w1, x0, t[1][0]); t[1][1] = fmaf(w1, x1, t[1][1]);
         }
-        As[(cb + j0) * LDA + rb + i] = -(t0 + t2);
-        As[(cb + j0 + 1) * LDA + rb + i] = -(t1 + t3);
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < 2; ++v) As[(cb + j0 + v) * LDA + rb + i0 + u] = -t[u][v];
     }
-    __syncthreads();
+    bar_sync(1, 128);
     {
-        const int i = tid >> 3, j0 = (tid & 7) * 4;
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
+        const int i0 = (tid >> 3) * 2, j0 = (tid & 7) * 4;
+        float a[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 8
         for (int k = 0; k < 32; ++k) {
-            const float a = As[(32 + i) * LDA + k];
+            const float u0 = As[(32 + i0) * LDA + k], u1 = As[(32 + i0 + 1) * LDA + k];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) acc[k & 1][q] = fmaf(a, Tget(As, k, j0 + q), acc[k & 1][q]);
+            for (int v = 0; v < 4; ++v) {
+                const float tv = Tget(As, k, j0 + v);
+                a[0][v] = fmaf(u0, tv, a[0][v]);
+                a[1][v] = fmaf(u1, tv, a[1][v]);
+            }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) X[i * 33 + j0 + q] = acc[0][q] + acc[1][q];
-        __syncthreads();
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) X[(i0 + u) * 33 + j0 + v] = a[u][v];
+        bar_sync(1, 128);
         float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
+#pragma unroll 8
         for (int k = 0; k < 32; ++k) {
-            const float w = Tget(As, 32 + i, 32 + k);
+            const float w0 = Tget(As, 32 + i0, 32 + k), w1 = Tget(As, 32 + i0 + 1, 32 + k);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) t[k & 1][q] = fmaf(w, X[k * 33 + j0 + q], t[k & 1][q]);
+            for (int v = 0; v < 4; ++v) {
+                const float xv = X[k * 33 + j0 + v];
+                t[0][v] = fmaf(w0, xv, t[0][v]);
+                t[1][v] = fmaf(w1, xv, t[1][v]);
+            }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) As[(j0 + q) * LDA + 32 + i] = -(t[0][q] + t[1][q]);
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) As[(j0 + v) * LDA + 32 + i0 + u] = -t[u][v];
     }
-    __syncthreads();
 }
 
 // K-major fp32 SW128 operand descriptor for MMA k-step kk (K = 8 per step):
@@ -245,14 +266,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     KDA_PHASE_DECL
     unsigned char* sm = align1024(smem_raw);
     unsigned char* A1 = sm + PL::R1;
-    unsigned char* Pb = sm + PL::P;
-    unsigned char* PTb = sm + PL::P;
     unsigned char* Top = sm + PL::TOP;
     float* As = reinterpret_cast<float*>(sm + PL::AS);
     float* Xs = reinterpret_cast<float*>(sm + PL::XS);
     unsigned char* Bx = sm + PL::R2;            // [B1 ; state operand], 128 rows
-    unsigned char* KBt = sm + PL::KBT;
-    unsigned char* Zb = sm + PL::KBT;
     unsigned char* Yb = sm + PL::Y;
     const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(sm + PL::STG);
     const __nv_bfloat16* ks = qs + C * DK;
@@ -269,7 +286,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int lt = tid & 127;          // TMEM lane owned by this thread
-    const int wg = tid >> 7;           // warpgroup: which 32-column half it loads
+    const int wg = tid >> 7;           // warpgroup: which 16-column quarter it handles
     const int nslice = p.DV / NV;
     const int slice = blockIdx.x % nslice;
     const int h = (blockIdx.x / nslice) % p.H;
@@ -306,20 +323,22 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_off = ((uint32_t)(warp & 3) * 32) << 16;
-    const uint32_t half_off = (uint32_t)wg * 32;
-    // TMEM columns: [PA | X] 0..127 (O accumulates onto X), Z 128, PT 192, dS 256
-    const uint32_t t_PA = tmem, t_X = tmem + 64, t_Z = tmem + 128, t_PT = tmem + 192, t_dS = tmem + 256;
+    const uint32_t q_off = (uint32_t)wg * 16;    // this warpgroup's 16-column quarter
+    const uint32_t t_PA = tmem, t_X = tmem + 64, t_Z = tmem + 128, t_PT = tmem + 192, t_S = tmem + 256;
+    const uint32_t t_KB = tmem + 320;
 
-    // fp32 state: thread (key channel lt < DK, half wg) owns S[lt][32 wg .. 32 wg + 32)
-    float S[32];
+    // initial state into TMEM (lane = key channel, 16 columns per warpgroup)
     {
-        const bool own = lt < DK;
-        const float* src = (p.s0 && own) ? p.s0 + (((size_t)n * H + h) * DK + lt) * DV + col0 + 32 * wg : nullptr;
+        float s16[16];
+        const bool own = lt < DK && p.s0;
+        const float* src = own ? p.s0 + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg : nullptr;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            const float4 v4 = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-            S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
+        for (int j = 0; j < 16; j += 4) {
+            const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            s16[j] = v4.x; s16[j + 1] = v4.y; s16[j + 2] = v4.z; s16[j + 3] = v4.w;
         }
+        tmem_st16(t_S + lane_off + q_off, s16);
+        tmem_wait_st();
     }
 
     unsigned pend = 0;                 // bit i: a completion of bars[i] is outstanding
@@ -331,41 +350,43 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     constexpr int kR128 = 128 * 128;  // atom-column strides (bytes) of 128-row and 64-row tiles
     constexpr int kR64 = 64 * 128;
     constexpr int NG = DK / 4;        // 4-channel groups per row
-    constexpr int RPP = NT / NG;      // rows per pass of the operand build (8 or 16)
+    constexpr int RPP = NT / NG;      // rows per pass of the operand build (16 or 32)
 
-    // gate cumsum of the chunk in the staging buffer (in place), channel
-    // vectors into buffer vb; beta of the chunk (prefetched value) alongside
+    // gate cumsum of the chunk in the staging buffer (in place; thread =
+    // (key channel, quarter of the rows)), channel vectors into buffer vb,
+    // beta of the chunk (prefetched value) alongside
     auto cumsum = [&](int Lc, int vb, float beta_v) {
         float* gml_s = vec0 + vb * PL::VECN;
         float* gm_s = gml_s + 128;
-        float* gam_s = gm_s + 128;
-        float* glm_s = gam_s + 128;
-        float* htot_s = glm_s + 128;
-        float* beta_s = htot_s + 128;
-        float G[32];
+        float* glm_s = gm_s + 256;
+        float* qtot = glm_s + 128;
+        float* beta_s = qtot + 4 * 128;
+        float G[16];
         if (lt < DK) {
 #pragma unroll
-            for (int rr = 0; rr < 32; ++rr) {
-                const int row = 32 * wg + rr;
+            for (int rr = 0; rr < 16; ++rr) {
+                const int row = 16 * wg + rr;
                 G[rr] = row < Lc ? gs[row * DK + lt] : 0.f;
             }
 #pragma unroll
-            for (int rr = 1; rr < 32; ++rr) G[rr] += G[rr - 1];
-            if (wg == 0) htot_s[lt] = G[31];
+            for (int rr = 1; rr < 16; ++rr) G[rr] += G[rr - 1];
+            qtot[wg * 128 + lt] = G[15];
         }
         if (tid < C) beta_s[tid] = beta_v;
         __syncthreads();
         if (lt < DK) {
-            const float off = wg ? htot_s[lt] : 0.f;
+            float off = 0.f;
+            for (int q = 0; q < wg; ++q) off += qtot[q * 128 + lt];
 #pragma unroll
-            for (int rr = 0; rr < 32; ++rr) gs[(32 * wg + rr) * DK + lt] = G[rr] + off;
-            if (wg == 0) {
-                gml_s[lt] = G[31];
-                gm_s[lt] = expf(G[31]);
-            } else {
-                const float Gl = G[31] + off;
-                gam_s[lt] = expf(Gl);
-                glm_s[lt] = expf(Gl - off);
+            for (int rr = 0; rr < 16; ++rr) gs[(16 * wg + rr) * DK + lt] = G[rr] + off;
+            if (wg == 1) {
+                const float Gm = G[15] + off;
+                gml_s[lt] = Gm;
+                gm_s[lt] = expf(Gm);
+            } else if (wg == 3) {
+                const float Gm = qtot[lt] + qtot[128 + lt];
+                const float Gl = G[15] + off;
+                glm_s[lt] = expf(Gl - Gm);
             }
         }
     };
@@ -392,18 +413,18 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         const int tokc = tok0 + c * C;
         const float* gml_s = vec0 + (c & 1) * PL::VECN;
         const float* gm_s = gml_s + 128;
-        const float* gam_s = gm_s + 128;
-        const float* glm_s = gam_s + 128;
-        const float* beta_s = gml_s + 5 * 128;
+        const float* beta_s = gml_s + 8 * 128;
         KDA_PHASE(0);
 
-        // values for Y: thread (chunk row s = lt - 64, half wg) owns v[s][32 wg .. + 32)
+        // values for Y: warpgroups 2 and 3 compute Y while warpgroup 0 runs the UT
+        // transform; thread (chunk row s = lt - 64, wg 2|3) owns v[s][32 (wg - 2) .. + 32)
         uint4 vraw[4];
         {
             const int s = lt - C;
-            const bool live = lt >= C && s < L;
+            const bool live = wg >= 2 && lt >= C && s < L;
             const uint4* src =
-                live ? reinterpret_cast<const uint4*>(p.v + ((size_t)(tokc + s) * H + h) * DV + col0 + 32 * wg) : nullptr;
+                live ? reinterpret_cast<const uint4*>(p.v + ((size_t)(tokc + s) * H + h) * DV + col0 + 32 * (wg - 2))
+                     : nullptr;
 #pragma unroll
             for (int u = 0; u < 4; ++u) vraw[u] = live ? __ldg(src + u) : make_uint4(0u, 0u, 0u, 0u);
         }
@@ -433,11 +454,25 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                     tf32r4(k4.x * rcp_nr(e0), k4.y * rcp_nr(e1), k4.z * rcp_nr(e2), k4.w * rcp_nr(e3));
             }
         }
-        if (lt < DK) {
-            const float sc = gm_s[lt];
+        // state operand Sm = diag(exp(G_m)) S.  TMEM holds S / exp(G_last - G_m)
+        // of the previous chunk (1 before the first), and Sm replaces it there so
+        // that MMA S += Z' Y leaves S_next / exp(G_last - G_m) of this chunk.
+        {
+            float s16[16];
+            tmem_ld16(t_S + lane_off + q_off, s16);
+            tmem_wait_ld();
+            if (lt < DK) {
+                const float sc = gm_s[lt] * (c > 0 ? vec0[((c + 1) & 1) * PL::VECN + 3 * 128 + lt] : 1.f);
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) swf(Bx, C + 32 * wg + jj, lt, 128) = tf32r(sc * S[jj]);
+                for (int jj = 0; jj < 16; ++jj) {
+                    s16[jj] *= sc;
+                    swf(Bx, C + 16 * wg + jj, lt, 128) = s16[jj];
+                }
+            }
+            tmem_st16(t_S + lane_off + q_off, s16);
+            tmem_wait_st();
         }
+        tc_fence_before();
         fence_proxy_async();
         __syncthreads();
         KDA_PHASE(1);
@@ -464,61 +499,42 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc_fence_after();
         KDA_PHASE(2);
 
-        // ---- P (lanes 0..63, lower incl.) and A = beta A~ (lanes 64..127, strictly lower)
+        // ---- P masked in place in TMEM (lanes 0..63, lower incl.); A = beta A~
+        // (lanes 64..127, strictly lower) to the fp32 UT scratch
         {
-            float pa[32];
-            tmem_ld32(t_PA + lane_off + half_off, pa);
+            float pa[16];
+            tmem_ld16(t_PA + lane_off + q_off, pa);
             tmem_wait_ld();
             if (lt < C) {
                 const int r = lt;
 #pragma unroll
-                for (int s2 = 0; s2 < 32; ++s2) pa[s2] = (32 * wg + s2 <= r) ? pa[s2] : 0.f;
-                st_row_swf<8>(Pb, r, 32 * wg, C, pa);
+                for (int s2 = 0; s2 < 16; ++s2) pa[s2] = (16 * wg + s2 <= r) ? pa[s2] : 0.f;
+                tmem_st16(t_PA + lane_off + q_off, pa);
             } else {
                 const int r = lt - C;
                 const float b = beta_s[r];
 #pragma unroll
-                for (int s2 = 0; s2 < 32; ++s2) As[r * LDA + 32 * wg + s2] = (32 * wg + s2 < r) ? b * pa[s2] : 0.f;
+                for (int s2 = 0; s2 < 16; ++s2) As[r * LDA + 16 * wg + s2] = (16 * wg + s2 < r) ? b * pa[s2] : 0.f;
             }
         }
-        // ---- B1 -> B1^T [c][s] (first 32 KB of R2), read fully before any write
+        // ---- B1^T [c][s] into TMEM (lane = key channel): A operand of MMA Z'
         {
-            float kb[32];
+            float kb[16];
 #pragma unroll
-            for (int s2 = 0; s2 < 32; ++s2) kb[s2] = lt < DK ? swf(Bx, 32 * wg + s2, lt, 128) : 0.f;
-            __syncthreads();
-            st_row_swf<8>(KBt, lt, 32 * wg, 128, kb);
+            for (int s2 = 0; s2 < 16; ++s2) kb[s2] = lt < DK ? swf(Bx, 16 * wg + s2, lt, 128) : 0.f;
+            tmem_st16(t_KB + lane_off + q_off, kb);
         }
+        tmem_wait_st();
+        __syncthreads();
         KDA_PHASE(3);
 
-        // ---- UT transform, then T^T into the operand tile (row j, column s)
-        ut_transform(As, Xs);
-        {
-            const int j = tid >> 2, c4 = (tid & 3) * 16;
-            float x[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) x[u] = (c4 + u >= j) ? As[j * LDA + c4 + u] : 0.f;
-            st_row_swf<4>(Top, j, c4, C, x);
-        }
-        fence_proxy_async();
-        __syncthreads();
-        KDA_PHASE(4);
-
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)    // Z' = B1^T T
-                umma_tf32(t_Z, kdesc(KBt, kk, kR128), kdesc(Top, kk, kR64), kI64, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)    // PT = P T  (rows 64..127 unused)
-                umma_tf32(t_PT, kdesc(Pb, kk, kR64), kdesc(Top, kk, kR64), kI64, kk > 0);
-            umma_commit(mb_z);
-        }
-        pend |= 4u;
-        // ---- while Z and PT run: Y = beta (V - (exp(G) k) S) from rows 64..127 of X
-        {
+        // ---- UT transform (warpgroup 0) while warpgroups 2, 3 form
+        // Y = beta (V - (exp(G) k) S) from rows 64..127 of X (K-major: row j, column s)
+        if (tid < 128) {
+            ut_transform(As, Xs);
+        } else if (wg >= 2) {
             float acc[32];
-            tmem_ld32(t_X + lane_off + half_off, acc);
+            tmem_ld32(t_X + lane_off + 32 * (wg - 2), acc);
             tmem_wait_ld();
             if (lt >= C) {
                 const int s2 = lt - C;
@@ -530,45 +546,54 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                     for (int w = 0; w < 4; ++w) {
                         const float2 f2 = __bfloat1622float2(v2[w]);
                         const int jj = u * 8 + w * 2;
-                        swf(Yb, 32 * wg + jj, s2, NV) = tf32r(b * (f2.x - acc[jj]));
-                        swf(Yb, 32 * wg + jj + 1, s2, NV) = tf32r(b * (f2.y - acc[jj + 1]));
+                        swf(Yb, 32 * (wg - 2) + jj, s2, NV) = tf32r(b * (f2.x - acc[jj]));
+                        swf(Yb, 32 * (wg - 2) + jj + 1, s2, NV) = tf32r(b * (f2.y - acc[jj + 1]));
                     }
                 }
             }
         }
+        tc_fence_before();
+        __syncthreads();
+        {
+            const int j = tid >> 3, c8 = (tid & 7) * 8;
+            float x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = (c8 + u >= j) ? As[j * LDA + c8 + u] : 0.f;
+            st_row_swf_raw<2>(Top, j, c8, C, x);
+        }
+        fence_proxy_async();
+        __syncthreads();
+        KDA_PHASE(4);
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C / 8; ++kk)    // Z' = B1^T T   (A from TMEM)
+                umma_tf32_ts(t_Z, t_KB + 8 * kk, kdesc(Top, kk, kR64), kI64, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < C / 8; ++kk)    // PT = P T  (A from TMEM; rows 64..127 unused)
+                umma_tf32_ts(t_PT, t_PA + 8 * kk, kdesc(Top, kk, kR64), kI64, kk > 0);
+            umma_commit(mb_z);
+        }
+        pend |= 4u;
         KDA_PHASE(5);
         KDA_WAIT_OR_EXIT(mb_z, 4u, c & 1);
         tc_fence_after();
         KDA_PHASE(6);
-        {
-            float acc[32];
-            tmem_ld32(t_Z + lane_off + half_off, acc);   // Z = diag(exp(G_last - G_m)) Z'
-            tmem_wait_ld();
-            const float sc = lt < DK ? glm_s[lt] : 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[j] *= sc;
-            st_row_swf<8>(Zb, lt, 32 * wg, 128, acc);
-            tmem_ld32(t_PT + lane_off + half_off, acc);
-            tmem_wait_ld();
-            if (lt < C) st_row_swf<8>(PTb, lt, 32 * wg, C, acc);
-        }
-        tc_fence_before();
-        fence_proxy_async();
-        __syncthreads();
         KDA_PHASE(7);
 
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)    // dS = Z Y
-                umma_tf32(t_dS, kdesc(Zb, kk, kR128), kdesc(Yb, kk, kR64), kI64, kk > 0);
+            for (int kk = 0; kk < C / 8; ++kk)    // S += Z' Y   (A from TMEM)
+                umma_tf32_ts(t_S, t_Z + 8 * kk, kdesc(Yb, kk, kR64), kI64, 1);
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)    // O += PT Y  (rows 0..63 of X)
-                umma_tf32(t_X, kdesc(PTb, kk, kR64), kdesc(Yb, kk, kR64), kI64, 1);
+            for (int kk = 0; kk < C / 8; ++kk)    // O += PT Y  (A from TMEM; rows 0..63 of X)
+                umma_tf32_ts(t_X, t_PT + 8 * kk, kdesc(Yb, kk, kR64), kI64, 1);
             umma_commit(mb_zy);
         }
         pend |= 8u;
-        // ---- while dS and O run: the next chunk's gate cumsum and vectors
+        // ---- while the state and O MMAs run: the next chunk's gate cumsum and vectors
         if (c + 1 < nchunks) {
             KDA_WAIT_OR_EXIT(mb_tma, 1u, (c + 1) & 1);
             cumsum(min(C, len - (c + 1) * C), (c + 1) & 1, beta_next);
@@ -580,27 +605,20 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc_fence_after();
         KDA_PHASE(9);
         {
-            float acc[32];
-            tmem_ld32(t_dS + lane_off + half_off, acc);
-            tmem_wait_ld();
-            if (lt < DK) {
-                const float gm = gam_s[lt];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) S[j] = fmaf(gm, S[j], acc[j]);
-            }
-            tmem_ld32(t_X + lane_off + half_off, acc);
+            float acc[16];
+            tmem_ld16(t_X + lane_off + q_off, acc);
             tmem_wait_ld();
             if (lt < L) {
-                const size_t off = ((size_t)(tokc + lt) * H + h) * DV + col0 + 32 * wg;
+                const size_t off = ((size_t)(tokc + lt) * H + h) * DV + col0 + 16 * wg;
                 if constexpr (sizeof(TO) == 4) {
                     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + off);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
+                    for (int u = 0; u < 4; ++u)
                         dst[u] = make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
                 } else {
                     uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
+                    for (int u = 0; u < 2; ++u)
                         dst[u] = make_uint4(pack_bf16(acc[8 * u], acc[8 * u + 1]), pack_bf16(acc[8 * u + 2], acc[8 * u + 3]),
                                             pack_bf16(acc[8 * u + 4], acc[8 * u + 5]), pack_bf16(acc[8 * u + 6], acc[8 * u + 7]));
                 }
@@ -611,11 +629,20 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         KDA_PHASE(10);
     }
 
-    if (p.sT && lt < DK) {
-        float* dst = p.sT + (((size_t)n * H + h) * DK + lt) * DV + col0 + 32 * wg;
+    if (p.sT) {
+        tc_fence_after();
+        float s16[16];
+        tmem_ld16(t_S + lane_off + q_off, s16);
+        tmem_wait_ld();
+        if (lt < DK) {
+            const float sc = nchunks > 0 ? vec0[((nchunks - 1) & 1) * PL::VECN + 3 * 128 + lt] : 1.f;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+            for (int j = 0; j < 16; ++j) s16[j] *= sc;
+            float* dst = p.sT + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg;
+#pragma unroll
+            for (int j = 0; j < 16; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(s16[j], s16[j + 1], s16[j + 2], s16[j + 3]);
+        }
     }
 
 finish:
