@@ -235,6 +235,9 @@ def run_ours(args, world, rank, local):
         # ---- decode: 64 consecutive steps over 256 x 32 fp32 states
         dec = run_decode(kda, device, stream, world, rank, max(1, args.warmup))
 
+        # ---- the other two chunk-forward workloads, timed once each (context)
+        others = {} if args.skip_others else run_other_workloads(kda, device, stream, world, rank)
+
         # ---- end to end through the public API from pinned host buffers
         e2e = run_e2e(kda, sets[0], w, device, stream, world, steps=max(1, min(args.steps, 5)))
 
@@ -259,6 +262,7 @@ def run_ours(args, world, rank, local):
                      "bytes_per_launch": nbytes, "launch_ms": launch_s * 1e3,
                      "tensor_frac": nflops / launch_s / 1e12 / pk["bf16_tflops"]},
         "decode": dec,
+        "other_workloads": others,
         "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": clocks,
@@ -302,6 +306,51 @@ def run_decode(kda, device, stream, world, rank, warmup):
                          "frac": per_launch / pk["hbm_gbs"], "traffic": recorded_traffic("decode_step"),
                          "peak_kind": f"{kind} copy bandwidth"},
             "gpu_launches": w.T}
+
+
+def run_other_workloads(kda, device, stream, world, rank, reps=3):
+    """Varlen (8 packed sequences, 65536 tokens, H32) and long-context (T131072,
+    H32) chunk forwards: one warm-up launch, `reps` timed launches each."""
+    from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
+    pk, kind = peaks()
+    out = {}
+    for name in ("varlen", "long"):
+        w = WORKLOADS[name]
+        d = make_inputs(w, device, seed=w.seed + 1000 * rank)
+        if name == "varlen":
+            cu = d["cu_seqlens"]
+            nseq = cu.numel() - 1
+            o = torch.empty(w.T, w.H, w.dv, dtype=torch.float32, device=device)
+            sN = torch.empty(nseq, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
+            call = lambda: kda.kda_varlen_fwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], cu, None,
+                                              o=o, final_state=sN, stream=stream)
+            tokens, states = w.T, nseq
+        else:
+            o = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32, device=device)
+            sN = torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
+            call = lambda: kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], None,
+                                             o=o, final_state=sN, stream=stream)
+            tokens, states = w.B * w.T, w.B
+        call()
+        torch.cuda.synchronize(device)
+        ev = event_pairs(reps)
+        barrier(world, device)
+        for a, b in ev:
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize(device)
+        kda.kda_check()
+        t = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3, world, device)
+        nbytes = tokens * w.H * bytes_per_token_head(w.dk, w.dv, 2, 4) + states * w.H * w.dk * w.dv * 4
+        nflops = tokens * w.H * flops_per_token_head(w.dk, w.dv)
+        out[name] = {"workload": f"{name}: {tokens} tokens, H={w.H}, d_k=d_v={w.dk}, bf16 q/k/v, fp32 o and state",
+                     "ms": t * 1e3, "tokens_per_s": tokens * world / t, "tflops": nflops * world / t / 1e12,
+                     "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                  "frac": nbytes / t / 1e9 / pk["hbm_gbs"], "peak_kind": f"{kind} copy bandwidth"}}
+        del d, o, sN
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(kda, d, w, device, stream, world, steps):
@@ -393,6 +442,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-others", action="store_true", help="skip the varlen / long-context timings")
     args = ap.parse_args(argv)
     world, rank, local = dist_env()
     if args.impl == "reference":

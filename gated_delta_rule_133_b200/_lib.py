@@ -23,6 +23,7 @@ SIGNATURES = {
     "kda_varlen_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "kda_recurrent_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "kda_check": (_I, [_P]),
+    "kda_selftest_timeout": (_I, [ctypes.c_longlong, _P]),
     "kda_status_string": (ctypes.c_char_p, [_I]),
     "kda_version": (_I, []),
 }

@@ -4,6 +4,7 @@
 #include <stdlib.h>
 
 #include "kda_chunk.cuh"
+#include "kda_sm100.cuh"
 
 namespace {
 
@@ -72,6 +73,21 @@ kda_status copy_state(const float* s0, float* sT, size_t elems, cudaStream_t s)
     return from_cuda(cudaMemsetAsync(sT, 0, elems * sizeof(float), s));
 }
 
+// One CTA waits, with the chunk kernel's bounded wait, on an mbarrier that
+// nobody arrives on; the wait records the timeout and the kernel returns.
+__global__ void selftest_timeout_kernel(long long limit_cycles)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        kda::sm100::mbar_init(&bar, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    (void)kda::sm100::mbar_wait(&bar, 0u, &abort_flag, limit_cycles);
+}
+
 }  // namespace
 
 extern "C" {
@@ -137,6 +153,13 @@ kda_status kda_check(void* stream)
         return KDA_ERR_CUDA;
     if (word & kda::KDA_DEV_ERR_TIMEOUT) return KDA_ERR_TIMEOUT;
     return KDA_OK;
+}
+
+kda_status kda_selftest_timeout(long long limit_cycles, void* stream)
+{
+    if (limit_cycles < 1 || limit_cycles > (1LL << 32)) return KDA_ERR_INVALID_ARG;
+    selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+    return from_cuda(cudaGetLastError());
 }
 
 const char* kda_status_string(kda_status status)

@@ -128,6 +128,17 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
  */
 kda_status kda_check(void* stream);
 
+/*
+ * Diagnostic: launches one CTA that waits on a shared-memory barrier no thread
+ * ever arrives on, through the same bounded wait the chunk kernel uses, with a
+ * budget of `limit_cycles` SM clock cycles (1 .. 2^32).  The wait gives up,
+ * records KDA_ERR_TIMEOUT in the device status word and the kernel exits
+ * normally: the next kda_check() must report KDA_ERR_TIMEOUT and the
+ * one after it KDA_OK.  Exercises the failure path without any GPU fault.
+ * Returns KDA_ERR_INVALID_ARG for a budget out of range.
+ */
+kda_status kda_selftest_timeout(long long limit_cycles, void* stream);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char* kda_status_string(kda_status status);
 

@@ -79,6 +79,13 @@ def test_recurrent_step_validation():
     assert f(None, None, None, None, None, None, None, 0, 2, 128, 128, 1, 0, None) == _lib.KDA_OK
 
 
+def test_selftest_timeout_validation():
+    f = _lib.load().kda_selftest_timeout
+    assert f(0, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f(-5, None) == _lib.KDA_ERR_INVALID_ARG
+    assert f((1 << 32) + 1, None) == _lib.KDA_ERR_INVALID_ARG
+
+
 def test_python_binding_rejects_bad_tensors():
     import torch
     import gated_delta_rule_133_b200 as kda
