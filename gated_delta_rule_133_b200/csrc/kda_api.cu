@@ -1,5 +1,6 @@
 // C ABI of the KDA library: argument validation, path selection, status codes.
 // Declarations and the contract of every entry point are in include/kda.h.
+#include <string.h>
 #include <cuda_runtime.h>
 #include <stdlib.h>
 
@@ -17,13 +18,21 @@ bool valid_dtype(kda_dtype t) { return t == KDA_F32 || t == KDA_BF16; }
 
 kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
-// KDA_FORCE_SIMT=1 routes bf16 inputs to the CUDA-core kernel (used by tests
-// that compare the two kernels); KDA_TIMEOUT_CYCLES bounds every device-side
-// wait of the tensor-core kernel (default 2^31 SM cycles, about one second).
-bool force_simt()
+// Kernel selection for bf16 inputs: the two-pass tensor-core forward by
+// default; KDA_CHUNK_KERNEL=fused selects the single-pass tensor-core kernel
+// and KDA_CHUNK_KERNEL=simt (or KDA_FORCE_SIMT=1) the CUDA-core kernel (used
+// by tests that compare the kernels).  KDA_TIMEOUT_CYCLES bounds every
+// device-side wait of the tensor-core kernels (default 2^31 SM cycles, about
+// one second).
+enum class ChunkKernel { split, fused, simt };
+ChunkKernel chunk_kernel()
 {
-    const char* e = getenv("KDA_FORCE_SIMT");
-    return e && e[0] == '1';
+    const char* f = getenv("KDA_FORCE_SIMT");
+    if (f && f[0] == '1') return ChunkKernel::simt;
+    const char* e = getenv("KDA_CHUNK_KERNEL");
+    if (e && strcmp(e, "fused") == 0) return ChunkKernel::fused;
+    if (e && strcmp(e, "simt") == 0) return ChunkKernel::simt;
+    return ChunkKernel::split;
 }
 
 long long timeout_cycles()
@@ -38,7 +47,11 @@ kda_status run_chunk(const void* q, const void* k, const void* v, const float* b
                      int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype dtype,
                      kda_dtype o_dtype, cudaStream_t s)
 {
-    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && !force_simt())
+    const ChunkKernel kind = chunk_kernel();
+    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && kind == ChunkKernel::split)
+        return from_cuda(kda::chunk_fwd_split(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk,
+                                              dv, o_dtype, timeout_cycles(), s));
+    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && kind == ChunkKernel::fused)
         return from_cuda(kda::chunk_fwd_tc(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk,
                                            dv, o_dtype, timeout_cycles(), s));
     return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, dtype,
@@ -152,6 +165,7 @@ kda_status kda_check(void* stream)
     if (word && cudaMemcpyToSymbol(kda::g_status, &zero, sizeof(zero)) != cudaSuccess)
         return KDA_ERR_CUDA;
     if (word & kda::KDA_DEV_ERR_TIMEOUT) return KDA_ERR_TIMEOUT;
+    if (word & kda::KDA_DEV_ERR_BAD_INPUT) return KDA_ERR_INVALID_ARG;
     return KDA_OK;
 }
 

@@ -25,4 +25,13 @@ cudaError_t chunk_fwd_tc(const void* q, const void* k, const void* v, const floa
                          int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
                          long long timeout_cycles, cudaStream_t stream);
 
+// Two-pass tensor-core forward (bf16 q/k/v only, same arguments): a parallel
+// pass over every (chunk, head) pair writes fp16 operand records to a
+// stream-ordered workspace, then a sequential pass per (sequence, head, 64
+// value columns) carries the state.
+cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const float* beta,
+                            const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
+                            int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
+                            long long timeout_cycles, cudaStream_t stream);
+
 }  // namespace kda

@@ -1,0 +1,935 @@
+// Chunkwise-parallel KDA forward in two passes on the sm_100a tensor cores
+// (bf16 q/k/v; fp32 gates, state and accumulation).
+//
+// The chunk algebra is that of the CUDA-core path ("Hybrid Linear Attention
+// Architecture: Making LLM Training and Inference More Efficient", section IV;
+// "... Technical Deep Dive ...", section 4; "Linear Attention Architecture Deep
+// Dive", section 5).  Per chunk of 64 tokens, G = cumsum(log alpha):
+//
+//   P  = lower-incl((q e^G)(k e^-G)^T)        A = beta strictly-lower((k e^G)(k e^-G)^T)
+//   T  = (I + A)^-1                           (UT transform)
+//   Z  = (e^(G_last - G) k)^T T   (d_k x 64)  PT = P T   (64 x 64)
+//   Qh = e^G q,  Kh = e^G k
+//   [O ; X] = [Qh ; Kh] S,   Y = diag(beta) (V - X)
+//   S <- diag(e^G_last) S + Z Y,   O += PT Y
+//
+// Everything above the last two lines depends on the chunk alone, so pass 1
+// (chunk_prep_kernel) computes it for every (chunk, head) pair at once, over
+// the whole GPU, and stores one operand record per pair.  Pass 2
+// (chunk_scan_kernel) is the only sequential part: one CTA per (sequence,
+// head, 64 value columns) walks its chunks with two MMA rounds per chunk.
+//
+// Precision.  The intra-chunk products P and A use the middle row m of the
+// chunk as reference, E = exp(G - G_m) and 1/E (each bounded by 32 tokens of
+// decay), and run as kind::tf32 MMAs with operands rounded to nearest; T is
+// fp32.  The record's operands are fp16, which has the tf32 mantissa: every
+// factor e^G, e^(G_last - G) is at most 1, so Qh, Kh, Z and PT stay in range,
+// and S and Y are rounded to fp16 as the scan's MMA operands (|S|, |Y| must
+// stay below 65504).  The scan accumulates in fp32 in TMEM.
+#include "kda_chunk.cuh"
+#include "kda_tc_util.cuh"
+
+namespace kda {
+namespace split {
+
+using namespace sm100;
+using namespace tcu;
+using namespace tcu_host;
+
+constexpr int NT = 512;     // threads per CTA (both kernels): four warpgroups
+constexpr int NV = 64;      // value columns per scan CTA
+
+// One operand record per (chunk, head), chunk-major (record index = chunk * H
+// + head).  Tiles are fp16 in the K-major 128-byte-swizzled layout, so a scan
+// CTA copies the record into shared memory with one bulk copy and feeds the
+// tiles to the tensor cores as they are.
+template <int DK>
+struct Rec {
+    static constexpr int QK = 0;                  // [128][DK]: rows 0..63 Qh, 64..127 Kh
+    static constexpr int Z = DK * 256;            // [DK][64]
+    static constexpr int PT = Z + DK * 128;       // [64][64]
+    static constexpr int EGL = PT + 8192;         // fp32 [DK]: exp(G_last)
+    static constexpr int BETA = EGL + DK * 4;     // fp32 [64]: beta (0 past the chunk end)
+    static constexpr int BYTES = BETA + 256;
+};
+static_assert(Rec<128>::BYTES % 16 == 0 && Rec<64>::BYTES % 16 == 0, "record size must allow bulk copies");
+static_assert(Rec<128>::BYTES <= 65536, "record must fit a 64 KB slot");
+
+// Stores 16 consecutive values of one row of a 16-bit SW128 tile as fp16
+// (col0 a multiple of 8: two 16-byte chunks).
+__device__ __forceinline__ void st_row_h16(unsigned char* tile, int row, int col0, int rows, const float* x)
+{
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+        *reinterpret_cast<uint4*>(tile + swh_off(row, col0 + 8 * u, rows)) =
+            make_uint4(pack_f16(x[8 * u], x[8 * u + 1]), pack_f16(x[8 * u + 2], x[8 * u + 3]),
+                       pack_f16(x[8 * u + 4], x[8 * u + 5]), pack_f16(x[8 * u + 6], x[8 * u + 7]));
+}
+
+
+// Every thread polls; a CTA-wide vote turns any timeout into a common exit.
+#define KDA_WAIT_OR_EXIT(bar, bit, parity)                                                   \
+    do {                                                                                     \
+        const bool ok_ = mbar_wait((bar), (uint32_t)(parity), abort_flag, p.timeout_cycles); \
+        if (__syncthreads_or(!ok_)) goto finish;                                             \
+        pend &= ~(bit);                                                                      \
+    } while (0)
+
+// ============================================================== pass 1: prep
+
+struct PrepParams {
+    const float* beta;
+    const int32_t* cu;       // varlen boundaries, or nullptr (dense)
+    const int32_t* choff;    // varlen: first chunk of each sequence, [nseq + 1]
+    unsigned char* rec;
+    int nseq, T, H, nch;     // dense: nch chunks per sequence
+    long long nitems;        // (chunk, head) items covered by the records
+    long long tokens;
+    long long timeout_cycles;
+};
+
+struct Item {
+    int tok0, L, h;
+    bool ok;
+};
+
+__device__ __forceinline__ Item resolve(const PrepParams& p, long long item)
+{
+    Item it{0, 0, 0, false};
+    if (item >= p.nitems) return it;
+    it.h = (int)(item % p.H);
+    const long long j = item / p.H;
+    if (p.cu) {
+        if (j >= p.choff[p.nseq]) return it;
+        int lo = 0, hi = p.nseq - 1;           // last sequence whose first chunk is <= j
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.choff[mid] <= j) lo = mid;
+            else hi = mid - 1;
+        }
+        it.tok0 = p.cu[lo] + (int)(j - p.choff[lo]) * C;
+        it.L = min(C, p.cu[lo + 1] - it.tok0);
+    } else {
+        const int n = (int)(j / p.nch), c = (int)(j % p.nch);
+        it.tok0 = n * p.T + c * C;
+        it.L = min(C, p.T - c * C);
+    }
+    it.ok = it.L > 0 && it.tok0 >= 0 && it.tok0 + it.L <= p.tokens;
+    return it;
+}
+
+// Shared memory of the prep kernel (byte offsets from a 1024-aligned base).
+//   R1: A1 = [q E; k E] (tf32, [128][d_k]) until MMA PA completes; then T^T
+//       [64][64] at +16 KB and the UT scratch at +32 KB.
+//   B1: k / E (tf32, [64][d_k]).
+//   STG: TMA staging of q, k (bf16) and log alpha (fp32 -> G in place).
+//   VEC: channel vectors G_m, e^G_m, e^(G_last - G_m), e^G_last, partial sums, beta.
+struct PrepPlan {
+    static constexpr int R1 = 0;
+    static constexpr int TOP = R1 + 16384, AS = R1 + 32768, XS = AS + C * LDA * 4;
+    static constexpr int B1 = 65536;
+    static constexpr int STG = 98304;
+    static constexpr int VEC = STG + 65536;
+    static constexpr int VECN = 8 * 128 + 64;
+    static constexpr int BAR = VEC + VECN * 4;
+    static constexpr int END = BAR + 128;
+    static constexpr int BYTES = END + 1024;
+};
+static_assert(PrepPlan::XS + 32 * 33 * 4 <= PrepPlan::B1, "UT scratch overflows R1");
+
+template <int DK>
+__global__ void __launch_bounds__(NT, 1)
+chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmg, const PrepParams p)
+{
+    using PL = PrepPlan;
+    using R = Rec<DK>;
+    extern __shared__ unsigned char smem_raw[];
+    KDA_PHASE_DECL(0)
+    unsigned char* sm = align1024(smem_raw);
+    unsigned char* A1 = sm + PL::R1;
+    unsigned char* Top = sm + PL::TOP;
+    float* As = reinterpret_cast<float*>(sm + PL::AS);
+    float* Xs = reinterpret_cast<float*>(sm + PL::XS);
+    unsigned char* B1 = sm + PL::B1;
+    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(sm + PL::STG);
+    const __nv_bfloat16* ks = qs + C * DK;
+    float* gs = reinterpret_cast<float*>(sm + PL::STG + 2 * C * DK * 2);
+    float* gml_s = reinterpret_cast<float*>(sm + PL::VEC);
+    float* gm_s = gml_s + 128;
+    float* glm_s = gml_s + 256;
+    float* egl_s = gml_s + 384;
+    float* qtot = gml_s + 512;
+    float* beta_s = gml_s + 1024;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::BAR);
+    uint64_t* mb_tma = bars + 0;
+    uint64_t* mb_pa = bars + 1;
+    uint64_t* mb_zp = bars + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int lt = tid & 127;
+    const int wg = tid >> 7;
+    const int H = p.H;
+
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(bars + i, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async();
+        prefetch_tmap(&tmq);
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmg);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32) << 16;
+    const uint32_t q_off = (uint32_t)wg * 16;
+    const uint32_t t_PA = tmem, t_KB = tmem + 64, t_Z = tmem + 128, t_PT = tmem + 192;
+
+    constexpr uint32_t kStageBytes = (uint32_t)C * DK * (2 + 2 + 4);
+    constexpr uint32_t kI64 = idesc_tf32(128, 64, 0, 0);
+    constexpr int kR128 = 128 * 128, kR64 = 64 * 128;
+    constexpr int NG = DK / 4;
+    constexpr int RPP = NT / NG;
+
+    unsigned pend = 0;
+    int tma_par = 0, it = 0;
+    long long item = blockIdx.x;
+    Item cur = resolve(p, item);
+    if (tid == 0 && cur.ok) {
+        mbar_expect_tx(mb_tma, kStageBytes);
+        tma_load_3d((void*)qs, &tmq, mb_tma, 0, cur.h, cur.tok0);
+        tma_load_3d((void*)ks, &tmk, mb_tma, 0, cur.h, cur.tok0);
+        tma_load_3d((void*)gs, &tmg, mb_tma, 0, cur.h, cur.tok0);
+    }
+    if (cur.ok) pend |= 1u;
+
+    for (; cur.ok; ++it) {
+        const int L = cur.L, h = cur.h, tok0 = cur.tok0;
+        unsigned char* rec = p.rec + (size_t)item * R::BYTES;
+        const float beta_v = (tid < C && tid < L) ? p.beta[(size_t)(tok0 + tid) * H + h] : 0.f;
+        KDA_PHASE(0);
+        KDA_WAIT_OR_EXIT(mb_tma, 1u, it & 1);
+
+        // ---- gate cumsum in place (thread = key channel x quarter of the rows)
+        {
+            float G[16];
+            if (lt < DK) {
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int row = 16 * wg + rr;
+                    G[rr] = row < L ? gs[row * DK + lt] : 0.f;
+                }
+#pragma unroll
+                for (int rr = 1; rr < 16; ++rr) G[rr] += G[rr - 1];
+                qtot[wg * 128 + lt] = G[15];
+            }
+            if (tid < C) beta_s[tid] = beta_v;
+            __syncthreads();
+            if (lt < DK) {
+                float off = 0.f;
+                for (int q = 0; q < wg; ++q) off += qtot[q * 128 + lt];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) gs[(16 * wg + rr) * DK + lt] = G[rr] + off;
+                if (wg == 1) {
+                    const float Gm = G[15] + off;
+                    gml_s[lt] = Gm;
+                    gm_s[lt] = expf(Gm);
+                } else if (wg == 3) {
+                    const float Gm = qtot[lt] + qtot[128 + lt];
+                    const float Gl = G[15] + off;
+                    glm_s[lt] = expf(Gl - Gm);
+                    egl_s[lt] = expf(Gl);
+                }
+            }
+            __syncthreads();
+        }
+        KDA_PHASE(1);
+
+        // ---- operands: A1 = [q E; k E] and B1 = k / E (tf32, smem) for the
+        // intra-chunk products; Qh = q e^G and Kh = k e^G (fp16) into the record
+        {
+            const int r0 = tid / NG, c0 = (tid % NG) * 4;
+            const float4 m4 = *reinterpret_cast<const float4*>(gml_s + c0);
+            const float4 gm4 = *reinterpret_cast<const float4*>(gm_s + c0);
+            const uint32_t oq = swf_off(r0, c0, 128), ok = swf_off(C + r0, c0, 128), ob = swf_off(r0, c0, 64);
+#pragma unroll
+            for (int i = 0; i < C / RPP; ++i) {
+                const int r = r0 + RPP * i;
+                const float4 g4 = *reinterpret_cast<const float4*>(gs + r * DK + c0);
+                float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = q4;
+                if (r < L) {
+                    q4 = bf16x4(qs + r * DK + c0);
+                    k4 = bf16x4(ks + r * DK + c0);
+                }
+                const float e0 = __expf(fminf(fmaxf(g4.x - m4.x, -80.f), 80.f));
+                const float e1 = __expf(fminf(fmaxf(g4.y - m4.y, -80.f), 80.f));
+                const float e2 = __expf(fminf(fmaxf(g4.z - m4.z, -80.f), 80.f));
+                const float e3 = __expf(fminf(fmaxf(g4.w - m4.w, -80.f), 80.f));
+                const uint32_t step = (uint32_t)(RPP * 128 * i);
+                *reinterpret_cast<float4*>(A1 + oq + step) = tf32r4(q4.x * e0, q4.y * e1, q4.z * e2, q4.w * e3);
+                *reinterpret_cast<float4*>(A1 + ok + step) = tf32r4(k4.x * e0, k4.y * e1, k4.z * e2, k4.w * e3);
+                *reinterpret_cast<float4*>(B1 + ob + step) =
+                    tf32r4(k4.x * rcp_nr(e0), k4.y * rcp_nr(e1), k4.z * rcp_nr(e2), k4.w * rcp_nr(e3));
+                const float f0 = e0 * gm4.x, f1 = e1 * gm4.y, f2 = e2 * gm4.z, f3 = e3 * gm4.w;
+                *reinterpret_cast<uint2*>(rec + R::QK + swh_off(r, c0, 128)) =
+                    make_uint2(pack_f16(q4.x * f0, q4.y * f1), pack_f16(q4.z * f2, q4.w * f3));
+                *reinterpret_cast<uint2*>(rec + R::QK + swh_off(C + r, c0, 128)) =
+                    make_uint2(pack_f16(k4.x * f0, k4.y * f1), pack_f16(k4.z * f2, k4.w * f3));
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        KDA_PHASE(2);
+
+        // ---- the staging buffer is free: fetch the next item; MMA [P ; A~] = A1 B1^T
+        const long long nitem = item + gridDim.x;
+        const Item nxt = resolve(p, nitem);
+        if (tid == 0) {
+            if (nxt.ok) {
+                mbar_expect_tx(mb_tma, kStageBytes);
+                tma_load_3d((void*)qs, &tmq, mb_tma, 0, nxt.h, nxt.tok0);
+                tma_load_3d((void*)ks, &tmk, mb_tma, 0, nxt.h, nxt.tok0);
+                tma_load_3d((void*)gs, &tmg, mb_tma, 0, nxt.h, nxt.tok0);
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < DK / 8; ++kk)
+                umma_tf32(t_PA, kdesc(A1, kk, kR128), kdesc(B1, kk, kR64), kI64, kk > 0);
+            umma_commit(mb_pa);
+        }
+        if (nxt.ok) {
+            pend |= 1u;
+            tma_par = (it + 1) & 1;
+        }
+        pend |= 2u;
+        KDA_WAIT_OR_EXIT(mb_pa, 2u, it & 1);
+        tc_fence_after();
+        KDA_PHASE(3);
+
+        // ---- P masked in place in TMEM (lanes 0..63, lower incl.); A = beta A~
+        // (lanes 64..127, strictly lower) to the fp32 UT scratch; B1^T into TMEM
+        {
+            float pa[16];
+            tmem_ld16(t_PA + lane_off + q_off, pa);
+            tmem_wait_ld();
+            if (lt < C) {
+                const int r = lt;
+#pragma unroll
+                for (int s2 = 0; s2 < 16; ++s2) pa[s2] = (16 * wg + s2 <= r) ? pa[s2] : 0.f;
+                tmem_st16(t_PA + lane_off + q_off, pa);
+            } else {
+                const int r = lt - C;
+                const float b = beta_s[r];
+#pragma unroll
+                for (int s2 = 0; s2 < 16; ++s2) As[r * LDA + 16 * wg + s2] = (16 * wg + s2 < r) ? b * pa[s2] : 0.f;
+            }
+            float kb[16];
+#pragma unroll
+            for (int s2 = 0; s2 < 16; ++s2) kb[s2] = lt < DK ? swf(B1, 16 * wg + s2, lt, 64) : 0.f;
+            tmem_st16(t_KB + lane_off + q_off, kb);
+        }
+        tmem_wait_st();
+        __syncthreads();
+        KDA_PHASE(4);
+
+        // ---- UT transform (warpgroup 0); channel vectors of the record alongside
+        if (tid < 128) {
+            ut_transform(As, Xs);
+        } else {
+            const int t = tid - 128;
+            float* egl_g = reinterpret_cast<float*>(rec + R::EGL);
+            float* beta_g = reinterpret_cast<float*>(rec + R::BETA);
+            if (t < DK) egl_g[t] = egl_s[t];
+            else if (t >= 128 && t < 128 + C) beta_g[t - 128] = beta_s[t - 128];
+        }
+        __syncthreads();
+        {
+            const int j = tid >> 3, c8 = (tid & 7) * 8;
+            float x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = (c8 + u >= j) ? As[j * LDA + c8 + u] : 0.f;
+            st_row_swf_raw<2>(Top, j, c8, C, x);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        KDA_PHASE(5);
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C / 8; ++kk)    // Z' = B1^T T   (A from TMEM)
+                umma_tf32_ts(t_Z, t_KB + 8 * kk, kdesc(Top, kk, kR64), kI64, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < C / 8; ++kk)    // PT = P T  (A from TMEM; rows 64..127 unused)
+                umma_tf32_ts(t_PT, t_PA + 8 * kk, kdesc(Top, kk, kR64), kI64, kk > 0);
+            umma_commit(mb_zp);
+        }
+        pend |= 4u;
+        KDA_WAIT_OR_EXIT(mb_zp, 4u, it & 1);
+        tc_fence_after();
+        KDA_PHASE(6);
+
+        // ---- Z = diag(e^(G_last - G_m)) Z' and PT, fp16, into the record
+        {
+            float z[16];
+            tmem_ld16(t_Z + lane_off + q_off, z);
+            tmem_wait_ld();
+            if (lt < DK) {
+                const float sc = glm_s[lt];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) z[u] *= sc;
+                st_row_h16(rec + R::Z, lt, 16 * wg, DK, z);
+            }
+            float pt[16];
+            tmem_ld16(t_PT + lane_off + q_off, pt);
+            tmem_wait_ld();
+            if (lt < C) st_row_h16(rec + R::PT, lt, 16 * wg, C, pt);
+        }
+        tc_fence_before();
+        __syncthreads();
+        KDA_PHASE(7);
+        item = nitem;
+        cur = nxt;
+    }
+
+finish:
+    KDA_PHASE_FLUSH
+    if (*abort_flag) {
+        volatile int never = 0;
+        for (int i = 0; i < 3; ++i)
+            if (pend & (1u << i))
+                (void)mbar_wait(bars + i, i == 0 ? (uint32_t)tma_par : (uint32_t)(it & 1), &never, p.timeout_cycles);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ============================================================== pass 2: scan
+
+struct ScanParams {
+    const __nv_bfloat16* v;
+    const float* s0;
+    void* o;
+    float* sT;
+    const int32_t* cu;
+    const int32_t* choff;
+    const unsigned char* rec;
+    int nseq, T, H, DV, nch;
+    long long max_chunks;    // records available per head
+    long long tokens;
+    long long timeout_cycles;
+};
+
+// Shared memory of the scan kernel: two 72 KB slots, each holding one record
+// (the M = 128 reads of the 64-row PT tile, and for d_k = 64 of the Z tile,
+// run on into the rest of the record's 64 KB, into rows whose products are
+// discarded) and the chunk's V tile [64][NV] (bf16, 128-byte swizzle) at
+// +64 KB; the state operand S [d_k][NV] and Y [64][NV] (fp16, MN-major B
+// operands: value columns contiguous, 128-byte swizzle); the o staging tile
+// [64][NV] (output type, 16-byte chunks XOR-swizzled by row).
+template <int DK>
+struct ScanPlan {
+    static constexpr int SLOT = 73728, VOFF = 65536;
+    static constexpr int SOP = 2 * SLOT;
+    static constexpr int YB = SOP + NV * DK * 2;
+    static constexpr int OST = YB + NV * C * 2;
+    static constexpr int BAR = OST + C * NV * 4;
+    static constexpr int END = BAR + 128;
+    static constexpr int BYTES = END + 1024;
+};
+
+// MN-major SW128 B operand (16-bit, NV = 64 columns = one 128-byte row per K
+// index): K-step kk (16 K rows = two 1 KB groups) starts 2 KB further on.
+__device__ __forceinline__ uint64_t mn_desc(const unsigned char* tile, int kk, int k_rows)
+{
+    return sdesc_sw128(smem_u32(tile) + kk * 2048, (uint32_t)(k_rows * 128), 1024);
+}
+
+// Output rows [0, L) of one chunk from the TMEM accumulator (lane = row, 16
+// columns per warpgroup), run by the 256 threads of lanes 0..63: rows go to a
+// staging tile, then every warp writes whole row segments (coalesced).
+template <typename TO>
+__device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost, void* o, size_t row0_off,
+                                             size_t row_stride, int L, int lt, int wg)
+{
+    constexpr int EB = (int)sizeof(TO), RB = NV * EB, CPR = RB / 16, CPT = 16 * EB / 16;
+    float acc[16];
+    tmem_ld16(t_acc, acc);
+    tmem_wait_ld();
+#pragma unroll
+    for (int u = 0; u < CPT; ++u) {
+        const int k = wg * CPT + u;
+        uint4 val;
+        if constexpr (EB == 4)
+            val = make_uint4(__float_as_uint(acc[4 * u]), __float_as_uint(acc[4 * u + 1]),
+                             __float_as_uint(acc[4 * u + 2]), __float_as_uint(acc[4 * u + 3]));
+        else
+            val = make_uint4(pack_bf16(acc[8 * u], acc[8 * u + 1]), pack_bf16(acc[8 * u + 2], acc[8 * u + 3]),
+                             pack_bf16(acc[8 * u + 4], acc[8 * u + 5]), pack_bf16(acc[8 * u + 6], acc[8 * u + 7]));
+        *reinterpret_cast<uint4*>(ost + lt * RB + ((k ^ (lt & (CPR - 1))) << 4)) = val;
+    }
+    bar_sync(1, 256);
+    const int t = wg * 64 + lt;
+#pragma unroll
+    for (int pss = 0; pss < C * CPR / 256; ++pss) {
+        const int idx = pss * 256 + t, row = idx / CPR, k = idx % CPR;
+        if (row < L) {
+            const uint4 val = *reinterpret_cast<const uint4*>(ost + row * RB + ((k ^ (row & (CPR - 1))) << 4));
+            *reinterpret_cast<uint4*>(static_cast<unsigned char*>(o) + (row0_off + (size_t)row * row_stride) * EB + k * 16) = val;
+        }
+    }
+}
+
+// One CTA per (sequence, head, NV value columns).  Thread (lane lt < d_k,
+// warpgroup wg) keeps S[lt][16 wg .. 16 wg + 16) of the state in registers.
+// Per chunk c (slot c % 2):
+//   S <- diag(e^G_last(c-1)) S + W(c-1)      W = Z Y of the chunk before, from TMEM
+//   S operand (fp16) -> smem;  MMA [O ; X] = [Qh ; Kh] S  -> TMEM buffer c % 2
+//   Y = diag(beta) (V - X) -> smem (lanes 64..127), while lanes 0..63 store
+//   the o rows of chunk c - 1
+//   MMA W = Z Y (commit), MMA O += PT Y
+// A slot is refilled in two parts as soon as the MMAs reading each part have
+// completed: the [Qh ; Kh] tile and V after chunk c's X MMA and Y phase, the
+// Z, PT, e^G_last and beta part after chunk c + 1's X MMA (tcgen05 MMAs of
+// one thread complete in issue order).
+template <typename TO, int DK>
+__global__ void __launch_bounds__(NT, 1)
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
+{
+    using PL = ScanPlan<DK>;
+    using R = Rec<DK>;
+    extern __shared__ unsigned char smem_raw[];
+    KDA_PHASE_DECL(1)
+    unsigned char* sm = align1024(smem_raw);
+    unsigned char* Sop = sm + PL::SOP;
+    unsigned char* Yb = sm + PL::YB;
+    unsigned char* Ost = sm + PL::OST;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::BAR);
+    uint64_t* mb_a = bars + 0;     // [2]: [Qh ; Kh] and V of a slot
+    uint64_t* mb_b = bars + 2;     // [2]: Z, PT, e^G_last and beta of a slot
+    uint64_t* mb_x = bars + 4;
+    uint64_t* mb_w = bars + 5;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* misc_slot = reinterpret_cast<int*>(tmem_slot + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int lt = tid & 127;
+    const int wg = tid >> 7;
+    const int nslice = p.DV / NV;
+    const int slice = blockIdx.x % nslice;
+    const int h = (blockIdx.x / nslice) % p.H;
+    const int rank = blockIdx.x / (nslice * p.H);
+    const int H = p.H, DV = p.DV;
+    int n, tok0, len;
+    long long j0;
+    if (p.cu) {
+        n = seq_by_rank(p.cu, p.nseq, rank, misc_slot);
+        tok0 = p.cu[n];
+        len = max(0, p.cu[n + 1] - tok0);
+        j0 = p.choff[n];
+    } else {
+        n = rank;
+        tok0 = n * p.T;
+        len = p.T;
+        j0 = (long long)n * p.nch;
+    }
+    const int col0 = slice * NV;
+    int nchunks = (len + C - 1) / C;
+    if (j0 < 0 || j0 + nchunks > p.max_chunks || (long long)tok0 + len > p.tokens || tok0 < 0) {
+        if (tid == 0) flag_bad_input();
+        nchunks = 0;
+        len = 0;
+    }
+
+    if (tid == 0) {
+        for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async();
+        prefetch_tmap(&tmv);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32) << 16;
+    const uint32_t q_off = (uint32_t)wg * 16;
+    const uint32_t t_W = tmem + 128;
+    constexpr uint32_t kI = idesc_f16(128, NV, 1);
+    constexpr uint32_t kBytesA = R::Z + C * NV * 2;     // [Qh ; Kh] tile + V tile
+    constexpr uint32_t kBytesB = R::BYTES - R::Z;       // Z, PT, e^G_last, beta
+
+    auto rec_of = [&](int cc) { return p.rec + ((size_t)(j0 + cc) * H + h) * R::BYTES; };
+    auto issue_a = [&](int cc) {
+        unsigned char* slot = sm + (cc & 1) * PL::SLOT;
+        mbar_expect_tx(mb_a + (cc & 1), kBytesA);
+        bulk_load(slot, rec_of(cc), R::Z, mb_a + (cc & 1));
+        tma_load_3d(slot + PL::VOFF, &tmv, mb_a + (cc & 1), col0, h, tok0 + cc * C);
+    };
+    auto issue_b = [&](int cc) {
+        unsigned char* slot = sm + (cc & 1) * PL::SLOT;
+        mbar_expect_tx(mb_b + (cc & 1), kBytesB);
+        bulk_load(slot + R::Z, rec_of(cc) + R::Z, kBytesB, mb_b + (cc & 1));
+    };
+
+    // state rows of this thread
+    float S[16];
+    {
+        const bool own = lt < DK && p.s0;
+        const float* src = own ? p.s0 + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg : nullptr;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+            const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
+        }
+    }
+
+    unsigned pend = 0;                 // bits: 0-1 mb_a[slot], 2-3 mb_b[slot], 4 mb_x, 5 mb_w
+    uint32_t apar = 0u, bpar = 0u;     // bit i: phase parity of the pending load of slot i
+    int xph = 0, wph = 0;              // commits issued to mb_x / mb_w
+    int c = 0;
+    if (tid == 0)
+        for (int cc = 0; cc < 2 && cc < nchunks; ++cc) {
+            issue_a(cc);
+            issue_b(cc);
+        }
+    for (int cc = 0; cc < 2 && cc < nchunks; ++cc) pend |= (1u | 4u) << cc;
+
+    float eglp = 1.f;                  // e^G_last of the previous chunk, key channel lt
+    int Lprev = 0;
+    for (c = 0; c < nchunks; ++c) {
+        const int b = c & 1;
+        unsigned char* slot = sm + b * PL::SLOT;
+        const uint32_t t_XO = tmem + 64 * b;
+        const int L = min(C, len - c * C);
+        KDA_PHASE(0);
+
+        // ---- state of chunk c - 1, then its fp16 operand (row = value column)
+        if (c > 0) {
+            KDA_WAIT_OR_EXIT(mb_w, 32u, (c - 1) & 1);
+            tc_fence_after();
+            float w[16];
+            tmem_ld16(t_W + lane_off + q_off, w);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
+        }
+        if (lt < DK) st_row_h16(Sop, lt, 16 * wg, DK, S);
+        fence_proxy_async();
+        tc_fence_before();
+        KDA_WAIT_OR_EXIT(mb_a + b, 1u << b, (apar >> b) & 1u);
+        KDA_PHASE(1);
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)    // [O ; X] = [Qh ; Kh] S
+                umma_f16(t_XO, kdesc(slot + R::QK, kk, 128 * 128), mn_desc(Sop, kk, DK), kI, kk > 0);
+            umma_commit(mb_x);
+        }
+        ++xph;
+        pend |= 16u;
+        KDA_WAIT_OR_EXIT(mb_x, 16u, c & 1);
+        tc_fence_after();
+        // chunk c - 1's PT Y has completed as well: refill the other slot's
+        // second part with chunk c + 1
+        if (c >= 1 && c + 1 < nchunks) {
+            if (tid == 0) {
+                fence_proxy_async();
+                issue_b(c + 1);
+            }
+            pend |= 4u << (b ^ 1);
+            bpar = (bpar & ~(1u << (b ^ 1))) | ((uint32_t)(((c + 1) >> 1) & 1) << (b ^ 1));
+        }
+        KDA_WAIT_OR_EXIT(mb_b + b, 4u << b, (bpar >> b) & 1u);
+        KDA_PHASE(2);
+
+        // ---- Y = beta (V - X) (lanes 64..127) | o rows of chunk c - 1 (lanes 0..63)
+        {
+            const float* egl = reinterpret_cast<const float*>(slot + R::EGL);
+            const float* beta = reinterpret_cast<const float*>(slot + R::BETA);
+            eglp = lt < DK ? egl[lt] : 1.f;
+            if (lt >= C) {
+                const int s = lt - C;
+                float x16[16];
+                tmem_ld16(t_XO + lane_off + q_off, x16);
+                tmem_wait_ld();
+                const float bs = beta[s];
+                const unsigned char* vt = slot + PL::VOFF;
+                uint4 vr[2];
+                vr[0] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg, C));
+                vr[1] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg + 8, C));
+                float y[16];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const float2 f2 = __bfloat1622float2(v2[w]);
+                        const int jj = 8 * u + 2 * w;
+                        y[jj] = bs * (f2.x - x16[jj]);
+                        y[jj + 1] = bs * (f2.y - x16[jj + 1]);
+                    }
+                }
+                st_row_h16(Yb, s, 16 * wg, C, y);
+            } else if (c > 0) {
+                store_o_tile<TO>(tmem + 64 * (b ^ 1) + lane_off + q_off, Ost, p.o,
+                                 ((size_t)(tok0 + (c - 1) * C) * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg);
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        KDA_PHASE(3);
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)     // W = Z Y
+                umma_f16(t_W, kdesc(slot + R::Z, kk, DK * 128), mn_desc(Yb, kk, C), kI, kk > 0);
+            umma_commit(mb_w);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)     // O += PT Y  (rows 64..127: discarded)
+                umma_f16(t_XO, kdesc(slot + R::PT, kk, C * 128), mn_desc(Yb, kk, C), kI, 1);
+            if (c + 2 < nchunks) {                  // X MMA done, V consumed: refill part one
+                fence_proxy_async();
+                issue_a(c + 2);
+            }
+        }
+        ++wph;
+        pend |= 32u;
+        if (c + 2 < nchunks) {
+            pend |= 1u << b;
+            apar = (apar & ~(1u << b)) | ((uint32_t)(((c + 2) >> 1) & 1) << b);
+        }
+        Lprev = L;
+        KDA_PHASE(4);
+    }
+
+    if (nchunks > 0) {
+        // W and O of the last chunk: one more commit covers every MMA issued
+        if (tid == 0) umma_commit(mb_x);
+        ++xph;
+        pend |= 16u;
+        KDA_WAIT_OR_EXIT(mb_x, 16u, nchunks & 1);
+        pend &= ~32u;
+        tc_fence_after();
+        float w[16];
+        tmem_ld16(t_W + lane_off + q_off, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
+        if (lt < C)
+            store_o_tile<TO>(tmem + 64 * ((nchunks - 1) & 1) + lane_off + q_off, Ost, p.o,
+                             ((size_t)(tok0 + (nchunks - 1) * C) * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg);
+    }
+    if (p.sT && lt < DK) {
+        float* dst = p.sT + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+
+finish:
+    KDA_PHASE_FLUSH
+    if (*abort_flag) {
+        // let every copy and MMA in flight land before the TMEM is released
+        volatile int never = 0;
+        for (int i = 0; i < 2; ++i) {
+            if (pend & (1u << i)) (void)mbar_wait(mb_a + i, (apar >> i) & 1u, &never, p.timeout_cycles);
+            if (pend & (4u << i)) (void)mbar_wait(mb_b + i, (bpar >> i) & 1u, &never, p.timeout_cycles);
+        }
+        if (pend & 16u) (void)mbar_wait(mb_x, (uint32_t)((xph - 1) & 1), &never, p.timeout_cycles);
+        if (pend & 32u) (void)mbar_wait(mb_w, (uint32_t)((wph - 1) & 1), &never, p.timeout_cycles);
+        __syncthreads();
+        if (tid == 0) umma_commit(mb_x);
+        (void)mbar_wait(mb_x, (uint32_t)(xph & 1), &never, p.timeout_cycles);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+#undef KDA_WAIT_OR_EXIT
+
+// ============================================================== host side
+
+// First chunk of every packed sequence: choff[i] = sum_{j<i} ceil(len_j / 64),
+// choff[nseq] = total.  One CTA; each thread sums a contiguous range of
+// sequences, then a block-wide scan.  Negative lengths count as empty.
+__global__ void chunk_offsets_kernel(const int32_t* cu, int nseq, int32_t* choff)
+{
+    __shared__ int warp_tot[32];
+    const int per = (nseq + blockDim.x - 1) / blockDim.x;
+    const int a = min(nseq, (int)threadIdx.x * per), b = min(nseq, a + per);
+    int local = 0;
+    for (int i = a; i < b; ++i) local += (max(0, cu[i + 1] - cu[i]) + C - 1) / C;
+    int x = local;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        int t = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        warp_tot[lane] = t;
+    }
+    __syncthreads();
+    int base = x - local + (w ? warp_tot[w - 1] : 0);
+    for (int i = a; i < b; ++i) {
+        choff[i] = base;
+        base += (max(0, cu[i + 1] - cu[i]) + C - 1) / C;
+    }
+    if (threadIdx.x == blockDim.x - 1) choff[nseq] = base;
+}
+
+static int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;
+    return n > 0 ? n : 148;
+}
+
+// Keeps freed stream-ordered allocations in the device's default pool, so
+// that the per-call workspace is recycled instead of returned to the driver.
+static void retain_pool_memory()
+{
+    static bool done[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || done[dev]) return;
+    cudaMemPool_t pool;
+    if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+        uint64_t keep = ~0ull;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    }
+    done[dev] = true;
+}
+
+template <typename TO, int DK>
+static cudaError_t run(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
+                       const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens,
+                       int H, int dv, long long timeout_cycles, cudaStream_t stream)
+{
+    using R = Rec<DK>;
+    const int nch = cu ? 0 : (T + C - 1) / C;
+    const long long max_chunks = cu ? tokens / C + nseq : (long long)nseq * nch;
+    const size_t off_bytes = (((size_t)nseq + 1) * 4 + 1023) & ~(size_t)1023;
+    const size_t bytes = off_bytes + (size_t)max_chunks * H * R::BYTES;
+
+    CUtensorMap tq, tk, tg;
+    if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
+        !make_tmap(&tg, log_alpha, tokens, H, DK, true))
+        return cudaErrorInvalidValue;
+    CUtensorMap tv;
+    if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true)) return cudaErrorInvalidValue;
+
+    retain_pool_memory();
+    unsigned char* ws = nullptr;
+    cudaError_t err = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
+    if (err != cudaSuccess) return err;
+    int32_t* choff = reinterpret_cast<int32_t*>(ws);
+    unsigned char* rec = ws + off_bytes;
+
+    if (cu) chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu, nseq, choff);
+
+    PrepParams pp;
+    pp.beta = beta;
+    pp.cu = cu;
+    pp.choff = choff;
+    pp.rec = rec;
+    pp.nseq = nseq;
+    pp.T = T;
+    pp.H = H;
+    pp.nch = nch;
+    pp.nitems = max_chunks * H;
+    pp.tokens = tokens;
+    pp.timeout_cycles = timeout_cycles;
+    auto pk = chunk_prep_kernel<DK>;
+    err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
+    if (err == cudaSuccess && pp.nitems > 0) {
+        const long long grid = std::min<long long>(pp.nitems, sm_count());
+        pk<<<(unsigned)grid, NT, PrepPlan::BYTES, stream>>>(tq, tk, tg, pp);
+        err = cudaGetLastError();
+    }
+
+    if (err == cudaSuccess) {
+        ScanParams sp;
+        sp.v = static_cast<const __nv_bfloat16*>(v);
+        sp.s0 = s0;
+        sp.o = o;
+        sp.sT = sT;
+        sp.cu = cu;
+        sp.choff = choff;
+        sp.rec = rec;
+        sp.nseq = nseq;
+        sp.T = T;
+        sp.H = H;
+        sp.DV = dv;
+        sp.nch = nch;
+        sp.max_chunks = max_chunks;
+        sp.tokens = tokens;
+        sp.timeout_cycles = timeout_cycles;
+        auto sk = chunk_scan_kernel<TO, DK>;
+        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
+        const long long blocks = (long long)nseq * H * (dv / NV);
+        if (err == cudaSuccess && blocks > 0) {
+            if (blocks > 0x7fffffffLL) err = cudaErrorInvalidConfiguration;
+            else {
+                sk<<<(unsigned)blocks, NT, ScanPlan<DK>::BYTES, stream>>>(tv, sp);
+                err = cudaGetLastError();
+            }
+        }
+    }
+    const cudaError_t ferr = cudaFreeAsync(ws, stream);
+    return err != cudaSuccess ? err : ferr;
+}
+
+}  // namespace split
+
+cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const float* beta,
+                            const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
+                            int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
+                            long long timeout_cycles, cudaStream_t stream)
+{
+    if (o_dtype == KDA_F32) {
+        if (dk == 128) return split::run<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 64) return split::run<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
+    } else {
+        if (dk == 128) return split::run<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 64) return split::run<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

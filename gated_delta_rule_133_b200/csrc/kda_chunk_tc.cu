@@ -28,19 +28,17 @@
 // (sequence, head, 64 value columns).  The CTA walks its chunks in order;
 // shared-memory regions are reused as each operand dies (see Plan).
 #include "kda_chunk.cuh"
-#include "kda_sm100.cuh"
-
-#include <cudaTypedefs.h>
+#include "kda_tc_util.cuh"
 
 namespace kda {
 namespace tc {
 
 using namespace sm100;
+using namespace tcu;
+using namespace tcu_host;
 
-constexpr int C = 64;      // chunk length
 constexpr int NV = 64;     // value columns per CTA
 constexpr int NT = 512;    // threads per CTA: four warpgroups
-constexpr int LDA = 65;    // fp32 pitch of the UT-transform scratch
 
 struct Params {
     const __nv_bfloat16* v;
@@ -87,166 +85,6 @@ struct Plan {
 };
 static_assert(Plan::XS + 32 * 33 * 4 <= Plan::R2, "UT scratch overflows R1");
 
-__device__ __forceinline__ unsigned char* align1024(unsigned char* p)
-{
-    const uint32_t a = smem_u32(p);
-    return p + (((a + 1023u) & ~1023u) - a);
-}
-
-// Rank-r sequence in longest-first order (ties: lower index first).
-__device__ int seq_by_rank(const int32_t* cu, int N, int rank, int* slot)
-{
-    if (threadIdx.x == 0) *slot = rank;
-    __syncthreads();
-    for (int i = threadIdx.x; i < N; i += blockDim.x) {
-        const int li = cu[i + 1] - cu[i];
-        int rk = 0;
-        for (int j = 0; j < N; ++j) {
-            const int lj = cu[j + 1] - cu[j];
-            rk += (lj > li) || (lj == li && j < i);
-        }
-        if (rk == rank) *slot = i;
-    }
-    __syncthreads();
-    const int n = *slot;
-    __syncthreads();
-    return n;
-}
-
-// 1/x for normal x by Newton-Raphson on the FMA pipe (keeps the exponent
-// unit free for exp): seed from the exponent bits (relative error < 5.1 %),
-// two iterations (< 1e-5, below tf32 resolution).
-__device__ __forceinline__ float rcp_nr(float x)
-{
-    float y = __int_as_float(0x7EF311C3 - __float_as_int(x));
-    y = y * fmaf(-x, y, 2.f);
-    y = y * fmaf(-x, y, 2.f);
-    return y;
-}
-
-// T[k][j] of the unit lower-triangular T, kept transposed in the upper
-// triangle (diagonal included) of the UT scratch.
-__device__ __forceinline__ float Tget(const float* As, int k, int j) { return k >= j ? As[j * LDA + k] : 0.f; }
-
-// UT transform, run by the first 128 threads (named barrier 1; the other
-// warps are free meanwhile).  On entry As[r*LDA + s] (s < r) holds the
-// strictly lower A; on return As[j*LDA + s] (s >= j) holds T[s][j],
-// T = (I + A)^-1, with A left intact below the diagonal.  Diagonal 16x16
-// blocks by column-sweep forward substitution (one lane per column), then
-// T10 = -T11 A10 T00, T32 = -T33 A32 T22 (2x2 register tiles) and the
-// lower-left 32x32 block -T_BB A_BA T_AA (2x4 register tiles).
-__device__ __forceinline__ void ut_transform(float* As, float* X)
-{
-    const int tid = threadIdx.x;
-    if (tid < 64) {
-        const int b0 = 16 * (tid >> 4), j = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-        for (int s = 0; s < 15; ++s) {
-            const float xs = x[s];
-#pragma unroll
-            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-As[(b0 + r) * LDA + b0 + s], xs, x[r]);
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r)
-            if (r >= j) As[(b0 + j) * LDA + b0 + r] = x[r];
-    }
-    bar_sync(1, 128);
-    {
-        const int blk = tid >> 6, tile = tid & 63, i0 = (tile >> 3) * 2, j0 = (tile & 7) * 2;
-        const int rb = blk ? 48 : 16, cb = blk ? 32 : 0;
-        float a[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float u0 = As[(rb + i0) * LDA + cb + k], u1 = As[(rb + i0 + 1) * LDA + cb + k];
-            const float t0 = Tget(As, cb + k, cb + j0), t1 = Tget(As, cb + k, cb + j0 + 1);
-            a[0][0] = fmaf(u0, t0, a[0][0]); a[0][1] = fmaf(u0, t1, a[0][1]);
-            a[1][0] = fmaf(u1, t0, a[1][0]); a[1][1] = fmaf(u1, t1, a[1][1]);
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < 2; ++v) X[(blk * 16 + i0 + u) * 33 + j0 + v] = a[u][v];
-        bar_sync(1, 128);
-        float t[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float w0 = Tget(As, rb + i0, rb + k), w1 = Tget(As, rb + i0 + 1, rb + k);
-            const float x0 = X[(blk * 16 + k) * 33 + j0], x1 = X[(blk * 16 + k) * 33 + j0 + 1];
-            t[0][0] = fmaf(w0, x0, t[0][0]); t[0][1] = fmaf(w0, x1, t[0][1]);
-            t[1][0] = fmaf(w1, x0, t[1][0]); t[1][1] = fmaf(w1, x1, t[1][1]);
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < 2; ++v) As[(cb + j0 + v) * LDA + rb + i0 + u] = -t[u][v];
-    }
-    bar_sync(1, 128);
-    {
-        const int i0 = (tid >> 3) * 2, j0 = (tid & 7) * 4;
-        float a[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-            const float u0 = As[(32 + i0) * LDA + k], u1 = As[(32 + i0 + 1) * LDA + k];
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const float tv = Tget(As, k, j0 + v);
-                a[0][v] = fmaf(u0, tv, a[0][v]);
-                a[1][v] = fmaf(u1, tv, a[1][v]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < 4; ++v) X[(i0 + u) * 33 + j0 + v] = a[u][v];
-        bar_sync(1, 128);
-        float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-            const float w0 = Tget(As, 32 + i0, 32 + k), w1 = Tget(As, 32 + i0 + 1, 32 + k);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const float xv = X[k * 33 + j0 + v];
-                t[0][v] = fmaf(w0, xv, t[0][v]);
-                t[1][v] = fmaf(w1, xv, t[1][v]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < 4; ++v) As[(j0 + v) * LDA + 32 + i0 + u] = -t[u][v];
-    }
-}
-
-// K-major fp32 SW128 operand descriptor for MMA k-step kk (K = 8 per step):
-// 4 steps per 128-byte atom column, atom columns `atom_stride` bytes apart.
-__device__ __forceinline__ uint64_t kdesc(const unsigned char* tile, int kk, int atom_stride)
-{
-    return sdesc_sw128(smem_u32(tile) + (kk >> 2) * atom_stride + (kk & 3) * 32, 16, 1024);
-}
-
-__device__ __forceinline__ float4 bf16x4(const __nv_bfloat16* p)
-{
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-}
-
-__device__ __forceinline__ float4 tf32r4(float a, float b, float c, float d)
-{
-    return make_float4(tf32r(a), tf32r(b), tf32r(c), tf32r(d));
-}
-
-// Phase markers: empty in the library build.  A profiling build may define
-// them to accumulate clock64() deltas per chunk stage.
-#ifndef KDA_PHASE
-#define KDA_PHASE_DECL
-#define KDA_PHASE(i) ((void)0)
-#define KDA_PHASE_FLUSH
-#endif
 
 // Every thread polls; a CTA-wide vote turns any timeout into a common exit.
 #define KDA_WAIT_OR_EXIT(bar, bit, parity)                                               \
@@ -263,7 +101,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 {
     using PL = Plan;
     extern __shared__ unsigned char smem_raw[];
-    KDA_PHASE_DECL
+    KDA_PHASE_DECL(2)
     unsigned char* sm = align1024(smem_raw);
     unsigned char* A1 = sm + PL::R1;
     unsigned char* Top = sm + PL::TOP;
@@ -665,40 +503,6 @@ finish:
     }
 }
 #undef KDA_WAIT_OR_EXIT
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// [tokens, H, DK] (bf16 or fp32), box = 64 tokens x 1 head x DK channels, no
-// swizzle; rows past the end of the tensor are filled with zeros.
-static bool make_tmap(CUtensorMap* m, const void* base, long long tokens, int H, int DK, bool fp32)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t es = fp32 ? 4 : 2;
-    const cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)H, (cuuint64_t)tokens};
-    const cuuint64_t strides[2] = {(cuuint64_t)DK * es, (cuuint64_t)H * DK * es};
-    const cuuint32_t box[3] = {(cuuint32_t)DK, 1, (cuuint32_t)C};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <typename TO, int DK>
 static cudaError_t launch(const void* q, const void* k, const float* log_alpha, const Params& prm,

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -10,12 +11,15 @@
 namespace kda {
 
 // Per-device status word (the library is one translation unit, so this is its
-// only definition).  Kernels set bits here when a bounded wait gives up;
+// only definition).  Kernels set bits here when a bounded wait gives up or
+// when device-resident arguments (sequence boundaries) fall outside the
+// buffers they index, in which case the affected sequence is skipped;
 // kda_check() reads and clears it.
-enum : unsigned { KDA_DEV_ERR_TIMEOUT = 1u };
+enum : unsigned { KDA_DEV_ERR_TIMEOUT = 1u, KDA_DEV_ERR_BAD_INPUT = 2u };
 __device__ unsigned g_status = 0;
 
 __device__ __forceinline__ void flag_timeout() { atomicOr(&g_status, KDA_DEV_ERR_TIMEOUT); }
+__device__ __forceinline__ void flag_bad_input() { atomicOr(&g_status, KDA_DEV_ERR_BAD_INPUT); }
 
 // Element access for the two supported q/k/v/o element types.
 template <typename T> struct Elem;

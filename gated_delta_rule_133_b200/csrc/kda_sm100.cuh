@@ -1,7 +1,8 @@
-// Thin wrappers over the sm_100a instructions the tensor-core chunk kernel uses:
-// mbarriers (bounded waits), TMA tile loads (no multicast), the async-proxy
-// fence, TMEM allocation, tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, one
-// CTA), tcgen05.commit, tcgen05.ld and the shared-memory matrix descriptors.
+// Thin wrappers over the sm_100a instructions the tensor-core chunk kernels use:
+// mbarriers (bounded waits), TMA tile and bulk loads (no multicast), the
+// async-proxy fence, TMEM allocation, tcgen05.mma (kind::tf32 and kind::f16
+// with fp16 operands, fp32 accumulation, one CTA), tcgen05.commit,
+// tcgen05.ld/st and the shared-memory matrix descriptors.
 #pragma once
 
 #include <cuda.h>
@@ -83,6 +84,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory (both addresses 16-byte
+// aligned, size a multiple of 16); completion is signalled on `bar` as
+// transaction bytes.  Never multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
 }
 
 // ---------------------------------------------------------------- TMEM
@@ -231,6 +242,25 @@ __device__ __forceinline__ void umma_tf32_ts(uint32_t tmem_d, uint32_t tmem_a, u
         : "memory");
 }
 
+// Instruction descriptor: kind::f16 with fp16 A (K-major) and B (K-major, or
+// MN-major when b_mn = 1), fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int b_mn = 0)
+{
+    return (1u << 4) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, one instruction (K = 16 fp16), issued by one thread.
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Named barrier over the first `count` threads of the CTA.
 __device__ __forceinline__ void bar_sync(int id, int count)
 {
@@ -290,6 +320,22 @@ __device__ __forceinline__ void st_row_swf_raw(unsigned char* tile, int row, int
     for (int ch = 0; ch < NCH; ++ch)
         *reinterpret_cast<float4*>(tile + swf_off(row, col0 + 4 * ch, rows)) =
             make_float4(x[4 * ch], x[4 * ch + 1], x[4 * ch + 2], x[4 * ch + 3]);
+}
+
+// Byte offset of element (row, col) of a 16-bit tile in the canonical K-major
+// 128-byte-swizzled layout: 64 columns (128 B) per atom column, otherwise as
+// swf_off.
+__device__ __forceinline__ uint32_t swh_off(int row, int col, int rows)
+{
+    const int atom = col >> 6, c = col & 63;
+    const int chunk = (c >> 3) ^ (row & 7);
+    return (uint32_t)(atom * rows * 128 + (row >> 3) * 1024 + (row & 7) * 128 + chunk * 16 + (c & 7) * 2);
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi)
+{
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)

@@ -124,7 +124,9 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
 /*
  * Synchronises `stream` and reports (then clears) the current device's
  * status word: KDA_ERR_TIMEOUT if a device-side bounded wait ran out since the
- * last check, KDA_ERR_CUDA if the stream reports an error, else KDA_OK.
+ * last check, KDA_ERR_INVALID_ARG if a kernel found device-resident sequence
+ * boundaries (cu_seqlens) outside the token range and skipped that sequence,
+ * KDA_ERR_CUDA if the stream reports an error, else KDA_OK.
  */
 kda_status kda_check(void* stream);
 
