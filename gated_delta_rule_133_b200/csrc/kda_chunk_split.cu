@@ -67,7 +67,8 @@ __device__ __forceinline__ void st_row_h16(unsigned char* tile, int row, int col
 }
 
 
-// Every thread polls; a CTA-wide vote turns any timeout into a common exit.
+// Every thread polls (measured faster than one poller per warp); a CTA-wide
+// vote turns any timeout into a common exit.
 #define KDA_WAIT_OR_EXIT(bar, bit, parity)                                                   \
     do {                                                                                     \
         const bool ok_ = mbar_wait((bar), (uint32_t)(parity), abort_flag, p.timeout_cycles); \
@@ -119,24 +120,139 @@ __device__ __forceinline__ Item resolve(const PrepParams& p, long long item)
 }
 
 // Shared memory of the prep kernel (byte offsets from a 1024-aligned base).
-//   R1: A1 = [q E; k E] (tf32, [128][d_k]) until MMA PA completes; then T^T
-//       [64][64] at +16 KB and the UT scratch at +32 KB.
+//   A1: [q E; k E] (tf32, [128][d_k]) of the item being built; once MMA PA
+//       has read it, the staging tile of the previous item's record tail
+//       (Z, PT, e^G_last, beta), which one bulk store copies out.
 //   B1: k / E (tf32, [64][d_k]).
 //   STG: TMA staging of q, k (bf16) and log alpha (fp32 -> G in place).
-//   VEC: channel vectors G_m, e^G_m, e^(G_last - G_m), e^G_last, partial sums, beta.
+//   TOP: T^T [64][64] (tf32 B operand of MMA Z', PT); AS/XS: UT scratch.
+//   VEC: per item (double-buffered): G_m, e^G_m, e^(G_last - G_m), e^G_last,
+//        partial sums, beta.
 struct PrepPlan {
-    static constexpr int R1 = 0;
-    static constexpr int TOP = R1 + 16384, AS = R1 + 32768, XS = AS + C * LDA * 4;
+    static constexpr int A1 = 0;
     static constexpr int B1 = 65536;
     static constexpr int STG = 98304;
-    static constexpr int VEC = STG + 65536;
+    static constexpr int TOP = 163840;
+    static constexpr int AS = TOP + 16384;
+    static constexpr int XS = AS + C * LDA * 4;
+    static constexpr int VEC = XS + 32 * 33 * 4;
     static constexpr int VECN = 8 * 128 + 64;
-    static constexpr int BAR = VEC + VECN * 4;
+    static constexpr int BAR = VEC + 2 * VECN * 4;
     static constexpr int END = BAR + 128;
     static constexpr int BYTES = END + 1024;
 };
-static_assert(PrepPlan::XS + 32 * 33 * 4 <= PrepPlan::B1, "UT scratch overflows R1");
 
+template <int DK>
+struct PrepCtx {
+    const __nv_bfloat16* qs;
+    const __nv_bfloat16* ks;
+    float* gs;
+    unsigned char* A1;
+    unsigned char* B1;
+};
+
+// Channel vectors of one item buffer.
+struct Vec {
+    float* gml;    // G_m
+    float* gm;     // e^G_m
+    float* glm;    // e^(G_last - G_m)
+    float* egl;    // e^G_last
+    float* qtot;   // partial sums [3][128]
+    float* beta;   // [64]
+};
+__device__ __forceinline__ Vec vec_at(unsigned char* base, int buf)
+{
+    float* f = reinterpret_cast<float*>(base) + buf * PrepPlan::VECN;
+    return Vec{f, f + 128, f + 256, f + 384, f + 512, f + 1024};
+}
+
+// Gate cumsum of the staged chunk in place, by 384 threads (t = 0..383:
+// key channel t % 128, rows [21 p, 21 p + 21) of part p = t / 128, the last
+// part 22 rows), and the item's channel vectors.  Named barrier 2.
+template <int DK>
+__device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t, float beta_v)
+{
+    const int ch = t & 127, part = t >> 7;
+    const int r0 = 21 * part, nr = part == 2 ? 22 : 21;
+    float G[22];
+    if (ch < DK) {
+#pragma unroll
+        for (int rr = 0; rr < 22; ++rr) {
+            const int row = r0 + rr;
+            G[rr] = (rr < nr && row < L) ? gs[row * DK + ch] : 0.f;
+        }
+#pragma unroll
+        for (int rr = 1; rr < 22; ++rr) G[rr] += G[rr - 1];
+        v.qtot[part * 128 + ch] = G[nr - 1];
+    }
+    if (t < C) v.beta[t] = beta_v;
+    bar_sync(2, 384);
+    if (ch < DK) {
+        float off = 0.f;
+        for (int q = 0; q < part; ++q) off += v.qtot[q * 128 + ch];
+#pragma unroll
+        for (int rr = 0; rr < 22; ++rr)
+            if (rr < nr) gs[(r0 + rr) * DK + ch] = G[rr] + off;
+        if (part == 1) {
+            const float Gm = off + G[31 - 21];
+            const float Gl = v.qtot[ch] + v.qtot[128 + ch] + v.qtot[256 + ch];
+            v.gml[ch] = Gm;
+            v.gm[ch] = expf(Gm);
+            v.glm[ch] = expf(Gl - Gm);
+            v.egl[ch] = expf(Gl);
+        }
+    }
+    bar_sync(2, 384);
+}
+
+// Operands of one item, by `nthr` threads (t = 0..nthr-1): A1 = [q E; k E]
+// and B1 = k / E (tf32, smem) for the intra-chunk products; Qh = q e^G and
+// Kh = k e^G (fp16) straight into the record.
+template <int DK>
+__device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& v, unsigned char* rec, int L, int t,
+                                               int nthr)
+{
+    using R = Rec<DK>;
+    constexpr int NG = DK / 4;
+    const int rpp = nthr / NG;
+    const int r0 = t / NG, c0 = (t % NG) * 4;
+    const float4 m4 = *reinterpret_cast<const float4*>(v.gml + c0);
+    const float4 gm4 = *reinterpret_cast<const float4*>(v.gm + c0);
+#pragma unroll 2
+    for (int r = r0; r < C; r += rpp) {
+        const float4 g4 = *reinterpret_cast<const float4*>(x.gs + r * DK + c0);
+        float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = q4;
+        if (r < L) {
+            q4 = bf16x4(x.qs + r * DK + c0);
+            k4 = bf16x4(x.ks + r * DK + c0);
+        }
+        const float e0 = __expf(fminf(fmaxf(g4.x - m4.x, -80.f), 80.f));
+        const float e1 = __expf(fminf(fmaxf(g4.y - m4.y, -80.f), 80.f));
+        const float e2 = __expf(fminf(fmaxf(g4.z - m4.z, -80.f), 80.f));
+        const float e3 = __expf(fminf(fmaxf(g4.w - m4.w, -80.f), 80.f));
+        *reinterpret_cast<float4*>(x.A1 + swf_off(r, c0, 128)) = tf32r4(q4.x * e0, q4.y * e1, q4.z * e2, q4.w * e3);
+        *reinterpret_cast<float4*>(x.A1 + swf_off(C + r, c0, 128)) = tf32r4(k4.x * e0, k4.y * e1, k4.z * e2, k4.w * e3);
+        *reinterpret_cast<float4*>(x.B1 + swf_off(r, c0, 64)) =
+            tf32r4(k4.x * rcp_nr(e0), k4.y * rcp_nr(e1), k4.z * rcp_nr(e2), k4.w * rcp_nr(e3));
+        const float f0 = e0 * gm4.x, f1 = e1 * gm4.y, f2 = e2 * gm4.z, f3 = e3 * gm4.w;
+        *reinterpret_cast<uint2*>(rec + R::QK + swh_off(r, c0, 128)) =
+            make_uint2(pack_f16(q4.x * f0, q4.y * f1), pack_f16(q4.z * f2, q4.w * f3));
+        *reinterpret_cast<uint2*>(rec + R::QK + swh_off(C + r, c0, 128)) =
+            make_uint2(pack_f16(k4.x * f0, k4.y * f1), pack_f16(k4.z * f2, k4.w * f3));
+    }
+}
+
+// One persistent CTA per SM walks items blockIdx.x, + gridDim.x, ...  The
+// UT transform of item k (warpgroup 0) overlaps the gate cumsum and operand
+// build of item k + 1 (warpgroups 1-3); one MMA round then forms Z', PT of
+// item k and [P ; A~] of item k + 1.
+//
+//   prologue: load, cumsum, build, MMA PA of item 0; P/A split of item 0
+//   loop k:   WG0: UT(k), T^T tile      | WG1-3: cumsum + build of item k + 1
+//             MMA Z'(k), PT(k), PA(k + 1)
+//             record tail of item k (staged in A1, one bulk store); P/A split of k + 1
+//
+// TMEM: [P ; A~] double-buffered (0, 64), B1^T 128, Z' 192, PT 256.
 template <int DK>
 __global__ void __launch_bounds__(NT, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -147,24 +263,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     extern __shared__ unsigned char smem_raw[];
     KDA_PHASE_DECL(0)
     unsigned char* sm = align1024(smem_raw);
-    unsigned char* A1 = sm + PL::R1;
+    PrepCtx<DK> x;
+    x.A1 = sm + PL::A1;
+    x.B1 = sm + PL::B1;
+    x.qs = reinterpret_cast<const __nv_bfloat16*>(sm + PL::STG);
+    x.ks = x.qs + C * DK;
+    x.gs = reinterpret_cast<float*>(sm + PL::STG + 2 * C * DK * 2);
     unsigned char* Top = sm + PL::TOP;
     float* As = reinterpret_cast<float*>(sm + PL::AS);
     float* Xs = reinterpret_cast<float*>(sm + PL::XS);
-    unsigned char* B1 = sm + PL::B1;
-    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(sm + PL::STG);
-    const __nv_bfloat16* ks = qs + C * DK;
-    float* gs = reinterpret_cast<float*>(sm + PL::STG + 2 * C * DK * 2);
-    float* gml_s = reinterpret_cast<float*>(sm + PL::VEC);
-    float* gm_s = gml_s + 128;
-    float* glm_s = gml_s + 256;
-    float* egl_s = gml_s + 384;
-    float* qtot = gml_s + 512;
-    float* beta_s = gml_s + 1024;
+    unsigned char* vbase = sm + PL::VEC;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::BAR);
     uint64_t* mb_tma = bars + 0;
-    uint64_t* mb_pa = bars + 1;
-    uint64_t* mb_zp = bars + 2;
+    uint64_t* mb_mma = bars + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -172,9 +283,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     const int lt = tid & 127;
     const int wg = tid >> 7;
     const int H = p.H;
+    constexpr int kStoreIssuer = 128;   // first thread of warpgroup 1
 
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 2; ++i) mbar_init(bars + i, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
@@ -183,7 +295,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         prefetch_tmap(&tmg);
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -192,230 +304,203 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_off = ((uint32_t)(warp & 3) * 32) << 16;
     const uint32_t q_off = (uint32_t)wg * 16;
-    const uint32_t t_PA = tmem, t_KB = tmem + 64, t_Z = tmem + 128, t_PT = tmem + 192;
+    const uint32_t t_KB = tmem + 128, t_Z = tmem + 192, t_PT = tmem + 256;
 
     constexpr uint32_t kStageBytes = (uint32_t)C * DK * (2 + 2 + 4);
     constexpr uint32_t kI64 = idesc_tf32(128, 64, 0, 0);
     constexpr int kR128 = 128 * 128, kR64 = 64 * 128;
-    constexpr int NG = DK / 4;
-    constexpr int RPP = NT / NG;
 
-    unsigned pend = 0;
-    int tma_par = 0, it = 0;
+    unsigned pend = 0;                 // bit 0: TMA load outstanding, bit 1: MMA commit outstanding
+    int tpar = 0;                      // parity of the outstanding TMA load
+    int nload = 0, nmma = 0;           // loads / commits issued so far
+    bool stored = false;               // the store issuer has bulk stores in flight
+
+    auto load_item = [&](const Item& it) {   // thread 0
+        mbar_expect_tx(mb_tma, kStageBytes);
+        tma_load_3d((void*)x.qs, &tmq, mb_tma, 0, it.h, it.tok0);
+        tma_load_3d((void*)x.ks, &tmk, mb_tma, 0, it.h, it.tok0);
+        tma_load_3d((void*)x.gs, &tmg, mb_tma, 0, it.h, it.tok0);
+    };
+    auto beta_of = [&](const Item& it, int t) {
+        return (it.ok && t < C && t < it.L) ? p.beta[(size_t)(it.tok0 + t) * H + it.h] : 0.f;
+    };
+    // P masked in place in TMEM (lanes 0..63, lower incl.); A = beta A~ (lanes
+    // 64..127, strictly lower) to the UT scratch; B1^T into TMEM
+    auto split_pa = [&](uint32_t t_PA, const Vec& v) {
+        float pa[16];
+        tmem_ld16(t_PA + lane_off + q_off, pa);
+        tmem_wait_ld();
+        if (lt < C) {
+#pragma unroll
+            for (int s2 = 0; s2 < 16; ++s2) pa[s2] = (16 * wg + s2 <= lt) ? pa[s2] : 0.f;
+            tmem_st16(t_PA + lane_off + q_off, pa);
+        } else {
+            const int r = lt - C;
+            const float b = v.beta[r];
+#pragma unroll
+            for (int s2 = 0; s2 < 16; ++s2) As[r * LDA + 16 * wg + s2] = (16 * wg + s2 < r) ? b * pa[s2] : 0.f;
+        }
+        float kb[16];
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) kb[s2] = lt < DK ? swf(x.B1, 16 * wg + s2, lt, 64) : 0.f;
+        tmem_st16(t_KB + lane_off + q_off, kb);
+        tmem_wait_st();
+    };
+
     long long item = blockIdx.x;
     Item cur = resolve(p, item);
-    if (tid == 0 && cur.ok) {
-        mbar_expect_tx(mb_tma, kStageBytes);
-        tma_load_3d((void*)qs, &tmq, mb_tma, 0, cur.h, cur.tok0);
-        tma_load_3d((void*)ks, &tmk, mb_tma, 0, cur.h, cur.tok0);
-        tma_load_3d((void*)gs, &tmg, mb_tma, 0, cur.h, cur.tok0);
+    Item nxt{0, 0, 0, false};
+    int k = 0;
+    if (!cur.ok) goto finish;
+
+    // ---- prologue: item 0 by all threads
+    if (tid == 0) load_item(cur);
+    ++nload;
+    pend |= 1u;
+    tpar = 0;
+    {
+        const float beta_v = tid >= 128 ? beta_of(cur, tid - 128) : 0.f;
+        KDA_WAIT_OR_EXIT(mb_tma, 1u, 0);
+        if (tid >= 128) cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v);
+        __syncthreads();
+        build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)item * R::BYTES, cur.L, tid, NT);
     }
-    if (cur.ok) pend |= 1u;
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    nxt = resolve(p, item + gridDim.x);
+    if (tid == 0) {
+        if (nxt.ok) load_item(nxt);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < DK / 8; ++kk)
+            umma_tf32(tmem, kdesc(x.A1, kk, kR128), kdesc(x.B1, kk, kR64), kI64, kk > 0);
+        umma_commit(mb_mma);
+    }
+    if (nxt.ok) {
+        pend |= 1u;
+        tpar = nload & 1;
+        ++nload;
+    }
+    pend |= 2u;
+    KDA_WAIT_OR_EXIT(mb_mma, 2u, 0);
+    ++nmma;
+    tc_fence_after();
+    split_pa(tmem, vec_at(vbase, 0));
+    tc_fence_before();
+    __syncthreads();
 
-    for (; cur.ok; ++it) {
-        const int L = cur.L, h = cur.h, tok0 = cur.tok0;
-        unsigned char* rec = p.rec + (size_t)item * R::BYTES;
-        const float beta_v = (tid < C && tid < L) ? p.beta[(size_t)(tok0 + tid) * H + h] : 0.f;
+    for (k = 0;; ++k) {
+        const int vb = k & 1, nb = vb ^ 1;
+        const Vec vcur = vec_at(vbase, vb), vnxt = vec_at(vbase, nb);
+        const uint32_t t_PAc = tmem + 64 * vb, t_PAn = tmem + 64 * nb;
+        const long long nitem = item + gridDim.x;
         KDA_PHASE(0);
-        KDA_WAIT_OR_EXIT(mb_tma, 1u, it & 1);
 
-        // ---- gate cumsum in place (thread = key channel x quarter of the rows)
-        {
-            float G[16];
-            if (lt < DK) {
+        // ---- UT transform of item k (WG0) | cumsum + operands of item k + 1 (WG1-3)
+        if (wg == 0) {
+            ut_transform(As, Xs);
+            bar_sync(1, 128);
+            {
+                const int j = tid >> 1, c0 = (tid & 1) * 32;
+                float tv[32];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int row = 16 * wg + rr;
-                    G[rr] = row < L ? gs[row * DK + lt] : 0.f;
-                }
-#pragma unroll
-                for (int rr = 1; rr < 16; ++rr) G[rr] += G[rr - 1];
-                qtot[wg * 128 + lt] = G[15];
+                for (int u = 0; u < 32; ++u) tv[u] = (c0 + u >= j) ? As[j * LDA + c0 + u] : 0.f;
+                st_row_swf_raw<8>(Top, j, c0, C, tv);
             }
-            if (tid < C) beta_s[tid] = beta_v;
-            __syncthreads();
-            if (lt < DK) {
-                float off = 0.f;
-                for (int q = 0; q < wg; ++q) off += qtot[q * 128 + lt];
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) gs[(16 * wg + rr) * DK + lt] = G[rr] + off;
-                if (wg == 1) {
-                    const float Gm = G[15] + off;
-                    gml_s[lt] = Gm;
-                    gm_s[lt] = expf(Gm);
-                } else if (wg == 3) {
-                    const float Gm = qtot[lt] + qtot[128 + lt];
-                    const float Gl = G[15] + off;
-                    glm_s[lt] = expf(Gl - Gm);
-                    egl_s[lt] = expf(Gl);
-                }
+        } else if (nxt.ok) {
+            const int t = tid - 128;
+            const float beta_v = beta_of(nxt, t);
+            if (tid == kStoreIssuer && stored) bulk_wait_read();   // A1 is about to be rewritten
+            const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
+            if (!bar_or(3, 384, !ok)) {
+                cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v);
+                build_operands<DK>(x, vnxt, p.rec + (size_t)nitem * R::BYTES, nxt.L, t, 384);
             }
-            __syncthreads();
         }
+        fence_proxy_async();
+        tc_fence_before();
+        if (__syncthreads_or(*abort_flag)) goto finish;
+        if (nxt.ok) pend &= ~1u;
         KDA_PHASE(1);
 
-        // ---- operands: A1 = [q E; k E] and B1 = k / E (tf32, smem) for the
-        // intra-chunk products; Qh = q e^G and Kh = k e^G (fp16) into the record
-        {
-            const int r0 = tid / NG, c0 = (tid % NG) * 4;
-            const float4 m4 = *reinterpret_cast<const float4*>(gml_s + c0);
-            const float4 gm4 = *reinterpret_cast<const float4*>(gm_s + c0);
-            const uint32_t oq = swf_off(r0, c0, 128), ok = swf_off(C + r0, c0, 128), ob = swf_off(r0, c0, 64);
-#pragma unroll
-            for (int i = 0; i < C / RPP; ++i) {
-                const int r = r0 + RPP * i;
-                const float4 g4 = *reinterpret_cast<const float4*>(gs + r * DK + c0);
-                float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = q4;
-                if (r < L) {
-                    q4 = bf16x4(qs + r * DK + c0);
-                    k4 = bf16x4(ks + r * DK + c0);
-                }
-                const float e0 = __expf(fminf(fmaxf(g4.x - m4.x, -80.f), 80.f));
-                const float e1 = __expf(fminf(fmaxf(g4.y - m4.y, -80.f), 80.f));
-                const float e2 = __expf(fminf(fmaxf(g4.z - m4.z, -80.f), 80.f));
-                const float e3 = __expf(fminf(fmaxf(g4.w - m4.w, -80.f), 80.f));
-                const uint32_t step = (uint32_t)(RPP * 128 * i);
-                *reinterpret_cast<float4*>(A1 + oq + step) = tf32r4(q4.x * e0, q4.y * e1, q4.z * e2, q4.w * e3);
-                *reinterpret_cast<float4*>(A1 + ok + step) = tf32r4(k4.x * e0, k4.y * e1, k4.z * e2, k4.w * e3);
-                *reinterpret_cast<float4*>(B1 + ob + step) =
-                    tf32r4(k4.x * rcp_nr(e0), k4.y * rcp_nr(e1), k4.z * rcp_nr(e2), k4.w * rcp_nr(e3));
-                const float f0 = e0 * gm4.x, f1 = e1 * gm4.y, f2 = e2 * gm4.z, f3 = e3 * gm4.w;
-                *reinterpret_cast<uint2*>(rec + R::QK + swh_off(r, c0, 128)) =
-                    make_uint2(pack_f16(q4.x * f0, q4.y * f1), pack_f16(q4.z * f2, q4.w * f3));
-                *reinterpret_cast<uint2*>(rec + R::QK + swh_off(C + r, c0, 128)) =
-                    make_uint2(pack_f16(k4.x * f0, k4.y * f1), pack_f16(k4.z * f2, k4.w * f3));
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        KDA_PHASE(2);
-
-        // ---- the staging buffer is free: fetch the next item; MMA [P ; A~] = A1 B1^T
-        const long long nitem = item + gridDim.x;
-        const Item nxt = resolve(p, nitem);
+        // ---- MMA round: Z'(k) = B1^T T, PT(k) = P T; [P ; A~](k + 1) = A1 B1^T
+        const Item nn = nxt.ok ? resolve(p, nitem + gridDim.x) : Item{0, 0, 0, false};
         if (tid == 0) {
-            if (nxt.ok) {
-                mbar_expect_tx(mb_tma, kStageBytes);
-                tma_load_3d((void*)qs, &tmq, mb_tma, 0, nxt.h, nxt.tok0);
-                tma_load_3d((void*)ks, &tmk, mb_tma, 0, nxt.h, nxt.tok0);
-                tma_load_3d((void*)gs, &tmg, mb_tma, 0, nxt.h, nxt.tok0);
-            }
+            if (nn.ok) load_item(nn);
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < DK / 8; ++kk)
-                umma_tf32(t_PA, kdesc(A1, kk, kR128), kdesc(B1, kk, kR64), kI64, kk > 0);
-            umma_commit(mb_pa);
-        }
-        if (nxt.ok) {
-            pend |= 1u;
-            tma_par = (it + 1) & 1;
-        }
-        pend |= 2u;
-        KDA_WAIT_OR_EXIT(mb_pa, 2u, it & 1);
-        tc_fence_after();
-        KDA_PHASE(3);
-
-        // ---- P masked in place in TMEM (lanes 0..63, lower incl.); A = beta A~
-        // (lanes 64..127, strictly lower) to the fp32 UT scratch; B1^T into TMEM
-        {
-            float pa[16];
-            tmem_ld16(t_PA + lane_off + q_off, pa);
-            tmem_wait_ld();
-            if (lt < C) {
-                const int r = lt;
-#pragma unroll
-                for (int s2 = 0; s2 < 16; ++s2) pa[s2] = (16 * wg + s2 <= r) ? pa[s2] : 0.f;
-                tmem_st16(t_PA + lane_off + q_off, pa);
-            } else {
-                const int r = lt - C;
-                const float b = beta_s[r];
-#pragma unroll
-                for (int s2 = 0; s2 < 16; ++s2) As[r * LDA + 16 * wg + s2] = (16 * wg + s2 < r) ? b * pa[s2] : 0.f;
-            }
-            float kb[16];
-#pragma unroll
-            for (int s2 = 0; s2 < 16; ++s2) kb[s2] = lt < DK ? swf(B1, 16 * wg + s2, lt, 64) : 0.f;
-            tmem_st16(t_KB + lane_off + q_off, kb);
-        }
-        tmem_wait_st();
-        __syncthreads();
-        KDA_PHASE(4);
-
-        // ---- UT transform (warpgroup 0); channel vectors of the record alongside
-        if (tid < 128) {
-            ut_transform(As, Xs);
-        } else {
-            const int t = tid - 128;
-            float* egl_g = reinterpret_cast<float*>(rec + R::EGL);
-            float* beta_g = reinterpret_cast<float*>(rec + R::BETA);
-            if (t < DK) egl_g[t] = egl_s[t];
-            else if (t >= 128 && t < 128 + C) beta_g[t - 128] = beta_s[t - 128];
-        }
-        __syncthreads();
-        {
-            const int j = tid >> 3, c8 = (tid & 7) * 8;
-            float x[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) x[u] = (c8 + u >= j) ? As[j * LDA + c8 + u] : 0.f;
-            st_row_swf_raw<2>(Top, j, c8, C, x);
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        KDA_PHASE(5);
-
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)    // Z' = B1^T T   (A from TMEM)
+            for (int kk = 0; kk < C / 8; ++kk)
                 umma_tf32_ts(t_Z, t_KB + 8 * kk, kdesc(Top, kk, kR64), kI64, kk > 0);
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)    // PT = P T  (A from TMEM; rows 64..127 unused)
-                umma_tf32_ts(t_PT, t_PA + 8 * kk, kdesc(Top, kk, kR64), kI64, kk > 0);
-            umma_commit(mb_zp);
+            for (int kk = 0; kk < C / 8; ++kk)
+                umma_tf32_ts(t_PT, t_PAc + 8 * kk, kdesc(Top, kk, kR64), kI64, kk > 0);
+            if (nxt.ok) {
+#pragma unroll
+                for (int kk = 0; kk < DK / 8; ++kk)
+                    umma_tf32(t_PAn, kdesc(x.A1, kk, kR128), kdesc(x.B1, kk, kR64), kI64, kk > 0);
+            }
+            umma_commit(mb_mma);
         }
-        pend |= 4u;
-        KDA_WAIT_OR_EXIT(mb_zp, 4u, it & 1);
+        if (nn.ok) {
+            pend |= 1u;
+            tpar = nload & 1;
+            ++nload;
+        }
+        pend |= 2u;
+        KDA_WAIT_OR_EXIT(mb_mma, 2u, nmma & 1);
+        ++nmma;
         tc_fence_after();
-        KDA_PHASE(6);
+        KDA_PHASE(2);
 
-        // ---- Z = diag(e^(G_last - G_m)) Z' and PT, fp16, into the record
+        // ---- record tail of item k, staged in A1: Z = diag(e^(G_last - G_m)) Z', PT, e^G_last, beta
         {
+            unsigned char* stg = x.A1;
             float z[16];
             tmem_ld16(t_Z + lane_off + q_off, z);
-            tmem_wait_ld();
-            if (lt < DK) {
-                const float sc = glm_s[lt];
-#pragma unroll
-                for (int u = 0; u < 16; ++u) z[u] *= sc;
-                st_row_h16(rec + R::Z, lt, 16 * wg, DK, z);
-            }
             float pt[16];
             tmem_ld16(t_PT + lane_off + q_off, pt);
             tmem_wait_ld();
-            if (lt < C) st_row_h16(rec + R::PT, lt, 16 * wg, C, pt);
+            if (lt < DK) {
+                const float sc = vcur.glm[lt];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) z[u] *= sc;
+                st_row_h16(stg, lt, 16 * wg, DK, z);
+            }
+            if (lt < C) st_row_h16(stg + (R::PT - R::Z), lt, 16 * wg, C, pt);
+            if (tid < DK) reinterpret_cast<float*>(stg + (R::EGL - R::Z))[tid] = vcur.egl[tid];
+            else if (tid >= 256 && tid < 256 + C) reinterpret_cast<float*>(stg + (R::BETA - R::Z))[tid - 256] = vcur.beta[tid - 256];
         }
+        // ---- P/A split of item k + 1
+        if (nxt.ok) split_pa(t_PAn, vnxt);
+        fence_proxy_async();
         tc_fence_before();
         __syncthreads();
-        KDA_PHASE(7);
+        if (tid == kStoreIssuer) {
+            bulk_store(p.rec + (size_t)item * R::BYTES + R::Z, x.A1, (uint32_t)(R::BYTES - R::Z));
+            bulk_commit();
+            stored = true;
+        }
+        KDA_PHASE(3);
+        if (!nxt.ok) break;
         item = nitem;
         cur = nxt;
+        nxt = nn;
     }
 
 finish:
     KDA_PHASE_FLUSH
     if (*abort_flag) {
         volatile int never = 0;
-        for (int i = 0; i < 3; ++i)
-            if (pend & (1u << i))
-                (void)mbar_wait(bars + i, i == 0 ? (uint32_t)tma_par : (uint32_t)(it & 1), &never, p.timeout_cycles);
+        if (pend & 1u) (void)mbar_wait(mb_tma, (uint32_t)tpar, &never, p.timeout_cycles);
+        if (pend & 2u) (void)mbar_wait(mb_mma, (uint32_t)(nmma & 1), &never, p.timeout_cycles);
     }
+    if (tid == kStoreIssuer && stored) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -461,19 +546,29 @@ __device__ __forceinline__ uint64_t mn_desc(const unsigned char* tile, int kk, i
 }
 
 // Output rows [0, L) of one chunk from the TMEM accumulator (lane = row, 16
-// columns per warpgroup), run by the 256 threads of lanes 0..63: rows go to a
-// staging tile, then every warp writes whole row segments (coalesced).
+// columns per warpgroup), run by the 256 threads of lanes 0..63.  Rows are
+// staged in the layout of the output tensor map's boxes (64 rows x 128 bytes,
+// 128-byte swizzle; two boxes for fp32 output); a full chunk leaves with TMA
+// stores issued by one thread, a partial one (the end of a sequence) with
+// coalesced 16-byte row-segment stores.
 template <typename TO>
-__device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost, void* o, size_t row0_off,
-                                             size_t row_stride, int L, int lt, int wg)
+__device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost, const CUtensorMap* tmo, void* o,
+                                             int tok, int h, int col0, size_t row0_off, size_t row_stride, int L,
+                                             int lt, int wg, bool issuer)
 {
-    constexpr int EB = (int)sizeof(TO), RB = NV * EB, CPR = RB / 16, CPT = 16 * EB / 16;
+    constexpr int EB = (int)sizeof(TO);
+    constexpr int CPB = 8;                 // 16-byte chunks per 128-byte box row
+    constexpr int CPT = EB;                // chunks per thread: 16 values
+    constexpr int NBOX = NV * EB / 128;
+    constexpr int CPR = NV * EB / 16;      // chunks per output row segment
     float acc[16];
     tmem_ld16(t_acc, acc);
+    if (issuer) bulk_wait_read();          // the previous chunk's stores have read the tile
     tmem_wait_ld();
+    bar_sync(1, 256);
 #pragma unroll
     for (int u = 0; u < CPT; ++u) {
-        const int k = wg * CPT + u;
+        const int k = wg * CPT + u, box = k / CPB, ci = k % CPB;
         uint4 val;
         if constexpr (EB == 4)
             val = make_uint4(__float_as_uint(acc[4 * u]), __float_as_uint(acc[4 * u + 1]),
@@ -481,16 +576,26 @@ __device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost,
         else
             val = make_uint4(pack_bf16(acc[8 * u], acc[8 * u + 1]), pack_bf16(acc[8 * u + 2], acc[8 * u + 3]),
                              pack_bf16(acc[8 * u + 4], acc[8 * u + 5]), pack_bf16(acc[8 * u + 6], acc[8 * u + 7]));
-        *reinterpret_cast<uint4*>(ost + lt * RB + ((k ^ (lt & (CPR - 1))) << 4)) = val;
+        *reinterpret_cast<uint4*>(ost + box * 8192 + lt * 128 + ((ci ^ (lt & 7)) << 4)) = val;
     }
+    fence_proxy_async();
     bar_sync(1, 256);
-    const int t = wg * 64 + lt;
+    if (L == C) {
+        if (issuer) {
 #pragma unroll
-    for (int pss = 0; pss < C * CPR / 256; ++pss) {
-        const int idx = pss * 256 + t, row = idx / CPR, k = idx % CPR;
-        if (row < L) {
-            const uint4 val = *reinterpret_cast<const uint4*>(ost + row * RB + ((k ^ (row & (CPR - 1))) << 4));
-            *reinterpret_cast<uint4*>(static_cast<unsigned char*>(o) + (row0_off + (size_t)row * row_stride) * EB + k * 16) = val;
+            for (int bx = 0; bx < NBOX; ++bx) tma_store_3d(tmo, ost + bx * 8192, col0 + bx * (128 / EB), h, tok);
+            bulk_commit();
+        }
+    } else {
+        const int t = wg * 64 + lt;
+#pragma unroll
+        for (int pss = 0; pss < C * CPR / 256; ++pss) {
+            const int idx = pss * 256 + t, row = idx / CPR, k = idx % CPR;
+            if (row < L) {
+                const int box = k / CPB, ci = k % CPB;
+                const uint4 val = *reinterpret_cast<const uint4*>(ost + box * 8192 + row * 128 + ((ci ^ (row & 7)) << 4));
+                *reinterpret_cast<uint4*>(static_cast<unsigned char*>(o) + (row0_off + (size_t)row * row_stride) * EB + k * 16) = val;
+            }
         }
     }
 }
@@ -509,7 +614,8 @@ __device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost,
 // one thread complete in issue order).
 template <typename TO, int DK>
 __global__ void __launch_bounds__(NT, 1)
-chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                  const ScanParams p)
 {
     using PL = ScanPlan<DK>;
     using R = Rec<DK>;
@@ -563,6 +669,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
         prefetch_tmap(&tmv);
+        prefetch_tmap(&tmo);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 256);
@@ -604,11 +711,15 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
         }
     }
 
+    // thread 0 issues the MMAs; thread kIssuer every copy (record refills, V
+    // tiles, output stores)
+    constexpr int kIssuer = 32;
+    const bool issuer = tid == kIssuer;
     unsigned pend = 0;                 // bits: 0-1 mb_a[slot], 2-3 mb_b[slot], 4 mb_x, 5 mb_w
     uint32_t apar = 0u, bpar = 0u;     // bit i: phase parity of the pending load of slot i
     int xph = 0, wph = 0;              // commits issued to mb_x / mb_w
     int c = 0;
-    if (tid == 0)
+    if (issuer)
         for (int cc = 0; cc < 2 && cc < nchunks; ++cc) {
             issue_a(cc);
             issue_b(cc);
@@ -654,7 +765,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
         // chunk c - 1's PT Y has completed as well: refill the other slot's
         // second part with chunk c + 1
         if (c >= 1 && c + 1 < nchunks) {
-            if (tid == 0) {
+            if (issuer) {
                 fence_proxy_async();
                 issue_b(c + 1);
             }
@@ -693,14 +804,19 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
                 }
                 st_row_h16(Yb, s, 16 * wg, C, y);
             } else if (c > 0) {
-                store_o_tile<TO>(tmem + 64 * (b ^ 1) + lane_off + q_off, Ost, p.o,
-                                 ((size_t)(tok0 + (c - 1) * C) * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg);
+                const int tk = tok0 + (c - 1) * C;
+                store_o_tile<TO>(tmem + 64 * (b ^ 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
+                                 ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
             }
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
         KDA_PHASE(3);
+        if (issuer && c + 2 < nchunks) {            // X MMA done, V consumed: refill part one
+            fence_proxy_async();
+            issue_a(c + 2);
+        }
 
         if (tid == 0) {
             tc_fence_after();
@@ -711,10 +827,6 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)     // O += PT Y  (rows 64..127: discarded)
                 umma_f16(t_XO, kdesc(slot + R::PT, kk, C * 128), mn_desc(Yb, kk, C), kI, 1);
-            if (c + 2 < nchunks) {                  // X MMA done, V consumed: refill part one
-                fence_proxy_async();
-                issue_a(c + 2);
-            }
         }
         ++wph;
         pend |= 32u;
@@ -739,9 +851,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
-        if (lt < C)
-            store_o_tile<TO>(tmem + 64 * ((nchunks - 1) & 1) + lane_off + q_off, Ost, p.o,
-                             ((size_t)(tok0 + (nchunks - 1) * C) * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg);
+        if (lt < C) {
+            const int tk = tok0 + (nchunks - 1) * C;
+            store_o_tile<TO>(tmem + 64 * ((nchunks - 1) & 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
+                             ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
+        }
     }
     if (p.sT && lt < DK) {
         float* dst = p.sT + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg;
@@ -765,6 +879,7 @@ finish:
         if (tid == 0) umma_commit(mb_x);
         (void)mbar_wait(mb_x, (uint32_t)(xph & 1), &never, p.timeout_cycles);
     }
+    if (issuer) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -851,8 +966,10 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
         !make_tmap(&tg, log_alpha, tokens, H, DK, true))
         return cudaErrorInvalidValue;
-    CUtensorMap tv;
-    if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true)) return cudaErrorInvalidValue;
+    CUtensorMap tv, to;
+    if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
+        !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
+        return cudaErrorInvalidValue;
 
     retain_pool_memory();
     unsigned char* ws = nullptr;
@@ -906,7 +1023,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         if (err == cudaSuccess && blocks > 0) {
             if (blocks > 0x7fffffffLL) err = cudaErrorInvalidConfiguration;
             else {
-                sk<<<(unsigned)blocks, NT, ScanPlan<DK>::BYTES, stream>>>(tv, sp);
+                sk<<<(unsigned)blocks, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
                 err = cudaGetLastError();
             }
         }
