@@ -29,6 +29,9 @@
 #include "kda_chunk.cuh"
 #include "kda_tc_util.cuh"
 
+#include <algorithm>
+#include <mutex>
+
 namespace kda {
 namespace split {
 
@@ -84,22 +87,25 @@ struct PrepParams {
     const int32_t* choff;    // varlen: first chunk of each sequence, [nseq + 1]
     unsigned char* rec;
     int nseq, T, H, nch;     // dense: nch chunks per sequence
-    long long nitems;        // (chunk, head) items covered by the records
+    int c_begin, cbs;        // dense: this launch covers chunks [c_begin, c_begin + cbs) of every sequence
+    long long nitems;        // (chunk, head) items of this launch
     long long tokens;
     long long timeout_cycles;
 };
 
 struct Item {
+    long long rec;           // record index: global chunk * H + head
     int tok0, L, h;
     bool ok;
 };
 
 __device__ __forceinline__ Item resolve(const PrepParams& p, long long item)
 {
-    Item it{0, 0, 0, false};
+    Item it{0, 0, 0, 0, false};
     if (item >= p.nitems) return it;
     it.h = (int)(item % p.H);
     const long long j = item / p.H;
+    it.rec = item;
     if (p.cu) {
         if (j >= p.choff[p.nseq]) return it;
         int lo = 0, hi = p.nseq - 1;           // last sequence whose first chunk is <= j
@@ -111,9 +117,10 @@ __device__ __forceinline__ Item resolve(const PrepParams& p, long long item)
         it.tok0 = p.cu[lo] + (int)(j - p.choff[lo]) * C;
         it.L = min(C, p.cu[lo + 1] - it.tok0);
     } else {
-        const int n = (int)(j / p.nch), c = (int)(j % p.nch);
+        const int n = (int)(j / p.cbs), c = p.c_begin + (int)(j % p.cbs);
         it.tok0 = n * p.T + c * C;
         it.L = min(C, p.T - c * C);
+        it.rec = ((long long)n * p.nch + c) * p.H + it.h;
     }
     it.ok = it.L > 0 && it.tok0 >= 0 && it.tok0 + it.L <= p.tokens;
     return it;
@@ -349,7 +356,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 
     long long item = blockIdx.x;
     Item cur = resolve(p, item);
-    Item nxt{0, 0, 0, false};
+    Item nxt{0, 0, 0, 0, false};
     int k = 0;
     if (!cur.ok) goto finish;
 
@@ -363,7 +370,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         KDA_WAIT_OR_EXIT(mb_tma, 1u, 0);
         if (tid >= 128) cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v);
         __syncthreads();
-        build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)item * R::BYTES, cur.L, tid, NT);
+        build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)cur.rec * R::BYTES, cur.L, tid, NT);
     }
     fence_proxy_async();
     tc_fence_before();
@@ -415,7 +422,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
             if (!bar_or(3, 384, !ok)) {
                 cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v);
-                build_operands<DK>(x, vnxt, p.rec + (size_t)nitem * R::BYTES, nxt.L, t, 384);
+                build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384);
             }
         }
         fence_proxy_async();
@@ -425,7 +432,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         KDA_PHASE(1);
 
         // ---- MMA round: Z'(k) = B1^T T, PT(k) = P T; [P ; A~](k + 1) = A1 B1^T
-        const Item nn = nxt.ok ? resolve(p, nitem + gridDim.x) : Item{0, 0, 0, false};
+        const Item nn = nxt.ok ? resolve(p, nitem + gridDim.x) : Item{0, 0, 0, 0, false};
         if (tid == 0) {
             if (nn.ok) load_item(nn);
             tc_fence_after();
@@ -477,7 +484,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         tc_fence_before();
         __syncthreads();
         if (tid == kStoreIssuer) {
-            bulk_store(p.rec + (size_t)item * R::BYTES + R::Z, x.A1, (uint32_t)(R::BYTES - R::Z));
+            bulk_store(p.rec + (size_t)cur.rec * R::BYTES + R::Z, x.A1, (uint32_t)(R::BYTES - R::Z));
             bulk_commit();
             stored = true;
         }
@@ -508,9 +515,10 @@ finish:
 
 struct ScanParams {
     const __nv_bfloat16* v;
-    const float* s0;
+    const float* s_in;       // state before chunk c_begin (nullptr: zeros)
     void* o;
-    float* sT;
+    float* s_out;            // state after this launch's last chunk (nullptr: not stored)
+    int c_begin, c_end;      // chunk range of this launch (per sequence)
     const int32_t* cu;
     const int32_t* choff;
     const unsigned char* rec;
@@ -658,10 +666,20 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant
     const int col0 = slice * NV;
     int nchunks = (len + C - 1) / C;
     if (j0 < 0 || j0 + nchunks > p.max_chunks || (long long)tok0 + len > p.tokens || tok0 < 0) {
-        if (tid == 0) flag_bad_input();
+        if (tid == 0 && p.c_begin == 0) flag_bad_input();
         nchunks = 0;
         len = 0;
     }
+    // this launch's part of the sequence: chunks [c_begin, c_end)
+    if (p.c_begin > 0 && p.c_begin >= nchunks) return;   // ended in an earlier launch; its state is final
+    {
+        const int lo = min(p.c_begin, nchunks), hi = min(p.c_end, nchunks);
+        tok0 += lo * C;
+        len = max(0, len - lo * C);
+        j0 += lo;
+        nchunks = max(0, hi - lo);
+    }
+    const float* s_src = p.s_in;
 
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
@@ -702,8 +720,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant
     // state rows of this thread
     float S[16];
     {
-        const bool own = lt < DK && p.s0;
-        const float* src = own ? p.s0 + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg : nullptr;
+        const bool own = lt < DK && s_src;
+        const float* src = own ? s_src + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg : nullptr;
 #pragma unroll
         for (int j = 0; j < 16; j += 4) {
             const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -857,8 +875,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant
                              ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
         }
     }
-    if (p.sT && lt < DK) {
-        float* dst = p.sT + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg;
+    if (p.s_out && lt < DK) {
+        float* dst = p.s_out + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg;
 #pragma unroll
         for (int j = 0; j < 16; j += 4)
             *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
@@ -951,16 +969,46 @@ static void retain_pool_memory()
     done[dev] = true;
 }
 
+// Second stream of the current device on which the prep of the next block of
+// chunks runs while the current block is scanned (created on first use).
+static cudaStream_t side_stream()
+{
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+        streams[dev] = nullptr;
+    return streams[dev];
+}
+
+constexpr int kMaxBlocks = 8;
+
+// Number of chunk blocks for a dense problem: the prep of block b + 1 runs on
+// the SMs the scan of block b leaves idle, so blocking pays only when the scan
+// grid leaves room.  KDA_SCAN_BLOCKS overrides (1 = no blocking).
+static int chunk_blocks(int nch, long long scan_ctas, int nsm)
+{
+    const char* e = getenv("KDA_SCAN_BLOCKS");
+    int nb = e ? atoi(e) : 0;
+    if (nb <= 0) nb = (scan_ctas + 32 <= nsm) ? nch / 32 : 1;   // measured: 32+ chunks per block
+    return std::max(1, std::min(std::min(nb, nch), kMaxBlocks));
+}
+
 template <typename TO, int DK>
 static cudaError_t run(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
                        const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens,
                        int H, int dv, long long timeout_cycles, cudaStream_t stream)
 {
     using R = Rec<DK>;
+    const int nsm = sm_count();
     const int nch = cu ? 0 : (T + C - 1) / C;
     const long long max_chunks = cu ? tokens / C + nseq : (long long)nseq * nch;
-    const size_t off_bytes = (((size_t)nseq + 1) * 4 + 1023) & ~(size_t)1023;
-    const size_t bytes = off_bytes + (size_t)max_chunks * H * R::BYTES;
+    const long long scan_ctas = (long long)nseq * H * (dv / NV);
+    if (scan_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const int nb = cu ? 1 : chunk_blocks(nch, scan_ctas, nsm);
+    cudaStream_t side = nb > 1 ? side_stream() : nullptr;
 
     CUtensorMap tq, tk, tg;
     if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
@@ -970,13 +1018,42 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
         !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
         return cudaErrorInvalidValue;
+    auto pk = chunk_prep_kernel<DK>;
+    auto sk = chunk_scan_kernel<TO, DK>;
+    cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
+    if (err != cudaSuccess) return err;
+
+    // events of the two-stream schedule (created last: no early return leaks them)
+    cudaEvent_t ev[kMaxBlocks + 1];
+    int nev = 0;
+    if (side) {
+        for (; nev <= nb; ++nev)
+            if (cudaEventCreateWithFlags(&ev[nev], cudaEventDisableTiming) != cudaSuccess) break;
+        if (nev <= nb) {   // fall back to one stream
+            for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+            nev = 0;
+            side = nullptr;
+        }
+    }
+    const int nblocks = side ? nb : 1;
+    const int cb = cu ? 0 : (nch + nblocks - 1) / nblocks;     // chunks per block (dense)
+    const size_t off_bytes = (((size_t)nseq + 1) * 4 + 1023) & ~(size_t)1023;
+    const size_t state_bytes = (nblocks > 1 && !sT) ? (size_t)nseq * H * DK * dv * 4 : 0;
+    const size_t rec_off = off_bytes + ((state_bytes + 1023) & ~(size_t)1023);
+    const size_t bytes = rec_off + (size_t)max_chunks * H * R::BYTES;
 
     retain_pool_memory();
     unsigned char* ws = nullptr;
-    cudaError_t err = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
-    if (err != cudaSuccess) return err;
+    err = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
+    if (err != cudaSuccess) {
+        for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+        return err;
+    }
     int32_t* choff = reinterpret_cast<int32_t*>(ws);
-    unsigned char* rec = ws + off_bytes;
+    float* carry = sT ? sT : reinterpret_cast<float*>(ws + off_bytes);
+    unsigned char* rec = ws + rec_off;
 
     if (cu) chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu, nseq, choff);
 
@@ -989,44 +1066,72 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     pp.T = T;
     pp.H = H;
     pp.nch = nch;
-    pp.nitems = max_chunks * H;
     pp.tokens = tokens;
     pp.timeout_cycles = timeout_cycles;
-    auto pk = chunk_prep_kernel<DK>;
-    err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
-    if (err == cudaSuccess && pp.nitems > 0) {
-        const long long grid = std::min<long long>(pp.nitems, sm_count());
-        pk<<<(unsigned)grid, NT, PrepPlan::BYTES, stream>>>(tq, tk, tg, pp);
-        err = cudaGetLastError();
-    }
+    ScanParams sp;
+    sp.v = static_cast<const __nv_bfloat16*>(v);
+    sp.o = o;
+    sp.cu = cu;
+    sp.choff = choff;
+    sp.rec = rec;
+    sp.nseq = nseq;
+    sp.T = T;
+    sp.H = H;
+    sp.DV = dv;
+    sp.nch = nch;
+    sp.max_chunks = max_chunks;
+    sp.tokens = tokens;
+    sp.timeout_cycles = timeout_cycles;
 
-    if (err == cudaSuccess) {
-        ScanParams sp;
-        sp.v = static_cast<const __nv_bfloat16*>(v);
-        sp.s0 = s0;
-        sp.o = o;
-        sp.sT = sT;
-        sp.cu = cu;
-        sp.choff = choff;
-        sp.rec = rec;
-        sp.nseq = nseq;
-        sp.T = T;
-        sp.H = H;
-        sp.DV = dv;
-        sp.nch = nch;
-        sp.max_chunks = max_chunks;
-        sp.tokens = tokens;
-        sp.timeout_cycles = timeout_cycles;
-        auto sk = chunk_scan_kernel<TO, DK>;
-        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
-        const long long blocks = (long long)nseq * H * (dv / NV);
-        if (err == cudaSuccess && blocks > 0) {
-            if (blocks > 0x7fffffffLL) err = cudaErrorInvalidConfiguration;
-            else {
-                sk<<<(unsigned)blocks, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
-                err = cudaGetLastError();
+    auto launch_prep = [&](int b, cudaStream_t st, long long grid_cap) {
+        if (cu) {
+            pp.c_begin = 0;
+            pp.cbs = 0;
+            pp.nitems = max_chunks * H;
+        } else {
+            pp.c_begin = b * cb;
+            pp.cbs = std::max(0, std::min(cb, nch - b * cb));
+            pp.nitems = (long long)nseq * pp.cbs * H;
+        }
+        if (pp.nitems <= 0) return cudaSuccess;
+        const long long grid = std::max(1LL, std::min(pp.nitems, grid_cap));
+        pk<<<(unsigned)grid, NT, PrepPlan::BYTES, st>>>(tq, tk, tg, pp);
+        return cudaGetLastError();
+    };
+    auto launch_scan = [&](int b) {
+        sp.c_begin = cu ? 0 : b * cb;
+        sp.c_end = (cu || b == nblocks - 1) ? 0x7fffffff : (b + 1) * cb;
+        sp.s_in = b == 0 ? s0 : carry;
+        sp.s_out = (b == nblocks - 1) ? sT : carry;
+        if (scan_ctas <= 0) return cudaSuccess;
+        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
+        return cudaGetLastError();
+    };
+
+    if (nblocks == 1) {
+        err = launch_prep(0, stream, nsm);
+        if (err == cudaSuccess) err = launch_scan(0);
+    } else {
+        // fork: the side stream starts after everything queued on `stream`;
+        // the scan of block b waits for the prep of block b; the prep of
+        // block b + 1 shares the GPU with that scan
+        err = cudaEventRecord(ev[0], stream);
+        if (err == cudaSuccess) err = cudaStreamWaitEvent(side, ev[0], 0);
+        if (err == cudaSuccess) err = launch_prep(0, side, nsm);
+        if (err == cudaSuccess) err = cudaEventRecord(ev[1], side);
+        for (int b = 0; b < nblocks && err == cudaSuccess; ++b) {
+            err = cudaStreamWaitEvent(stream, ev[b + 1], 0);
+            if (err == cudaSuccess) err = launch_scan(b);
+            if (err == cudaSuccess && b + 1 < nblocks) {
+                err = launch_prep(b + 1, side, std::max(1LL, nsm - scan_ctas));
+                if (err == cudaSuccess) err = cudaEventRecord(ev[b + 2], side);
             }
         }
+        if (err != cudaSuccess) {   // join the side stream back whatever happened
+            cudaEventRecord(ev[nblocks], side);
+            cudaStreamWaitEvent(stream, ev[nblocks], 0);
+        }
+        for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
     }
     const cudaError_t ferr = cudaFreeAsync(ws, stream);
     return err != cudaSuccess ? err : ferr;

@@ -1,0 +1,90 @@
+"""GPU: the two-stream blocked schedule of the tensor-core chunk forward.
+
+For dense inputs the library splits the chunk axis into blocks: the prep pass
+of block b + 1 runs on a second stream while block b is scanned, and the state
+crosses block boundaries through memory as the same fp32 values it has in
+registers.  Every block count must therefore give results bit-identical to
+the single-block schedule (KDA_SCAN_BLOCKS=1), which itself matches the
+oracle.  The block count is read from the environment on every call.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import gated_delta_rule_133_b200 as kda
+from gated_delta_rule_133_b200.inputs import Workload, make_inputs
+from tests._helpers import TOL_BF16, f64, norm_max_err
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _inputs(B, T, H, d, seed, init=0.05):
+    w = Workload("blocked", "dense", B, T, H, d, d, "bf16", -3.0, init, seed=seed)
+    x = make_inputs(w, "cpu")
+    return x, {k: (None if v is None else v.to(DEV)) for k, v in x.items()}
+
+
+def _call(g, blocks, initial_state="inputs", **kw):
+    s0 = g["initial_state"] if isinstance(initial_state, str) else initial_state
+    old = os.environ.get("KDA_SCAN_BLOCKS")
+    os.environ["KDA_SCAN_BLOCKS"] = str(blocks)
+    try:
+        out = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], s0, **kw)
+        torch.cuda.synchronize()
+        kda.kda_check()
+    finally:
+        if old is None:
+            del os.environ["KDA_SCAN_BLOCKS"]
+        else:
+            os.environ["KDA_SCAN_BLOCKS"] = old
+    return out
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_block_counts_bit_identical(d):
+    """T = 33 chunks + a ragged tail: even, uneven and empty trailing blocks."""
+    x, g = _inputs(2, 33 * 64 + 37, 3, d, seed=41)
+    o1, s1 = _call(g, 1)
+    for nb in (2, 3, 5, 8):
+        o, s = _call(g, nb)
+        assert torch.equal(o, o1), nb
+        assert torch.equal(s, s1), nb
+    # and the single-block result is the oracle's
+    B, T, H = x["q"].shape[:3]
+    flat = lambda t: f64(t).reshape(B * T, H, *t.shape[3:])
+    o_ref, s_ref = oracle.recurrence(flat(x["q"]), flat(x["k"]), flat(x["v"]), f64(x["beta"]).reshape(B * T, H),
+                                     flat(x["log_alpha"]), np.arange(B + 1) * T, f64(x["initial_state"]))
+    assert norm_max_err(f64(o1).reshape(B * T, H, d), o_ref) <= TOL_BF16
+    assert norm_max_err(f64(s1), s_ref) <= TOL_BF16
+
+
+def test_blocked_without_final_state():
+    """No final state requested: the carry lives in the workspace."""
+    x, g = _inputs(2, 40 * 64, 2, 128, seed=42)
+    o1, _ = _call(g, 1)
+    o4, s4 = _call(g, 4, output_final_state=False)
+    assert s4 is None
+    assert torch.equal(o4, o1)
+
+
+def test_blocked_in_place_state():
+    """initial_state and final_state the same buffer, several blocks."""
+    x, g = _inputs(1, 48 * 64, 2, 128, seed=43)
+    o1, s1 = _call(g, 1)
+    st = g["initial_state"].clone()
+    o3, _ = _call(g, 3, initial_state=st, final_state=st)
+    assert torch.equal(o3, o1)
+    assert torch.equal(st, s1)
+
+
+def test_blocked_bf16_output():
+    x, g = _inputs(2, 36 * 64, 2, 128, seed=44)
+    o1, s1 = _call(g, 1, o_dtype=torch.bfloat16)
+    o4, s4 = _call(g, 4, o_dtype=torch.bfloat16)
+    assert torch.equal(o4, o1)
+    assert torch.equal(s4, s1)
