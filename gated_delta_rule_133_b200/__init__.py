@@ -18,7 +18,7 @@ import torch
 from . import _lib
 from ._lib import KdaError
 
-__all__ = ["kda_chunk_fwd", "kda_varlen_fwd", "kda_recurrent_step", "kda_check", "KdaError"]
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_varlen_fwd", "kda_recurrent_step", "kda_check", "KdaError"]
 
 _DTYPES = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
 
@@ -52,6 +52,21 @@ def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final
     log_alpha [B, T, H, dk] fp32; initial_state [B, H, dk, dv] fp32 or None.
     Returns (o [B, T, H, dv] in o_dtype (or o's dtype when o is given),
     final_state [B, H, dk, dv] or None)."""
+    return _dense_fwd("kda_chunk_fwd", q, k, v, beta, log_alpha, initial_state, o, final_state,
+                      output_final_state, o_dtype, chunk, stream)
+
+
+def kda_chunk_fwd_noalloc(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final_state=None,
+                          output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None):
+    """kda_chunk_fwd with every intermediate in the library's fixed per-device
+    area (no allocation by the library).  Calls must be ordered with respect to
+    each other; raises KdaError (unsupported) when the problem does not fit."""
+    return _dense_fwd("kda_chunk_fwd_noalloc", q, k, v, beta, log_alpha, initial_state, o, final_state,
+                      output_final_state, o_dtype, chunk, stream)
+
+
+def _dense_fwd(symbol, q, k, v, beta, log_alpha, initial_state, o, final_state, output_final_state, o_dtype,
+               chunk, stream):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev, dt = q.device, q.dtype
@@ -72,7 +87,7 @@ def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final
         final_state = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
     if final_state is not None:
         _check(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
-    _lib.call("kda_chunk_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
+    _lib.call(symbol, _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
               _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk,
               _DTYPES[dt], _DTYPES[o.dtype], _stream(stream))
     return o, final_state

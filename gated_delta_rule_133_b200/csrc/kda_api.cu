@@ -122,6 +122,27 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
                      dv, dtype, o_dtype, s);
 }
 
+kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* beta,
+                                 const float* log_alpha, const float* initial_state, void* o,
+                                 float* final_state, int B, int T, int H, int dk, int dv, int chunk,
+                                 kda_dtype dtype, kda_dtype o_dtype, void* stream)
+{
+    if (B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    const long long tokens = (long long)B * T;
+    kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, tokens, H,
+                              dk, dv, chunk, dtype, o_dtype);
+    if (st != KDA_OK) return st;
+    if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tokens == 0) return copy_state(initial_state, final_state, (size_t)B * H * dk * dv, s);
+    if (!kda::chunk_fwd_tc_supported(dk, dv, dtype))   // the CUDA-core kernel needs no scratch
+        return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, initial_state, o, final_state, nullptr, B,
+                                             T, H, dk, dv, dtype, o_dtype, s));
+    if (!kda::chunk_fwd_noalloc_fits(B, T, H, dk, dv, final_state != nullptr)) return KDA_ERR_UNSUPPORTED;
+    return from_cuda(kda::chunk_fwd_noalloc(q, k, v, beta, log_alpha, initial_state, o, final_state, B, T, tokens,
+                                            H, dk, dv, o_dtype, timeout_cycles(), s));
+}
+
 kda_status kda_varlen_fwd(const void* q, const void* k, const void* v, const float* beta,
                           const float* log_alpha, const int32_t* cu_seqlens, int N,
                           const float* initial_state, void* o, float* final_state, int T, int H,

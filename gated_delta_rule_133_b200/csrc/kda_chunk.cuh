@@ -34,4 +34,13 @@ cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const f
                             int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
                             long long timeout_cycles, cudaStream_t stream);
 
+// Same as chunk_fwd_split for dense inputs, with every intermediate in a
+// fixed library-owned device area instead of a stream-ordered allocation;
+// chunk_fwd_noalloc_fits tells whether a problem fits that area.
+bool chunk_fwd_noalloc_fits(int nseq, int T, int H, int dk, int dv, bool has_final);
+cudaError_t chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* beta,
+                              const float* log_alpha, const float* s0, void* o, float* sT, int nseq, int T,
+                              long long tokens, int H, int dk, int dv, kda_dtype o_dtype, long long timeout_cycles,
+                              cudaStream_t stream);
+
 }  // namespace kda

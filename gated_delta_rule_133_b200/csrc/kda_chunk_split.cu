@@ -88,6 +88,7 @@ struct PrepParams {
     unsigned char* rec;
     int nseq, T, H, nch;     // dense: nch chunks per sequence
     int c_begin, cbs;        // dense: this launch covers chunks [c_begin, c_begin + cbs) of every sequence
+    int rs, rc0;             // dense: record of (n, c, h) = (n * rs + c - rc0) * H + h
     long long nitems;        // (chunk, head) items of this launch
     long long tokens;
     long long timeout_cycles;
@@ -120,7 +121,7 @@ __device__ __forceinline__ Item resolve(const PrepParams& p, long long item)
         const int n = (int)(j / p.cbs), c = p.c_begin + (int)(j % p.cbs);
         it.tok0 = n * p.T + c * C;
         it.L = min(C, p.T - c * C);
-        it.rec = ((long long)n * p.nch + c) * p.H + it.h;
+        it.rec = ((long long)n * p.rs + c - p.rc0) * p.H + it.h;
     }
     it.ok = it.L > 0 && it.tok0 >= 0 && it.tok0 + it.L <= p.tokens;
     return it;
@@ -523,6 +524,7 @@ struct ScanParams {
     const int32_t* choff;
     const unsigned char* rec;
     int nseq, T, H, DV, nch;
+    int rs, rc0;             // dense: record of (n, c, h) = (n * rs + c - rc0) * H + h
     long long max_chunks;    // records available per head
     long long tokens;
     long long timeout_cycles;
@@ -661,11 +663,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant
         n = rank;
         tok0 = n * p.T;
         len = p.T;
-        j0 = (long long)n * p.nch;
+        j0 = (long long)n * p.rs - p.rc0;
     }
     const int col0 = slice * NV;
     int nchunks = (len + C - 1) / C;
-    if (j0 < 0 || j0 + nchunks > p.max_chunks || (long long)tok0 + len > p.tokens || tok0 < 0) {
+    if ((long long)tok0 + len > p.tokens || tok0 < 0) {
         if (tid == 0 && p.c_begin == 0) flag_bad_input();
         nchunks = 0;
         len = 0;
@@ -678,6 +680,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant
         len = max(0, len - lo * C);
         j0 += lo;
         nchunks = max(0, hi - lo);
+    }
+    if (nchunks > 0 && (j0 < 0 || j0 + nchunks > p.max_chunks)) {   // records outside the buffer
+        if (tid == 0) flag_bad_input();
+        nchunks = 0;
+        len = 0;
     }
     const float* s_src = p.s_in;
 
@@ -1066,6 +1073,8 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     pp.T = T;
     pp.H = H;
     pp.nch = nch;
+    pp.rs = nch;
+    pp.rc0 = 0;
     pp.tokens = tokens;
     pp.timeout_cycles = timeout_cycles;
     ScanParams sp;
@@ -1079,6 +1088,8 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     sp.H = H;
     sp.DV = dv;
     sp.nch = nch;
+    sp.rs = nch;
+    sp.rc0 = 0;
     sp.max_chunks = max_chunks;
     sp.tokens = tokens;
     sp.timeout_cycles = timeout_cycles;
@@ -1137,6 +1148,161 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     return err != cudaSuccess ? err : ferr;
 }
 
+// ============================================================== allocation-free variant
+
+// Library-owned scratch of kda_chunk_fwd_noalloc: the operand records of two
+// blocks of chunks used as a ring, and the carried state when the caller
+// keeps no final state.  One area per device, so calls that use it must be
+// ordered with respect to each other (one stream, or synchronised).
+constexpr size_t kScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+static unsigned char* scratch_area()
+{
+    static std::mutex mu;
+    static void* areas[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!areas[dev] && cudaGetSymbolAddress(&areas[dev], g_scratch) != cudaSuccess) areas[dev] = nullptr;
+    return static_cast<unsigned char*>(areas[dev]);
+}
+
+static size_t carry_bytes(int nseq, int H, int dk, int dv, bool has_final)
+{
+    return has_final ? 0 : (((size_t)nseq * H * dk * dv * 4 + 1023) & ~(size_t)1023);
+}
+
+template <int DK>
+static long long noalloc_block(int nseq, int H, int dv, bool has_final, int nch)
+{
+    const size_t per_chunk = (size_t)nseq * H * Rec<DK>::BYTES;   // one chunk of every (sequence, head)
+    const size_t carry = carry_bytes(nseq, H, DK, dv, has_final);
+    if (per_chunk == 0 || carry + 2 * per_chunk > kScratchBytes) return 0;
+    return std::min<long long>(nch, (long long)((kScratchBytes - carry) / (2 * per_chunk)));
+}
+
+template <typename TO, int DK>
+static cudaError_t run_noalloc(const void* q, const void* k, const void* v, const float* beta,
+                               const float* log_alpha, const float* s0, void* o, float* sT, int nseq, int T,
+                               long long tokens, int H, int dv, long long timeout_cycles, cudaStream_t stream)
+{
+    using R = Rec<DK>;
+    const int nsm = sm_count();
+    const int nch = (T + C - 1) / C;
+    const long long cb = noalloc_block<DK>(nseq, H, dv, sT != nullptr, nch);
+    if (cb <= 0) return cudaErrorInvalidValue;
+    const int nblocks = (int)((nch + cb - 1) / cb);
+    const long long scan_ctas = (long long)nseq * H * (dv / NV);
+    if (scan_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    unsigned char* area = scratch_area();
+    if (!area) return cudaErrorInvalidSymbol;
+    const size_t carry_sz = carry_bytes(nseq, H, DK, dv, sT != nullptr);
+    float* carry = sT ? sT : reinterpret_cast<float*>(area);
+    unsigned char* ring[2] = {area + carry_sz, area + carry_sz + (size_t)cb * nseq * H * R::BYTES};
+
+    CUtensorMap tq, tk, tg, tv, to;
+    if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
+        !make_tmap(&tg, log_alpha, tokens, H, DK, true) || !make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
+        !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
+        return cudaErrorInvalidValue;
+    auto pk = chunk_prep_kernel<DK>;
+    auto sk = chunk_scan_kernel<TO, DK>;
+    cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
+    if (err != cudaSuccess) return err;
+
+    PrepParams pp{};
+    pp.beta = beta;
+    pp.nseq = nseq;
+    pp.T = T;
+    pp.H = H;
+    pp.nch = nch;
+    pp.rs = (int)cb;
+    pp.tokens = tokens;
+    pp.timeout_cycles = timeout_cycles;
+    ScanParams sp{};
+    sp.v = static_cast<const __nv_bfloat16*>(v);
+    sp.o = o;
+    sp.nseq = nseq;
+    sp.T = T;
+    sp.H = H;
+    sp.DV = dv;
+    sp.nch = nch;
+    sp.rs = (int)cb;
+    sp.max_chunks = (long long)nseq * cb;
+    sp.tokens = tokens;
+    sp.timeout_cycles = timeout_cycles;
+
+    // block b: chunks [b cb, (b + 1) cb) of every sequence, records in ring[b % 2]
+    auto launch_prep = [&](int b, cudaStream_t st, long long grid_cap) {
+        pp.rec = ring[b & 1];
+        pp.c_begin = (int)(b * cb);
+        pp.rc0 = pp.c_begin;
+        pp.cbs = (int)std::min<long long>(cb, nch - b * cb);
+        pp.nitems = (long long)nseq * pp.cbs * H;
+        if (pp.nitems <= 0) return cudaSuccess;
+        const long long grid = std::max(1LL, std::min(pp.nitems, grid_cap));
+        pk<<<(unsigned)grid, NT, PrepPlan::BYTES, st>>>(tq, tk, tg, pp);
+        return cudaGetLastError();
+    };
+    auto launch_scan = [&](int b) {
+        sp.rec = ring[b & 1];
+        sp.c_begin = (int)(b * cb);
+        sp.rc0 = sp.c_begin;
+        sp.c_end = b == nblocks - 1 ? 0x7fffffff : (int)((b + 1) * cb);
+        sp.s_in = b == 0 ? s0 : carry;
+        sp.s_out = b == nblocks - 1 ? sT : carry;
+        if (scan_ctas <= 0) return cudaSuccess;
+        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
+        return cudaGetLastError();
+    };
+
+    cudaStream_t side = nblocks > 1 ? side_stream() : nullptr;
+    cudaEvent_t ev[5];
+    int nev = 0;
+    if (side) {
+        for (; nev < 5; ++nev)
+            if (cudaEventCreateWithFlags(&ev[nev], cudaEventDisableTiming) != cudaSuccess) break;
+        if (nev < 5) {
+            for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+            nev = 0;
+            side = nullptr;
+        }
+    }
+    if (!side) {   // one stream: blocks in order, no overlap
+        for (int b = 0; b < nblocks && err == cudaSuccess; ++b) {
+            err = launch_prep(b, stream, nsm);
+            if (err == cudaSuccess) err = launch_scan(b);
+        }
+        return err;
+    }
+    // two streams: prep(b + 1) overlaps scan(b); prep(b + 2) reuses the ring
+    // slot of block b only after scan(b) has finished with it
+    cudaEvent_t ev_prep[2] = {ev[1], ev[2]}, ev_scan[2] = {ev[3], ev[4]};
+    err = cudaEventRecord(ev[0], stream);
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(side, ev[0], 0);
+    if (err == cudaSuccess) err = launch_prep(0, side, nsm);
+    if (err == cudaSuccess) err = cudaEventRecord(ev_prep[0], side);
+    for (int b = 0; b < nblocks && err == cudaSuccess; ++b) {
+        err = cudaStreamWaitEvent(stream, ev_prep[b & 1], 0);
+        if (err == cudaSuccess) err = launch_scan(b);
+        if (err == cudaSuccess) err = cudaEventRecord(ev_scan[b & 1], stream);
+        if (err == cudaSuccess && b + 1 < nblocks) {
+            if (b + 1 >= 2) err = cudaStreamWaitEvent(side, ev_scan[(b + 1) & 1], 0);
+            if (err == cudaSuccess) err = launch_prep(b + 1, side, scan_ctas < nsm ? nsm - scan_ctas : nsm);
+            if (err == cudaSuccess) err = cudaEventRecord(ev_prep[(b + 1) & 1], side);
+        }
+    }
+    if (err != cudaSuccess) {   // join the side stream back whatever happened
+        cudaEventRecord(ev[0], side);
+        cudaStreamWaitEvent(stream, ev[0], 0);
+    }
+    for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+    return err;
+}
+
 }  // namespace split
 
 cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const float* beta,
@@ -1150,6 +1316,28 @@ cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const f
     } else {
         if (dk == 128) return split::run<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
         if (dk == 64) return split::run<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+bool chunk_fwd_noalloc_fits(int nseq, int T, int H, int dk, int dv, bool has_final)
+{
+    const int nch = (T + tcu::C - 1) / tcu::C;
+    return dk == 128 ? split::noalloc_block<128>(nseq, H, dv, has_final, nch) > 0
+                     : split::noalloc_block<64>(nseq, H, dv, has_final, nch) > 0;
+}
+
+cudaError_t chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* beta,
+                              const float* log_alpha, const float* s0, void* o, float* sT, int nseq, int T,
+                              long long tokens, int H, int dk, int dv, kda_dtype o_dtype, long long timeout_cycles,
+                              cudaStream_t stream)
+{
+    if (o_dtype == KDA_F32) {
+        if (dk == 128) return split::run_noalloc<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 64) return split::run_noalloc<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+    } else {
+        if (dk == 128) return split::run_noalloc<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 64) return split::run_noalloc<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
     }
     return cudaErrorInvalidValue;
 }

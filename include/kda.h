@@ -84,6 +84,30 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          kda_dtype dtype, kda_dtype o_dtype, void* stream);
 
 /*
+ * kda_chunk_fwd computed without allocating any memory.  The method the pages
+ * describe has no counterpart of this call: it differs from kda_chunk_fwd
+ * only in where the tensor-core path keeps its intermediates (the per-chunk
+ * operand records and, when final_state is NULL, the state carried between
+ * blocks of chunks), namely a fixed 64 MiB area the library owns on each
+ * device, instead of stream-ordered allocations.  Arguments, layouts and
+ * results are those of kda_chunk_fwd (results bit-identical to it).
+ *
+ *   - Problems whose records for one 64-token chunk of every (sequence, head),
+ *     twice over, plus the carried state do not fit the area return
+ *     KDA_ERR_UNSUPPORTED before anything is launched (bf16 inputs, d_k = 128:
+ *     B * H up to 577 with final_state, fewer without).
+ *   - The area is shared by all calls on a device: calls of this function
+ *     must be ordered with respect to each other (one stream, or synchronised
+ *     by the caller).  Inputs the tensor-core path does not take (fp32) run on
+ *     the CUDA-core kernel, which needs no scratch.
+ */
+kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                 const float* beta, const float* log_alpha,
+                                 const float* initial_state, void* o, float* final_state,
+                                 int B, int T, int H, int dk, int dv, int chunk,
+                                 kda_dtype dtype, kda_dtype o_dtype, void* stream);
+
+/*
  * Same computation over N variable-length sequences packed along one token
  * axis (B = 1).  The state restarts (from initial_state[n] or zero) at every
  * sequence boundary; the last chunk of each sequence may be shorter than 64.

@@ -94,3 +94,15 @@ def test_python_binding_rejects_bad_tensors():
         kda.kda_chunk_fwd(q, q, q, torch.zeros(1, 8, 2), torch.zeros(1, 8, 2, 64))
     with pytest.raises(ValueError):
         kda.kda_chunk_fwd(q, q, q.to(torch.float64), torch.zeros(1, 8, 2), q)
+
+
+def test_noalloc_validation():
+    """The allocation-free entry point validates like kda_chunk_fwd and rejects,
+    on the host, problems whose intermediates do not fit its fixed area."""
+    f = _lib.load().kda_chunk_fwd_noalloc
+    ok = (P, P, P, P, P, None, P, P, 1, 8, 2, 128, 128, 64, 1, 0, None)
+    assert f(*ok[:8], -1, *ok[9:]) == _lib.KDA_ERR_INVALID_ARG
+    assert f(None, *ok[1:]) == _lib.KDA_ERR_INVALID_ARG
+    assert f(*ok[:11], 96, *ok[12:]) == _lib.KDA_ERR_UNSUPPORTED
+    # 10 x 64 (sequence, head) pairs: two chunks of records exceed the 64 MiB area
+    assert f(*ok[:8], 10, 8, 64, *ok[11:]) == _lib.KDA_ERR_UNSUPPORTED
