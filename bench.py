@@ -182,6 +182,21 @@ def recorded_traffic(kernel_key):
     return rec.get("dram_bytes_per_launch")
 
 
+def chunk_launches(B, T, H, dv, device):
+    """Kernels one dense chunk-forward call launches: the tensor-core path runs
+    a prep and a scan kernel per block of chunks, with one block per 32 chunks
+    (at most 8) when the scan grid leaves at least 32 SMs for the prep of the
+    next block (the library's own rule; KDA_SCAN_BLOCKS overrides it)."""
+    kind = os.environ.get("KDA_CHUNK_KERNEL", "")
+    if kind in ("fused", "simt") or os.environ.get("KDA_FORCE_SIMT") == "1":
+        return 1
+    nch = (T + 63) // 64
+    nsm = torch.cuda.get_device_properties(device).multi_processor_count
+    env = int(os.environ.get("KDA_SCAN_BLOCKS", "0") or 0)
+    nb = env if env > 0 else (nch // 32 if B * H * (dv // 64) + 32 <= nsm else 1)
+    return 2 * max(1, min(nb, nch, 8))
+
+
 def event_pairs(n):
     return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
 
@@ -264,7 +279,7 @@ def run_ours(args, world, rank, local):
         "decode": dec,
         "other_workloads": others,
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * chunk_launches(w.B, w.T, w.H, w.dv, device),
         "clocks": clocks,
     }
     return line, rank
