@@ -160,10 +160,17 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {
+    # the files whose code a recorded ncu capture of each path depends on
+    "chunk_fwd_prefill": ["kda_chunk_split.cu", "kda_tc_util.cuh", "kda_sm100.cuh", "kda_common.cuh"],
+    "decode_step": ["kda_decode.cu", "kda_common.cuh"],
+}
+
+
+def kernel_source_hash(kernel_key="chunk_fwd_prefill"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_133_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel_key]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -177,7 +184,7 @@ def recorded_traffic(kernel_key):
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel_key)
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(kernel_key):
         return None
     return rec.get("dram_bytes_per_launch")
 
