@@ -190,17 +190,22 @@ def recorded_traffic(kernel_key):
 
 
 def chunk_launches(B, T, H, dv, device):
-    """Kernels one dense chunk-forward call launches: the tensor-core path runs
-    a prep and a scan kernel per block of chunks, with one block per 32 chunks
-    (at most 8) when the scan grid leaves at least 32 SMs for the prep of the
-    next block (the library's own rule; KDA_SCAN_BLOCKS overrides it)."""
+    """Kernels one dense chunk-forward call launches (the library's own rule):
+    one cooperative kernel (prep and scan CTAs together) when the scan grid
+    leaves at least 32 SMs; otherwise a prep and a scan kernel per block of
+    chunks, one block per 32 chunks (at most 8) when the scan grid leaves 32 SMs
+    (KDA_SCAN_BLOCKS / KDA_CHUNK_SCHEDULE override)."""
     kind = os.environ.get("KDA_CHUNK_KERNEL", "")
     if kind in ("fused", "simt") or os.environ.get("KDA_FORCE_SIMT") == "1":
         return 1
     nch = (T + 63) // 64
     nsm = torch.cuda.get_device_properties(device).multi_processor_count
+    room = B * H * (dv // 64) + 32 <= nsm
+    sched = os.environ.get("KDA_CHUNK_SCHEDULE")
     env = int(os.environ.get("KDA_SCAN_BLOCKS", "0") or 0)
-    nb = env if env > 0 else (nch // 32 if B * H * (dv // 64) + 32 <= nsm else 1)
+    if room and not env and (sched is None or sched == "coop"):
+        return 1
+    nb = env if env > 0 else (nch // 32 if room else 1)
     return 2 * max(1, min(nb, nch, 8))
 
 

@@ -30,6 +30,7 @@
 #include "kda_tc_util.cuh"
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 namespace kda {
@@ -79,6 +80,38 @@ __device__ __forceinline__ void st_row_h16(unsigned char* tile, int row, int col
         pend &= ~(bit);                                                                      \
     } while (0)
 
+// Cooperative schedule: a prep CTA publishes a finished record (its generic
+// stores ordered by a CTA barrier, its bulk stores completed) with a release
+// store; a scan CTA's copy thread acquires the flag, with a bounded wait,
+// before its bulk copies read the record.
+__device__ __forceinline__ void publish(unsigned* flag)
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __threadfence();
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(1u) : "memory");
+}
+
+__device__ __forceinline__ bool wait_ready(const unsigned* flag, volatile int* abort, long long limit_cycles)
+{
+    const long long t0 = clock64();
+    for (uint32_t i = 0;; ++i) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            return true;
+        }
+        __nanosleep(32);
+        if ((i & 15u) == 15u) {
+            if (*abort) return false;
+            if (clock64() - t0 > limit_cycles) break;
+        }
+    }
+    *abort = 1;
+    flag_timeout();
+    return false;
+}
+
 // ============================================================== pass 1: prep
 
 struct PrepParams {
@@ -92,6 +125,7 @@ struct PrepParams {
     long long nitems;        // (chunk, head) items of this launch
     long long tokens;
     long long timeout_cycles;
+    unsigned* ready;         // cooperative schedule: ready[record] = 1 once the record is complete
 };
 
 struct Item {
@@ -117,8 +151,8 @@ __device__ __forceinline__ Item resolve(const PrepParams& p, long long item)
         }
         it.tok0 = p.cu[lo] + (int)(j - p.choff[lo]) * C;
         it.L = min(C, p.cu[lo + 1] - it.tok0);
-    } else {
-        const int n = (int)(j / p.cbs), c = p.c_begin + (int)(j % p.cbs);
+    } else {   // chunk outermost, then sequence: the scans of all sequences advance together
+        const int n = (int)(j % p.nseq), c = p.c_begin + (int)(j / p.nseq);
         it.tok0 = n * p.T + c * C;
         it.L = min(C, p.T - c * C);
         it.rec = ((long long)n * p.rs + c - p.rc0) * p.H + it.h;
@@ -213,12 +247,12 @@ __device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t,
     bar_sync(2, 384);
 }
 
-// Operands of one item, by `nthr` threads (t = 0..nthr-1): A1 = [q E; k E]
+// Operands of rows [row_lo, row_hi) of one item, by `nthr` threads (t = 0..nthr-1): A1 = [q E; k E]
 // and B1 = k / E (tf32, smem) for the intra-chunk products; Qh = q e^G and
 // Kh = k e^G (fp16) straight into the record.
 template <int DK>
 __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& v, unsigned char* rec, int L, int t,
-                                               int nthr)
+                                               int nthr, int row_lo, int row_hi)
 {
     using R = Rec<DK>;
     constexpr int NG = DK / 4;
@@ -227,7 +261,7 @@ __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& 
     const float4 m4 = *reinterpret_cast<const float4*>(v.gml + c0);
     const float4 gm4 = *reinterpret_cast<const float4*>(v.gm + c0);
 #pragma unroll 2
-    for (int r = r0; r < C; r += rpp) {
+    for (int r = row_lo + r0; r < row_hi; r += rpp) {
         const float4 g4 = *reinterpret_cast<const float4*>(x.gs + r * DK + c0);
         float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = q4;
         if (r < L) {
@@ -262,9 +296,8 @@ __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& 
 //
 // TMEM: [P ; A~] double-buffered (0, 64), B1^T 128, Z' 192, PT 256.
 template <int DK>
-__global__ void __launch_bounds__(NT, 1)
-chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                  const __grid_constant__ CUtensorMap tmg, const PrepParams p)
+__device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmg,
+                                          const PrepParams& p, int bid, int nblk)
 {
     using PL = PrepPlan;
     using R = Rec<DK>;
@@ -322,6 +355,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     int tpar = 0;                      // parity of the outstanding TMA load
     int nload = 0, nmma = 0;           // loads / commits issued so far
     bool stored = false;               // the store issuer has bulk stores in flight
+    bool unpublished = false;
+    long long stored_rec = 0;
 
     auto load_item = [&](const Item& it) {   // thread 0
         mbar_expect_tx(mb_tma, kStageBytes);
@@ -355,7 +390,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         tmem_wait_st();
     };
 
-    long long item = blockIdx.x;
+    long long item = bid;
     Item cur = resolve(p, item);
     Item nxt{0, 0, 0, 0, false};
     int k = 0;
@@ -371,12 +406,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         KDA_WAIT_OR_EXIT(mb_tma, 1u, 0);
         if (tid >= 128) cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v);
         __syncthreads();
-        build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)cur.rec * R::BYTES, cur.L, tid, NT);
+        build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)cur.rec * R::BYTES, cur.L, tid, NT, 0, C);
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    nxt = resolve(p, item + gridDim.x);
+    nxt = resolve(p, item + nblk);
     if (tid == 0) {
         if (nxt.ok) load_item(nxt);
         tc_fence_after();
@@ -402,7 +437,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         const int vb = k & 1, nb = vb ^ 1;
         const Vec vcur = vec_at(vbase, vb), vnxt = vec_at(vbase, nb);
         const uint32_t t_PAc = tmem + 64 * vb, t_PAn = tmem + 64 * nb;
-        const long long nitem = item + gridDim.x;
+        const long long nitem = item + nblk;
         KDA_PHASE(0);
 
         // ---- UT transform of item k (WG0) | cumsum + operands of item k + 1 (WG1-3)
@@ -423,17 +458,22 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
             if (!bar_or(3, 384, !ok)) {
                 cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v);
-                build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384);
+                build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384, 0, C);
             }
         }
         fence_proxy_async();
         tc_fence_before();
         if (__syncthreads_or(*abort_flag)) goto finish;
         if (nxt.ok) pend &= ~1u;
+        if (p.ready && tid == kStoreIssuer && unpublished) {
+            bulk_wait_all();
+            publish(p.ready + stored_rec);
+            unpublished = false;
+        }
         KDA_PHASE(1);
 
         // ---- MMA round: Z'(k) = B1^T T, PT(k) = P T; [P ; A~](k + 1) = A1 B1^T
-        const Item nn = nxt.ok ? resolve(p, nitem + gridDim.x) : Item{0, 0, 0, 0, false};
+        const Item nn = nxt.ok ? resolve(p, nitem + nblk) : Item{0, 0, 0, 0, false};
         if (tid == 0) {
             if (nn.ok) load_item(nn);
             tc_fence_after();
@@ -488,6 +528,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             bulk_store(p.rec + (size_t)cur.rec * R::BYTES + R::Z, x.A1, (uint32_t)(R::BYTES - R::Z));
             bulk_commit();
             stored = true;
+            unpublished = true;
+            stored_rec = cur.rec;
         }
         KDA_PHASE(3);
         if (!nxt.ok) break;
@@ -503,7 +545,10 @@ finish:
         if (pend & 1u) (void)mbar_wait(mb_tma, (uint32_t)tpar, &never, p.timeout_cycles);
         if (pend & 2u) (void)mbar_wait(mb_mma, (uint32_t)(nmma & 1), &never, p.timeout_cycles);
     }
-    if (tid == kStoreIssuer && stored) bulk_wait_all();
+    if (tid == kStoreIssuer && stored) {
+        bulk_wait_all();
+        if (p.ready && unpublished && !*abort_flag) publish(p.ready + stored_rec);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -528,6 +573,7 @@ struct ScanParams {
     long long max_chunks;    // records available per head
     long long tokens;
     long long timeout_cycles;
+    const unsigned* ready;   // cooperative schedule: wait for ready[record] before loading it
 };
 
 // Shared memory of the scan kernel: two 72 KB slots, each holding one record
@@ -623,9 +669,8 @@ __device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost,
 // Z, PT, e^G_last and beta part after chunk c + 1's X MMA (tcgen05 MMAs of
 // one thread complete in issue order).
 template <typename TO, int DK>
-__global__ void __launch_bounds__(NT, 1)
-chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
-                  const ScanParams p)
+__device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensorMap& tmo, const ScanParams& p,
+                                          int bid)
 {
     using PL = ScanPlan<DK>;
     using R = Rec<DK>;
@@ -648,9 +693,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant
     const int lt = tid & 127;
     const int wg = tid >> 7;
     const int nslice = p.DV / NV;
-    const int slice = blockIdx.x % nslice;
-    const int h = (blockIdx.x / nslice) % p.H;
-    const int rank = blockIdx.x / (nslice * p.H);
+    const int slice = bid % nslice;
+    const int h = (bid / nslice) % p.H;
+    const int rank = bid / (nslice * p.H);
     const int H = p.H, DV = p.DV;
     int n, tok0, len;
     long long j0;
@@ -714,6 +759,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant
     auto rec_of = [&](int cc) { return p.rec + ((size_t)(j0 + cc) * H + h) * R::BYTES; };
     auto issue_a = [&](int cc) {
         unsigned char* slot = sm + (cc & 1) * PL::SLOT;
+        if (p.ready && !wait_ready(p.ready + (size_t)(j0 + cc) * H + h, abort_flag, p.timeout_cycles)) return;
         mbar_expect_tx(mb_a + (cc & 1), kBytesA);
         bulk_load(slot, rec_of(cc), R::Z, mb_a + (cc & 1));
         tma_load_3d(slot + PL::VOFF, &tmv, mb_a + (cc & 1), col0, h, tok0 + cc * C);
@@ -914,6 +960,35 @@ finish:
 }
 #undef KDA_WAIT_OR_EXIT
 
+template <int DK>
+__global__ void __launch_bounds__(NT, 1)
+chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmg, const PrepParams p)
+{
+    prep_body<DK>(tmq, tmk, tmg, p, blockIdx.x, gridDim.x);
+}
+
+template <typename TO, int DK>
+__global__ void __launch_bounds__(NT, 1)
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                  const ScanParams p)
+{
+    scan_body<TO, DK>(tmv, tmo, p, blockIdx.x);
+}
+
+// Cooperative schedule: CTAs [0, n_scan) scan, the others prep; the scan
+// waits on the records' ready flags, the prep never waits on the scan, and a
+// cooperative launch keeps every CTA resident, so the hand-off cannot stall.
+template <typename TO, int DK>
+__global__ void __launch_bounds__(NT, 1)
+chunk_coop_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmg, const __grid_constant__ CUtensorMap tmv,
+                  const __grid_constant__ CUtensorMap tmo, const PrepParams pp, const ScanParams sp, int n_scan)
+{
+    if ((int)blockIdx.x < n_scan) scan_body<TO, DK>(tmv, tmo, sp, blockIdx.x);
+    else prep_body<DK>(tmq, tmk, tmg, pp, blockIdx.x - n_scan, gridDim.x - n_scan);
+}
+
 // ============================================================== host side
 
 // First chunk of every packed sequence: choff[i] = sum_{j<i} ceil(len_j / 64),
@@ -1014,7 +1089,14 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     const long long max_chunks = cu ? tokens / C + nseq : (long long)nseq * nch;
     const long long scan_ctas = (long long)nseq * H * (dv / NV);
     if (scan_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    const int nb = cu ? 1 : chunk_blocks(nch, scan_ctas, nsm);
+    // schedule: one cooperative launch (prep CTAs publish records, scan CTAs
+    // consume them) when the scan grid leaves at least 32 SMs; otherwise
+    // blocks of chunks on two streams, or prep then scan.  KDA_CHUNK_SCHEDULE
+    // (coop | streams) and KDA_SCAN_BLOCKS select explicitly.
+    const char* sched_env = getenv("KDA_CHUNK_SCHEDULE");
+    const bool coop = !cu && scan_ctas > 0 && scan_ctas + 32 <= nsm && !getenv("KDA_SCAN_BLOCKS") &&
+                      !(sched_env && strcmp(sched_env, "coop") != 0);
+    const int nb = (cu || coop) ? 1 : chunk_blocks(nch, scan_ctas, nsm);
     cudaStream_t side = nb > 1 ? side_stream() : nullptr;
 
     CUtensorMap tq, tk, tg;
@@ -1048,7 +1130,9 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     const int cb = cu ? 0 : (nch + nblocks - 1) / nblocks;     // chunks per block (dense)
     const size_t off_bytes = (((size_t)nseq + 1) * 4 + 1023) & ~(size_t)1023;
     const size_t state_bytes = (nblocks > 1 && !sT) ? (size_t)nseq * H * DK * dv * 4 : 0;
-    const size_t rec_off = off_bytes + ((state_bytes + 1023) & ~(size_t)1023);
+    const size_t flag_off = off_bytes + ((state_bytes + 1023) & ~(size_t)1023);
+    const size_t flag_bytes = coop ? (((size_t)max_chunks * H * 4 + 1023) & ~(size_t)1023) : 0;
+    const size_t rec_off = flag_off + flag_bytes;
     const size_t bytes = rec_off + (size_t)max_chunks * H * R::BYTES;
 
     retain_pool_memory();
@@ -1064,7 +1148,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
 
     if (cu) chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu, nseq, choff);
 
-    PrepParams pp;
+    PrepParams pp{};
     pp.beta = beta;
     pp.cu = cu;
     pp.choff = choff;
@@ -1077,7 +1161,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     pp.rc0 = 0;
     pp.tokens = tokens;
     pp.timeout_cycles = timeout_cycles;
-    ScanParams sp;
+    ScanParams sp{};
     sp.v = static_cast<const __nv_bfloat16*>(v);
     sp.o = o;
     sp.cu = cu;
@@ -1119,8 +1203,43 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         return cudaGetLastError();
     };
 
-    if (nblocks == 1) {
-        err = launch_prep(0, stream, nsm);
+    bool done = false;
+    if (coop) {
+        unsigned* flags = reinterpret_cast<unsigned*>(ws + flag_off);
+        err = cudaMemsetAsync(flags, 0, flag_bytes, stream);
+        auto ck = chunk_coop_kernel<TO, DK>;
+        const int smem = std::max(PrepPlan::BYTES, ScanPlan<DK>::BYTES);
+        if (err == cudaSuccess) err = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (err == cudaSuccess) {
+            pp.ready = flags;
+            pp.c_begin = 0;
+            pp.cbs = nch;
+            pp.nitems = max_chunks * H;
+            sp.ready = flags;
+            sp.c_begin = 0;
+            sp.c_end = 0x7fffffff;
+            sp.s_in = s0;
+            sp.s_out = sT;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)nsm);
+            cfg.blockDim = dim3(NT);
+            cfg.dynamicSmemBytes = (size_t)smem;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeCooperative;
+            attr[0].val.cooperative = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            const int n_scan = (int)scan_ctas;
+            if (cudaLaunchKernelEx(&cfg, ck, tq, tk, tg, tv, to, pp, sp, n_scan) == cudaSuccess) done = true;
+            else (void)cudaGetLastError();   // not co-residable here: fall back to prep then scan
+            pp.ready = nullptr;
+            sp.ready = nullptr;
+        }
+    }
+    if (done) {
+    } else if (nblocks == 1) {
+        if (err == cudaSuccess) err = launch_prep(0, stream, nsm);
         if (err == cudaSuccess) err = launch_scan(0);
     } else {
         // fork: the side stream starts after everything queued on `stream`;

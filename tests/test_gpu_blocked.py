@@ -88,3 +88,26 @@ def test_blocked_bf16_output():
     o4, s4 = _call(g, 4, o_dtype=torch.bfloat16)
     assert torch.equal(o4, o1)
     assert torch.equal(s4, s1)
+
+
+def _call_coop(g, **kw):
+    """Default schedule: one cooperative launch (prep CTAs publish records,
+    scan CTAs consume them) whenever the scan grid leaves 32 SMs free."""
+    assert "KDA_SCAN_BLOCKS" not in os.environ
+    out = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"], **kw)
+    torch.cuda.synchronize()
+    kda.kda_check()
+    return out
+
+
+@pytest.mark.parametrize("B,T,H,d", [(2, 33 * 64 + 37, 3, 128), (1, 64, 1, 128), (3, 20 * 64 + 1, 5, 64),
+                                     (2, 4096, 16, 128)])
+def test_cooperative_schedule_bit_identical(B, T, H, d):
+    x, g = _inputs(B, T, H, d, seed=70 + H)
+    o1, s1 = _call(g, 1)
+    o2, s2 = _call_coop(g)
+    assert torch.equal(o2, o1)
+    assert torch.equal(s2, s1)
+    o3, s3 = _call_coop(g, output_final_state=False, o_dtype=torch.bfloat16)
+    o4, _ = _call(g, 1, output_final_state=False, o_dtype=torch.bfloat16)
+    assert s3 is None and torch.equal(o3, o4)
