@@ -412,8 +412,8 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     tc_fence_before();
     __syncthreads();
     nxt = resolve(p, item + nblk);
+    if (tid == 32 && nxt.ok) load_item(nxt);
     if (tid == 0) {
-        if (nxt.ok) load_item(nxt);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < DK / 8; ++kk)
@@ -474,8 +474,8 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
 
         // ---- MMA round: Z'(k) = B1^T T, PT(k) = P T; [P ; A~](k + 1) = A1 B1^T
         const Item nn = nxt.ok ? resolve(p, nitem + nblk) : Item{0, 0, 0, 0, false};
+        if (tid == 32 && nn.ok) load_item(nn);
         if (tid == 0) {
-            if (nn.ok) load_item(nn);
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk)
