@@ -451,14 +451,19 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
                 for (int u = 0; u < 32; ++u) tv[u] = (c0 + u >= j) ? As[j * LDA + c0 + u] : 0.f;
                 st_row_swf_raw<8>(Top, j, c0, C, tv);
             }
-        } else if (nxt.ok) {
-            const int t = tid - 128;
-            const float beta_v = beta_of(nxt, t);
-            if (tid == kStoreIssuer && stored) bulk_wait_read();   // A1 is about to be rewritten
-            const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
-            if (!bar_or(3, 384, !ok)) {
-                cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v);
-                build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384, 0, C);
+        } else {
+            // A1 is rewritten in this iteration (operands of item k + 1, or the
+            // record tail of item k when it is the last): the previous tail's
+            // bulk store must have finished reading it
+            if (tid == kStoreIssuer && stored) bulk_wait_read();
+            if (nxt.ok) {
+                const int t = tid - 128;
+                const float beta_v = beta_of(nxt, t);
+                const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
+                if (!bar_or(3, 384, !ok)) {
+                    cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v);
+                    build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384, 0, C);
+                }
             }
         }
         fence_proxy_async();
