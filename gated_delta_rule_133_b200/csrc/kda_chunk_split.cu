@@ -161,28 +161,37 @@ __device__ __forceinline__ Item resolve(const PrepParams& p, long long item)
     return it;
 }
 
+constexpr int LDT = 68;     // row stride (floats) of the UT matrix: 16-byte rows, conflict-free quads
+
 // Shared memory of the prep kernel (byte offsets from a 1024-aligned base).
-//   A1: [q E; k E] (tf32, [128][d_k]) of the item being built; once MMA PA
-//       has read it, the staging tile of the previous item's record tail
-//       (Z, PT, e^G_last, beta), which one bulk store copies out.
+//   A1: [q E; k E] (tf32, [128][d_k]) of the item being built.
 //   B1: k / E (tf32, [64][d_k]).
 //   STG: TMA staging of q, k (bf16) and log alpha (fp32 -> G in place).
-//   TOP: T^T [64][64] (tf32 B operand of MMA Z', PT); AS/XS: UT scratch.
+//   TOP: T^T [64][64] (tf32 B operand of MMA Z', PT); before T^T is written,
+//        the UT product scratch XS.
+//   AS: A, then T in place (fp32, row-major, row stride LDT).
 //   VEC: per item (double-buffered): G_m, e^G_m, e^(G_last - G_m), e^G_last,
 //        partial sums, beta.
+//   TST: staging of the previous item's record tail (Z, PT, e^G_last, beta),
+//        which one bulk store copies out.
 struct PrepPlan {
     static constexpr int A1 = 0;
     static constexpr int B1 = 65536;
     static constexpr int STG = 98304;
     static constexpr int TOP = 163840;
+    static constexpr int XS = TOP;
     static constexpr int AS = TOP + 16384;
-    static constexpr int XS = AS + C * LDA * 4;
-    static constexpr int VEC = XS + 32 * 33 * 4;
-    static constexpr int VECN = 8 * 128 + 64;
-    static constexpr int BAR = VEC + 2 * VECN * 4;
+    static constexpr int VEC = AS + C * LDT * 4;
+    static constexpr int VECN = 7 * 128 + 64;
+    static constexpr int TST = VEC + 2 * VECN * 4;
+    static constexpr int TST_BYTES = 25344;
+    static constexpr int BAR = TST + TST_BYTES;
     static constexpr int END = BAR + 128;
     static constexpr int BYTES = END + 1024;
 };
+static_assert(PrepPlan::BYTES <= 232448, "prep shared memory exceeds the per-CTA limit");
+static_assert(Rec<128>::BYTES - Rec<128>::Z <= PrepPlan::TST_BYTES, "record tail staging too small");
+static_assert(32 * 36 * 4 <= 16384, "UT scratch must fit the T^T tile");
 
 template <int DK>
 struct PrepCtx {
@@ -205,7 +214,7 @@ struct Vec {
 __device__ __forceinline__ Vec vec_at(unsigned char* base, int buf)
 {
     float* f = reinterpret_cast<float*>(base) + buf * PrepPlan::VECN;
-    return Vec{f, f + 128, f + 256, f + 384, f + 512, f + 1024};
+    return Vec{f, f + 128, f + 256, f + 384, f + 512, f + 896};
 }
 
 // Gate cumsum of the staged chunk in place, by 384 threads (t = 0..383:
@@ -284,6 +293,121 @@ __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& 
     }
 }
 
+// d += s * b for two float4 accumulators, as four packed fp32x2 FMAs (each
+// lane rounds exactly as fmaf does).
+__device__ __forceinline__ void fma_s8(float4& d0, float4& d1, float s, const float4& b0, const float4& b1)
+{
+    asm("{\n\t.reg .b64 ss, bb, dd;\n\t"
+        "mov.b64 ss, {%8, %8};\n\t"
+        "mov.b64 bb, {%9, %10};\n\tmov.b64 dd, {%0, %1};\n\tfma.rn.f32x2 dd, ss, bb, dd;\n\tmov.b64 {%0, %1}, dd;\n\t"
+        "mov.b64 bb, {%11, %12};\n\tmov.b64 dd, {%2, %3};\n\tfma.rn.f32x2 dd, ss, bb, dd;\n\tmov.b64 {%2, %3}, dd;\n\t"
+        "mov.b64 bb, {%13, %14};\n\tmov.b64 dd, {%4, %5};\n\tfma.rn.f32x2 dd, ss, bb, dd;\n\tmov.b64 {%4, %5}, dd;\n\t"
+        "mov.b64 bb, {%15, %16};\n\tmov.b64 dd, {%6, %7};\n\tfma.rn.f32x2 dd, ss, bb, dd;\n\tmov.b64 {%6, %7}, dd;\n\t}"
+        : "+f"(d0.x), "+f"(d0.y), "+f"(d0.z), "+f"(d0.w), "+f"(d1.x), "+f"(d1.y), "+f"(d1.z), "+f"(d1.w)
+        : "f"(s), "f"(b0.x), "f"(b0.y), "f"(b0.z), "f"(b0.w), "f"(b1.x), "f"(b1.y), "f"(b1.z), "f"(b1.w));
+}
+__device__ __forceinline__ void fma_s4(float4& d, float s, const float4& b)
+{
+    asm("{\n\t.reg .b64 ss, bb, dd;\n\t"
+        "mov.b64 ss, {%4, %4};\n\t"
+        "mov.b64 bb, {%5, %6};\n\tmov.b64 dd, {%0, %1};\n\tfma.rn.f32x2 dd, ss, bb, dd;\n\tmov.b64 {%0, %1}, dd;\n\t"
+        "mov.b64 bb, {%7, %8};\n\tmov.b64 dd, {%2, %3};\n\tfma.rn.f32x2 dd, ss, bb, dd;\n\tmov.b64 {%2, %3}, dd;\n\t}"
+        : "+f"(d.x), "+f"(d.y), "+f"(d.z), "+f"(d.w)
+        : "f"(s), "f"(b.x), "f"(b.y), "f"(b.z), "f"(b.w));
+}
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 neg4(const float4& a) { return make_float4(-a.x, -a.y, -a.z, -a.w); }
+__device__ __forceinline__ float f4at(const float4& a, int u) { return u == 0 ? a.x : u == 1 ? a.y : u == 2 ? a.z : a.w; }
+
+// UT transform T = (I + A)^-1 of the strictly lower 64 x 64 A, in place, by
+// the first 128 threads (named barrier 1).  On entry As[r * LDT + s] holds
+// A[r][s] (zero for s >= r); on return it holds T[r][s] (T[r][r] = 1, zero for
+// s > r).  Diagonal 16 x 16 blocks by forward substitution (one lane per
+// column), then T10 = -T11 A10 T00 and T32 = -T33 A32 T22, then the lower-left
+// 32 x 32 block -T_BB A_BA T_AA.  Every sum runs in ascending index order
+// (terms that the triangular factors make zero are skipped where a whole warp
+// can skip them); X is the product scratch.
+__device__ __forceinline__ void ut_rows(float* As, float* X)
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid < 64) {
+        const int b0 = 16 * (tid >> 4), j = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = 0.f;
+        x[0] = j == 0 ? 1.f : 0.f;
+#pragma unroll
+        for (int r = 1; r < 16; ++r) {
+            float acc = (r == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int q = 0; 4 * q < r; ++q) {   // A[r][s] = 0 and x[s] = 0 for s >= r
+                const float4 a = ld4(As + (b0 + r) * LDT + b0 + 4 * q);
+                acc = fmaf(-a.x, x[4 * q], acc);
+                acc = fmaf(-a.y, x[4 * q + 1], acc);
+                acc = fmaf(-a.z, x[4 * q + 2], acc);
+                acc = fmaf(-a.w, x[4 * q + 3], acc);
+            }
+            x[r] = acc;
+        }
+        __syncwarp();   // every lane has read its A block before T overwrites it
+#pragma unroll
+        for (int r = 0; r < 16; ++r)
+            if (r >= j) As[(b0 + r) * LDT + b0 + j] = x[r];
+    }
+    bar_sync(1, 128);
+    {   // T10 (warps 0, 1) and T32 (warps 2, 3): lane -> row i, columns j0 .. j0 + 3
+        const int pr = warp >> 1, half = warp & 1;
+        const int rb = 16 + 32 * pr, cb = 32 * pr;
+        const int i = lane & 15, j0 = 8 * half + 4 * (lane >> 4);
+        float* Xp = X + pr * 16 * 20;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 2 * half; q < 4; ++q) {   // T_cc[t][j] = 0 for t < j
+            const float4 a = ld4(As + (rb + i) * LDT + cb + 4 * q);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) fma_s4(acc, f4at(a, u), ld4(As + (cb + 4 * q + u) * LDT + cb + j0));
+        }
+        *reinterpret_cast<float4*>(Xp + i * 20 + j0) = acc;
+        bar_sync(1, 128);
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 t = ld4(As + (rb + i) * LDT + rb + 4 * q);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) fma_s4(acc, f4at(t, u), ld4(Xp + (4 * q + u) * 20 + j0));
+        }
+        *reinterpret_cast<float4*>(As + (rb + i) * LDT + cb + j0) = neg4(acc);
+    }
+    bar_sync(1, 128);
+    {   // lower-left 32 x 32: lane -> row i (0..31), warp -> columns c0 .. c0 + 7
+        const int i = lane, c0 = 8 * warp;
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+        for (int q = 2 * warp; q < 8; ++q) {   // T_AA[t][c] = 0 for t < c0 <= c
+            const float4 a = ld4(As + (32 + i) * LDT + 4 * q);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float* tr = As + (4 * q + u) * LDT + c0;
+                fma_s8(a0, a1, f4at(a, u), ld4(tr), ld4(tr + 4));
+            }
+        }
+        *reinterpret_cast<float4*>(X + i * 36 + c0) = a0;
+        *reinterpret_cast<float4*>(X + i * 36 + c0 + 4) = a1;
+        bar_sync(1, 128);
+        a0 = make_float4(0.f, 0.f, 0.f, 0.f);
+        a1 = a0;
+#pragma unroll 2
+        for (int q = 0; q < 8; ++q) {
+            const float4 t = ld4(As + (32 + i) * LDT + 32 + 4 * q);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float* xr = X + (4 * q + u) * 36 + c0;
+                fma_s8(a0, a1, f4at(t, u), ld4(xr), ld4(xr + 4));
+            }
+        }
+        *reinterpret_cast<float4*>(As + (32 + i) * LDT + c0) = neg4(a0);
+        *reinterpret_cast<float4*>(As + (32 + i) * LDT + c0 + 4) = neg4(a1);
+    }
+}
+
 // One persistent CTA per SM walks items blockIdx.x, + gridDim.x, ...  The
 // UT transform of item k (warpgroup 0) overlaps the gate cumsum and operand
 // build of item k + 1 (warpgroups 1-3); one MMA round then forms Z', PT of
@@ -292,7 +416,7 @@ __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& 
 //   prologue: load, cumsum, build, MMA PA of item 0; P/A split of item 0
 //   loop k:   WG0: UT(k), T^T tile      | WG1-3: cumsum + build of item k + 1
 //             MMA Z'(k), PT(k), PA(k + 1)
-//             record tail of item k (staged in A1, one bulk store); P/A split of k + 1
+//             record tail of item k (staged in TST, one bulk store); P/A split of k + 1
 //
 // TMEM: [P ; A~] double-buffered (0, 64), B1^T 128, Z' 192, PT 256.
 template <int DK>
@@ -380,8 +504,13 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         } else {
             const int r = lt - C;
             const float b = v.beta[r];
+            float a[16];
 #pragma unroll
-            for (int s2 = 0; s2 < 16; ++s2) As[r * LDA + 16 * wg + s2] = (16 * wg + s2 < r) ? b * pa[s2] : 0.f;
+            for (int s2 = 0; s2 < 16; ++s2) a[s2] = (16 * wg + s2 < r) ? b * pa[s2] : 0.f;
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4)
+                *reinterpret_cast<float4*>(As + r * LDT + 16 * wg + 4 * s4) =
+                    make_float4(a[4 * s4], a[4 * s4 + 1], a[4 * s4 + 2], a[4 * s4 + 3]);
         }
         float kb[16];
 #pragma unroll
@@ -442,20 +571,16 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
 
         // ---- UT transform of item k (WG0) | cumsum + operands of item k + 1 (WG1-3)
         if (wg == 0) {
-            ut_transform(As, Xs);
+            ut_rows(As, Xs);
             bar_sync(1, 128);
-            {
+            {   // T^T row j = column j of T (zero above the diagonal)
                 const int j = tid >> 1, c0 = (tid & 1) * 32;
                 float tv[32];
 #pragma unroll
-                for (int u = 0; u < 32; ++u) tv[u] = (c0 + u >= j) ? As[j * LDA + c0 + u] : 0.f;
+                for (int u = 0; u < 32; ++u) tv[u] = As[(c0 + u) * LDT + j];
                 st_row_swf_raw<8>(Top, j, c0, C, tv);
             }
         } else {
-            // A1 is rewritten in this iteration (operands of item k + 1, or the
-            // record tail of item k when it is the last): the previous tail's
-            // bulk store must have finished reading it
-            if (tid == kStoreIssuer && stored) bulk_wait_read();
             if (nxt.ok) {
                 const int t = tid - 128;
                 const float beta_v = beta_of(nxt, t);
@@ -501,14 +626,17 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
             ++nload;
         }
         pend |= 2u;
+        // the staging area is rewritten below: the previous tail's bulk store
+        // (issued an iteration ago) must have read it
+        if (tid == kStoreIssuer && stored) bulk_wait_read();
         KDA_WAIT_OR_EXIT(mb_mma, 2u, nmma & 1);
         ++nmma;
         tc_fence_after();
         KDA_PHASE(2);
 
-        // ---- record tail of item k, staged in A1: Z = diag(e^(G_last - G_m)) Z', PT, e^G_last, beta
+        // ---- record tail of item k, staged in TST: Z = diag(e^(G_last - G_m)) Z', PT, e^G_last, beta
         {
-            unsigned char* stg = x.A1;
+            unsigned char* stg = sm + PL::TST;
             float z[16];
             tmem_ld16(t_Z + lane_off + q_off, z);
             float pt[16];
@@ -530,7 +658,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         tc_fence_before();
         __syncthreads();
         if (tid == kStoreIssuer) {
-            bulk_store(p.rec + (size_t)cur.rec * R::BYTES + R::Z, x.A1, (uint32_t)(R::BYTES - R::Z));
+            bulk_store(p.rec + (size_t)cur.rec * R::BYTES + R::Z, sm + PL::TST, (uint32_t)(R::BYTES - R::Z));
             bulk_commit();
             stored = true;
             unpublished = true;
