@@ -22,7 +22,9 @@
 // Precision.  The intra-chunk products P and A use the middle row m of the
 // chunk as reference, E = exp(G - G_m) and 1/E (each bounded by 32 tokens of
 // decay), and run as kind::tf32 MMAs with operands rounded to nearest; T is
-// fp32.  The record's operands are fp16, which has the tf32 mantissa: every
+// fp32.  Z and PT are kind::f16 MMAs: T, P and k e^(G_last - G) are rounded to
+// fp16, which has the tf32 mantissa and holds them (every factor is at most 1).
+// The record's operands are fp16 too: every
 // factor e^G, e^(G_last - G) is at most 1, so Qh, Kh, Z and PT stay in range,
 // and S and Y are rounded to fp16 as the scan's MMA operands (|S|, |Y| must
 // stay below 65504).  The scan accumulates in fp32 in TMEM.
@@ -167,7 +169,7 @@ constexpr int LDT = 68;     // row stride (floats) of the UT matrix: 16-byte row
 //   A1: [q E; k E] (tf32, [128][d_k]) of the item being built.
 //   B1: k / E (tf32, [64][d_k]).
 //   STG: TMA staging of q, k (bf16) and log alpha (fp32 -> G in place).
-//   TOP: T^T [64][64] (tf32 B operand of MMA Z', PT); before T^T is written,
+//   TOP: T^T [64][64] (fp16 B operand of MMAs Z, PT); before T^T is written,
 //        the UT product scratch XS.
 //   AS: A, then T in place (fp32, row-major, row stride LDT).
 //   VEC: per item (double-buffered): G_m, e^G_m, e^(G_last - G_m), e^G_last,
@@ -410,15 +412,17 @@ __device__ __forceinline__ void ut_rows(float* As, float* X)
 
 // One persistent CTA per SM walks items blockIdx.x, + gridDim.x, ...  The
 // UT transform of item k (warpgroup 0) overlaps the gate cumsum and operand
-// build of item k + 1 (warpgroups 1-3); one MMA round then forms Z', PT of
+// build of item k + 1 (warpgroups 1-3); one MMA round then forms Z, PT of
 // item k and [P ; A~] of item k + 1.
 //
 //   prologue: load, cumsum, build, MMA PA of item 0; P/A split of item 0
 //   loop k:   WG0: UT(k), T^T tile      | WG1-3: cumsum + build of item k + 1
-//             MMA Z'(k), PT(k), PA(k + 1)
+//             MMA Z(k), PT(k) (kind::f16), PA(k + 1) (kind::tf32)
 //             record tail of item k (staged in TST, one bulk store); P/A split of k + 1
 //
-// TMEM: [P ; A~] double-buffered (0, 64), B1^T 128, Z' 192, PT 256.
+// TMEM: [P ; A~] double-buffered (0, 64); the fp16 A operands of Z and PT,
+// k e^(G_last - G) transposed (128) and masked P (160), two per 32-bit column;
+// Z 192, PT 256.
 template <int DK>
 __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmg,
                                           const PrepParams& p, int bid, int nblk)
@@ -469,7 +473,8 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_off = ((uint32_t)(warp & 3) * 32) << 16;
     const uint32_t q_off = (uint32_t)wg * 16;
-    const uint32_t t_KB = tmem + 128, t_Z = tmem + 192, t_PT = tmem + 256;
+    const uint32_t t_K16 = tmem + 128, t_P16 = tmem + 160, t_Z = tmem + 192, t_PT = tmem + 256;
+    constexpr uint32_t kH64 = idesc_f16(128, 64);
 
     constexpr uint32_t kStageBytes = (uint32_t)C * DK * (2 + 2 + 4);
     constexpr uint32_t kI64 = idesc_tf32(128, 64, 0, 0);
@@ -491,16 +496,19 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     auto beta_of = [&](const Item& it, int t) {
         return (it.ok && t < C && t < it.L) ? p.beta[(size_t)(it.tok0 + t) * H + it.h] : 0.f;
     };
-    // P masked in place in TMEM (lanes 0..63, lower incl.); A = beta A~ (lanes
-    // 64..127, strictly lower) to the UT scratch; B1^T into TMEM
+    // P masked (lanes 0..63, lower incl.) into the fp16 operand of PT; A = beta
+    // A~ (lanes 64..127, strictly lower) to the UT scratch; (k / E)^T
+    // e^(G_last - G_m) = (k e^(G_last - G))^T into the fp16 operand of Z
     auto split_pa = [&](uint32_t t_PA, const Vec& v) {
         float pa[16];
         tmem_ld16(t_PA + lane_off + q_off, pa);
         tmem_wait_ld();
-        if (lt < C) {
+        if (lt < C) {   // P, lower incl., packed fp16 (warps of lanes 0..63)
+            uint32_t p16[8];
 #pragma unroll
-            for (int s2 = 0; s2 < 16; ++s2) pa[s2] = (16 * wg + s2 <= lt) ? pa[s2] : 0.f;
-            tmem_st16(t_PA + lane_off + q_off, pa);
+            for (int s2 = 0; s2 < 8; ++s2)
+                p16[s2] = pack_f16((16 * wg + 2 * s2 <= lt) ? pa[2 * s2] : 0.f, (16 * wg + 2 * s2 + 1 <= lt) ? pa[2 * s2 + 1] : 0.f);
+            tmem_st8(t_P16 + lane_off + wg * 8, p16);
         } else {
             const int r = lt - C;
             const float b = v.beta[r];
@@ -512,10 +520,12 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
                 *reinterpret_cast<float4*>(As + r * LDT + 16 * wg + 4 * s4) =
                     make_float4(a[4 * s4], a[4 * s4 + 1], a[4 * s4 + 2], a[4 * s4 + 3]);
         }
-        float kb[16];
+        const float gl = lt < DK ? v.glm[lt] : 0.f;   // k e^(G_last - G) = (k / E) e^(G_last - G_m)
+        uint32_t kb[8];
 #pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2) kb[s2] = lt < DK ? swf(x.B1, 16 * wg + s2, lt, 64) : 0.f;
-        tmem_st16(t_KB + lane_off + q_off, kb);
+        for (int s2 = 0; s2 < 8; ++s2)
+            kb[s2] = lt < DK ? pack_f16(swf(x.B1, 16 * wg + 2 * s2, lt, 64) * gl, swf(x.B1, 16 * wg + 2 * s2 + 1, lt, 64) * gl) : 0u;
+        tmem_st8(t_K16 + lane_off + wg * 8, kb);
         tmem_wait_st();
     };
 
@@ -565,7 +575,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     for (k = 0;; ++k) {
         const int vb = k & 1, nb = vb ^ 1;
         const Vec vcur = vec_at(vbase, vb), vnxt = vec_at(vbase, nb);
-        const uint32_t t_PAc = tmem + 64 * vb, t_PAn = tmem + 64 * nb;
+        const uint32_t t_PAn = tmem + 64 * nb;
         const long long nitem = item + nblk;
         KDA_PHASE(0);
 
@@ -578,7 +588,8 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
                 float tv[32];
 #pragma unroll
                 for (int u = 0; u < 32; ++u) tv[u] = As[(c0 + u) * LDT + j];
-                st_row_swf_raw<8>(Top, j, c0, C, tv);
+                st_row_h16(Top, j, c0, C, tv);
+                st_row_h16(Top, j, c0 + 16, C, tv + 16);
             }
         } else {
             if (nxt.ok) {
@@ -602,17 +613,17 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         }
         KDA_PHASE(1);
 
-        // ---- MMA round: Z'(k) = B1^T T, PT(k) = P T; [P ; A~](k + 1) = A1 B1^T
+        // ---- MMA round: Z(k) = (k e^(G_last - G))^T T, PT(k) = P T; [P ; A~](k + 1) = A1 B1^T
         const Item nn = nxt.ok ? resolve(p, nitem + nblk) : Item{0, 0, 0, 0, false};
         if (tid == 32 && nn.ok) load_item(nn);
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)
-                umma_tf32_ts(t_Z, t_KB + 8 * kk, kdesc(Top, kk, kR64), kI64, kk > 0);
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_f16_ts(t_Z, t_K16 + 8 * kk, kdesc(Top, kk, kR64), kH64, kk > 0);
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)
-                umma_tf32_ts(t_PT, t_PAc + 8 * kk, kdesc(Top, kk, kR64), kI64, kk > 0);
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_f16_ts(t_PT, t_P16 + 8 * kk, kdesc(Top, kk, kR64), kH64, kk > 0);
             if (nxt.ok) {
 #pragma unroll
                 for (int kk = 0; kk < DK / 8; ++kk)
@@ -634,7 +645,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         tc_fence_after();
         KDA_PHASE(2);
 
-        // ---- record tail of item k, staged in TST: Z = diag(e^(G_last - G_m)) Z', PT, e^G_last, beta
+        // ---- record tail of item k, staged in TST: Z, PT, e^G_last, beta
         {
             unsigned char* stg = sm + PL::TST;
             float z[16];
@@ -642,12 +653,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
             float pt[16];
             tmem_ld16(t_PT + lane_off + q_off, pt);
             tmem_wait_ld();
-            if (lt < DK) {
-                const float sc = vcur.glm[lt];
-#pragma unroll
-                for (int u = 0; u < 16; ++u) z[u] *= sc;
-                st_row_h16(stg, lt, 16 * wg, DK, z);
-            }
+            if (lt < DK) st_row_h16(stg, lt, 16 * wg, DK, z);
             if (lt < C) st_row_h16(stg + (R::PT - R::Z), lt, 16 * wg, C, pt);
             if (tid < DK) reinterpret_cast<float*>(stg + (R::EGL - R::Z))[tid] = vcur.egl[tid];
             else if (tid >= 256 && tid < 256 + C) reinterpret_cast<float*>(stg + (R::BETA - R::Z))[tid - 256] = vcur.beta[tid - 256];
