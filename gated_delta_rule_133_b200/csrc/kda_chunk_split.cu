@@ -140,8 +140,15 @@ __device__ __forceinline__ Item resolve(const PrepParams& p, long long item)
 {
     Item it{0, 0, 0, 0, false};
     if (item >= p.nitems) return it;
-    it.h = (int)(item % p.H);
-    const long long j = item / p.H;
+    long long j;
+    if (p.nitems <= 0xffffffffll) {   // 32-bit divisions (a fraction of the 64-bit routine's cost)
+        const uint32_t i32 = (uint32_t)item, q = i32 / (uint32_t)p.H;
+        it.h = (int)(i32 - q * (uint32_t)p.H);
+        j = q;
+    } else {
+        it.h = (int)(item % p.H);
+        j = item / p.H;
+    }
     it.rec = item;
     if (p.cu) {
         if (j >= p.choff[p.nseq]) return it;
@@ -154,7 +161,15 @@ __device__ __forceinline__ Item resolve(const PrepParams& p, long long item)
         it.tok0 = p.cu[lo] + (int)(j - p.choff[lo]) * C;
         it.L = min(C, p.cu[lo + 1] - it.tok0);
     } else {   // chunk outermost, then sequence: the scans of all sequences advance together
-        const int n = (int)(j % p.nseq), c = p.c_begin + (int)(j / p.nseq);
+        int n, c;
+        if (p.nitems <= 0xffffffffll) {
+            const uint32_t j32 = (uint32_t)j, jq = j32 / (uint32_t)p.nseq;
+            n = (int)(j32 - jq * (uint32_t)p.nseq);
+            c = p.c_begin + (int)jq;
+        } else {
+            n = (int)(j % p.nseq);
+            c = p.c_begin + (int)(j / p.nseq);
+        }
         it.tok0 = n * p.T + c * C;
         it.L = min(C, p.T - c * C);
         it.rec = ((long long)n * p.rs + c - p.rc0) * p.H + it.h;
@@ -614,8 +629,6 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         KDA_PHASE(1);
 
         // ---- MMA round: Z(k) = (k e^(G_last - G))^T T, PT(k) = P T; [P ; A~](k + 1) = A1 B1^T
-        const Item nn = nxt.ok ? resolve(p, nitem + nblk) : Item{0, 0, 0, 0, false};
-        if (tid == 32 && nn.ok) load_item(nn);
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -631,6 +644,8 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
             }
             umma_commit(mb_mma);
         }
+        const Item nn = nxt.ok ? resolve(p, nitem + nblk) : Item{0, 0, 0, 0, false};
+        if (tid == 32 && nn.ok) load_item(nn);
         if (nn.ok) {
             pend |= 1u;
             tpar = nload & 1;
