@@ -645,17 +645,19 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
             umma_commit(mb_mma);
         }
         const Item nn = nxt.ok ? resolve(p, nitem + nblk) : Item{0, 0, 0, 0, false};
+        pend |= 2u;
+        // the staging area is rewritten below: the previous tail's bulk store
+        // (issued an iteration ago) must have read it
+        if (tid == kStoreIssuer && stored) bulk_wait_read();
+        KDA_WAIT_OR_EXIT(mb_mma, 2u, nmma & 1);
+        // the next load lands in shared memory only now: a TMA copy arriving
+        // while the MMAs read their operands slows the round by ~30 %
         if (tid == 32 && nn.ok) load_item(nn);
         if (nn.ok) {
             pend |= 1u;
             tpar = nload & 1;
             ++nload;
         }
-        pend |= 2u;
-        // the staging area is rewritten below: the previous tail's bulk store
-        // (issued an iteration ago) must have read it
-        if (tid == kStoreIssuer && stored) bulk_wait_read();
-        KDA_WAIT_OR_EXIT(mb_mma, 2u, nmma & 1);
         ++nmma;
         tc_fence_after();
         KDA_PHASE(2);
