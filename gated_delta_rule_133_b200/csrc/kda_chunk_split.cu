@@ -184,8 +184,8 @@ constexpr int LDT = 68;     // row stride (floats) of the UT matrix: 16-byte row
 //   A1: [q E; k E] (tf32, [128][d_k]) of the item being built.
 //   B1: k / E (tf32, [64][d_k]).
 //   STG: TMA staging of q, k (bf16) and log alpha (fp32 -> G in place).
-//   TOP: T^T [64][64] (fp16 B operand of MMAs Z, PT); before T^T is written,
-//        the UT product scratch XS.
+//   TOP: T^T [64][64] (fp16 B operand of MMAs Z, PT; entries below its
+//        diagonal stay zero), then the UT product scratch XS.
 //   AS: A, then T in place (fp32, row-major, row stride LDT).
 //   VEC: per item (double-buffered): G_m, e^G_m, e^(G_last - G_m), e^G_last,
 //        partial sums, beta.
@@ -196,7 +196,7 @@ struct PrepPlan {
     static constexpr int B1 = 65536;
     static constexpr int STG = 98304;
     static constexpr int TOP = 163840;
-    static constexpr int XS = TOP;
+    static constexpr int XS = TOP + 8192;
     static constexpr int AS = TOP + 16384;
     static constexpr int VEC = AS + C * LDT * 4;
     static constexpr int VECN = 7 * 128 + 64;
@@ -208,7 +208,7 @@ struct PrepPlan {
 };
 static_assert(PrepPlan::BYTES <= 232448, "prep shared memory exceeds the per-CTA limit");
 static_assert(Rec<128>::BYTES - Rec<128>::Z <= PrepPlan::TST_BYTES, "record tail staging too small");
-static_assert(32 * 36 * 4 <= 16384, "UT scratch must fit the T^T tile");
+static_assert(32 * 36 * 4 <= 8192, "UT scratch must fit behind the T^T tile");
 
 template <int DK>
 struct PrepCtx {
@@ -336,15 +336,17 @@ __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast
 __device__ __forceinline__ float4 neg4(const float4& a) { return make_float4(-a.x, -a.y, -a.z, -a.w); }
 __device__ __forceinline__ float f4at(const float4& a, int u) { return u == 0 ? a.x : u == 1 ? a.y : u == 2 ? a.z : a.w; }
 
-// UT transform T = (I + A)^-1 of the strictly lower 64 x 64 A, in place, by
-// the first 128 threads (named barrier 1).  On entry As[r * LDT + s] holds
-// A[r][s] (zero for s >= r); on return it holds T[r][s] (T[r][r] = 1, zero for
-// s > r).  Diagonal 16 x 16 blocks by forward substitution (one lane per
+// UT transform T = (I + A)^-1 of the strictly lower 64 x 64 A, by the first
+// 128 threads (named barrier 1).  On entry As[r * LDT + s] holds A[r][s] (zero
+// for s >= r).  T^T goes to Top (fp16, K-major 128-byte swizzle: row j =
+// column j of T) as each block of T is final; the entries of Top below its
+// diagonal are never written (they hold zeros).  As keeps the blocks of T that
+// later steps read (T[r][r] = 1, zero above the diagonal).  Diagonal 16 x 16 blocks by forward substitution (one lane per
 // column), then T10 = -T11 A10 T00 and T32 = -T33 A32 T22, then the lower-left
 // 32 x 32 block -T_BB A_BA T_AA.  Every sum runs in ascending index order
 // (terms that the triangular factors make zero are skipped where a whole warp
 // can skip them); X is the product scratch.
-__device__ __forceinline__ void ut_rows(float* As, float* X)
+__device__ __forceinline__ void ut_rows(float* As, float* X, unsigned char* Top)
 {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid < 64) {
@@ -370,6 +372,7 @@ __device__ __forceinline__ void ut_rows(float* As, float* X)
 #pragma unroll
         for (int r = 0; r < 16; ++r)
             if (r >= j) As[(b0 + r) * LDT + b0 + j] = x[r];
+        st_row_h16(Top, b0 + j, b0, C, x);   // x[r] = 0 for r < j
     }
     bar_sync(1, 128);
     {   // T10 (warps 0, 1) and T32 (warps 2, 3): lane -> row i, columns j0 .. j0 + 3
@@ -392,7 +395,10 @@ __device__ __forceinline__ void ut_rows(float* As, float* X)
 #pragma unroll
             for (int u = 0; u < 4; ++u) fma_s4(acc, f4at(t, u), ld4(Xp + (4 * q + u) * 20 + j0));
         }
-        *reinterpret_cast<float4*>(As + (rb + i) * LDT + cb + j0) = neg4(acc);
+        const float4 t4 = neg4(acc);
+        *reinterpret_cast<float4*>(As + (rb + i) * LDT + cb + j0) = t4;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) *reinterpret_cast<__half*>(Top + swh_off(cb + j0 + u, rb + i, C)) = __float2half_rn(f4at(t4, u));
     }
     bar_sync(1, 128);
     {   // lower-left 32 x 32: lane -> row i (0..31), warp -> columns c0 .. c0 + 7
@@ -420,8 +426,11 @@ __device__ __forceinline__ void ut_rows(float* As, float* X)
                 fma_s8(a0, a1, f4at(t, u), ld4(xr), ld4(xr + 4));
             }
         }
-        *reinterpret_cast<float4*>(As + (32 + i) * LDT + c0) = neg4(a0);
-        *reinterpret_cast<float4*>(As + (32 + i) * LDT + c0 + 4) = neg4(a1);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            *reinterpret_cast<__half*>(Top + swh_off(c0 + u, 32 + i, C)) = __float2half_rn(-f4at(a0, u));
+            *reinterpret_cast<__half*>(Top + swh_off(c0 + 4 + u, 32 + i, C)) = __float2half_rn(-f4at(a1, u));
+        }
     }
 }
 
@@ -551,6 +560,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     if (!cur.ok) goto finish;
 
     // ---- prologue: item 0 by all threads
+    for (int i = tid; i < C * C * 2 / 16; i += NT) reinterpret_cast<uint4*>(Top)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (tid == 0) load_item(cur);
     ++nload;
     pend |= 1u;
@@ -596,16 +606,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
 
         // ---- UT transform of item k (WG0) | cumsum + operands of item k + 1 (WG1-3)
         if (wg == 0) {
-            ut_rows(As, Xs);
-            bar_sync(1, 128);
-            {   // T^T row j = column j of T (zero above the diagonal)
-                const int j = tid >> 1, c0 = (tid & 1) * 32;
-                float tv[32];
-#pragma unroll
-                for (int u = 0; u < 32; ++u) tv[u] = As[(c0 + u) * LDT + j];
-                st_row_h16(Top, j, c0, C, tv);
-                st_row_h16(Top, j, c0 + 16, C, tv + 16);
-            }
+            ut_rows(As, Xs, Top);
         } else {
             if (nxt.ok) {
                 const int t = tid - 128;
