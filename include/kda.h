@@ -37,7 +37,11 @@
  *    factored around the chunk's middle token; that requires the decay of any
  *    32 consecutive tokens of one channel to stay below about 80 nats
  *    (average alpha above ~0.08).  Stronger gates lose accuracy in the
- *    intra-chunk terms (results stay finite).
+ *    intra-chunk terms (results stay finite).  The tensor-core path rounds
+ *    its operands to fp16: entries of e^G q, e^G k, the state, beta (v - k S)
+ *    and of the intra-chunk inverse (I + A)^-1 must stay below 65504 in
+ *    magnitude.  With keys of norm at most 1 and beta <= 1 the inverse's
+ *    entries are at most 1 in magnitude.
  */
 #ifndef KDA_H
 #define KDA_H
