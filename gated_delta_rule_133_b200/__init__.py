@@ -10,6 +10,10 @@ the computation runs in the library's CUDA kernels.  There is no CPU path.
     o      = kda_recurrent_step(q, k, v, beta, log_alpha, state)   # state updated in place
 
 The output o is fp32 by default (``o_dtype=torch.bfloat16`` rounds it to bf16).
+Two variants of the layer are keyword flags of the three calls (the
+``KDA_MODE_*`` flags of the C ABI): ``head_gate=True`` takes one forget gate per
+(token, head) -- log_alpha without its d_k axis -- and ``erase=False`` drops the
+delta rule's erase term (S_t = Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T).
 """
 from __future__ import annotations
 
@@ -25,6 +29,10 @@ _DTYPES = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
 
 def _ptr(t):
     return None if t is None else t.data_ptr()
+
+
+def _mode(head_gate, erase):
+    return (_lib.KDA_MODE_HEAD_GATE if head_gate else 0) | (0 if erase else _lib.KDA_MODE_NO_ERASE)
 
 
 def _stream(stream):
@@ -45,15 +53,16 @@ def _check(t, name, shape, dtype, device):
 
 
 def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final_state=None,
-                  output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None):
+                  output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None,
+                  head_gate=False, erase=True):
     """Chunkwise forward over equal-length sequences.
 
     q, k [B, T, H, dk] and v [B, T, H, dv] (bf16 or fp32); beta [B, T, H] and
-    log_alpha [B, T, H, dk] fp32; initial_state [B, H, dk, dv] fp32 or None.
-    Returns (o [B, T, H, dv] in o_dtype (or o's dtype when o is given),
-    final_state [B, H, dk, dv] or None)."""
+    log_alpha [B, T, H, dk] fp32 ([B, T, H] with head_gate); initial_state
+    [B, H, dk, dv] fp32 or None.  Returns (o [B, T, H, dv] in o_dtype (or o's
+    dtype when o is given), final_state [B, H, dk, dv] or None)."""
     return _dense_fwd("kda_chunk_fwd", q, k, v, beta, log_alpha, initial_state, o, final_state,
-                      output_final_state, o_dtype, chunk, stream)
+                      output_final_state, o_dtype, chunk, stream, _mode(head_gate, erase))
 
 
 def kda_chunk_fwd_noalloc(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final_state=None,
@@ -66,7 +75,7 @@ def kda_chunk_fwd_noalloc(q, k, v, beta, log_alpha, initial_state=None, *, o=Non
 
 
 def _dense_fwd(symbol, q, k, v, beta, log_alpha, initial_state, o, final_state, output_final_state, o_dtype,
-               chunk, stream):
+               chunk, stream, mode=0):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev, dt = q.device, q.dtype
@@ -74,7 +83,8 @@ def _dense_fwd(symbol, q, k, v, beta, log_alpha, initial_state, o, final_state, 
         raise ValueError(f"unsupported dtype {dt}")
     for t, n, s, d in ((q, "q", (B, T, H, dk), dt), (k, "k", (B, T, H, dk), dt),
                        (v, "v", (B, T, H, dv), dt), (beta, "beta", (B, T, H), torch.float32),
-                       (log_alpha, "log_alpha", (B, T, H, dk), torch.float32)):
+                       (log_alpha, "log_alpha", (B, T, H) if mode & _lib.KDA_MODE_HEAD_GATE else (B, T, H, dk),
+                        torch.float32)):
         _check(t, n, s, d, dev)
     if initial_state is not None:
         _check(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
@@ -87,18 +97,22 @@ def _dense_fwd(symbol, q, k, v, beta, log_alpha, initial_state, o, final_state, 
         final_state = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
     if final_state is not None:
         _check(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
+    extra = ()
+    if mode:
+        symbol, extra = symbol + "_mode", (mode,)
     _lib.call(symbol, _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
               _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk,
-              _DTYPES[dt], _DTYPES[o.dtype], _stream(stream))
+              _DTYPES[dt], _DTYPES[o.dtype], *extra, _stream(stream))
     return o, final_state
 
 
 def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, o=None,
                    final_state=None, output_final_state=True, o_dtype=torch.float32, chunk=64,
-                   stream=None):
+                   stream=None, head_gate=False, erase=True):
     """Chunkwise forward over N packed variable-length sequences.
 
-    q, k [T, H, dk], v [T, H, dv]; beta [T, H]; log_alpha [T, H, dk];
+    q, k [T, H, dk], v [T, H, dv]; beta [T, H]; log_alpha [T, H, dk] ([T, H]
+    with head_gate);
     cu_seqlens [N + 1] int32 on the device; initial_state [N, H, dk, dv] or None.
     Returns (o [T, H, dv], final_state [N, H, dk, dv] or None)."""
     T, H, dk = q.shape
@@ -109,7 +123,7 @@ def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, 
         raise ValueError(f"unsupported dtype {dt}")
     for t, n, s, d in ((q, "q", (T, H, dk), dt), (k, "k", (T, H, dk), dt), (v, "v", (T, H, dv), dt),
                        (beta, "beta", (T, H), torch.float32),
-                       (log_alpha, "log_alpha", (T, H, dk), torch.float32),
+                       (log_alpha, "log_alpha", (T, H) if head_gate else (T, H, dk), torch.float32),
                        (cu_seqlens, "cu_seqlens", (N + 1,), torch.int32)):
         _check(t, n, s, d, dev)
     if initial_state is not None:
@@ -123,17 +137,18 @@ def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, 
         final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
     if final_state is not None:
         _check(final_state, "final_state", (N, H, dk, dv), torch.float32, dev)
-    _lib.call("kda_varlen_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
-              _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(o), _ptr(final_state), T, H, dk, dv,
-              chunk, _DTYPES[dt], _DTYPES[o.dtype], _stream(stream))
+    mode = _mode(head_gate, erase)
+    _lib.call("kda_varlen_fwd_mode" if mode else "kda_varlen_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+              _ptr(log_alpha), _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(o), _ptr(final_state), T, H, dk,
+              dv, chunk, _DTYPES[dt], _DTYPES[o.dtype], *((mode,) if mode else ()), _stream(stream))
     return o, final_state
 
 
 def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, o_dtype=torch.float32,
-                       stream=None):
+                       stream=None, head_gate=False, erase=True):
     """One decode step: q, k [N, H, dk], v [N, H, dv], beta [N, H],
-    log_alpha [N, H, dk]; state [N, H, dk, dv] fp32 is updated in place.
-    Returns o [N, H, dv]."""
+    log_alpha [N, H, dk] ([N, H] with head_gate); state [N, H, dk, dv] fp32 is
+    updated in place.  Returns o [N, H, dv]."""
     N, H, dk = q.shape
     dv = v.shape[-1]
     dev, dt = q.device, q.dtype
@@ -141,7 +156,7 @@ def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, o_dtype=torch
         raise ValueError(f"unsupported dtype {dt}")
     for t, n, s, d in ((q, "q", (N, H, dk), dt), (k, "k", (N, H, dk), dt), (v, "v", (N, H, dv), dt),
                        (beta, "beta", (N, H), torch.float32),
-                       (log_alpha, "log_alpha", (N, H, dk), torch.float32),
+                       (log_alpha, "log_alpha", (N, H) if head_gate else (N, H, dk), torch.float32),
                        (state, "state", (N, H, dk, dv), torch.float32)):
         _check(t, n, s, d, dev)
     if o is None:
@@ -149,8 +164,10 @@ def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, o_dtype=torch
     _check(o, "o", (N, H, dv), o.dtype, dev)
     if o.dtype not in _DTYPES:
         raise ValueError(f"unsupported output dtype {o.dtype}")
-    _lib.call("kda_recurrent_step", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
-              _ptr(state), _ptr(o), N, H, dk, dv, _DTYPES[dt], _DTYPES[o.dtype], _stream(stream))
+    mode = _mode(head_gate, erase)
+    _lib.call("kda_recurrent_step_mode" if mode else "kda_recurrent_step", _ptr(q), _ptr(k), _ptr(v),
+              _ptr(beta), _ptr(log_alpha), _ptr(state), _ptr(o), N, H, dk, dv, _DTYPES[dt], _DTYPES[o.dtype],
+              *((mode,) if mode else ()), _stream(stream))
     return o
 
 

@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(HERE, "libkda.so")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
 KDA_F32, KDA_BF16 = 0, 1
+KDA_MODE_HEAD_GATE, KDA_MODE_NO_ERASE = 1, 2
 
 # Every symbol include/kda.h declares, with its ctypes signature.
 _P = ctypes.c_void_p
@@ -23,6 +24,9 @@ SIGNATURES = {
     "kda_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "kda_varlen_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "kda_recurrent_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_chunk_fwd_mode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_varlen_fwd_mode": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_recurrent_step_mode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "kda_check": (_I, [_P]),
     "kda_selftest_timeout": (_I, [ctypes.c_longlong, _P]),
     "kda_status_string": (ctypes.c_char_p, [_I]),

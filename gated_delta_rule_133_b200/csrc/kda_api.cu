@@ -45,31 +45,34 @@ long long timeout_cycles()
 kda_status run_chunk(const void* q, const void* k, const void* v, const float* beta,
                      const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
                      int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype dtype,
-                     kda_dtype o_dtype, cudaStream_t s)
+                     kda_dtype o_dtype, int mode, cudaStream_t s)
 {
     const ChunkKernel kind = chunk_kernel();
-    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && kind == ChunkKernel::split)
-        return from_cuda(kda::chunk_fwd_split(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk,
-                                              dv, o_dtype, timeout_cycles(), s));
-    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && kind == ChunkKernel::fused)
+    // the single-pass kernel implements the plain layer only: variants take the two-pass path
+    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && kind == ChunkKernel::fused && mode == 0)
         return from_cuda(kda::chunk_fwd_tc(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk,
                                            dv, o_dtype, timeout_cycles(), s));
+    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && kind != ChunkKernel::simt)
+        return from_cuda(kda::chunk_fwd_split(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk,
+                                              dv, o_dtype, timeout_cycles(), mode, s));
     return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, dtype,
-                                         o_dtype, s));
+                                         o_dtype, mode, s));
 }
+
+bool valid_mode(int mode) { return (mode & ~(KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE)) == 0; }
 
 // Shared checks of the forward entry points.
 kda_status check_fwd(const void* q, const void* k, const void* v, const float* beta,
                      const float* log_alpha, const float* s0, const void* o, const float* sT,
                      long long tokens, int H, int dk, int dv, int chunk, kda_dtype dtype,
-                     kda_dtype o_dtype)
+                     kda_dtype o_dtype, int mode)
 {
     if (H <= 0 || dk <= 0 || dv <= 0 || tokens < 0) return KDA_ERR_INVALID_ARG;
-    if (!valid_dtype(dtype) || !valid_dtype(o_dtype)) return KDA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype) || !valid_dtype(o_dtype) || !valid_mode(mode)) return KDA_ERR_INVALID_ARG;
+    const bool gate_ok = (mode & KDA_MODE_HEAD_GATE) ? aligned4(log_alpha) : aligned16(log_alpha);
     if (tokens > 0) {
         if (!q || !k || !v || !beta || !log_alpha || !o) return KDA_ERR_INVALID_ARG;
-        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(beta) ||
-            !aligned16(log_alpha) || !aligned16(o))
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(beta) || !gate_ok || !aligned16(o))
             return KDA_ERR_INVALID_ARG;
     }
     if ((s0 && !aligned16(s0)) || (sT && !aligned16(sT))) return KDA_ERR_INVALID_ARG;
@@ -105,21 +108,30 @@ __global__ void selftest_timeout_kernel(long long limit_cycles)
 
 extern "C" {
 
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
-                         const float* log_alpha, const float* initial_state, void* o,
-                         float* final_state, int B, int T, int H, int dk, int dv, int chunk,
-                         kda_dtype dtype, kda_dtype o_dtype, void* stream)
+kda_status kda_chunk_fwd_mode(const void* q, const void* k, const void* v, const float* beta,
+                              const float* log_alpha, const float* initial_state, void* o,
+                              float* final_state, int B, int T, int H, int dk, int dv, int chunk,
+                              kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream)
 {
     if (B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
     const long long tokens = (long long)B * T;
     kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, tokens, H,
-                              dk, dv, chunk, dtype, o_dtype);
+                              dk, dv, chunk, dtype, o_dtype, mode);
     if (st != KDA_OK) return st;
     if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (tokens == 0) return copy_state(initial_state, final_state, (size_t)B * H * dk * dv, s);
     return run_chunk(q, k, v, beta, log_alpha, initial_state, o, final_state, nullptr, B, T, tokens, H, dk,
-                     dv, dtype, o_dtype, s);
+                     dv, dtype, o_dtype, mode, s);
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
+                         const float* log_alpha, const float* initial_state, void* o,
+                         float* final_state, int B, int T, int H, int dk, int dv, int chunk,
+                         kda_dtype dtype, kda_dtype o_dtype, void* stream)
+{
+    return kda_chunk_fwd_mode(q, k, v, beta, log_alpha, initial_state, o, final_state, B, T, H, dk, dv, chunk,
+                              dtype, o_dtype, 0, stream);
 }
 
 kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* beta,
@@ -130,17 +142,35 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, co
     if (B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
     const long long tokens = (long long)B * T;
     kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, tokens, H,
-                              dk, dv, chunk, dtype, o_dtype);
+                              dk, dv, chunk, dtype, o_dtype, 0);
     if (st != KDA_OK) return st;
     if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (tokens == 0) return copy_state(initial_state, final_state, (size_t)B * H * dk * dv, s);
     if (!kda::chunk_fwd_tc_supported(dk, dv, dtype))   // the CUDA-core kernel needs no scratch
         return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, initial_state, o, final_state, nullptr, B,
-                                             T, H, dk, dv, dtype, o_dtype, s));
+                                             T, H, dk, dv, dtype, o_dtype, 0, s));
     if (!kda::chunk_fwd_noalloc_fits(B, T, H, dk, dv, final_state != nullptr)) return KDA_ERR_UNSUPPORTED;
     return from_cuda(kda::chunk_fwd_noalloc(q, k, v, beta, log_alpha, initial_state, o, final_state, B, T, tokens,
                                             H, dk, dv, o_dtype, timeout_cycles(), s));
+}
+
+kda_status kda_varlen_fwd_mode(const void* q, const void* k, const void* v, const float* beta,
+                               const float* log_alpha, const int32_t* cu_seqlens, int N,
+                               const float* initial_state, void* o, float* final_state, int T, int H,
+                               int dk, int dv, int chunk, kda_dtype dtype, kda_dtype o_dtype, int mode,
+                               void* stream)
+{
+    if (N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, T, H, dk,
+                              dv, chunk, dtype, o_dtype, mode);
+    if (st != KDA_OK) return st;
+    if (N == 0) return T == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
+    if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) return copy_state(initial_state, final_state, (size_t)N * H * dk * dv, s);
+    return run_chunk(q, k, v, beta, log_alpha, initial_state, o, final_state, cu_seqlens, N, T, T, H, dk,
+                     dv, dtype, o_dtype, mode, s);
 }
 
 kda_status kda_varlen_fwd(const void* q, const void* k, const void* v, const float* beta,
@@ -149,32 +179,32 @@ kda_status kda_varlen_fwd(const void* q, const void* k, const void* v, const flo
                           int dk, int dv, int chunk, kda_dtype dtype, kda_dtype o_dtype,
                           void* stream)
 {
-    if (N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
-    kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, T, H, dk,
-                              dv, chunk, dtype, o_dtype);
-    if (st != KDA_OK) return st;
-    if (N == 0) return T == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
-    if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARG;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (T == 0) return copy_state(initial_state, final_state, (size_t)N * H * dk * dv, s);
-    return run_chunk(q, k, v, beta, log_alpha, initial_state, o, final_state, cu_seqlens, N, T, T, H, dk,
-                     dv, dtype, o_dtype, s);
+    return kda_varlen_fwd_mode(q, k, v, beta, log_alpha, cu_seqlens, N, initial_state, o, final_state, T, H,
+                               dk, dv, chunk, dtype, o_dtype, 0, stream);
+}
+
+kda_status kda_recurrent_step_mode(const void* q, const void* k, const void* v, const float* beta,
+                                   const float* log_alpha, float* state, void* o, int N, int H, int dk,
+                                   int dv, kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream)
+{
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype) || !valid_dtype(o_dtype) || !valid_mode(mode)) return KDA_ERR_INVALID_ARG;
+    if (N == 0) return KDA_OK;
+    if (!q || !k || !v || !beta || !log_alpha || !state || !o) return KDA_ERR_INVALID_ARG;
+    const bool gate_ok = (mode & KDA_MODE_HEAD_GATE) ? aligned4(log_alpha) : aligned16(log_alpha);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(beta) || !gate_ok ||
+        !aligned16(state) || !aligned16(o))
+        return KDA_ERR_INVALID_ARG;
+    if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_UNSUPPORTED;
+    return from_cuda(kda::decode_step(q, k, v, beta, log_alpha, state, o, (long long)N * H, dk,
+                                      dv, dtype, o_dtype, mode, static_cast<cudaStream_t>(stream)));
 }
 
 kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* beta,
                               const float* log_alpha, float* state, void* o, int N, int H, int dk,
                               int dv, kda_dtype dtype, kda_dtype o_dtype, void* stream)
 {
-    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
-    if (!valid_dtype(dtype) || !valid_dtype(o_dtype)) return KDA_ERR_INVALID_ARG;
-    if (N == 0) return KDA_OK;
-    if (!q || !k || !v || !beta || !log_alpha || !state || !o) return KDA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(beta) ||
-        !aligned16(log_alpha) || !aligned16(state) || !aligned16(o))
-        return KDA_ERR_INVALID_ARG;
-    if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_UNSUPPORTED;
-    return from_cuda(kda::decode_step(q, k, v, beta, log_alpha, state, o, (long long)N * H, dk,
-                                      dv, dtype, o_dtype, static_cast<cudaStream_t>(stream)));
+    return kda_recurrent_step_mode(q, k, v, beta, log_alpha, state, o, N, H, dk, dv, dtype, o_dtype, 0, stream);
 }
 
 kda_status kda_check(void* stream)

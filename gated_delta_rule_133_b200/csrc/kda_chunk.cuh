@@ -6,16 +6,17 @@
 namespace kda {
 
 // Decode step over NH = N * H independent (sequence, head) states.
+// `mode`: KDA_MODE_* flags of kda.h (0 = the KDA layer).
 cudaError_t decode_step(const void* q, const void* k, const void* v, const float* beta,
                         const float* log_alpha, float* state, void* o, long long NH, int dk,
-                        int dv, kda_dtype dtype, kda_dtype o_dtype, cudaStream_t stream);
+                        int dv, kda_dtype dtype, kda_dtype o_dtype, int mode, cudaStream_t stream);
 
 // Chunkwise forward on CUDA cores (fp32 arithmetic).  cu == nullptr: nseq
 // sequences of T tokens each; otherwise nseq packed sequences given by cu.
 cudaError_t chunk_fwd_simt(const void* q, const void* k, const void* v, const float* beta,
                            const float* log_alpha, const float* s0, void* o, float* sT,
                            const int32_t* cu, int nseq, int T, int H, int dk, int dv,
-                           kda_dtype dtype, kda_dtype o_dtype, cudaStream_t stream);
+                           kda_dtype dtype, kda_dtype o_dtype, int mode, cudaStream_t stream);
 
 // Chunkwise forward on the tensor cores (bf16 q/k/v only).  `tokens` is the
 // length of the packed token axis (B * T, or the varlen total).
@@ -32,7 +33,7 @@ cudaError_t chunk_fwd_tc(const void* q, const void* k, const void* v, const floa
 cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const float* beta,
                             const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
                             int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
-                            long long timeout_cycles, cudaStream_t stream);
+                            long long timeout_cycles, int mode, cudaStream_t stream);
 
 // Same as chunk_fwd_split for dense inputs, with every intermediate in a
 // fixed library-owned device area instead of a stream-ordered allocation;

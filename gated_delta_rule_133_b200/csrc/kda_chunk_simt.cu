@@ -102,8 +102,10 @@ __global__ void __launch_bounds__(NT)
 chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                       const TIn* __restrict__ v, const float* __restrict__ beta,
                       const float* __restrict__ log_alpha, const float* s0, TOut* __restrict__ o,
-                      float* sT, const int32_t* __restrict__ cu, int nseq, int T, int H, int DV)
+                      float* sT, const int32_t* __restrict__ cu, int nseq, int T, int H, int DV, int mode)
 {
+    const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;   // log_alpha [tokens, H]
+    const bool erase = (mode & KDA_MODE_NO_ERASE) == 0;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Smem<DK>& sm = *reinterpret_cast<Smem<DK>*>(smem_raw);
     constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC;
@@ -143,7 +145,7 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                 const size_t off = ((size_t)(tok0 + t0 + r) * H + h) * DK + c;
                 qv = Elem<TIn>::load(q + off);
                 kv = Elem<TIn>::load(k + off);
-                gv = log_alpha[off];
+                gv = head_gate ? log_alpha[(size_t)(tok0 + t0 + r) * H + h] : log_alpha[off];
             }
             sm.qm[r * LDK + c] = qv;
             sm.km[r * LDK + c] = kv;
@@ -190,7 +192,7 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                 for (int j = 0; j < 4; ++j) {
                     const int r = tm + 16 * i, s = tn + 16 * j;
                     sm.P[r * LDC + s] = s <= r ? p[i][j] : 0.f;
-                    sm.A[r * LDC + s] = s < r ? sm.beta[r] * a[i][j] : 0.f;
+                    sm.A[r * LDC + s] = (erase && s < r) ? sm.beta[r] * a[i][j] : 0.f;
                 }
             // Sm = exp(G_m) * S  (state rows scaled per key channel)
             for (int e = tid; e < DK * NV; e += NT) sm.Sm[e] = sm.gm[e / NV] * sm.S[e];
@@ -222,7 +224,7 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int r = tm + 16 * i, cc = tn + 16 * j;
-                    sm.V[r * NV + cc] = sm.beta[r] * (sm.V[r * NV + cc] - x[i][j]);
+                    sm.V[r * NV + cc] = sm.beta[r] * (sm.V[r * NV + cc] - (erase ? x[i][j] : 0.f));
                 }
         }
         __syncthreads();
@@ -281,7 +283,7 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 template <typename TIn, typename TOut, int DK>
 cudaError_t launch(const void* q, const void* k, const void* v, const float* beta,
                    const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
-                   int nseq, int T, int H, int dv, cudaStream_t stream)
+                   int nseq, int T, int H, int dv, int mode, cudaStream_t stream)
 {
     const size_t smem = sizeof(Smem<DK>);
     auto kern = chunk_fwd_simt_kernel<TIn, TOut, DK>;
@@ -292,17 +294,17 @@ cudaError_t launch(const void* q, const void* k, const void* v, const float* bet
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     kern<<<(unsigned)blocks, NT, smem, stream>>>(
         static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), beta,
-        log_alpha, s0, static_cast<TOut*>(o), sT, cu, nseq, T, H, dv);
+        log_alpha, s0, static_cast<TOut*>(o), sT, cu, nseq, T, H, dv, mode);
     return cudaGetLastError();
 }
 
 template <typename TIn, typename TOut>
 cudaError_t launch_dk(const void* q, const void* k, const void* v, const float* beta,
                       const float* log_alpha, const float* s0, void* o, float* sT,
-                      const int32_t* cu, int nseq, int T, int H, int dk, int dv, cudaStream_t s)
+                      const int32_t* cu, int nseq, int T, int H, int dk, int dv, int mode, cudaStream_t s)
 {
-    if (dk == 128) return launch<TIn, TOut, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, s);
-    if (dk == 64) return launch<TIn, TOut, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, s);
+    if (dk == 128) return launch<TIn, TOut, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, mode, s);
+    if (dk == 64) return launch<TIn, TOut, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, mode, s);
     return cudaErrorInvalidValue;
 }
 
@@ -311,16 +313,16 @@ cudaError_t launch_dk(const void* q, const void* k, const void* v, const float* 
 cudaError_t chunk_fwd_simt(const void* q, const void* k, const void* v, const float* beta,
                            const float* log_alpha, const float* s0, void* o, float* sT,
                            const int32_t* cu, int nseq, int T, int H, int dk, int dv,
-                           kda_dtype dtype, kda_dtype o_dtype, cudaStream_t s)
+                           kda_dtype dtype, kda_dtype o_dtype, int mode, cudaStream_t s)
 {
     using bf = __nv_bfloat16;
     if (dtype == KDA_BF16 && o_dtype == KDA_BF16)
-        return simt::launch_dk<bf, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, s);
+        return simt::launch_dk<bf, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, mode, s);
     if (dtype == KDA_BF16 && o_dtype == KDA_F32)
-        return simt::launch_dk<bf, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, s);
+        return simt::launch_dk<bf, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, mode, s);
     if (dtype == KDA_F32 && o_dtype == KDA_BF16)
-        return simt::launch_dk<float, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, s);
-    return simt::launch_dk<float, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, s);
+        return simt::launch_dk<float, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, mode, s);
+    return simt::launch_dk<float, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, mode, s);
 }
 
 }  // namespace kda

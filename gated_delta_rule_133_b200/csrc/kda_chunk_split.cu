@@ -128,6 +128,8 @@ struct PrepParams {
     long long tokens;
     long long timeout_cycles;
     unsigned* ready;         // cooperative schedule: ready[record] = 1 once the record is complete
+    const float* gh;         // one gate per (token, head), [tokens, H] (KDA_MODE_HEAD_GATE), or nullptr
+    int no_erase;            // KDA_MODE_NO_ERASE: A = 0, so T = I
 };
 
 struct Item {
@@ -238,7 +240,8 @@ __device__ __forceinline__ Vec vec_at(unsigned char* base, int buf)
 // key channel t % 128, rows [21 p, 21 p + 21) of part p = t / 128, the last
 // part 22 rows), and the item's channel vectors.  Named barrier 2.
 template <int DK>
-__device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t, float beta_v)
+__device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t, float beta_v,
+                                          const float* gh, long long gbase, int H)
 {
     const int ch = t & 127, part = t >> 7;
     const int r0 = 21 * part, nr = part == 2 ? 22 : 21;
@@ -247,7 +250,7 @@ __device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t,
 #pragma unroll
         for (int rr = 0; rr < 22; ++rr) {
             const int row = r0 + rr;
-            G[rr] = (rr < nr && row < L) ? gs[row * DK + ch] : 0.f;
+            G[rr] = (rr < nr && row < L) ? (gh ? gh[gbase + (long long)row * H] : gs[row * DK + ch]) : 0.f;
         }
 #pragma unroll
         for (int rr = 1; rr < 22; ++rr) G[rr] += G[rr - 1];
@@ -485,7 +488,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         fence_proxy_async();
         prefetch_tmap(&tmq);
         prefetch_tmap(&tmk);
-        prefetch_tmap(&tmg);
+        if (!p.gh) prefetch_tmap(&tmg);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -511,11 +514,11 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     bool unpublished = false;
     long long stored_rec = 0;
 
-    auto load_item = [&](const Item& it) {   // thread 0
-        mbar_expect_tx(mb_tma, kStageBytes);
+    auto load_item = [&](const Item& it) {   // one thread; per-head gates are read by the cumsum
+        mbar_expect_tx(mb_tma, p.gh ? (uint32_t)C * DK * 4 : kStageBytes);
         tma_load_3d((void*)x.qs, &tmq, mb_tma, 0, it.h, it.tok0);
         tma_load_3d((void*)x.ks, &tmk, mb_tma, 0, it.h, it.tok0);
-        tma_load_3d((void*)x.gs, &tmg, mb_tma, 0, it.h, it.tok0);
+        if (!p.gh) tma_load_3d((void*)x.gs, &tmg, mb_tma, 0, it.h, it.tok0);
     };
     auto beta_of = [&](const Item& it, int t) {
         return (it.ok && t < C && t < it.L) ? p.beta[(size_t)(it.tok0 + t) * H + it.h] : 0.f;
@@ -538,7 +541,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
             const float b = v.beta[r];
             float a[16];
 #pragma unroll
-            for (int s2 = 0; s2 < 16; ++s2) a[s2] = (16 * wg + s2 < r) ? b * pa[s2] : 0.f;
+            for (int s2 = 0; s2 < 16; ++s2) a[s2] = (!p.no_erase && 16 * wg + s2 < r) ? b * pa[s2] : 0.f;
 #pragma unroll
             for (int s4 = 0; s4 < 4; ++s4)
                 *reinterpret_cast<float4*>(As + r * LDT + 16 * wg + 4 * s4) =
@@ -568,7 +571,8 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     {
         const float beta_v = tid >= 128 ? beta_of(cur, tid - 128) : 0.f;
         KDA_WAIT_OR_EXIT(mb_tma, 1u, 0);
-        if (tid >= 128) cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v);
+        if (tid >= 128)
+            cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v, p.gh, (long long)cur.tok0 * H + cur.h, H);
         __syncthreads();
         build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)cur.rec * R::BYTES, cur.L, tid, NT, 0, C);
     }
@@ -613,7 +617,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
                 const float beta_v = beta_of(nxt, t);
                 const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
                 if (!bar_or(3, 384, !ok)) {
-                    cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v);
+                    cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v, p.gh, (long long)nxt.tok0 * H + nxt.h, H);
                     build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384, 0, C);
                 }
             }
@@ -731,6 +735,7 @@ struct ScanParams {
     long long tokens;
     long long timeout_cycles;
     const unsigned* ready;   // cooperative schedule: wait for ready[record] before loading it
+    int no_erase;            // KDA_MODE_NO_ERASE: Y = beta V (no X term)
 };
 
 // Shared memory of the scan kernel: two 72 KB slots, each holding one record
@@ -1026,8 +1031,8 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
                     for (int w = 0; w < 4; ++w) {
                         const float2 f2 = __bfloat1622float2(v2[w]);
                         const int jj = 8 * u + 2 * w;
-                        y[jj] = bs * (f2.x - x16[jj]);
-                        y[jj + 1] = bs * (f2.y - x16[jj + 1]);
+                        y[jj] = bs * (f2.x - (p.no_erase ? 0.f : x16[jj]));
+                        y[jj + 1] = bs * (f2.y - (p.no_erase ? 0.f : x16[jj + 1]));
                     }
                 }
                 st_row_h16(Yb, s, 16 * wg, C, y);
@@ -1238,8 +1243,9 @@ static int chunk_blocks(int nch, long long scan_ctas, int nsm)
 template <typename TO, int DK>
 static cudaError_t run(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
                        const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens,
-                       int H, int dv, long long timeout_cycles, cudaStream_t stream)
+                       int H, int dv, long long timeout_cycles, int mode, cudaStream_t stream)
 {
+    const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;
     using R = Rec<DK>;
     const int nsm = sm_count();
     const int nch = cu ? 0 : (T + C - 1) / C;
@@ -1257,8 +1263,9 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     cudaStream_t side = nb > 1 ? side_stream() : nullptr;
 
     CUtensorMap tq, tk, tg;
+    memset(&tg, 0, sizeof(tg));   // per-head gates: no gate tile to load (the map is never used)
     if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
-        !make_tmap(&tg, log_alpha, tokens, H, DK, true))
+        (!head_gate && !make_tmap(&tg, log_alpha, tokens, H, DK, true)))
         return cudaErrorInvalidValue;
     CUtensorMap tv, to;
     if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
@@ -1318,7 +1325,10 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     pp.rc0 = 0;
     pp.tokens = tokens;
     pp.timeout_cycles = timeout_cycles;
+    pp.gh = head_gate ? log_alpha : nullptr;
+    pp.no_erase = (mode & KDA_MODE_NO_ERASE) ? 1 : 0;
     ScanParams sp{};
+    sp.no_erase = pp.no_erase;
     sp.v = static_cast<const __nv_bfloat16*>(v);
     sp.o = o;
     sp.cu = cu;
@@ -1584,14 +1594,14 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
 cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const float* beta,
                             const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
                             int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
-                            long long timeout_cycles, cudaStream_t stream)
+                            long long timeout_cycles, int mode, cudaStream_t stream)
 {
     if (o_dtype == KDA_F32) {
-        if (dk == 128) return split::run<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
-        if (dk == 64) return split::run<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 128) return split::run<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, stream);
+        if (dk == 64) return split::run<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, stream);
     } else {
-        if (dk == 128) return split::run<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
-        if (dk == 64) return split::run<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 128) return split::run<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, stream);
+        if (dk == 64) return split::run<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -21,8 +21,10 @@ template <typename T, typename TO, int DK, int DV>
 __global__ void __launch_bounds__(256)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ log_alpha,
-                   float* __restrict__ state, TO* __restrict__ o)
+                   float* __restrict__ state, TO* __restrict__ o, int mode)
 {
+    const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;   // log_alpha [NH]: one gate per head
+    const bool erase = (mode & KDA_MODE_NO_ERASE) == 0;
     constexpr int COLS = 64;
     constexpr int SPLIT = DV / COLS;
     constexpr int RPT = DK / 16;          // key rows per thread
@@ -44,7 +46,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     for (int i = t; i < DK; i += 256) {
         sk[i] = Elem<T>::load(k + (size_t)head * DK + i);
         sq[i] = Elem<T>::load(q + (size_t)head * DK + i);
-        sa[i] = expf(log_alpha[(size_t)head * DK + i]);
+        sa[i] = expf(head_gate ? log_alpha[head] : log_alpha[(size_t)head * DK + i]);
     }
     __syncthreads();
 
@@ -87,7 +89,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     float d[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-        d[j] = b * (Elem<T>::load(v + (size_t)head * DV + col0 + 4 * cg + j) - R[j]);
+        d[j] = b * (Elem<T>::load(v + (size_t)head * DV + col0 + 4 * cg + j) - (erase ? R[j] : 0.f));
 
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
@@ -107,37 +109,37 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 template <typename T, typename TO, int DK, int DV>
 static cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* beta,
                                  const float* log_alpha, float* state, void* o, long long NH,
-                                 cudaStream_t stream)
+                                 int mode, cudaStream_t stream)
 {
     const long long blocks = NH * (DV / 64);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     decode_step_kernel<T, TO, DK, DV><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), beta,
-        log_alpha, state, static_cast<TO*>(o));
+        log_alpha, state, static_cast<TO*>(o), mode);
     return cudaGetLastError();
 }
 
 template <typename T, typename TO>
 static cudaError_t decode_dims(const void* q, const void* k, const void* v, const float* beta,
                                const float* log_alpha, float* state, void* o, long long NH, int dk,
-                               int dv, cudaStream_t s)
+                               int dv, int mode, cudaStream_t s)
 {
-    if (dk == 128 && dv == 128) return launch_decode<T, TO, 128, 128>(q, k, v, beta, log_alpha, state, o, NH, s);
-    if (dk == 128 && dv == 64) return launch_decode<T, TO, 128, 64>(q, k, v, beta, log_alpha, state, o, NH, s);
-    if (dk == 64 && dv == 128) return launch_decode<T, TO, 64, 128>(q, k, v, beta, log_alpha, state, o, NH, s);
-    if (dk == 64 && dv == 64) return launch_decode<T, TO, 64, 64>(q, k, v, beta, log_alpha, state, o, NH, s);
+    if (dk == 128 && dv == 128) return launch_decode<T, TO, 128, 128>(q, k, v, beta, log_alpha, state, o, NH, mode, s);
+    if (dk == 128 && dv == 64) return launch_decode<T, TO, 128, 64>(q, k, v, beta, log_alpha, state, o, NH, mode, s);
+    if (dk == 64 && dv == 128) return launch_decode<T, TO, 64, 128>(q, k, v, beta, log_alpha, state, o, NH, mode, s);
+    if (dk == 64 && dv == 64) return launch_decode<T, TO, 64, 64>(q, k, v, beta, log_alpha, state, o, NH, mode, s);
     return cudaErrorInvalidValue;
 }
 
 cudaError_t decode_step(const void* q, const void* k, const void* v, const float* beta,
                         const float* log_alpha, float* state, void* o, long long NH, int dk,
-                        int dv, kda_dtype dtype, kda_dtype o_dtype, cudaStream_t s)
+                        int dv, kda_dtype dtype, kda_dtype o_dtype, int mode, cudaStream_t s)
 {
     using bf = __nv_bfloat16;
-    if (dtype == KDA_BF16 && o_dtype == KDA_BF16) return decode_dims<bf, bf>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, s);
-    if (dtype == KDA_BF16 && o_dtype == KDA_F32) return decode_dims<bf, float>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, s);
-    if (dtype == KDA_F32 && o_dtype == KDA_BF16) return decode_dims<float, bf>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, s);
-    return decode_dims<float, float>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, s);
+    if (dtype == KDA_BF16 && o_dtype == KDA_BF16) return decode_dims<bf, bf>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, mode, s);
+    if (dtype == KDA_BF16 && o_dtype == KDA_F32) return decode_dims<bf, float>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, mode, s);
+    if (dtype == KDA_F32 && o_dtype == KDA_BF16) return decode_dims<float, bf>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, mode, s);
+    return decode_dims<float, float>(q, k, v, beta, log_alpha, state, o, NH, dk, dv, mode, s);
 }
 
 }  // namespace kda

@@ -150,6 +150,46 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
                               kda_dtype dtype, kda_dtype o_dtype, void* stream);
 
 /*
+ * Variants of the layer, selected by the bit flags `mode` of the *_mode entry
+ * points below (mode = 0 is the layer above; unknown bits return
+ * KDA_ERR_INVALID_ARG).  Both are gate tiers of "Hybrid Linear Attention
+ * Architecture: Making LLM Training and Inference More Efficient", section 3.3:
+ *
+ *  KDA_MODE_HEAD_GATE  one forget gate per (token, head), the scalar gate:
+ *      log_alpha has no d_k axis ([B, T, H], [T, H] or [N, H]; 4-byte
+ *      aligned) and alpha_t scales every key channel of the state alike.  With
+ *      a scalar gate the decay commutes with the erase, so the section's two
+ *      orderings coincide.
+ *  KDA_MODE_NO_ERASE   no erase term: S_t = Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *      the element-wise gate without the delta rule (beta_t = 1 gives the
+ *      section's form; per-channel decay of the key rows as in this layer).
+ *
+ * The flags combine.  Every other argument, layout and rule is that of the
+ * plain entry point of the same name.
+ */
+#define KDA_MODE_HEAD_GATE 1
+#define KDA_MODE_NO_ERASE 2
+
+kda_status kda_chunk_fwd_mode(const void* q, const void* k, const void* v,
+                              const float* beta, const float* log_alpha,
+                              const float* initial_state, void* o, float* final_state,
+                              int B, int T, int H, int dk, int dv, int chunk,
+                              kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream);
+
+kda_status kda_varlen_fwd_mode(const void* q, const void* k, const void* v,
+                               const float* beta, const float* log_alpha,
+                               const int32_t* cu_seqlens, int N,
+                               const float* initial_state, void* o, float* final_state,
+                               int T, int H, int dk, int dv, int chunk,
+                               kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream);
+
+kda_status kda_recurrent_step_mode(const void* q, const void* k, const void* v,
+                                   const float* beta, const float* log_alpha,
+                                   float* state, void* o,
+                                   int N, int H, int dk, int dv,
+                                   kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream);
+
+/*
  * Synchronises `stream` and reports (then clears) the current device's
  * status word: KDA_ERR_TIMEOUT if a device-side bounded wait ran out since the
  * last check, KDA_ERR_INVALID_ARG if a kernel found device-resident sequence

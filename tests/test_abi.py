@@ -106,3 +106,23 @@ def test_noalloc_validation():
     assert f(*ok[:11], 96, *ok[12:]) == _lib.KDA_ERR_UNSUPPORTED
     # 10 x 64 (sequence, head) pairs: two chunks of records exceed the 64 MiB area
     assert f(*ok[:8], 10, 8, 64, *ok[11:]) == _lib.KDA_ERR_UNSUPPORTED
+
+
+def test_mode_validation():
+    """Layer variants: unknown mode bits are rejected; a per-head gate array
+    needs only 4-byte alignment, a per-channel one 16 bytes."""
+    lib = _lib.load()
+    base = (P, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 1, 0)
+    assert lib.kda_chunk_fwd_mode(*base, 4, None) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_fwd_mode(*base, -1, None) == _lib.KDA_ERR_INVALID_ARG
+    gate4 = base[:4] + (P + 4,) + base[5:]
+    assert lib.kda_chunk_fwd_mode(*gate4, _lib.KDA_MODE_NO_ERASE, None) == _lib.KDA_ERR_INVALID_ARG
+    # 4-byte-aligned per-head gates pass validation: an unsupported head size then decides
+    gate4_d96 = gate4[:11] + (96,) + gate4[12:]
+    assert lib.kda_chunk_fwd_mode(*gate4_d96, _lib.KDA_MODE_HEAD_GATE, None) == _lib.KDA_ERR_UNSUPPORTED
+    v = lib.kda_varlen_fwd_mode
+    assert v(P, P, P, P, P, P, 1, None, P, None, 8, 2, 128, 128, 64, 1, 0, 8, None) == _lib.KDA_ERR_INVALID_ARG
+    r = lib.kda_recurrent_step_mode
+    assert r(P, P, P, P, P, P, P, 3, 2, 128, 128, 1, 0, 4, None) == _lib.KDA_ERR_INVALID_ARG
+    assert r(P, P, P, P, P + 4, P, P, 3, 2, 128, 128, 1, 0, 0, None) == _lib.KDA_ERR_INVALID_ARG
+    assert r(P, P, P, P, P + 4, P, P, 3, 2, 96, 128, 1, 0, _lib.KDA_MODE_HEAD_GATE, None) == _lib.KDA_ERR_UNSUPPORTED
