@@ -337,14 +337,29 @@ def run_decode(kda, device, stream, world, rank, warmup):
 
 def run_other_workloads(kda, device, stream, world, rank, reps=3):
     """Varlen (8 packed sequences, 65536 tokens, H32) and long-context (T131072,
-    H32) chunk forwards: one warm-up launch, `reps` timed launches each."""
+    H32) chunk forwards, and the prefill shape with the two layer variants (one
+    gate per head; no erase term): one warm-up launch, `reps` timed launches
+    each."""
     from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
     pk, kind = peaks()
     out = {}
-    for name in ("varlen", "long"):
-        w = WORKLOADS[name]
+    for name in ("varlen", "long", "prefill_head_gate", "prefill_no_erase"):
+        w = WORKLOADS[name.split("_")[0]]
         d = make_inputs(w, device, seed=w.seed + 1000 * rank)
-        if name == "varlen":
+        gate_bytes = 4 * w.dk
+        desc = f"{name}: {w.B * w.T if w.kind != 'varlen' else w.T} tokens, H={w.H}, d_k=d_v={w.dk}, bf16 q/k/v, fp32 o and state"
+        if name.startswith("prefill"):
+            head_gate, erase = name == "prefill_head_gate", name != "prefill_no_erase"
+            if head_gate:
+                d["log_alpha"] = d["log_alpha"][..., 0].contiguous()
+                gate_bytes = 4
+            o = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32, device=device)
+            sN = torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
+            call = lambda: kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], d["initial_state"],
+                                             o=o, final_state=sN, stream=stream, head_gate=head_gate, erase=erase)
+            tokens, states = w.B * w.T, 2 * w.B
+            desc += ", " + ("one forget gate per (token, head)" if head_gate else "no erase term")
+        elif name == "varlen":
             cu = d["cu_seqlens"]
             nseq = cu.numel() - 1
             o = torch.empty(w.T, w.H, w.dv, dtype=torch.float32, device=device)
@@ -369,12 +384,14 @@ def run_other_workloads(kda, device, stream, world, rank, reps=3):
         torch.cuda.synchronize(device)
         kda.kda_check()
         t = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3, world, device)
-        nbytes = tokens * w.H * bytes_per_token_head(w.dk, w.dv, 2, 4) + states * w.H * w.dk * w.dv * 4
-        nflops = tokens * w.H * flops_per_token_head(w.dk, w.dv)
-        out[name] = {"workload": f"{name}: {tokens} tokens, H={w.H}, d_k=d_v={w.dk}, bf16 q/k/v, fp32 o and state",
-                     "ms": t * 1e3, "tokens_per_s": tokens * world / t, "tflops": nflops * world / t / 1e12,
+        nbytes = (tokens * w.H * (bytes_per_token_head(w.dk, w.dv, 2, 4) - 4 * w.dk + gate_bytes)
+                  + states * w.H * w.dk * w.dv * 4)
+        out[name] = {"workload": desc, "ms": t * 1e3, "tokens_per_s": tokens * world / t,
                      "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                  "frac": nbytes / t / 1e9 / pk["hbm_gbs"], "peak_kind": f"{kind} copy bandwidth"}}
+                                  "frac": nbytes / t / 1e9 / pk["hbm_gbs"], "peak_kind": f"{kind} copy bandwidth",
+                                  "bytes_per_launch": nbytes}}
+        if not name.startswith("prefill"):   # the layer's FLOPs (the variants do less arithmetic)
+            out[name]["tflops"] = tokens * w.H * flops_per_token_head(w.dk, w.dv) * world / t / 1e12
         del d, o, sN
         torch.cuda.empty_cache()
     return out

@@ -450,10 +450,13 @@ __device__ __forceinline__ void ut_rows(float* As, float* X, unsigned char* Top)
 // TMEM: [P ; A~] double-buffered (0, 64); the fp16 A operands of Z and PT,
 // k e^(G_last - G) transposed (128) and masked P (160), two per 32-bit column;
 // Z 192, PT 256.
-template <int DK>
+template <int DK, bool VAR>
 __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmg,
                                           const PrepParams& p, int bid, int nblk)
 {
+    // layer variants (VAR instantiations only; the plain layer compiles without them)
+    const float* const gh = VAR ? p.gh : nullptr;
+    const bool no_erase = VAR && p.no_erase;
     using PL = PrepPlan;
     using R = Rec<DK>;
     extern __shared__ unsigned char smem_raw[];
@@ -488,7 +491,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         fence_proxy_async();
         prefetch_tmap(&tmq);
         prefetch_tmap(&tmk);
-        if (!p.gh) prefetch_tmap(&tmg);
+        if (!gh) prefetch_tmap(&tmg);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -515,10 +518,10 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     long long stored_rec = 0;
 
     auto load_item = [&](const Item& it) {   // one thread; per-head gates are read by the cumsum
-        mbar_expect_tx(mb_tma, p.gh ? (uint32_t)C * DK * 4 : kStageBytes);
+        mbar_expect_tx(mb_tma, gh ? (uint32_t)C * DK * 4 : kStageBytes);
         tma_load_3d((void*)x.qs, &tmq, mb_tma, 0, it.h, it.tok0);
         tma_load_3d((void*)x.ks, &tmk, mb_tma, 0, it.h, it.tok0);
-        if (!p.gh) tma_load_3d((void*)x.gs, &tmg, mb_tma, 0, it.h, it.tok0);
+        if (!gh) tma_load_3d((void*)x.gs, &tmg, mb_tma, 0, it.h, it.tok0);
     };
     auto beta_of = [&](const Item& it, int t) {
         return (it.ok && t < C && t < it.L) ? p.beta[(size_t)(it.tok0 + t) * H + it.h] : 0.f;
@@ -541,7 +544,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
             const float b = v.beta[r];
             float a[16];
 #pragma unroll
-            for (int s2 = 0; s2 < 16; ++s2) a[s2] = (!p.no_erase && 16 * wg + s2 < r) ? b * pa[s2] : 0.f;
+            for (int s2 = 0; s2 < 16; ++s2) a[s2] = (!no_erase && 16 * wg + s2 < r) ? b * pa[s2] : 0.f;
 #pragma unroll
             for (int s4 = 0; s4 < 4; ++s4)
                 *reinterpret_cast<float4*>(As + r * LDT + 16 * wg + 4 * s4) =
@@ -572,7 +575,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         const float beta_v = tid >= 128 ? beta_of(cur, tid - 128) : 0.f;
         KDA_WAIT_OR_EXIT(mb_tma, 1u, 0);
         if (tid >= 128)
-            cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v, p.gh, (long long)cur.tok0 * H + cur.h, H);
+            cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v, gh, (long long)cur.tok0 * H + cur.h, H);
         __syncthreads();
         build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)cur.rec * R::BYTES, cur.L, tid, NT, 0, C);
     }
@@ -617,7 +620,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
                 const float beta_v = beta_of(nxt, t);
                 const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
                 if (!bar_or(3, 384, !ok)) {
-                    cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v, p.gh, (long long)nxt.tok0 * H + nxt.h, H);
+                    cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v, gh, (long long)nxt.tok0 * H + nxt.h, H);
                     build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384, 0, C);
                 }
             }
@@ -830,10 +833,11 @@ __device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost,
 // completed: the [Qh ; Kh] tile and V after chunk c's X MMA and Y phase, the
 // Z, PT, e^G_last and beta part after chunk c + 1's X MMA (tcgen05 MMAs of
 // one thread complete in issue order).
-template <typename TO, int DK>
+template <typename TO, int DK, bool VAR>
 __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensorMap& tmo, const ScanParams& p,
                                           int bid)
 {
+    const bool no_erase = VAR && p.no_erase;   // layer variant (VAR instantiations only)
     using PL = ScanPlan<DK>;
     using R = Rec<DK>;
     extern __shared__ unsigned char smem_raw[];
@@ -1031,8 +1035,8 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
                     for (int w = 0; w < 4; ++w) {
                         const float2 f2 = __bfloat1622float2(v2[w]);
                         const int jj = 8 * u + 2 * w;
-                        y[jj] = bs * (f2.x - (p.no_erase ? 0.f : x16[jj]));
-                        y[jj + 1] = bs * (f2.y - (p.no_erase ? 0.f : x16[jj + 1]));
+                        y[jj] = bs * (f2.x - (no_erase ? 0.f : x16[jj]));
+                        y[jj + 1] = bs * (f2.y - (no_erase ? 0.f : x16[jj + 1]));
                     }
                 }
                 st_row_h16(Yb, s, 16 * wg, C, y);
@@ -1122,33 +1126,33 @@ finish:
 }
 #undef KDA_WAIT_OR_EXIT
 
-template <int DK>
+template <int DK, bool VAR>
 __global__ void __launch_bounds__(NT, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmg, const PrepParams p)
 {
-    prep_body<DK>(tmq, tmk, tmg, p, blockIdx.x, gridDim.x);
+    prep_body<DK, VAR>(tmq, tmk, tmg, p, blockIdx.x, gridDim.x);
 }
 
-template <typename TO, int DK>
+template <typename TO, int DK, bool VAR>
 __global__ void __launch_bounds__(NT, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
                   const ScanParams p)
 {
-    scan_body<TO, DK>(tmv, tmo, p, blockIdx.x);
+    scan_body<TO, DK, VAR>(tmv, tmo, p, blockIdx.x);
 }
 
 // Cooperative schedule: CTAs [0, n_scan) scan, the others prep; the scan
 // waits on the records' ready flags, the prep never waits on the scan, and a
 // cooperative launch keeps every CTA resident, so the hand-off cannot stall.
-template <typename TO, int DK>
+template <typename TO, int DK, bool VAR>
 __global__ void __launch_bounds__(NT, 1)
 chunk_coop_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmg, const __grid_constant__ CUtensorMap tmv,
                   const __grid_constant__ CUtensorMap tmo, const PrepParams pp, const ScanParams sp, int n_scan)
 {
-    if ((int)blockIdx.x < n_scan) scan_body<TO, DK>(tmv, tmo, sp, blockIdx.x);
-    else prep_body<DK>(tmq, tmk, tmg, pp, blockIdx.x - n_scan, gridDim.x - n_scan);
+    if ((int)blockIdx.x < n_scan) scan_body<TO, DK, VAR>(tmv, tmo, sp, blockIdx.x);
+    else prep_body<DK, VAR>(tmq, tmk, tmg, pp, blockIdx.x - n_scan, gridDim.x - n_scan);
 }
 
 // ============================================================== host side
@@ -1271,8 +1275,8 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
         !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
         return cudaErrorInvalidValue;
-    auto pk = chunk_prep_kernel<DK>;
-    auto sk = chunk_scan_kernel<TO, DK>;
+    auto pk = mode ? chunk_prep_kernel<DK, true> : chunk_prep_kernel<DK, false>;
+    auto sk = mode ? chunk_scan_kernel<TO, DK, true> : chunk_scan_kernel<TO, DK, false>;
     cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
@@ -1374,7 +1378,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (coop) {
         unsigned* flags = reinterpret_cast<unsigned*>(ws + flag_off);
         err = cudaMemsetAsync(flags, 0, flag_bytes, stream);
-        auto ck = chunk_coop_kernel<TO, DK>;
+        auto ck = mode ? chunk_coop_kernel<TO, DK, true> : chunk_coop_kernel<TO, DK, false>;
         const int smem = std::max(PrepPlan::BYTES, ScanPlan<DK>::BYTES);
         if (err == cudaSuccess) err = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err == cudaSuccess) {
@@ -1492,8 +1496,8 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
         !make_tmap(&tg, log_alpha, tokens, H, DK, true) || !make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
         !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
         return cudaErrorInvalidValue;
-    auto pk = chunk_prep_kernel<DK>;
-    auto sk = chunk_scan_kernel<TO, DK>;
+    auto pk = chunk_prep_kernel<DK, false>;
+    auto sk = chunk_scan_kernel<TO, DK, false>;
     cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
