@@ -245,12 +245,16 @@ __device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t,
 {
     const int ch = t & 127, part = t >> 7;
     const int r0 = 21 * part, nr = part == 2 ? 22 : 21;
+    if (gh) {   // one gate per (token, head): column 0 of the staging holds the chunk's 64 gates
+        if (t < C) gs[t * DK] = t < L ? gh[gbase + (long long)t * H] : 0.f;
+        bar_sync(2, 384);
+    }
     float G[22];
     if (ch < DK) {
 #pragma unroll
         for (int rr = 0; rr < 22; ++rr) {
             const int row = r0 + rr;
-            G[rr] = (rr < nr && row < L) ? (gh ? gh[gbase + (long long)row * H] : gs[row * DK + ch]) : 0.f;
+            G[rr] = (rr < nr && row < L) ? gs[row * DK + (gh ? 0 : ch)] : 0.f;
         }
 #pragma unroll
         for (int rr = 1; rr < 22; ++rr) G[rr] += G[rr - 1];
