@@ -13,7 +13,10 @@ The output o is fp32 by default (``o_dtype=torch.bfloat16`` rounds it to bf16).
 Two variants of the layer are keyword flags of the three calls (the
 ``KDA_MODE_*`` flags of the C ABI): ``head_gate=True`` takes one forget gate per
 (token, head) -- log_alpha without its d_k axis -- and ``erase=False`` drops the
-delta rule's erase term (S_t = Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T).
+delta rule's erase term (S_t = Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T).  Two
+more flags move input pre-processing into the kernels: ``normalize_qk=True``
+divides every q and k row by its L2 norm, and ``gate_logits=True`` reads
+log_alpha as logits z (log alpha = -softplus(z)).
 """
 from __future__ import annotations
 
@@ -31,8 +34,9 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-def _mode(head_gate, erase):
-    return (_lib.KDA_MODE_HEAD_GATE if head_gate else 0) | (0 if erase else _lib.KDA_MODE_NO_ERASE)
+def _mode(head_gate, erase, normalize_qk=False, gate_logits=False):
+    return ((_lib.KDA_MODE_HEAD_GATE if head_gate else 0) | (0 if erase else _lib.KDA_MODE_NO_ERASE)
+            | (_lib.KDA_MODE_NORM_QK if normalize_qk else 0) | (_lib.KDA_MODE_GATE_LOGITS if gate_logits else 0))
 
 
 def _stream(stream):
@@ -54,7 +58,7 @@ def _check(t, name, shape, dtype, device):
 
 def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final_state=None,
                   output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None,
-                  head_gate=False, erase=True):
+                  head_gate=False, erase=True, normalize_qk=False, gate_logits=False):
     """Chunkwise forward over equal-length sequences.
 
     q, k [B, T, H, dk] and v [B, T, H, dv] (bf16 or fp32); beta [B, T, H] and
@@ -62,7 +66,8 @@ def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final
     [B, H, dk, dv] fp32 or None.  Returns (o [B, T, H, dv] in o_dtype (or o's
     dtype when o is given), final_state [B, H, dk, dv] or None)."""
     return _dense_fwd("kda_chunk_fwd", q, k, v, beta, log_alpha, initial_state, o, final_state,
-                      output_final_state, o_dtype, chunk, stream, _mode(head_gate, erase))
+                      output_final_state, o_dtype, chunk, stream,
+                      _mode(head_gate, erase, normalize_qk, gate_logits))
 
 
 def kda_chunk_fwd_noalloc(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final_state=None,
@@ -108,7 +113,7 @@ def _dense_fwd(symbol, q, k, v, beta, log_alpha, initial_state, o, final_state, 
 
 def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, o=None,
                    final_state=None, output_final_state=True, o_dtype=torch.float32, chunk=64,
-                   stream=None, head_gate=False, erase=True):
+                   stream=None, head_gate=False, erase=True, normalize_qk=False, gate_logits=False):
     """Chunkwise forward over N packed variable-length sequences.
 
     q, k [T, H, dk], v [T, H, dv]; beta [T, H]; log_alpha [T, H, dk] ([T, H]
@@ -137,7 +142,7 @@ def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, 
         final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
     if final_state is not None:
         _check(final_state, "final_state", (N, H, dk, dv), torch.float32, dev)
-    mode = _mode(head_gate, erase)
+    mode = _mode(head_gate, erase, normalize_qk, gate_logits)
     _lib.call("kda_varlen_fwd_mode" if mode else "kda_varlen_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
               _ptr(log_alpha), _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(o), _ptr(final_state), T, H, dk,
               dv, chunk, _DTYPES[dt], _DTYPES[o.dtype], *((mode,) if mode else ()), _stream(stream))
@@ -145,7 +150,7 @@ def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, 
 
 
 def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, o_dtype=torch.float32,
-                       stream=None, head_gate=False, erase=True):
+                       stream=None, head_gate=False, erase=True, normalize_qk=False, gate_logits=False):
     """One decode step: q, k [N, H, dk], v [N, H, dv], beta [N, H],
     log_alpha [N, H, dk] ([N, H] with head_gate); state [N, H, dk, dv] fp32 is
     updated in place.  Returns o [N, H, dv]."""
@@ -164,7 +169,7 @@ def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, o_dtype=torch
     _check(o, "o", (N, H, dv), o.dtype, dev)
     if o.dtype not in _DTYPES:
         raise ValueError(f"unsupported output dtype {o.dtype}")
-    mode = _mode(head_gate, erase)
+    mode = _mode(head_gate, erase, normalize_qk, gate_logits)
     _lib.call("kda_recurrent_step_mode" if mode else "kda_recurrent_step", _ptr(q), _ptr(k), _ptr(v),
               _ptr(beta), _ptr(log_alpha), _ptr(state), _ptr(o), N, H, dk, dv, _DTYPES[dt], _DTYPES[o.dtype],
               *((mode,) if mode else ()), _stream(stream))

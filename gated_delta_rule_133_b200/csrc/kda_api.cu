@@ -59,7 +59,10 @@ kda_status run_chunk(const void* q, const void* k, const void* v, const float* b
                                          o_dtype, mode, s));
 }
 
-bool valid_mode(int mode) { return (mode & ~(KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE)) == 0; }
+bool valid_mode(int mode)
+{
+    return (mode & ~(KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE | KDA_MODE_NORM_QK | KDA_MODE_GATE_LOGITS)) == 0;
+}
 
 // Shared checks of the forward entry points.
 kda_status check_fwd(const void* q, const void* k, const void* v, const float* beta,

@@ -106,6 +106,8 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 {
     const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;   // log_alpha [tokens, H]
     const bool erase = (mode & KDA_MODE_NO_ERASE) == 0;
+    const bool logits = (mode & KDA_MODE_GATE_LOGITS) != 0;
+    const bool norm_qk = (mode & KDA_MODE_NORM_QK) != 0;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Smem<DK>& sm = *reinterpret_cast<Smem<DK>*>(smem_raw);
     constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC;
@@ -146,6 +148,7 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                 qv = Elem<TIn>::load(q + off);
                 kv = Elem<TIn>::load(k + off);
                 gv = head_gate ? log_alpha[(size_t)(tok0 + t0 + r) * H + h] : log_alpha[off];
+                if (logits) gv = neg_softplus(gv);
             }
             sm.qm[r * LDK + c] = qv;
             sm.km[r * LDK + c] = kv;
@@ -157,6 +160,17 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
         }
         if (tid < C) sm.beta[tid] = tid < L ? beta[(size_t)(tok0 + t0 + tid) * H + h] : 0.f;
         __syncthreads();
+        if (norm_qk) {   // raw q, k: each row divided by its L2 norm, one warp per row
+            const int lane = tid & 31;
+            for (int rw = tid >> 5; rw < 2 * C; rw += NT / 32) {
+                float* row = (rw < C ? sm.qm : sm.km) + (rw % C) * LDK;
+                float ss = 0.f;
+                for (int c = lane; c < DK; c += 32) ss = fmaf(row[c], row[c], ss);
+                const float inv = inv_norm(warp_sum(ss));
+                for (int c = lane; c < DK; c += 32) row[c] *= inv;
+            }
+            __syncthreads();
+        }
 
         // ---- gate cumsum per channel (fp32, log space) and the factor split
         if (tid < DK) {

@@ -130,6 +130,8 @@ struct PrepParams {
     unsigned* ready;         // cooperative schedule: ready[record] = 1 once the record is complete
     const float* gh;         // one gate per (token, head), [tokens, H] (KDA_MODE_HEAD_GATE), or nullptr
     int no_erase;            // KDA_MODE_NO_ERASE: A = 0, so T = I
+    int norm_qk;             // KDA_MODE_NORM_QK: q, k rows divided by their L2 norms in the build
+    int logits;              // KDA_MODE_GATE_LOGITS: gates are logits z, log alpha = -softplus(z)
 };
 
 struct Item {
@@ -241,12 +243,15 @@ __device__ __forceinline__ Vec vec_at(unsigned char* base, int buf)
 // part 22 rows), and the item's channel vectors.  Named barrier 2.
 template <int DK>
 __device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t, float beta_v,
-                                          const float* gh, long long gbase, int H)
+                                          const float* gh, long long gbase, int H, bool logits)
 {
     const int ch = t & 127, part = t >> 7;
     const int r0 = 21 * part, nr = part == 2 ? 22 : 21;
     if (gh) {   // one gate per (token, head): column 0 of the staging holds the chunk's 64 gates
-        if (t < C) gs[t * DK] = t < L ? gh[gbase + (long long)t * H] : 0.f;
+        if (t < C) {
+            const float z = t < L ? gh[gbase + (long long)t * H] : 0.f;
+            gs[t * DK] = (logits && t < L) ? neg_softplus(z) : z;
+        }
         bar_sync(2, 384);
     }
     float G[22];
@@ -255,6 +260,7 @@ __device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t,
         for (int rr = 0; rr < 22; ++rr) {
             const int row = r0 + rr;
             G[rr] = (rr < nr && row < L) ? gs[row * DK + (gh ? 0 : ch)] : 0.f;
+            if (logits && !gh && rr < nr && row < L) G[rr] = neg_softplus(G[rr]);
         }
 #pragma unroll
         for (int rr = 1; rr < 22; ++rr) G[rr] += G[rr - 1];
@@ -285,7 +291,7 @@ __device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t,
 // Kh = k e^G (fp16) straight into the record.
 template <int DK>
 __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& v, unsigned char* rec, int L, int t,
-                                               int nthr, int row_lo, int row_hi)
+                                               int nthr, int row_lo, int row_hi, bool norm_qk = false)
 {
     using R = Rec<DK>;
     constexpr int NG = DK / 4;
@@ -300,6 +306,18 @@ __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& 
         if (r < L) {
             q4 = bf16x4(x.qs + r * DK + c0);
             k4 = bf16x4(x.ks + r * DK + c0);
+        }
+        if (norm_qk) {   // the NG lanes holding row r are consecutive, and every lane runs the same rows
+            float sq = q4.x * q4.x + q4.y * q4.y + q4.z * q4.z + q4.w * q4.w;
+            float sk = k4.x * k4.x + k4.y * k4.y + k4.z * k4.z + k4.w * k4.w;
+#pragma unroll
+            for (int o = NG / 2; o > 0; o >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                sk += __shfl_xor_sync(0xffffffffu, sk, o);
+            }
+            const float iq = inv_norm(sq), ik = inv_norm(sk);
+            q4 = make_float4(q4.x * iq, q4.y * iq, q4.z * iq, q4.w * iq);
+            k4 = make_float4(k4.x * ik, k4.y * ik, k4.z * ik, k4.w * ik);
         }
         const float e0 = __expf(fminf(fmaxf(g4.x - m4.x, -80.f), 80.f));
         const float e1 = __expf(fminf(fmaxf(g4.y - m4.y, -80.f), 80.f));
@@ -461,6 +479,8 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     // layer variants (VAR instantiations only; the plain layer compiles without them)
     const float* const gh = VAR ? p.gh : nullptr;
     const bool no_erase = VAR && p.no_erase;
+    const bool norm_qk = VAR && p.norm_qk;
+    const bool logits = VAR && p.logits;
     using PL = PrepPlan;
     using R = Rec<DK>;
     extern __shared__ unsigned char smem_raw[];
@@ -579,9 +599,9 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         const float beta_v = tid >= 128 ? beta_of(cur, tid - 128) : 0.f;
         KDA_WAIT_OR_EXIT(mb_tma, 1u, 0);
         if (tid >= 128)
-            cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v, gh, (long long)cur.tok0 * H + cur.h, H);
+            cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v, gh, (long long)cur.tok0 * H + cur.h, H, logits);
         __syncthreads();
-        build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)cur.rec * R::BYTES, cur.L, tid, NT, 0, C);
+        build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)cur.rec * R::BYTES, cur.L, tid, NT, 0, C, norm_qk);
     }
     fence_proxy_async();
     tc_fence_before();
@@ -624,8 +644,8 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
                 const float beta_v = beta_of(nxt, t);
                 const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
                 if (!bar_or(3, 384, !ok)) {
-                    cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v, gh, (long long)nxt.tok0 * H + nxt.h, H);
-                    build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384, 0, C);
+                    cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v, gh, (long long)nxt.tok0 * H + nxt.h, H, logits);
+                    build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384, 0, C, norm_qk);
                 }
             }
         }
@@ -1335,6 +1355,8 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     pp.timeout_cycles = timeout_cycles;
     pp.gh = head_gate ? log_alpha : nullptr;
     pp.no_erase = (mode & KDA_MODE_NO_ERASE) ? 1 : 0;
+    pp.norm_qk = (mode & KDA_MODE_NORM_QK) ? 1 : 0;
+    pp.logits = (mode & KDA_MODE_GATE_LOGITS) ? 1 : 0;
     ScanParams sp{};
     sp.no_erase = pp.no_erase;
     sp.v = static_cast<const __nv_bfloat16*>(v);

@@ -38,4 +38,11 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// log alpha from a gate logit z (KDA_MODE_GATE_LOGITS): -softplus(z) =
+// -(max(z, 0) + log(1 + e^-|z|)), without overflow for any finite z.
+__device__ __forceinline__ float neg_softplus(float z) { return -(fmaxf(z, 0.f) + log1pf(expf(-fabsf(z)))); }
+
+// 1 / max(||x||, 1e-15) from ||x||^2 (KDA_MODE_NORM_QK; rows of zero norm stay zero).
+__device__ __forceinline__ float inv_norm(float sq) { return rsqrtf(fmaxf(sq, 1e-30f)); }
+
 }  // namespace kda

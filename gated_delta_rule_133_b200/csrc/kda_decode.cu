@@ -25,6 +25,8 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 {
     const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;   // log_alpha [NH]: one gate per head
     const bool erase = (mode & KDA_MODE_NO_ERASE) == 0;
+    const bool logits = (mode & KDA_MODE_GATE_LOGITS) != 0;
+    const bool norm_qk = (mode & KDA_MODE_NORM_QK) != 0;
     constexpr int COLS = 64;
     constexpr int SPLIT = DV / COLS;
     constexpr int RPT = DK / 16;          // key rows per thread
@@ -46,9 +48,23 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     for (int i = t; i < DK; i += 256) {
         sk[i] = Elem<T>::load(k + (size_t)head * DK + i);
         sq[i] = Elem<T>::load(q + (size_t)head * DK + i);
-        sa[i] = expf(head_gate ? log_alpha[head] : log_alpha[(size_t)head * DK + i]);
+        const float g = head_gate ? log_alpha[head] : log_alpha[(size_t)head * DK + i];
+        sa[i] = logits ? 1.f / (1.f + expf(g)) : expf(g);   // sigmoid(-z) = exp(-softplus(z))
     }
     __syncthreads();
+    if (norm_qk) {   // raw q, k: divide each by its L2 norm
+        __shared__ float s_inv[2];
+        if (w == 0) {
+            float nk = 0.f, nq = 0.f;
+            for (int i = lane; i < DK; i += 32) { nk = fmaf(sk[i], sk[i], nk); nq = fmaf(sq[i], sq[i], nq); }
+            nk = warp_sum(nk);
+            nq = warp_sum(nq);
+            if (lane == 0) { s_inv[0] = inv_norm(nk); s_inv[1] = inv_norm(nq); }
+        }
+        __syncthreads();
+        for (int i = t; i < DK; i += 256) { sk[i] *= s_inv[0]; sq[i] *= s_inv[1]; }
+        __syncthreads();
+    }
 
     float r[4] = {0.f, 0.f, 0.f, 0.f}, y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

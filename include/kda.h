@@ -164,11 +164,22 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
  *      the element-wise gate without the delta rule (beta_t = 1 gives the
  *      section's form; per-channel decay of the key rows as in this layer).
  *
+ * Two more flags move the inputs' pre-processing into the kernels (the pages
+ * give unit-norm q, k and a gate from a sigmoid of a projection: section 3.4
+ * of the same page):
+ *
+ *  KDA_MODE_NORM_QK      q and k are raw: every (token, head) row of q and of k
+ *      is divided by its L2 norm (rows of norm below 1e-15 count as zero).
+ *  KDA_MODE_GATE_LOGITS  log_alpha holds gate logits z: the layer uses
+ *      log alpha = -softplus(z), i.e. alpha = sigmoid(-z).
+ *
  * The flags combine.  Every other argument, layout and rule is that of the
  * plain entry point of the same name.
  */
 #define KDA_MODE_HEAD_GATE 1
 #define KDA_MODE_NO_ERASE 2
+#define KDA_MODE_NORM_QK 4
+#define KDA_MODE_GATE_LOGITS 8
 
 kda_status kda_chunk_fwd_mode(const void* q, const void* k, const void* v,
                               const float* beta, const float* log_alpha,

@@ -113,7 +113,7 @@ def test_mode_validation():
     needs only 4-byte alignment, a per-channel one 16 bytes."""
     lib = _lib.load()
     base = (P, P, P, P, P, None, P, None, 1, 8, 2, 128, 128, 64, 1, 0)
-    assert lib.kda_chunk_fwd_mode(*base, 4, None) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_fwd_mode(*base, 16, None) == _lib.KDA_ERR_INVALID_ARG
     assert lib.kda_chunk_fwd_mode(*base, -1, None) == _lib.KDA_ERR_INVALID_ARG
     gate4 = base[:4] + (P + 4,) + base[5:]
     assert lib.kda_chunk_fwd_mode(*gate4, _lib.KDA_MODE_NO_ERASE, None) == _lib.KDA_ERR_INVALID_ARG
@@ -121,8 +121,8 @@ def test_mode_validation():
     gate4_d96 = gate4[:11] + (96,) + gate4[12:]
     assert lib.kda_chunk_fwd_mode(*gate4_d96, _lib.KDA_MODE_HEAD_GATE, None) == _lib.KDA_ERR_UNSUPPORTED
     v = lib.kda_varlen_fwd_mode
-    assert v(P, P, P, P, P, P, 1, None, P, None, 8, 2, 128, 128, 64, 1, 0, 8, None) == _lib.KDA_ERR_INVALID_ARG
+    assert v(P, P, P, P, P, P, 1, None, P, None, 8, 2, 128, 128, 64, 1, 0, 32, None) == _lib.KDA_ERR_INVALID_ARG
     r = lib.kda_recurrent_step_mode
-    assert r(P, P, P, P, P, P, P, 3, 2, 128, 128, 1, 0, 4, None) == _lib.KDA_ERR_INVALID_ARG
+    assert r(P, P, P, P, P, P, P, 3, 2, 128, 128, 1, 0, 16, None) == _lib.KDA_ERR_INVALID_ARG
     assert r(P, P, P, P, P + 4, P, P, 3, 2, 128, 128, 1, 0, 0, None) == _lib.KDA_ERR_INVALID_ARG
     assert r(P, P, P, P, P + 4, P, P, 3, 2, 96, 128, 1, 0, _lib.KDA_MODE_HEAD_GATE, None) == _lib.KDA_ERR_UNSUPPORTED
