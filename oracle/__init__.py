@@ -11,7 +11,10 @@ of the method's arithmetic.
 LLM Training and Inference More Efficient" section 3.3 and "Demystifying Hybrid
 LLM Architectures" section 2.3 (read-out after the write).  ``forms`` holds
 independent restatements (closed forms, brute force, the chunkwise algebra)
-that pin it.
+that pin it.  ``backward`` holds the reverse-mode gradients of the same
+recurrence in fp64 (the reference for a backward pass), pinned by finite
+differences of ``recurrence`` and by the closed-form gradients of causal
+linear attention.
 """
 from __future__ import annotations
 
