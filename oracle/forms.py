@@ -136,3 +136,82 @@ def chunkwise(q, k, v, beta, log_alpha, s0, C):
         o[c0:c1] = (np.exp(G) * Q) @ S + P @ Vp
         S = np.exp(G[-1])[:, None] * S + (np.exp(G[-1][None, :] - G) * K).T @ Vp
     return o, S
+
+
+def chunkwise_backward(q, k, v, beta, log_alpha, s0, do, dsT, C):
+    """Gradients of L = sum(o * do) + sum(S_T * dsT) through the chunkwise
+    algorithm of ``chunkwise`` (fp64, one (sequence, head)): the adjoint of
+    each chunk's map, a reverse scan over chunks carrying dS.  Per chunk, with
+    E = exp(G), gamma = exp(G_last), Qh = E * Q, Kh = E * K, Kn = K / E,
+    Kl = gamma * Kn, A = beta strictly-lower(Kh Kn^T), P = lower-incl(Qh Kn^T),
+    T = (I + A)^-1, Y = beta (V - Kh S), U = T Y:
+      O = Qh S + P U,   S_next = Diag(gamma) S + Kl^T U.
+    Returns (dq, dk, dv, dbeta, dlog_alpha, ds0); the same quantities as
+    ``oracle.backward.recurrence_backward`` by a different route."""
+    T = q.shape[0]
+    dk_, dv_ = q.shape[1], v.shape[1]
+    starts = list(range(0, T, C))
+    S = np.array(s0, dtype=np.float64)
+    states = []
+    for c0 in starts:                                   # forward: the state entering each chunk
+        states.append(S)
+        c1 = min(T, c0 + C)
+        G = np.cumsum(log_alpha[c0:c1], axis=0)
+        E, gam = np.exp(G), np.exp(G[-1])
+        L = c1 - c0
+        Kh, Kn = k[c0:c1] * E, k[c0:c1] / E
+        A = beta[c0:c1, None] * np.tril(Kh @ Kn.T, -1)
+        U = np.linalg.inv(np.eye(L) + A) @ (beta[c0:c1, None] * (v[c0:c1] - Kh @ S))
+        S = gam[:, None] * S + (gam[None, :] * Kn).T @ U
+    grads = [np.zeros_like(q), np.zeros_like(k), np.zeros_like(v), np.zeros_like(beta), np.zeros_like(log_alpha)]
+    gq, gk, gv, gb, gg = grads
+    dS = np.zeros((dk_, dv_)) if dsT is None else np.array(dsT, dtype=np.float64)
+    for ci in range(len(starts) - 1, -1, -1):
+        c0 = starts[ci]
+        c1 = min(T, c0 + C)
+        L = c1 - c0
+        S = states[ci]
+        Q, K, V, b, dO = q[c0:c1], k[c0:c1], v[c0:c1], beta[c0:c1], do[c0:c1]
+        G = np.cumsum(log_alpha[c0:c1], axis=0)
+        E, En, gam = np.exp(G), np.exp(-G), np.exp(G[-1])
+        Qh, Kh, Kn = Q * E, K * E, K * En
+        Kl = Kn * gam[None, :]
+        low, strict = np.tril(np.ones((L, L))), np.tril(np.ones((L, L)), -1)
+        MA, MP = Kh @ Kn.T, Qh @ Kn.T
+        A, P = b[:, None] * MA * strict, MP * low
+        Tm = np.linalg.inv(np.eye(L) + A)
+        X = Kh @ S
+        Y = b[:, None] * (V - X)
+        U = Tm @ Y
+        dSn = dS
+        # adjoint of O = Qh S + P U and S_next = Diag(gamma) S + Kl^T U
+        dU = P.T @ dO + Kl @ dSn
+        dP = (dO @ U.T) * low
+        dKl = U @ dSn.T
+        dgam = np.sum(dSn * S, axis=1)
+        dS = gam[:, None] * dSn + Qh.T @ dO
+        dQh = dO @ S.T
+        # U = T Y,  Y = beta (V - Kh S)
+        dY = Tm.T @ dU
+        dTm = dU @ Y.T
+        gv[c0:c1] = b[:, None] * dY
+        dX = -b[:, None] * dY
+        db = np.sum((V - X) * dY, axis=1)
+        dKh = dX @ S.T
+        dS = dS + Kh.T @ dX
+        # T = (I + A)^-1,  A = beta strictly-lower(Kh Kn^T),  P = lower-incl(Qh Kn^T)
+        dA = -(Tm.T @ dTm @ Tm.T) * strict
+        db += np.sum(MA * strict * dA, axis=1)
+        dMA = b[:, None] * dA
+        dKh += dMA @ Kn
+        dKn = dMA.T @ Kh + dP.T @ Qh + dKl * gam[None, :]
+        dQh += dP @ Kn
+        dgam += np.sum(dKl * Kn, axis=0)
+        # Qh = E Q, Kh = E K, Kn = K / E, gamma = E[-1]; G = cumsum(log alpha)
+        gq[c0:c1] = dQh * E
+        gk[c0:c1] = dKh * E + dKn * En
+        dG = dQh * Qh + dKh * Kh - dKn * Kn
+        dG[-1] += dgam * gam
+        gg[c0:c1] = np.cumsum(dG[::-1], axis=0)[::-1]
+        gb[c0:c1] = db
+    return gq, gk, gv, gb, gg, dS

@@ -7,6 +7,10 @@
 - Causal linear attention (alpha = 1, no erase) has closed-form gradients of
   the scores-times-values form of "Hybrid Linear Attention Architecture: ...",
   section 3.1.
+- The adjoint of the chunkwise algorithm (``oracle.forms.chunkwise_backward``:
+  a reverse scan over chunks carrying dS plus per-chunk local gradients, the
+  blueprint of a backward pass) equals the token-level gradients for chunk
+  sizes 1, 3, 4 and 16 with a ragged last chunk.
 """
 import numpy as np
 import pytest
@@ -81,3 +85,24 @@ def test_linear_attention_closed_form_gradients():
     for name in ("q", "k", "v", "beta"):
         assert np.allclose(got[name][:, 0], want[name], rtol=1e-12, atol=1e-12), name
     assert np.allclose(got["s0"][0, 0], want["s0"], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("C", [1, 3, 4, 16])
+def test_chunkwise_backward_matches_token_backward(C):
+    """The chunk algebra's adjoint (a reverse scan over chunks plus per-chunk
+    local gradients) gives the token recurrence's gradients, ragged last chunk
+    included."""
+    from oracle.forms import chunkwise_backward
+    rng = np.random.default_rng(7 + C)
+    T, dk, dv = 11, 4, 3
+    q, k, v = rng.standard_normal((T, dk)), rng.standard_normal((T, dk)) * 0.6, rng.standard_normal((T, dv))
+    beta = rng.uniform(0.1, 0.9, T)
+    la = -rng.uniform(0.02, 0.3, (T, dk))
+    s0 = rng.standard_normal((dk, dv))
+    do, dsT = rng.standard_normal((T, dv)), rng.standard_normal((dk, dv))
+    want = recurrence_backward(q[:, None], k[:, None], v[:, None], beta[:, None], la[:, None], None,
+                               s0[None, None], do[:, None], dsT[None, None])
+    got = chunkwise_backward(q, k, v, beta, la, s0, do, dsT, C)
+    for name, w, g in zip(("q", "k", "v", "beta", "log_alpha"), want[:5], got[:5]):
+        assert np.allclose(g, w[:, 0], rtol=1e-10, atol=1e-10), name
+    assert np.allclose(got[5], want[5][0, 0], rtol=1e-10, atol=1e-10)
