@@ -2,12 +2,13 @@
 """Benchmark of the KDA layer on B200.
 
 One step = one chunkwise forward (gate cumsum, intra-chunk A, UT transform,
-state scan, intra-chunk output, final state) over the prefill workload
-(B=2, H=16, T=4096, d_k=d_v=128, bf16 q/k/v, fp32 state, chunk 64), inputs
-resident in HBM.  Two input sets of ~200 MB each (larger than the 126 MB L2)
-alternate between steps, so no step starts with its inputs in L2.  The decode
-step (256 sequences x 32 heads, 64 consecutive tokens) is timed in the same
-run and reported under "decode".
+state scan, intra-chunk output, final state) over the long-context workload
+(B=1, H=32, T=131072, d_k=d_v=128, bf16 q/k/v, fp32 state, chunk 64; the
+largest single-GPU configuration), inputs resident in HBM (5.4 GB, far larger
+than the 126 MB L2).  The prefill (B=2, H=16, T=4096) and packed variable-length
+(8 sequences, 65536 tokens, H=32) forwards, the layer variants and the decode
+step (256 sequences x 32 heads, 64 consecutive tokens) are timed in the same
+run and reported under "other_workloads" and "decode".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -40,9 +41,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ----------------------------------------------------------------------------- work model
-def bytes_per_token_head(dk, dv, elem, o_elem=4):
+def bytes_per_token_head(dk, dv, elem, o_elem=2):
     """Algorithmic HBM bytes per (token, head): q, k, v in (elem bytes each),
-    o out (o_elem bytes), log alpha (fp32 per key channel) and beta (fp32) in."""
+    o out (o_elem bytes), log alpha (fp32 per key channel) and beta (fp32) in.
+    With bf16 q/k/v/o and d = 128 this is the 1540 B of the roofline; the
+    library's default fp32 o adds 2 d_v bytes (1796 B)."""
     return elem * (2 * dk + dv) + o_elem * dv + 4 * dk + 4
 
 
@@ -53,7 +56,7 @@ def flops_per_token_head(dk, dv, C=64):
     return (2 * (C - 1) + (C + 1)) * dk + 2 * C * dv + 6 * dk * dv + C * C / 3.0
 
 
-def chunk_work(B, T, H, dk, dv, elem=2, o_elem=4, state_in=True, state_out=True):
+def chunk_work(B, T, H, dk, dv, elem=2, o_elem=2, state_in=True, state_out=True):
     th = B * T * H
     nbytes = th * bytes_per_token_head(dk, dv, elem, o_elem)
     nbytes += (int(state_in) + int(state_out)) * B * H * dk * dv * 4
@@ -163,6 +166,7 @@ def peaks():
 KERNEL_SOURCES = {
     # the files whose code a recorded ncu capture of each path depends on
     "chunk_fwd_prefill": ["kda_chunk_split.cu", "kda_tc_util.cuh", "kda_sm100.cuh", "kda_common.cuh"],
+    "chunk_fwd_long": ["kda_chunk_split.cu", "kda_tc_util.cuh", "kda_sm100.cuh", "kda_common.cuh"],
     "decode_step": ["kda_decode.cu", "kda_common.cuh"],
 }
 
@@ -189,28 +193,39 @@ def recorded_traffic(kernel_key):
     return rec.get("dram_bytes_per_launch")
 
 
-def chunk_launches(B, T, H, dv, device):
-    """Kernels one dense chunk-forward call launches (the library's own rule):
-    one cooperative kernel (prep and scan CTAs together) when the scan grid
-    leaves at least 32 SMs; otherwise a prep and a scan kernel per block of
-    chunks, one block per 32 chunks (at most 8) when the scan grid leaves 32 SMs
-    (KDA_SCAN_BLOCKS / KDA_CHUNK_SCHEDULE override)."""
-    kind = os.environ.get("KDA_CHUNK_KERNEL", "")
-    if kind in ("fused", "simt") or os.environ.get("KDA_FORCE_SIMT") == "1":
-        return 1
-    nch = (T + 63) // 64
+def chunk_launches(B, T, H, dv, device, varlen=False):
+    """Kernels one chunk-forward call launches (the library's rule): dense
+    inputs whose scan grid (B * H * dv / 64 CTAs) leaves at least 32 SMs run as
+    one cooperative kernel (prep and scan CTAs together); otherwise a prep and
+    a scan kernel, plus the index kernel of a packed batch."""
     nsm = torch.cuda.get_device_properties(device).multi_processor_count
-    room = B * H * (dv // 64) + 32 <= nsm
-    sched = os.environ.get("KDA_CHUNK_SCHEDULE")
-    env = int(os.environ.get("KDA_SCAN_BLOCKS", "0") or 0)
-    if room and not env and (sched is None or sched == "coop"):
+    if not varlen and B * H * (dv // 64) + 32 <= nsm:
         return 1
-    nb = env if env > 0 else (nch // 32 if room else 1)
-    return 2 * max(1, min(nb, nch, 8))
+    return 3 if varlen else 2
 
 
 def event_pairs(n):
     return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+
+
+def chunk_roofline(nbytes, nbytes_f32o, nflops, launch_s, traffic=None):
+    """Roofline of one chunk-forward call: algorithmic bytes (bf16 o, the
+    survey's count) over the call's CUDA-event time, against the measured copy
+    bandwidth; the fp32-o byte count (what the default call writes) beside it."""
+    pk, kind = peaks()
+    achieved = nbytes / launch_s / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "peak_kind": f"{kind} copy bandwidth",
+            "bytes_per_launch": nbytes, "launch_ms": launch_s * 1e3,
+            "fp32_o": {"bytes_per_launch": nbytes_f32o, "achieved": nbytes_f32o / launch_s / 1e9,
+                       "frac": nbytes_f32o / launch_s / 1e9 / pk["hbm_gbs"]},
+            "tensor_frac": nflops / launch_s / 1e12 / pk["bf16_tflops"]}
+
+
+def dense_work(w, state_in):
+    nbytes, nflops = chunk_work(w.B, w.T, w.H, w.dk, w.dv, state_in=state_in)
+    nbytes_f32o, _ = chunk_work(w.B, w.T, w.H, w.dk, w.dv, o_elem=4, state_in=state_in)
+    return nbytes, nbytes_f32o, nflops
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -221,20 +236,19 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     init_dist(world, "nccl")
-    w = WORKLOADS["prefill"]
+    w = WORKLOADS["long"]
     stream = torch.cuda.current_stream(device)
 
-    nsets = 2
-    sets = [make_inputs(w, device, seed=w.seed + 1000 * rank + i) for i in range(nsets)]
-    outs = [(torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32, device=device),
-             torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)) for _ in range(nsets)]
-    nbytes, nflops = chunk_work(w.B, w.T, w.H, w.dk, w.dv)
-    set_bytes = sum(t.numel() * t.element_size() for t in sets[0].values() if t is not None)
+    d = make_inputs(w, device, seed=w.seed + 1000 * rank)
+    o = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32, device=device)
+    sN = torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
+    ws = torch.empty(kda.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv), dtype=torch.uint8, device=device)
+    nbytes, nbytes_f32o, nflops = dense_work(w, state_in=d["initial_state"] is not None)
+    set_bytes = sum(t.numel() * t.element_size() for t in d.values() if t is not None)
 
     def step(i):
-        d, (o, s) = sets[i % nsets], outs[i % nsets]
         kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], d["initial_state"],
-                          o=o, final_state=s, stream=stream)
+                          o=o, final_state=sN, workspace=ws, stream=stream)
 
     sampler = ClockSampler(device.index)
     with sampler:
@@ -259,35 +273,36 @@ def run_ours(args, world, rank, local):
         elapsed = reduce_max(t_start.elapsed_time(t_end) / 1e3, world, device)
         launch_s = statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3
 
-        # ---- decode: 64 consecutive steps over 256 x 32 fp32 states
-        dec = run_decode(kda, device, stream, world, rank, max(1, args.warmup))
-
-        # ---- the other two chunk-forward workloads, timed once each (context)
-        others = {} if args.skip_others else run_other_workloads(kda, device, stream, world, rank)
-
         # ---- end to end through the public API from pinned host buffers
-        e2e = run_e2e(kda, sets[0], w, device, stream, world, steps=max(2, min(args.steps, 10)))
+        host = {k: (None if v is None else v.cpu()) for k, v in d.items()}
+        del d, o, sN
+        torch.cuda.empty_cache()
+        e2e = run_e2e(kda, host, w, device, stream, world, ws, steps=max(3, min(args.steps, 10)))
+        del host, ws
+        torch.cuda.empty_cache()
+
+        # ---- decode: 64 consecutive steps over 256 x 32 fp32 states
+        dec = run_decode(kda, device, stream, world, rank, max(3, args.warmup))
+
+        # ---- the other chunk-forward workloads (context)
+        others = {} if args.skip_others else run_other_workloads(kda, device, stream, world, rank,
+                                                                 reps=max(3, min(args.steps, 20)))
 
     clocks = sampler.summary()
     tokens = w.B * w.T * world
     value = tokens * args.steps / elapsed
-    pk, pk_kind = peaks()
-    achieved = nbytes / launch_s / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"prefill: B={w.B} H={w.H} T={w.T} d_k={w.dk} d_v={w.dv} chunk={w.chunk}, "
-                               "bf16 q/k/v, fp32 state and fp32 output, random fp32 initial state",
+        "config": {"workload": f"long context: B={w.B} H={w.H} T={w.T} d_k={w.dk} d_v={w.dv} chunk={w.chunk}, "
+                               "bf16 q/k/v, fp32 state and fp32 output, log alpha = -softplus(z), z ~ N(-1, 1), "
+                               "zero initial state",
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: {nsets} input sets of {set_bytes / 1e6:.0f} MB alternate"},
+                   "l2": f"inputs larger than L2: one input set of {set_bytes / 1e9:.1f} GB"},
         "tflops": nflops * world * args.steps / elapsed / 1e12,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic("chunk_fwd_prefill"),
-                     "peak_kind": f"{pk_kind} copy bandwidth",
-                     "bytes_per_launch": nbytes, "launch_ms": launch_s * 1e3,
-                     "tensor_frac": nflops / launch_s / 1e12 / pk["bf16_tflops"]},
+        "roofline": chunk_roofline(nbytes, nbytes_f32o, nflops, launch_s, recorded_traffic("chunk_fwd_long")),
         "decode": dec,
         "other_workloads": others,
         "e2e": e2e,
@@ -335,44 +350,48 @@ def run_decode(kda, device, stream, world, rank, warmup):
             "gpu_launches": w.T}
 
 
-def run_other_workloads(kda, device, stream, world, rank, reps=3):
-    """Varlen (8 packed sequences, 65536 tokens, H32) and long-context (T131072,
+def run_other_workloads(kda, device, stream, world, rank, reps=20):
+    """The prefill (B2 H16 T4096) and varlen (8 packed sequences, 65536 tokens,
     H32) chunk forwards, and the prefill shape with the two layer variants (one
     gate per head; no erase term): one warm-up launch, `reps` timed launches
-    each."""
+    each, inputs resident in HBM."""
     from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
-    pk, kind = peaks()
     out = {}
-    for name in ("varlen", "long", "prefill_head_gate", "prefill_no_erase"):
+    for name in ("prefill", "varlen", "prefill_head_gate", "prefill_no_erase"):
         w = WORKLOADS[name.split("_")[0]]
         d = make_inputs(w, device, seed=w.seed + 1000 * rank)
-        gate_bytes = 4 * w.dk
         desc = f"{name}: {w.B * w.T if w.kind != 'varlen' else w.T} tokens, H={w.H}, d_k=d_v={w.dk}, bf16 q/k/v, fp32 o and state"
+        kw = {}
+        gate_bytes = 4 * w.dk
         if name.startswith("prefill"):
-            head_gate, erase = name == "prefill_head_gate", name != "prefill_no_erase"
-            if head_gate:
+            if name == "prefill_head_gate":
                 d["log_alpha"] = d["log_alpha"][..., 0].contiguous()
+                kw["head_gate"] = True
                 gate_bytes = 4
+                desc += ", one forget gate per (token, head)"
+            if name == "prefill_no_erase":
+                kw["erase"] = False
+                desc += ", no erase term"
             o = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32, device=device)
             sN = torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
+            mode = (1 if kw.get("head_gate") else 0) | (0 if kw.get("erase", True) else 2)
+            ws = torch.empty(kda.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, mode=mode), dtype=torch.uint8,
+                             device=device)
             call = lambda: kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], d["initial_state"],
-                                             o=o, final_state=sN, stream=stream, head_gate=head_gate, erase=erase)
-            tokens, states = w.B * w.T, 2 * w.B
-            desc += ", " + ("one forget gate per (token, head)" if head_gate else "no erase term")
-        elif name == "varlen":
+                                             o=o, final_state=sN, stream=stream, workspace=ws, **kw)
+            tokens, s_in, s_out = w.B * w.T, w.B, w.B
+            launches = chunk_launches(w.B, w.T, w.H, w.dv, device)
+        else:
             cu = d["cu_seqlens"]
             nseq = cu.numel() - 1
             o = torch.empty(w.T, w.H, w.dv, dtype=torch.float32, device=device)
             sN = torch.empty(nseq, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
+            ws = torch.empty(kda.varlen_fwd_workspace_size(nseq, w.T, w.H, w.dk, w.dv), dtype=torch.uint8,
+                             device=device)
             call = lambda: kda.kda_varlen_fwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], cu, None,
-                                              o=o, final_state=sN, stream=stream)
-            tokens, states = w.T, nseq
-        else:
-            o = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32, device=device)
-            sN = torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
-            call = lambda: kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], None,
-                                             o=o, final_state=sN, stream=stream)
-            tokens, states = w.B * w.T, w.B
+                                              o=o, final_state=sN, stream=stream, workspace=ws)
+            tokens, s_in, s_out = w.T, 0, nseq
+            launches = chunk_launches(1, w.T, w.H, w.dv, device, varlen=True)
         call()
         torch.cuda.synchronize(device)
         ev = event_pairs(reps)
@@ -384,31 +403,34 @@ def run_other_workloads(kda, device, stream, world, rank, reps=3):
         torch.cuda.synchronize(device)
         kda.kda_check()
         t = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3, world, device)
-        nbytes = (tokens * w.H * (bytes_per_token_head(w.dk, w.dv, 2, 4) - 4 * w.dk + gate_bytes)
-                  + states * w.H * w.dk * w.dv * 4)
+        per_th = lambda o_elem: bytes_per_token_head(w.dk, w.dv, 2, o_elem) - 4 * w.dk + gate_bytes
+        states = (s_in + s_out) * w.H * w.dk * w.dv * 4
+        nbytes = tokens * w.H * per_th(2) + states
+        nbytes_f32o = tokens * w.H * per_th(4) + states
+        nflops = tokens * w.H * flops_per_token_head(w.dk, w.dv)
         out[name] = {"workload": desc, "ms": t * 1e3, "tokens_per_s": tokens * world / t,
-                     "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                  "frac": nbytes / t / 1e9 / pk["hbm_gbs"], "peak_kind": f"{kind} copy bandwidth",
-                                  "bytes_per_launch": nbytes}}
-        if not name.startswith("prefill"):   # the layer's FLOPs (the variants do less arithmetic)
-            out[name]["tflops"] = tokens * w.H * flops_per_token_head(w.dk, w.dv) * world / t / 1e12
-        del d, o, sN
+                     "roofline": chunk_roofline(nbytes, nbytes_f32o, nflops, t,
+                                                recorded_traffic("chunk_fwd_prefill") if name == "prefill" else None),
+                     "gpu_launches_per_call": launches}
+        if not name.startswith("prefill_"):   # the layer's FLOPs (the variants do less arithmetic)
+            out[name]["tflops"] = nflops * world / t / 1e12
+        del d, o, sN, ws
         torch.cuda.empty_cache()
     return out
 
 
-def run_e2e(kda, d, w, device, stream, world, steps):
+def run_e2e(kda, host_inputs, w, device, stream, world, ws, steps):
     """Same metric through the public API with pinned host buffers, as a
     pipelined loop over steps: every step copies its inputs host->device on a
     copy-in stream, runs the chunk forward on the compute stream and reads o
     and the final state back on a copy-out stream; two buffer sets let step
     i + 1's inputs travel while step i computes and its results return (PCIe
     is full duplex).  Events order each buffer set's reuse."""
-    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in d.items()}
+    host = {k: (None if v is None else v.pin_memory()) for k, v in host_inputs.items()}
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
     sets = []
     for _ in range(2):
-        dev = {k: (None if v is None else torch.empty_like(v, device=device)) for k, v in d.items()}
+        dev = {k: (None if v is None else torch.empty_like(v, device=device)) for k, v in host.items()}
         o_d = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32, device=device)
         s_d = torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
         o_h = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.float32).pin_memory()
@@ -436,7 +458,7 @@ def run_e2e(kda, d, w, device, stream, world, steps):
         if done_out[j] is not None:
             stream.wait_event(done_out[j])
         kda.kda_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_alpha"], dev["initial_state"],
-                          o=o_d, final_state=s_d, stream=stream)
+                          o=o_d, final_state=s_d, workspace=ws, stream=stream)
         e_c = ev()
         e_c.record(stream)
         done_compute[j] = e_c
@@ -466,31 +488,33 @@ def run_e2e(kda, d, w, device, stream, world, steps):
 
 
 # ----------------------------------------------------------------------------- oracle arm
+ORACLE_SAMPLE_TOKENS = 8192
+
+
 def oracle_sample(heads_max=16):
-    """Times the fp64 oracle on the prefill workload (all tokens of both
-    sequences for up to `heads_max` heads; all 16 by default, about 1 s on 8
-    cores).  Returns the equivalent whole-workload tokens/s, the threads used
-    and the sample description."""
-    import numpy as np
+    """Times the fp64 oracle on a bounded sample of the long-context workload:
+    up to `heads_max` heads (one thread each, at most the host's cores) of one
+    sequence of ORACLE_SAMPLE_TOKENS tokens drawn with the workload's recipe.
+    The recurrence costs the same per token, so the rate scales to the whole
+    workload (131072 tokens x 32 heads).  Returns its tokens/s, the threads
+    used and the sample description."""
     import oracle
-    from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
-    w = WORKLOADS["prefill"]
-    d = make_inputs(w, "cpu")
+    from gated_delta_rule_133_b200.inputs import WORKLOADS, draw_tokens
+    w = WORKLOADS["long"]
     cores = os.cpu_count() or 1
-    heads = max(1, min(heads_max, w.H))
-    f = lambda x: x[:, :, :heads].to(torch.float64).numpy().reshape(w.B * w.T, heads, *x.shape[3:])
-    q, k, v, la = f(d["q"]), f(d["k"]), f(d["v"]), f(d["log_alpha"])
-    beta = d["beta"][:, :, :heads].to(torch.float64).numpy().reshape(w.B * w.T, heads)
-    s0 = d["initial_state"][:, :heads].to(torch.float64).numpy()
-    cu = np.array([0, w.T, 2 * w.T])
+    heads = max(1, min(heads_max, w.H, cores))
+    T = ORACLE_SAMPLE_TOKENS
+    d = draw_tokens(T, heads, w.dk, w.dv, w.dtype, w.gate_mu, w.seed, "cpu")
+    f = lambda x: x.to(torch.float64).numpy()
+    import numpy as np
     t0 = time.perf_counter()
-    oracle.recurrence(q, k, v, beta, la, cu, s0, nthreads=cores)
+    oracle.recurrence(f(d["q"]), f(d["k"]), f(d["v"]), f(d["beta"]), f(d["log_alpha"]), np.array([0, T]), None,
+                      nthreads=heads)
     dt = time.perf_counter() - t0
-    full_time = dt * w.H / heads
-    return {"value": w.B * w.T / full_time, "unit": "tokens/s", "cores": min(cores, w.B * heads),
-            "kind": "oracle",
-            "sample": f"prefill workload, {heads} of {w.H} heads x both sequences x all {w.T} tokens "
-                      f"({dt:.1f} s), scaled to all heads"}
+    full_time = dt * (w.T / T) * (w.H / heads)
+    return {"value": w.B * w.T / full_time, "unit": "tokens/s", "cores": heads, "kind": "oracle",
+            "sample": f"long-context recipe, {heads} heads x {T} tokens ({dt:.2f} s, {heads} threads), "
+                      f"scaled to {w.H} heads x {w.T} tokens"}
 
 
 def run_reference(args, world, rank):
@@ -504,12 +528,16 @@ def run_reference(args, world, rank):
             vals.append(info["value"])
     value = statistics.mean(vals) if vals else info["value"]
     from gated_delta_rule_133_b200.inputs import WORKLOADS
-    w = WORKLOADS["prefill"]
+    w = WORKLOADS["long"]
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": w.B * w.T / value * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"prefill: B={w.B} H={w.H} T={w.T} d_k={w.dk} d_v={w.dv} (fp64 CPU oracle)"},
+            "config": {"workload": f"long context: B={w.B} H={w.H} T={w.T} d_k={w.dk} d_v={w.dv} chunk={w.chunk}, "
+                                   "bf16 q/k/v, fp32 state and fp32 output, log alpha = -softplus(z), z ~ N(-1, 1), "
+                                   "zero initial state",
+                       "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"replicas x{world}",
+                       "oracle": "fp64 CPU token recurrence"},
             "cpu_baseline": {**info, "value": value},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -517,11 +545,11 @@ def run_reference(args, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--skip-others", action="store_true", help="skip the varlen / long-context timings")
+    ap.add_argument("--skip-others", action="store_true", help="skip the prefill / varlen / variant timings")
     args = ap.parse_args(argv)
     world, rank, local = dist_env()
     if args.impl == "reference":

@@ -17,6 +17,12 @@ delta rule's erase term (S_t = Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T).  Two
 more flags move input pre-processing into the kernels: ``normalize_qk=True``
 divides every q and k row by its L2 norm, and ``gate_logits=True`` reads
 log_alpha as logits z (log alpha = -softplus(z)).
+
+The tensor-core chunk forward needs scratch memory: these calls ask the library
+for its size (``kda_chunk_fwd_workspace_size`` / ``kda_varlen_fwd_workspace_size``)
+and allocate it with PyTorch's caching allocator, or take a caller's uint8
+``workspace`` tensor.  ``cuda_cores=True`` runs the fp32 CUDA-core kernel and
+``blocks=n`` the two-stream blocked schedule (cross-checks; same results).
 """
 from __future__ import annotations
 
@@ -25,7 +31,8 @@ import torch
 from . import _lib
 from ._lib import KdaError
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_varlen_fwd", "kda_recurrent_step", "kda_check", "KdaError"]
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_varlen_fwd", "kda_recurrent_step", "kda_check",
+           "chunk_fwd_workspace_size", "varlen_fwd_workspace_size", "KdaError"]
 
 _DTYPES = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
 
@@ -34,9 +41,32 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-def _mode(head_gate, erase, normalize_qk=False, gate_logits=False):
+def _mode(head_gate, erase, normalize_qk=False, gate_logits=False, cuda_cores=False, blocks=0):
     return ((_lib.KDA_MODE_HEAD_GATE if head_gate else 0) | (0 if erase else _lib.KDA_MODE_NO_ERASE)
-            | (_lib.KDA_MODE_NORM_QK if normalize_qk else 0) | (_lib.KDA_MODE_GATE_LOGITS if gate_logits else 0))
+            | (_lib.KDA_MODE_NORM_QK if normalize_qk else 0) | (_lib.KDA_MODE_GATE_LOGITS if gate_logits else 0)
+            | (_lib.KDA_MODE_CUDA_CORES if cuda_cores else 0) | _lib.KDA_MODE_BLOCKS(int(blocks)))
+
+
+def chunk_fwd_workspace_size(B, T, H, dk, dv, dtype=torch.bfloat16, chunk=64, mode=0):
+    """Workspace bytes kda_chunk_fwd needs for these sizes (0 on the CUDA-core path)."""
+    return _lib.workspace_size("kda_chunk_fwd_workspace_size", B, T, H, dk, dv, chunk, _DTYPES[dtype], mode)
+
+
+def varlen_fwd_workspace_size(N, T, H, dk, dv, dtype=torch.bfloat16, chunk=64, mode=0):
+    """Workspace bytes kda_varlen_fwd needs for N packed sequences of T tokens in all."""
+    return _lib.workspace_size("kda_varlen_fwd_workspace_size", N, T, H, dk, dv, chunk, _DTYPES[dtype], mode)
+
+
+def _workspace(nbytes, workspace, device):
+    """(pointer, bytes) of the scratch a call needs: the caller's uint8 tensor,
+    or a fresh one from PyTorch's caching allocator."""
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if workspace.device != device or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor on the inputs' device")
+    return workspace.data_ptr(), workspace.numel()
 
 
 def _stream(stream):
@@ -58,7 +88,8 @@ def _check(t, name, shape, dtype, device):
 
 def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final_state=None,
                   output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None,
-                  head_gate=False, erase=True, normalize_qk=False, gate_logits=False):
+                  head_gate=False, erase=True, normalize_qk=False, gate_logits=False,
+                  workspace=None, cuda_cores=False, blocks=0):
     """Chunkwise forward over equal-length sequences.
 
     q, k [B, T, H, dk] and v [B, T, H, dv] (bf16 or fp32); beta [B, T, H] and
@@ -67,7 +98,7 @@ def kda_chunk_fwd(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final
     dtype when o is given), final_state [B, H, dk, dv] or None)."""
     return _dense_fwd("kda_chunk_fwd", q, k, v, beta, log_alpha, initial_state, o, final_state,
                       output_final_state, o_dtype, chunk, stream,
-                      _mode(head_gate, erase, normalize_qk, gate_logits))
+                      _mode(head_gate, erase, normalize_qk, gate_logits, cuda_cores, blocks), workspace)
 
 
 def kda_chunk_fwd_noalloc(q, k, v, beta, log_alpha, initial_state=None, *, o=None, final_state=None,
@@ -80,7 +111,7 @@ def kda_chunk_fwd_noalloc(q, k, v, beta, log_alpha, initial_state=None, *, o=Non
 
 
 def _dense_fwd(symbol, q, k, v, beta, log_alpha, initial_state, o, final_state, output_final_state, o_dtype,
-               chunk, stream, mode=0):
+               chunk, stream, mode=0, workspace=None):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev, dt = q.device, q.dtype
@@ -102,18 +133,23 @@ def _dense_fwd(symbol, q, k, v, beta, log_alpha, initial_state, o, final_state, 
         final_state = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
     if final_state is not None:
         _check(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
-    extra = ()
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha), _ptr(initial_state), _ptr(o),
+            _ptr(final_state), B, T, H, dk, dv, chunk, _DTYPES[dt], _DTYPES[o.dtype])
+    if symbol == "kda_chunk_fwd_noalloc":
+        _lib.call(symbol, *args, _stream(stream))
+        return o, final_state
+    ws = _workspace(chunk_fwd_workspace_size(B, T, H, dk, dv, dt, chunk, mode), workspace, dev)
     if mode:
-        symbol, extra = symbol + "_mode", (mode,)
-    _lib.call(symbol, _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha),
-              _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk,
-              _DTYPES[dt], _DTYPES[o.dtype], *extra, _stream(stream))
+        _lib.call("kda_chunk_fwd_mode", *args, mode, *ws, _stream(stream))
+    else:
+        _lib.call("kda_chunk_fwd", *args, *ws, _stream(stream))
     return o, final_state
 
 
 def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, o=None,
                    final_state=None, output_final_state=True, o_dtype=torch.float32, chunk=64,
-                   stream=None, head_gate=False, erase=True, normalize_qk=False, gate_logits=False):
+                   stream=None, head_gate=False, erase=True, normalize_qk=False, gate_logits=False,
+                   workspace=None, cuda_cores=False):
     """Chunkwise forward over N packed variable-length sequences.
 
     q, k [T, H, dk], v [T, H, dv]; beta [T, H]; log_alpha [T, H, dk] ([T, H]
@@ -142,10 +178,11 @@ def kda_varlen_fwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state=None, *, 
         final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
     if final_state is not None:
         _check(final_state, "final_state", (N, H, dk, dv), torch.float32, dev)
-    mode = _mode(head_gate, erase, normalize_qk, gate_logits)
+    mode = _mode(head_gate, erase, normalize_qk, gate_logits, cuda_cores)
+    ws = _workspace(varlen_fwd_workspace_size(N, T, H, dk, dv, dt, chunk, mode), workspace, dev)
     _lib.call("kda_varlen_fwd_mode" if mode else "kda_varlen_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
               _ptr(log_alpha), _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(o), _ptr(final_state), T, H, dk,
-              dv, chunk, _DTYPES[dt], _DTYPES[o.dtype], *((mode,) if mode else ()), _stream(stream))
+              dv, chunk, _DTYPES[dt], _DTYPES[o.dtype], *((mode,) if mode else ()), *ws, _stream(stream))
     return o, final_state
 
 

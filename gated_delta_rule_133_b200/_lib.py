@@ -15,17 +15,28 @@ LIB_PATH = os.path.join(HERE, "libkda.so")
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
 KDA_F32, KDA_BF16 = 0, 1
 KDA_MODE_HEAD_GATE, KDA_MODE_NO_ERASE, KDA_MODE_NORM_QK, KDA_MODE_GATE_LOGITS = 1, 2, 4, 8
+KDA_MODE_CUDA_CORES = 16
+
+
+def KDA_MODE_BLOCKS(n: int) -> int:
+    return n << 8
+
 
 # Every symbol include/kda.h declares, with its ctypes signature.
 _P = ctypes.c_void_p
 _I = ctypes.c_int
+_Z = ctypes.c_size_t
+_ZP = ctypes.POINTER(ctypes.c_size_t)
 SIGNATURES = {
-    "kda_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    "kda_chunk_fwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _ZP]),
     "kda_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
-    "kda_varlen_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_varlen_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    "kda_varlen_fwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _ZP]),
     "kda_recurrent_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
-    "kda_chunk_fwd_mode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
-    "kda_varlen_fwd_mode": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_chunk_fwd_mode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    "kda_varlen_fwd_mode": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _Z,
+                                 _P]),
     "kda_recurrent_step_mode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "kda_check": (_I, [_P]),
     "kda_selftest_timeout": (_I, [ctypes.c_longlong, _P]),
@@ -66,3 +77,10 @@ def call(name: str, *args) -> None:
     st = getattr(load(), name)(*args)
     if st != KDA_OK:
         raise KdaError(st, name)
+
+
+def workspace_size(name: str, *args) -> int:
+    """Bytes returned by one of the *_workspace_size entry points."""
+    out = ctypes.c_size_t(0)
+    call(name, *args, ctypes.byref(out))
+    return int(out.value)

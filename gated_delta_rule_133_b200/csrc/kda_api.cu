@@ -2,7 +2,6 @@
 // Declarations and the contract of every entry point are in include/kda.h.
 #include <string.h>
 #include <cuda_runtime.h>
-#include <stdlib.h>
 
 #include "kda_chunk.cuh"
 #include "kda_sm100.cuh"
@@ -18,50 +17,27 @@ bool valid_dtype(kda_dtype t) { return t == KDA_F32 || t == KDA_BF16; }
 
 kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
-// Kernel selection for bf16 inputs: the two-pass tensor-core forward by
-// default; KDA_CHUNK_KERNEL=fused selects the single-pass tensor-core kernel
-// and KDA_CHUNK_KERNEL=simt (or KDA_FORCE_SIMT=1) the CUDA-core kernel (used
-// by tests that compare the kernels).  KDA_TIMEOUT_CYCLES bounds every
-// device-side wait of the tensor-core kernels (default 2^31 SM cycles, about
-// one second).
-enum class ChunkKernel { split, fused, simt };
-ChunkKernel chunk_kernel()
+// Budget of every device-side bounded wait of the tensor-core kernels, in SM
+// clock cycles (about one second).
+constexpr long long kTimeoutCycles = 1LL << 31;
+
+constexpr int kLayerBits = KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE | KDA_MODE_NORM_QK | KDA_MODE_GATE_LOGITS;
+
+int mode_blocks(int mode) { return (mode >> 8) & 0xff; }
+
+bool valid_mode(int mode, bool chunk_call)
 {
-    const char* f = getenv("KDA_FORCE_SIMT");
-    if (f && f[0] == '1') return ChunkKernel::simt;
-    const char* e = getenv("KDA_CHUNK_KERNEL");
-    if (e && strcmp(e, "fused") == 0) return ChunkKernel::fused;
-    if (e && strcmp(e, "simt") == 0) return ChunkKernel::simt;
-    return ChunkKernel::split;
+    if (!chunk_call) return (mode & ~kLayerBits) == 0;
+    const int nb = mode_blocks(mode);
+    return (mode & ~(kLayerBits | KDA_MODE_CUDA_CORES | KDA_MODE_BLOCKS(0xff))) == 0 && nb <= 8;
 }
 
-long long timeout_cycles()
+// bf16 inputs with supported head sizes run on the tensor cores unless the
+// caller asks for the CUDA-core kernel; fp32 inputs always run on the CUDA
+// cores (their fp32 arithmetic is what meets the fp32 bar).
+bool use_tensor_cores(int dk, int dv, kda_dtype dtype, int mode)
 {
-    const char* e = getenv("KDA_TIMEOUT_CYCLES");
-    long long v = e ? atoll(e) : 0;
-    return v > 0 ? v : (1LL << 31);
-}
-
-kda_status run_chunk(const void* q, const void* k, const void* v, const float* beta,
-                     const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
-                     int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype dtype,
-                     kda_dtype o_dtype, int mode, cudaStream_t s)
-{
-    const ChunkKernel kind = chunk_kernel();
-    // the single-pass kernel implements the plain layer only: variants take the two-pass path
-    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && kind == ChunkKernel::fused && mode == 0)
-        return from_cuda(kda::chunk_fwd_tc(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk,
-                                           dv, o_dtype, timeout_cycles(), s));
-    if (kda::chunk_fwd_tc_supported(dk, dv, dtype) && kind != ChunkKernel::simt)
-        return from_cuda(kda::chunk_fwd_split(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk,
-                                              dv, o_dtype, timeout_cycles(), mode, s));
-    return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, dtype,
-                                         o_dtype, mode, s));
-}
-
-bool valid_mode(int mode)
-{
-    return (mode & ~(KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE | KDA_MODE_NORM_QK | KDA_MODE_GATE_LOGITS)) == 0;
+    return kda::chunk_fwd_split_supported(dk, dv, dtype) && !(mode & KDA_MODE_CUDA_CORES);
 }
 
 // Shared checks of the forward entry points.
@@ -71,7 +47,7 @@ kda_status check_fwd(const void* q, const void* k, const void* v, const float* b
                      kda_dtype o_dtype, int mode)
 {
     if (H <= 0 || dk <= 0 || dv <= 0 || tokens < 0) return KDA_ERR_INVALID_ARG;
-    if (!valid_dtype(dtype) || !valid_dtype(o_dtype) || !valid_mode(mode)) return KDA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype) || !valid_dtype(o_dtype) || !valid_mode(mode, true)) return KDA_ERR_INVALID_ARG;
     const bool gate_ok = (mode & KDA_MODE_HEAD_GATE) ? aligned4(log_alpha) : aligned16(log_alpha);
     if (tokens > 0) {
         if (!q || !k || !v || !beta || !log_alpha || !o) return KDA_ERR_INVALID_ARG;
@@ -81,6 +57,40 @@ kda_status check_fwd(const void* q, const void* k, const void* v, const float* b
     if ((s0 && !aligned16(s0)) || (sT && !aligned16(sT))) return KDA_ERR_INVALID_ARG;
     if (chunk != 64 || !supported_d(dk) || !supported_d(dv)) return KDA_ERR_UNSUPPORTED;
     return KDA_OK;
+}
+
+// Size checks shared by the workspace queries and the forward calls.
+kda_status check_sizes(int H, int dk, int dv, int chunk, kda_dtype dtype, int mode)
+{
+    if (H <= 0 || dk <= 0 || dv <= 0 || !valid_dtype(dtype) || !valid_mode(mode, true)) return KDA_ERR_INVALID_ARG;
+    if (chunk != 64 || !supported_d(dk) || !supported_d(dv)) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+size_t workspace_bytes(int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype dtype, int mode,
+                       bool varlen)
+{
+    if (!use_tensor_cores(dk, dv, dtype, mode) || tokens <= 0) return 0;
+    return kda::chunk_fwd_split_workspace(nseq, T, tokens, H, dk, dv, varlen, mode);
+}
+
+kda_status check_workspace(const void* ws, size_t have, size_t need)
+{
+    if (need == 0) return KDA_OK;
+    if (!ws || have < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
+kda_status run_chunk(const void* q, const void* k, const void* v, const float* beta,
+                     const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
+                     int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype dtype,
+                     kda_dtype o_dtype, int mode, void* ws, size_t ws_bytes, cudaStream_t s)
+{
+    if (use_tensor_cores(dk, dv, dtype, mode))
+        return from_cuda(kda::chunk_fwd_split(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv,
+                                              o_dtype, kTimeoutCycles, mode, ws, ws_bytes, s));
+    return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv, dtype,
+                                         o_dtype, mode & kLayerBits, s));
 }
 
 // Writes final = initial (or zeros) for sequences that have no tokens at all.
@@ -111,10 +121,33 @@ __global__ void selftest_timeout_kernel(long long limit_cycles)
 
 extern "C" {
 
+kda_status kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, kda_dtype dtype, int mode,
+                                        size_t* bytes)
+{
+    if (!bytes || B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    const kda_status st = check_sizes(H, dk, dv, chunk, dtype, mode);
+    if (st != KDA_OK) return st;
+    const long long tokens = (long long)B * T;
+    if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    *bytes = workspace_bytes(B, T, tokens, H, dk, dv, dtype, mode, false);
+    return KDA_OK;
+}
+
+kda_status kda_varlen_fwd_workspace_size(int N, int T, int H, int dk, int dv, int chunk, kda_dtype dtype, int mode,
+                                         size_t* bytes)
+{
+    if (!bytes || N < 0 || N > 65535 || T < 0 || (mode_blocks(mode) != 0)) return KDA_ERR_INVALID_ARG;
+    const kda_status st = check_sizes(H, dk, dv, chunk, dtype, mode);
+    if (st != KDA_OK) return st;
+    *bytes = N == 0 ? 0 : workspace_bytes(N, 0, T, H, dk, dv, dtype, mode, true);
+    return KDA_OK;
+}
+
 kda_status kda_chunk_fwd_mode(const void* q, const void* k, const void* v, const float* beta,
                               const float* log_alpha, const float* initial_state, void* o,
                               float* final_state, int B, int T, int H, int dk, int dv, int chunk,
-                              kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream)
+                              kda_dtype dtype, kda_dtype o_dtype, int mode, void* workspace,
+                              size_t workspace_bytes_, void* stream)
 {
     if (B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
     const long long tokens = (long long)B * T;
@@ -122,19 +155,22 @@ kda_status kda_chunk_fwd_mode(const void* q, const void* k, const void* v, const
                               dk, dv, chunk, dtype, o_dtype, mode);
     if (st != KDA_OK) return st;
     if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes_, workspace_bytes(B, T, tokens, H, dk, dv, dtype, mode, false));
+    if (st != KDA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (tokens == 0) return copy_state(initial_state, final_state, (size_t)B * H * dk * dv, s);
     return run_chunk(q, k, v, beta, log_alpha, initial_state, o, final_state, nullptr, B, T, tokens, H, dk,
-                     dv, dtype, o_dtype, mode, s);
+                     dv, dtype, o_dtype, mode, workspace, workspace_bytes_, s);
 }
 
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
                          const float* log_alpha, const float* initial_state, void* o,
                          float* final_state, int B, int T, int H, int dk, int dv, int chunk,
-                         kda_dtype dtype, kda_dtype o_dtype, void* stream)
+                         kda_dtype dtype, kda_dtype o_dtype, void* workspace, size_t workspace_bytes_,
+                         void* stream)
 {
     return kda_chunk_fwd_mode(q, k, v, beta, log_alpha, initial_state, o, final_state, B, T, H, dk, dv, chunk,
-                              dtype, o_dtype, 0, stream);
+                              dtype, o_dtype, 0, workspace, workspace_bytes_, stream);
 }
 
 kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* beta,
@@ -150,40 +186,42 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, co
     if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (tokens == 0) return copy_state(initial_state, final_state, (size_t)B * H * dk * dv, s);
-    if (!kda::chunk_fwd_tc_supported(dk, dv, dtype))   // the CUDA-core kernel needs no scratch
+    if (!kda::chunk_fwd_split_supported(dk, dv, dtype))   // the CUDA-core kernel needs no scratch
         return from_cuda(kda::chunk_fwd_simt(q, k, v, beta, log_alpha, initial_state, o, final_state, nullptr, B,
-                                             T, H, dk, dv, dtype, o_dtype, 0, s));
+                                             T, tokens, H, dk, dv, dtype, o_dtype, 0, s));
     if (!kda::chunk_fwd_noalloc_fits(B, T, H, dk, dv, final_state != nullptr)) return KDA_ERR_UNSUPPORTED;
     return from_cuda(kda::chunk_fwd_noalloc(q, k, v, beta, log_alpha, initial_state, o, final_state, B, T, tokens,
-                                            H, dk, dv, o_dtype, timeout_cycles(), s));
+                                            H, dk, dv, o_dtype, kTimeoutCycles, s));
 }
 
 kda_status kda_varlen_fwd_mode(const void* q, const void* k, const void* v, const float* beta,
                                const float* log_alpha, const int32_t* cu_seqlens, int N,
                                const float* initial_state, void* o, float* final_state, int T, int H,
                                int dk, int dv, int chunk, kda_dtype dtype, kda_dtype o_dtype, int mode,
-                               void* stream)
+                               void* workspace, size_t workspace_bytes_, void* stream)
 {
-    if (N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
+    if (N < 0 || N > 65535 || T < 0 || mode_blocks(mode) != 0) return KDA_ERR_INVALID_ARG;
     kda_status st = check_fwd(q, k, v, beta, log_alpha, initial_state, o, final_state, T, H, dk,
                               dv, chunk, dtype, o_dtype, mode);
     if (st != KDA_OK) return st;
     if (N == 0) return T == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
     if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARG;
+    st = check_workspace(workspace, workspace_bytes_, workspace_bytes(N, 0, T, H, dk, dv, dtype, mode, true));
+    if (st != KDA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0) return copy_state(initial_state, final_state, (size_t)N * H * dk * dv, s);
     return run_chunk(q, k, v, beta, log_alpha, initial_state, o, final_state, cu_seqlens, N, T, T, H, dk,
-                     dv, dtype, o_dtype, mode, s);
+                     dv, dtype, o_dtype, mode, workspace, workspace_bytes_, s);
 }
 
 kda_status kda_varlen_fwd(const void* q, const void* k, const void* v, const float* beta,
                           const float* log_alpha, const int32_t* cu_seqlens, int N,
                           const float* initial_state, void* o, float* final_state, int T, int H,
                           int dk, int dv, int chunk, kda_dtype dtype, kda_dtype o_dtype,
-                          void* stream)
+                          void* workspace, size_t workspace_bytes_, void* stream)
 {
     return kda_varlen_fwd_mode(q, k, v, beta, log_alpha, cu_seqlens, N, initial_state, o, final_state, T, H,
-                               dk, dv, chunk, dtype, o_dtype, 0, stream);
+                               dk, dv, chunk, dtype, o_dtype, 0, workspace, workspace_bytes_, stream);
 }
 
 kda_status kda_recurrent_step_mode(const void* q, const void* k, const void* v, const float* beta,
@@ -191,7 +229,7 @@ kda_status kda_recurrent_step_mode(const void* q, const void* k, const void* v, 
                                    int dv, kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream)
 {
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
-    if (!valid_dtype(dtype) || !valid_dtype(o_dtype) || !valid_mode(mode)) return KDA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype) || !valid_dtype(o_dtype) || !valid_mode(mode, false)) return KDA_ERR_INVALID_ARG;
     if (N == 0) return KDA_OK;
     if (!q || !k || !v || !beta || !log_alpha || !state || !o) return KDA_ERR_INVALID_ARG;
     const bool gate_ok = (mode & KDA_MODE_HEAD_GATE) ? aligned4(log_alpha) : aligned16(log_alpha);
@@ -242,6 +280,6 @@ const char* kda_status_string(kda_status status)
     return "KDA_ERR_UNKNOWN";
 }
 
-int kda_version(void) { return 100; }
+int kda_version(void) { return 200; }
 
 }  // extern "C"

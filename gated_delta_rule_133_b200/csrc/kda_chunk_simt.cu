@@ -77,32 +77,13 @@ struct Smem {
     float beta[C];
 };
 
-// Rank-r sequence in longest-first order (ties: lower index first).  N is small.
-__device__ int seq_by_rank(const int32_t* cu, int N, int rank, int* s_out)
-{
-    if (threadIdx.x == 0) *s_out = rank;
-    __syncthreads();
-    for (int i = threadIdx.x; i < N; i += blockDim.x) {
-        const int li = cu[i + 1] - cu[i];
-        int rk = 0;
-        for (int j = 0; j < N; ++j) {
-            const int lj = cu[j + 1] - cu[j];
-            rk += (lj > li) || (lj == li && j < i);
-        }
-        if (rk == rank) *s_out = i;
-    }
-    __syncthreads();
-    const int n = *s_out;
-    __syncthreads();
-    return n;
-}
-
 template <typename TIn, typename TOut, int DK>
 __global__ void __launch_bounds__(NT)
 chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                       const TIn* __restrict__ v, const float* __restrict__ beta,
                       const float* __restrict__ log_alpha, const float* s0, TOut* __restrict__ o,
-                      float* sT, const int32_t* __restrict__ cu, int nseq, int T, int H, int DV, int mode)
+                      float* sT, const int32_t* __restrict__ cu, int nseq, int T, long long tokens, int H, int DV,
+                      int mode)
 {
     const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;   // log_alpha [tokens, H]
     const bool erase = (mode & KDA_MODE_NO_ERASE) == 0;
@@ -111,17 +92,21 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Smem<DK>& sm = *reinterpret_cast<Smem<DK>*>(smem_raw);
     constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC;
-    __shared__ int s_tmp;
 
     const int nslice = DV / NV;
     const int slice = blockIdx.x % nslice;
     const int h = (blockIdx.x / nslice) % H;
     const int rank = blockIdx.x / (nslice * H);
     int n, tok0, len;
-    if (cu) {
-        n = seq_by_rank(cu, nseq, rank, &s_tmp);
+    if (cu) {   // packed sequences in their own order; a range outside the token axis is skipped
+        n = rank;
         tok0 = cu[n];
-        len = cu[n + 1] - tok0;
+        len = max(0, cu[n + 1] - tok0);
+        if (tok0 < 0 || (long long)tok0 + len > tokens) {   // no tokens read; final state = initial
+            if (threadIdx.x == 0) flag_bad_input();
+            tok0 = 0;
+            len = 0;
+        }
     } else {
         n = rank;
         tok0 = n * T;
@@ -297,7 +282,7 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 template <typename TIn, typename TOut, int DK>
 cudaError_t launch(const void* q, const void* k, const void* v, const float* beta,
                    const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
-                   int nseq, int T, int H, int dv, int mode, cudaStream_t stream)
+                   int nseq, int T, long long tokens, int H, int dv, int mode, cudaStream_t stream)
 {
     const size_t smem = sizeof(Smem<DK>);
     auto kern = chunk_fwd_simt_kernel<TIn, TOut, DK>;
@@ -308,17 +293,18 @@ cudaError_t launch(const void* q, const void* k, const void* v, const float* bet
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     kern<<<(unsigned)blocks, NT, smem, stream>>>(
         static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), beta,
-        log_alpha, s0, static_cast<TOut*>(o), sT, cu, nseq, T, H, dv, mode);
+        log_alpha, s0, static_cast<TOut*>(o), sT, cu, nseq, T, tokens, H, dv, mode);
     return cudaGetLastError();
 }
 
 template <typename TIn, typename TOut>
 cudaError_t launch_dk(const void* q, const void* k, const void* v, const float* beta,
                       const float* log_alpha, const float* s0, void* o, float* sT,
-                      const int32_t* cu, int nseq, int T, int H, int dk, int dv, int mode, cudaStream_t s)
+                      const int32_t* cu, int nseq, int T, long long tokens, int H, int dk, int dv, int mode,
+                      cudaStream_t s)
 {
-    if (dk == 128) return launch<TIn, TOut, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, mode, s);
-    if (dk == 64) return launch<TIn, TOut, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dv, mode, s);
+    if (dk == 128) return launch<TIn, TOut, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, mode, s);
+    if (dk == 64) return launch<TIn, TOut, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, mode, s);
     return cudaErrorInvalidValue;
 }
 
@@ -326,17 +312,17 @@ cudaError_t launch_dk(const void* q, const void* k, const void* v, const float* 
 
 cudaError_t chunk_fwd_simt(const void* q, const void* k, const void* v, const float* beta,
                            const float* log_alpha, const float* s0, void* o, float* sT,
-                           const int32_t* cu, int nseq, int T, int H, int dk, int dv,
+                           const int32_t* cu, int nseq, int T, long long tokens, int H, int dk, int dv,
                            kda_dtype dtype, kda_dtype o_dtype, int mode, cudaStream_t s)
 {
     using bf = __nv_bfloat16;
     if (dtype == KDA_BF16 && o_dtype == KDA_BF16)
-        return simt::launch_dk<bf, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, mode, s);
+        return simt::launch_dk<bf, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv, mode, s);
     if (dtype == KDA_BF16 && o_dtype == KDA_F32)
-        return simt::launch_dk<bf, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, mode, s);
+        return simt::launch_dk<bf, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv, mode, s);
     if (dtype == KDA_F32 && o_dtype == KDA_BF16)
-        return simt::launch_dk<float, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, mode, s);
-    return simt::launch_dk<float, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, H, dk, dv, mode, s);
+        return simt::launch_dk<float, bf>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv, mode, s);
+    return simt::launch_dk<float, float>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv, mode, s);
 }
 
 }  // namespace kda

@@ -326,7 +326,7 @@ __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& 
         *reinterpret_cast<float4*>(x.A1 + swf_off(r, c0, 128)) = tf32r4(q4.x * e0, q4.y * e1, q4.z * e2, q4.w * e3);
         *reinterpret_cast<float4*>(x.A1 + swf_off(C + r, c0, 128)) = tf32r4(k4.x * e0, k4.y * e1, k4.z * e2, k4.w * e3);
         *reinterpret_cast<float4*>(x.B1 + swf_off(r, c0, 64)) =
-            tf32r4(k4.x * rcp_nr(e0), k4.y * rcp_nr(e1), k4.z * rcp_nr(e2), k4.w * rcp_nr(e3));
+            tf32r4(k4.x * rcp_approx(e0), k4.y * rcp_approx(e1), k4.z * rcp_approx(e2), k4.w * rcp_approx(e3));
         const float f0 = e0 * gm4.x, f1 = e1 * gm4.y, f2 = e2 * gm4.z, f3 = e3 * gm4.w;
         *reinterpret_cast<uint2*>(rec + R::QK + swh_off(r, c0, 128)) =
             make_uint2(pack_f16(q4.x * f0, q4.y * f1), pack_f16(q4.z * f2, q4.w * f3));
@@ -755,6 +755,7 @@ struct ScanParams {
     int c_begin, c_end;      // chunk range of this launch (per sequence)
     const int32_t* cu;
     const int32_t* choff;
+    const int32_t* order;    // varlen: sequence of each scan rank (longest first)
     const unsigned char* rec;
     int nseq, T, H, DV, nch;
     int rs, rc0;             // dense: record of (n, c, h) = (n * rs + c - rc0) * H + h
@@ -877,7 +878,6 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
     uint64_t* mb_w = bars + 5;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* misc_slot = reinterpret_cast<int*>(tmem_slot + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int lt = tid & 127;
@@ -890,7 +890,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
     int n, tok0, len;
     long long j0;
     if (p.cu) {
-        n = seq_by_rank(p.cu, p.nseq, rank, misc_slot);
+        n = p.order[rank];
         tok0 = p.cu[n];
         len = max(0, p.cu[n + 1] - tok0);
         j0 = p.choff[n];
@@ -1181,18 +1181,29 @@ chunk_coop_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 
 // ============================================================== host side
 
-// First chunk of every packed sequence: choff[i] = sum_{j<i} ceil(len_j / 64),
-// choff[nseq] = total.  One CTA; each thread sums a contiguous range of
-// sequences, then a block-wide scan.  Negative lengths count as empty.
-__global__ void chunk_offsets_kernel(const int32_t* cu, int nseq, int32_t* choff)
+// Per-call index arrays of a packed (varlen) batch, one CTA of 1024 threads:
+//   choff[i] = sum_{j<i} ceil(len_j / 64) (first record of sequence i),
+//   choff[nseq] = total;
+//   order[r] = the sequence the scan CTAs of rank r take: longest first, ties
+//   by lower index (negative lengths count as empty).
+// The order is a bitonic sort of 64-bit keys (complemented length, index) of
+// the next power of two of nseq, in shared memory when it fits, else in the
+// workspace `gkeys`.
+constexpr int kIndexThreads = 1024;
+constexpr int kSmemKeys = 16384;
+
+__global__ void __launch_bounds__(kIndexThreads)
+varlen_index_kernel(const int32_t* cu, int nseq, int32_t* choff, int32_t* order, unsigned long long* gkeys)
 {
     __shared__ int warp_tot[32];
-    const int per = (nseq + blockDim.x - 1) / blockDim.x;
-    const int a = min(nseq, (int)threadIdx.x * per), b = min(nseq, a + per);
+    extern __shared__ unsigned long long skeys[];
+    const int tid = threadIdx.x;
+    const int per = (nseq + kIndexThreads - 1) / kIndexThreads;
+    const int a = min(nseq, tid * per), b = min(nseq, a + per);
     int local = 0;
     for (int i = a; i < b; ++i) local += (max(0, cu[i + 1] - cu[i]) + C - 1) / C;
     int x = local;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int lane = tid & 31, w = tid >> 5;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -1201,7 +1212,7 @@ __global__ void chunk_offsets_kernel(const int32_t* cu, int nseq, int32_t* choff
     if (lane == 31) warp_tot[w] = x;
     __syncthreads();
     if (w == 0) {
-        int t = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+        int t = warp_tot[lane];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, t, o);
@@ -1215,7 +1226,33 @@ __global__ void chunk_offsets_kernel(const int32_t* cu, int nseq, int32_t* choff
         choff[i] = base;
         base += (max(0, cu[i + 1] - cu[i]) + C - 1) / C;
     }
-    if (threadIdx.x == blockDim.x - 1) choff[nseq] = base;
+    if (tid == kIndexThreads - 1) choff[nseq] = base;
+
+    int npad = 1;
+    while (npad < nseq) npad <<= 1;
+    unsigned long long* keys = npad <= kSmemKeys ? skeys : gkeys;
+    for (int i = tid; i < npad; i += kIndexThreads) {
+        const unsigned len = i < nseq ? (unsigned)max(0, cu[i + 1] - cu[i]) : 0u;
+        // ascending keys: longer first, then lower index; padding sorts last
+        keys[i] = i < nseq ? ((unsigned long long)(0x7fffffffu - len) << 32) | (unsigned)i : ~0ull;
+    }
+    __syncthreads();
+    for (int size = 2; size <= npad; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = tid; t < npad / 2; t += kIndexThreads) {
+                const int lo = 2 * t - (t & (stride - 1));    // index whose `stride` bit is clear
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const unsigned long long kl = keys[lo], kh = keys[hi];
+                if ((kl > kh) == up) {
+                    keys[lo] = kh;
+                    keys[hi] = kl;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int r = tid; r < nseq; r += kIndexThreads) order[r] = (int32_t)(keys[r] & 0xffffffffu);
 }
 
 static int sm_count()
@@ -1226,68 +1263,105 @@ static int sm_count()
     return n > 0 ? n : 148;
 }
 
-// Keeps freed stream-ordered allocations in the device's default pool, so
-// that the per-call workspace is recycled instead of returned to the driver.
-static void retain_pool_memory()
+// Second stream on which the parallel pass of the next block of chunks runs
+// while the current block is scanned.  Cached per CUDA context (created on
+// first use in that context), so a context that is destroyed and re-created
+// gets a stream of its own.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+static CUcontext current_context()
 {
-    static bool done[64] = {false};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || done[dev]) return;
-    cudaMemPool_t pool;
-    if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
-        uint64_t keep = ~0ull;
-        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
     }
-    done[dev] = true;
+    CUcontext ctx = nullptr;
+    if (cudaFree(nullptr) != cudaSuccess) return nullptr;   // makes the device's primary context current
+    return fn(&ctx) == CUDA_SUCCESS ? ctx : nullptr;
 }
 
-// Second stream of the current device on which the prep of the next block of
-// chunks runs while the current block is scanned (created on first use).
 static cudaStream_t side_stream()
 {
     static std::mutex mu;
+    static CUcontext ctxs[64] = {};
     static cudaStream_t streams[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    const CUcontext ctx = current_context();
+    if (!ctx) return nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
-        streams[dev] = nullptr;
-    return streams[dev];
+    int slot = -1;
+    for (int i = 0; i < 64; ++i) {
+        if (ctxs[i] == ctx) return streams[i];
+        if (!ctxs[i] && slot < 0) slot = i;
+    }
+    if (slot < 0) return nullptr;
+    cudaStream_t st = nullptr;
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    ctxs[slot] = ctx;
+    streams[slot] = st;
+    return st;
 }
 
 constexpr int kMaxBlocks = 8;
 
-// Number of chunk blocks for a dense problem: the prep of block b + 1 runs on
-// the SMs the scan of block b leaves idle, so blocking pays only when the scan
-// grid leaves room.  KDA_SCAN_BLOCKS overrides (1 = no blocking).
-static int chunk_blocks(int nch, long long scan_ctas, int nsm)
+// Offsets (bytes) of the parts of a call's workspace.
+struct WsLayout {
+    size_t choff, order, keys, carry, flags, rec, bytes;
+    long long max_chunks;
+};
+
+static size_t align1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
+
+template <int DK>
+static WsLayout ws_layout(int nseq, int T, long long tokens, int H, int dv, bool varlen)
 {
-    const char* e = getenv("KDA_SCAN_BLOCKS");
-    int nb = e ? atoi(e) : 0;
-    if (nb <= 0) nb = (scan_ctas + 32 <= nsm) ? nch / 32 : 1;   // measured: 32+ chunks per block
-    return std::max(1, std::min(std::min(nb, nch), kMaxBlocks));
+    WsLayout w{};
+    w.max_chunks = varlen ? tokens / C + nseq : (long long)nseq * ((T + C - 1) / C);
+    int npad = 1;
+    while (npad < nseq) npad <<= 1;
+    size_t off = 0;
+    w.choff = off;
+    off += varlen ? align1k(((size_t)nseq + 1) * 4) : 0;
+    w.order = off;
+    off += varlen ? align1k((size_t)nseq * 4) : 0;
+    w.keys = off;
+    off += (varlen && npad > kSmemKeys) ? align1k((size_t)npad * 8) : 0;
+    w.carry = off;                                         // state between blocks when no final state is kept
+    off += varlen ? 0 : align1k((size_t)nseq * H * DK * dv * 4);
+    w.flags = off;                                         // cooperative hand-off flags, one per record
+    off += varlen ? 0 : align1k((size_t)w.max_chunks * H * 4);
+    w.rec = off;
+    off += (size_t)w.max_chunks * H * Rec<DK>::BYTES;
+    w.bytes = off;
+    return w;
 }
 
 template <typename TO, int DK>
 static cudaError_t run(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
                        const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens,
-                       int H, int dv, long long timeout_cycles, int mode, cudaStream_t stream)
+                       int H, int dv, long long timeout_cycles, int mode, unsigned char* ws, size_t ws_bytes,
+                       cudaStream_t stream)
 {
     const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;
-    using R = Rec<DK>;
+    const bool variant = (mode & (KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE | KDA_MODE_NORM_QK | KDA_MODE_GATE_LOGITS)) != 0;
+    const int req_blocks = (mode >> 8) & 0xff;     // KDA_MODE_BLOCKS(n), 0 = automatic
     const int nsm = sm_count();
     const int nch = cu ? 0 : (T + C - 1) / C;
-    const long long max_chunks = cu ? tokens / C + nseq : (long long)nseq * nch;
+    const WsLayout L = ws_layout<DK>(nseq, T, tokens, H, dv, cu != nullptr);
+    if (!ws || ws_bytes < L.bytes) return cudaErrorInvalidValue;
+    const long long max_chunks = L.max_chunks;
     const long long scan_ctas = (long long)nseq * H * (dv / NV);
     if (scan_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     // schedule: one cooperative launch (prep CTAs publish records, scan CTAs
-    // consume them) when the scan grid leaves at least 32 SMs; otherwise
-    // blocks of chunks on two streams, or prep then scan.  KDA_CHUNK_SCHEDULE
-    // (coop | streams) and KDA_SCAN_BLOCKS select explicitly.
-    const char* sched_env = getenv("KDA_CHUNK_SCHEDULE");
-    const bool coop = !cu && scan_ctas > 0 && scan_ctas + 32 <= nsm && !getenv("KDA_SCAN_BLOCKS") &&
-                      !(sched_env && strcmp(sched_env, "coop") != 0);
-    const int nb = (cu || coop) ? 1 : chunk_blocks(nch, scan_ctas, nsm);
+    // consume them) when the scan grid leaves at least 32 SMs; otherwise prep
+    // then scan.  KDA_MODE_BLOCKS(n) asks for n blocks of chunks on two
+    // streams instead (dense inputs).
+    const bool coop = !cu && req_blocks == 0 && scan_ctas > 0 && scan_ctas + 32 <= nsm;
+    const int nb = (cu || coop || req_blocks == 0) ? 1 : std::max(1, std::min(std::min(req_blocks, nch), kMaxBlocks));
     cudaStream_t side = nb > 1 ? side_stream() : nullptr;
 
     CUtensorMap tq, tk, tg;
@@ -1299,8 +1373,8 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
         !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
         return cudaErrorInvalidValue;
-    auto pk = mode ? chunk_prep_kernel<DK, true> : chunk_prep_kernel<DK, false>;
-    auto sk = mode ? chunk_scan_kernel<TO, DK, true> : chunk_scan_kernel<TO, DK, false>;
+    auto pk = variant ? chunk_prep_kernel<DK, true> : chunk_prep_kernel<DK, false>;
+    auto sk = variant ? chunk_scan_kernel<TO, DK, true> : chunk_scan_kernel<TO, DK, false>;
     cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
@@ -1318,27 +1392,29 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
             side = nullptr;
         }
     }
-    const int nblocks = side ? nb : 1;
+    // without a second stream the blocks run one after the other (same results)
+    const int nblocks = nb;
     const int cb = cu ? 0 : (nch + nblocks - 1) / nblocks;     // chunks per block (dense)
-    const size_t off_bytes = (((size_t)nseq + 1) * 4 + 1023) & ~(size_t)1023;
-    const size_t state_bytes = (nblocks > 1 && !sT) ? (size_t)nseq * H * DK * dv * 4 : 0;
-    const size_t flag_off = off_bytes + ((state_bytes + 1023) & ~(size_t)1023);
-    const size_t flag_bytes = coop ? (((size_t)max_chunks * H * 4 + 1023) & ~(size_t)1023) : 0;
-    const size_t rec_off = flag_off + flag_bytes;
-    const size_t bytes = rec_off + (size_t)max_chunks * H * R::BYTES;
+    int32_t* choff = reinterpret_cast<int32_t*>(ws + L.choff);
+    int32_t* order = reinterpret_cast<int32_t*>(ws + L.order);
+    float* carry = sT ? sT : reinterpret_cast<float*>(ws + L.carry);
+    unsigned char* rec = ws + L.rec;
 
-    retain_pool_memory();
-    unsigned char* ws = nullptr;
-    err = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
-    if (err != cudaSuccess) {
-        for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
-        return err;
+    if (cu) {
+        int npad = 1;
+        while (npad < nseq) npad <<= 1;
+        const int smem = npad <= kSmemKeys ? npad * 8 : 0;
+        err = cudaFuncSetAttribute(varlen_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 8);
+        if (err == cudaSuccess) {
+            varlen_index_kernel<<<1, kIndexThreads, smem, stream>>>(cu, nseq, choff, order,
+                                                                    reinterpret_cast<unsigned long long*>(ws + L.keys));
+            err = cudaGetLastError();
+        }
+        if (err != cudaSuccess) {
+            for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+            return err;
+        }
     }
-    int32_t* choff = reinterpret_cast<int32_t*>(ws);
-    float* carry = sT ? sT : reinterpret_cast<float*>(ws + off_bytes);
-    unsigned char* rec = ws + rec_off;
-
-    if (cu) chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu, nseq, choff);
 
     PrepParams pp{};
     pp.beta = beta;
@@ -1363,6 +1439,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     sp.o = o;
     sp.cu = cu;
     sp.choff = choff;
+    sp.order = order;
     sp.rec = rec;
     sp.nseq = nseq;
     sp.T = T;
@@ -1402,9 +1479,9 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
 
     bool done = false;
     if (coop) {
-        unsigned* flags = reinterpret_cast<unsigned*>(ws + flag_off);
-        err = cudaMemsetAsync(flags, 0, flag_bytes, stream);
-        auto ck = mode ? chunk_coop_kernel<TO, DK, true> : chunk_coop_kernel<TO, DK, false>;
+        unsigned* flags = reinterpret_cast<unsigned*>(ws + L.flags);
+        err = cudaMemsetAsync(flags, 0, (size_t)max_chunks * H * 4, stream);
+        auto ck = variant ? chunk_coop_kernel<TO, DK, true> : chunk_coop_kernel<TO, DK, false>;
         const int smem = std::max(PrepPlan::BYTES, ScanPlan<DK>::BYTES);
         if (err == cudaSuccess) err = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err == cudaSuccess) {
@@ -1435,9 +1512,11 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         }
     }
     if (done) {
-    } else if (nblocks == 1) {
-        if (err == cudaSuccess) err = launch_prep(0, stream, nsm);
-        if (err == cudaSuccess) err = launch_scan(0);
+    } else if (nblocks == 1 || !side) {
+        for (int b = 0; b < nblocks && err == cudaSuccess; ++b) {
+            err = launch_prep(b, stream, nsm);
+            if (err == cudaSuccess) err = launch_scan(b);
+        }
     } else {
         // fork: the side stream starts after everything queued on `stream`;
         // the scan of block b waits for the prep of block b; the prep of
@@ -1458,10 +1537,9 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
             cudaEventRecord(ev[nblocks], side);
             cudaStreamWaitEvent(stream, ev[nblocks], 0);
         }
-        for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
     }
-    const cudaError_t ferr = cudaFreeAsync(ws, stream);
-    return err != cudaSuccess ? err : ferr;
+    for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+    return err;
 }
 
 // ============================================================== allocation-free variant
@@ -1473,15 +1551,13 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
 constexpr size_t kScratchBytes = size_t(64) << 20;
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
+// Device address of this device's scratch area, looked up on every call
+// (cheap), so that it always belongs to the current context.
 static unsigned char* scratch_area()
 {
-    static std::mutex mu;
-    static void* areas[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!areas[dev] && cudaGetSymbolAddress(&areas[dev], g_scratch) != cudaSuccess) areas[dev] = nullptr;
-    return static_cast<unsigned char*>(areas[dev]);
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess) return nullptr;
+    return static_cast<unsigned char*>(p);
 }
 
 static size_t carry_bytes(int nseq, int H, int dk, int dv, bool has_final)
@@ -1489,12 +1565,17 @@ static size_t carry_bytes(int nseq, int H, int dk, int dv, bool has_final)
     return has_final ? 0 : (((size_t)nseq * H * dk * dv * 4 + 1023) & ~(size_t)1023);
 }
 
+// Chunks per block of the ring: all nch in one block when their records fit
+// (no carried state is needed then), else the most that fit twice over next
+// to the carried state; 0 when not even one chunk fits that way.
 template <int DK>
 static long long noalloc_block(int nseq, int H, int dv, bool has_final, int nch)
 {
     const size_t per_chunk = (size_t)nseq * H * Rec<DK>::BYTES;   // one chunk of every (sequence, head)
+    if (per_chunk == 0) return 0;
+    if ((size_t)nch * per_chunk <= kScratchBytes) return nch;
     const size_t carry = carry_bytes(nseq, H, DK, dv, has_final);
-    if (per_chunk == 0 || carry + 2 * per_chunk > kScratchBytes) return 0;
+    if (carry + 2 * per_chunk > kScratchBytes) return 0;
     return std::min<long long>(nch, (long long)((kScratchBytes - carry) / (2 * per_chunk)));
 }
 
@@ -1513,9 +1594,10 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
     if (scan_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     unsigned char* area = scratch_area();
     if (!area) return cudaErrorInvalidSymbol;
-    const size_t carry_sz = carry_bytes(nseq, H, DK, dv, sT != nullptr);
-    float* carry = sT ? sT : reinterpret_cast<float*>(area);
-    unsigned char* ring[2] = {area + carry_sz, area + carry_sz + (size_t)cb * nseq * H * R::BYTES};
+    const size_t carry_sz = nblocks > 1 ? carry_bytes(nseq, H, DK, dv, sT != nullptr) : 0;
+    float* carry = sT ? sT : reinterpret_cast<float*>(area);   // unused with one block
+    unsigned char* ring[2] = {area + carry_sz, nullptr};
+    if (nblocks > 1) ring[1] = area + carry_sz + (size_t)cb * nseq * H * R::BYTES;
 
     CUtensorMap tq, tk, tg, tv, to;
     if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
@@ -1621,17 +1703,30 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
 
 }  // namespace split
 
+bool chunk_fwd_split_supported(int dk, int dv, kda_dtype dtype)
+{
+    return dtype == KDA_BF16 && (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
+}
+
+size_t chunk_fwd_split_workspace(int nseq, int T, long long tokens, int H, int dk, int dv, bool varlen, int mode)
+{
+    (void)mode;
+    return dk == 128 ? split::ws_layout<128>(nseq, T, tokens, H, dv, varlen).bytes
+                     : split::ws_layout<64>(nseq, T, tokens, H, dv, varlen).bytes;
+}
+
 cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const float* beta,
                             const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
                             int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
-                            long long timeout_cycles, int mode, cudaStream_t stream)
+                            long long timeout_cycles, int mode, void* ws, size_t ws_bytes, cudaStream_t stream)
 {
+    unsigned char* w = static_cast<unsigned char*>(ws);
     if (o_dtype == KDA_F32) {
-        if (dk == 128) return split::run<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, stream);
-        if (dk == 64) return split::run<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, stream);
+        if (dk == 128) return split::run<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 64) return split::run<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
     } else {
-        if (dk == 128) return split::run<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, stream);
-        if (dk == 64) return split::run<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, stream);
+        if (dk == 128) return split::run<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 64) return split::run<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
     }
     return cudaErrorInvalidValue;
 }

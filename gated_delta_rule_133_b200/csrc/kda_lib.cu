@@ -4,5 +4,4 @@
 #include "kda_api.cu"
 #include "kda_decode.cu"
 #include "kda_chunk_simt.cu"
-#include "kda_chunk_tc.cu"
 #include "kda_chunk_split.cu"

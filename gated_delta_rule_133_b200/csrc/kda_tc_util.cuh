@@ -29,34 +29,14 @@ __device__ __forceinline__ unsigned char* align1024(unsigned char* p)
     return p + (((a + 1023u) & ~1023u) - a);
 }
 
-// Rank-r sequence in longest-first order (ties: lower index first).
-__device__ int seq_by_rank(const int32_t* cu, int N, int rank, int* slot)
+// 1/x by the hardware reciprocal (PTX rcp.approx.ftz.f32: relative error
+// within 2^-23 for normal x; subnormal inputs and results flush to zero).
+// Used for factors e^(G_m - G) in [e^-80, e^80], whose products are then
+// rounded to tf32 (2^-11).
+__device__ __forceinline__ float rcp_approx(float x)
 {
-    if (threadIdx.x == 0) *slot = rank;
-    __syncthreads();
-    for (int i = threadIdx.x; i < N; i += blockDim.x) {
-        const int li = cu[i + 1] - cu[i];
-        int rk = 0;
-        for (int j = 0; j < N; ++j) {
-            const int lj = cu[j + 1] - cu[j];
-            rk += (lj > li) || (lj == li && j < i);
-        }
-        if (rk == rank) *slot = i;
-    }
-    __syncthreads();
-    const int n = *slot;
-    __syncthreads();
-    return n;
-}
-
-// 1/x for normal x by Newton-Raphson on the FMA pipe (keeps the exponent
-// unit free for exp): seed from the exponent bits (relative error < 5.1 %),
-// two iterations (< 1e-5, below tf32 resolution).
-__device__ __forceinline__ float rcp_nr(float x)
-{
-    float y = __int_as_float(0x7EF311C3 - __float_as_int(x));
-    y = y * fmaf(-x, y, 2.f);
-    y = y * fmaf(-x, y, 2.f);
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 

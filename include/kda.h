@@ -15,8 +15,16 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - Every tensor pointer is a DEVICE pointer owned by the caller; the library
- *    allocates no device memory and keeps no pointer after the call returns.
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller.  The
+ *    library allocates no device memory and keeps no pointer after the call
+ *    returns.  The tensor-core chunk forward needs scratch memory (per-chunk
+ *    operand records and a few index arrays): the caller passes it as
+ *    `workspace` / `workspace_bytes`, sized by kda_chunk_fwd_workspace_size() or
+ *    kda_varlen_fwd_workspace_size() for the same arguments.  The workspace is
+ *    used asynchronously on `stream` (it must stay allocated until the work
+ *    queued there has run) and its contents need no initialisation.  The one
+ *    exception is kda_chunk_fwd_noalloc(), which keeps its scratch in a fixed
+ *    library-owned area (see there).
  *  - Layouts are dense, row-major, token-major ("[B, T, H, d]": d fastest).
  *  - q, k and v have the element type `dtype` (KDA_BF16 or KDA_F32); the
  *    output o has the element type `o_dtype` (either, independently; KDA_F32
@@ -46,6 +54,7 @@
 #ifndef KDA_H
 #define KDA_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -78,6 +87,10 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
  *   o           [B, T, H, dv]  o_dtype, written
  *   final_state [B, H, dk, dv] fp32, or NULL if not wanted; written.  It may
  *               alias initial_state (in-place state update).
+ *   workspace   device scratch of at least kda_chunk_fwd_workspace_size()
+ *               bytes for these sizes (256-byte aligned), or NULL when that
+ *               size is 0; a smaller workspace_bytes returns
+ *               KDA_ERR_INVALID_ARG before anything is launched.
  *   B >= 0, T >= 0 (B*T == 0 is a no-op that still writes final_state from
  *   initial_state), H >= 1, chunk must be 64.
  */
@@ -85,7 +98,18 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          const float* beta, const float* log_alpha,
                          const float* initial_state, void* o, float* final_state,
                          int B, int T, int H, int dk, int dv, int chunk,
-                         kda_dtype dtype, kda_dtype o_dtype, void* stream);
+                         kda_dtype dtype, kda_dtype o_dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Bytes of workspace kda_chunk_fwd / kda_chunk_fwd_mode need for these
+ * arguments (`mode` as in kda_chunk_fwd_mode; 0 for the plain call), written
+ * to *bytes.  Pure host computation (it reads the current device's SM count);
+ * 0 when the call runs on the CUDA-core kernel.  Argument errors as in the
+ * forward call.
+ */
+kda_status kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
+                                        kda_dtype dtype, int mode, size_t* bytes);
 
 /*
  * kda_chunk_fwd computed without allocating any memory.  The method the pages
@@ -93,7 +117,7 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
  * only in where the tensor-core path keeps its intermediates (the per-chunk
  * operand records and, when final_state is NULL, the state carried between
  * blocks of chunks), namely a fixed 64 MiB area the library owns on each
- * device, instead of stream-ordered allocations.  Arguments, layouts and
+ * device, instead of a caller-provided workspace.  Arguments, layouts and
  * results are those of kda_chunk_fwd (results bit-identical to it).
  *
  *   - Problems whose records for one 64-token chunk of every (sequence, head),
@@ -119,17 +143,29 @@ kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
  *   q, k [T, H, dk], v [T, H, dv] (dtype), beta [T, H], log_alpha [T, H, dk],
  *   o [T, H, dv] (o_dtype)
  *   cu_seqlens  [N + 1] int32, DEVICE pointer, cu_seqlens[0] = 0,
- *               non-decreasing, cu_seqlens[N] = T (not checked on the device;
- *               a violation is undefined behaviour).
+ *               non-decreasing, cu_seqlens[N] = T.  The boundaries are read on
+ *               the device and guarded there: a sequence whose token range
+ *               leaves [0, T) is skipped (its o rows are not written, its
+ *               final state is its initial state) and the next kda_check()
+ *               reports KDA_ERR_INVALID_ARG; a decreasing pair counts as an
+ *               empty sequence; o rows outside every sequence are not written.
  *   initial_state / final_state [N, H, dk, dv] fp32 or NULL.
- *   N <= 65535.  Work is ordered longest sequence first.
+ *   workspace   as for kda_chunk_fwd, sized by kda_varlen_fwd_workspace_size().
+ *   N <= 65535.  The tensor-core path scans the longest sequences first (an
+ *   order computed on the device once per call).
  */
 kda_status kda_varlen_fwd(const void* q, const void* k, const void* v,
                           const float* beta, const float* log_alpha,
                           const int32_t* cu_seqlens, int N,
                           const float* initial_state, void* o, float* final_state,
                           int T, int H, int dk, int dv, int chunk,
-                          kda_dtype dtype, kda_dtype o_dtype, void* stream);
+                          kda_dtype dtype, kda_dtype o_dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of kda_varlen_fwd / kda_varlen_fwd_mode (see
+ * kda_chunk_fwd_workspace_size); T is the packed token count. */
+kda_status kda_varlen_fwd_workspace_size(int N, int T, int H, int dk, int dv, int chunk,
+                                         kda_dtype dtype, int mode, size_t* bytes);
 
 /*
  * One decode step of the recurrence for N independent sequences (one new
@@ -137,6 +173,7 @@ kda_status kda_varlen_fwd(const void* q, const void* k, const void* v,
  * Linear Attention Architecture: Making LLM Training and Inference More
  * Efficient", section 3.3, one state update and one state read per token
  * (its section I).  Memory bound: every state is read once and written once.
+ * Needs no workspace.
  *
  *   q, k [N, H, dk], v [N, H, dv]  dtype
  *   beta [N, H], log_alpha [N, H, dk]  fp32
@@ -173,6 +210,17 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
  *  KDA_MODE_GATE_LOGITS  log_alpha holds gate logits z: the layer uses
  *      log alpha = -softplus(z), i.e. alpha = sigmoid(-z).
  *
+ * Execution options of the chunk forwards (they change how, not what, is
+ * computed; used to cross-check the kernels against each other):
+ *
+ *  KDA_MODE_CUDA_CORES   run the fp32 CUDA-core kernel whatever the input
+ *      dtype (the reference-precision path; it needs no workspace).
+ *  KDA_MODE_BLOCKS(n)    tensor-core path, dense inputs: cut the chunk axis
+ *      into n blocks (1 <= n <= 8) and overlap the parallel pass of block b + 1
+ *      with the sequential pass of block b on a second stream; n = 1 runs the
+ *      parallel pass over every chunk, then the sequential pass.  Results are
+ *      bit-identical to the default schedule for every n.
+ *
  * The flags combine.  Every other argument, layout and rule is that of the
  * plain entry point of the same name.
  */
@@ -180,19 +228,23 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
 #define KDA_MODE_NO_ERASE 2
 #define KDA_MODE_NORM_QK 4
 #define KDA_MODE_GATE_LOGITS 8
+#define KDA_MODE_CUDA_CORES 16
+#define KDA_MODE_BLOCKS(n) ((n) << 8)
 
 kda_status kda_chunk_fwd_mode(const void* q, const void* k, const void* v,
                               const float* beta, const float* log_alpha,
                               const float* initial_state, void* o, float* final_state,
                               int B, int T, int H, int dk, int dv, int chunk,
-                              kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream);
+                              kda_dtype dtype, kda_dtype o_dtype, int mode,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 kda_status kda_varlen_fwd_mode(const void* q, const void* k, const void* v,
                                const float* beta, const float* log_alpha,
                                const int32_t* cu_seqlens, int N,
                                const float* initial_state, void* o, float* final_state,
                                int T, int H, int dk, int dv, int chunk,
-                               kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream);
+                               kda_dtype dtype, kda_dtype o_dtype, int mode,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 kda_status kda_recurrent_step_mode(const void* q, const void* k, const void* v,
                                    const float* beta, const float* log_alpha,

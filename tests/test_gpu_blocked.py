@@ -3,11 +3,10 @@
 For dense inputs the library splits the chunk axis into blocks: the prep pass
 of block b + 1 runs on a second stream while block b is scanned, and the state
 crosses block boundaries through memory as the same fp32 values it has in
-registers.  Every block count must therefore give results bit-identical to
-the single-block schedule (KDA_SCAN_BLOCKS=1), which itself matches the
-oracle.  The block count is read from the environment on every call.
+registers.  Every block count (KDA_MODE_BLOCKS(n), the ``blocks`` keyword)
+must therefore give results bit-identical to the single-block schedule, which
+itself matches the oracle.
 """
-import os
 
 import numpy as np
 import pytest
@@ -31,17 +30,9 @@ def _inputs(B, T, H, d, seed, init=0.05):
 
 def _call(g, blocks, initial_state="inputs", **kw):
     s0 = g["initial_state"] if isinstance(initial_state, str) else initial_state
-    old = os.environ.get("KDA_SCAN_BLOCKS")
-    os.environ["KDA_SCAN_BLOCKS"] = str(blocks)
-    try:
-        out = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], s0, **kw)
-        torch.cuda.synchronize()
-        kda.kda_check()
-    finally:
-        if old is None:
-            del os.environ["KDA_SCAN_BLOCKS"]
-        else:
-            os.environ["KDA_SCAN_BLOCKS"] = old
+    out = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], s0, blocks=blocks, **kw)
+    torch.cuda.synchronize()
+    kda.kda_check()
     return out
 
 
@@ -93,7 +84,6 @@ def test_blocked_bf16_output():
 def _call_coop(g, **kw):
     """Default schedule: one cooperative launch (prep CTAs publish records,
     scan CTAs consume them) whenever the scan grid leaves 32 SMs free."""
-    assert "KDA_SCAN_BLOCKS" not in os.environ
     out = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"], **kw)
     torch.cuda.synchronize()
     kda.kda_check()

@@ -203,16 +203,15 @@ def test_bf16_output_is_the_rounded_fp32_output():
 
 
 @pytest.mark.parametrize("d", [128, 64])
-def test_tensor_core_and_cuda_core_kernels_agree(monkeypatch, d):
-    """bf16 inputs go to the tcgen05 kernel; KDA_FORCE_SIMT=1 sends them to the
-    CUDA-core kernel.  Both meet the bar against the oracle and agree closely."""
+def test_tensor_core_and_cuda_core_kernels_agree(d):
+    """bf16 inputs go to the tcgen05 kernel; KDA_MODE_CUDA_CORES sends them to
+    the CUDA-core kernel.  Both meet the bar against the oracle."""
     w = Workload("case", "dense", 2, 333, 2, d, d, "bf16", -1.0, 0.05, seed=28)
     d_cpu = make_inputs(w, "cpu")
     g = _to(d_cpu, DEV)
     args = (g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"])
     o_tc, s_tc = kda.kda_chunk_fwd(*args)
-    monkeypatch.setenv("KDA_FORCE_SIMT", "1")
-    o_cc, s_cc = kda.kda_chunk_fwd(*args)
+    o_cc, s_cc = kda.kda_chunk_fwd(*args, cuda_cores=True)
     torch.cuda.synchronize()
     o_ref, s_ref = _dense_oracle(d_cpu, 2, 333)
     flat = lambda t: f64(t).reshape(2 * 333, 2, d)

@@ -116,19 +116,6 @@ def test_recurrent_step_variants(head_gate, erase, dtype):
         assert norm_max_err(f64(state), S_ref) <= tol
 
 
-def test_single_pass_kernel_setting_runs_variants_on_the_two_pass_kernels(monkeypatch):
-    """KDA_CHUNK_KERNEL=fused selects a kernel that implements the plain layer
-    only; a variant then runs on the default kernels and gives their result."""
-    B, T, H, d = 1, 130, 2, 128
-    x = make_inputs(Workload("variant", "dense", B, T, H, d, d, "bf16", -2.0, 0.05, seed=66), "cpu")
-    g = {n: (None if t is None else t.to(DEV)) for n, t in x.items()}
-    o1, s1 = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"], erase=False)
-    monkeypatch.setenv("KDA_CHUNK_KERNEL", "fused")
-    o2, s2 = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"], erase=False)
-    torch.cuda.synchronize()
-    assert torch.equal(o1, o2) and torch.equal(s1, s2)
-
-
 def _raw(x, seed):
     """Raw projections: q, k rows scaled by random factors (0.2 .. 5) and gate
     logits z with log alpha = -softplus(z) (z ~ N(-3, 1), the generator's)."""

@@ -61,8 +61,30 @@ def test_noalloc_in_place_state():
     assert torch.equal(st, s1)
 
 
+def test_noalloc_in_place_state_across_ring_blocks():
+    """256 (sequence, head) pairs, 11 chunks: 2 chunks per block, 6 blocks, each
+    block reading and writing the caller's state in place."""
+    g = _inputs(4, 657, 64, 128, seed=65)
+    o1, s1 = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"])
+    st = g["initial_state"].clone()
+    o2, _ = kda.kda_chunk_fwd_noalloc(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], st, final_state=st)
+    torch.cuda.synchronize()
+    kda.kda_check()
+    assert torch.equal(o2, o1)
+    assert torch.equal(st, s1)
+
+
+def test_noalloc_single_block_needs_no_second_slot():
+    """1000 (sequence, head) pairs of one chunk, no final state: the records of
+    one block fill most of the area, which is enough when there is one block."""
+    g = _inputs(10, 50, 100, 128, seed=66)
+    (o1, _), (o2, s2) = _both(g, output_final_state=False)
+    assert s2 is None
+    assert torch.equal(o2, o1)
+
+
 def test_noalloc_rejects_oversize():
-    g = _inputs(10, 64, 64, 128, seed=63)
+    g = _inputs(20, 64, 64, 128, seed=63)
     with pytest.raises(_lib.KdaError) as e:
         kda.kda_chunk_fwd_noalloc(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"])
     assert e.value.status == _lib.KDA_ERR_UNSUPPORTED
