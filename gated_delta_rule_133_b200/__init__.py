@@ -32,7 +32,7 @@ from . import _lib
 from ._lib import KdaError
 
 __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_varlen_fwd", "kda_recurrent_step", "kda_check",
-           "chunk_fwd_workspace_size", "varlen_fwd_workspace_size", "KdaError"]
+           "kda_chunk_bwd", "kda_varlen_bwd", "chunk_fwd_workspace_size", "varlen_fwd_workspace_size", "KdaError"]
 
 _DTYPES = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
 
@@ -211,6 +211,68 @@ def kda_recurrent_step(q, k, v, beta, log_alpha, state, *, o=None, o_dtype=torch
               _ptr(beta), _ptr(log_alpha), _ptr(state), _ptr(o), N, H, dk, dv, _DTYPES[dt], _DTYPES[o.dtype],
               *((mode,) if mode else ()), _stream(stream))
     return o
+
+
+def _bwd_outputs(q, v, beta, nstates, H, dk, dv, want_ds0):
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = (torch.empty(q.shape, **f32), torch.empty(q.shape, **f32), torch.empty(v.shape, **f32),
+             torch.empty(beta.shape, **f32), torch.empty(q.shape, **f32))
+    ds0 = torch.empty(nstates, H, dk, dv, **f32) if want_ds0 else None
+    return grads, ds0
+
+
+def kda_chunk_bwd(q, k, v, beta, log_alpha, initial_state, grad_o, grad_final_state=None, *,
+                  want_initial_state_grad=True, chunk=64, stream=None, workspace=None):
+    """Backward of kda_chunk_fwd: gradients of sum(o * grad_o) + sum(S_T * grad_final_state).
+
+    Inputs as for kda_chunk_fwd (plain layer); grad_o [B, T, H, dv] fp32,
+    grad_final_state [B, H, dk, dv] fp32 or None.  Returns fp32
+    (dq, dk, dv, dbeta, dlog_alpha, dinitial_state or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for t, n, s_, d in ((q, "q", (B, T, H, dk), dt), (k, "k", (B, T, H, dk), dt), (v, "v", (B, T, H, dv), dt),
+                        (beta, "beta", (B, T, H), torch.float32), (log_alpha, "log_alpha", (B, T, H, dk), torch.float32),
+                        (grad_o, "grad_o", (B, T, H, dv), torch.float32)):
+        _check(t, n, s_, d, dev)
+    for t, n in ((initial_state, "initial_state"), (grad_final_state, "grad_final_state")):
+        if t is not None:
+            _check(t, n, (B, H, dk, dv), torch.float32, dev)
+    (gq, gk, gv, gb, gla), gs0 = _bwd_outputs(q, v, beta, B, H, dk, dv, want_initial_state_grad)
+    nbytes = _lib.workspace_size("kda_chunk_bwd_workspace_size", B, T, H, dk, dv, chunk, _DTYPES[dt])
+    ws = _workspace(nbytes, workspace, dev)
+    _lib.call("kda_chunk_bwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha), _ptr(initial_state),
+              _ptr(grad_o), _ptr(grad_final_state), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gb), _ptr(gla), _ptr(gs0),
+              B, T, H, dk, dv, chunk, _DTYPES[dt], *ws, _stream(stream))
+    return gq, gk, gv, gb, gla, gs0
+
+
+def kda_varlen_bwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state, grad_o, grad_final_state=None, *,
+                   want_initial_state_grad=True, chunk=64, stream=None, workspace=None):
+    """Backward of kda_varlen_fwd (packed [T, H, ...] layouts, states [N, H, dk, dv])."""
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.shape[0] - 1
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for t, n, s_, d in ((q, "q", (T, H, dk), dt), (k, "k", (T, H, dk), dt), (v, "v", (T, H, dv), dt),
+                        (beta, "beta", (T, H), torch.float32), (log_alpha, "log_alpha", (T, H, dk), torch.float32),
+                        (grad_o, "grad_o", (T, H, dv), torch.float32), (cu_seqlens, "cu_seqlens", (N + 1,), torch.int32)):
+        _check(t, n, s_, d, dev)
+    for t, n in ((initial_state, "initial_state"), (grad_final_state, "grad_final_state")):
+        if t is not None:
+            _check(t, n, (N, H, dk, dv), torch.float32, dev)
+    (gq, gk, gv, gb, gla), gs0 = _bwd_outputs(q, v, beta, N, H, dk, dv, want_initial_state_grad)
+    nbytes = _lib.workspace_size("kda_varlen_bwd_workspace_size", N, T, H, dk, dv, chunk, _DTYPES[dt])
+    ws = _workspace(nbytes, workspace, dev)
+    _lib.call("kda_varlen_bwd", _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha), _ptr(cu_seqlens), N,
+              _ptr(initial_state), _ptr(grad_o), _ptr(grad_final_state), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gb),
+              _ptr(gla), _ptr(gs0), T, H, dk, dv, chunk, _DTYPES[dt], *ws, _stream(stream))
+    return gq, gk, gv, gb, gla, gs0
 
 
 def kda_check(stream=None):

@@ -38,6 +38,10 @@ SIGNATURES = {
     "kda_varlen_fwd_mode": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _Z,
                                  _P]),
     "kda_recurrent_step_mode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_chunk_bwd": (_I, [_P] * 14 + [_I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    "kda_chunk_bwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _ZP]),
+    "kda_varlen_bwd": (_I, [_P] * 6 + [_I] + [_P] * 9 + [_I, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    "kda_varlen_bwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _ZP]),
     "kda_check": (_I, [_P]),
     "kda_selftest_timeout": (_I, [ctypes.c_longlong, _P]),
     "kda_status_string": (ctypes.c_char_p, [_I]),

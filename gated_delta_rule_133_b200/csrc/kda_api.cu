@@ -248,6 +248,94 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
     return kda_recurrent_step_mode(q, k, v, beta, log_alpha, state, o, N, H, dk, dv, dtype, o_dtype, 0, stream);
 }
 
+kda_status kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                                        size_t* bytes)
+{
+    if (!bytes || B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    const kda_status st = check_sizes(H, dk, dv, chunk, dtype, 0);
+    if (st != KDA_OK) return st;
+    const long long tokens = (long long)B * T;
+    if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    *bytes = tokens == 0 ? 0 : kda::chunk_bwd_workspace(B, T, tokens, H, dk, dv, false);
+    return KDA_OK;
+}
+
+kda_status kda_varlen_bwd_workspace_size(int N, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                                         size_t* bytes)
+{
+    if (!bytes || N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
+    const kda_status st = check_sizes(H, dk, dv, chunk, dtype, 0);
+    if (st != KDA_OK) return st;
+    *bytes = (N == 0 || T == 0) ? 0 : kda::chunk_bwd_workspace(N, 0, T, H, dk, dv, true);
+    return KDA_OK;
+}
+
+namespace {
+
+kda_status check_bwd(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
+                     const float* s0, const float* go, const float* gsT, const float* gq, const float* gk,
+                     const float* gv, const float* gb, const float* gla, const float* gs0, long long tokens, int H,
+                     int dk, int dv, int chunk, kda_dtype dtype)
+{
+    if (H <= 0 || dk <= 0 || dv <= 0 || tokens < 0 || !valid_dtype(dtype)) return KDA_ERR_INVALID_ARG;
+    if (tokens > 0) {
+        if (!q || !k || !v || !beta || !log_alpha || !go || !gq || !gk || !gv || !gb || !gla)
+            return KDA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(beta) || !aligned16(log_alpha) ||
+            !aligned16(go) || !aligned16(gq) || !aligned16(gk) || !aligned16(gv) || !aligned4(gb) || !aligned16(gla))
+            return KDA_ERR_INVALID_ARG;
+    }
+    if ((s0 && !aligned16(s0)) || (gsT && !aligned16(gsT)) || (gs0 && !aligned16(gs0))) return KDA_ERR_INVALID_ARG;
+    if (chunk != 64 || !supported_d(dk) || !supported_d(dv)) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+}  // namespace
+
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
+                         const float* initial_state, const float* grad_o, const float* grad_final_state,
+                         float* grad_q, float* grad_k, float* grad_v, float* grad_beta, float* grad_log_alpha,
+                         float* grad_initial_state, int B, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                         void* workspace, size_t workspace_bytes_, void* stream)
+{
+    if (B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    const long long tokens = (long long)B * T;
+    kda_status st = check_bwd(q, k, v, beta, log_alpha, initial_state, grad_o, grad_final_state, grad_q, grad_k,
+                              grad_v, grad_beta, grad_log_alpha, grad_initial_state, tokens, H, dk, dv, chunk, dtype);
+    if (st != KDA_OK) return st;
+    if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    const size_t need = tokens == 0 ? 0 : kda::chunk_bwd_workspace(B, T, tokens, H, dk, dv, false);
+    st = check_workspace(workspace, workspace_bytes_, need);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tokens == 0) return copy_state(grad_final_state, grad_initial_state, (size_t)B * H * dk * dv, s);
+    return from_cuda(kda::chunk_bwd(q, k, v, beta, log_alpha, initial_state, grad_o, grad_final_state, grad_q, grad_k,
+                                    grad_v, grad_beta, grad_log_alpha, grad_initial_state, nullptr, B, T, tokens, H, dk,
+                                    dv, dtype, workspace, workspace_bytes_, s));
+}
+
+kda_status kda_varlen_bwd(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
+                          const int32_t* cu_seqlens, int N, const float* initial_state, const float* grad_o,
+                          const float* grad_final_state, float* grad_q, float* grad_k, float* grad_v,
+                          float* grad_beta, float* grad_log_alpha, float* grad_initial_state, int T, int H, int dk,
+                          int dv, int chunk, kda_dtype dtype, void* workspace, size_t workspace_bytes_, void* stream)
+{
+    if (N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_bwd(q, k, v, beta, log_alpha, initial_state, grad_o, grad_final_state, grad_q, grad_k,
+                              grad_v, grad_beta, grad_log_alpha, grad_initial_state, T, H, dk, dv, chunk, dtype);
+    if (st != KDA_OK) return st;
+    if (N == 0) return T == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
+    if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARG;
+    const size_t need = T == 0 ? 0 : kda::chunk_bwd_workspace(N, 0, T, H, dk, dv, true);
+    st = check_workspace(workspace, workspace_bytes_, need);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) return copy_state(grad_final_state, grad_initial_state, (size_t)N * H * dk * dv, s);
+    return from_cuda(kda::chunk_bwd(q, k, v, beta, log_alpha, initial_state, grad_o, grad_final_state, grad_q, grad_k,
+                                    grad_v, grad_beta, grad_log_alpha, grad_initial_state, cu_seqlens, N, 0, T, H, dk,
+                                    dv, dtype, workspace, workspace_bytes_, s));
+}
+
 kda_status kda_check(void* stream)
 {
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -42,4 +42,14 @@ cudaError_t chunk_fwd_noalloc(const void* q, const void* k, const void* v, const
                               long long tokens, int H, int dk, int dv, kda_dtype o_dtype, long long timeout_cycles,
                               cudaStream_t stream);
 
+// Chunkwise backward on CUDA cores (fp32): gradients of sum(o * dout) +
+// sum(S_T * dsT) into fp32 dq, dk, dv, dbeta, dla (the library zeroes the
+// accumulated ones) and ds0 (or nullptr).  chunk_bwd_workspace gives the bytes
+// of workspace a call needs.
+size_t chunk_bwd_workspace(int nseq, int T, long long tokens, int H, int dk, int dv, bool varlen);
+cudaError_t chunk_bwd(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
+                      const float* s0, const float* dout, const float* dsT, float* dq, float* dk, float* dv,
+                      float* dbeta, float* dla, float* ds0, const int32_t* cu, int nseq, int T, long long tokens,
+                      int H, int dkd, int dvd, kda_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 }  // namespace kda

@@ -702,7 +702,11 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
             float pt[16];
             tmem_ld16(t_PT + lane_off + q_off, pt);
             tmem_wait_ld();
-            if (lt < DK) st_row_h16(stg, lt, 16 * wg, DK, z);
+            if (lt < DK) {   // the record keeps Z diag(beta)
+#pragma unroll
+                for (int j = 0; j < 16; ++j) z[j] *= vcur.beta[16 * wg + j];
+                st_row_h16(stg, lt, 16 * wg, DK, z);
+            }
             if (lt < C) st_row_h16(stg + (R::PT - R::Z), lt, 16 * wg, C, pt);
             if (tid < DK) reinterpret_cast<float*>(stg + (R::EGL - R::Z))[tid] = vcur.egl[tid];
             else if (tid >= 256 && tid < 256 + C) reinterpret_cast<float*>(stg + (R::BETA - R::Z))[tid - 256] = vcur.beta[tid - 256];
@@ -766,127 +770,104 @@ struct ScanParams {
     int no_erase;            // KDA_MODE_NO_ERASE: Y = beta V (no X term)
 };
 
-// Shared memory of the scan kernel: two 72 KB slots, each holding one record
-// (the M = 128 reads of the 64-row PT tile, and for d_k = 64 of the Z tile,
-// run on into the rest of the record's 64 KB, into rows whose products are
-// discarded) and the chunk's V tile [64][NV] (bf16, 128-byte swizzle) at
-// +64 KB; the state operand S [d_k][NV] and Y [64][NV] (fp16, MN-major B
-// operands: value columns contiguous, 128-byte swizzle); the o staging tile
-// [64][NV] (output type, 16-byte chunks XOR-swizzled by row).
-template <int DK>
+// Shared memory of the scan kernel (one CTA per (sequence, head), all d_v
+// columns).  Two record slots, each holding one record as stored followed by
+// the chunk's V tile [64][DV] (bf16 from TMA, converted to fp16 in place; the
+// M = 128 reads of the 64-row PT tile, and for d_k = 64 of the Z tile, run on
+// into rows whose products are discarded); the state operand S [DK][DV] twice
+// (fp16, MN-major: value columns contiguous, 128-byte swizzle); Y [64][DV]
+// (fp16, MN-major).  The mbarriers sit in the gap between slot 0's record and
+// its V tile.
+template <int DK, int DV>
 struct ScanPlan {
-    static constexpr int SLOT = 73728, VOFF = 65536;
+    static constexpr int VOFF = (Rec<DK>::BYTES + 1023) & ~1023;
+    static constexpr int SLOT = VOFF + C * DV * 2;
     static constexpr int SOP = 2 * SLOT;
-    static constexpr int YB = SOP + NV * DK * 2;
-    static constexpr int OST = YB + NV * C * 2;
-    static constexpr int BAR = OST + C * NV * 4;
-    static constexpr int END = BAR + 128;
+    static constexpr int YB = SOP + 2 * DK * DV * 2;
+    static constexpr int END = YB + C * DV * 2;
+    static constexpr int BAR = Rec<DK>::BYTES;
     static constexpr int BYTES = END + 1024;
 };
+static_assert(ScanPlan<128, 128>::BYTES <= 232448, "scan shared memory exceeds the per-CTA limit");
+static_assert(ScanPlan<128, 128>::VOFF - ScanPlan<128, 128>::BAR >= 128, "no room for the scan's barriers");
+static_assert(ScanPlan<64, 128>::VOFF - ScanPlan<64, 128>::BAR >= 128, "no room for the scan's barriers");
 
-// MN-major SW128 B operand (16-bit, NV = 64 columns = one 128-byte row per K
-// index): K-step kk (16 K rows = two 1 KB groups) starts 2 KB further on.
-__device__ __forceinline__ uint64_t mn_desc(const unsigned char* tile, int kk, int k_rows)
+// MN-major SW128 16-bit operand: K-step kk (16 K rows = two 1 KB groups)
+// starts 2 KB further on; 64-column atoms `atom_stride` bytes apart.
+__device__ __forceinline__ uint64_t mn_desc(const unsigned char* tile, int kk, int atom_stride)
 {
-    return sdesc_sw128(smem_u32(tile) + kk * 2048, (uint32_t)(k_rows * 128), 1024);
+    return sdesc_sw128(smem_u32(tile) + kk * 2048, (uint32_t)atom_stride, 1024);
 }
 
-// Output rows [0, L) of one chunk from the TMEM accumulator (lane = row, 16
-// columns per warpgroup), run by the 256 threads of lanes 0..63.  Rows are
-// staged in the layout of the output tensor map's boxes (64 rows x 128 bytes,
-// 128-byte swizzle; two boxes for fp32 output); a full chunk leaves with TMA
-// stores issued by one thread, a partial one (the end of a sequence) with
-// coalesced 16-byte row-segment stores.
-template <typename TO>
-__device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost, const CUtensorMap* tmo, void* o,
-                                             int tok, int h, int col0, size_t row0_off, size_t row_stride, int L,
-                                             int lt, int wg, bool issuer)
+// Stores NC consecutive values of one row of a 16-bit SW128 tile as fp16
+// (col0 a multiple of 8).
+template <int NC>
+__device__ __forceinline__ void st_row_h16n(unsigned char* tile, int row, int col0, int rows, const float* x)
 {
-    constexpr int EB = (int)sizeof(TO);
-    constexpr int CPB = 8;                 // 16-byte chunks per 128-byte box row
-    constexpr int CPT = EB;                // chunks per thread: 16 values
-    constexpr int NBOX = NV * EB / 128;
-    constexpr int CPR = NV * EB / 16;      // chunks per output row segment
-    float acc[16];
-    tmem_ld16(t_acc, acc);
-    if (issuer) bulk_wait_read();          // the previous chunk's stores have read the tile
-    tmem_wait_ld();
-    bar_sync(1, 256);
 #pragma unroll
-    for (int u = 0; u < CPT; ++u) {
-        const int k = wg * CPT + u, box = k / CPB, ci = k % CPB;
-        uint4 val;
-        if constexpr (EB == 4)
-            val = make_uint4(__float_as_uint(acc[4 * u]), __float_as_uint(acc[4 * u + 1]),
-                             __float_as_uint(acc[4 * u + 2]), __float_as_uint(acc[4 * u + 3]));
-        else
-            val = make_uint4(pack_bf16(acc[8 * u], acc[8 * u + 1]), pack_bf16(acc[8 * u + 2], acc[8 * u + 3]),
-                             pack_bf16(acc[8 * u + 4], acc[8 * u + 5]), pack_bf16(acc[8 * u + 6], acc[8 * u + 7]));
-        *reinterpret_cast<uint4*>(ost + box * 8192 + lt * 128 + ((ci ^ (lt & 7)) << 4)) = val;
-    }
-    fence_proxy_async();
-    bar_sync(1, 256);
-    if (L == C) {
-        if (issuer) {
-#pragma unroll
-            for (int bx = 0; bx < NBOX; ++bx) tma_store_3d(tmo, ost + bx * 8192, col0 + bx * (128 / EB), h, tok);
-            bulk_commit();
-        }
-    } else {
-        const int t = wg * 64 + lt;
-#pragma unroll
-        for (int pss = 0; pss < C * CPR / 256; ++pss) {
-            const int idx = pss * 256 + t, row = idx / CPR, k = idx % CPR;
-            if (row < L) {
-                const int box = k / CPB, ci = k % CPB;
-                const uint4 val = *reinterpret_cast<const uint4*>(ost + box * 8192 + row * 128 + ((ci ^ (row & 7)) << 4));
-                *reinterpret_cast<uint4*>(static_cast<unsigned char*>(o) + (row0_off + (size_t)row * row_stride) * EB + k * 16) = val;
-            }
-        }
-    }
+    for (int u = 0; u < NC / 8; ++u)
+        *reinterpret_cast<uint4*>(tile + swh_off(row, col0 + 8 * u, rows)) =
+            make_uint4(pack_f16(x[8 * u], x[8 * u + 1]), pack_f16(x[8 * u + 2], x[8 * u + 3]),
+                       pack_f16(x[8 * u + 4], x[8 * u + 5]), pack_f16(x[8 * u + 6], x[8 * u + 7]));
 }
 
-// One CTA per (sequence, head, NV value columns).  Thread (lane lt < d_k,
-// warpgroup wg) keeps S[lt][16 wg .. 16 wg + 16) of the state in registers.
-// Per chunk c (slot c % 2):
-//   S <- diag(e^G_last(c-1)) S + W(c-1)      W = Z Y of the chunk before, from TMEM
-//   S operand (fp16) -> smem;  MMA [O ; X] = [Qh ; Kh] S  -> TMEM buffer c % 2
-//   Y = diag(beta) (V - X) -> smem (lanes 64..127), while lanes 0..63 store
-//   the o rows of chunk c - 1
-//   MMA W = Z Y (commit), MMA O += PT Y
-// A slot is refilled in two parts as soon as the MMAs reading each part have
-// completed: the [Qh ; Kh] tile and V after chunk c's X MMA and Y phase, the
-// Z, PT, e^G_last and beta part after chunk c + 1's X MMA (tcgen05 MMAs of
-// one thread complete in issue order).
-template <typename TO, int DK, bool VAR>
-__device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensorMap& tmo, const ScanParams& p,
-                                          int bid)
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[N])
+{
+    if constexpr (N == 32) tmem_ld32(taddr, v);
+    else tmem_ld16(taddr, v);
+}
+
+// One CTA per (sequence, head).  The state update of a chunk is one MMA
+// round on the critical path:
+//
+//   S_{c+1} = diag(e^G_last) S_c + M'_c S_c + B_c,
+//   M'_c = -(Z diag(beta)) Kh  (d_k x d_k),   B_c = (Z diag(beta)) V  (d_k x d_v)
+//
+// (the record's Z tile already carries the beta factors).  M'_c and B_c depend
+// on the chunk alone: they are formed by MMAs issued a chunk ahead, M'_c
+// converted to fp16 in TMEM (the A operand of a TS-form MMA) and B_c left in
+// the accumulator the chain MMA adds to.  The output leaves the chain:
+// [O ; X] = [Qh ; Kh] S_c, Y = beta (V - X), O += PT Y.
+//
+// Thread (warp w, lane l) owns state row 32 (w % 4) + l (the TMEM lane its
+// warp may access) and the NC = DV / 4 value columns of its warpgroup, in
+// fp32 registers.  TMEM columns: D_S[2] (0, 128), D_O (256), D_M (384; M'
+// packed over its first DK / 2 columns).
+//
+// Per chunk c (record in slot c % 2):
+//   (A) S_c from D_S of chunk c - 1, its fp16 operand to S_op[c % 2]
+//   (B) chain MMA D_S[c % 2] += M'_c S_op; X/O MMA D_O = [Qh ; Kh] S_op
+//   (C) chunk c + 1: V tile to fp16, MMAs D_M = Zb Kh, D_S[(c+1) % 2] = Zb V
+//   (D) Y = beta (V - X) (lanes 64..127); MMA D_O += PT Y
+//   (F) M'_{c+1} = -D_M to fp16 in TMEM
+//   (E) o rows of chunk c (lanes 0..63); slot c % 2 refilled with chunk c + 2
+template <typename TO, int DK, int DV, bool VAR>
+__device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const ScanParams& p, int bid)
 {
     const bool no_erase = VAR && p.no_erase;   // layer variant (VAR instantiations only)
-    using PL = ScanPlan<DK>;
+    using PL = ScanPlan<DK, DV>;
     using R = Rec<DK>;
+    constexpr int NC = DV / 4;                 // value columns per warpgroup
     extern __shared__ unsigned char smem_raw[];
     KDA_PHASE_DECL(1)
     unsigned char* sm = align1024(smem_raw);
-    unsigned char* Sop = sm + PL::SOP;
     unsigned char* Yb = sm + PL::YB;
-    unsigned char* Ost = sm + PL::OST;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::BAR);
-    uint64_t* mb_a = bars + 0;     // [2]: [Qh ; Kh] and V of a slot
-    uint64_t* mb_b = bars + 2;     // [2]: Z, PT, e^G_last and beta of a slot
-    uint64_t* mb_x = bars + 4;
-    uint64_t* mb_w = bars + 5;
+    uint64_t* mb_rec = bars + 0;   // [2]: record + V tile of a slot
+    uint64_t* mb_chain = bars + 2;
+    uint64_t* mb_xo = bars + 3;
+    uint64_t* mb_m = bars + 4;
+    uint64_t* mb_o = bars + 5;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int lt = tid & 127;
+    const int lt = (warp & 3) * 32 + (tid & 31);   // TMEM lane of this thread
     const int wg = tid >> 7;
-    const int nslice = p.DV / NV;
-    const int slice = bid % nslice;
-    const int h = (bid / nslice) % p.H;
-    const int rank = bid / (nslice * p.H);
-    const int H = p.H, DV = p.DV;
+    const int h = bid % p.H;
+    const int rank = bid / p.H;
+    const int H = p.H;
     int n, tok0, len;
     long long j0;
     if (p.cu) {
@@ -900,7 +881,6 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
         len = p.T;
         j0 = (long long)n * p.rs - p.rc0;
     }
-    const int col0 = slice * NV;
     int nchunks = (len + C - 1) / C;
     if ((long long)tok0 + len > p.tokens || tok0 < 0) {
         if (tid == 0 && p.c_begin == 0) flag_bad_input();
@@ -921,7 +901,6 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
         nchunks = 0;
         len = 0;
     }
-    const float* s_src = p.s_in;
 
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
@@ -929,10 +908,9 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
         prefetch_tmap(&tmv);
-        prefetch_tmap(&tmo);
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -940,188 +918,267 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_off = ((uint32_t)(warp & 3) * 32) << 16;
-    const uint32_t q_off = (uint32_t)wg * 16;
-    const uint32_t t_W = tmem + 128;
-    constexpr uint32_t kI = idesc_f16(128, NV, 1);
-    constexpr uint32_t kBytesA = R::Z + C * NV * 2;     // [Qh ; Kh] tile + V tile
-    constexpr uint32_t kBytesB = R::BYTES - R::Z;       // Z, PT, e^G_last, beta
+    const uint32_t t_O = tmem + 256, t_M = tmem + 384;
+    constexpr uint32_t kIdv = idesc_f16(128, DV, 1);    // N = d_v, B MN-major
+    constexpr uint32_t kIdk = idesc_f16(128, DK, 1);    // N = d_k, B MN-major
+    constexpr uint32_t kRecBytes = (uint32_t)R::BYTES + C * DV * 2;
 
-    auto rec_of = [&](int cc) { return p.rec + ((size_t)(j0 + cc) * H + h) * R::BYTES; };
-    auto issue_a = [&](int cc) {
-        unsigned char* slot = sm + (cc & 1) * PL::SLOT;
-        if (p.ready && !wait_ready(p.ready + (size_t)(j0 + cc) * H + h, abort_flag, p.timeout_cycles)) return;
-        mbar_expect_tx(mb_a + (cc & 1), kBytesA);
-        bulk_load(slot, rec_of(cc), R::Z, mb_a + (cc & 1));
-        tma_load_3d(slot + PL::VOFF, &tmv, mb_a + (cc & 1), col0, h, tok0 + cc * C);
-    };
-    auto issue_b = [&](int cc) {
-        unsigned char* slot = sm + (cc & 1) * PL::SLOT;
-        mbar_expect_tx(mb_b + (cc & 1), kBytesB);
-        bulk_load(slot + R::Z, rec_of(cc) + R::Z, kBytesB, mb_b + (cc & 1));
-    };
-
-    // state rows of this thread
-    float S[16];
-    {
-        const bool own = lt < DK && s_src;
-        const float* src = own ? s_src + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg : nullptr;
+    auto slot_of = [&](int cc) { return sm + (cc & 1) * PL::SLOT; };
+    auto issue_rec = [&](int cc) {   // one thread: record and V tile of chunk cc into its slot
+        unsigned char* slot = slot_of(cc);
+        const size_t ri = (size_t)(j0 + cc) * H + h;
+        if (p.ready && !wait_ready(p.ready + ri, abort_flag, p.timeout_cycles)) return;
+        mbar_expect_tx(mb_rec + (cc & 1), kRecBytes);
+        bulk_load(slot, p.rec + ri * R::BYTES, (uint32_t)R::BYTES, mb_rec + (cc & 1));
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) {
+        for (int a = 0; a < DV / 64; ++a)
+            tma_load_3d(slot + PL::VOFF + a * 8192, &tmv, mb_rec + (cc & 1), 64 * a, h, tok0 + cc * C);
+    };
+    // V tile of a slot from bf16 to fp16 in place (all threads, 16 bytes each per pass)
+    auto convert_v = [&](unsigned char* slot) {
+        uint4* vt = reinterpret_cast<uint4*>(slot + PL::VOFF);
+#pragma unroll
+        for (int i = tid; i < C * DV * 2 / 16; i += NT) {
+            uint4 u = vt[i];
+            uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                w[e] = pack_f16(f.x, f.y);
+            }
+            vt[i] = u;
+        }
+    };
+    // MMAs of the state-independent terms of chunk cc: D_M = Zb Kh, D_S[cc % 2] = Zb V (one thread)
+    auto issue_chunk_terms = [&](int cc) {
+        const unsigned char* slot = slot_of(cc);
+        if (!no_erase) {
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_f16(t_M, kdesc(slot + R::Z, kk, 0), mn_desc(slot + R::QK + C * 128 + 0, kk, 128 * 128), kIdk,
+                         kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+            umma_f16(tmem + 128 * (cc & 1), kdesc(slot + R::Z, kk, 0), mn_desc(slot + PL::VOFF, kk, C * 128), kIdv,
+                     kk > 0);
+        umma_commit(mb_m);
+    };
+    // M' = -D_M to packed fp16 in TMEM (A operand of the chain MMA); the four
+    // warps sharing a lane quadrant read all their columns before any writes
+    auto convert_m = [&]() {
+        constexpr int MC = DK / 4;   // D_M columns per warpgroup
+        float m[MC];
+        tmem_ldn<MC>(t_M + lane_off + (uint32_t)(wg * MC), m);
+        tmem_wait_ld();
+        bar_sync(2 + (warp & 3), 128);
+        uint32_t pk[MC / 2];
+#pragma unroll
+        for (int i = 0; i < MC / 2; ++i) pk[i] = pack_f16(-m[2 * i], -m[2 * i + 1]);
+        if constexpr (MC == 32) {
+            tmem_st8(t_M + lane_off + (uint32_t)(wg * 16), *reinterpret_cast<const uint32_t(*)[8]>(pk));
+            tmem_st8(t_M + lane_off + (uint32_t)(wg * 16 + 8), *reinterpret_cast<const uint32_t(*)[8]>(pk + 8));
+        } else {
+            tmem_st8(t_M + lane_off + (uint32_t)(wg * 8), *reinterpret_cast<const uint32_t(*)[8]>(pk));
+        }
+        tmem_wait_st();
+    };
+
+    // state rows of this thread (rows >= DK unused)
+    float S[NC];
+    {
+        const bool own = lt < DK && p.s_in;
+        const float* src = own ? p.s_in + (((size_t)n * H + h) * DK + lt) * DV + wg * NC : nullptr;
+#pragma unroll
+        for (int j = 0; j < NC; j += 4) {
             const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
             S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
         }
     }
 
-    // thread 0 issues the MMAs; thread kIssuer every copy (record refills, V
-    // tiles, output stores)
-    constexpr int kIssuer = 32;
-    const bool issuer = tid == kIssuer;
-    unsigned pend = 0;                 // bits: 0-1 mb_a[slot], 2-3 mb_b[slot], 4 mb_x, 5 mb_w
-    uint32_t apar = 0u, bpar = 0u;     // bit i: phase parity of the pending load of slot i
-    int xph = 0, wph = 0;              // commits issued to mb_x / mb_w
+    constexpr int kMma = 0, kCopy = 32;        // MMA issuer and copy issuer threads
+    unsigned pend = 0;                         // bits: 0-1 mb_rec[slot], 2 chain, 3 xo, 4 m, 5 o
+    uint32_t rpar = 0u;                        // bit i: phase parity of the pending load of slot i
+    int nchain = 0, nxo = 0, nm = 0, no = 0;   // commits issued to mb_chain / mb_xo / mb_m / mb_o
+    float egl = 1.f;                           // e^G_last of the chunk before, row lt
     int c = 0;
-    if (issuer)
-        for (int cc = 0; cc < 2 && cc < nchunks; ++cc) {
-            issue_a(cc);
-            issue_b(cc);
-        }
-    for (int cc = 0; cc < 2 && cc < nchunks; ++cc) pend |= (1u | 4u) << cc;
 
-    float eglp = 1.f;                  // e^G_last of the previous chunk, key channel lt
-    int Lprev = 0;
+    if (nchunks > 0) {
+        if (tid == kCopy) {
+            issue_rec(0);
+            if (nchunks > 1) issue_rec(1);
+        }
+        pend |= 1u | (nchunks > 1 ? 2u : 0u);
+        rpar = 0u;
+        KDA_WAIT_OR_EXIT(mb_rec, 1u, 0u);
+        convert_v(slot_of(0));
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == kMma) {
+            tc_fence_after();
+            issue_chunk_terms(0);
+        }
+        ++nm;
+        pend |= 16u;
+        KDA_WAIT_OR_EXIT(mb_m, 16u, 0u);
+        tc_fence_after();
+        if (!no_erase) convert_m();
+    }
+
     for (c = 0; c < nchunks; ++c) {
         const int b = c & 1;
-        unsigned char* slot = sm + b * PL::SLOT;
-        const uint32_t t_XO = tmem + 64 * b;
+        unsigned char* slot = slot_of(c);
+        unsigned char* Sop = sm + PL::SOP + b * (DK * DV * 2);
         const int L = min(C, len - c * C);
         KDA_PHASE(0);
 
-        // ---- state of chunk c - 1, then its fp16 operand (row = value column)
+        // ---- (A) state entering chunk c and its fp16 operand
         if (c > 0) {
-            KDA_WAIT_OR_EXIT(mb_w, 32u, (c - 1) & 1);
+            KDA_WAIT_OR_EXIT(mb_chain, 4u, (nchain - 1) & 1);
             tc_fence_after();
-            float w[16];
-            tmem_ld16(t_W + lane_off + q_off, w);
+            float d[NC];
+            tmem_ldn<NC>(tmem + 128 * (b ^ 1) + lane_off + (uint32_t)(wg * NC), d);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
+            for (int j = 0; j < NC; ++j) S[j] = fmaf(egl, S[j], d[j]);
         }
-        if (lt < DK) st_row_h16(Sop, lt, 16 * wg, DK, S);
+        if (lt < DK) st_row_h16n<NC>(Sop, lt, wg * NC, DK, S);
         fence_proxy_async();
         tc_fence_before();
-        KDA_WAIT_OR_EXIT(mb_a + b, 1u << b, (apar >> b) & 1u);
+        __syncthreads();
         KDA_PHASE(1);
 
-        if (tid == 0) {
+        // ---- (B) chain MMA and the output products of chunk c
+        if (tid == kMma) {
             tc_fence_after();
+            if (!no_erase) {
 #pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)    // [O ; X] = [Qh ; Kh] S
-                umma_f16(t_XO, kdesc(slot + R::QK, kk, 128 * 128), mn_desc(Sop, kk, DK), kI, kk > 0);
-            umma_commit(mb_x);
-        }
-        ++xph;
-        pend |= 16u;
-        KDA_WAIT_OR_EXIT(mb_x, 16u, c & 1);
-        tc_fence_after();
-        // chunk c - 1's PT Y has completed as well: refill the other slot's
-        // second part with chunk c + 1
-        if (c >= 1 && c + 1 < nchunks) {
-            if (issuer) {
-                fence_proxy_async();
-                issue_b(c + 1);
+                for (int kk = 0; kk < DK / 16; ++kk)   // D_S += M' S  (M' from TMEM)
+                    umma_f16_ts(tmem + 128 * b, t_M + 8 * kk, mn_desc(Sop, kk, DK * 128), kIdv, 1);
             }
-            pend |= 4u << (b ^ 1);
-            bpar = (bpar & ~(1u << (b ^ 1))) | ((uint32_t)(((c + 1) >> 1) & 1) << (b ^ 1));
+            umma_commit(mb_chain);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)       // [O ; X] = [Qh ; Kh] S
+                umma_f16(t_O, kdesc(slot + R::QK, kk, 128 * 128), mn_desc(Sop, kk, DK * 128), kIdv, kk > 0);
+            umma_commit(mb_xo);
         }
-        KDA_WAIT_OR_EXIT(mb_b + b, 4u << b, (bpar >> b) & 1u);
+        ++nchain;
+        ++nxo;
+        pend |= 4u | 8u;
+
+        // ---- (C) chunk c + 1: V to fp16, then its M' and B MMAs
+        const bool more = c + 1 < nchunks;
+        if (more) {
+            KDA_WAIT_OR_EXIT(mb_rec + (b ^ 1), 1u << (b ^ 1), (rpar >> (b ^ 1)) & 1u);
+            convert_v(slot_of(c + 1));
+            fence_proxy_async();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == kMma) {
+                tc_fence_after();
+                issue_chunk_terms(c + 1);
+            }
+            ++nm;
+            pend |= 16u;
+        }
         KDA_PHASE(2);
 
-        // ---- Y = beta (V - X) (lanes 64..127) | o rows of chunk c - 1 (lanes 0..63)
+        // ---- (D) Y = beta (V - X) (lanes 64..127), then O += PT Y
+        KDA_WAIT_OR_EXIT(mb_xo, 8u, (nxo - 1) & 1);
+        tc_fence_after();
         {
-            const float* egl = reinterpret_cast<const float*>(slot + R::EGL);
-            const float* beta = reinterpret_cast<const float*>(slot + R::BETA);
-            eglp = lt < DK ? egl[lt] : 1.f;
+            const float* eg = reinterpret_cast<const float*>(slot + R::EGL);
+            egl = lt < DK ? eg[lt] : 1.f;
             if (lt >= C) {
                 const int s = lt - C;
-                float x16[16];
-                tmem_ld16(t_XO + lane_off + q_off, x16);
+                const float bs = reinterpret_cast<const float*>(slot + R::BETA)[s];
+                float x[NC];
+                tmem_ldn<NC>(t_O + lane_off + (uint32_t)(wg * NC), x);
                 tmem_wait_ld();
-                const float bs = beta[s];
-                const unsigned char* vt = slot + PL::VOFF;
-                uint4 vr[2];
-                vr[0] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg, C));
-                vr[1] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg + 8, C));
-                float y[16];
+                float y[NC];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
+                for (int u = 0; u < NC / 8; ++u) {
+                    const uint4 vr = *reinterpret_cast<const uint4*>(slot + PL::VOFF + swh_off(s, wg * NC + 8 * u, C));
+                    const __half2* v2 = reinterpret_cast<const __half2*>(&vr);
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const float2 f2 = __bfloat1622float2(v2[w]);
-                        const int jj = 8 * u + 2 * w;
-                        y[jj] = bs * (f2.x - (no_erase ? 0.f : x16[jj]));
-                        y[jj + 1] = bs * (f2.y - (no_erase ? 0.f : x16[jj + 1]));
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f2 = __half22float2(v2[e]);
+                        const int jj = 8 * u + 2 * e;
+                        y[jj] = bs * (f2.x - (no_erase ? 0.f : x[jj]));
+                        y[jj + 1] = bs * (f2.y - (no_erase ? 0.f : x[jj + 1]));
                     }
                 }
-                st_row_h16(Yb, s, 16 * wg, C, y);
-            } else if (c > 0) {
-                const int tk = tok0 + (c - 1) * C;
-                store_o_tile<TO>(tmem + 64 * (b ^ 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
-                                 ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
+                st_row_h16n<NC>(Yb, s, wg * NC, C, y);
             }
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
-        KDA_PHASE(3);
-        if (issuer && c + 2 < nchunks) {            // X MMA done, V consumed: refill part one
-            fence_proxy_async();
-            issue_a(c + 2);
-        }
-
-        if (tid == 0) {
+        if (tid == kMma) {
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)     // W = Z Y
-                umma_f16(t_W, kdesc(slot + R::Z, kk, DK * 128), mn_desc(Yb, kk, C), kI, kk > 0);
-            umma_commit(mb_w);
-#pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)     // O += PT Y  (rows 64..127: discarded)
-                umma_f16(t_XO, kdesc(slot + R::PT, kk, C * 128), mn_desc(Yb, kk, C), kI, 1);
+                umma_f16(t_O, kdesc(slot + R::PT, kk, 0), mn_desc(Yb, kk, C * 128), kIdv, 1);
+            umma_commit(mb_o);
         }
-        ++wph;
+        ++no;
         pend |= 32u;
-        if (c + 2 < nchunks) {
-            pend |= 1u << b;
-            apar = (apar & ~(1u << b)) | ((uint32_t)(((c + 2) >> 1) & 1) << b);
+        KDA_PHASE(3);
+
+        // ---- (F) M' of chunk c + 1
+        if (more) {
+            KDA_WAIT_OR_EXIT(mb_m, 16u, (nm - 1) & 1);
+            tc_fence_after();
+            if (!no_erase) convert_m();
         }
-        Lprev = L;
+
+        // ---- (E) o rows of chunk c (lanes 0..63); slot c % 2 then takes chunk c + 2
+        KDA_WAIT_OR_EXIT(mb_o, 32u, (no - 1) & 1);
+        tc_fence_after();
+        if (lt < C) {
+            float acc[NC];
+            tmem_ldn<NC>(t_O + lane_off + (uint32_t)(wg * NC), acc);
+            tmem_wait_ld();
+            if (lt < L) {
+                TO* dst = static_cast<TO*>(p.o) + ((size_t)(tok0 + c * C + lt) * H + h) * DV + wg * NC;
+                if constexpr (sizeof(TO) == 4) {
+#pragma unroll
+                    for (int j = 0; j < NC; j += 4)
+                        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < NC; j += 8)
+                        *reinterpret_cast<uint4*>(dst + j) =
+                            make_uint4(pack_bf16(acc[j], acc[j + 1]), pack_bf16(acc[j + 2], acc[j + 3]),
+                                       pack_bf16(acc[j + 4], acc[j + 5]), pack_bf16(acc[j + 6], acc[j + 7]));
+                }
+            }
+        }
+        if (c + 2 < nchunks) {
+            if (tid == kCopy) {
+                fence_proxy_async();
+                issue_rec(c + 2);
+            }
+            pend |= 1u << b;
+            rpar = (rpar & ~(1u << b)) | ((uint32_t)(((c + 2) >> 1) & 1) << b);
+        }
         KDA_PHASE(4);
     }
 
-    if (nchunks > 0) {
-        // W and O of the last chunk: one more commit covers every MMA issued
-        if (tid == 0) umma_commit(mb_x);
-        ++xph;
-        pend |= 16u;
-        KDA_WAIT_OR_EXIT(mb_x, 16u, nchunks & 1);
-        pend &= ~32u;
+    if (nchunks > 0) {   // state after the last chunk
+        KDA_WAIT_OR_EXIT(mb_chain, 4u, (nchain - 1) & 1);
         tc_fence_after();
-        float w[16];
-        tmem_ld16(t_W + lane_off + q_off, w);
+        float d[NC];
+        tmem_ldn<NC>(tmem + 128 * ((nchunks - 1) & 1) + lane_off + (uint32_t)(wg * NC), d);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
-        if (lt < C) {
-            const int tk = tok0 + (nchunks - 1) * C;
-            store_o_tile<TO>(tmem + 64 * ((nchunks - 1) & 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
-                             ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
-        }
+        for (int j = 0; j < NC; ++j) S[j] = fmaf(egl, S[j], d[j]);
     }
     if (p.s_out && lt < DK) {
-        float* dst = p.s_out + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg;
+        float* dst = p.s_out + (((size_t)n * H + h) * DK + lt) * DV + wg * NC;
 #pragma unroll
-        for (int j = 0; j < 16; j += 4)
+        for (int j = 0; j < NC; j += 4)
             *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
 
@@ -1130,22 +1187,21 @@ finish:
     if (*abort_flag) {
         // let every copy and MMA in flight land before the TMEM is released
         volatile int never = 0;
-        for (int i = 0; i < 2; ++i) {
-            if (pend & (1u << i)) (void)mbar_wait(mb_a + i, (apar >> i) & 1u, &never, p.timeout_cycles);
-            if (pend & (4u << i)) (void)mbar_wait(mb_b + i, (bpar >> i) & 1u, &never, p.timeout_cycles);
-        }
-        if (pend & 16u) (void)mbar_wait(mb_x, (uint32_t)((xph - 1) & 1), &never, p.timeout_cycles);
-        if (pend & 32u) (void)mbar_wait(mb_w, (uint32_t)((wph - 1) & 1), &never, p.timeout_cycles);
+        for (int i = 0; i < 2; ++i)
+            if (pend & (1u << i)) (void)mbar_wait(mb_rec + i, (rpar >> i) & 1u, &never, p.timeout_cycles);
+        if (pend & 4u) (void)mbar_wait(mb_chain, (uint32_t)((nchain - 1) & 1), &never, p.timeout_cycles);
+        if (pend & 8u) (void)mbar_wait(mb_xo, (uint32_t)((nxo - 1) & 1), &never, p.timeout_cycles);
+        if (pend & 16u) (void)mbar_wait(mb_m, (uint32_t)((nm - 1) & 1), &never, p.timeout_cycles);
+        if (pend & 32u) (void)mbar_wait(mb_o, (uint32_t)((no - 1) & 1), &never, p.timeout_cycles);
         __syncthreads();
-        if (tid == 0) umma_commit(mb_x);
-        (void)mbar_wait(mb_x, (uint32_t)(xph & 1), &never, p.timeout_cycles);
+        if (tid == kMma) umma_commit(mb_o);
+        (void)mbar_wait(mb_o, (uint32_t)(no & 1), &never, p.timeout_cycles);
     }
-    if (issuer) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 #undef KDA_WAIT_OR_EXIT
@@ -1158,24 +1214,23 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     prep_body<DK, VAR>(tmq, tmk, tmg, p, blockIdx.x, gridDim.x);
 }
 
-template <typename TO, int DK, bool VAR>
+template <typename TO, int DK, int DV, bool VAR>
 __global__ void __launch_bounds__(NT, 1)
-chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
-                  const ScanParams p)
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
 {
-    scan_body<TO, DK, VAR>(tmv, tmo, p, blockIdx.x);
+    scan_body<TO, DK, DV, VAR>(tmv, p, blockIdx.x);
 }
 
 // Cooperative schedule: CTAs [0, n_scan) scan, the others prep; the scan
 // waits on the records' ready flags, the prep never waits on the scan, and a
 // cooperative launch keeps every CTA resident, so the hand-off cannot stall.
-template <typename TO, int DK, bool VAR>
+template <typename TO, int DK, int DV, bool VAR>
 __global__ void __launch_bounds__(NT, 1)
 chunk_coop_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmg, const __grid_constant__ CUtensorMap tmv,
-                  const __grid_constant__ CUtensorMap tmo, const PrepParams pp, const ScanParams sp, int n_scan)
+                  const PrepParams pp, const ScanParams sp, int n_scan)
 {
-    if ((int)blockIdx.x < n_scan) scan_body<TO, DK, VAR>(tmv, tmo, sp, blockIdx.x);
+    if ((int)blockIdx.x < n_scan) scan_body<TO, DK, DV, VAR>(tmv, sp, blockIdx.x);
     else prep_body<DK, VAR>(tmq, tmk, tmg, pp, blockIdx.x - n_scan, gridDim.x - n_scan);
 }
 
@@ -1340,12 +1395,13 @@ static WsLayout ws_layout(int nseq, int T, long long tokens, int H, int dv, bool
     return w;
 }
 
-template <typename TO, int DK>
+template <typename TO, int DK, int DV>
 static cudaError_t run(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
                        const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens,
-                       int H, int dv, long long timeout_cycles, int mode, unsigned char* ws, size_t ws_bytes,
+                       int H, long long timeout_cycles, int mode, unsigned char* ws, size_t ws_bytes,
                        cudaStream_t stream)
 {
+    constexpr int dv = DV;
     const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;
     const bool variant = (mode & (KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE | KDA_MODE_NORM_QK | KDA_MODE_GATE_LOGITS)) != 0;
     const int req_blocks = (mode >> 8) & 0xff;     // KDA_MODE_BLOCKS(n), 0 = automatic
@@ -1354,7 +1410,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     const WsLayout L = ws_layout<DK>(nseq, T, tokens, H, dv, cu != nullptr);
     if (!ws || ws_bytes < L.bytes) return cudaErrorInvalidValue;
     const long long max_chunks = L.max_chunks;
-    const long long scan_ctas = (long long)nseq * H * (dv / NV);
+    const long long scan_ctas = (long long)nseq * H;   // one scan CTA per (sequence, head)
     if (scan_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     // schedule: one cooperative launch (prep CTAs publish records, scan CTAs
     // consume them) when the scan grid leaves at least 32 SMs; otherwise prep
@@ -1369,15 +1425,13 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
         (!head_gate && !make_tmap(&tg, log_alpha, tokens, H, DK, true)))
         return cudaErrorInvalidValue;
-    CUtensorMap tv, to;
-    if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
-        !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
-        return cudaErrorInvalidValue;
+    CUtensorMap tv;
+    if (!make_tmap(&tv, v, tokens, H, dv, false, 64, true)) return cudaErrorInvalidValue;
     auto pk = variant ? chunk_prep_kernel<DK, true> : chunk_prep_kernel<DK, false>;
-    auto sk = variant ? chunk_scan_kernel<TO, DK, true> : chunk_scan_kernel<TO, DK, false>;
+    auto sk = variant ? chunk_scan_kernel<TO, DK, DV, true> : chunk_scan_kernel<TO, DK, DV, false>;
     cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
     if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
+        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK, DV>::BYTES);
     if (err != cudaSuccess) return err;
 
     // events of the two-stream schedule (created last: no early return leaks them)
@@ -1473,7 +1527,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         sp.s_in = b == 0 ? s0 : carry;
         sp.s_out = (b == nblocks - 1) ? sT : carry;
         if (scan_ctas <= 0) return cudaSuccess;
-        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
+        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK, DV>::BYTES, stream>>>(tv, sp);
         return cudaGetLastError();
     };
 
@@ -1481,8 +1535,8 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (coop) {
         unsigned* flags = reinterpret_cast<unsigned*>(ws + L.flags);
         err = cudaMemsetAsync(flags, 0, (size_t)max_chunks * H * 4, stream);
-        auto ck = variant ? chunk_coop_kernel<TO, DK, true> : chunk_coop_kernel<TO, DK, false>;
-        const int smem = std::max(PrepPlan::BYTES, ScanPlan<DK>::BYTES);
+        auto ck = variant ? chunk_coop_kernel<TO, DK, DV, true> : chunk_coop_kernel<TO, DK, DV, false>;
+        const int smem = std::max(PrepPlan::BYTES, ScanPlan<DK, DV>::BYTES);
         if (err == cudaSuccess) err = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err == cudaSuccess) {
             pp.ready = flags;
@@ -1505,7 +1559,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             const int n_scan = (int)scan_ctas;
-            if (cudaLaunchKernelEx(&cfg, ck, tq, tk, tg, tv, to, pp, sp, n_scan) == cudaSuccess) done = true;
+            if (cudaLaunchKernelEx(&cfg, ck, tq, tk, tg, tv, pp, sp, n_scan) == cudaSuccess) done = true;
             else (void)cudaGetLastError();   // not co-residable here: fall back to prep then scan
             pp.ready = nullptr;
             sp.ready = nullptr;
@@ -1579,18 +1633,19 @@ static long long noalloc_block(int nseq, int H, int dv, bool has_final, int nch)
     return std::min<long long>(nch, (long long)((kScratchBytes - carry) / (2 * per_chunk)));
 }
 
-template <typename TO, int DK>
+template <typename TO, int DK, int DV>
 static cudaError_t run_noalloc(const void* q, const void* k, const void* v, const float* beta,
                                const float* log_alpha, const float* s0, void* o, float* sT, int nseq, int T,
-                               long long tokens, int H, int dv, long long timeout_cycles, cudaStream_t stream)
+                               long long tokens, int H, long long timeout_cycles, cudaStream_t stream)
 {
+    constexpr int dv = DV;
     using R = Rec<DK>;
     const int nsm = sm_count();
     const int nch = (T + C - 1) / C;
     const long long cb = noalloc_block<DK>(nseq, H, dv, sT != nullptr, nch);
     if (cb <= 0) return cudaErrorInvalidValue;
     const int nblocks = (int)((nch + cb - 1) / cb);
-    const long long scan_ctas = (long long)nseq * H * (dv / NV);
+    const long long scan_ctas = (long long)nseq * H;   // one scan CTA per (sequence, head)
     if (scan_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     unsigned char* area = scratch_area();
     if (!area) return cudaErrorInvalidSymbol;
@@ -1599,16 +1654,15 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
     unsigned char* ring[2] = {area + carry_sz, nullptr};
     if (nblocks > 1) ring[1] = area + carry_sz + (size_t)cb * nseq * H * R::BYTES;
 
-    CUtensorMap tq, tk, tg, tv, to;
+    CUtensorMap tq, tk, tg, tv;
     if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
-        !make_tmap(&tg, log_alpha, tokens, H, DK, true) || !make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
-        !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
+        !make_tmap(&tg, log_alpha, tokens, H, DK, true) || !make_tmap(&tv, v, tokens, H, dv, false, 64, true))
         return cudaErrorInvalidValue;
     auto pk = chunk_prep_kernel<DK, false>;
-    auto sk = chunk_scan_kernel<TO, DK, false>;
+    auto sk = chunk_scan_kernel<TO, DK, DV, false>;
     cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
     if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
+        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK, DV>::BYTES);
     if (err != cudaSuccess) return err;
 
     PrepParams pp{};
@@ -1653,7 +1707,7 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
         sp.s_in = b == 0 ? s0 : carry;
         sp.s_out = b == nblocks - 1 ? sT : carry;
         if (scan_ctas <= 0) return cudaSuccess;
-        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
+        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK, DV>::BYTES, stream>>>(tv, sp);
         return cudaGetLastError();
     };
 
@@ -1715,6 +1769,21 @@ size_t chunk_fwd_split_workspace(int nseq, int T, long long tokens, int H, int d
                      : split::ws_layout<64>(nseq, T, tokens, H, dv, varlen).bytes;
 }
 
+template <typename TO, int DK>
+static cudaError_t run_dv(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
+                          const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens,
+                          int H, int dv, long long timeout_cycles, int mode, unsigned char* ws, size_t ws_bytes,
+                          cudaStream_t stream)
+{
+    if (dv == 128)
+        return split::run<TO, DK, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, timeout_cycles,
+                                       mode, ws, ws_bytes, stream);
+    if (dv == 64)
+        return split::run<TO, DK, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, timeout_cycles,
+                                      mode, ws, ws_bytes, stream);
+    return cudaErrorInvalidValue;
+}
+
 cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const float* beta,
                             const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
                             int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
@@ -1722,11 +1791,11 @@ cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const f
 {
     unsigned char* w = static_cast<unsigned char*>(ws);
     if (o_dtype == KDA_F32) {
-        if (dk == 128) return split::run<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
-        if (dk == 64) return split::run<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 128) return run_dv<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 64) return run_dv<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
     } else {
-        if (dk == 128) return split::run<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
-        if (dk == 64) return split::run<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 128) return run_dv<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 64) return run_dv<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -1738,17 +1807,31 @@ bool chunk_fwd_noalloc_fits(int nseq, int T, int H, int dk, int dv, bool has_fin
                      : split::noalloc_block<64>(nseq, H, dv, has_final, nch) > 0;
 }
 
+template <typename TO, int DK>
+static cudaError_t noalloc_dv(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
+                              const float* s0, void* o, float* sT, int nseq, int T, long long tokens, int H, int dv,
+                              long long timeout_cycles, cudaStream_t stream)
+{
+    if (dv == 128)
+        return split::run_noalloc<TO, DK, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H,
+                                               timeout_cycles, stream);
+    if (dv == 64)
+        return split::run_noalloc<TO, DK, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H,
+                                              timeout_cycles, stream);
+    return cudaErrorInvalidValue;
+}
+
 cudaError_t chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* beta,
                               const float* log_alpha, const float* s0, void* o, float* sT, int nseq, int T,
                               long long tokens, int H, int dk, int dv, kda_dtype o_dtype, long long timeout_cycles,
                               cudaStream_t stream)
 {
     if (o_dtype == KDA_F32) {
-        if (dk == 128) return split::run_noalloc<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
-        if (dk == 64) return split::run_noalloc<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 128) return noalloc_dv<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 64) return noalloc_dv<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
     } else {
-        if (dk == 128) return split::run_noalloc<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
-        if (dk == 64) return split::run_noalloc<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 128) return noalloc_dv<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 64) return noalloc_dv<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -5,3 +5,4 @@
 #include "kda_decode.cu"
 #include "kda_chunk_simt.cu"
 #include "kda_chunk_split.cu"
+#include "kda_chunk_bwd.cu"

@@ -253,6 +253,52 @@ kda_status kda_recurrent_step_mode(const void* q, const void* k, const void* v,
                                    kda_dtype dtype, kda_dtype o_dtype, int mode, void* stream);
 
 /*
+ * Chunkwise backward pass: gradients of L = sum(o * grad_o) + sum(S_T * grad_final_state)
+ * through kda_chunk_fwd's computation ("Hybrid Linear Attention Architecture:
+ * Making LLM Training and Inference More Efficient", section IV: backpropagation
+ * reuses the chunked structure of the forward pass).  It recomputes the
+ * forward (the states entering every chunk go to the workspace), then walks
+ * the chunks in reverse carrying the state's gradient, with the per-chunk
+ * adjoint of the UT transform and of the gate factors.  fp32 arithmetic on
+ * CUDA cores throughout; the plain layer only (no KDA_MODE_* variants).
+ *
+ *   q, k, v, beta, log_alpha, initial_state: as in kda_chunk_fwd (dtype bf16 or fp32)
+ *   grad_o           [B, T, H, dv] fp32
+ *   grad_final_state [B, H, dk, dv] fp32, or NULL (zero)
+ *   grad_q, grad_k   [B, T, H, dk] fp32, written
+ *   grad_v           [B, T, H, dv] fp32, written
+ *   grad_beta        [B, T, H]     fp32, written
+ *   grad_log_alpha   [B, T, H, dk] fp32, written
+ *   grad_initial_state [B, H, dk, dv] fp32, or NULL if not wanted
+ *   workspace        at least kda_chunk_bwd_workspace_size() bytes, 256-byte aligned
+ * All tensor pointers 16-byte aligned (beta, grad_beta: 4).  d_k, d_v in
+ * {64, 128}, chunk 64.  The gradient buffers must not alias the inputs.
+ */
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const float* beta,
+                         const float* log_alpha, const float* initial_state,
+                         const float* grad_o, const float* grad_final_state,
+                         float* grad_q, float* grad_k, float* grad_v, float* grad_beta,
+                         float* grad_log_alpha, float* grad_initial_state,
+                         int B, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+kda_status kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
+                                        kda_dtype dtype, size_t* bytes);
+
+/* The same over N packed variable-length sequences (layouts of
+ * kda_varlen_fwd; initial/final state gradients [N, H, dk, dv]). */
+kda_status kda_varlen_bwd(const void* q, const void* k, const void* v, const float* beta,
+                          const float* log_alpha, const int32_t* cu_seqlens, int N,
+                          const float* initial_state, const float* grad_o, const float* grad_final_state,
+                          float* grad_q, float* grad_k, float* grad_v, float* grad_beta,
+                          float* grad_log_alpha, float* grad_initial_state,
+                          int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+kda_status kda_varlen_bwd_workspace_size(int N, int T, int H, int dk, int dv, int chunk,
+                                         kda_dtype dtype, size_t* bytes);
+
+/*
  * Synchronises `stream` and reports (then clears) the current device's
  * status word: KDA_ERR_TIMEOUT if a device-side bounded wait ran out since the
  * last check, KDA_ERR_INVALID_ARG if a kernel found device-resident sequence

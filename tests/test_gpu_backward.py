@@ -1,0 +1,95 @@
+"""GPU: the chunkwise backward (kda_chunk_bwd / kda_varlen_bwd through the C
+ABI) against the fp64 oracle's reverse-mode gradients of the token recurrence
+(oracle.backward.recurrence_backward, itself pinned by finite differences).
+
+The kernel computes in fp32 from the exact input values; the bar is 1e-4
+(max-abs error / RMS of the reference, per gradient), the fp32 forward's bar.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import backward
+import gated_delta_rule_133_b200 as kda
+from gated_delta_rule_133_b200.inputs import Workload, cu_from_lengths, draw_tokens, make_inputs
+from tests._helpers import f64, norm_max_err
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+TOL = 1e-4
+NAMES = ("dq", "dk", "dv", "dbeta", "dlog_alpha", "ds0")
+
+
+def _grads_out(B, T, H, dv, seed):
+    g = torch.Generator().manual_seed(seed)
+    do = torch.randn(B, T, H, dv, generator=g)
+    dsT = torch.randn(B, H, 128 if dv == 128 else dv, dv, generator=g)
+    return do, dsT
+
+
+def _check(got, ref):
+    for n, a, b in zip(NAMES, got, ref):
+        e = norm_max_err(a, b)
+        assert e <= TOL, f"{n}: {e:.2e}"
+
+
+@pytest.mark.parametrize("B,T,H,d,dtype,mu", [
+    (2, 150, 2, 128, "bf16", -3.0),     # two full chunks and a ragged one
+    (1, 64, 3, 64, "fp32", -1.0),       # one full chunk, strong gates
+    (1, 1, 2, 128, "bf16", -3.0),       # a single token
+    (2, 200, 1, 64, "bf16", -6.0),      # weak gates
+])
+def test_chunk_bwd_matches_oracle(B, T, H, d, dtype, mu):
+    w = Workload("bwd", "dense", B, T, H, d, d, dtype, mu, 0.05, seed=300 + T)
+    x = make_inputs(w, "cpu")
+    g = torch.Generator().manual_seed(400 + T)
+    do = torch.randn(B, T, H, d, generator=g)
+    dsT = torch.randn(B, H, d, d, generator=g)
+    dev = {n: (None if t is None else t.to(DEV)) for n, t in x.items()}
+    got = kda.kda_chunk_bwd(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_alpha"], dev["initial_state"],
+                            do.to(DEV), dsT.to(DEV))
+    torch.cuda.synchronize()
+    kda.kda_check()
+    flat = lambda t: f64(t).reshape(B * T, H, *t.shape[3:])
+    ref = backward.recurrence_backward(flat(x["q"]), flat(x["k"]), flat(x["v"]), f64(x["beta"]).reshape(B * T, H),
+                                       flat(x["log_alpha"]), np.arange(B + 1) * T, f64(x["initial_state"]),
+                                       flat(do), f64(dsT))
+    got = [flat(t) for t in got[:5]] + [f64(got[5])]
+    got[3] = got[3].reshape(B * T, H)
+    _check(got, ref)
+
+
+def test_chunk_bwd_without_state_gradients():
+    """No initial state and no final-state gradient: both read as zeros."""
+    B, T, H, d = 1, 130, 2, 128
+    w = Workload("bwd", "dense", B, T, H, d, d, "bf16", -3.0, 0.0, seed=310)
+    x = make_inputs(w, "cpu")
+    do = torch.randn(B, T, H, d, generator=torch.Generator().manual_seed(311))
+    dev = {n: (None if t is None else t.to(DEV)) for n, t in x.items()}
+    got = kda.kda_chunk_bwd(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_alpha"], None, do.to(DEV), None)
+    torch.cuda.synchronize()
+    flat = lambda t: f64(t).reshape(B * T, H, *t.shape[3:])
+    ref = backward.recurrence_backward(flat(x["q"]), flat(x["k"]), flat(x["v"]), f64(x["beta"]).reshape(B * T, H),
+                                       flat(x["log_alpha"]), None, None, flat(do), None)
+    got = [flat(t) for t in got[:5]] + [f64(got[5])]
+    got[3] = got[3].reshape(B * T, H)
+    _check(got, ref)
+
+
+def test_varlen_bwd_matches_oracle():
+    lens = [1, 63, 64, 65, 0, 200, 129]
+    cu = cu_from_lengths(lens)
+    H, d = 2, 128
+    t = draw_tokens(int(cu[-1]), H, d, d, "bf16", -3.0, 320, "cpu", init_states=len(lens), init_std=0.05)
+    g = torch.Generator().manual_seed(321)
+    do = torch.randn(int(cu[-1]), H, d, generator=g)
+    dsT = torch.randn(len(lens), H, d, d, generator=g)
+    dev = {n: (None if v is None else v.to(DEV)) for n, v in t.items()}
+    got = kda.kda_varlen_bwd(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_alpha"],
+                             torch.from_numpy(cu).to(DEV), dev["initial_state"], do.to(DEV), dsT.to(DEV))
+    torch.cuda.synchronize()
+    kda.kda_check()
+    ref = backward.recurrence_backward(f64(t["q"]), f64(t["k"]), f64(t["v"]), f64(t["beta"]), f64(t["log_alpha"]),
+                                       cu, f64(t["initial_state"]), f64(do), f64(dsT))
+    _check([f64(x) for x in got], ref)
