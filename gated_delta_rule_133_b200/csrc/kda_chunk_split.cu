@@ -459,6 +459,40 @@ __device__ __forceinline__ void ut_rows(float* As, float* X, unsigned char* Top)
     }
 }
 
+// UT transform T = (I + A)^-1 of the strictly lower 64 x 64 A by forward
+// substitution, one column of T per thread (threads 0..63):
+//   T[j][j] = 1,   T[r][j] = -sum_{j <= s < r} A[r][s] T[s][j]   (r > j).
+// The column lives in registers (T[s][j] = 0 for s < j, so the sum may run
+// from s = 0); rows of A (As[r * LDT + s], zero for s >= r) are read as
+// float4s that every lane of a warp reads at the same address (broadcast), and
+// eight partial sums shorten the dependent chain.  Column j of T is row j of
+// T^T, written to Top as fp16 (K-major 128-byte swizzle).
+__device__ __forceinline__ void ut_columns(const float* As, unsigned char* Top)
+{
+    const int j = threadIdx.x;
+    float x[C];
+#pragma unroll
+    for (int r = 0; r < C; ++r) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; 4 * q < r; ++q) {
+            const float4 a = ld4(As + r * LDT + 4 * q);
+            const int b = 4 * (q & 1);
+            if (4 * q + 0 < r) acc[b + 0] = fmaf(a.x, x[4 * q + 0], acc[b + 0]);
+            if (4 * q + 1 < r) acc[b + 1] = fmaf(a.y, x[4 * q + 1], acc[b + 1]);
+            if (4 * q + 2 < r) acc[b + 2] = fmaf(a.z, x[4 * q + 2], acc[b + 2]);
+            if (4 * q + 3 < r) acc[b + 3] = fmaf(a.w, x[4 * q + 3], acc[b + 3]);
+        }
+        const float sum = ((acc[0] + acc[4]) + (acc[1] + acc[5])) + ((acc[2] + acc[6]) + (acc[3] + acc[7]));
+        x[r] = r > j ? -sum : (r == j ? 1.f : 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < C / 8; ++u)
+        *reinterpret_cast<uint4*>(Top + swh_off(j, 8 * u, C)) =
+            make_uint4(pack_f16(x[8 * u], x[8 * u + 1]), pack_f16(x[8 * u + 2], x[8 * u + 3]),
+                       pack_f16(x[8 * u + 4], x[8 * u + 5]), pack_f16(x[8 * u + 6], x[8 * u + 7]));
+}
+
 // One persistent CTA per SM walks items blockIdx.x, + gridDim.x, ...  The
 // UT transform of item k (warpgroup 0) overlaps the gate cumsum and operand
 // build of item k + 1 (warpgroups 1-3); one MMA round then forms Z, PT of
@@ -818,8 +852,8 @@ __device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[N])
     else tmem_ld16(taddr, v);
 }
 
-// One CTA per (sequence, head).  The state update of a chunk is one MMA
-// round on the critical path:
+// One CTA per (sequence, head), warp-specialised.  The state update of a
+// chunk is one MMA round on the critical path:
 //
 //   S_{c+1} = diag(e^G_last) S_c + M'_c S_c + B_c,
 //   M'_c = -(Z diag(beta)) Kh  (d_k x d_k),   B_c = (Z diag(beta)) V  (d_k x d_v)
@@ -830,41 +864,46 @@ __device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[N])
 // the accumulator the chain MMA adds to.  The output leaves the chain:
 // [O ; X] = [Qh ; Kh] S_c, Y = beta (V - X), O += PT Y.
 //
-// Thread (warp w, lane l) owns state row 32 (w % 4) + l (the TMEM lane its
-// warp may access) and the NC = DV / 4 value columns of its warpgroup, in
-// fp32 registers.  TMEM columns: D_S[2] (0, 128), D_O (256), D_M (384; M'
-// packed over its first DK / 2 columns).
-//
-// Per chunk c (record in slot c % 2):
-//   (A) S_c from D_S of chunk c - 1, its fp16 operand to S_op[c % 2]
-//   (B) chain MMA D_S[c % 2] += M'_c S_op; X/O MMA D_O = [Qh ; Kh] S_op
-//   (C) chunk c + 1: V tile to fp16, MMAs D_M = Zb Kh, D_S[(c+1) % 2] = Zb V
-//   (D) Y = beta (V - X) (lanes 64..127); MMA D_O += PT Y
-//   (F) M'_{c+1} = -D_M to fp16 in TMEM
-//   (E) o rows of chunk c (lanes 0..63); slot c % 2 refilled with chunk c + 2
+// Warp roles (they synchronise through mbarriers, never CTA-wide barriers):
+//   warp 0       MMA issuer: issues each MMA group as soon as its inputs are
+//                ready, the state chain first;
+//   warps 1..3   V tile bf16 -> fp16, in place;
+//   warps 4..11  state: row 32 (w % 4) + lane, half of the value columns, in
+//                fp32 registers; S_op writes; M' conversion;
+//   warps 12..15 output: Y = beta (V - X) (lanes 64..127), o rows (lanes 0..63);
+//                lane 0 of warp 12 also issues the copies: the record and V
+//                tile of chunk c + 2 into the slot chunk c frees.
+// TMEM columns: D_S[2] (0, 128), D_O (256), D_M (384; M' packed over its
+// columns [DK / 4, 3 DK / 4)).
 template <typename TO, int DK, int DV, bool VAR>
 __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const ScanParams& p, int bid)
 {
     const bool no_erase = VAR && p.no_erase;   // layer variant (VAR instantiations only)
     using PL = ScanPlan<DK, DV>;
     using R = Rec<DK>;
-    constexpr int NC = DV / 4;                 // value columns per warpgroup
+    constexpr int SC = DV / 2;                 // value columns per state warp
     extern __shared__ unsigned char smem_raw[];
     KDA_PHASE_DECL(1)
     unsigned char* sm = align1024(smem_raw);
     unsigned char* Yb = sm + PL::YB;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::BAR);
-    uint64_t* mb_rec = bars + 0;   // [2]: record + V tile of a slot
-    uint64_t* mb_chain = bars + 2;
-    uint64_t* mb_xo = bars + 3;
-    uint64_t* mb_m = bars + 4;
-    uint64_t* mb_o = bars + 5;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+    uint64_t* mb_rec = bars + 0;     // [2] record + V tile of a slot (transaction bytes)
+    uint64_t* mb_chain = bars + 2;   // commits: chain MMA of a chunk
+    uint64_t* mb_m = bars + 3;       //          M' and B MMAs of a chunk
+    uint64_t* mb_xo = bars + 4;      //          [O ; X] MMA
+    uint64_t* mb_o = bars + 5;       //          PT Y MMA
+    uint64_t* bar_v16 = bars + 6;    // [2] V tile of a slot converted (warps 1..3)
+    uint64_t* bar_sop = bars + 8;    // S_op written (8 state warps)
+    uint64_t* bar_mconv = bars + 9;  // M' converted (8 state warps)
+    uint64_t* bar_y = bars + 10;     // Y written (2 output warps)
+    uint64_t* bar_ofree = bars + 11; // o rows read from D_O (2 output warps)
+    uint64_t* mb_fin = bars + 12;    // final commit of an aborted CTA
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int lt = (warp & 3) * 32 + (tid & 31);   // TMEM lane of this thread
-    const int wg = tid >> 7;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3;
+    const int lt = quad * 32 + lane;           // TMEM lane of this thread
     const int h = bid % p.H;
     const int rank = bid / p.H;
     const int H = p.H;
@@ -904,6 +943,13 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const ScanPara
 
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
+        mbar_init(bar_v16 + 0, 3);
+        mbar_init(bar_v16 + 1, 3);
+        mbar_init(bar_sop, 8);
+        mbar_init(bar_mconv, 8);
+        mbar_init(bar_y, 2);
+        mbar_init(bar_ofree, 2);
+        mbar_init(mb_fin, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
@@ -917,285 +963,322 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const ScanPara
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32) << 16;
+    const uint32_t lane_off = ((uint32_t)quad * 32) << 16;
     const uint32_t t_O = tmem + 256, t_M = tmem + 384;
     constexpr uint32_t kIdv = idesc_f16(128, DV, 1);    // N = d_v, B MN-major
     constexpr uint32_t kIdk = idesc_f16(128, DK, 1);    // N = d_k, B MN-major
     constexpr uint32_t kRecBytes = (uint32_t)R::BYTES + C * DV * 2;
-
+    const long long tmo = p.timeout_cycles;
     auto slot_of = [&](int cc) { return sm + (cc & 1) * PL::SLOT; };
-    auto issue_rec = [&](int cc) {   // one thread: record and V tile of chunk cc into its slot
+    auto sop_of = [&](int cc) { return sm + PL::SOP + (cc & 1) * (DK * DV * 2); };
+    // bounded wait; false once this CTA has aborted (every role then leaves)
+    auto wt = [&](uint64_t* bar, int par) { return mbar_wait(bar, (uint32_t)(par & 1), abort_flag, tmo); };
+
+    // state of the roles that outlive their loops (cleanup of an aborted CTA)
+    int rec_issued = 0;         // copy issuer: loads issued
+    bool mma_issued = false;    // MMA issuer: any MMA issued
+    constexpr int kCopy = 384;  // copy issuer: lane 0 of the output warp of lane quadrant 0
+    auto issue_rec = [&](int cc) {   // record and V tile of chunk cc into its slot (one thread)
         unsigned char* slot = slot_of(cc);
         const size_t ri = (size_t)(j0 + cc) * H + h;
-        if (p.ready && !wait_ready(p.ready + ri, abort_flag, p.timeout_cycles)) return;
+        if (p.ready && !wait_ready(p.ready + ri, abort_flag, tmo)) return false;
         mbar_expect_tx(mb_rec + (cc & 1), kRecBytes);
         bulk_load(slot, p.rec + ri * R::BYTES, (uint32_t)R::BYTES, mb_rec + (cc & 1));
 #pragma unroll
         for (int a = 0; a < DV / 64; ++a)
             tma_load_3d(slot + PL::VOFF + a * 8192, &tmv, mb_rec + (cc & 1), 64 * a, h, tok0 + cc * C);
+        ++rec_issued;
+        return true;
     };
-    // V tile of a slot from bf16 to fp16 in place (all threads, 16 bytes each per pass)
-    auto convert_v = [&](unsigned char* slot) {
-        uint4* vt = reinterpret_cast<uint4*>(slot + PL::VOFF);
-#pragma unroll
-        for (int i = tid; i < C * DV * 2 / 16; i += NT) {
-            uint4 u = vt[i];
-            uint32_t* w = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-                w[e] = pack_f16(f.x, f.y);
-            }
-            vt[i] = u;
-        }
-    };
-    // MMAs of the state-independent terms of chunk cc: D_M = Zb Kh, D_S[cc % 2] = Zb V (one thread)
-    auto issue_chunk_terms = [&](int cc) {
-        const unsigned char* slot = slot_of(cc);
-        if (!no_erase) {
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                umma_f16(t_M, kdesc(slot + R::Z, kk, 0), mn_desc(slot + R::QK + C * 128 + 0, kk, 128 * 128), kIdk,
-                         kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-            umma_f16(tmem + 128 * (cc & 1), kdesc(slot + R::Z, kk, 0), mn_desc(slot + PL::VOFF, kk, C * 128), kIdv,
-                     kk > 0);
-        umma_commit(mb_m);
-    };
-    // M' = -D_M to packed fp16 in TMEM (A operand of the chain MMA); the four
-    // warps sharing a lane quadrant read all their columns before any writes
-    auto convert_m = [&]() {
-        constexpr int MC = DK / 4;   // D_M columns per warpgroup
-        float m[MC];
-        tmem_ldn<MC>(t_M + lane_off + (uint32_t)(wg * MC), m);
-        tmem_wait_ld();
-        bar_sync(2 + (warp & 3), 128);
-        uint32_t pk[MC / 2];
-#pragma unroll
-        for (int i = 0; i < MC / 2; ++i) pk[i] = pack_f16(-m[2 * i], -m[2 * i + 1]);
-        if constexpr (MC == 32) {
-            tmem_st8(t_M + lane_off + (uint32_t)(wg * 16), *reinterpret_cast<const uint32_t(*)[8]>(pk));
-            tmem_st8(t_M + lane_off + (uint32_t)(wg * 16 + 8), *reinterpret_cast<const uint32_t(*)[8]>(pk + 8));
-        } else {
-            tmem_st8(t_M + lane_off + (uint32_t)(wg * 8), *reinterpret_cast<const uint32_t(*)[8]>(pk));
-        }
-        tmem_wait_st();
-    };
-
-    // state rows of this thread (rows >= DK unused)
-    float S[NC];
-    {
-        const bool own = lt < DK && p.s_in;
-        const float* src = own ? p.s_in + (((size_t)n * H + h) * DK + lt) * DV + wg * NC : nullptr;
-#pragma unroll
-        for (int j = 0; j < NC; j += 4) {
-            const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-            S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
-        }
+    if (tid == kCopy && nchunks > 0) {   // the first two records; chunk c's slot takes chunk c + 2 after its o rows
+        // a failed wait for a record sets the abort flag, which every role checks
+        if (issue_rec(0) && nchunks > 1) (void)issue_rec(1);
     }
 
-    constexpr int kMma = 0, kCopy = 32;        // MMA issuer and copy issuer threads
-    unsigned pend = 0;                         // bits: 0-1 mb_rec[slot], 2 chain, 3 xo, 4 m, 5 o
-    uint32_t rpar = 0u;                        // bit i: phase parity of the pending load of slot i
-    int nchain = 0, nxo = 0, nm = 0, no = 0;   // commits issued to mb_chain / mb_xo / mb_m / mb_o
-    float egl = 1.f;                           // e^G_last of the chunk before, row lt
-    int c = 0;
+    const bool state_warp = warp >= 4 && warp < 12;
+    const int hh = (warp - 4) >> 2;            // state warps: value-column half
 
-    if (nchunks > 0) {
-        if (tid == kCopy) {
-            issue_rec(0);
-            if (nchunks > 1) issue_rec(1);
-        }
-        pend |= 1u | (nchunks > 1 ? 2u : 0u);
-        rpar = 0u;
-        KDA_WAIT_OR_EXIT(mb_rec, 1u, 0u);
-        convert_v(slot_of(0));
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == kMma) {
+    if (warp == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && nchunks > 0) {
+            auto issue_chunk_terms = [&](int cc) {   // D_M = Zb Kh, D_S[cc % 2] = Zb V
+                const unsigned char* slot = slot_of(cc);
+                if (!no_erase) {
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        umma_f16(t_M, kdesc(slot + R::Z, kk, 0), mn_desc(slot + R::QK + C * 128, kk, 128 * 128), kIdk,
+                                 kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_f16(tmem + 128 * (cc & 1), kdesc(slot + R::Z, kk, 0), mn_desc(slot + PL::VOFF, kk, C * 128),
+                             kIdv, kk > 0);
+                umma_commit(mb_m);
+            };
+            if (!wt(bar_v16, 0)) goto finish;
             tc_fence_after();
             issue_chunk_terms(0);
-        }
-        ++nm;
-        pend |= 16u;
-        KDA_WAIT_OR_EXIT(mb_m, 16u, 0u);
-        tc_fence_after();
-        if (!no_erase) convert_m();
-    }
-
-    for (c = 0; c < nchunks; ++c) {
-        const int b = c & 1;
-        unsigned char* slot = slot_of(c);
-        unsigned char* Sop = sm + PL::SOP + b * (DK * DV * 2);
-        const int L = min(C, len - c * C);
-        KDA_PHASE(0);
-
-        // ---- (A) state entering chunk c and its fp16 operand
-        if (c > 0) {
-            KDA_WAIT_OR_EXIT(mb_chain, 4u, (nchain - 1) & 1);
-            tc_fence_after();
-            float d[NC];
-            tmem_ldn<NC>(tmem + 128 * (b ^ 1) + lane_off + (uint32_t)(wg * NC), d);
-            tmem_wait_ld();
+            mma_issued = true;
+            int ci = 0, cm = 1, cx = 0, cp = 0;     // next chain, M'/B, [O ; X], PT Y chunk
+            long long t0 = clock64();
+            while (cp < nchunks) {
+                bool did = false;
+                if (ci < nchunks && (ci == 0 || cx >= ci) && mbar_test(bar_mconv, ci & 1) &&
+                    mbar_test(bar_sop, ci & 1)) {
+                    tc_fence_after();
+                    unsigned char* Sop = sop_of(ci);
+                    if (!no_erase) {
 #pragma unroll
-            for (int j = 0; j < NC; ++j) S[j] = fmaf(egl, S[j], d[j]);
-        }
-        if (lt < DK) st_row_h16n<NC>(Sop, lt, wg * NC, DK, S);
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        KDA_PHASE(1);
-
-        // ---- (B) chain MMA and the output products of chunk c
-        if (tid == kMma) {
-            tc_fence_after();
-            if (!no_erase) {
+                        for (int kk = 0; kk < DK / 16; ++kk)   // D_S += M' S  (M' from TMEM)
+                            umma_f16_ts(tmem + 128 * (ci & 1), t_M + DK / 4 + 8 * kk, mn_desc(Sop, kk, DK * 128), kIdv, 1);
+                    }
+                    umma_commit(mb_chain);
+                    ++ci;
+                    did = true;
+                } else if (cp < cx && mbar_test(bar_y, cp & 1)) {
+                    tc_fence_after();
+                    const unsigned char* slot = slot_of(cp);
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)   // D_S += M' S  (M' from TMEM)
-                    umma_f16_ts(tmem + 128 * b, t_M + 8 * kk, mn_desc(Sop, kk, DK * 128), kIdv, 1);
-            }
-            umma_commit(mb_chain);
+                    for (int kk = 0; kk < C / 16; ++kk)       // O += PT Y  (rows 64..127: discarded)
+                        umma_f16(t_O, kdesc(slot + R::PT, kk, 0), mn_desc(Yb, kk, C * 128), kIdv, 1);
+                    umma_commit(mb_o);
+                    ++cp;
+                    did = true;
+                } else if (cx < ci && cx == cp && (cx == 0 || mbar_test(bar_ofree, (cx - 1) & 1))) {
+                    tc_fence_after();
+                    const unsigned char* slot = slot_of(cx);
+                    unsigned char* Sop = sop_of(cx);
 #pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)       // [O ; X] = [Qh ; Kh] S
-                umma_f16(t_O, kdesc(slot + R::QK, kk, 128 * 128), mn_desc(Sop, kk, DK * 128), kIdv, kk > 0);
-            umma_commit(mb_xo);
-        }
-        ++nchain;
-        ++nxo;
-        pend |= 4u | 8u;
-
-        // ---- (C) chunk c + 1: V to fp16, then its M' and B MMAs
-        const bool more = c + 1 < nchunks;
-        if (more) {
-            KDA_WAIT_OR_EXIT(mb_rec + (b ^ 1), 1u << (b ^ 1), (rpar >> (b ^ 1)) & 1u);
-            convert_v(slot_of(c + 1));
-            fence_proxy_async();
-            tc_fence_before();
-            __syncthreads();
-            if (tid == kMma) {
-                tc_fence_after();
-                issue_chunk_terms(c + 1);
-            }
-            ++nm;
-            pend |= 16u;
-        }
-        KDA_PHASE(2);
-
-        // ---- (D) Y = beta (V - X) (lanes 64..127), then O += PT Y
-        KDA_WAIT_OR_EXIT(mb_xo, 8u, (nxo - 1) & 1);
-        tc_fence_after();
-        {
-            const float* eg = reinterpret_cast<const float*>(slot + R::EGL);
-            egl = lt < DK ? eg[lt] : 1.f;
-            if (lt >= C) {
-                const int s = lt - C;
-                const float bs = reinterpret_cast<const float*>(slot + R::BETA)[s];
-                float x[NC];
-                tmem_ldn<NC>(t_O + lane_off + (uint32_t)(wg * NC), x);
-                tmem_wait_ld();
-                float y[NC];
-#pragma unroll
-                for (int u = 0; u < NC / 8; ++u) {
-                    const uint4 vr = *reinterpret_cast<const uint4*>(slot + PL::VOFF + swh_off(s, wg * NC + 8 * u, C));
-                    const __half2* v2 = reinterpret_cast<const __half2*>(&vr);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f2 = __half22float2(v2[e]);
-                        const int jj = 8 * u + 2 * e;
-                        y[jj] = bs * (f2.x - (no_erase ? 0.f : x[jj]));
-                        y[jj + 1] = bs * (f2.y - (no_erase ? 0.f : x[jj + 1]));
+                    for (int kk = 0; kk < DK / 16; ++kk)       // [O ; X] = [Qh ; Kh] S
+                        umma_f16(t_O, kdesc(slot + R::QK, kk, 128 * 128), mn_desc(Sop, kk, DK * 128), kIdv, kk > 0);
+                    umma_commit(mb_xo);
+                    ++cx;
+                    did = true;
+                } else if (cm < nchunks && ci >= cm && mbar_test(bar_v16 + (cm & 1), (cm >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_chunk_terms(cm);
+                    ++cm;
+                    did = true;
+                }
+                if (did) {
+                    t0 = clock64();
+                } else {
+                    __nanosleep(16);
+                    if (*abort_flag) goto finish;
+                    if (clock64() - t0 > tmo) {
+                        *abort_flag = 1;
+                        flag_timeout();
+                        goto finish;
                     }
                 }
-                st_row_h16n<NC>(Yb, s, wg * NC, C, y);
             }
         }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == kMma) {
-            tc_fence_after();
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ V tiles to fp16
+        const int t = tid - 32;
+        for (int c = 0; c < nchunks; ++c) {
+            if (!wt(mb_rec + (c & 1), c >> 1)) goto finish;
+            uint4* vt = reinterpret_cast<uint4*>(slot_of(c) + PL::VOFF);
+#pragma unroll 4
+            for (int i = t; i < C * DV * 2 / 16; i += 96) {
+                uint4 u = vt[i];
+                uint32_t* w = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)     // O += PT Y  (rows 64..127: discarded)
-                umma_f16(t_O, kdesc(slot + R::PT, kk, 0), mn_desc(Yb, kk, C * 128), kIdv, 1);
-            umma_commit(mb_o);
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                    w[e] = pack_f16(f.x, f.y);
+                }
+                vt[i] = u;
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_v16 + (c & 1));
         }
-        ++no;
-        pend |= 32u;
-        KDA_PHASE(3);
-
-        // ---- (F) M' of chunk c + 1
-        if (more) {
-            KDA_WAIT_OR_EXIT(mb_m, 16u, (nm - 1) & 1);
+    } else if (state_warp) {
+        // ------------------------------------------------------------ state
+        float S[SC];   // rows >= DK unused
+        {
+            const bool own = lt < DK && p.s_in;
+            const float* src = own ? p.s_in + (((size_t)n * H + h) * DK + lt) * DV + hh * SC : nullptr;
+#pragma unroll
+            for (int j = 0; j < SC; j += 4) {
+                const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
+            }
+        }
+        // M' = -D_M to packed fp16 in TMEM at t_M + DK / 4.  Warp half hh reads
+        // fp32 columns [hh DK / 2, (hh + 1) DK / 2) and writes its packed columns
+        // inside that range, 16 columns at a time, in an order that only
+        // overwrites columns it has already read (descending for hh = 0,
+        // ascending for hh = 1), so no other warp's reads are in the way.
+        auto convert_m = [&]() {
+            constexpr int NP = DK / 32;   // 16-column pieces per warp
+#pragma unroll
+            for (int i = 0; i < NP; ++i) {
+                const int piece = hh == 0 ? NP - 1 - i : i;
+                const int col = hh * (DK / 2) + 16 * piece;          // fp32 source column
+                float m[16];
+                tmem_ld16(t_M + lane_off + (uint32_t)col, m);
+                tmem_wait_ld();
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pk[e] = pack_f16(-m[2 * e], -m[2 * e + 1]);
+                tmem_st8(t_M + lane_off + (uint32_t)(DK / 4 + col / 2), pk);   // K pair (col, col + 1) -> col / 2
+            }
+            tmem_wait_st();
+        };
+        // bar_mconv(c) is raised only after mb_m(c) completed (with or without
+        // the conversion), so it also tells the issuer that B_c is in D_S, and
+        // it cannot run a phase ahead of the issuer
+        float egl_prev = 1.f;
+        if (nchunks > 0) {
+            if (!wt(mb_m, 0)) goto finish;
             tc_fence_after();
             if (!no_erase) convert_m();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_mconv);
         }
-
-        // ---- (E) o rows of chunk c (lanes 0..63); slot c % 2 then takes chunk c + 2
-        KDA_WAIT_OR_EXIT(mb_o, 32u, (no - 1) & 1);
-        tc_fence_after();
-        if (lt < C) {
-            float acc[NC];
-            tmem_ldn<NC>(t_O + lane_off + (uint32_t)(wg * NC), acc);
-            tmem_wait_ld();
-            if (lt < L) {
-                TO* dst = static_cast<TO*>(p.o) + ((size_t)(tok0 + c * C + lt) * H + h) * DV + wg * NC;
-                if constexpr (sizeof(TO) == 4) {
+        for (int c = 0; c < nchunks; ++c) {
+            unsigned char* slot = slot_of(c);
+            KDA_PHASE(0);
+            if (!wt(bar_v16 + (c & 1), c >> 1)) goto finish;   // record c is in its slot
+            if (c > 0) {
+                if (!wt(mb_chain, c - 1)) goto finish;
+                tc_fence_after();
+            }
+            {
+                unsigned char* Sop = sop_of(c);
 #pragma unroll
-                    for (int j = 0; j < NC; j += 4)
-                        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-                } else {
+                for (int u = 0; u < SC / 16; ++u) {   // 16 columns at a time: update, then the fp16 operand
+                    if (c > 0) {
+                        float d[16];
+                        tmem_ld16(tmem + 128 * ((c - 1) & 1) + lane_off + (uint32_t)(hh * SC + 16 * u), d);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < NC; j += 8)
-                        *reinterpret_cast<uint4*>(dst + j) =
-                            make_uint4(pack_bf16(acc[j], acc[j + 1]), pack_bf16(acc[j + 2], acc[j + 3]),
-                                       pack_bf16(acc[j + 4], acc[j + 5]), pack_bf16(acc[j + 6], acc[j + 7]));
+                        for (int j = 0; j < 16; ++j) S[16 * u + j] = fmaf(egl_prev, S[16 * u + j], d[j]);
+                    }
+                    if (lt < DK) st_row_h16n<16>(Sop, lt, hh * SC + 16 * u, DK, S + 16 * u);
                 }
             }
-        }
-        if (c + 2 < nchunks) {
-            if (tid == kCopy) {
-                fence_proxy_async();
-                issue_rec(c + 2);
+            egl_prev = lt < DK ? reinterpret_cast<const float*>(slot + R::EGL)[lt] : 1.f;
+            fence_proxy_async();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_sop);
+            KDA_PHASE(1);
+            if (c + 1 < nchunks) {   // M' of chunk c + 1
+                if (!wt(mb_m, c + 1)) goto finish;
+                tc_fence_after();
+                if (!no_erase) convert_m();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_mconv);
             }
-            pend |= 1u << b;
-            rpar = (rpar & ~(1u << b)) | ((uint32_t)(((c + 2) >> 1) & 1) << b);
+            KDA_PHASE(2);
         }
-        KDA_PHASE(4);
-    }
-
-    if (nchunks > 0) {   // state after the last chunk
-        KDA_WAIT_OR_EXIT(mb_chain, 4u, (nchain - 1) & 1);
-        tc_fence_after();
-        float d[NC];
-        tmem_ldn<NC>(tmem + 128 * ((nchunks - 1) & 1) + lane_off + (uint32_t)(wg * NC), d);
-        tmem_wait_ld();
+        if (nchunks > 0) {   // state after the last chunk
+            if (!wt(mb_chain, nchunks - 1)) goto finish;
+            tc_fence_after();
 #pragma unroll
-        for (int j = 0; j < NC; ++j) S[j] = fmaf(egl, S[j], d[j]);
-    }
-    if (p.s_out && lt < DK) {
-        float* dst = p.s_out + (((size_t)n * H + h) * DK + lt) * DV + wg * NC;
+            for (int u = 0; u < SC / 16; ++u) {
+                float d[16];
+                tmem_ld16(tmem + 128 * ((nchunks - 1) & 1) + lane_off + (uint32_t)(hh * SC + 16 * u), d);
+                tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < NC; j += 4)
-            *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                for (int j = 0; j < 16; ++j) S[16 * u + j] = fmaf(egl_prev, S[16 * u + j], d[j]);
+            }
+        }
+        if (p.s_out && lt < DK) {
+            float* dst = p.s_out + (((size_t)n * H + h) * DK + lt) * DV + hh * SC;
+#pragma unroll
+            for (int j = 0; j < SC; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+    } else {
+        // ------------------------------------------------------------ output
+        for (int c = 0; c < nchunks; ++c) {
+            unsigned char* slot = slot_of(c);
+            const int L = min(C, len - c * C);
+            if (quad >= 2) {   // Y = beta (V - X), rows s = lane - 64 of D_O
+                if (!wt(bar_v16 + (c & 1), c >> 1)) goto finish;   // V tile in fp16, beta in the slot
+                if (!wt(mb_xo, c)) goto finish;
+                tc_fence_after();
+                const int s = lt - C;
+                const float bs = reinterpret_cast<const float*>(slot + R::BETA)[s];
+#pragma unroll
+                for (int u = 0; u < DV / 16; ++u) {
+                    float x[16];
+                    tmem_ld16(t_O + lane_off + (uint32_t)(16 * u), x);
+                    tmem_wait_ld();
+                    float y[16];
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        const uint4 vr = *reinterpret_cast<const uint4*>(slot + PL::VOFF + swh_off(s, 16 * u + 8 * g, C));
+                        const __half2* v2 = reinterpret_cast<const __half2*>(&vr);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f2 = __half22float2(v2[e]);
+                            const int jj = 8 * g + 2 * e;
+                            y[jj] = bs * (f2.x - (no_erase ? 0.f : x[jj]));
+                            y[jj + 1] = bs * (f2.y - (no_erase ? 0.f : x[jj + 1]));
+                        }
+                    }
+                    st_row_h16n<16>(Yb, s, 16 * u, C, y);
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_y);
+            } else {           // o rows s = lane of D_O
+                if (!wt(mb_o, c)) goto finish;
+                tc_fence_after();
+                if (tid == kCopy && c + 2 < nchunks) {   // PT Y of chunk c has completed: its slot is free
+                    fence_proxy_async();
+                    if (!issue_rec(c + 2)) goto finish;
+                }
+                const int s = lt;
+                TO* dst = static_cast<TO*>(p.o) + ((size_t)(tok0 + c * C + s) * H + h) * DV;
+#pragma unroll
+                for (int u = 0; u < DV / 16; ++u) {
+                    float acc[16];
+                    tmem_ld16(t_O + lane_off + (uint32_t)(16 * u), acc);
+                    tmem_wait_ld();
+                    if (s < L) {
+                        if constexpr (sizeof(TO) == 4) {
+#pragma unroll
+                            for (int j = 0; j < 16; j += 4)
+                                *reinterpret_cast<float4*>(dst + 16 * u + j) =
+                                    make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; j += 8)
+                                *reinterpret_cast<uint4*>(dst + 16 * u + j) =
+                                    make_uint4(pack_bf16(acc[j], acc[j + 1]), pack_bf16(acc[j + 2], acc[j + 3]),
+                                               pack_bf16(acc[j + 4], acc[j + 5]), pack_bf16(acc[j + 6], acc[j + 7]));
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_ofree);
+            }
+        }
     }
 
 finish:
     KDA_PHASE_FLUSH
+    __syncthreads();
     if (*abort_flag) {
         // let every copy and MMA in flight land before the TMEM is released
         volatile int never = 0;
-        for (int i = 0; i < 2; ++i)
-            if (pend & (1u << i)) (void)mbar_wait(mb_rec + i, (rpar >> i) & 1u, &never, p.timeout_cycles);
-        if (pend & 4u) (void)mbar_wait(mb_chain, (uint32_t)((nchain - 1) & 1), &never, p.timeout_cycles);
-        if (pend & 8u) (void)mbar_wait(mb_xo, (uint32_t)((nxo - 1) & 1), &never, p.timeout_cycles);
-        if (pend & 16u) (void)mbar_wait(mb_m, (uint32_t)((nm - 1) & 1), &never, p.timeout_cycles);
-        if (pend & 32u) (void)mbar_wait(mb_o, (uint32_t)((no - 1) & 1), &never, p.timeout_cycles);
-        __syncthreads();
-        if (tid == kMma) umma_commit(mb_o);
-        (void)mbar_wait(mb_o, (uint32_t)(no & 1), &never, p.timeout_cycles);
+        if (tid == 0 && mma_issued) {
+            umma_commit(mb_fin);
+            (void)mbar_wait(mb_fin, 0u, &never, tmo);
+        }
+        if (tid == kCopy)
+            for (int i = max(0, rec_issued - 2); i < rec_issued; ++i)
+                (void)mbar_wait(mb_rec + (i & 1), (uint32_t)((i >> 1) & 1), &never, tmo);
     }
     tc_fence_before();
     __syncthreads();
