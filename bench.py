@@ -56,6 +56,28 @@ def flops_per_token_head(dk, dv, C=64):
     return (2 * (C - 1) + (C + 1)) * dk + 2 * C * dv + 6 * dk * dv + C * C / 3.0
 
 
+def bwd_flops_per_token_head(dk, dv, C=64):
+    """Algorithmic FLOPs per (token, head) of the chunkwise backward (dense
+    products, per chunk, divided by C): the forward recompute (MA and P over
+    d_k, X = Kh S, U = T Y, the state update, the UT transform) and the adjoint
+    products (dU, dY, dP, dT, T^T dT T^T, the three d_k-wide gradient
+    accumulations and the state-gradient update)."""
+    fwd = 2 * (2 * C * C * dk) + 2 * C * dk * dv + 2 * C * C * dv + 2 * dk * C * dv + C ** 3 / 3
+    adj = (2 * C * C * dv + 2 * C * dk * dv          # dU = P^T dO + Kl dS'
+           + 2 * C * C * dv + 2 * C * C * dv         # dY = T^T dU, dP = dO U^T
+           + 2 * C * C * dv + 2 * 2 * C * C * C      # dT = dU Y^T, T^T dT T^T
+           + 3 * 2 * C * dk * dv + 5 * 2 * C * C * dk  # dO S^T, dX S^T, U dS'^T; dP, dMA products
+           + 2 * 2 * dk * C * dv)                    # dS = Qh^T dO + Kh^T dX
+    return (fwd + adj) / C
+
+
+def fp32_alu_peak_tflops(device=None):
+    """CUDA-core fp32 peak from unit counts: SMs x 128 FP32 lanes x 2 FLOP (FMA)
+    x the maximum SM clock (1965 MHz on these B200s)."""
+    nsm = torch.cuda.get_device_properties(device).multi_processor_count if device is not None else 148
+    return nsm * 128 * 2 * 1.965e9 / 1e12
+
+
 def chunk_work(B, T, H, dk, dv, elem=2, o_elem=2, state_in=True, state_out=True):
     th = B * T * H
     nbytes = th * bytes_per_token_head(dk, dv, elem, o_elem)
@@ -416,7 +438,43 @@ def run_other_workloads(kda, device, stream, world, rank, reps=20):
             out[name]["tflops"] = nflops * world / t / 1e12
         del d, o, sN, ws
         torch.cuda.empty_cache()
+    out["prefill_backward"] = run_backward(kda, device, stream, world, rank, reps=max(3, min(reps, 5)))
     return out
+
+
+def run_backward(kda, device, stream, world, rank, reps=3):
+    """The chunkwise backward (fp32, CUDA cores) on the prefill shape: gradients
+    of sum(o * dO) + sum(S_T * dS_T) for random dO, dS_T."""
+    from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
+    w = WORKLOADS["prefill"]
+    d = make_inputs(w, device, seed=w.seed + 1000 * rank)
+    g = torch.Generator(device=device).manual_seed(7 + rank)
+    do = torch.randn(w.B, w.T, w.H, w.dv, generator=g, device=device)
+    dsT = torch.randn(w.B, w.H, w.dk, w.dv, generator=g, device=device)
+    call = lambda: kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], d["initial_state"], do, dsT,
+                                     stream=stream)
+    call()
+    torch.cuda.synchronize(device)
+    ev = event_pairs(reps)
+    barrier(world, device)
+    for a, b in ev:
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    kda.kda_check()
+    t = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3, world, device)
+    th = w.B * w.T * w.H
+    nflops = th * bwd_flops_per_token_head(w.dk, w.dv)
+    peak = fp32_alu_peak_tflops(device)
+    achieved = nflops / t / 1e12
+    return {"workload": f"backward, prefill shape: B={w.B} H={w.H} T={w.T} d_k=d_v={w.dk}, bf16 q/k/v, fp32 "
+                        "gradients, CUDA-core kernel",
+            "ms": t * 1e3, "tokens_per_s": w.B * w.T * world / t,
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_kind": "fp32 FMA: SMs x 128 lanes x 2 x 1965 MHz",
+                         "flops_per_launch": nflops},
+            "gpu_launches_per_call": 1}
 
 
 def run_e2e(kda, host_inputs, w, device, stream, world, ws, steps):
