@@ -71,6 +71,16 @@ def bwd_flops_per_token_head(dk, dv, C=64):
     return (fwd + adj) / C
 
 
+def dplr_flops_per_token_head(dk, dv, C=64):
+    """Algorithmic FLOPs per (token, head) of the diagonal-plus-low-rank chunk
+    forward (dense products per chunk / C): the four intra-chunk products over
+    d_k, (e^Gx a) S and A_ak V, U = T W, the output's three products, the two
+    state-update products, and the triangular solve."""
+    per_chunk = (4 * 2 * C * C * dk + 2 * C * dk * dv + 2 * C * C * dv + 2 * C * C * dv
+                 + 2 * C * dk * dv + 2 * 2 * C * C * dv + 2 * 2 * dk * C * dv + C ** 3 / 3)
+    return per_chunk / C
+
+
 def fp32_alu_peak_tflops(device=None):
     """CUDA-core fp32 peak from unit counts: SMs x 128 FP32 lanes x 2 FLOP (FMA)
     x the maximum SM clock (1965 MHz on these B200s)."""
@@ -439,7 +449,43 @@ def run_other_workloads(kda, device, stream, world, rank, reps=20):
         del d, o, sN, ws
         torch.cuda.empty_cache()
     out["prefill_backward"] = run_backward(kda, device, stream, world, rank, reps=max(3, min(reps, 5)))
+    out["prefill_dplr"] = run_dplr(kda, device, stream, world, rank, reps=max(3, min(reps, 5)))
     return out
+
+
+def run_dplr(kda, device, stream, world, rank, reps=3):
+    """The diagonal-plus-low-rank transition's chunk forward (fp32, CUDA cores)
+    on the prefill shape, with a, b ~ N(0, 0.7^2 / d_k)."""
+    from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
+    w = WORKLOADS["prefill"]
+    d = make_inputs(w, device, seed=w.seed + 1000 * rank)
+    g = torch.Generator(device=device).manual_seed(11 + rank)
+    ab = [(torch.randn(w.B, w.T, w.H, w.dk, generator=g, device=device) * 0.7 / w.dk ** 0.5).to(torch.bfloat16)
+          for _ in range(2)]
+    o = torch.empty(w.B, w.T, w.H, w.dv, device=device)
+    sN = torch.empty(w.B, w.H, w.dk, w.dv, device=device)
+    call = lambda: kda.kda_dplr_fwd(d["q"], d["k"], d["v"], ab[0], ab[1], d["log_alpha"], d["initial_state"],
+                                    o=o, final_state=sN, stream=stream)
+    call()
+    torch.cuda.synchronize(device)
+    ev = event_pairs(reps)
+    barrier(world, device)
+    for a, b in ev:
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    kda.kda_check()
+    t = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3, world, device)
+    nflops = w.B * w.T * w.H * dplr_flops_per_token_head(w.dk, w.dv)
+    peak = fp32_alu_peak_tflops(device)
+    return {"workload": f"diagonal-plus-low-rank transition, prefill shape: B={w.B} H={w.H} T={w.T} "
+                        f"d_k=d_v={w.dk}, bf16 q/k/v/a/b, fp32 o and state, CUDA-core kernel",
+            "ms": t * 1e3, "tokens_per_s": w.B * w.T * world / t,
+            "roofline": {"bound": "alu", "achieved": nflops / t / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": nflops / t / 1e12 / peak, "peak_kind": "fp32 FMA: SMs x 128 lanes x 2 x 1965 MHz",
+                         "flops_per_launch": nflops},
+            "gpu_launches_per_call": 1}
 
 
 def run_backward(kda, device, stream, world, rank, reps=3):
@@ -600,6 +646,41 @@ def run_reference(args, world, rank):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_case(args):
+    """One library call of the named workload, --warmup + --steps times on cuda:0
+    (for profiler command lines: a handful of launches, nothing else timed)."""
+    import gated_delta_rule_133_b200 as kda
+    from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    name = {"backward": "prefill", "dplr": "prefill"}.get(args.case, args.case)
+    w = WORKLOADS[name]
+    if args.case == "long" and args.case_tokens:
+        w = type(w)(**{**w.__dict__, "T": args.case_tokens})
+    d = make_inputs(w, device)
+    if args.case == "decode":
+        state = d["initial_state"].clone()
+        call = lambda i: kda.kda_recurrent_step(d["q"][i % w.T], d["k"][i % w.T], d["v"][i % w.T], d["beta"][i % w.T],
+                                                d["log_alpha"][i % w.T], state)
+    elif args.case == "backward":
+        g = torch.Generator(device=device).manual_seed(7)
+        do = torch.randn(w.B, w.T, w.H, w.dv, generator=g, device=device)
+        call = lambda i: kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], d["initial_state"], do)
+    elif args.case == "dplr":
+        g = torch.Generator(device=device).manual_seed(11)
+        a, b = [(torch.randn(w.B, w.T, w.H, w.dk, generator=g, device=device) * 0.7 / w.dk ** 0.5).to(torch.bfloat16)
+                for _ in range(2)]
+        call = lambda i: kda.kda_dplr_fwd(d["q"], d["k"], d["v"], a, b, d["log_alpha"], d["initial_state"])
+    else:
+        ws = torch.empty(kda.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv), dtype=torch.uint8, device=device)
+        call = lambda i: kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["log_alpha"], d["initial_state"],
+                                           workspace=ws)
+    for i in range(args.warmup + args.steps):
+        call(i)
+    torch.cuda.synchronize(device)
+    kda.kda_check()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -608,8 +689,15 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-others", action="store_true", help="skip the prefill / varlen / variant timings")
+    ap.add_argument("--case", choices=["prefill", "long", "decode", "backward", "dplr"], default=None,
+                    help="profiling aid: run only this call --steps times after --warmup calls, print nothing")
+    ap.add_argument("--case-tokens", type=int, default=0,
+                    help="with --case long: tokens of the sequence (default: the workload's 131072)")
     args = ap.parse_args(argv)
     world, rank, local = dist_env()
+    if args.case:
+        run_case(args)
+        return 0
     if args.impl == "reference":
         line = run_reference(args, world, rank)
         if line is not None:

@@ -32,7 +32,8 @@ from . import _lib
 from ._lib import KdaError
 
 __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_varlen_fwd", "kda_recurrent_step", "kda_check",
-           "kda_chunk_bwd", "kda_varlen_bwd", "chunk_fwd_workspace_size", "varlen_fwd_workspace_size", "KdaError"]
+           "kda_chunk_bwd", "kda_varlen_bwd", "kda_dplr_fwd", "kda_dplr_varlen_fwd", "chunk_fwd_workspace_size",
+           "varlen_fwd_workspace_size", "KdaError"]
 
 _DTYPES = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
 
@@ -273,6 +274,59 @@ def kda_varlen_bwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state, grad_o, 
               _ptr(initial_state), _ptr(grad_o), _ptr(grad_final_state), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gb),
               _ptr(gla), _ptr(gs0), T, H, dk, dv, chunk, _DTYPES[dt], *ws, _stream(stream))
     return gq, gk, gv, gb, gla, gs0
+
+
+def kda_dplr_fwd(q, k, v, a, b, log_alpha, initial_state=None, *, o=None, final_state=None,
+                 output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None):
+    """Diagonal-plus-low-rank transition S_t = (Diag(alpha_t) + b_t a_t^T) S_{t-1} + k_t v_t^T,
+    o_t = S_t^T q_t.  q, k, a, b [B, T, H, dk], v [B, T, H, dv] (bf16 or fp32);
+    log_alpha [B, T, H, dk] fp32; initial_state [B, H, dk, dv] or None.
+    Returns (o, final_state or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for t, n, s_, d in ((q, "q", (B, T, H, dk), dt), (k, "k", (B, T, H, dk), dt), (v, "v", (B, T, H, dv), dt),
+                        (a, "a", (B, T, H, dk), dt), (b, "b", (B, T, H, dk), dt),
+                        (log_alpha, "log_alpha", (B, T, H, dk), torch.float32)):
+        _check(t, n, s_, d, dev)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=o_dtype, device=dev)
+    _check(o, "o", (B, T, H, dv), o.dtype, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    _lib.call("kda_dplr_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(log_alpha), _ptr(initial_state),
+              _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk, _DTYPES[dt], _DTYPES[o.dtype], _stream(stream))
+    return o, final_state
+
+
+def kda_dplr_varlen_fwd(q, k, v, a, b, log_alpha, cu_seqlens, initial_state=None, *, o=None, final_state=None,
+                        output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None):
+    """kda_dplr_fwd over N packed variable-length sequences ([T, H, ...] layouts)."""
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.shape[0] - 1
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for t, n, s_, d in ((q, "q", (T, H, dk), dt), (k, "k", (T, H, dk), dt), (v, "v", (T, H, dv), dt),
+                        (a, "a", (T, H, dk), dt), (b, "b", (T, H, dk), dt),
+                        (log_alpha, "log_alpha", (T, H, dk), torch.float32), (cu_seqlens, "cu_seqlens", (N + 1,), torch.int32)):
+        _check(t, n, s_, d, dev)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (N, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=o_dtype, device=dev)
+    _check(o, "o", (T, H, dv), o.dtype, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    _lib.call("kda_dplr_varlen_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(log_alpha), _ptr(cu_seqlens),
+              N, _ptr(initial_state), _ptr(o), _ptr(final_state), T, H, dk, dv, chunk, _DTYPES[dt], _DTYPES[o.dtype],
+              _stream(stream))
+    return o, final_state
 
 
 def kda_check(stream=None):

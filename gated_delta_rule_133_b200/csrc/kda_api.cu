@@ -336,6 +336,41 @@ kda_status kda_varlen_bwd(const void* q, const void* k, const void* v, const flo
                                     dv, dtype, workspace, workspace_bytes_, s));
 }
 
+kda_status kda_dplr_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
+                        const float* log_alpha, const float* initial_state, void* o, float* final_state, int B, int T,
+                        int H, int dk, int dv, int chunk, kda_dtype dtype, kda_dtype o_dtype, void* stream)
+{
+    if (B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    const long long tokens = (long long)B * T;
+    kda_status st = check_fwd(q, k, v, (const float*)q, log_alpha, initial_state, o, final_state, tokens, H, dk, dv,
+                              chunk, dtype, o_dtype, 0);
+    if (st != KDA_OK) return st;
+    if (tokens > 0 && (!a || !b || !aligned16(a) || !aligned16(b))) return KDA_ERR_INVALID_ARG;
+    if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tokens == 0) return copy_state(initial_state, final_state, (size_t)B * H * dk * dv, s);
+    return from_cuda(kda::dplr_fwd(q, k, v, a, b, log_alpha, initial_state, o, final_state, nullptr, B, T, tokens, H, dk,
+                                   dv, dtype, o_dtype, s));
+}
+
+kda_status kda_dplr_varlen_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
+                               const float* log_alpha, const int32_t* cu_seqlens, int N, const float* initial_state,
+                               void* o, float* final_state, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                               kda_dtype o_dtype, void* stream)
+{
+    if (N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_fwd(q, k, v, (const float*)q, log_alpha, initial_state, o, final_state, T, H, dk, dv, chunk,
+                              dtype, o_dtype, 0);
+    if (st != KDA_OK) return st;
+    if (T > 0 && (!a || !b || !aligned16(a) || !aligned16(b))) return KDA_ERR_INVALID_ARG;
+    if (N == 0) return T == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
+    if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) return copy_state(initial_state, final_state, (size_t)N * H * dk * dv, s);
+    return from_cuda(kda::dplr_fwd(q, k, v, a, b, log_alpha, initial_state, o, final_state, cu_seqlens, N, 0, T, H, dk,
+                                   dv, dtype, o_dtype, s));
+}
+
 kda_status kda_check(void* stream)
 {
     cudaStream_t s = static_cast<cudaStream_t>(stream);

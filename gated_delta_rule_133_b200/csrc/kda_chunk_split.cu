@@ -459,40 +459,6 @@ __device__ __forceinline__ void ut_rows(float* As, float* X, unsigned char* Top)
     }
 }
 
-// UT transform T = (I + A)^-1 of the strictly lower 64 x 64 A by forward
-// substitution, one column of T per thread (threads 0..63):
-//   T[j][j] = 1,   T[r][j] = -sum_{j <= s < r} A[r][s] T[s][j]   (r > j).
-// The column lives in registers (T[s][j] = 0 for s < j, so the sum may run
-// from s = 0); rows of A (As[r * LDT + s], zero for s >= r) are read as
-// float4s that every lane of a warp reads at the same address (broadcast), and
-// eight partial sums shorten the dependent chain.  Column j of T is row j of
-// T^T, written to Top as fp16 (K-major 128-byte swizzle).
-__device__ __forceinline__ void ut_columns(const float* As, unsigned char* Top)
-{
-    const int j = threadIdx.x;
-    float x[C];
-#pragma unroll
-    for (int r = 0; r < C; ++r) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int q = 0; 4 * q < r; ++q) {
-            const float4 a = ld4(As + r * LDT + 4 * q);
-            const int b = 4 * (q & 1);
-            if (4 * q + 0 < r) acc[b + 0] = fmaf(a.x, x[4 * q + 0], acc[b + 0]);
-            if (4 * q + 1 < r) acc[b + 1] = fmaf(a.y, x[4 * q + 1], acc[b + 1]);
-            if (4 * q + 2 < r) acc[b + 2] = fmaf(a.z, x[4 * q + 2], acc[b + 2]);
-            if (4 * q + 3 < r) acc[b + 3] = fmaf(a.w, x[4 * q + 3], acc[b + 3]);
-        }
-        const float sum = ((acc[0] + acc[4]) + (acc[1] + acc[5])) + ((acc[2] + acc[6]) + (acc[3] + acc[7]));
-        x[r] = r > j ? -sum : (r == j ? 1.f : 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < C / 8; ++u)
-        *reinterpret_cast<uint4*>(Top + swh_off(j, 8 * u, C)) =
-            make_uint4(pack_f16(x[8 * u], x[8 * u + 1]), pack_f16(x[8 * u + 2], x[8 * u + 3]),
-                       pack_f16(x[8 * u + 4], x[8 * u + 5]), pack_f16(x[8 * u + 6], x[8 * u + 7]));
-}
-
 // One persistent CTA per SM walks items blockIdx.x, + gridDim.x, ...  The
 // UT transform of item k (warpgroup 0) overlaps the gate cumsum and operand
 // build of item k + 1 (warpgroups 1-3); one MMA round then forms Z, PT of
@@ -736,11 +702,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
             float pt[16];
             tmem_ld16(t_PT + lane_off + q_off, pt);
             tmem_wait_ld();
-            if (lt < DK) {   // the record keeps Z diag(beta)
-#pragma unroll
-                for (int j = 0; j < 16; ++j) z[j] *= vcur.beta[16 * wg + j];
-                st_row_h16(stg, lt, 16 * wg, DK, z);
-            }
+            if (lt < DK) st_row_h16(stg, lt, 16 * wg, DK, z);
             if (lt < C) st_row_h16(stg + (R::PT - R::Z), lt, 16 * wg, C, pt);
             if (tid < DK) reinterpret_cast<float*>(stg + (R::EGL - R::Z))[tid] = vcur.egl[tid];
             else if (tid >= 256 && tid < 256 + C) reinterpret_cast<float*>(stg + (R::BETA - R::Z))[tid - 256] = vcur.beta[tid - 256];
@@ -804,109 +766,127 @@ struct ScanParams {
     int no_erase;            // KDA_MODE_NO_ERASE: Y = beta V (no X term)
 };
 
-// Shared memory of the scan kernel (one CTA per (sequence, head), all d_v
-// columns).  Two record slots, each holding one record as stored followed by
-// the chunk's V tile [64][DV] (bf16 from TMA, converted to fp16 in place; the
-// M = 128 reads of the 64-row PT tile, and for d_k = 64 of the Z tile, run on
-// into rows whose products are discarded); the state operand S [DK][DV] twice
-// (fp16, MN-major: value columns contiguous, 128-byte swizzle); Y [64][DV]
-// (fp16, MN-major).  The mbarriers sit in the gap between slot 0's record and
-// its V tile.
-template <int DK, int DV>
+// Shared memory of the scan kernel: two 72 KB slots, each holding one record
+// (the M = 128 reads of the 64-row PT tile, and for d_k = 64 of the Z tile,
+// run on into the rest of the record's 64 KB, into rows whose products are
+// discarded) and the chunk's V tile [64][NV] (bf16, 128-byte swizzle) at
+// +64 KB; the state operand S [d_k][NV] and Y [64][NV] (fp16, MN-major B
+// operands: value columns contiguous, 128-byte swizzle); the o staging tile
+// [64][NV] (output type, 16-byte chunks XOR-swizzled by row).
+template <int DK>
 struct ScanPlan {
-    static constexpr int VOFF = (Rec<DK>::BYTES + 1023) & ~1023;
-    static constexpr int SLOT = VOFF + C * DV * 2;
+    static constexpr int SLOT = 73728, VOFF = 65536;
     static constexpr int SOP = 2 * SLOT;
-    static constexpr int YB = SOP + 2 * DK * DV * 2;
-    static constexpr int END = YB + C * DV * 2;
-    static constexpr int BAR = Rec<DK>::BYTES;
+    static constexpr int YB = SOP + NV * DK * 2;
+    static constexpr int OST = YB + NV * C * 2;
+    static constexpr int BAR = OST + C * NV * 4;
+    static constexpr int END = BAR + 128;
     static constexpr int BYTES = END + 1024;
 };
-static_assert(ScanPlan<128, 128>::BYTES <= 232448, "scan shared memory exceeds the per-CTA limit");
-static_assert(ScanPlan<128, 128>::VOFF - ScanPlan<128, 128>::BAR >= 128, "no room for the scan's barriers");
-static_assert(ScanPlan<64, 128>::VOFF - ScanPlan<64, 128>::BAR >= 128, "no room for the scan's barriers");
 
-// MN-major SW128 16-bit operand: K-step kk (16 K rows = two 1 KB groups)
-// starts 2 KB further on; 64-column atoms `atom_stride` bytes apart.
-__device__ __forceinline__ uint64_t mn_desc(const unsigned char* tile, int kk, int atom_stride)
+// MN-major SW128 B operand (16-bit, NV = 64 columns = one 128-byte row per K
+// index): K-step kk (16 K rows = two 1 KB groups) starts 2 KB further on.
+__device__ __forceinline__ uint64_t mn_desc(const unsigned char* tile, int kk, int k_rows)
 {
-    return sdesc_sw128(smem_u32(tile) + kk * 2048, (uint32_t)atom_stride, 1024);
+    return sdesc_sw128(smem_u32(tile) + kk * 2048, (uint32_t)(k_rows * 128), 1024);
 }
 
-// Stores NC consecutive values of one row of a 16-bit SW128 tile as fp16
-// (col0 a multiple of 8).
-template <int NC>
-__device__ __forceinline__ void st_row_h16n(unsigned char* tile, int row, int col0, int rows, const float* x)
+// Output rows [0, L) of one chunk from the TMEM accumulator (lane = row, 16
+// columns per warpgroup), run by the 256 threads of lanes 0..63.  Rows are
+// staged in the layout of the output tensor map's boxes (64 rows x 128 bytes,
+// 128-byte swizzle; two boxes for fp32 output); a full chunk leaves with TMA
+// stores issued by one thread, a partial one (the end of a sequence) with
+// coalesced 16-byte row-segment stores.
+template <typename TO>
+__device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost, const CUtensorMap* tmo, void* o,
+                                             int tok, int h, int col0, size_t row0_off, size_t row_stride, int L,
+                                             int lt, int wg, bool issuer)
 {
+    constexpr int EB = (int)sizeof(TO);
+    constexpr int CPB = 8;                 // 16-byte chunks per 128-byte box row
+    constexpr int CPT = EB;                // chunks per thread: 16 values
+    constexpr int NBOX = NV * EB / 128;
+    constexpr int CPR = NV * EB / 16;      // chunks per output row segment
+    float acc[16];
+    tmem_ld16(t_acc, acc);
+    if (issuer) bulk_wait_read();          // the previous chunk's stores have read the tile
+    tmem_wait_ld();
+    bar_sync(1, 256);
 #pragma unroll
-    for (int u = 0; u < NC / 8; ++u)
-        *reinterpret_cast<uint4*>(tile + swh_off(row, col0 + 8 * u, rows)) =
-            make_uint4(pack_f16(x[8 * u], x[8 * u + 1]), pack_f16(x[8 * u + 2], x[8 * u + 3]),
-                       pack_f16(x[8 * u + 4], x[8 * u + 5]), pack_f16(x[8 * u + 6], x[8 * u + 7]));
+    for (int u = 0; u < CPT; ++u) {
+        const int k = wg * CPT + u, box = k / CPB, ci = k % CPB;
+        uint4 val;
+        if constexpr (EB == 4)
+            val = make_uint4(__float_as_uint(acc[4 * u]), __float_as_uint(acc[4 * u + 1]),
+                             __float_as_uint(acc[4 * u + 2]), __float_as_uint(acc[4 * u + 3]));
+        else
+            val = make_uint4(pack_bf16(acc[8 * u], acc[8 * u + 1]), pack_bf16(acc[8 * u + 2], acc[8 * u + 3]),
+                             pack_bf16(acc[8 * u + 4], acc[8 * u + 5]), pack_bf16(acc[8 * u + 6], acc[8 * u + 7]));
+        *reinterpret_cast<uint4*>(ost + box * 8192 + lt * 128 + ((ci ^ (lt & 7)) << 4)) = val;
+    }
+    fence_proxy_async();
+    bar_sync(1, 256);
+    if (L == C) {
+        if (issuer) {
+#pragma unroll
+            for (int bx = 0; bx < NBOX; ++bx) tma_store_3d(tmo, ost + bx * 8192, col0 + bx * (128 / EB), h, tok);
+            bulk_commit();
+        }
+    } else {
+        const int t = wg * 64 + lt;
+#pragma unroll
+        for (int pss = 0; pss < C * CPR / 256; ++pss) {
+            const int idx = pss * 256 + t, row = idx / CPR, k = idx % CPR;
+            if (row < L) {
+                const int box = k / CPB, ci = k % CPB;
+                const uint4 val = *reinterpret_cast<const uint4*>(ost + box * 8192 + row * 128 + ((ci ^ (row & 7)) << 4));
+                *reinterpret_cast<uint4*>(static_cast<unsigned char*>(o) + (row0_off + (size_t)row * row_stride) * EB + k * 16) = val;
+            }
+        }
+    }
 }
 
-template <int N>
-__device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[N])
-{
-    if constexpr (N == 32) tmem_ld32(taddr, v);
-    else tmem_ld16(taddr, v);
-}
-
-// One CTA per (sequence, head), warp-specialised.  The state update of a
-// chunk is one MMA round on the critical path:
-//
-//   S_{c+1} = diag(e^G_last) S_c + M'_c S_c + B_c,
-//   M'_c = -(Z diag(beta)) Kh  (d_k x d_k),   B_c = (Z diag(beta)) V  (d_k x d_v)
-//
-// (the record's Z tile already carries the beta factors).  M'_c and B_c depend
-// on the chunk alone: they are formed by MMAs issued a chunk ahead, M'_c
-// converted to fp16 in TMEM (the A operand of a TS-form MMA) and B_c left in
-// the accumulator the chain MMA adds to.  The output leaves the chain:
-// [O ; X] = [Qh ; Kh] S_c, Y = beta (V - X), O += PT Y.
-//
-// Warp roles (they synchronise through mbarriers, never CTA-wide barriers):
-//   warp 0       MMA issuer: issues each MMA group as soon as its inputs are
-//                ready, the state chain first;
-//   warps 1..3   V tile bf16 -> fp16, in place;
-//   warps 4..11  state: row 32 (w % 4) + lane, half of the value columns, in
-//                fp32 registers; S_op writes; M' conversion;
-//   warps 12..15 output: Y = beta (V - X) (lanes 64..127), o rows (lanes 0..63);
-//                lane 0 of warp 12 also issues the copies: the record and V
-//                tile of chunk c + 2 into the slot chunk c frees.
-// TMEM columns: D_S[2] (0, 128), D_O (256), D_M (384; M' packed over its
-// columns [DK / 4, 3 DK / 4)).
-template <typename TO, int DK, int DV, bool VAR>
-__device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const ScanParams& p, int bid)
+// One CTA per (sequence, head, NV value columns).  Thread (lane lt < d_k,
+// warpgroup wg) keeps S[lt][16 wg .. 16 wg + 16) of the state in registers.
+// Per chunk c (slot c % 2):
+//   S <- diag(e^G_last(c-1)) S + W(c-1)      W = Z Y of the chunk before, from TMEM
+//   S operand (fp16) -> smem;  MMA [O ; X] = [Qh ; Kh] S  -> TMEM buffer c % 2
+//   Y = diag(beta) (V - X) -> smem (lanes 64..127), while lanes 0..63 store
+//   the o rows of chunk c - 1
+//   MMA W = Z Y (commit), MMA O += PT Y
+// A slot is refilled in two parts as soon as the MMAs reading each part have
+// completed: the [Qh ; Kh] tile and V after chunk c's X MMA and Y phase, the
+// Z, PT, e^G_last and beta part after chunk c + 1's X MMA (tcgen05 MMAs of
+// one thread complete in issue order).
+template <typename TO, int DK, bool VAR>
+__device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensorMap& tmo, const ScanParams& p,
+                                          int bid)
 {
     const bool no_erase = VAR && p.no_erase;   // layer variant (VAR instantiations only)
-    using PL = ScanPlan<DK, DV>;
+    using PL = ScanPlan<DK>;
     using R = Rec<DK>;
-    constexpr int SC = DV / 2;                 // value columns per state warp
     extern __shared__ unsigned char smem_raw[];
     KDA_PHASE_DECL(1)
     unsigned char* sm = align1024(smem_raw);
+    unsigned char* Sop = sm + PL::SOP;
     unsigned char* Yb = sm + PL::YB;
+    unsigned char* Ost = sm + PL::OST;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::BAR);
-    uint64_t* mb_rec = bars + 0;     // [2] record + V tile of a slot (transaction bytes)
-    uint64_t* mb_chain = bars + 2;   // commits: chain MMA of a chunk
-    uint64_t* mb_m = bars + 3;       //          M' and B MMAs of a chunk
-    uint64_t* mb_xo = bars + 4;      //          [O ; X] MMA
-    uint64_t* mb_o = bars + 5;       //          PT Y MMA
-    uint64_t* bar_v16 = bars + 6;    // [2] V tile of a slot converted (warps 1..3)
-    uint64_t* bar_sop = bars + 8;    // S_op written (8 state warps)
-    uint64_t* bar_mconv = bars + 9;  // M' converted (8 state warps)
-    uint64_t* bar_y = bars + 10;     // Y written (2 output warps)
-    uint64_t* bar_ofree = bars + 11; // o rows read from D_O (2 output warps)
-    uint64_t* mb_fin = bars + 12;    // final commit of an aborted CTA
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+    uint64_t* mb_a = bars + 0;     // [2]: [Qh ; Kh] and V of a slot
+    uint64_t* mb_b = bars + 2;     // [2]: Z, PT, e^G_last and beta of a slot
+    uint64_t* mb_x = bars + 4;
+    uint64_t* mb_w = bars + 5;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3;
-    const int lt = quad * 32 + lane;           // TMEM lane of this thread
-    const int h = bid % p.H;
-    const int rank = bid / p.H;
-    const int H = p.H;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int lt = tid & 127;
+    const int wg = tid >> 7;
+    const int nslice = p.DV / NV;
+    const int slice = bid % nslice;
+    const int h = (bid / nslice) % p.H;
+    const int rank = bid / (nslice * p.H);
+    const int H = p.H, DV = p.DV;
     int n, tok0, len;
     long long j0;
     if (p.cu) {
@@ -920,6 +900,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const ScanPara
         len = p.T;
         j0 = (long long)n * p.rs - p.rc0;
     }
+    const int col0 = slice * NV;
     int nchunks = (len + C - 1) / C;
     if ((long long)tok0 + len > p.tokens || tok0 < 0) {
         if (tid == 0 && p.c_begin == 0) flag_bad_input();
@@ -940,351 +921,231 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const ScanPara
         nchunks = 0;
         len = 0;
     }
+    const float* s_src = p.s_in;
 
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
-        mbar_init(bar_v16 + 0, 3);
-        mbar_init(bar_v16 + 1, 3);
-        mbar_init(bar_sop, 8);
-        mbar_init(bar_mconv, 8);
-        mbar_init(bar_y, 2);
-        mbar_init(bar_ofree, 2);
-        mbar_init(mb_fin, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
         prefetch_tmap(&tmv);
+        prefetch_tmap(&tmo);
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_off = ((uint32_t)quad * 32) << 16;
-    const uint32_t t_O = tmem + 256, t_M = tmem + 384;
-    constexpr uint32_t kIdv = idesc_f16(128, DV, 1);    // N = d_v, B MN-major
-    constexpr uint32_t kIdk = idesc_f16(128, DK, 1);    // N = d_k, B MN-major
-    constexpr uint32_t kRecBytes = (uint32_t)R::BYTES + C * DV * 2;
-    const long long tmo = p.timeout_cycles;
-    auto slot_of = [&](int cc) { return sm + (cc & 1) * PL::SLOT; };
-    auto sop_of = [&](int cc) { return sm + PL::SOP + (cc & 1) * (DK * DV * 2); };
-    // bounded wait; false once this CTA has aborted (every role then leaves)
-    auto wt = [&](uint64_t* bar, int par) { return mbar_wait(bar, (uint32_t)(par & 1), abort_flag, tmo); };
+    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32) << 16;
+    const uint32_t q_off = (uint32_t)wg * 16;
+    const uint32_t t_W = tmem + 128;
+    constexpr uint32_t kI = idesc_f16(128, NV, 1);
+    constexpr uint32_t kBytesA = R::Z + C * NV * 2;     // [Qh ; Kh] tile + V tile
+    constexpr uint32_t kBytesB = R::BYTES - R::Z;       // Z, PT, e^G_last, beta
 
-    // state of the roles that outlive their loops (cleanup of an aborted CTA)
-    int rec_issued = 0;         // copy issuer: loads issued
-    bool mma_issued = false;    // MMA issuer: any MMA issued
-    constexpr int kCopy = 384;  // copy issuer: lane 0 of the output warp of lane quadrant 0
-    auto issue_rec = [&](int cc) {   // record and V tile of chunk cc into its slot (one thread)
-        unsigned char* slot = slot_of(cc);
-        const size_t ri = (size_t)(j0 + cc) * H + h;
-        if (p.ready && !wait_ready(p.ready + ri, abort_flag, tmo)) return false;
-        mbar_expect_tx(mb_rec + (cc & 1), kRecBytes);
-        bulk_load(slot, p.rec + ri * R::BYTES, (uint32_t)R::BYTES, mb_rec + (cc & 1));
-#pragma unroll
-        for (int a = 0; a < DV / 64; ++a)
-            tma_load_3d(slot + PL::VOFF + a * 8192, &tmv, mb_rec + (cc & 1), 64 * a, h, tok0 + cc * C);
-        ++rec_issued;
-        return true;
+    auto rec_of = [&](int cc) { return p.rec + ((size_t)(j0 + cc) * H + h) * R::BYTES; };
+    auto issue_a = [&](int cc) {
+        unsigned char* slot = sm + (cc & 1) * PL::SLOT;
+        if (p.ready && !wait_ready(p.ready + (size_t)(j0 + cc) * H + h, abort_flag, p.timeout_cycles)) return;
+        mbar_expect_tx(mb_a + (cc & 1), kBytesA);
+        bulk_load(slot, rec_of(cc), R::Z, mb_a + (cc & 1));
+        tma_load_3d(slot + PL::VOFF, &tmv, mb_a + (cc & 1), col0, h, tok0 + cc * C);
     };
-    if (tid == kCopy && nchunks > 0) {   // the first two records; chunk c's slot takes chunk c + 2 after its o rows
-        // a failed wait for a record sets the abort flag, which every role checks
-        if (issue_rec(0) && nchunks > 1) (void)issue_rec(1);
+    auto issue_b = [&](int cc) {
+        unsigned char* slot = sm + (cc & 1) * PL::SLOT;
+        mbar_expect_tx(mb_b + (cc & 1), kBytesB);
+        bulk_load(slot + R::Z, rec_of(cc) + R::Z, kBytesB, mb_b + (cc & 1));
+    };
+
+    // state rows of this thread
+    float S[16];
+    {
+        const bool own = lt < DK && s_src;
+        const float* src = own ? s_src + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg : nullptr;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+            const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
+        }
     }
 
-    const bool state_warp = warp >= 4 && warp < 12;
-    const int hh = (warp - 4) >> 2;            // state warps: value-column half
+    // thread 0 issues the MMAs; thread kIssuer every copy (record refills, V
+    // tiles, output stores)
+    constexpr int kIssuer = 32;
+    const bool issuer = tid == kIssuer;
+    unsigned pend = 0;                 // bits: 0-1 mb_a[slot], 2-3 mb_b[slot], 4 mb_x, 5 mb_w
+    uint32_t apar = 0u, bpar = 0u;     // bit i: phase parity of the pending load of slot i
+    int xph = 0, wph = 0;              // commits issued to mb_x / mb_w
+    int c = 0;
+    if (issuer)
+        for (int cc = 0; cc < 2 && cc < nchunks; ++cc) {
+            issue_a(cc);
+            issue_b(cc);
+        }
+    for (int cc = 0; cc < 2 && cc < nchunks; ++cc) pend |= (1u | 4u) << cc;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && nchunks > 0) {
-            auto issue_chunk_terms = [&](int cc) {   // D_M = Zb Kh, D_S[cc % 2] = Zb V
-                const unsigned char* slot = slot_of(cc);
-                if (!no_erase) {
-#pragma unroll
-                    for (int kk = 0; kk < C / 16; ++kk)
-                        umma_f16(t_M, kdesc(slot + R::Z, kk, 0), mn_desc(slot + R::QK + C * 128, kk, 128 * 128), kIdk,
-                                 kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_f16(tmem + 128 * (cc & 1), kdesc(slot + R::Z, kk, 0), mn_desc(slot + PL::VOFF, kk, C * 128),
-                             kIdv, kk > 0);
-                umma_commit(mb_m);
-            };
-            if (!wt(bar_v16, 0)) goto finish;
+    float eglp = 1.f;                  // e^G_last of the previous chunk, key channel lt
+    int Lprev = 0;
+    for (c = 0; c < nchunks; ++c) {
+        const int b = c & 1;
+        unsigned char* slot = sm + b * PL::SLOT;
+        const uint32_t t_XO = tmem + 64 * b;
+        const int L = min(C, len - c * C);
+        KDA_PHASE(0);
+
+        // ---- state of chunk c - 1, then its fp16 operand (row = value column)
+        if (c > 0) {
+            KDA_WAIT_OR_EXIT(mb_w, 32u, (c - 1) & 1);
             tc_fence_after();
-            issue_chunk_terms(0);
-            mma_issued = true;
-            int ci = 0, cm = 1, cx = 0, cp = 0;     // next chain, M'/B, [O ; X], PT Y chunk
-            long long t0 = clock64();
-            while (cp < nchunks) {
-                bool did = false;
-                if (ci < nchunks && (ci == 0 || cx >= ci) && mbar_test(bar_mconv, ci & 1) &&
-                    mbar_test(bar_sop, ci & 1)) {
-                    tc_fence_after();
-                    unsigned char* Sop = sop_of(ci);
-                    if (!no_erase) {
+            float w[16];
+            tmem_ld16(t_W + lane_off + q_off, w);
+            tmem_wait_ld();
 #pragma unroll
-                        for (int kk = 0; kk < DK / 16; ++kk)   // D_S += M' S  (M' from TMEM)
-                            umma_f16_ts(tmem + 128 * (ci & 1), t_M + DK / 4 + 8 * kk, mn_desc(Sop, kk, DK * 128), kIdv, 1);
-                    }
-                    umma_commit(mb_chain);
-                    ++ci;
-                    did = true;
-                } else if (cp < cx && mbar_test(bar_y, cp & 1)) {
-                    tc_fence_after();
-                    const unsigned char* slot = slot_of(cp);
-#pragma unroll
-                    for (int kk = 0; kk < C / 16; ++kk)       // O += PT Y  (rows 64..127: discarded)
-                        umma_f16(t_O, kdesc(slot + R::PT, kk, 0), mn_desc(Yb, kk, C * 128), kIdv, 1);
-                    umma_commit(mb_o);
-                    ++cp;
-                    did = true;
-                } else if (cx < ci && cx == cp && (cx == 0 || mbar_test(bar_ofree, (cx - 1) & 1))) {
-                    tc_fence_after();
-                    const unsigned char* slot = slot_of(cx);
-                    unsigned char* Sop = sop_of(cx);
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk)       // [O ; X] = [Qh ; Kh] S
-                        umma_f16(t_O, kdesc(slot + R::QK, kk, 128 * 128), mn_desc(Sop, kk, DK * 128), kIdv, kk > 0);
-                    umma_commit(mb_xo);
-                    ++cx;
-                    did = true;
-                } else if (cm < nchunks && ci >= cm && mbar_test(bar_v16 + (cm & 1), (cm >> 1) & 1)) {
-                    tc_fence_after();
-                    issue_chunk_terms(cm);
-                    ++cm;
-                    did = true;
-                }
-                if (did) {
-                    t0 = clock64();
-                } else {
-                    __nanosleep(16);
-                    if (*abort_flag) goto finish;
-                    if (clock64() - t0 > tmo) {
-                        *abort_flag = 1;
-                        flag_timeout();
-                        goto finish;
-                    }
-                }
-            }
+            for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ V tiles to fp16
-        const int t = tid - 32;
-        for (int c = 0; c < nchunks; ++c) {
-            if (!wt(mb_rec + (c & 1), c >> 1)) goto finish;
-            uint4* vt = reinterpret_cast<uint4*>(slot_of(c) + PL::VOFF);
-#pragma unroll 4
-            for (int i = t; i < C * DV * 2 / 16; i += 96) {
-                uint4 u = vt[i];
-                uint32_t* w = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-                    w[e] = pack_f16(f.x, f.y);
-                }
-                vt[i] = u;
-            }
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_v16 + (c & 1));
-        }
-    } else if (state_warp) {
-        // ------------------------------------------------------------ state
-        float S[SC];   // rows >= DK unused
-        {
-            const bool own = lt < DK && p.s_in;
-            const float* src = own ? p.s_in + (((size_t)n * H + h) * DK + lt) * DV + hh * SC : nullptr;
-#pragma unroll
-            for (int j = 0; j < SC; j += 4) {
-                const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-                S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
-            }
-        }
-        // M' = -D_M to packed fp16 in TMEM at t_M + DK / 4.  Warp half hh reads
-        // fp32 columns [hh DK / 2, (hh + 1) DK / 2) and writes its packed columns
-        // inside that range, 16 columns at a time, in an order that only
-        // overwrites columns it has already read (descending for hh = 0,
-        // ascending for hh = 1), so no other warp's reads are in the way.
-        auto convert_m = [&]() {
-            constexpr int NP = DK / 32;   // 16-column pieces per warp
-#pragma unroll
-            for (int i = 0; i < NP; ++i) {
-                const int piece = hh == 0 ? NP - 1 - i : i;
-                const int col = hh * (DK / 2) + 16 * piece;          // fp32 source column
-                float m[16];
-                tmem_ld16(t_M + lane_off + (uint32_t)col, m);
-                tmem_wait_ld();
-                uint32_t pk[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) pk[e] = pack_f16(-m[2 * e], -m[2 * e + 1]);
-                tmem_st8(t_M + lane_off + (uint32_t)(DK / 4 + col / 2), pk);   // K pair (col, col + 1) -> col / 2
-            }
-            tmem_wait_st();
-        };
-        // bar_mconv(c) is raised only after mb_m(c) completed (with or without
-        // the conversion), so it also tells the issuer that B_c is in D_S, and
-        // it cannot run a phase ahead of the issuer
-        float egl_prev = 1.f;
-        if (nchunks > 0) {
-            if (!wt(mb_m, 0)) goto finish;
-            tc_fence_after();
-            if (!no_erase) convert_m();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_mconv);
-        }
-        for (int c = 0; c < nchunks; ++c) {
-            unsigned char* slot = slot_of(c);
-            KDA_PHASE(0);
-            if (!wt(bar_v16 + (c & 1), c >> 1)) goto finish;   // record c is in its slot
-            if (c > 0) {
-                if (!wt(mb_chain, c - 1)) goto finish;
-                tc_fence_after();
-            }
-            {
-                unsigned char* Sop = sop_of(c);
-#pragma unroll
-                for (int u = 0; u < SC / 16; ++u) {   // 16 columns at a time: update, then the fp16 operand
-                    if (c > 0) {
-                        float d[16];
-                        tmem_ld16(tmem + 128 * ((c - 1) & 1) + lane_off + (uint32_t)(hh * SC + 16 * u), d);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) S[16 * u + j] = fmaf(egl_prev, S[16 * u + j], d[j]);
-                    }
-                    if (lt < DK) st_row_h16n<16>(Sop, lt, hh * SC + 16 * u, DK, S + 16 * u);
-                }
-            }
-            egl_prev = lt < DK ? reinterpret_cast<const float*>(slot + R::EGL)[lt] : 1.f;
-            fence_proxy_async();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_sop);
-            KDA_PHASE(1);
-            if (c + 1 < nchunks) {   // M' of chunk c + 1
-                if (!wt(mb_m, c + 1)) goto finish;
-                tc_fence_after();
-                if (!no_erase) convert_m();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_mconv);
-            }
-            KDA_PHASE(2);
-        }
-        if (nchunks > 0) {   // state after the last chunk
-            if (!wt(mb_chain, nchunks - 1)) goto finish;
+        if (lt < DK) st_row_h16(Sop, lt, 16 * wg, DK, S);
+        fence_proxy_async();
+        tc_fence_before();
+        KDA_WAIT_OR_EXIT(mb_a + b, 1u << b, (apar >> b) & 1u);
+        KDA_PHASE(1);
+
+        if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int u = 0; u < SC / 16; ++u) {
-                float d[16];
-                tmem_ld16(tmem + 128 * ((nchunks - 1) & 1) + lane_off + (uint32_t)(hh * SC + 16 * u), d);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; ++j) S[16 * u + j] = fmaf(egl_prev, S[16 * u + j], d[j]);
-            }
+            for (int kk = 0; kk < DK / 16; ++kk)    // [O ; X] = [Qh ; Kh] S
+                umma_f16(t_XO, kdesc(slot + R::QK, kk, 128 * 128), mn_desc(Sop, kk, DK), kI, kk > 0);
+            umma_commit(mb_x);
         }
-        if (p.s_out && lt < DK) {
-            float* dst = p.s_out + (((size_t)n * H + h) * DK + lt) * DV + hh * SC;
-#pragma unroll
-            for (int j = 0; j < SC; j += 4)
-                *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-        }
-    } else {
-        // ------------------------------------------------------------ output
-        for (int c = 0; c < nchunks; ++c) {
-            unsigned char* slot = slot_of(c);
-            const int L = min(C, len - c * C);
-            if (quad >= 2) {   // Y = beta (V - X), rows s = lane - 64 of D_O
-                if (!wt(bar_v16 + (c & 1), c >> 1)) goto finish;   // V tile in fp16, beta in the slot
-                if (!wt(mb_xo, c)) goto finish;
-                tc_fence_after();
-                const int s = lt - C;
-                const float bs = reinterpret_cast<const float*>(slot + R::BETA)[s];
-#pragma unroll
-                for (int u = 0; u < DV / 16; ++u) {
-                    float x[16];
-                    tmem_ld16(t_O + lane_off + (uint32_t)(16 * u), x);
-                    tmem_wait_ld();
-                    float y[16];
-#pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        const uint4 vr = *reinterpret_cast<const uint4*>(slot + PL::VOFF + swh_off(s, 16 * u + 8 * g, C));
-                        const __half2* v2 = reinterpret_cast<const __half2*>(&vr);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f2 = __half22float2(v2[e]);
-                            const int jj = 8 * g + 2 * e;
-                            y[jj] = bs * (f2.x - (no_erase ? 0.f : x[jj]));
-                            y[jj + 1] = bs * (f2.y - (no_erase ? 0.f : x[jj + 1]));
-                        }
-                    }
-                    st_row_h16n<16>(Yb, s, 16 * u, C, y);
-                }
+        ++xph;
+        pend |= 16u;
+        KDA_WAIT_OR_EXIT(mb_x, 16u, c & 1);
+        tc_fence_after();
+        // chunk c - 1's PT Y has completed as well: refill the other slot's
+        // second part with chunk c + 1
+        if (c >= 1 && c + 1 < nchunks) {
+            if (issuer) {
                 fence_proxy_async();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_y);
-            } else {           // o rows s = lane of D_O
-                if (!wt(mb_o, c)) goto finish;
-                tc_fence_after();
-                if (tid == kCopy && c + 2 < nchunks) {   // PT Y of chunk c has completed: its slot is free
-                    fence_proxy_async();
-                    if (!issue_rec(c + 2)) goto finish;
-                }
-                const int s = lt;
-                TO* dst = static_cast<TO*>(p.o) + ((size_t)(tok0 + c * C + s) * H + h) * DV;
+                issue_b(c + 1);
+            }
+            pend |= 4u << (b ^ 1);
+            bpar = (bpar & ~(1u << (b ^ 1))) | ((uint32_t)(((c + 1) >> 1) & 1) << (b ^ 1));
+        }
+        KDA_WAIT_OR_EXIT(mb_b + b, 4u << b, (bpar >> b) & 1u);
+        KDA_PHASE(2);
+
+        // ---- Y = beta (V - X) (lanes 64..127) | o rows of chunk c - 1 (lanes 0..63)
+        {
+            const float* egl = reinterpret_cast<const float*>(slot + R::EGL);
+            const float* beta = reinterpret_cast<const float*>(slot + R::BETA);
+            eglp = lt < DK ? egl[lt] : 1.f;
+            if (lt >= C) {
+                const int s = lt - C;
+                float x16[16];
+                tmem_ld16(t_XO + lane_off + q_off, x16);
+                tmem_wait_ld();
+                const float bs = beta[s];
+                const unsigned char* vt = slot + PL::VOFF;
+                uint4 vr[2];
+                vr[0] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg, C));
+                vr[1] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg + 8, C));
+                float y[16];
 #pragma unroll
-                for (int u = 0; u < DV / 16; ++u) {
-                    float acc[16];
-                    tmem_ld16(t_O + lane_off + (uint32_t)(16 * u), acc);
-                    tmem_wait_ld();
-                    if (s < L) {
-                        if constexpr (sizeof(TO) == 4) {
+                for (int u = 0; u < 2; ++u) {
+                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
 #pragma unroll
-                            for (int j = 0; j < 16; j += 4)
-                                *reinterpret_cast<float4*>(dst + 16 * u + j) =
-                                    make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 16; j += 8)
-                                *reinterpret_cast<uint4*>(dst + 16 * u + j) =
-                                    make_uint4(pack_bf16(acc[j], acc[j + 1]), pack_bf16(acc[j + 2], acc[j + 3]),
-                                               pack_bf16(acc[j + 4], acc[j + 5]), pack_bf16(acc[j + 6], acc[j + 7]));
-                        }
+                    for (int w = 0; w < 4; ++w) {
+                        const float2 f2 = __bfloat1622float2(v2[w]);
+                        const int jj = 8 * u + 2 * w;
+                        y[jj] = bs * (f2.x - (no_erase ? 0.f : x16[jj]));
+                        y[jj + 1] = bs * (f2.y - (no_erase ? 0.f : x16[jj + 1]));
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_ofree);
+                st_row_h16(Yb, s, 16 * wg, C, y);
+            } else if (c > 0) {
+                const int tk = tok0 + (c - 1) * C;
+                store_o_tile<TO>(tmem + 64 * (b ^ 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
+                                 ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
             }
         }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        KDA_PHASE(3);
+        if (issuer && c + 2 < nchunks) {            // X MMA done, V consumed: refill part one
+            fence_proxy_async();
+            issue_a(c + 2);
+        }
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)     // W = Z Y
+                umma_f16(t_W, kdesc(slot + R::Z, kk, DK * 128), mn_desc(Yb, kk, C), kI, kk > 0);
+            umma_commit(mb_w);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)     // O += PT Y  (rows 64..127: discarded)
+                umma_f16(t_XO, kdesc(slot + R::PT, kk, C * 128), mn_desc(Yb, kk, C), kI, 1);
+        }
+        ++wph;
+        pend |= 32u;
+        if (c + 2 < nchunks) {
+            pend |= 1u << b;
+            apar = (apar & ~(1u << b)) | ((uint32_t)(((c + 2) >> 1) & 1) << b);
+        }
+        Lprev = L;
+        KDA_PHASE(4);
+    }
+
+    if (nchunks > 0) {
+        // W and O of the last chunk: one more commit covers every MMA issued
+        if (tid == 0) umma_commit(mb_x);
+        ++xph;
+        pend |= 16u;
+        KDA_WAIT_OR_EXIT(mb_x, 16u, nchunks & 1);
+        pend &= ~32u;
+        tc_fence_after();
+        float w[16];
+        tmem_ld16(t_W + lane_off + q_off, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
+        if (lt < C) {
+            const int tk = tok0 + (nchunks - 1) * C;
+            store_o_tile<TO>(tmem + 64 * ((nchunks - 1) & 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
+                             ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
+        }
+    }
+    if (p.s_out && lt < DK) {
+        float* dst = p.s_out + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
 
 finish:
     KDA_PHASE_FLUSH
-    __syncthreads();
     if (*abort_flag) {
         // let every copy and MMA in flight land before the TMEM is released
         volatile int never = 0;
-        if (tid == 0 && mma_issued) {
-            umma_commit(mb_fin);
-            (void)mbar_wait(mb_fin, 0u, &never, tmo);
+        for (int i = 0; i < 2; ++i) {
+            if (pend & (1u << i)) (void)mbar_wait(mb_a + i, (apar >> i) & 1u, &never, p.timeout_cycles);
+            if (pend & (4u << i)) (void)mbar_wait(mb_b + i, (bpar >> i) & 1u, &never, p.timeout_cycles);
         }
-        if (tid == kCopy)
-            for (int i = max(0, rec_issued - 2); i < rec_issued; ++i)
-                (void)mbar_wait(mb_rec + (i & 1), (uint32_t)((i >> 1) & 1), &never, tmo);
+        if (pend & 16u) (void)mbar_wait(mb_x, (uint32_t)((xph - 1) & 1), &never, p.timeout_cycles);
+        if (pend & 32u) (void)mbar_wait(mb_w, (uint32_t)((wph - 1) & 1), &never, p.timeout_cycles);
+        __syncthreads();
+        if (tid == 0) umma_commit(mb_x);
+        (void)mbar_wait(mb_x, (uint32_t)(xph & 1), &never, p.timeout_cycles);
     }
+    if (issuer) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, 256);
     }
 }
 #undef KDA_WAIT_OR_EXIT
@@ -1297,23 +1158,24 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     prep_body<DK, VAR>(tmq, tmk, tmg, p, blockIdx.x, gridDim.x);
 }
 
-template <typename TO, int DK, int DV, bool VAR>
+template <typename TO, int DK, bool VAR>
 __global__ void __launch_bounds__(NT, 1)
-chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const ScanParams p)
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                  const ScanParams p)
 {
-    scan_body<TO, DK, DV, VAR>(tmv, p, blockIdx.x);
+    scan_body<TO, DK, VAR>(tmv, tmo, p, blockIdx.x);
 }
 
 // Cooperative schedule: CTAs [0, n_scan) scan, the others prep; the scan
 // waits on the records' ready flags, the prep never waits on the scan, and a
 // cooperative launch keeps every CTA resident, so the hand-off cannot stall.
-template <typename TO, int DK, int DV, bool VAR>
+template <typename TO, int DK, bool VAR>
 __global__ void __launch_bounds__(NT, 1)
 chunk_coop_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmg, const __grid_constant__ CUtensorMap tmv,
-                  const PrepParams pp, const ScanParams sp, int n_scan)
+                  const __grid_constant__ CUtensorMap tmo, const PrepParams pp, const ScanParams sp, int n_scan)
 {
-    if ((int)blockIdx.x < n_scan) scan_body<TO, DK, DV, VAR>(tmv, sp, blockIdx.x);
+    if ((int)blockIdx.x < n_scan) scan_body<TO, DK, VAR>(tmv, tmo, sp, blockIdx.x);
     else prep_body<DK, VAR>(tmq, tmk, tmg, pp, blockIdx.x - n_scan, gridDim.x - n_scan);
 }
 
@@ -1478,13 +1340,12 @@ static WsLayout ws_layout(int nseq, int T, long long tokens, int H, int dv, bool
     return w;
 }
 
-template <typename TO, int DK, int DV>
+template <typename TO, int DK>
 static cudaError_t run(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
                        const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens,
-                       int H, long long timeout_cycles, int mode, unsigned char* ws, size_t ws_bytes,
+                       int H, int dv, long long timeout_cycles, int mode, unsigned char* ws, size_t ws_bytes,
                        cudaStream_t stream)
 {
-    constexpr int dv = DV;
     const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;
     const bool variant = (mode & (KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE | KDA_MODE_NORM_QK | KDA_MODE_GATE_LOGITS)) != 0;
     const int req_blocks = (mode >> 8) & 0xff;     // KDA_MODE_BLOCKS(n), 0 = automatic
@@ -1493,7 +1354,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     const WsLayout L = ws_layout<DK>(nseq, T, tokens, H, dv, cu != nullptr);
     if (!ws || ws_bytes < L.bytes) return cudaErrorInvalidValue;
     const long long max_chunks = L.max_chunks;
-    const long long scan_ctas = (long long)nseq * H;   // one scan CTA per (sequence, head)
+    const long long scan_ctas = (long long)nseq * H * (dv / NV);
     if (scan_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     // schedule: one cooperative launch (prep CTAs publish records, scan CTAs
     // consume them) when the scan grid leaves at least 32 SMs; otherwise prep
@@ -1508,13 +1369,15 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
         (!head_gate && !make_tmap(&tg, log_alpha, tokens, H, DK, true)))
         return cudaErrorInvalidValue;
-    CUtensorMap tv;
-    if (!make_tmap(&tv, v, tokens, H, dv, false, 64, true)) return cudaErrorInvalidValue;
+    CUtensorMap tv, to;
+    if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
+        !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
+        return cudaErrorInvalidValue;
     auto pk = variant ? chunk_prep_kernel<DK, true> : chunk_prep_kernel<DK, false>;
-    auto sk = variant ? chunk_scan_kernel<TO, DK, DV, true> : chunk_scan_kernel<TO, DK, DV, false>;
+    auto sk = variant ? chunk_scan_kernel<TO, DK, true> : chunk_scan_kernel<TO, DK, false>;
     cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
     if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK, DV>::BYTES);
+        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
     if (err != cudaSuccess) return err;
 
     // events of the two-stream schedule (created last: no early return leaks them)
@@ -1610,7 +1473,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         sp.s_in = b == 0 ? s0 : carry;
         sp.s_out = (b == nblocks - 1) ? sT : carry;
         if (scan_ctas <= 0) return cudaSuccess;
-        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK, DV>::BYTES, stream>>>(tv, sp);
+        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
         return cudaGetLastError();
     };
 
@@ -1618,8 +1481,8 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (coop) {
         unsigned* flags = reinterpret_cast<unsigned*>(ws + L.flags);
         err = cudaMemsetAsync(flags, 0, (size_t)max_chunks * H * 4, stream);
-        auto ck = variant ? chunk_coop_kernel<TO, DK, DV, true> : chunk_coop_kernel<TO, DK, DV, false>;
-        const int smem = std::max(PrepPlan::BYTES, ScanPlan<DK, DV>::BYTES);
+        auto ck = variant ? chunk_coop_kernel<TO, DK, true> : chunk_coop_kernel<TO, DK, false>;
+        const int smem = std::max(PrepPlan::BYTES, ScanPlan<DK>::BYTES);
         if (err == cudaSuccess) err = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err == cudaSuccess) {
             pp.ready = flags;
@@ -1642,7 +1505,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             const int n_scan = (int)scan_ctas;
-            if (cudaLaunchKernelEx(&cfg, ck, tq, tk, tg, tv, pp, sp, n_scan) == cudaSuccess) done = true;
+            if (cudaLaunchKernelEx(&cfg, ck, tq, tk, tg, tv, to, pp, sp, n_scan) == cudaSuccess) done = true;
             else (void)cudaGetLastError();   // not co-residable here: fall back to prep then scan
             pp.ready = nullptr;
             sp.ready = nullptr;
@@ -1716,19 +1579,18 @@ static long long noalloc_block(int nseq, int H, int dv, bool has_final, int nch)
     return std::min<long long>(nch, (long long)((kScratchBytes - carry) / (2 * per_chunk)));
 }
 
-template <typename TO, int DK, int DV>
+template <typename TO, int DK>
 static cudaError_t run_noalloc(const void* q, const void* k, const void* v, const float* beta,
                                const float* log_alpha, const float* s0, void* o, float* sT, int nseq, int T,
-                               long long tokens, int H, long long timeout_cycles, cudaStream_t stream)
+                               long long tokens, int H, int dv, long long timeout_cycles, cudaStream_t stream)
 {
-    constexpr int dv = DV;
     using R = Rec<DK>;
     const int nsm = sm_count();
     const int nch = (T + C - 1) / C;
     const long long cb = noalloc_block<DK>(nseq, H, dv, sT != nullptr, nch);
     if (cb <= 0) return cudaErrorInvalidValue;
     const int nblocks = (int)((nch + cb - 1) / cb);
-    const long long scan_ctas = (long long)nseq * H;   // one scan CTA per (sequence, head)
+    const long long scan_ctas = (long long)nseq * H * (dv / NV);
     if (scan_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     unsigned char* area = scratch_area();
     if (!area) return cudaErrorInvalidSymbol;
@@ -1737,15 +1599,16 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
     unsigned char* ring[2] = {area + carry_sz, nullptr};
     if (nblocks > 1) ring[1] = area + carry_sz + (size_t)cb * nseq * H * R::BYTES;
 
-    CUtensorMap tq, tk, tg, tv;
+    CUtensorMap tq, tk, tg, tv, to;
     if (!make_tmap(&tq, q, tokens, H, DK, false) || !make_tmap(&tk, k, tokens, H, DK, false) ||
-        !make_tmap(&tg, log_alpha, tokens, H, DK, true) || !make_tmap(&tv, v, tokens, H, dv, false, 64, true))
+        !make_tmap(&tg, log_alpha, tokens, H, DK, true) || !make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
+        !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
         return cudaErrorInvalidValue;
     auto pk = chunk_prep_kernel<DK, false>;
-    auto sk = chunk_scan_kernel<TO, DK, DV, false>;
+    auto sk = chunk_scan_kernel<TO, DK, false>;
     cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
     if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK, DV>::BYTES);
+        err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
     if (err != cudaSuccess) return err;
 
     PrepParams pp{};
@@ -1790,7 +1653,7 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
         sp.s_in = b == 0 ? s0 : carry;
         sp.s_out = b == nblocks - 1 ? sT : carry;
         if (scan_ctas <= 0) return cudaSuccess;
-        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK, DV>::BYTES, stream>>>(tv, sp);
+        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
         return cudaGetLastError();
     };
 
@@ -1852,21 +1715,6 @@ size_t chunk_fwd_split_workspace(int nseq, int T, long long tokens, int H, int d
                      : split::ws_layout<64>(nseq, T, tokens, H, dv, varlen).bytes;
 }
 
-template <typename TO, int DK>
-static cudaError_t run_dv(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
-                          const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens,
-                          int H, int dv, long long timeout_cycles, int mode, unsigned char* ws, size_t ws_bytes,
-                          cudaStream_t stream)
-{
-    if (dv == 128)
-        return split::run<TO, DK, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, timeout_cycles,
-                                       mode, ws, ws_bytes, stream);
-    if (dv == 64)
-        return split::run<TO, DK, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, timeout_cycles,
-                                      mode, ws, ws_bytes, stream);
-    return cudaErrorInvalidValue;
-}
-
 cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const float* beta,
                             const float* log_alpha, const float* s0, void* o, float* sT, const int32_t* cu,
                             int nseq, int T, long long tokens, int H, int dk, int dv, kda_dtype o_dtype,
@@ -1874,11 +1722,11 @@ cudaError_t chunk_fwd_split(const void* q, const void* k, const void* v, const f
 {
     unsigned char* w = static_cast<unsigned char*>(ws);
     if (o_dtype == KDA_F32) {
-        if (dk == 128) return run_dv<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
-        if (dk == 64) return run_dv<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 128) return split::run<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 64) return split::run<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
     } else {
-        if (dk == 128) return run_dv<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
-        if (dk == 64) return run_dv<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 128) return split::run<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
+        if (dk == 64) return split::run<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dv, timeout_cycles, mode, w, ws_bytes, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -1890,31 +1738,17 @@ bool chunk_fwd_noalloc_fits(int nseq, int T, int H, int dk, int dv, bool has_fin
                      : split::noalloc_block<64>(nseq, H, dv, has_final, nch) > 0;
 }
 
-template <typename TO, int DK>
-static cudaError_t noalloc_dv(const void* q, const void* k, const void* v, const float* beta, const float* log_alpha,
-                              const float* s0, void* o, float* sT, int nseq, int T, long long tokens, int H, int dv,
-                              long long timeout_cycles, cudaStream_t stream)
-{
-    if (dv == 128)
-        return split::run_noalloc<TO, DK, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H,
-                                               timeout_cycles, stream);
-    if (dv == 64)
-        return split::run_noalloc<TO, DK, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H,
-                                              timeout_cycles, stream);
-    return cudaErrorInvalidValue;
-}
-
 cudaError_t chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* beta,
                               const float* log_alpha, const float* s0, void* o, float* sT, int nseq, int T,
                               long long tokens, int H, int dk, int dv, kda_dtype o_dtype, long long timeout_cycles,
                               cudaStream_t stream)
 {
     if (o_dtype == KDA_F32) {
-        if (dk == 128) return noalloc_dv<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
-        if (dk == 64) return noalloc_dv<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 128) return split::run_noalloc<float, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 64) return split::run_noalloc<float, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
     } else {
-        if (dk == 128) return noalloc_dv<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
-        if (dk == 64) return noalloc_dv<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 128) return split::run_noalloc<__nv_bfloat16, 128>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
+        if (dk == 64) return split::run_noalloc<__nv_bfloat16, 64>(q, k, v, beta, log_alpha, s0, o, sT, nseq, T, tokens, H, dv, timeout_cycles, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -6,3 +6,4 @@
 #include "kda_chunk_simt.cu"
 #include "kda_chunk_split.cu"
 #include "kda_chunk_bwd.cu"
+#include "kda_dplr.cu"

@@ -299,6 +299,39 @@ kda_status kda_varlen_bwd_workspace_size(int N, int T, int H, int dk, int dv, in
                                          kda_dtype dtype, size_t* bytes);
 
 /*
+ * Chunkwise forward of the diagonal-plus-low-rank transition, the "finer
+ * granularity" gate of "Hybrid Linear Attention Architecture: Making LLM
+ * Training and Inference More Efficient", section 3.3 (a low-rank correction
+ * on top of the element-wise decay; also the RWKV-7 line of "... Technical Deep
+ * Dive ...", section 3), in this library's d_k x d_v orientation:
+ *
+ *     S_t = (Diag(alpha_t) + b_t a_t^T) S_{t-1} + k_t v_t^T,     o_t = S_t^T q_t
+ *
+ * (the pages write S_{t-1} (Diag(alpha_t) + a_t b_t^T) + v_t k_t^T for the
+ * transposed d_v x d_k state).  With a_t = alpha_t * k_t, b_t = -beta_t k_t and
+ * the key beta_t k_t it is the KDA layer.  fp32 arithmetic on CUDA cores; no
+ * workspace.
+ *
+ *   q, k, a, b  [B, T, H, dk]  dtype;   v [B, T, H, dv]  dtype
+ *   log_alpha   [B, T, H, dk]  fp32 (<= 0)
+ *   initial_state / final_state [B, H, dk, dv] fp32 or NULL (final may alias initial)
+ *   o           [B, T, H, dv]  o_dtype
+ * d_k, d_v in {64, 128}, chunk 64; pointers 16-byte aligned.
+ */
+kda_status kda_dplr_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
+                        const float* log_alpha, const float* initial_state, void* o, float* final_state,
+                        int B, int T, int H, int dk, int dv, int chunk,
+                        kda_dtype dtype, kda_dtype o_dtype, void* stream);
+
+/* The same over N packed variable-length sequences (layouts and boundary
+ * rules of kda_varlen_fwd). */
+kda_status kda_dplr_varlen_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
+                               const float* log_alpha, const int32_t* cu_seqlens, int N,
+                               const float* initial_state, void* o, float* final_state,
+                               int T, int H, int dk, int dv, int chunk,
+                               kda_dtype dtype, kda_dtype o_dtype, void* stream);
+
+/*
  * Synchronises `stream` and reports (then clears) the current device's
  * status word: KDA_ERR_TIMEOUT if a device-side bounded wait ran out since the
  * last check, KDA_ERR_INVALID_ARG if a kernel found device-resident sequence
