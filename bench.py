@@ -384,15 +384,20 @@ def run_decode(kda, device, stream, world, rank, warmup):
 
 def run_other_workloads(kda, device, stream, world, rank, reps=20):
     """The prefill (B2 H16 T4096) and varlen (8 packed sequences, 65536 tokens,
-    H32) chunk forwards, and the prefill shape with the two layer variants (one
+    H32) chunk forwards, the same 65536 tokens packed as 1024 short sequences
+    (lengths 16..112), and the prefill shape with the two layer variants (one
     gate per head; no erase term): one warm-up launch, `reps` timed launches
     each, inputs resident in HBM."""
     from gated_delta_rule_133_b200.inputs import WORKLOADS, make_inputs
     out = {}
-    for name in ("prefill", "varlen", "prefill_head_gate", "prefill_no_erase"):
+    for name in ("prefill", "varlen", "varlen_1024", "prefill_head_gate", "prefill_no_erase"):
         w = WORKLOADS[name.split("_")[0]]
+        if name == "varlen_1024":
+            w = type(w)(**{**w.__dict__, "B": 1024, "extra": {"min_len": 16, "max_len": 112}})
         d = make_inputs(w, device, seed=w.seed + 1000 * rank)
         desc = f"{name}: {w.B * w.T if w.kind != 'varlen' else w.T} tokens, H={w.H}, d_k=d_v={w.dk}, bf16 q/k/v, fp32 o and state"
+        if w.kind == "varlen":
+            desc += f", {w.B} sequences of {w.extra['min_len']}..{w.extra['max_len']} tokens"
         kw = {}
         gate_bytes = 4 * w.dk
         if name.startswith("prefill"):

@@ -116,6 +116,12 @@ __device__ __forceinline__ bool wait_ready(const unsigned* flag, volatile int* a
 
 // ============================================================== pass 1: prep
 
+// Layer-variant instantiations of the kernels: the plain layer, the two gate
+// tiers alone (each with the work it no longer needs removed), and one
+// instantiation for every other combination of KDA_MODE_* flags (runtime
+// branches).
+constexpr int kVarPlain = 0, kVarHeadGate = 1, kVarNoErase = 2, kVarAny = 3;
+
 struct PrepParams {
     const float* beta;
     const int32_t* cu;       // varlen boundaries, or nullptr (dense)
@@ -241,17 +247,17 @@ __device__ __forceinline__ Vec vec_at(unsigned char* base, int buf)
 // Gate cumsum of the staged chunk in place, by 384 threads (t = 0..383:
 // key channel t % 128, rows [21 p, 21 p + 21) of part p = t / 128, the last
 // part 22 rows), and the item's channel vectors.  Named barrier 2.
+//
+// gate_v is the gate of row t (t < 64) when gates are per (token, head), read
+// by the caller ahead of the wait for the tile.
 template <int DK>
 __device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t, float beta_v,
-                                          const float* gh, long long gbase, int H, bool logits)
+                                          bool gh, float gate_v, bool logits)
 {
     const int ch = t & 127, part = t >> 7;
     const int r0 = 21 * part, nr = part == 2 ? 22 : 21;
     if (gh) {   // one gate per (token, head): column 0 of the staging holds the chunk's 64 gates
-        if (t < C) {
-            const float z = t < L ? gh[gbase + (long long)t * H] : 0.f;
-            gs[t * DK] = (logits && t < L) ? neg_softplus(z) : z;
-        }
+        if (t < C) gs[t * DK] = (logits && t < L) ? neg_softplus(gate_v) : gate_v;
         bar_sync(2, 384);
     }
     float G[22];
@@ -286,10 +292,56 @@ __device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t,
     bar_sync(2, 384);
 }
 
+// Gate cumsum of one gate per (token, head), by 384 threads (named barrier 2):
+// column 0 of the staging receives G and every key channel gets the same
+// channel vectors.  Three lanes run the three row parts of cumsum384 for one
+// channel, additions in the same order, so the result is bit-identical to the
+// per-channel path fed the same gate on every channel.
+template <int DK>
+__device__ __forceinline__ void cumsum_head384(float* gs, const Vec& v, int L, int t, float beta_v, float gate_v)
+{
+    if (t < C) {
+        gs[t * DK] = t < L ? gate_v : 0.f;
+        v.beta[t] = beta_v;
+    }
+    bar_sync(2, 384);
+    float G[22];
+    const int r0 = 21 * t, nr = t == 2 ? 22 : 21;
+    if (t < 3) {
+#pragma unroll
+        for (int rr = 0; rr < 22; ++rr) G[rr] = rr < nr ? gs[(r0 + rr) * DK] : 0.f;
+#pragma unroll
+        for (int rr = 1; rr < 22; ++rr) G[rr] += G[rr - 1];
+        v.qtot[t * 128] = G[nr - 1];
+    }
+    bar_sync(2, 384);
+    if (t < 3) {
+        float off = 0.f;
+        for (int q = 0; q < t; ++q) off += v.qtot[q * 128];
+#pragma unroll
+        for (int rr = 0; rr < 22; ++rr)
+            if (rr < nr) gs[(r0 + rr) * DK] = G[rr] + off;
+        if (t == 1) v.qtot[1] = off + G[31 - 21];   // G_m (slot 1 of part 0 is free)
+    }
+    bar_sync(2, 384);
+    if (t < DK) {
+        const float Gm = v.qtot[1];
+        const float Gl = v.qtot[0] + v.qtot[128] + v.qtot[256];
+        v.gml[t] = Gm;
+        v.gm[t] = expf(Gm);
+        v.glm[t] = expf(Gl - Gm);
+        v.egl[t] = expf(Gl);
+    }
+    bar_sync(2, 384);
+}
+
 // Operands of rows [row_lo, row_hi) of one item, by `nthr` threads (t = 0..nthr-1): A1 = [q E; k E]
 // and B1 = k / E (tf32, smem) for the intra-chunk products; Qh = q e^G and
 // Kh = k e^G (fp16) straight into the record.
-template <int DK>
+//
+// HG: one gate per (token, head): G is read from column 0 and every channel of
+// a row shares one exponential and one reciprocal.
+template <int DK, bool HG = false>
 __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& v, unsigned char* rec, int L, int t,
                                                int nthr, int row_lo, int row_hi, bool norm_qk = false)
 {
@@ -301,7 +353,8 @@ __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& 
     const float4 gm4 = *reinterpret_cast<const float4*>(v.gm + c0);
 #pragma unroll 2
     for (int r = row_lo + r0; r < row_hi; r += rpp) {
-        const float4 g4 = *reinterpret_cast<const float4*>(x.gs + r * DK + c0);
+        const float4 g4 = HG ? make_float4(x.gs[r * DK], 0.f, 0.f, 0.f)
+                             : *reinterpret_cast<const float4*>(x.gs + r * DK + c0);
         float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = q4;
         if (r < L) {
             q4 = bf16x4(x.qs + r * DK + c0);
@@ -319,14 +372,24 @@ __device__ __forceinline__ void build_operands(const PrepCtx<DK>& x, const Vec& 
             q4 = make_float4(q4.x * iq, q4.y * iq, q4.z * iq, q4.w * iq);
             k4 = make_float4(k4.x * ik, k4.y * ik, k4.z * ik, k4.w * ik);
         }
-        const float e0 = __expf(fminf(fmaxf(g4.x - m4.x, -80.f), 80.f));
-        const float e1 = __expf(fminf(fmaxf(g4.y - m4.y, -80.f), 80.f));
-        const float e2 = __expf(fminf(fmaxf(g4.z - m4.z, -80.f), 80.f));
-        const float e3 = __expf(fminf(fmaxf(g4.w - m4.w, -80.f), 80.f));
+        float e0, e1, e2, e3, i0, i1, i2, i3;
+        if (HG) {
+            e0 = e1 = e2 = e3 = __expf(fminf(fmaxf(g4.x - m4.x, -80.f), 80.f));
+            i0 = i1 = i2 = i3 = rcp_approx(e0);
+        } else {
+            e0 = __expf(fminf(fmaxf(g4.x - m4.x, -80.f), 80.f));
+            e1 = __expf(fminf(fmaxf(g4.y - m4.y, -80.f), 80.f));
+            e2 = __expf(fminf(fmaxf(g4.z - m4.z, -80.f), 80.f));
+            e3 = __expf(fminf(fmaxf(g4.w - m4.w, -80.f), 80.f));
+            i0 = rcp_approx(e0);
+            i1 = rcp_approx(e1);
+            i2 = rcp_approx(e2);
+            i3 = rcp_approx(e3);
+        }
         *reinterpret_cast<float4*>(x.A1 + swf_off(r, c0, 128)) = tf32r4(q4.x * e0, q4.y * e1, q4.z * e2, q4.w * e3);
         *reinterpret_cast<float4*>(x.A1 + swf_off(C + r, c0, 128)) = tf32r4(k4.x * e0, k4.y * e1, k4.z * e2, k4.w * e3);
         *reinterpret_cast<float4*>(x.B1 + swf_off(r, c0, 64)) =
-            tf32r4(k4.x * rcp_approx(e0), k4.y * rcp_approx(e1), k4.z * rcp_approx(e2), k4.w * rcp_approx(e3));
+            tf32r4(k4.x * i0, k4.y * i1, k4.z * i2, k4.w * i3);
         const float f0 = e0 * gm4.x, f1 = e1 * gm4.y, f2 = e2 * gm4.z, f3 = e3 * gm4.w;
         *reinterpret_cast<uint2*>(rec + R::QK + swh_off(r, c0, 128)) =
             make_uint2(pack_f16(q4.x * f0, q4.y * f1), pack_f16(q4.z * f2, q4.w * f3));
@@ -469,18 +532,24 @@ __device__ __forceinline__ void ut_rows(float* As, float* X, unsigned char* Top)
 //             MMA Z(k), PT(k) (kind::f16), PA(k + 1) (kind::tf32)
 //             record tail of item k (staged in TST, one bulk store); P/A split of k + 1
 //
+// Without the erase term A = 0 and T = I: the T^T tile is the identity from
+// the start, no UT transform runs, and warpgroup 0 joins the build.
+//
 // TMEM: [P ; A~] double-buffered (0, 64); the fp16 A operands of Z and PT,
 // k e^(G_last - G) transposed (128) and masked P (160), two per 32-bit column;
 // Z 192, PT 256.
-template <int DK, bool VAR>
+template <int DK, int VK>
 __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmg,
                                           const PrepParams& p, int bid, int nblk)
 {
-    // layer variants (VAR instantiations only; the plain layer compiles without them)
-    const float* const gh = VAR ? p.gh : nullptr;
-    const bool no_erase = VAR && p.no_erase;
-    const bool norm_qk = VAR && p.norm_qk;
-    const bool logits = VAR && p.logits;
+    // layer variants: kVarHeadGate and kVarNoErase fix one flag at compile
+    // time; kVarAny reads every flag at run time
+    constexpr bool kHG = VK == kVarHeadGate;   // per-head gates only
+    constexpr bool kNE = VK == kVarNoErase;    // no erase term only
+    const float* const gh = (kHG || VK == kVarAny) ? p.gh : nullptr;
+    const bool no_erase = kNE || (VK == kVarAny && p.no_erase);
+    const bool norm_qk = VK == kVarAny && p.norm_qk;
+    const bool logits = VK == kVarAny && p.logits;
     using PL = PrepPlan;
     using R = Rec<DK>;
     extern __shared__ unsigned char smem_raw[];
@@ -550,6 +619,13 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
     auto beta_of = [&](const Item& it, int t) {
         return (it.ok && t < C && t < it.L) ? p.beta[(size_t)(it.tok0 + t) * H + it.h] : 0.f;
     };
+    auto gate_of = [&](const Item& it, int t) {   // per-head gate of row t (0 past the chunk)
+        return (gh && it.ok && t < C && t < it.L) ? gh[(size_t)(it.tok0 + t) * H + it.h] : 0.f;
+    };
+    auto cumsum = [&](const Vec& v, const Item& it, int t, float beta_v, float gate_v) {
+        if (kHG) cumsum_head384<DK>(x.gs, v, it.L, t, beta_v, gate_v);
+        else cumsum384<DK>(x.gs, v, it.L, t, beta_v, gh != nullptr, gate_v, logits);
+    };
     // P masked (lanes 0..63, lower incl.) into the fp16 operand of PT; A = beta
     // A~ (lanes 64..127, strictly lower) to the UT scratch; (k / E)^T
     // e^(G_last - G_m) = (k e^(G_last - G))^T into the fp16 operand of Z
@@ -563,7 +639,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
             for (int s2 = 0; s2 < 8; ++s2)
                 p16[s2] = pack_f16((16 * wg + 2 * s2 <= lt) ? pa[2 * s2] : 0.f, (16 * wg + 2 * s2 + 1 <= lt) ? pa[2 * s2 + 1] : 0.f);
             tmem_st8(t_P16 + lane_off + wg * 8, p16);
-        } else {
+        } else if (!kNE) {
             const int r = lt - C;
             const float b = v.beta[r];
             float a[16];
@@ -591,17 +667,21 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
 
     // ---- prologue: item 0 by all threads
     for (int i = tid; i < C * C * 2 / 16; i += NT) reinterpret_cast<uint4*>(Top)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (kNE) {   // T = I for good
+        __syncthreads();
+        if (tid < C) *reinterpret_cast<__half*>(Top + swh_off(tid, tid, C)) = __float2half_rn(1.f);
+    }
     if (tid == 0) load_item(cur);
     ++nload;
     pend |= 1u;
     tpar = 0;
     {
         const float beta_v = tid >= 128 ? beta_of(cur, tid - 128) : 0.f;
+        const float gate_v = tid >= 128 ? gate_of(cur, tid - 128) : 0.f;
         KDA_WAIT_OR_EXIT(mb_tma, 1u, 0);
-        if (tid >= 128)
-            cumsum384<DK>(x.gs, vec_at(vbase, 0), cur.L, tid - 128, beta_v, gh, (long long)cur.tok0 * H + cur.h, H, logits);
+        if (tid >= 128) cumsum(vec_at(vbase, 0), cur, tid - 128, beta_v, gate_v);
         __syncthreads();
-        build_operands<DK>(x, vec_at(vbase, 0), p.rec + (size_t)cur.rec * R::BYTES, cur.L, tid, NT, 0, C, norm_qk);
+        build_operands<DK, kHG>(x, vec_at(vbase, 0), p.rec + (size_t)cur.rec * R::BYTES, cur.L, tid, NT, 0, C, norm_qk);
     }
     fence_proxy_async();
     tc_fence_before();
@@ -636,16 +716,28 @@ __device__ __forceinline__ void prep_body(const CUtensorMap& tmq, const CUtensor
         KDA_PHASE(0);
 
         // ---- UT transform of item k (WG0) | cumsum + operands of item k + 1 (WG1-3)
-        if (wg == 0) {
+        if (kNE) {   // no UT transform: all four warpgroups build
+            if (nxt.ok) {
+                const int t = tid - 128;
+                const float beta_v = wg ? beta_of(nxt, t) : 0.f;
+                const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
+                if (!__syncthreads_or(!ok)) {
+                    if (wg) cumsum(vnxt, nxt, t, beta_v, 0.f);
+                    __syncthreads();
+                    build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, tid, NT, 0, C, false);
+                }
+            }
+        } else if (wg == 0) {
             ut_rows(As, Xs, Top);
         } else {
             if (nxt.ok) {
                 const int t = tid - 128;
                 const float beta_v = beta_of(nxt, t);
+                const float gate_v = gate_of(nxt, t);
                 const bool ok = mbar_wait(mb_tma, (uint32_t)tpar, abort_flag, p.timeout_cycles);
                 if (!bar_or(3, 384, !ok)) {
-                    cumsum384<DK>(x.gs, vnxt, nxt.L, t, beta_v, gh, (long long)nxt.tok0 * H + nxt.h, H, logits);
-                    build_operands<DK>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384, 0, C, norm_qk);
+                    cumsum(vnxt, nxt, t, beta_v, gate_v);
+                    build_operands<DK, kHG>(x, vnxt, p.rec + (size_t)nxt.rec * R::BYTES, nxt.L, t, 384, 0, C, norm_qk);
                 }
             }
         }
@@ -858,11 +950,11 @@ __device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost,
 // completed: the [Qh ; Kh] tile and V after chunk c's X MMA and Y phase, the
 // Z, PT, e^G_last and beta part after chunk c + 1's X MMA (tcgen05 MMAs of
 // one thread complete in issue order).
-template <typename TO, int DK, bool VAR>
+template <typename TO, int DK, int VK>
 __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensorMap& tmo, const ScanParams& p,
                                           int bid)
 {
-    const bool no_erase = VAR && p.no_erase;   // layer variant (VAR instantiations only)
+    const bool no_erase = VK == kVarNoErase || (VK == kVarAny && p.no_erase);   // layer variant
     using PL = ScanPlan<DK>;
     using R = Rec<DK>;
     extern __shared__ unsigned char smem_raw[];
@@ -1150,34 +1242,44 @@ finish:
 }
 #undef KDA_WAIT_OR_EXIT
 
-template <int DK, bool VAR>
+template <int DK, int VK>
 __global__ void __launch_bounds__(NT, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmg, const PrepParams p)
 {
-    prep_body<DK, VAR>(tmq, tmk, tmg, p, blockIdx.x, gridDim.x);
+    prep_body<DK, VK>(tmq, tmk, tmg, p, blockIdx.x, gridDim.x);
 }
 
-template <typename TO, int DK, bool VAR>
+template <typename TO, int DK, int VK>
 __global__ void __launch_bounds__(NT, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
                   const ScanParams p)
 {
-    scan_body<TO, DK, VAR>(tmv, tmo, p, blockIdx.x);
+    scan_body<TO, DK, VK>(tmv, tmo, p, blockIdx.x);
 }
 
 // Cooperative schedule: CTAs [0, n_scan) scan, the others prep; the scan
 // waits on the records' ready flags, the prep never waits on the scan, and a
 // cooperative launch keeps every CTA resident, so the hand-off cannot stall.
-template <typename TO, int DK, bool VAR>
+template <typename TO, int DK, int VK>
 __global__ void __launch_bounds__(NT, 1)
 chunk_coop_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmg, const __grid_constant__ CUtensorMap tmv,
                   const __grid_constant__ CUtensorMap tmo, const PrepParams pp, const ScanParams sp, int n_scan)
 {
-    if ((int)blockIdx.x < n_scan) scan_body<TO, DK, VAR>(tmv, tmo, sp, blockIdx.x);
-    else prep_body<DK, VAR>(tmq, tmk, tmg, pp, blockIdx.x - n_scan, gridDim.x - n_scan);
+    // the scan of a per-head-gate call is the plain layer's
+    if ((int)blockIdx.x < n_scan) scan_body<TO, DK, VK == kVarHeadGate ? kVarPlain : VK>(tmv, tmo, sp, blockIdx.x);
+    else prep_body<DK, VK>(tmq, tmk, tmg, pp, blockIdx.x - n_scan, gridDim.x - n_scan);
 }
+
+// Kernel entry points of one variant kind.
+template <typename TO, int DK, int VK>
+struct Kernels {
+    static constexpr int kScanVK = VK == kVarHeadGate ? kVarPlain : VK;
+    static constexpr auto prep = chunk_prep_kernel<DK, VK>;
+    static constexpr auto scan = chunk_scan_kernel<TO, DK, kScanVK>;
+    static constexpr auto coop = chunk_coop_kernel<TO, DK, VK>;
+};
 
 // ============================================================== host side
 
@@ -1347,7 +1449,10 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
                        cudaStream_t stream)
 {
     const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;
-    const bool variant = (mode & (KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE | KDA_MODE_NORM_QK | KDA_MODE_GATE_LOGITS)) != 0;
+    const int vflags = mode & (KDA_MODE_HEAD_GATE | KDA_MODE_NO_ERASE | KDA_MODE_NORM_QK | KDA_MODE_GATE_LOGITS);
+    const int vk = vflags == 0 ? kVarPlain
+                 : vflags == KDA_MODE_HEAD_GATE ? kVarHeadGate
+                 : vflags == KDA_MODE_NO_ERASE ? kVarNoErase : kVarAny;
     const int req_blocks = (mode >> 8) & 0xff;     // KDA_MODE_BLOCKS(n), 0 = automatic
     const int nsm = sm_count();
     const int nch = cu ? 0 : (T + C - 1) / C;
@@ -1373,8 +1478,12 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (!make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
         !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
         return cudaErrorInvalidValue;
-    auto pk = variant ? chunk_prep_kernel<DK, true> : chunk_prep_kernel<DK, false>;
-    auto sk = variant ? chunk_scan_kernel<TO, DK, true> : chunk_scan_kernel<TO, DK, false>;
+    using K0 = Kernels<TO, DK, kVarPlain>;
+    using K1 = Kernels<TO, DK, kVarHeadGate>;
+    using K2 = Kernels<TO, DK, kVarNoErase>;
+    using K3 = Kernels<TO, DK, kVarAny>;
+    auto pk = vk == kVarPlain ? K0::prep : vk == kVarHeadGate ? K1::prep : vk == kVarNoErase ? K2::prep : K3::prep;
+    auto sk = vk == kVarPlain ? K0::scan : vk == kVarHeadGate ? K1::scan : vk == kVarNoErase ? K2::scan : K3::scan;
     cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);
@@ -1481,7 +1590,7 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     if (coop) {
         unsigned* flags = reinterpret_cast<unsigned*>(ws + L.flags);
         err = cudaMemsetAsync(flags, 0, (size_t)max_chunks * H * 4, stream);
-        auto ck = variant ? chunk_coop_kernel<TO, DK, true> : chunk_coop_kernel<TO, DK, false>;
+        auto ck = vk == kVarPlain ? K0::coop : vk == kVarHeadGate ? K1::coop : vk == kVarNoErase ? K2::coop : K3::coop;
         const int smem = std::max(PrepPlan::BYTES, ScanPlan<DK>::BYTES);
         if (err == cudaSuccess) err = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err == cudaSuccess) {
@@ -1604,8 +1713,8 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
         !make_tmap(&tg, log_alpha, tokens, H, DK, true) || !make_tmap(&tv, v, tokens, H, dv, false, NV, true) ||
         !make_tmap(&to, o, tokens, H, dv, sizeof(TO) == 4, 128 / (int)sizeof(TO), true))
         return cudaErrorInvalidValue;
-    auto pk = chunk_prep_kernel<DK, false>;
-    auto sk = chunk_scan_kernel<TO, DK, false>;
+    auto pk = chunk_prep_kernel<DK, kVarPlain>;
+    auto sk = chunk_scan_kernel<TO, DK, kVarPlain>;
     cudaError_t err = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepPlan::BYTES);
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanPlan<DK>::BYTES);

@@ -93,3 +93,25 @@ def test_varlen_bwd_matches_oracle():
     ref = backward.recurrence_backward(f64(t["q"]), f64(t["k"]), f64(t["v"]), f64(t["beta"]), f64(t["log_alpha"]),
                                        cu, f64(t["initial_state"]), f64(do), f64(dsT))
     _check([f64(x) for x in got], ref)
+
+
+def test_chunk_bwd_prefill_shape_sampled_heads():
+    """The prefill workload at full size (B2 H16 T4096, bf16), gradients of two
+    whole (sequence, head) pairs against the oracle (heads are independent)."""
+    from gated_delta_rule_133_b200.inputs import WORKLOADS
+    w = WORKLOADS["prefill"]
+    x = make_inputs(w, DEV)
+    g = torch.Generator(device=DEV).manual_seed(330)
+    do = torch.randn(w.B, w.T, w.H, w.dv, generator=g, device=DEV)
+    dsT = torch.randn(w.B, w.H, w.dk, w.dv, generator=g, device=DEV)
+    got = kda.kda_chunk_bwd(x["q"], x["k"], x["v"], x["beta"], x["log_alpha"], x["initial_state"], do, dsT)
+    torch.cuda.synchronize()
+    kda.kda_check()
+    for n, h in ((0, 3), (1, 12)):
+        sl = lambda t: f64(t[n, :, h:h + 1])
+        ref = backward.recurrence_backward(sl(x["q"]), sl(x["k"]), sl(x["v"]), f64(x["beta"][n, :, h:h + 1]),
+                                           sl(x["log_alpha"]), None, f64(x["initial_state"][n:n + 1, h:h + 1]),
+                                           sl(do), f64(dsT[n:n + 1, h:h + 1]))
+        mine = [sl(t) for t in got[:3]] + [f64(got[3][n, :, h:h + 1]), sl(got[4]),
+                                            f64(got[5][n:n + 1, h:h + 1])]
+        _check(mine, ref)
