@@ -597,32 +597,38 @@ def run_e2e(kda, host_inputs, w, device, stream, world, ws, steps):
 
 
 # ----------------------------------------------------------------------------- oracle arm
-ORACLE_SAMPLE_TOKENS = 8192
+ORACLE_SAMPLE_TOKENS = 65536
 
 
 def oracle_sample(heads_max=16):
     """Times the fp64 oracle on a bounded sample of the long-context workload:
-    up to `heads_max` heads (one thread each, at most the host's cores) of one
-    sequence of ORACLE_SAMPLE_TOKENS tokens drawn with the workload's recipe.
-    The recurrence costs the same per token, so the rate scales to the whole
-    workload (131072 tokens x 32 heads).  Returns its tokens/s, the threads
-    used and the sample description."""
+    every head (in groups of up to `heads_max`, one thread per head, at most
+    the host's cores) of one sequence of ORACLE_SAMPLE_TOKENS tokens drawn with
+    the workload's recipe, each group drawn with its own seed.  The recurrence
+    costs the same per token, so the rate scales to the whole workload (131072
+    tokens x 32 heads).  Returns its tokens/s, the threads used and the sample
+    description."""
+    import numpy as np
     import oracle
     from gated_delta_rule_133_b200.inputs import WORKLOADS, draw_tokens
     w = WORKLOADS["long"]
     cores = os.cpu_count() or 1
     heads = max(1, min(heads_max, w.H, cores))
+    groups = max(1, min(w.H // heads, 2))
     T = ORACLE_SAMPLE_TOKENS
-    d = draw_tokens(T, heads, w.dk, w.dv, w.dtype, w.gate_mu, w.seed, "cpu")
     f = lambda x: x.to(torch.float64).numpy()
-    import numpy as np
-    t0 = time.perf_counter()
-    oracle.recurrence(f(d["q"]), f(d["k"]), f(d["v"]), f(d["beta"]), f(d["log_alpha"]), np.array([0, T]), None,
-                      nthreads=heads)
-    dt = time.perf_counter() - t0
-    full_time = dt * (w.T / T) * (w.H / heads)
+    dt = 0.0
+    for g in range(groups):
+        d = draw_tokens(T, heads, w.dk, w.dv, w.dtype, w.gate_mu, w.seed + g, "cpu")
+        args = [f(d[n]) for n in ("q", "k", "v", "beta", "log_alpha")]
+        del d
+        t0 = time.perf_counter()
+        oracle.recurrence(*args, np.array([0, T]), None, nthreads=heads)
+        dt += time.perf_counter() - t0
+        del args
+    full_time = dt * (w.T / T) * (w.H / (heads * groups))
     return {"value": w.B * w.T / full_time, "unit": "tokens/s", "cores": heads, "kind": "oracle",
-            "sample": f"long-context recipe, {heads} heads x {T} tokens ({dt:.2f} s, {heads} threads), "
+            "sample": f"long-context recipe, {groups} x {heads} heads x {T} tokens ({dt:.1f} s, {heads} threads), "
                       f"scaled to {w.H} heads x {w.T} tokens"}
 
 

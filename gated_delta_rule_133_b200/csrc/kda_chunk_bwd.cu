@@ -26,12 +26,19 @@
 //   depend on differences of G only), and dlog alpha is the reverse
 //   cumulative sum of dG inside the chunk.
 //
-// One CTA (256 threads) per (sequence, head, 16 value columns).  A forward
-// walk over the chunks stores the state entering every chunk in the
-// workspace; a reverse walk then carries dS.  Gradients that sum over value
-// columns (dq, dk, dbeta, dlog alpha) are added with atomics into outputs the
-// launcher has zeroed; dv and the initial state's gradient belong to one
-// slice each.
+// Only the two walks over the chunks are sequential, and they carry nothing
+// but [d_k x 16] slices of S and dS.  Four launches:
+//   1. factors   one CTA per (chunk, head): the V-independent factors (Q~, K~,
+//                K~n, G, P, T, MA and the channel vectors), once per chunk,
+//                stored as a record;
+//   2. forward   one CTA per (sequence, head, 16 value columns): the state
+//                entering every chunk, and U = T Y;
+//   3. reverse   the same CTAs carry dS back: the gradient reaching every
+//                chunk's end state, dU and dY; dv and dS_0 are written here;
+//   4. gradients one CTA per (chunk, head): every product that sums over
+//                value columns (dP, dT, the a_* terms) over all columns at
+//                once, then dA, and dq, dk, dbeta and dlog alpha of the
+//                chunk's rows, written without atomics.
 #include "kda_chunk.cuh"
 
 namespace kda {
@@ -41,35 +48,17 @@ namespace bwd {
 using simt::mma_tile;
 
 constexpr int C = 64;       // chunk length
-constexpr int NV = 16;      // value columns per CTA
+constexpr int NV = 16;      // value columns per walk CTA, and per pass of the gradient kernel
 constexpr int NT = 256;     // threads per CTA
 
+// Factor record of one (chunk, head), in floats: Q~, K~, K~n, G [C][DK];
+// P, T, MA [C][C]; e^G_m, e^G_last, e^(G_last - G_m) [DK]; beta [C].
 template <int DK>
-struct Smem {
-    static constexpr int LDK = DK + 1;   // padded row pitch of the [C][DK] tiles
-    static constexpr int LDC = C + 1;    // padded pitch of the [C][C] tiles
-    float qm[C * LDK];    // q E, then dG
-    float km[C * LDK];    // k E
-    float kf[C * LDK];    // cumulative gate G, then k F
-    float MA[C * LDC];    // strictly-lower (k E)(k F)^T
-    float P[C * LDC];     // lower-incl (q E)(k F)^T, then T^T dT
-    float T[C * LDC];     // (I + A)^-1
-    float D[C * LDC];     // A, then dP, dT, dA, dMA
-    float S[DK * NV];     // state entering the chunk (slice)
-    float Sm[DK * NV];    // e^G_m S, then the state gradient entering the chunk
-    float dS[DK * NV];    // gradient reaching the state after the chunk
-    float dSg[DK * NV];   // e^(G_last - G_m) dS
-    float V[C * NV];      // V, then V - X
-    float Y[C * NV];      // beta (V - X)
-    float U[C * NV];      // T Y
-    float dO[C * NV];
-    float dU[C * NV];
-    float dY[C * NV];     // T^T dU, then dX = -beta dY
-    float gm[DK];         // e^G_m
-    float gam[DK];        // e^G_last
-    float glm[DK];        // e^(G_last - G_m)
-    float dgl[DK];        // rowsum(dS' S'): the last row's extra dG
-    float beta[C];
+struct Rec {
+    static constexpr int QM = 0, KM = QM + C * DK, KF = KM + C * DK, G = KF + C * DK;
+    static constexpr int P = G + C * DK, T = P + C * C, MA = T + C * C;
+    static constexpr int GM = MA + C * C, GAM = GM + DK, GLM = GAM + DK, BETA = GLM + DK;
+    static constexpr int FLOATS = (BETA + C + 63) & ~63;
 };
 
 struct Params {
@@ -78,33 +67,176 @@ struct Params {
     const float* s0;         // [nseq, H, DK, DV] or nullptr
     const float* dout;       // [tokens, H, DV]
     const float* dsT;        // [nseq, H, DK, DV] or nullptr
-    float* dq;               // [tokens, H, DK], zeroed
+    float* dq;               // [tokens, H, DK]
     float* dk;
     float* dv;               // [tokens, H, DV]
-    float* dbeta;            // [tokens, H], zeroed
-    float* dla;              // [tokens, H, DK], zeroed
+    float* dbeta;            // [tokens, H]
+    float* dla;              // [tokens, H, DK]
     float* ds0;              // [nseq, H, DK, DV] or nullptr
-    float* states;           // workspace: state entering every chunk, and the final one
-    float* escr;             // workspace: E of the current chunk, per CTA [C][DK]
+    float* states;           // state entering every chunk, and the final one: [slot][H][DK][DV]
+    float* rec;              // factor records [record][H][Rec::FLOATS]
+    float* U;                // [record][H][C][DV]
+    float* dU;
+    float* dY;
+    float* dSn;              // gradient reaching the state after each chunk: [record][H][DK][DV]
     const int32_t* cu;
-    const int32_t* choff;    // varlen: first chunk of each sequence
+    const int32_t* choff;    // varlen: first record of each sequence, [nseq + 1]
     long long tokens;
-    int nseq, T, H, DV;
+    long long nrec;          // records per head the workspace holds
+    int nseq, T, H, DV, nch; // nch: chunks per sequence (dense)
 };
 
-// Loads chunk [t0, t0 + L) of one (sequence, head) and forms the gate
-// factors, the intra-chunk products and T = (I + A)^-1 (all threads).
-template <typename TIn, int DK>
-__device__ void prepare(Smem<DK>& sm, const TIn* q, const TIn* k, const TIn* v, const Params& p, int tok,
-                        int L, int h, int col0, float* escr)
+// Chunks of packed sequence i: none for a decreasing pair or a token range
+// that leaves [0, tokens).
+__device__ __forceinline__ int seq_chunks(const int32_t* cu, int i, long long tokens)
 {
-    constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC;
-    const int tid = threadIdx.x, H = p.H;
+    const int a = cu[i], b = cu[i + 1];
+    if (b <= a || a < 0 || (long long)b > tokens) return 0;
+    return (b - a + C - 1) / C;
+}
+
+// Walk range of sequence n: first token, length, first record, first state
+// slot.  A packed sequence whose token range leaves [0, tokens), or whose
+// records would not fit the workspace, is skipped (length 0, no state slot)
+// and reported.
+struct Walk {
+    int tok0, len;
+    long long rbase, sbase;
+    bool has_slots;
+};
+
+__device__ __forceinline__ Walk walk_of(const Params& p, int n, bool report)
+{
+    Walk w{};
+    w.has_slots = true;
+    if (p.cu) {
+        const int a = p.cu[n], b = p.cu[n + 1];
+        w.tok0 = a;
+        w.len = max(0, b - a);
+        w.rbase = p.choff[n];
+        w.sbase = w.rbase + n;
+        const bool bad = w.len > 0 && (a < 0 || (long long)b > p.tokens);
+        if (bad || w.rbase + (w.len + C - 1) / C > p.nrec) {
+            if (report && threadIdx.x == 0) flag_bad_input();
+            w.tok0 = 0;
+            w.len = 0;
+            w.has_slots = !bad && w.rbase <= p.nrec;
+        }
+    } else {
+        w.tok0 = n * p.T;
+        w.len = p.T;
+        w.rbase = (long long)n * p.nch;
+        w.sbase = (long long)n * (p.nch + 1);
+    }
+    return w;
+}
+
+// Position of one (record, head) item.  Records of packed sequences are
+// numbered through choff; items past the last record, or of a sequence whose
+// token range leaves [0, tokens), are not ok.
+struct Pos {
+    long long rc;     // record (chunk) index
+    long long slot;   // state slot of the state entering the chunk
+    int n, tok, L, h;
+    bool ok;
+};
+
+__device__ __forceinline__ Pos locate(const Params& p, long long item)
+{
+    Pos x{};
+    x.h = (int)(item % p.H);
+    x.rc = item / p.H;
+    x.ok = false;
+    if (p.cu) {
+        if (x.rc >= p.choff[p.nseq]) return x;
+        int lo = 0, hi = p.nseq - 1;   // the last sequence whose first record is <= rc
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.choff[mid] <= x.rc) lo = mid;
+            else hi = mid - 1;
+        }
+        const int nc = seq_chunks(p.cu, lo, p.tokens);
+        if (nc == 0 || p.choff[lo] + nc > p.nrec) return x;   // skipped by the walks too
+        const int t0 = p.cu[lo], len = p.cu[lo + 1] - t0;
+        const int c = (int)(x.rc - p.choff[lo]);
+        x.n = lo;
+        x.tok = t0 + c * C;
+        x.L = min(C, len - c * C);
+        x.slot = (long long)p.choff[lo] + lo + c;
+    } else {
+        const int c = (int)(x.rc % p.nch);
+        x.n = (int)(x.rc / p.nch);
+        x.tok = x.n * p.T + c * C;
+        x.L = min(C, p.T - c * C);
+        x.slot = (long long)x.n * (p.nch + 1) + c;
+    }
+    x.ok = x.L > 0;
+    return x;
+}
+
+// Sum over the 16 threads (consecutive lanes) that share tm.
+__device__ __forceinline__ float sum16(float x)
+{
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Copies a [rows][cols] row-major block from global memory into shared
+// memory with row pitch ld, optionally scaling column c by sc[c] (cols a
+// multiple of 4, src 16-byte aligned).
+__device__ __forceinline__ void stage(float* dst, int ld, const float* src, int rows, int cols,
+                                      const float* sc = nullptr)
+{
+    const int q4 = cols / 4;
+    for (int e = threadIdx.x; e < rows * q4; e += NT) {
+        const int r = e / q4, c = 4 * (e % q4);
+        float4 x = *reinterpret_cast<const float4*>(src + (size_t)r * cols + c);
+        if (sc) {
+            x.x *= sc[c];
+            x.y *= sc[c + 1];
+            x.z *= sc[c + 2];
+            x.w *= sc[c + 3];
+        }
+        float* d = dst + r * ld + c;
+        d[0] = x.x;
+        d[1] = x.y;
+        d[2] = x.z;
+        d[3] = x.w;
+    }
+}
+
+// ================================================================ 1. factors
+
+template <int DK>
+struct FacSmem {
+    static constexpr int LDK = DK + 1, LDC = C + 1;
+    float qm[C * LDK];    // q, then q E
+    float km[C * LDK];    // k, then k E
+    float kf[C * LDK];    // log alpha, then G, then k F
+    float D[C * LDC];     // A = beta MA
+    float T[C * LDC];     // (I + A)^-1
+    float beta[C];
+};
+
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(NT, 1)
+bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Params p)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    FacSmem<DK>& sm = *reinterpret_cast<FacSmem<DK>*>(smem_raw);
+    using R = Rec<DK>;
+    constexpr int LDK = FacSmem<DK>::LDK, LDC = FacSmem<DK>::LDC;
+    const Pos x = locate(p, blockIdx.x);
+    if (!x.ok) return;
+    const int tid = threadIdx.x, H = p.H, L = x.L, h = x.h;
+    float* rec = p.rec + (size_t)blockIdx.x * R::FLOATS;
+
     for (int e = tid; e < C * DK; e += NT) {
         const int r = e / DK, c = e % DK;
         float qv = 0.f, kv = 0.f, gv = 0.f;
         if (r < L) {
-            const size_t off = ((size_t)(tok + r) * H + h) * DK + c;
+            const size_t off = ((size_t)(x.tok + r) * H + h) * DK + c;
             qv = Elem<TIn>::load(q + off);
             kv = Elem<TIn>::load(k + off);
             gv = p.log_alpha[off];
@@ -113,32 +245,39 @@ __device__ void prepare(Smem<DK>& sm, const TIn* q, const TIn* k, const TIn* v, 
         sm.km[r * LDK + c] = kv;
         sm.kf[r * LDK + c] = gv;
     }
-    for (int e = tid; e < C * NV; e += NT) {
-        const int r = e / NV, j = e % NV;
-        sm.V[e] = r < L ? Elem<TIn>::load(v + ((size_t)(tok + r) * H + h) * p.DV + col0 + j) : 0.f;
+    if (tid < C) {
+        const float b = tid < L ? p.beta[(size_t)(x.tok + tid) * H + h] : 0.f;
+        sm.beta[tid] = b;
+        rec[R::BETA + tid] = b;
     }
-    if (tid < C) sm.beta[tid] = tid < L ? p.beta[(size_t)(tok + tid) * H + h] : 0.f;
     __syncthreads();
     if (tid < DK) {   // gate cumsum per channel (fp32, log space) and the factor split
         const int c = tid;
         float acc = 0.f;
-        for (int r = 0; r < C; ++r) { acc += sm.kf[r * LDK + c]; sm.kf[r * LDK + c] = acc; }
-        const float Gm = sm.kf[(C / 2 - 1) * LDK + c];
-        sm.gm[c] = expf(Gm);
-        sm.gam[c] = expf(acc);
-        sm.glm[c] = expf(acc - Gm);
         for (int r = 0; r < C; ++r) {
-            const float x = fminf(fmaxf(sm.kf[r * LDK + c] - Gm, -80.f), 80.f);
-            const float E = expf(x), F = expf(-x);
-            if (escr) escr[r * DK + c] = E;
-            sm.qm[r * LDK + c] *= E;
+            acc += sm.kf[r * LDK + c];
+            sm.kf[r * LDK + c] = acc;
+            rec[R::G + r * DK + c] = acc;
+        }
+        const float Gm = sm.kf[(C / 2 - 1) * LDK + c];
+        rec[R::GM + c] = expf(Gm);
+        rec[R::GAM + c] = expf(acc);
+        rec[R::GLM + c] = expf(acc - Gm);
+        for (int r = 0; r < C; ++r) {
+            const float e = fminf(fmaxf(sm.kf[r * LDK + c] - Gm, -80.f), 80.f);
+            const float E = expf(e), F = expf(-e);
+            const float qe = sm.qm[r * LDK + c] * E;
             const float kk = sm.km[r * LDK + c];
+            sm.qm[r * LDK + c] = qe;
             sm.km[r * LDK + c] = kk * E;
             sm.kf[r * LDK + c] = kk * F;
+            rec[R::QM + r * DK + c] = qe;
+            rec[R::KM + r * DK + c] = kk * E;
+            rec[R::KF + r * DK + c] = kk * F;
         }
     }
     __syncthreads();
-    {   // MA (strictly lower), P (lower incl.), A = beta MA -> D
+    {   // MA (strictly lower), P (lower incl.) to the record; A = beta MA -> D
         const int tn = tid % 16, tm = tid / 16;
         float pp[4][4] = {}, a[4][4] = {};
         mma_tile<4, 4>(pp, sm.qm, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
@@ -148,8 +287,8 @@ __device__ void prepare(Smem<DK>& sm, const TIn* q, const TIn* k, const TIn* v, 
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int r = tm + 16 * i, s = tn + 16 * j;
-                sm.P[r * LDC + s] = s <= r ? pp[i][j] : 0.f;
-                sm.MA[r * LDC + s] = s < r ? a[i][j] : 0.f;
+                rec[R::P + r * C + s] = s <= r ? pp[i][j] : 0.f;
+                rec[R::MA + r * C + s] = s < r ? a[i][j] : 0.f;
                 sm.D[r * LDC + s] = s < r ? sm.beta[r] * a[i][j] : 0.f;
             }
     }
@@ -167,46 +306,35 @@ __device__ void prepare(Smem<DK>& sm, const TIn* q, const TIn* k, const TIn* v, 
         }
     }
     __syncthreads();
+    for (int e = tid; e < C * C; e += NT) rec[R::T + e] = sm.T[(e / C) * LDC + e % C];
 }
 
-// X = (k E)(e^G_m S), V <- V - X, Y = beta (V - X), U = T Y   (Sm must hold e^G_m S)
+// ================================================================ 2. forward walk
+
 template <int DK>
-__device__ void chunk_uy(Smem<DK>& sm)
-{
-    constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC;
-    const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
-    float x[4][1] = {};
-    mma_tile<4, 1>(x, sm.km, LDK, 1, sm.Sm, NV, 1, DK, tm, 16, tn, 16);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = tm + 16 * i;
-        const float d = sm.V[r * NV + tn] - x[i][0];
-        sm.V[r * NV + tn] = d;
-        sm.Y[r * NV + tn] = sm.beta[r] * d;
-    }
-    __syncthreads();
-    float u[4][1] = {};
-    mma_tile<4, 1>(u, sm.T, LDC, 1, sm.Y, NV, 1, C, tm, 16, tn, 16);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sm.U[(tm + 16 * i) * NV + tn] = u[i][0];
-    __syncthreads();
-}
-
-// Sum over the 16 threads (consecutive lanes) that share tm.
-__device__ __forceinline__ float sum16(float x)
-{
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
+struct FwdSmem {
+    static constexpr int LDK = DK + 1, LDC = C + 1;
+    float Kh[C * LDK];    // e^G_m K~
+    float Kl[C * LDK];    // e^(G_last - G_m) K~n
+    float T[C * LDC];
+    float S[DK * NV];     // state slice entering the chunk
+    float V[C * NV];
+    float Y[C * NV];
+    float U[C * NV];
+    float gm[DK];
+    float glm[DK];
+    float gam[DK];
+    float beta[C];
+};
 
 template <typename TIn, int DK>
-__global__ void __launch_bounds__(NT, 1)
-chunk_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v, const Params p)
+__global__ void __launch_bounds__(NT, 2)
+bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    Smem<DK>& sm = *reinterpret_cast<Smem<DK>*>(smem_raw);
-    constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC;
+    FwdSmem<DK>& sm = *reinterpret_cast<FwdSmem<DK>*>(smem_raw);
+    using R = Rec<DK>;
+    constexpr int LDK = FwdSmem<DK>::LDK, LDC = FwdSmem<DK>::LDC;
     constexpr int TK = DK / 16;
     const int DV = p.DV, H = p.H;
     const int nslice = DV / NV;
@@ -215,224 +343,183 @@ chunk_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn
     const int n = blockIdx.x / (nslice * H);
     const int col0 = slice * NV;
     const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
-    float* escr = p.escr + (size_t)blockIdx.x * C * DK;
 
-    int tok0, len;
-    long long sbase;   // state slot of the sequence's first chunk
-    if (p.cu) {
-        tok0 = p.cu[n];
-        len = max(0, p.cu[n + 1] - tok0);
-        sbase = (long long)p.choff[n] + n;
-        if (tok0 < 0 || (long long)tok0 + len > p.tokens) {   // no tokens read; the state passes through
-            if (tid == 0) flag_bad_input();
-            tok0 = 0;
-            len = 0;
-        }
-    } else {
-        tok0 = n * p.T;
-        len = p.T;
-        sbase = (long long)n * ((p.T + C - 1) / C + 1);
-    }
+    const Walk wk = walk_of(p, n, true);
+    if (!wk.has_slots) return;   // nothing of this sequence is read again
+    const int tok0 = wk.tok0, len = wk.len;
+    const long long sbase = wk.sbase, rbase = wk.rbase;
     const int nch = (len + C - 1) / C;
-    auto state_at = [&](int c) { return p.states + ((sbase + c) * H + h) * (size_t)DK * DV + col0; };
 
-    // ---- forward walk: the state entering every chunk (and after the last)
     for (int e = tid; e < DK * NV; e += NT) {
         const int c = e / NV, j = e % NV;
         sm.S[e] = p.s0 ? p.s0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
     }
     __syncthreads();
     for (int ci = 0; ci < nch; ++ci) {
-        const int L = min(C, len - ci * C);
-        float* st = state_at(ci);
+        const int L = min(C, len - ci * C), tok = tok0 + ci * C;
+        const size_t item = (size_t)(rbase + ci) * H + h;
+        const float* rec = p.rec + item * R::FLOATS;
+        float* st = p.states + ((sbase + ci) * H + h) * (size_t)DK * DV + col0;
         for (int e = tid; e < DK * NV; e += NT) st[(e / NV) * DV + e % NV] = sm.S[e];
-        prepare<TIn, DK>(sm, q, k, v, p, tok0 + ci * C, L, h, col0, nullptr);
-        for (int e = tid; e < DK * NV; e += NT) sm.Sm[e] = sm.gm[e / NV] * sm.S[e];
+        if (tid < DK) {
+            sm.gm[tid] = rec[R::GM + tid];
+            sm.glm[tid] = rec[R::GLM + tid];
+            sm.gam[tid] = rec[R::GAM + tid];
+        }
+        if (tid < C) sm.beta[tid] = rec[R::BETA + tid];
+        for (int e = tid; e < C * NV; e += NT) {
+            const int r = e / NV, j = e % NV;
+            sm.V[e] = r < L ? Elem<TIn>::load(v + ((size_t)(tok + r) * H + h) * DV + col0 + j) : 0.f;
+        }
         __syncthreads();
-        chunk_uy<DK>(sm);
-        {   // S <- gamma S + e^(G_last - G_m) (k F)^T U
+        stage(sm.Kh, LDK, rec + R::KM, C, DK, sm.gm);
+        stage(sm.Kl, LDK, rec + R::KF, C, DK, sm.glm);
+        stage(sm.T, LDC, rec + R::T, C, C);
+        __syncthreads();
+        {   // X = Kh S, Y = beta (V - X)
+            float xx[4][1] = {};
+            mma_tile<4, 1>(xx, sm.Kh, LDK, 1, sm.S, NV, 1, DK, tm, 16, tn, 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = tm + 16 * i;
+                sm.Y[r * NV + tn] = sm.beta[r] * (sm.V[r * NV + tn] - xx[i][0]);
+            }
+        }
+        __syncthreads();
+        {   // U = T Y
+            float u[4][1] = {};
+            mma_tile<4, 1>(u, sm.T, LDC, 1, sm.Y, NV, 1, C, tm, 16, tn, 16);
+            float* ug = p.U + item * (size_t)C * DV + col0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = tm + 16 * i;
+                sm.U[r * NV + tn] = u[i][0];
+                ug[(size_t)r * DV + tn] = u[i][0];
+            }
+        }
+        __syncthreads();
+        {   // S <- gamma S + Kl^T U
             float ds[TK][1] = {};
-            mma_tile<TK, 1>(ds, sm.kf, 1, LDK, sm.U, NV, 1, C, tm, 16, tn, 16);
+            mma_tile<TK, 1>(ds, sm.Kl, 1, LDK, sm.U, NV, 1, C, tm, 16, tn, 16);
 #pragma unroll
             for (int i = 0; i < TK; ++i) {
                 const int c = tm + 16 * i, e = c * NV + tn;
-                sm.S[e] = fmaf(sm.gam[c], sm.S[e], sm.glm[c] * ds[i][0]);
+                sm.S[e] = fmaf(sm.gam[c], sm.S[e], ds[i][0]);
             }
         }
         __syncthreads();
     }
-    {
-        float* st = state_at(nch);
-        for (int e = tid; e < DK * NV; e += NT) st[(e / NV) * DV + e % NV] = sm.S[e];
-    }
+    float* st = p.states + ((sbase + nch) * H + h) * (size_t)DK * DV + col0;
+    for (int e = tid; e < DK * NV; e += NT) st[(e / NV) * DV + e % NV] = sm.S[e];
+}
 
-    // ---- reverse walk carrying dS
+// ================================================================ 3. reverse walk
+
+template <int DK>
+struct RevSmem {
+    static constexpr int LDK = DK + 1, LDC = C + 1;
+    float Qh[C * LDK];    // e^G_m Q~
+    float Kh[C * LDK];    // e^G_m K~
+    float Kl[C * LDK];    // e^(G_last - G_m) K~n
+    float P[C * LDC];
+    float T[C * LDC];
+    float dS[DK * NV];    // gradient reaching the state after the chunk, then before it
+    float dO[C * NV];
+    float dU[C * NV];
+    float dY[C * NV];     // dX = -beta dY
+    float gm[DK];
+    float glm[DK];
+    float gam[DK];
+    float beta[C];
+};
+
+template <int DK>
+__global__ void __launch_bounds__(NT, 1)
+bwd_reverse_kernel(const Params p)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    RevSmem<DK>& sm = *reinterpret_cast<RevSmem<DK>*>(smem_raw);
+    using R = Rec<DK>;
+    constexpr int LDK = RevSmem<DK>::LDK, LDC = RevSmem<DK>::LDC;
+    constexpr int TK = DK / 16;
+    const int DV = p.DV, H = p.H;
+    const int nslice = DV / NV;
+    const int slice = blockIdx.x % nslice;
+    const int h = (blockIdx.x / nslice) % H;
+    const int n = blockIdx.x / (nslice * H);
+    const int col0 = slice * NV;
+    const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
+
+    const Walk wk = walk_of(p, n, false);   // a skipped sequence was reported by the forward walk
+    const int tok0 = wk.tok0, len = wk.len;
+    const long long rbase = wk.rbase;
+    const int nch = (len + C - 1) / C;
+
     for (int e = tid; e < DK * NV; e += NT) {
         const int c = e / NV, j = e % NV;
         sm.dS[e] = p.dsT ? p.dsT[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
     }
-    __threadfence_block();
     __syncthreads();
     for (int ci = nch - 1; ci >= 0; --ci) {
         const int L = min(C, len - ci * C), tok = tok0 + ci * C;
-        prepare<TIn, DK>(sm, q, k, v, p, tok, L, h, col0, escr);
-        {
-            const float* st = state_at(ci);
-            const float* st1 = state_at(ci + 1);
-            for (int e = tid; e < DK * NV; e += NT) {
-                const int c = e / NV, j = e % NV;
-                const float s = st[c * DV + j];
-                sm.S[e] = s;
-                sm.Sm[e] = sm.gm[c] * s;
-                sm.dSg[e] = sm.glm[c] * sm.dS[e];
-            }
-            for (int e = tid; e < C * NV; e += NT) {
-                const int r = e / NV, j = e % NV;
-                sm.dO[e] = r < L ? p.dout[((size_t)(tok + r) * H + h) * DV + col0 + j] : 0.f;
-            }
-            if (tid < DK) {   // rowsum(dS' S'), S' = the state after this chunk
-                float a = 0.f;
-                for (int j = 0; j < NV; ++j) a = fmaf(sm.dS[tid * NV + j], st1[tid * DV + j], a);
-                sm.dgl[tid] = a;
-            }
+        const size_t item = (size_t)(rbase + ci) * H + h;
+        const float* rec = p.rec + item * R::FLOATS;
+        float* dsn = p.dSn + item * (size_t)DK * DV + col0;
+        for (int e = tid; e < DK * NV; e += NT) dsn[(e / NV) * DV + e % NV] = sm.dS[e];
+        if (tid < DK) {
+            sm.gm[tid] = rec[R::GM + tid];
+            sm.glm[tid] = rec[R::GLM + tid];
+            sm.gam[tid] = rec[R::GAM + tid];
+        }
+        if (tid < C) sm.beta[tid] = rec[R::BETA + tid];
+        for (int e = tid; e < C * NV; e += NT) {
+            const int r = e / NV, j = e % NV;
+            sm.dO[e] = r < L ? p.dout[((size_t)(tok + r) * H + h) * DV + col0 + j] : 0.f;
         }
         __syncthreads();
-        chunk_uy<DK>(sm);
-
-        float aq[4][TK] = {}, ak[4][TK] = {}, an[4][TK] = {};
-        // a_q = e^G_m dO S^T, a_n = e^(G_last - G_m) U dS'^T
-        mma_tile<4, TK>(aq, sm.dO, NV, 1, sm.Sm, 1, NV, NV, tm, 16, tn, 16);
-        mma_tile<4, TK>(an, sm.U, NV, 1, sm.dSg, 1, NV, NV, tm, 16, tn, 16);
+        stage(sm.Qh, LDK, rec + R::QM, C, DK, sm.gm);
+        stage(sm.Kh, LDK, rec + R::KM, C, DK, sm.gm);
+        stage(sm.Kl, LDK, rec + R::KF, C, DK, sm.glm);
+        stage(sm.P, LDC, rec + R::P, C, C);
+        stage(sm.T, LDC, rec + R::T, C, C);
+        __syncthreads();
         {   // dU = P^T dO + Kl dS'
             float du[4][1] = {};
             mma_tile<4, 1>(du, sm.P, 1, LDC, sm.dO, NV, 1, C, tm, 16, tn, 16);
-            mma_tile<4, 1>(du, sm.kf, LDK, 1, sm.dSg, NV, 1, DK, tm, 16, tn, 16);
+            mma_tile<4, 1>(du, sm.Kl, LDK, 1, sm.dS, NV, 1, DK, tm, 16, tn, 16);
+            float* g = p.dU + item * (size_t)C * DV + col0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) sm.dU[(tm + 16 * i) * NV + tn] = du[i][0];
+            for (int i = 0; i < 4; ++i) {
+                const int r = tm + 16 * i;
+                sm.dU[r * NV + tn] = du[i][0];
+                g[(size_t)r * DV + tn] = du[i][0];
+            }
         }
         __syncthreads();
-        float db[4];
-        {   // dY = T^T dU; dv = beta dY; dbeta = rowsum((V - X) dY)
+        {   // dY = T^T dU; dv = beta dY; dX = -beta dY
             float dy[4][1] = {};
             mma_tile<4, 1>(dy, sm.T, 1, LDC, sm.dU, NV, 1, C, tm, 16, tn, 16);
+            float* g = p.dY + item * (size_t)C * DV + col0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = tm + 16 * i;
-                sm.dY[r * NV + tn] = dy[i][0];
-                if (r < L) p.dv[((size_t)(tok + r) * H + h) * DV + col0 + tn] = sm.beta[r] * dy[i][0];
-                db[i] = sum16(sm.V[r * NV + tn] * dy[i][0]);
-            }
-        }
-        {   // dP = lower-incl(dO U^T) -> D
-            float dp[4][4] = {};
-            mma_tile<4, 4>(dp, sm.dO, NV, 1, sm.U, 1, NV, NV, tm, 16, tn, 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int r = tm + 16 * i, s = tn + 16 * j;
-                    sm.D[r * LDC + s] = s <= r ? dp[i][j] : 0.f;
-                }
-        }
-        __syncthreads();
-        // a_k = e^G_m dX S^T (dX = -beta dY); a_q += dP K~n; a_n += dP^T Q~
-        {
-            float t[4][TK] = {};
-            mma_tile<4, TK>(t, sm.dY, NV, 1, sm.Sm, 1, NV, NV, tm, 16, tn, 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < TK; ++j) ak[i][j] = -sm.beta[tm + 16 * i] * t[i][j];
-        }
-        mma_tile<4, TK>(aq, sm.D, LDC, 1, sm.kf, LDK, 1, C, tm, 16, tn, 16);
-        mma_tile<4, TK>(an, sm.D, 1, LDC, sm.qm, LDK, 1, C, tm, 16, tn, 16);
-        __syncthreads();
-        {   // dT = dU Y^T -> D
-            float dt[4][4] = {};
-            mma_tile<4, 4>(dt, sm.dU, NV, 1, sm.Y, 1, NV, NV, tm, 16, tn, 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) sm.D[(tm + 16 * i) * LDC + tn + 16 * j] = dt[i][j];
-        }
-        __syncthreads();
-        {   // T^T dT -> P
-            float z[4][4] = {};
-            mma_tile<4, 4>(z, sm.T, 1, LDC, sm.D, LDC, 1, C, tm, 16, tn, 16);
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) sm.P[(tm + 16 * i) * LDC + tn + 16 * j] = z[i][j];
-        }
-        __syncthreads();
-        {   // dA = -strictly-lower((T^T dT) T^T); dbeta += rowsum(MA dA); dMA = beta dA -> D
-            float da[4][4] = {};
-            mma_tile<4, 4>(da, sm.P, LDC, 1, sm.T, 1, LDC, C, tm, 16, tn, 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = tm + 16 * i;
-                float part = 0.f;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int s = tn + 16 * j;
-                    const float a = s < r ? -da[i][j] : 0.f;
-                    part = fmaf(sm.MA[r * LDC + s], a, part);
-                    sm.D[r * LDC + s] = sm.beta[r] * a;
-                }
-                db[i] += sum16(part);
+                const float b = sm.beta[r];
+                g[(size_t)r * DV + tn] = dy[i][0];
+                sm.dY[r * NV + tn] = -b * dy[i][0];
+                if (r < L) p.dv[((size_t)(tok + r) * H + h) * DV + col0 + tn] = b * dy[i][0];
             }
         }
         __syncthreads();
-        // a_k += dMA K~n; a_n += dMA^T K~
-        mma_tile<4, TK>(ak, sm.D, LDC, 1, sm.kf, LDK, 1, C, tm, 16, tn, 16);
-        mma_tile<4, TK>(an, sm.D, 1, LDC, sm.km, LDK, 1, C, tm, 16, tn, 16);
-        {   // dX = -beta dY (in dY); then dS = diag(gamma) dS' + e^G_m ((q E)^T dO + (k E)^T dX) -> Sm
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = tm + 16 * i;
-                sm.dY[r * NV + tn] *= -sm.beta[r];
-            }
-            __syncthreads();
+        {   // dS = diag(gamma) dS' + Qh^T dO + Kh^T dX
             float ds[TK][1] = {};
-            mma_tile<TK, 1>(ds, sm.qm, 1, LDK, sm.dO, NV, 1, C, tm, 16, tn, 16);
-            mma_tile<TK, 1>(ds, sm.km, 1, LDK, sm.dY, NV, 1, C, tm, 16, tn, 16);
+            mma_tile<TK, 1>(ds, sm.Qh, 1, LDK, sm.dO, NV, 1, C, tm, 16, tn, 16);
+            mma_tile<TK, 1>(ds, sm.Kh, 1, LDK, sm.dY, NV, 1, C, tm, 16, tn, 16);
 #pragma unroll
             for (int i = 0; i < TK; ++i) {
                 const int c = tm + 16 * i, e = c * NV + tn;
-                sm.Sm[e] = fmaf(sm.gam[c], sm.dS[e], sm.gm[c] * ds[i][0]);
+                sm.dS[e] = fmaf(sm.gam[c], sm.dS[e], ds[i][0]);
             }
         }
-        __syncthreads();
-        // dG = Q~ a_q + K~ a_k - K~n a_n (into qm); dq = E a_q, dk = E a_k + a_n / E
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = tm + 16 * i;
-#pragma unroll
-            for (int j = 0; j < TK; ++j) {
-                const int c = tn + 16 * j;
-                const float g = sm.qm[r * LDK + c] * aq[i][j] + sm.km[r * LDK + c] * ak[i][j] -
-                                sm.kf[r * LDK + c] * an[i][j];
-                sm.qm[r * LDK + c] = g;
-                if (r < L) {
-                    const float E = escr[r * DK + c];
-                    const size_t off = ((size_t)(tok + r) * H + h) * DK + c;
-                    atomicAdd(p.dq + off, E * aq[i][j]);
-                    atomicAdd(p.dk + off, E * ak[i][j] + an[i][j] / E);
-                }
-            }
-            if (tn == 0 && r < L) atomicAdd(p.dbeta + (size_t)(tok + r) * H + h, db[i]);
-        }
-        __syncthreads();
-        if (tid < DK) {   // dlog alpha: reverse cumulative sum of dG inside the chunk
-            const int c = tid;
-            float acc = sm.dgl[c];
-            for (int r = L - 1; r >= 0; --r) {
-                acc += sm.qm[r * LDK + c];
-                atomicAdd(p.dla + ((size_t)(tok + r) * H + h) * DK + c, acc);
-            }
-        }
-        for (int e = tid; e < DK * NV; e += NT) sm.dS[e] = sm.Sm[e];
         __syncthreads();
     }
     if (p.ds0)
@@ -442,17 +529,216 @@ chunk_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn
         }
 }
 
-// First chunk of every packed sequence: choff[i] = sum_{j<i} ceil(len_j / 64)
-// (negative lengths count as empty).  One CTA; each thread sums a contiguous
-// range of sequences, then a block-wide scan.
-__global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, int nseq, int32_t* choff)
+// ================================================================ 4. gradients
+
+template <int DK>
+struct GradSmem {
+    static constexpr int LDK = DK + 1, LDC = C + 1;
+    float qm[C * LDK];    // Q~, then dG
+    float km[C * LDK];    // K~
+    float kf[C * LDK];    // K~n
+    float MA[C * LDC];
+    float T[C * LDC];
+    float D1[C * LDC];    // dP, then T^T dT
+    float D2[C * LDC];    // dT, then dMA
+    float Sm[DK * NV];    // e^G_m S (value columns of this pass)
+    float dSg[DK * NV];   // e^(G_last - G_m) dS'
+    float VX[C * NV];     // V, then V - X
+    float dO[C * NV];
+    float U[C * NV];
+    float dU[C * NV];
+    float Y[C * NV];      // beta (V - X)
+    float dX[C * NV];     // -beta dY
+    float gm[DK];
+    float glm[DK];
+    float dgl[DK];        // rowsum(dS' S'): the last row's extra dG
+    float beta[C];
+    float db[C];
+};
+
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(NT, 1)
+bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    GradSmem<DK>& sm = *reinterpret_cast<GradSmem<DK>*>(smem_raw);
+    using R = Rec<DK>;
+    constexpr int LDK = GradSmem<DK>::LDK, LDC = GradSmem<DK>::LDC;
+    constexpr int TK = DK / 16;
+    const Pos x = locate(p, blockIdx.x);
+    if (!x.ok) return;
+    const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
+    const int DV = p.DV, H = p.H, L = x.L, h = x.h;
+    const size_t item = blockIdx.x;
+    const float* rec = p.rec + item * R::FLOATS;
+    const float* S0 = p.states + ((size_t)x.slot * H + h) * (size_t)DK * DV;          // entering the chunk
+    const float* S1 = p.states + ((size_t)(x.slot + 1) * H + h) * (size_t)DK * DV;    // after it
+    const float* dS1 = p.dSn + item * (size_t)DK * DV;
+    const float* Ug = p.U + item * (size_t)C * DV;
+    const float* dUg = p.dU + item * (size_t)C * DV;
+    const float* dYg = p.dY + item * (size_t)C * DV;
+
+    if (tid < DK) {
+        sm.gm[tid] = rec[R::GM + tid];
+        sm.glm[tid] = rec[R::GLM + tid];
+    }
+    if (tid < C) sm.beta[tid] = rec[R::BETA + tid];
+    stage(sm.qm, LDK, rec + R::QM, C, DK);
+    stage(sm.km, LDK, rec + R::KM, C, DK);
+    stage(sm.kf, LDK, rec + R::KF, C, DK);
+    stage(sm.MA, LDC, rec + R::MA, C, C);
+    stage(sm.T, LDC, rec + R::T, C, C);
+
+    float aq[4][TK] = {}, ak[4][TK] = {}, an[4][TK] = {};
+    float dp[4][4] = {}, dt[4][4] = {};
+    float db1[4] = {0.f, 0.f, 0.f, 0.f};
+    float dgl[TK] = {};   // channel tm + 16 i, summed over this thread's columns
+    for (int j0 = 0; j0 < DV; j0 += NV) {
+        __syncthreads();   // the previous pass has read its slices (first pass: the vectors are in place)
+        for (int e = tid; e < DK * NV; e += NT) {
+            const int c = e / NV, j = e % NV;
+            const size_t g = (size_t)c * DV + j0 + j;
+            sm.Sm[e] = sm.gm[c] * S0[g];
+            sm.dSg[e] = sm.glm[c] * dS1[g];
+        }
+#pragma unroll
+        for (int i = 0; i < TK; ++i) {   // thread (tm, tn): channel tm + 16 i, column tn
+            const size_t g = (size_t)(tm + 16 * i) * DV + j0 + tn;
+            dgl[i] = fmaf(dS1[g], S1[g], dgl[i]);
+        }
+        for (int e = tid; e < C * NV; e += NT) {
+            const int r = e / NV, j = e % NV;
+            const size_t g = (size_t)r * DV + j0 + j;
+            const bool in = r < L;
+            sm.VX[e] = in ? Elem<TIn>::load(v + ((size_t)(x.tok + r) * H + h) * DV + j0 + j) : 0.f;
+            sm.dO[e] = in ? p.dout[((size_t)(x.tok + r) * H + h) * DV + j0 + j] : 0.f;
+            sm.U[e] = Ug[g];
+            sm.dU[e] = dUg[g];
+            sm.dX[e] = -sm.beta[r] * dYg[g];
+        }
+        __syncthreads();
+        {   // X = K~ (e^G_m S); V - X; Y = beta (V - X); rowsum((V - X) dY)
+            float xx[4][1] = {};
+            mma_tile<4, 1>(xx, sm.km, LDK, 1, sm.Sm, NV, 1, DK, tm, 16, tn, 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = tm + 16 * i, e = r * NV + tn;
+                const float vx = sm.VX[e] - xx[i][0];
+                sm.VX[e] = vx;
+                sm.Y[e] = sm.beta[r] * vx;
+                db1[i] = fmaf(vx, dYg[(size_t)r * DV + j0 + tn], db1[i]);
+            }
+        }
+        __syncthreads();
+        // a_q += dO Sm^T, a_k += dX Sm^T, a_n += U dSg^T; dP += dO U^T, dT += dU Y^T
+        mma_tile<4, TK>(aq, sm.dO, NV, 1, sm.Sm, 1, NV, NV, tm, 16, tn, 16);
+        mma_tile<4, TK>(ak, sm.dX, NV, 1, sm.Sm, 1, NV, NV, tm, 16, tn, 16);
+        mma_tile<4, TK>(an, sm.U, NV, 1, sm.dSg, 1, NV, NV, tm, 16, tn, 16);
+        mma_tile<4, 4>(dp, sm.dO, NV, 1, sm.U, 1, NV, NV, tm, 16, tn, 16);
+        mma_tile<4, 4>(dt, sm.dU, NV, 1, sm.Y, 1, NV, NV, tm, 16, tn, 16);
+    }
+    // dP (lower incl.) -> D1, dT -> D2; dgl and the first part of dbeta
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = tm + 16 * i;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int s = tn + 16 * j;
+            sm.D1[r * LDC + s] = s <= r ? dp[i][j] : 0.f;
+            sm.D2[r * LDC + s] = dt[i][j];
+        }
+        const float b = sum16(db1[i]);
+        if (tn == 0) sm.db[r] = b;
+    }
+#pragma unroll
+    for (int i = 0; i < TK; ++i) {
+        const float g = sum16(dgl[i]);
+        if (tn == 0) sm.dgl[tm + 16 * i] = g;
+    }
+    __syncthreads();
+    // a_q += dP K~n; a_n += dP^T Q~
+    mma_tile<4, TK>(aq, sm.D1, LDC, 1, sm.kf, LDK, 1, C, tm, 16, tn, 16);
+    mma_tile<4, TK>(an, sm.D1, 1, LDC, sm.qm, LDK, 1, C, tm, 16, tn, 16);
+    {   // T^T dT
+        float z[4][4] = {};
+        mma_tile<4, 4>(z, sm.T, 1, LDC, sm.D2, LDC, 1, C, tm, 16, tn, 16);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sm.D1[(tm + 16 * i) * LDC + tn + 16 * j] = z[i][j];
+    }
+    __syncthreads();
+    {   // dA = -strictly-lower((T^T dT) T^T); dbeta += rowsum(MA dA); dMA = beta dA -> D2
+        float da[4][4] = {};
+        mma_tile<4, 4>(da, sm.D1, LDC, 1, sm.T, 1, LDC, C, tm, 16, tn, 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = tm + 16 * i;
+            float part = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int s = tn + 16 * j;
+                const float a = s < r ? -da[i][j] : 0.f;
+                part = fmaf(sm.MA[r * LDC + s], a, part);
+                sm.D2[r * LDC + s] = sm.beta[r] * a;
+            }
+            const float b = sum16(part);
+            if (tn == 0) sm.db[r] += b;
+        }
+    }
+    __syncthreads();
+    // a_k += dMA K~n; a_n += dMA^T K~
+    mma_tile<4, TK>(ak, sm.D2, LDC, 1, sm.kf, LDK, 1, C, tm, 16, tn, 16);
+    mma_tile<4, TK>(an, sm.D2, 1, LDC, sm.km, LDK, 1, C, tm, 16, tn, 16);
+    // dG = Q~ a_q + K~ a_k - K~n a_n into qm (each thread rewrites only the
+    // elements it reads; no product reads Q~ any more); dq = E a_q,
+    // dk = E a_k + a_n / E
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = tm + 16 * i;
+#pragma unroll
+        for (int j = 0; j < TK; ++j) {
+            const int c = tn + 16 * j;
+            const float g = sm.qm[r * LDK + c] * aq[i][j] + sm.km[r * LDK + c] * ak[i][j] -
+                            sm.kf[r * LDK + c] * an[i][j];
+            sm.qm[r * LDK + c] = g;
+            if (r < L) {
+                const float e = fminf(fmaxf(rec[R::G + r * DK + c] - rec[R::G + (C / 2 - 1) * DK + c], -80.f), 80.f);
+                const float E = expf(e);
+                const size_t off = ((size_t)(x.tok + r) * H + h) * DK + c;
+                p.dq[off] = E * aq[i][j];
+                p.dk[off] = E * ak[i][j] + an[i][j] / E;
+            }
+        }
+    }
+    __syncthreads();
+    if (tid < DK) {   // dlog alpha: reverse cumulative sum of dG inside the chunk
+        const int c = tid;
+        float acc = sm.dgl[c];
+        for (int r = L - 1; r >= 0; --r) {
+            acc += sm.qm[r * LDK + c];
+            p.dla[((size_t)(x.tok + r) * H + h) * DK + c] = acc;
+        }
+    }
+    if (tid < L) p.dbeta[(size_t)(x.tok + tid) * H + h] = sm.db[tid];
+}
+
+// ================================================================ host side
+
+// First record of every packed sequence: choff[i] = sum_{j<i} of its chunks
+// (seq_chunks: none for an empty or out-of-range sequence), choff[nseq] = the
+// total.  One CTA; each
+// thread sums a contiguous range of sequences, then a block-wide scan.
+__global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, int nseq, long long tokens,
+                                                             int32_t* choff)
 {
     __shared__ int warp_tot[32];
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int per = (nseq + 1023) / 1024;
     const int a = min(nseq, tid * per), b = min(nseq, a + per);
     int local = 0;
-    for (int i = a; i < b; ++i) local += (max(0, cu[i + 1] - cu[i]) + C - 1) / C;
+    for (int i = a; i < b; ++i) local += seq_chunks(cu, i, tokens);
     int x = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -474,35 +760,85 @@ __global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, 
     int base = x - local + (w ? warp_tot[w - 1] : 0);
     for (int i = a; i < b; ++i) {
         choff[i] = base;
-        base += (max(0, cu[i + 1] - cu[i]) + C - 1) / C;
+        base += seq_chunks(cu, i, tokens);
     }
+    if (tid == 1023) choff[nseq] = base;
 }
 
-// Bytes of workspace: states (chunks + 1 per sequence), the E scratch of
-// every CTA, and for packed batches the chunk offsets.
+// Parts of a call's workspace (byte offsets).
+struct Ws {
+    size_t states, rec, U, dU, dY, dSn, choff, bytes;
+    long long nrec;   // records per head (an upper bound for packed batches)
+};
+
+static size_t al1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
+
+static Ws ws_layout(int nseq, int T, long long tokens, int H, int dk, int dv, bool varlen)
+{
+    Ws w{};
+    const int nch = (T + C - 1) / C;
+    w.nrec = varlen ? tokens / C + nseq : (long long)nseq * nch;
+    const long long slots = varlen ? tokens / C + 2LL * nseq : (long long)nseq * (nch + 1);
+    const size_t recf = dk == 128 ? Rec<128>::FLOATS : Rec<64>::FLOATS;
+    size_t off = 0;
+    w.states = off;
+    off += al1k((size_t)slots * H * dk * dv * 4);
+    w.rec = off;
+    off += al1k((size_t)w.nrec * H * recf * 4);
+    w.U = off;
+    off += al1k((size_t)w.nrec * H * C * dv * 4);
+    w.dU = off;
+    off += al1k((size_t)w.nrec * H * C * dv * 4);
+    w.dY = off;
+    off += al1k((size_t)w.nrec * H * C * dv * 4);
+    w.dSn = off;
+    off += al1k((size_t)w.nrec * H * dk * dv * 4);
+    w.choff = off;
+    off += varlen ? al1k(((size_t)nseq + 1) * 4) : 0;
+    w.bytes = off;
+    return w;
+}
+
 size_t workspace(int nseq, int T, long long tokens, int H, int dk, int dv, bool varlen)
 {
-    const long long slots = varlen ? tokens / C + 2LL * nseq : (long long)nseq * ((T + C - 1) / C + 1);
-    const long long ctas = (long long)nseq * H * (dv / NV);
-    auto al = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
-    return al((size_t)slots * H * dk * dv * 4) + al((size_t)ctas * C * dk * 4) +
-           (varlen ? al(((size_t)nseq + 1) * 4) : 0);
+    return ws_layout(nseq, T, tokens, H, dk, dv, varlen).bytes;
 }
 
 template <typename TIn, int DK>
-cudaError_t launch(const void* q, const void* k, const void* v, Params p, int dv, unsigned char* ws,
-                   cudaStream_t stream)
+cudaError_t launch(const void* q, const void* k, const void* v, const Params& p, long long nrec, cudaStream_t stream)
 {
-    const long long ctas = (long long)p.nseq * p.H * (dv / NV);
-    if (ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    auto kern = chunk_bwd_kernel<TIn, DK>;
-    const size_t smem = sizeof(Smem<DK>);
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const long long walk_ctas = (long long)p.nseq * p.H * (p.DV / NV);
+    const long long items = nrec * p.H;
+    if (walk_ctas > 0x7fffffffLL || items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    auto kf = bwd_factor_kernel<TIn, DK>;
+    auto kw = bwd_forward_kernel<TIn, DK>;
+    auto kr = bwd_reverse_kernel<DK>;
+    auto kg = bwd_grad_kernel<TIn, DK>;
+    cudaError_t err = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(FacSmem<DK>));
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(kw, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(FwdSmem<DK>));
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RevSmem<DK>));
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(GradSmem<DK>));
     if (err != cudaSuccess) return err;
-    if (ctas == 0) return cudaSuccess;
-    kern<<<(unsigned)ctas, NT, smem, stream>>>(static_cast<const TIn*>(q), static_cast<const TIn*>(k),
-                                               static_cast<const TIn*>(v), p);
-    return cudaGetLastError();
+    if (walk_ctas == 0) return cudaSuccess;
+    const TIn* qq = static_cast<const TIn*>(q);
+    const TIn* kk = static_cast<const TIn*>(k);
+    const TIn* vv = static_cast<const TIn*>(v);
+    if (items > 0) {
+        kf<<<(unsigned)items, NT, sizeof(FacSmem<DK>), stream>>>(qq, kk, p);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    kw<<<(unsigned)walk_ctas, NT, sizeof(FwdSmem<DK>), stream>>>(vv, p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    kr<<<(unsigned)walk_ctas, NT, sizeof(RevSmem<DK>), stream>>>(p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (items > 0) {
+        kg<<<(unsigned)items, NT, sizeof(GradSmem<DK>), stream>>>(vv, p);
+        err = cudaGetLastError();
+    }
+    return err;
 }
 
 }  // namespace bwd
@@ -518,10 +854,8 @@ cudaError_t chunk_bwd(const void* q, const void* k, const void* v, const float* 
                       int H, int dkd, int dvd, kda_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream)
 {
     const bool varlen = cu != nullptr;
-    if (!ws || ws_bytes < bwd::workspace(nseq, T, tokens, H, dkd, dvd, varlen)) return cudaErrorInvalidValue;
-    auto al = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
-    const long long slots = varlen ? tokens / bwd::C + 2LL * nseq : (long long)nseq * ((T + bwd::C - 1) / bwd::C + 1);
-    const long long ctas = (long long)nseq * H * (dvd / bwd::NV);
+    const bwd::Ws L = bwd::ws_layout(nseq, T, tokens, H, dkd, dvd, varlen);
+    if (!ws || ws_bytes < L.bytes) return cudaErrorInvalidValue;
     unsigned char* w = static_cast<unsigned char*>(ws);
     bwd::Params p{};
     p.beta = beta;
@@ -535,32 +869,41 @@ cudaError_t chunk_bwd(const void* q, const void* k, const void* v, const float* 
     p.dbeta = dbeta;
     p.dla = dla;
     p.ds0 = ds0;
-    p.states = reinterpret_cast<float*>(w);
-    p.escr = reinterpret_cast<float*>(w + al((size_t)slots * H * dkd * dvd * 4));
-    int32_t* choff = reinterpret_cast<int32_t*>(w + al((size_t)slots * H * dkd * dvd * 4) +
-                                                al((size_t)ctas * bwd::C * dkd * 4));
+    p.states = reinterpret_cast<float*>(w + L.states);
+    p.rec = reinterpret_cast<float*>(w + L.rec);
+    p.U = reinterpret_cast<float*>(w + L.U);
+    p.dU = reinterpret_cast<float*>(w + L.dU);
+    p.dY = reinterpret_cast<float*>(w + L.dY);
+    p.dSn = reinterpret_cast<float*>(w + L.dSn);
+    int32_t* choff = reinterpret_cast<int32_t*>(w + L.choff);
     p.cu = cu;
     p.choff = varlen ? choff : nullptr;
     p.tokens = tokens;
+    p.nrec = L.nrec;
     p.nseq = nseq;
     p.T = T;
     p.H = H;
     p.DV = dvd;
-    const size_t th = (size_t)tokens * H;
-    cudaError_t err = cudaMemsetAsync(dq, 0, th * dkd * 4, stream);
-    if (err == cudaSuccess) err = cudaMemsetAsync(dk, 0, th * dkd * 4, stream);
-    if (err == cudaSuccess) err = cudaMemsetAsync(dla, 0, th * dkd * 4, stream);
-    if (err == cudaSuccess) err = cudaMemsetAsync(dbeta, 0, th * 4, stream);
-    if (err == cudaSuccess && varlen) {
-        bwd::chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu, nseq, choff);
-        err = cudaGetLastError();
+    p.nch = varlen ? 0 : (T + bwd::C - 1) / bwd::C;
+    cudaError_t err = cudaSuccess;
+    if (varlen) {   // rows outside every sequence get zero gradients (dense batches write every row)
+        const size_t th = (size_t)tokens * H;
+        err = cudaMemsetAsync(dq, 0, th * dkd * 4, stream);
+        if (err == cudaSuccess) err = cudaMemsetAsync(dk, 0, th * dkd * 4, stream);
+        if (err == cudaSuccess) err = cudaMemsetAsync(dla, 0, th * dkd * 4, stream);
+        if (err == cudaSuccess) err = cudaMemsetAsync(dbeta, 0, th * 4, stream);
+        if (err == cudaSuccess) {
+            bwd::chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu, nseq, tokens, choff);
+            err = cudaGetLastError();
+        }
     }
     if (err != cudaSuccess) return err;
     using bf = __nv_bfloat16;
     if (dtype == KDA_BF16)
-        return dkd == 128 ? bwd::launch<bf, 128>(q, k, v, p, dvd, w, stream) : bwd::launch<bf, 64>(q, k, v, p, dvd, w, stream);
-    return dkd == 128 ? bwd::launch<float, 128>(q, k, v, p, dvd, w, stream)
-                      : bwd::launch<float, 64>(q, k, v, p, dvd, w, stream);
+        return dkd == 128 ? bwd::launch<bf, 128>(q, k, v, p, L.nrec, stream)
+                          : bwd::launch<bf, 64>(q, k, v, p, L.nrec, stream);
+    return dkd == 128 ? bwd::launch<float, 128>(q, k, v, p, L.nrec, stream)
+                      : bwd::launch<float, 64>(q, k, v, p, L.nrec, stream);
 }
 
 }  // namespace kda
