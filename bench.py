@@ -469,8 +469,9 @@ def run_dplr(kda, device, stream, world, rank, reps=3):
           for _ in range(2)]
     o = torch.empty(w.B, w.T, w.H, w.dv, device=device)
     sN = torch.empty(w.B, w.H, w.dk, w.dv, device=device)
+    ws = torch.empty(kda.dplr_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv), dtype=torch.uint8, device=device)
     call = lambda: kda.kda_dplr_fwd(d["q"], d["k"], d["v"], ab[0], ab[1], d["log_alpha"], d["initial_state"],
-                                    o=o, final_state=sN, stream=stream)
+                                    o=o, final_state=sN, stream=stream, workspace=ws)
     call()
     torch.cuda.synchronize(device)
     ev = event_pairs(reps)

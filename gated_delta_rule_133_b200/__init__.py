@@ -33,7 +33,7 @@ from ._lib import KdaError
 
 __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_varlen_fwd", "kda_recurrent_step", "kda_check",
            "kda_chunk_bwd", "kda_varlen_bwd", "kda_dplr_fwd", "kda_dplr_varlen_fwd", "chunk_fwd_workspace_size",
-           "varlen_fwd_workspace_size", "KdaError"]
+           "varlen_fwd_workspace_size", "dplr_fwd_workspace_size", "KdaError"]
 
 _DTYPES = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
 
@@ -56,6 +56,11 @@ def chunk_fwd_workspace_size(B, T, H, dk, dv, dtype=torch.bfloat16, chunk=64, mo
 def varlen_fwd_workspace_size(N, T, H, dk, dv, dtype=torch.bfloat16, chunk=64, mode=0):
     """Workspace bytes kda_varlen_fwd needs for N packed sequences of T tokens in all."""
     return _lib.workspace_size("kda_varlen_fwd_workspace_size", N, T, H, dk, dv, chunk, _DTYPES[dtype], mode)
+
+
+def dplr_fwd_workspace_size(B, T, H, dk, dv, dtype=torch.bfloat16, chunk=64):
+    """Workspace bytes kda_dplr_fwd needs for these sizes."""
+    return _lib.workspace_size("kda_dplr_fwd_workspace_size", B, T, H, dk, dv, chunk, _DTYPES[dtype])
 
 
 def _workspace(nbytes, workspace, device):
@@ -277,7 +282,7 @@ def kda_varlen_bwd(q, k, v, beta, log_alpha, cu_seqlens, initial_state, grad_o, 
 
 
 def kda_dplr_fwd(q, k, v, a, b, log_alpha, initial_state=None, *, o=None, final_state=None,
-                 output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None):
+                 output_final_state=True, o_dtype=torch.float32, chunk=64, workspace=None, stream=None):
     """Diagonal-plus-low-rank transition S_t = (Diag(alpha_t) + b_t a_t^T) S_{t-1} + k_t v_t^T,
     o_t = S_t^T q_t.  q, k, a, b [B, T, H, dk], v [B, T, H, dv] (bf16 or fp32);
     log_alpha [B, T, H, dk] fp32; initial_state [B, H, dk, dv] or None.
@@ -298,13 +303,16 @@ def kda_dplr_fwd(q, k, v, a, b, log_alpha, initial_state=None, *, o=None, final_
     _check(o, "o", (B, T, H, dv), o.dtype, dev)
     if final_state is None and output_final_state:
         final_state = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    nbytes = _lib.workspace_size("kda_dplr_fwd_workspace_size", B, T, H, dk, dv, chunk, _DTYPES[dt])
+    ws = _workspace(nbytes, workspace, dev)
     _lib.call("kda_dplr_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(log_alpha), _ptr(initial_state),
-              _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk, _DTYPES[dt], _DTYPES[o.dtype], _stream(stream))
+              _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk, _DTYPES[dt], _DTYPES[o.dtype], *ws,
+              _stream(stream))
     return o, final_state
 
 
 def kda_dplr_varlen_fwd(q, k, v, a, b, log_alpha, cu_seqlens, initial_state=None, *, o=None, final_state=None,
-                        output_final_state=True, o_dtype=torch.float32, chunk=64, stream=None):
+                        output_final_state=True, o_dtype=torch.float32, chunk=64, workspace=None, stream=None):
     """kda_dplr_fwd over N packed variable-length sequences ([T, H, ...] layouts)."""
     T, H, dk = q.shape
     dv = v.shape[-1]
@@ -323,9 +331,11 @@ def kda_dplr_varlen_fwd(q, k, v, a, b, log_alpha, cu_seqlens, initial_state=None
     _check(o, "o", (T, H, dv), o.dtype, dev)
     if final_state is None and output_final_state:
         final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    nbytes = _lib.workspace_size("kda_dplr_varlen_fwd_workspace_size", N, T, H, dk, dv, chunk, _DTYPES[dt])
+    ws = _workspace(nbytes, workspace, dev)
     _lib.call("kda_dplr_varlen_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(log_alpha), _ptr(cu_seqlens),
               N, _ptr(initial_state), _ptr(o), _ptr(final_state), T, H, dk, dv, chunk, _DTYPES[dt], _DTYPES[o.dtype],
-              _stream(stream))
+              *ws, _stream(stream))
     return o, final_state
 
 

@@ -42,8 +42,10 @@ SIGNATURES = {
     "kda_chunk_bwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _ZP]),
     "kda_varlen_bwd": (_I, [_P] * 6 + [_I] + [_P] * 9 + [_I, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "kda_varlen_bwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _ZP]),
-    "kda_dplr_fwd": (_I, [_P] * 9 + [_I] * 8 + [_P]),
-    "kda_dplr_varlen_fwd": (_I, [_P] * 7 + [_I] + [_P] * 3 + [_I] * 7 + [_P]),
+    "kda_dplr_fwd": (_I, [_P] * 9 + [_I] * 8 + [_P, _Z, _P]),
+    "kda_dplr_fwd_workspace_size": (_I, [_I] * 7 + [_ZP]),
+    "kda_dplr_varlen_fwd": (_I, [_P] * 7 + [_I] + [_P] * 3 + [_I] * 7 + [_P, _Z, _P]),
+    "kda_dplr_varlen_fwd_workspace_size": (_I, [_I] * 7 + [_ZP]),
     "kda_check": (_I, [_P]),
     "kda_selftest_timeout": (_I, [ctypes.c_longlong, _P]),
     "kda_status_string": (ctypes.c_char_p, [_I]),

@@ -336,9 +336,32 @@ kda_status kda_varlen_bwd(const void* q, const void* k, const void* v, const flo
                                     dv, dtype, workspace, workspace_bytes_, s));
 }
 
+kda_status kda_dplr_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                                       size_t* bytes)
+{
+    if (!bytes || B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    const kda_status st = check_sizes(H, dk, dv, chunk, dtype, 0);
+    if (st != KDA_OK) return st;
+    const long long tokens = (long long)B * T;
+    if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    *bytes = tokens == 0 ? 0 : kda::dplr_fwd_workspace(B, T, tokens, H, dk, dv, false);
+    return KDA_OK;
+}
+
+kda_status kda_dplr_varlen_fwd_workspace_size(int N, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                                              size_t* bytes)
+{
+    if (!bytes || N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
+    const kda_status st = check_sizes(H, dk, dv, chunk, dtype, 0);
+    if (st != KDA_OK) return st;
+    *bytes = (N == 0 || T == 0) ? 0 : kda::dplr_fwd_workspace(N, 0, T, H, dk, dv, true);
+    return KDA_OK;
+}
+
 kda_status kda_dplr_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
                         const float* log_alpha, const float* initial_state, void* o, float* final_state, int B, int T,
-                        int H, int dk, int dv, int chunk, kda_dtype dtype, kda_dtype o_dtype, void* stream)
+                        int H, int dk, int dv, int chunk, kda_dtype dtype, kda_dtype o_dtype, void* workspace,
+                        size_t workspace_bytes, void* stream)
 {
     if (B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
     const long long tokens = (long long)B * T;
@@ -349,14 +372,16 @@ kda_status kda_dplr_fwd(const void* q, const void* k, const void* v, const void*
     if (tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (tokens == 0) return copy_state(initial_state, final_state, (size_t)B * H * dk * dv, s);
+    st = check_workspace(workspace, workspace_bytes, kda::dplr_fwd_workspace(B, T, tokens, H, dk, dv, false));
+    if (st != KDA_OK) return st;
     return from_cuda(kda::dplr_fwd(q, k, v, a, b, log_alpha, initial_state, o, final_state, nullptr, B, T, tokens, H, dk,
-                                   dv, dtype, o_dtype, s));
+                                   dv, dtype, o_dtype, workspace, workspace_bytes, s));
 }
 
 kda_status kda_dplr_varlen_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
                                const float* log_alpha, const int32_t* cu_seqlens, int N, const float* initial_state,
                                void* o, float* final_state, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
-                               kda_dtype o_dtype, void* stream)
+                               kda_dtype o_dtype, void* workspace, size_t workspace_bytes, void* stream)
 {
     if (N < 0 || N > 65535 || T < 0) return KDA_ERR_INVALID_ARG;
     kda_status st = check_fwd(q, k, v, (const float*)q, log_alpha, initial_state, o, final_state, T, H, dk, dv, chunk,
@@ -367,8 +392,10 @@ kda_status kda_dplr_varlen_fwd(const void* q, const void* k, const void* v, cons
     if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0) return copy_state(initial_state, final_state, (size_t)N * H * dk * dv, s);
+    st = check_workspace(workspace, workspace_bytes, kda::dplr_fwd_workspace(N, 0, T, H, dk, dv, true));
+    if (st != KDA_OK) return st;
     return from_cuda(kda::dplr_fwd(q, k, v, a, b, log_alpha, initial_state, o, final_state, cu_seqlens, N, 0, T, H, dk,
-                                   dv, dtype, o_dtype, s));
+                                   dv, dtype, o_dtype, workspace, workspace_bytes, s));
 }
 
 kda_status kda_check(void* stream)

@@ -54,8 +54,10 @@ cudaError_t chunk_bwd(const void* q, const void* k, const void* v, const float* 
 
 // Chunkwise forward of the diagonal-plus-low-rank transition on CUDA cores
 // (fp32): S_t = (Diag(alpha_t) + b_t a_t^T) S_{t-1} + k_t v_t^T, o_t = S_t^T q_t.
+// dplr_fwd_workspace gives the bytes of workspace a call needs.
+size_t dplr_fwd_workspace(int nseq, int T, long long tokens, int H, int dk, int dv, bool varlen);
 cudaError_t dplr_fwd(const void* q, const void* k, const void* v, const void* a, const void* b, const float* log_alpha,
                      const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens, int H,
-                     int dk, int dv, kda_dtype dtype, kda_dtype o_dtype, cudaStream_t s);
+                     int dk, int dv, kda_dtype dtype, kda_dtype o_dtype, void* ws, size_t ws_bytes, cudaStream_t s);
 
 }  // namespace kda

@@ -27,11 +27,11 @@
 //   cumulative sum of dG inside the chunk.
 //
 // Only the two walks over the chunks are sequential, and they carry nothing
-// but [d_k x 16] slices of S and dS.  Four launches:
+// but [d_k x 32] slices of S and dS.  Four launches:
 //   1. factors   one CTA per (chunk, head): the V-independent factors (Q~, K~,
 //                K~n, G, P, T, MA and the channel vectors), once per chunk,
 //                stored as a record;
-//   2. forward   one CTA per (sequence, head, 16 value columns): the state
+//   2. forward   one CTA per (sequence, head, 32 value columns): the state
 //                entering every chunk, and U = T Y;
 //   3. reverse   the same CTAs carry dS back: the gradient reaching every
 //                chunk's end state, dU and dY; dv and dS_0 are written here;
@@ -40,6 +40,7 @@
 //                once, then dA, and dq, dk, dbeta and dlog alpha of the
 //                chunk's rows, written without atomics.
 #include "kda_chunk.cuh"
+#include "kda_packed.cuh"
 
 namespace kda {
 
@@ -48,7 +49,8 @@ namespace bwd {
 using simt::mma_tile;
 
 constexpr int C = 64;       // chunk length
-constexpr int NV = 16;      // value columns per walk CTA, and per pass of the gradient kernel
+constexpr int NW = 32;      // value columns per walk CTA
+constexpr int NV = 16;      // value columns per pass of the gradient kernel
 constexpr int NT = 256;     // threads per CTA
 
 // Factor record of one (chunk, head), in floats: Q~, K~, K~n, G [C][DK];
@@ -86,92 +88,9 @@ struct Params {
     int nseq, T, H, DV, nch; // nch: chunks per sequence (dense)
 };
 
-// Chunks of packed sequence i: none for a decreasing pair or a token range
-// that leaves [0, tokens).
-__device__ __forceinline__ int seq_chunks(const int32_t* cu, int i, long long tokens)
+__device__ __forceinline__ packed::Layout layout_of(const Params& p)
 {
-    const int a = cu[i], b = cu[i + 1];
-    if (b <= a || a < 0 || (long long)b > tokens) return 0;
-    return (b - a + C - 1) / C;
-}
-
-// Walk range of sequence n: first token, length, first record, first state
-// slot.  A packed sequence whose token range leaves [0, tokens), or whose
-// records would not fit the workspace, is skipped (length 0, no state slot)
-// and reported.
-struct Walk {
-    int tok0, len;
-    long long rbase, sbase;
-    bool has_slots;
-};
-
-__device__ __forceinline__ Walk walk_of(const Params& p, int n, bool report)
-{
-    Walk w{};
-    w.has_slots = true;
-    if (p.cu) {
-        const int a = p.cu[n], b = p.cu[n + 1];
-        w.tok0 = a;
-        w.len = max(0, b - a);
-        w.rbase = p.choff[n];
-        w.sbase = w.rbase + n;
-        const bool bad = w.len > 0 && (a < 0 || (long long)b > p.tokens);
-        if (bad || w.rbase + (w.len + C - 1) / C > p.nrec) {
-            if (report && threadIdx.x == 0) flag_bad_input();
-            w.tok0 = 0;
-            w.len = 0;
-            w.has_slots = !bad && w.rbase <= p.nrec;
-        }
-    } else {
-        w.tok0 = n * p.T;
-        w.len = p.T;
-        w.rbase = (long long)n * p.nch;
-        w.sbase = (long long)n * (p.nch + 1);
-    }
-    return w;
-}
-
-// Position of one (record, head) item.  Records of packed sequences are
-// numbered through choff; items past the last record, or of a sequence whose
-// token range leaves [0, tokens), are not ok.
-struct Pos {
-    long long rc;     // record (chunk) index
-    long long slot;   // state slot of the state entering the chunk
-    int n, tok, L, h;
-    bool ok;
-};
-
-__device__ __forceinline__ Pos locate(const Params& p, long long item)
-{
-    Pos x{};
-    x.h = (int)(item % p.H);
-    x.rc = item / p.H;
-    x.ok = false;
-    if (p.cu) {
-        if (x.rc >= p.choff[p.nseq]) return x;
-        int lo = 0, hi = p.nseq - 1;   // the last sequence whose first record is <= rc
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (p.choff[mid] <= x.rc) lo = mid;
-            else hi = mid - 1;
-        }
-        const int nc = seq_chunks(p.cu, lo, p.tokens);
-        if (nc == 0 || p.choff[lo] + nc > p.nrec) return x;   // skipped by the walks too
-        const int t0 = p.cu[lo], len = p.cu[lo + 1] - t0;
-        const int c = (int)(x.rc - p.choff[lo]);
-        x.n = lo;
-        x.tok = t0 + c * C;
-        x.L = min(C, len - c * C);
-        x.slot = (long long)p.choff[lo] + lo + c;
-    } else {
-        const int c = (int)(x.rc % p.nch);
-        x.n = (int)(x.rc / p.nch);
-        x.tok = x.n * p.T + c * C;
-        x.L = min(C, p.T - c * C);
-        x.slot = (long long)x.n * (p.nch + 1) + c;
-    }
-    x.ok = x.L > 0;
-    return x;
+    return packed::Layout{p.cu, p.choff, p.tokens, p.nrec, p.nseq, p.T, p.nch, p.H};
 }
 
 // Sum over the 16 threads (consecutive lanes) that share tm.
@@ -182,27 +101,36 @@ __device__ __forceinline__ float sum16(float x)
     return x;
 }
 
-// Copies a [rows][cols] row-major block from global memory into shared
-// memory with row pitch ld, optionally scaling column c by sc[c] (cols a
-// multiple of 4, src 16-byte aligned).
-__device__ __forceinline__ void stage(float* dst, int ld, const float* src, int rows, int cols,
-                                      const float* sc = nullptr)
+// Copies a [ROWS][COLS] row-major block from global memory into shared
+// memory with row pitch ld, optionally scaling column c by sc[c].  Every load
+// of a thread is issued before its first store (src 16-byte aligned, read-only
+// for the kernel's lifetime).
+template <int ROWS, int COLS>
+__device__ __forceinline__ void stage(float* dst, int ld, const float* src, const float* sc = nullptr)
 {
-    const int q4 = cols / 4;
-    for (int e = threadIdx.x; e < rows * q4; e += NT) {
-        const int r = e / q4, c = 4 * (e % q4);
-        float4 x = *reinterpret_cast<const float4*>(src + (size_t)r * cols + c);
+    constexpr int Q4 = COLS / 4, N = ROWS * Q4 / NT;
+    static_assert(ROWS * Q4 % NT == 0, "tile not a multiple of the CTA");
+    float4 x[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int e = threadIdx.x + i * NT;
+        x[i] = __ldg(reinterpret_cast<const float4*>(src + (size_t)(e / Q4) * COLS + 4 * (e % Q4)));
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int e = threadIdx.x + i * NT;
+        const int r = e / Q4, c = 4 * (e % Q4);
         if (sc) {
-            x.x *= sc[c];
-            x.y *= sc[c + 1];
-            x.z *= sc[c + 2];
-            x.w *= sc[c + 3];
+            x[i].x *= sc[c];
+            x[i].y *= sc[c + 1];
+            x[i].z *= sc[c + 2];
+            x[i].w *= sc[c + 3];
         }
         float* d = dst + r * ld + c;
-        d[0] = x.x;
-        d[1] = x.y;
-        d[2] = x.z;
-        d[3] = x.w;
+        d[0] = x[i].x;
+        d[1] = x[i].y;
+        d[2] = x[i].z;
+        d[3] = x[i].w;
     }
 }
 
@@ -227,7 +155,7 @@ bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Pa
     FacSmem<DK>& sm = *reinterpret_cast<FacSmem<DK>*>(smem_raw);
     using R = Rec<DK>;
     constexpr int LDK = FacSmem<DK>::LDK, LDC = FacSmem<DK>::LDC;
-    const Pos x = locate(p, blockIdx.x);
+    const packed::Pos x = packed::locate(layout_of(p), blockIdx.x);
     if (!x.ok) return;
     const int tid = threadIdx.x, H = p.H, L = x.L, h = x.h;
     float* rec = p.rec + (size_t)blockIdx.x * R::FLOATS;
@@ -317,10 +245,10 @@ struct FwdSmem {
     float Kh[C * LDK];    // e^G_m K~
     float Kl[C * LDK];    // e^(G_last - G_m) K~n
     float T[C * LDC];
-    float S[DK * NV];     // state slice entering the chunk
-    float V[C * NV];
-    float Y[C * NV];
-    float U[C * NV];
+    float S[DK * NW];     // state slice entering the chunk
+    float V[C * NW];
+    float Y[C * NW];
+    float U[C * NW];
     float gm[DK];
     float glm[DK];
     float gam[DK];
@@ -328,7 +256,7 @@ struct FwdSmem {
 };
 
 template <typename TIn, int DK>
-__global__ void __launch_bounds__(NT, 2)
+__global__ void __launch_bounds__(NT, 1)
 bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -337,21 +265,21 @@ bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
     constexpr int LDK = FwdSmem<DK>::LDK, LDC = FwdSmem<DK>::LDC;
     constexpr int TK = DK / 16;
     const int DV = p.DV, H = p.H;
-    const int nslice = DV / NV;
+    const int nslice = DV / NW;
     const int slice = blockIdx.x % nslice;
     const int h = (blockIdx.x / nslice) % H;
     const int n = blockIdx.x / (nslice * H);
-    const int col0 = slice * NV;
+    const int col0 = slice * NW;
     const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
 
-    const Walk wk = walk_of(p, n, true);
+    const packed::Walk wk = packed::walk_of(layout_of(p), n, true);
     if (!wk.has_slots) return;   // nothing of this sequence is read again
     const int tok0 = wk.tok0, len = wk.len;
     const long long sbase = wk.sbase, rbase = wk.rbase;
     const int nch = (len + C - 1) / C;
 
-    for (int e = tid; e < DK * NV; e += NT) {
-        const int c = e / NV, j = e % NV;
+    for (int e = tid; e < DK * NW; e += NT) {
+        const int c = e / NW, j = e % NW;
         sm.S[e] = p.s0 ? p.s0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
     }
     __syncthreads();
@@ -360,57 +288,63 @@ bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
         const size_t item = (size_t)(rbase + ci) * H + h;
         const float* rec = p.rec + item * R::FLOATS;
         float* st = p.states + ((sbase + ci) * H + h) * (size_t)DK * DV + col0;
-        for (int e = tid; e < DK * NV; e += NT) st[(e / NV) * DV + e % NV] = sm.S[e];
+        for (int e = tid; e < DK * NW; e += NT) st[(e / NW) * DV + e % NW] = sm.S[e];
         if (tid < DK) {
             sm.gm[tid] = rec[R::GM + tid];
             sm.glm[tid] = rec[R::GLM + tid];
             sm.gam[tid] = rec[R::GAM + tid];
         }
         if (tid < C) sm.beta[tid] = rec[R::BETA + tid];
-        for (int e = tid; e < C * NV; e += NT) {
-            const int r = e / NV, j = e % NV;
+        for (int e = tid; e < C * NW; e += NT) {
+            const int r = e / NW, j = e % NW;
             sm.V[e] = r < L ? Elem<TIn>::load(v + ((size_t)(tok + r) * H + h) * DV + col0 + j) : 0.f;
         }
         __syncthreads();
-        stage(sm.Kh, LDK, rec + R::KM, C, DK, sm.gm);
-        stage(sm.Kl, LDK, rec + R::KF, C, DK, sm.glm);
-        stage(sm.T, LDC, rec + R::T, C, C);
+        stage<C, DK>(sm.Kh, LDK, rec + R::KM, sm.gm);
+        stage<C, DK>(sm.Kl, LDK, rec + R::KF, sm.glm);
+        stage<C, C>(sm.T, LDC, rec + R::T);
         __syncthreads();
         {   // X = Kh S, Y = beta (V - X)
-            float xx[4][1] = {};
-            mma_tile<4, 1>(xx, sm.Kh, LDK, 1, sm.S, NV, 1, DK, tm, 16, tn, 16);
+            float xx[4][2] = {};
+            mma_tile<4, 2>(xx, sm.Kh, LDK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = tm + 16 * i;
-                sm.Y[r * NV + tn] = sm.beta[r] * (sm.V[r * NV + tn] - xx[i][0]);
-            }
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int r = tm + 16 * i, e = r * NW + tn + 16 * j;
+                    sm.Y[e] = sm.beta[r] * (sm.V[e] - xx[i][j]);
+                }
         }
         __syncthreads();
         {   // U = T Y
-            float u[4][1] = {};
-            mma_tile<4, 1>(u, sm.T, LDC, 1, sm.Y, NV, 1, C, tm, 16, tn, 16);
+            float u[4][2] = {};
+            mma_tile<4, 2>(u, sm.T, LDC, 1, sm.Y, NW, 1, C, tm, 16, tn, 16);
             float* ug = p.U + item * (size_t)C * DV + col0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = tm + 16 * i;
-                sm.U[r * NV + tn] = u[i][0];
-                ug[(size_t)r * DV + tn] = u[i][0];
-            }
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int r = tm + 16 * i, cc = tn + 16 * j;
+                    sm.U[r * NW + cc] = u[i][j];
+                    ug[(size_t)r * DV + cc] = u[i][j];
+                }
         }
         __syncthreads();
         {   // S <- gamma S + Kl^T U
-            float ds[TK][1] = {};
-            mma_tile<TK, 1>(ds, sm.Kl, 1, LDK, sm.U, NV, 1, C, tm, 16, tn, 16);
+            float ds[TK][2] = {};
+            mma_tile<TK, 2>(ds, sm.Kl, 1, LDK, sm.U, NW, 1, C, tm, 16, tn, 16);
 #pragma unroll
-            for (int i = 0; i < TK; ++i) {
-                const int c = tm + 16 * i, e = c * NV + tn;
-                sm.S[e] = fmaf(sm.gam[c], sm.S[e], ds[i][0]);
-            }
+            for (int i = 0; i < TK; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
+                    sm.S[e] = fmaf(sm.gam[c], sm.S[e], ds[i][j]);
+                }
         }
         __syncthreads();
     }
     float* st = p.states + ((sbase + nch) * H + h) * (size_t)DK * DV + col0;
-    for (int e = tid; e < DK * NV; e += NT) st[(e / NV) * DV + e % NV] = sm.S[e];
+    for (int e = tid; e < DK * NW; e += NT) st[(e / NW) * DV + e % NW] = sm.S[e];
 }
 
 // ================================================================ 3. reverse walk
@@ -423,10 +357,10 @@ struct RevSmem {
     float Kl[C * LDK];    // e^(G_last - G_m) K~n
     float P[C * LDC];
     float T[C * LDC];
-    float dS[DK * NV];    // gradient reaching the state after the chunk, then before it
-    float dO[C * NV];
-    float dU[C * NV];
-    float dY[C * NV];     // dX = -beta dY
+    float dS[DK * NW];    // gradient reaching the state after the chunk, then before it
+    float dO[C * NW];
+    float dU[C * NW];
+    float dY[C * NW];     // dX = -beta dY
     float gm[DK];
     float glm[DK];
     float gam[DK];
@@ -443,20 +377,21 @@ bwd_reverse_kernel(const Params p)
     constexpr int LDK = RevSmem<DK>::LDK, LDC = RevSmem<DK>::LDC;
     constexpr int TK = DK / 16;
     const int DV = p.DV, H = p.H;
-    const int nslice = DV / NV;
+    const int nslice = DV / NW;
     const int slice = blockIdx.x % nslice;
     const int h = (blockIdx.x / nslice) % H;
     const int n = blockIdx.x / (nslice * H);
-    const int col0 = slice * NV;
+    const int col0 = slice * NW;
     const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
 
-    const Walk wk = walk_of(p, n, false);   // a skipped sequence was reported by the forward walk
+    // a skipped sequence was reported by the forward walk
+    const packed::Walk wk = packed::walk_of(layout_of(p), n, false);
     const int tok0 = wk.tok0, len = wk.len;
     const long long rbase = wk.rbase;
     const int nch = (len + C - 1) / C;
 
-    for (int e = tid; e < DK * NV; e += NT) {
-        const int c = e / NV, j = e % NV;
+    for (int e = tid; e < DK * NW; e += NT) {
+        const int c = e / NW, j = e % NW;
         sm.dS[e] = p.dsT ? p.dsT[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
     }
     __syncthreads();
@@ -465,66 +400,72 @@ bwd_reverse_kernel(const Params p)
         const size_t item = (size_t)(rbase + ci) * H + h;
         const float* rec = p.rec + item * R::FLOATS;
         float* dsn = p.dSn + item * (size_t)DK * DV + col0;
-        for (int e = tid; e < DK * NV; e += NT) dsn[(e / NV) * DV + e % NV] = sm.dS[e];
+        for (int e = tid; e < DK * NW; e += NT) dsn[(e / NW) * DV + e % NW] = sm.dS[e];
         if (tid < DK) {
             sm.gm[tid] = rec[R::GM + tid];
             sm.glm[tid] = rec[R::GLM + tid];
             sm.gam[tid] = rec[R::GAM + tid];
         }
         if (tid < C) sm.beta[tid] = rec[R::BETA + tid];
-        for (int e = tid; e < C * NV; e += NT) {
-            const int r = e / NV, j = e % NV;
+        for (int e = tid; e < C * NW; e += NT) {
+            const int r = e / NW, j = e % NW;
             sm.dO[e] = r < L ? p.dout[((size_t)(tok + r) * H + h) * DV + col0 + j] : 0.f;
         }
         __syncthreads();
-        stage(sm.Qh, LDK, rec + R::QM, C, DK, sm.gm);
-        stage(sm.Kh, LDK, rec + R::KM, C, DK, sm.gm);
-        stage(sm.Kl, LDK, rec + R::KF, C, DK, sm.glm);
-        stage(sm.P, LDC, rec + R::P, C, C);
-        stage(sm.T, LDC, rec + R::T, C, C);
+        stage<C, DK>(sm.Qh, LDK, rec + R::QM, sm.gm);
+        stage<C, DK>(sm.Kh, LDK, rec + R::KM, sm.gm);
+        stage<C, DK>(sm.Kl, LDK, rec + R::KF, sm.glm);
+        stage<C, C>(sm.P, LDC, rec + R::P);
+        stage<C, C>(sm.T, LDC, rec + R::T);
         __syncthreads();
         {   // dU = P^T dO + Kl dS'
-            float du[4][1] = {};
-            mma_tile<4, 1>(du, sm.P, 1, LDC, sm.dO, NV, 1, C, tm, 16, tn, 16);
-            mma_tile<4, 1>(du, sm.Kl, LDK, 1, sm.dS, NV, 1, DK, tm, 16, tn, 16);
+            float du[4][2] = {};
+            mma_tile<4, 2>(du, sm.P, 1, LDC, sm.dO, NW, 1, C, tm, 16, tn, 16);
+            mma_tile<4, 2>(du, sm.Kl, LDK, 1, sm.dS, NW, 1, DK, tm, 16, tn, 16);
             float* g = p.dU + item * (size_t)C * DV + col0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = tm + 16 * i;
-                sm.dU[r * NV + tn] = du[i][0];
-                g[(size_t)r * DV + tn] = du[i][0];
-            }
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int r = tm + 16 * i, cc = tn + 16 * j;
+                    sm.dU[r * NW + cc] = du[i][j];
+                    g[(size_t)r * DV + cc] = du[i][j];
+                }
         }
         __syncthreads();
         {   // dY = T^T dU; dv = beta dY; dX = -beta dY
-            float dy[4][1] = {};
-            mma_tile<4, 1>(dy, sm.T, 1, LDC, sm.dU, NV, 1, C, tm, 16, tn, 16);
+            float dy[4][2] = {};
+            mma_tile<4, 2>(dy, sm.T, 1, LDC, sm.dU, NW, 1, C, tm, 16, tn, 16);
             float* g = p.dY + item * (size_t)C * DV + col0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = tm + 16 * i;
-                const float b = sm.beta[r];
-                g[(size_t)r * DV + tn] = dy[i][0];
-                sm.dY[r * NV + tn] = -b * dy[i][0];
-                if (r < L) p.dv[((size_t)(tok + r) * H + h) * DV + col0 + tn] = b * dy[i][0];
-            }
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int r = tm + 16 * i, cc = tn + 16 * j;
+                    const float b = sm.beta[r];
+                    g[(size_t)r * DV + cc] = dy[i][j];
+                    sm.dY[r * NW + cc] = -b * dy[i][j];
+                    if (r < L) p.dv[((size_t)(tok + r) * H + h) * DV + col0 + cc] = b * dy[i][j];
+                }
         }
         __syncthreads();
         {   // dS = diag(gamma) dS' + Qh^T dO + Kh^T dX
-            float ds[TK][1] = {};
-            mma_tile<TK, 1>(ds, sm.Qh, 1, LDK, sm.dO, NV, 1, C, tm, 16, tn, 16);
-            mma_tile<TK, 1>(ds, sm.Kh, 1, LDK, sm.dY, NV, 1, C, tm, 16, tn, 16);
+            float ds[TK][2] = {};
+            mma_tile<TK, 2>(ds, sm.Qh, 1, LDK, sm.dO, NW, 1, C, tm, 16, tn, 16);
+            mma_tile<TK, 2>(ds, sm.Kh, 1, LDK, sm.dY, NW, 1, C, tm, 16, tn, 16);
 #pragma unroll
-            for (int i = 0; i < TK; ++i) {
-                const int c = tm + 16 * i, e = c * NV + tn;
-                sm.dS[e] = fmaf(sm.gam[c], sm.dS[e], ds[i][0]);
-            }
+            for (int i = 0; i < TK; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
+                    sm.dS[e] = fmaf(sm.gam[c], sm.dS[e], ds[i][j]);
+                }
         }
         __syncthreads();
     }
     if (p.ds0)
-        for (int e = tid; e < DK * NV; e += NT) {
-            const int c = e / NV, j = e % NV;
+        for (int e = tid; e < DK * NW; e += NT) {
+            const int c = e / NW, j = e % NW;
             p.ds0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] = sm.dS[e];
         }
 }
@@ -565,7 +506,7 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
     using R = Rec<DK>;
     constexpr int LDK = GradSmem<DK>::LDK, LDC = GradSmem<DK>::LDC;
     constexpr int TK = DK / 16;
-    const Pos x = locate(p, blockIdx.x);
+    const packed::Pos x = packed::locate(layout_of(p), blockIdx.x);
     if (!x.ok) return;
     const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
     const int DV = p.DV, H = p.H, L = x.L, h = x.h;
@@ -583,11 +524,11 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
         sm.glm[tid] = rec[R::GLM + tid];
     }
     if (tid < C) sm.beta[tid] = rec[R::BETA + tid];
-    stage(sm.qm, LDK, rec + R::QM, C, DK);
-    stage(sm.km, LDK, rec + R::KM, C, DK);
-    stage(sm.kf, LDK, rec + R::KF, C, DK);
-    stage(sm.MA, LDC, rec + R::MA, C, C);
-    stage(sm.T, LDC, rec + R::T, C, C);
+    stage<C, DK>(sm.qm, LDK, rec + R::QM);
+    stage<C, DK>(sm.km, LDK, rec + R::KM);
+    stage<C, DK>(sm.kf, LDK, rec + R::KF);
+    stage<C, C>(sm.MA, LDC, rec + R::MA);
+    stage<C, C>(sm.T, LDC, rec + R::T);
 
     float aq[4][TK] = {}, ak[4][TK] = {}, an[4][TK] = {};
     float dp[4][4] = {}, dt[4][4] = {};
@@ -726,45 +667,6 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
 
 // ================================================================ host side
 
-// First record of every packed sequence: choff[i] = sum_{j<i} of its chunks
-// (seq_chunks: none for an empty or out-of-range sequence), choff[nseq] = the
-// total.  One CTA; each
-// thread sums a contiguous range of sequences, then a block-wide scan.
-__global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, int nseq, long long tokens,
-                                                             int32_t* choff)
-{
-    __shared__ int warp_tot[32];
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int per = (nseq + 1023) / 1024;
-    const int a = min(nseq, tid * per), b = min(nseq, a + per);
-    int local = 0;
-    for (int i = a; i < b; ++i) local += seq_chunks(cu, i, tokens);
-    int x = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_tot[w] = x;
-    __syncthreads();
-    if (w == 0) {
-        int t = warp_tot[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, t, o);
-            if (lane >= o) t += y;
-        }
-        warp_tot[lane] = t;
-    }
-    __syncthreads();
-    int base = x - local + (w ? warp_tot[w - 1] : 0);
-    for (int i = a; i < b; ++i) {
-        choff[i] = base;
-        base += seq_chunks(cu, i, tokens);
-    }
-    if (tid == 1023) choff[nseq] = base;
-}
-
 // Parts of a call's workspace (byte offsets).
 struct Ws {
     size_t states, rec, U, dU, dY, dSn, choff, bytes;
@@ -776,9 +678,8 @@ static size_t al1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
 static Ws ws_layout(int nseq, int T, long long tokens, int H, int dk, int dv, bool varlen)
 {
     Ws w{};
-    const int nch = (T + C - 1) / C;
-    w.nrec = varlen ? tokens / C + nseq : (long long)nseq * nch;
-    const long long slots = varlen ? tokens / C + 2LL * nseq : (long long)nseq * (nch + 1);
+    w.nrec = packed::records(nseq, T, tokens, varlen);
+    const long long slots = packed::state_slots(nseq, T, tokens, varlen);
     const size_t recf = dk == 128 ? Rec<128>::FLOATS : Rec<64>::FLOATS;
     size_t off = 0;
     w.states = off;
@@ -807,7 +708,7 @@ size_t workspace(int nseq, int T, long long tokens, int H, int dk, int dv, bool 
 template <typename TIn, int DK>
 cudaError_t launch(const void* q, const void* k, const void* v, const Params& p, long long nrec, cudaStream_t stream)
 {
-    const long long walk_ctas = (long long)p.nseq * p.H * (p.DV / NV);
+    const long long walk_ctas = (long long)p.nseq * p.H * (p.DV / NW);
     const long long items = nrec * p.H;
     if (walk_ctas > 0x7fffffffLL || items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     auto kf = bwd_factor_kernel<TIn, DK>;
@@ -893,7 +794,7 @@ cudaError_t chunk_bwd(const void* q, const void* k, const void* v, const float* 
         if (err == cudaSuccess) err = cudaMemsetAsync(dla, 0, th * dkd * 4, stream);
         if (err == cudaSuccess) err = cudaMemsetAsync(dbeta, 0, th * 4, stream);
         if (err == cudaSuccess) {
-            bwd::chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu, nseq, tokens, choff);
+            packed::chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu, nseq, tokens, choff);
             err = cudaGetLastError();
         }
     }

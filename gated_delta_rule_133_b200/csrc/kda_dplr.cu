@@ -15,15 +15,19 @@
 //   O = (e^G q) S + P_qb U + P_qk V
 //   S <- Diag(e^{G_last}) S + (e^{G_last - G} b)^T U + (e^{G_last - G} k)^T V
 //
-// The relative decays are factored around the chunk's middle row m (every
-// factor bounded by the decay of 32 tokens): ax = a e^{Gx - G_m},
-// qx = q e^{G - G_m}, bf = b e^{G_m - G}, kf = k e^{G_m - G}, and the
-// per-channel e^{G_m}, e^{G_last - G_m} are folded into the state products.
-//
-// One CTA (256 threads) per (sequence, head, 16 value columns); columns of S
-// evolve independently (the transition acts on the d_k side).  The operand
-// tiles are retired in two rounds so that everything fits in shared memory.
+// Two launches (plus, for packed batches, the chunk-offset kernel):
+//   1. factors  one CTA per (chunk, head): the intra-chunk products, with the
+//               relative decays factored around the chunk's middle row m so
+//               that every factor is bounded by the decay of 32 tokens
+//               (a e^{Gx - G_m}, q e^{G - G_m}, b e^{G_m - G}, k e^{G_m - G}),
+//               the inverse (I - A_ab)^-1 by forward substitution, and the
+//               state-side factors e^{Gx} a, e^G q, e^{G_last - G} b,
+//               e^{G_last - G} k, stored as one record;
+//   2. walk     one CTA per (sequence, head, 32 value columns; the columns of
+//               S evolve independently, the transition acts on the d_k side)
+//               carries the state through the chunks from the records.
 #include "kda_chunk.cuh"
+#include "kda_packed.cuh"
 
 namespace kda {
 
@@ -32,253 +36,369 @@ namespace dplr {
 using simt::mma_tile;
 
 constexpr int C = 64;
-constexpr int NV = 16;
+constexpr int NW = 32;      // value columns per walk CTA
 constexpr int NT = 256;
 
+// Record of one (chunk, head), in floats: e^{Gx} a, e^G q, e^{G_last - G} b,
+// e^{G_last - G} k [C][DK]; (I - A_ab)^-1, A_ak, P_qb, P_qk [C][C]; e^{G_last} [DK].
 template <int DK>
-struct Smem {
-    static constexpr int LDK = DK + 1;
-    static constexpr int LDC = C + 1;
-    float ax[C * LDK];    // a e^{Gx - G_m}, then q e^{G - G_m}
-    float bf[C * LDK];    // b e^{G_m - G}
-    float kf[C * LDK];    // k e^{G_m - G}
-    float gq[C * LDK];    // cumulative gate G
-    float M1[C * LDC];    // A_ab, then P_qb
-    float M2[C * LDC];    // A_ak, then P_qk
-    float T[C * LDC];     // (I - A_ab)^-1
-    float S[DK * NV];     // state slice
-    float Sm[DK * NV];    // e^{G_m} S
-    float V[C * NV];
-    float W[C * NV];      // (e^{Gx} a) S + A_ak V, then U
-    float O[C * NV];      // (e^G q) S, then the output rows
-    float gm[DK], gam[DK], glm[DK];
+struct Rec {
+    static constexpr int AX = 0, QX = AX + C * DK, BL = QX + C * DK, KL = BL + C * DK;
+    static constexpr int TI = KL + C * DK, AAK = TI + C * C, PQB = AAK + C * C, PQK = PQB + C * C;
+    static constexpr int GAM = PQK + C * C;
+    static constexpr int FLOATS = (GAM + DK + 63) & ~63;
 };
 
-template <typename TIn, typename TOut, int DK>
-__global__ void __launch_bounds__(NT)
-dplr_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
-                const TIn* __restrict__ a, const TIn* __restrict__ b, const float* __restrict__ log_alpha,
-                const float* s0, TOut* __restrict__ o, float* sT, const int32_t* __restrict__ cu, int nseq, int T,
-                long long tokens, int H, int DV)
+struct Params {
+    const float* log_alpha;
+    const float* s0;
+    float* sT;
+    float* rec;
+    packed::Layout lay;
+    int DV;
+};
+
+// Copies a [ROWS][COLS] row-major block from global memory into shared
+// memory with row pitch ld; every load of a thread is issued before its first
+// store (src 16-byte aligned, read-only for the kernel's lifetime).
+template <int ROWS, int COLS>
+__device__ __forceinline__ void stage(float* dst, int ld, const float* src)
+{
+    constexpr int Q4 = COLS / 4, N = ROWS * Q4 / NT;
+    static_assert(ROWS * Q4 % NT == 0, "tile not a multiple of the CTA");
+    float4 x[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int e = threadIdx.x + i * NT;
+        x[i] = __ldg(reinterpret_cast<const float4*>(src + (size_t)(e / Q4) * COLS + 4 * (e % Q4)));
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int e = threadIdx.x + i * NT;
+        float* d = dst + (e / Q4) * ld + 4 * (e % Q4);
+        d[0] = x[i].x;
+        d[1] = x[i].y;
+        d[2] = x[i].z;
+        d[3] = x[i].w;
+    }
+}
+
+// ================================================================ 1. factors
+
+template <int DK>
+struct FacSmem {
+    static constexpr int LDK = DK + 1, LDC = C + 1;
+    float ax[C * LDK];    // a e^{Gx - G_m}
+    float bf[C * LDK];    // b e^{G_m - G}
+    float kf[C * LDK];    // k e^{G_m - G}
+    float qx[C * LDK];    // q e^{G - G_m}
+    float M[C * LDC];     // A_ab
+    float T[C * LDC];     // (I - A_ab)^-1
+};
+
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(NT, 1)
+dplr_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ a,
+                   const TIn* __restrict__ b, const Params p)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    Smem<DK>& sm = *reinterpret_cast<Smem<DK>*>(smem_raw);
-    constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC;
-    constexpr int TK = DK / 16;
-    const int nslice = DV / NV;
-    const int slice = blockIdx.x % nslice;
-    const int h = (blockIdx.x / nslice) % H;
-    const int n = blockIdx.x / (nslice * H);
-    const int col0 = slice * NV;
-    const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
-    int tok0, len;
-    if (cu) {   // a range outside the token axis is skipped (its final state is its initial one)
-        tok0 = cu[n];
-        len = max(0, cu[n + 1] - tok0);
-        if (tok0 < 0 || (long long)tok0 + len > tokens) {
-            if (tid == 0) flag_bad_input();
-            tok0 = 0;
-            len = 0;
-        }
-    } else {
-        tok0 = n * T;
-        len = T;
-    }
-    for (int e = tid; e < DK * NV; e += NT) {
-        const int c = e / NV, j = e % NV;
-        sm.S[e] = s0 ? s0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
-    }
+    FacSmem<DK>& sm = *reinterpret_cast<FacSmem<DK>*>(smem_raw);
+    using R = Rec<DK>;
+    constexpr int LDK = FacSmem<DK>::LDK, LDC = FacSmem<DK>::LDC;
+    const packed::Pos x = packed::locate(p.lay, blockIdx.x);
+    if (!x.ok) return;
+    const int tid = threadIdx.x, H = p.lay.H, L = x.L, h = x.h;
+    float* rec = p.rec + (size_t)blockIdx.x * R::FLOATS;
 
-    for (int t0 = 0; t0 < len; t0 += C) {
-        const int L = min(C, len - t0);
-        __syncthreads();
-        // ---- load (rows >= L are zero: no key, no value, no decay)
-        for (int e = tid; e < C * DK; e += NT) {
-            const int r = e / DK, c = e % DK;
-            float av = 0.f, bv = 0.f, kv = 0.f, gv = 0.f;
-            if (r < L) {
-                const size_t off = ((size_t)(tok0 + t0 + r) * H + h) * DK + c;
-                av = Elem<TIn>::load(a + off);
-                bv = Elem<TIn>::load(b + off);
-                kv = Elem<TIn>::load(k + off);
-                gv = log_alpha[off];
-            }
-            sm.ax[r * LDK + c] = av;
-            sm.bf[r * LDK + c] = bv;
-            sm.kf[r * LDK + c] = kv;
-            sm.gq[r * LDK + c] = gv;
+    // rows >= L are zero: no key, no value, no decay
+    for (int e = tid; e < C * DK; e += NT) {
+        const int r = e / DK, c = e % DK;
+        float av = 0.f, bv = 0.f, kv = 0.f, qv = 0.f;
+        if (r < L) {
+            const size_t off = ((size_t)(x.tok + r) * H + h) * DK + c;
+            av = Elem<TIn>::load(a + off);
+            bv = Elem<TIn>::load(b + off);
+            kv = Elem<TIn>::load(k + off);
+            qv = Elem<TIn>::load(q + off);
         }
-        for (int e = tid; e < C * NV; e += NT) {
-            const int r = e / NV, j = e % NV;
-            sm.V[e] = r < L ? Elem<TIn>::load(v + ((size_t)(tok0 + t0 + r) * H + h) * DV + col0 + j) : 0.f;
-        }
-        __syncthreads();
-        // ---- gate cumsum per channel and the factor split around the middle row
-        if (tid < DK) {
-            const int c = tid;
-            float acc = 0.f;
-            for (int r = 0; r < C; ++r) { acc += sm.gq[r * LDK + c]; sm.gq[r * LDK + c] = acc; }
-            const float Gm = sm.gq[(C / 2 - 1) * LDK + c];
-            sm.gm[c] = expf(Gm);
-            sm.gam[c] = expf(acc);
-            sm.glm[c] = expf(acc - Gm);
-            float gprev = 0.f;   // Gx of row r = G of row r - 1
-            for (int r = 0; r < C; ++r) {
-                const float G = sm.gq[r * LDK + c];
-                const float f = expf(fminf(Gm - G, 80.f));
-                sm.ax[r * LDK + c] *= expf(fminf(gprev - Gm, 80.f));
-                sm.bf[r * LDK + c] *= f;
-                sm.kf[r * LDK + c] *= f;
-                gprev = G;
-            }
-        }
-        __syncthreads();
-        for (int e = tid; e < DK * NV; e += NT) sm.Sm[e] = sm.gm[e / NV] * sm.S[e];
-        // ---- round 1: A_ab, A_ak (strictly lower) and (e^{Gx} a) S = ax Sm
-        {
-            float p1[4][4] = {}, p2[4][4] = {};
-            mma_tile<4, 4>(p1, sm.ax, LDK, 1, sm.bf, 1, LDK, DK, tm, 16, tn, 16);
-            mma_tile<4, 4>(p2, sm.ax, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
+        sm.ax[r * LDK + c] = av;
+        sm.bf[r * LDK + c] = bv;
+        sm.kf[r * LDK + c] = kv;
+        sm.qx[r * LDK + c] = qv;
+    }
+    __syncthreads();
+    if (tid < DK) {   // gate cumsum per channel (fp32, log space), factors and the record's scaled rows
+        const int c = tid;
+        float G[C];
+        float acc = 0.f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int r = tm + 16 * i, s = tn + 16 * j;
-                    sm.M1[r * LDC + s] = s < r ? p1[i][j] : 0.f;
-                    sm.M2[r * LDC + s] = s < r ? p2[i][j] : 0.f;
-                }
+        for (int r = 0; r < C; ++r) {
+            acc += r < L ? p.log_alpha[((size_t)(x.tok + r) * H + h) * DK + c] : 0.f;
+            G[r] = acc;
         }
-        __syncthreads();
-        {
-            float w[4][1] = {};
-            mma_tile<4, 1>(w, sm.ax, LDK, 1, sm.Sm, NV, 1, DK, tm, 16, tn, 16);
-            mma_tile<4, 1>(w, sm.M2, LDC, 1, sm.V, NV, 1, C, tm, 16, tn, 16);
-            __syncthreads();
+        const float Gm = G[C / 2 - 1], Gl = G[C - 1];
+        rec[R::GAM + c] = expf(Gl);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) sm.W[(tm + 16 * i) * NV + tn] = w[i][0];
-        }
-        // ---- T = (I - A_ab)^-1 by forward substitution (column j per 4 lanes)
-        {
-            const int j = tid >> 2, pq = tid & 3;
-            for (int r = 0; r < C; ++r) {
-                float acc = 0.f;
-                if (r > j)
-                    for (int s = j + pq; s < r; s += 4) acc = fmaf(sm.M1[r * LDC + s], sm.T[s * LDC + j], acc);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                if (pq == 0) sm.T[r * LDC + j] = (r == j ? 1.f : 0.f) + (r > j ? acc : 0.f);
-                __syncwarp();
-            }
-        }
-        // ---- reload q as q e^{G - G_m} into ax (ax is retired)
-        __syncthreads();
-        for (int e = tid; e < C * DK; e += NT) {
-            const int r = e / DK, c = e % DK;
-            float qv = 0.f;
-            if (r < L) qv = Elem<TIn>::load(q + ((size_t)(tok0 + t0 + r) * H + h) * DK + c);
-            const float G = sm.gq[r * LDK + c], Gm = sm.gq[(C / 2 - 1) * LDK + c];
-            sm.ax[r * LDK + c] = qv * expf(fminf(G - Gm, 80.f));
-        }
-        __syncthreads();
-        // ---- round 2: P_qb, P_qk (lower incl.), (e^G q) S = qx Sm; U = T W
-        {
-            float p1[4][4] = {}, p2[4][4] = {};
-            mma_tile<4, 4>(p1, sm.ax, LDK, 1, sm.bf, 1, LDK, DK, tm, 16, tn, 16);
-            mma_tile<4, 4>(p2, sm.ax, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
-            float oq[4][1] = {}, u[4][1] = {};
-            mma_tile<4, 1>(oq, sm.ax, LDK, 1, sm.Sm, NV, 1, DK, tm, 16, tn, 16);
-            mma_tile<4, 1>(u, sm.T, LDC, 1, sm.W, NV, 1, C, tm, 16, tn, 16);
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int r = tm + 16 * i, s = tn + 16 * j;
-                    sm.M1[r * LDC + s] = s <= r ? p1[i][j] : 0.f;
-                    sm.M2[r * LDC + s] = s <= r ? p2[i][j] : 0.f;
-                }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                sm.O[(tm + 16 * i) * NV + tn] = oq[i][0];
-                sm.W[(tm + 16 * i) * NV + tn] = u[i][0];
-            }
-        }
-        __syncthreads();
-        // ---- O = (e^G q) S + P_qb U + P_qk V  -> output rows < L
-        {
-            float ov[4][1] = {};
-            mma_tile<4, 1>(ov, sm.M1, LDC, 1, sm.W, NV, 1, C, tm, 16, tn, 16);
-            mma_tile<4, 1>(ov, sm.M2, LDC, 1, sm.V, NV, 1, C, tm, 16, tn, 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = tm + 16 * i;
-                if (r < L)
-                    Elem<TOut>::store(o + ((size_t)(tok0 + t0 + r) * H + h) * DV + col0 + tn,
-                                      sm.O[r * NV + tn] + ov[i][0]);
-            }
-        }
-        // ---- S <- gamma S + e^{G_last - G_m} (bf^T U + kf^T V)
-        {
-            float ds[TK][1] = {};
-            mma_tile<TK, 1>(ds, sm.bf, 1, LDK, sm.W, NV, 1, C, tm, 16, tn, 16);
-            mma_tile<TK, 1>(ds, sm.kf, 1, LDK, sm.V, NV, 1, C, tm, 16, tn, 16);
-#pragma unroll
-            for (int i = 0; i < TK; ++i) {
-                const int c = tm + 16 * i, e = c * NV + tn;
-                sm.S[e] = fmaf(sm.gam[c], sm.S[e], sm.glm[c] * ds[i][0]);
-            }
+        for (int r = 0; r < C; ++r) {
+            const float g = G[r], gx = r ? G[r - 1] : 0.f;
+            const float f = expf(fminf(Gm - g, 80.f));
+            const float av = sm.ax[r * LDK + c], bv = sm.bf[r * LDK + c], kv = sm.kf[r * LDK + c];
+            const float qv = sm.qx[r * LDK + c];
+            sm.ax[r * LDK + c] = av * expf(fminf(gx - Gm, 80.f));
+            sm.bf[r * LDK + c] = bv * f;
+            sm.kf[r * LDK + c] = kv * f;
+            sm.qx[r * LDK + c] = qv * expf(fminf(g - Gm, 80.f));
+            const float el = expf(Gl - g);
+            rec[R::AX + r * DK + c] = av * expf(gx);
+            rec[R::QX + r * DK + c] = qv * expf(g);
+            rec[R::BL + r * DK + c] = bv * el;
+            rec[R::KL + r * DK + c] = kv * el;
         }
     }
     __syncthreads();
-    if (sT)
-        for (int e = tid; e < DK * NV; e += NT) {
-            const int c = e / NV, j = e % NV;
-            sT[(((size_t)n * H + h) * DK + c) * DV + col0 + j] = sm.S[e];
+    const int tn = tid % 16, tm = tid / 16;
+    {   // A_ab (strictly lower) -> M; A_ak (strictly lower) -> the record
+        float p1[4][4] = {}, p2[4][4] = {};
+        mma_tile<4, 4>(p1, sm.ax, LDK, 1, sm.bf, 1, LDK, DK, tm, 16, tn, 16);
+        mma_tile<4, 4>(p2, sm.ax, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = tm + 16 * i, s = tn + 16 * j;
+                sm.M[r * LDC + s] = s < r ? p1[i][j] : 0.f;
+                rec[R::AAK + r * C + s] = s < r ? p2[i][j] : 0.f;
+            }
+    }
+    {   // P_qb, P_qk (lower incl.) -> the record
+        float p1[4][4] = {}, p2[4][4] = {};
+        mma_tile<4, 4>(p1, sm.qx, LDK, 1, sm.bf, 1, LDK, DK, tm, 16, tn, 16);
+        mma_tile<4, 4>(p2, sm.qx, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = tm + 16 * i, s = tn + 16 * j;
+                rec[R::PQB + r * C + s] = s <= r ? p1[i][j] : 0.f;
+                rec[R::PQK + r * C + s] = s <= r ? p2[i][j] : 0.f;
+            }
+    }
+    __syncthreads();
+    {   // T = (I - A_ab)^-1 by forward substitution; 4 lanes share one column
+        const int j = tid >> 2, pq = tid & 3;
+        for (int r = 0; r < C; ++r) {
+            float acc = 0.f;
+            if (r > j)
+                for (int s = j + pq; s < r; s += 4) acc = fmaf(sm.M[r * LDC + s], sm.T[s * LDC + j], acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (pq == 0) sm.T[r * LDC + j] = (r == j ? 1.f : 0.f) + (r > j ? acc : 0.f);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < C * C; e += NT) rec[R::TI + e] = sm.T[(e / C) * LDC + e % C];
+}
+
+// ================================================================ 2. walk
+
+template <int DK>
+struct WalkSmem {
+    static constexpr int LDK = DK + 1, LDC = C + 1;
+    float AX[C * LDK];
+    float QX[C * LDK];
+    float BL[C * LDK];
+    float KL[C * LDK];
+    float TI[C * LDC];
+    float AAK[C * LDC];
+    float PQB[C * LDC];
+    float PQK[C * LDC];
+    float S[DK * NW];     // state slice
+    float V[C * NW];
+    float W[C * NW];      // (e^{Gx} a) S + A_ak V, then U
+    float gam[DK];
+};
+
+template <typename TIn, typename TOut, int DK>
+__global__ void __launch_bounds__(NT, 1)
+dplr_walk_kernel(const TIn* __restrict__ v, TOut* __restrict__ o, const Params p)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    WalkSmem<DK>& sm = *reinterpret_cast<WalkSmem<DK>*>(smem_raw);
+    using R = Rec<DK>;
+    constexpr int LDK = WalkSmem<DK>::LDK, LDC = WalkSmem<DK>::LDC;
+    constexpr int TK = DK / 16;
+    const int DV = p.DV, H = p.lay.H;
+    const int nslice = DV / NW;
+    const int slice = blockIdx.x % nslice;
+    const int h = (blockIdx.x / nslice) % H;
+    const int n = blockIdx.x / (nslice * H);
+    const int col0 = slice * NW;
+    const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
+    const packed::Walk wk = packed::walk_of(p.lay, n, true);   // a skipped sequence keeps its initial state
+
+    for (int e = tid; e < DK * NW; e += NT) {
+        const int c = e / NW, j = e % NW;
+        sm.S[e] = p.s0 ? p.s0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
+    }
+    const int nch = (wk.len + C - 1) / C;
+    for (int ci = 0; ci < nch; ++ci) {
+        const int L = min(C, wk.len - ci * C), tok = wk.tok0 + ci * C;
+        const float* rec = p.rec + ((size_t)(wk.rbase + ci) * H + h) * R::FLOATS;
+        __syncthreads();   // the previous chunk has read every tile
+        stage<C, DK>(sm.AX, LDK, rec + R::AX);
+        stage<C, DK>(sm.QX, LDK, rec + R::QX);
+        stage<C, DK>(sm.BL, LDK, rec + R::BL);
+        stage<C, DK>(sm.KL, LDK, rec + R::KL);
+        stage<C, C>(sm.TI, LDC, rec + R::TI);
+        stage<C, C>(sm.AAK, LDC, rec + R::AAK);
+        stage<C, C>(sm.PQB, LDC, rec + R::PQB);
+        stage<C, C>(sm.PQK, LDC, rec + R::PQK);
+        if (tid < DK) sm.gam[tid] = rec[R::GAM + tid];
+        for (int e = tid; e < C * NW; e += NT) {
+            const int r = e / NW, j = e % NW;
+            sm.V[e] = r < L ? Elem<TIn>::load(v + ((size_t)(tok + r) * H + h) * DV + col0 + j) : 0.f;
+        }
+        __syncthreads();
+        // W = (e^{Gx} a) S + A_ak V;  OQ = (e^G q) S
+        float w[4][2] = {}, oq[4][2] = {};
+        mma_tile<4, 2>(w, sm.AX, LDK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
+        mma_tile<4, 2>(w, sm.AAK, LDC, 1, sm.V, NW, 1, C, tm, 16, tn, 16);
+        mma_tile<4, 2>(oq, sm.QX, LDK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) sm.W[(tm + 16 * i) * NW + tn + 16 * j] = w[i][j];
+        __syncthreads();
+        // U = (I - A_ab)^-1 W
+        float u[4][2] = {};
+        mma_tile<4, 2>(u, sm.TI, LDC, 1, sm.W, NW, 1, C, tm, 16, tn, 16);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) sm.W[(tm + 16 * i) * NW + tn + 16 * j] = u[i][j];
+        __syncthreads();
+        // O = OQ + P_qb U + P_qk V -> rows < L
+        mma_tile<4, 2>(oq, sm.PQB, LDC, 1, sm.W, NW, 1, C, tm, 16, tn, 16);
+        mma_tile<4, 2>(oq, sm.PQK, LDC, 1, sm.V, NW, 1, C, tm, 16, tn, 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = tm + 16 * i;
+            if (r < L)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+                    Elem<TOut>::store(o + ((size_t)(tok + r) * H + h) * DV + col0 + tn + 16 * j, oq[i][j]);
+        }
+        // S <- e^{G_last} S + (e^{G_last - G} b)^T U + (e^{G_last - G} k)^T V
+        float ds[TK][2] = {};
+        mma_tile<TK, 2>(ds, sm.BL, 1, LDK, sm.W, NW, 1, C, tm, 16, tn, 16);
+        mma_tile<TK, 2>(ds, sm.KL, 1, LDK, sm.V, NW, 1, C, tm, 16, tn, 16);
+#pragma unroll
+        for (int i = 0; i < TK; ++i)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
+                sm.S[e] = fmaf(sm.gam[c], sm.S[e], ds[i][j]);
+            }
+    }
+    __syncthreads();
+    if (p.sT)
+        for (int e = tid; e < DK * NW; e += NT) {
+            const int c = e / NW, j = e % NW;
+            p.sT[(((size_t)n * H + h) * DK + c) * DV + col0 + j] = sm.S[e];
         }
 }
 
-template <typename TIn, typename TOut, int DK>
-cudaError_t launch(const void* q, const void* k, const void* v, const void* a, const void* b, const float* la,
-                   const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens, int H,
-                   int dv, cudaStream_t stream)
+// ================================================================ host side
+
+struct Ws {
+    size_t rec, choff, bytes;
+    long long nrec;
+};
+
+static size_t al1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
+
+static Ws ws_layout(int nseq, int T, long long tokens, int H, int dk, bool varlen)
 {
-    const size_t smem = sizeof(Smem<DK>);
-    auto kern = dplr_fwd_kernel<TIn, TOut, DK>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    Ws w{};
+    w.nrec = packed::records(nseq, T, tokens, varlen);
+    const size_t recf = dk == 128 ? Rec<128>::FLOATS : Rec<64>::FLOATS;
+    w.rec = 0;
+    w.choff = al1k((size_t)w.nrec * H * recf * 4);
+    w.bytes = w.choff + (varlen ? al1k(((size_t)nseq + 1) * 4) : 0);
+    return w;
+}
+
+template <typename TIn, typename TOut, int DK>
+cudaError_t launch(const void* q, const void* k, const void* v, const void* a, const void* b, void* o, const Params& p,
+                   long long nrec, cudaStream_t stream)
+{
+    const long long walk_ctas = (long long)p.lay.nseq * p.lay.H * (p.DV / NW);
+    const long long items = nrec * p.lay.H;
+    if (walk_ctas > 0x7fffffffLL || items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    auto kf = dplr_factor_kernel<TIn, DK>;
+    auto kw = dplr_walk_kernel<TIn, TOut, DK>;
+    cudaError_t err = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(FacSmem<DK>));
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(kw, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(WalkSmem<DK>));
     if (err != cudaSuccess) return err;
-    const long long blocks = (long long)nseq * H * (dv / NV);
-    if (blocks == 0) return cudaSuccess;
-    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    kern<<<(unsigned)blocks, NT, smem, stream>>>(
-        static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), static_cast<const TIn*>(a),
-        static_cast<const TIn*>(b), la, s0, static_cast<TOut*>(o), sT, cu, nseq, T, tokens, H, dv);
+    if (walk_ctas == 0) return cudaSuccess;
+    if (items > 0) {
+        kf<<<(unsigned)items, NT, sizeof(FacSmem<DK>), stream>>>(
+            static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(a),
+            static_cast<const TIn*>(b), p);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    kw<<<(unsigned)walk_ctas, NT, sizeof(WalkSmem<DK>), stream>>>(static_cast<const TIn*>(v),
+                                                                   static_cast<TOut*>(o), p);
     return cudaGetLastError();
 }
 
 template <typename TIn, typename TOut>
-cudaError_t launch_dk(const void* q, const void* k, const void* v, const void* a, const void* b, const float* la,
-                      const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens,
-                      int H, int dk, int dv, cudaStream_t s)
+cudaError_t launch_dk(const void* q, const void* k, const void* v, const void* a, const void* b, void* o,
+                      const Params& p, int dk, long long nrec, cudaStream_t s)
 {
-    if (dk == 128) return launch<TIn, TOut, 128>(q, k, v, a, b, la, s0, o, sT, cu, nseq, T, tokens, H, dv, s);
-    if (dk == 64) return launch<TIn, TOut, 64>(q, k, v, a, b, la, s0, o, sT, cu, nseq, T, tokens, H, dv, s);
+    if (dk == 128) return launch<TIn, TOut, 128>(q, k, v, a, b, o, p, nrec, s);
+    if (dk == 64) return launch<TIn, TOut, 64>(q, k, v, a, b, o, p, nrec, s);
     return cudaErrorInvalidValue;
 }
 
 }  // namespace dplr
 
+size_t dplr_fwd_workspace(int nseq, int T, long long tokens, int H, int dk, int dv, bool varlen)
+{
+    (void)dv;
+    return dplr::ws_layout(nseq, T, tokens, H, dk, varlen).bytes;
+}
+
 cudaError_t dplr_fwd(const void* q, const void* k, const void* v, const void* a, const void* b, const float* log_alpha,
                      const float* s0, void* o, float* sT, const int32_t* cu, int nseq, int T, long long tokens, int H,
-                     int dk, int dv, kda_dtype dtype, kda_dtype o_dtype, cudaStream_t s)
+                     int dk, int dv, kda_dtype dtype, kda_dtype o_dtype, void* ws, size_t ws_bytes, cudaStream_t s)
 {
+    const bool varlen = cu != nullptr;
+    const dplr::Ws L = dplr::ws_layout(nseq, T, tokens, H, dk, varlen);
+    if (!ws || ws_bytes < L.bytes) return cudaErrorInvalidValue;
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    int32_t* choff = reinterpret_cast<int32_t*>(w + L.choff);
+    dplr::Params p{};
+    p.log_alpha = log_alpha;
+    p.s0 = s0;
+    p.sT = sT;
+    p.rec = reinterpret_cast<float*>(w + L.rec);
+    p.lay = packed::Layout{cu, varlen ? choff : nullptr, tokens, L.nrec, nseq, T,
+                           varlen ? 0 : (T + dplr::C - 1) / dplr::C, H};
+    p.DV = dv;
+    if (varlen) {
+        packed::chunk_offsets_kernel<<<1, 1024, 0, s>>>(cu, nseq, tokens, choff);
+        const cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
     using bf = __nv_bfloat16;
-    if (dtype == KDA_BF16 && o_dtype == KDA_BF16)
-        return dplr::launch_dk<bf, bf>(q, k, v, a, b, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv, s);
-    if (dtype == KDA_BF16)
-        return dplr::launch_dk<bf, float>(q, k, v, a, b, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv, s);
-    if (o_dtype == KDA_BF16)
-        return dplr::launch_dk<float, bf>(q, k, v, a, b, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv, s);
-    return dplr::launch_dk<float, float>(q, k, v, a, b, log_alpha, s0, o, sT, cu, nseq, T, tokens, H, dk, dv, s);
+    if (dtype == KDA_BF16 && o_dtype == KDA_BF16) return dplr::launch_dk<bf, bf>(q, k, v, a, b, o, p, dk, L.nrec, s);
+    if (dtype == KDA_BF16) return dplr::launch_dk<bf, float>(q, k, v, a, b, o, p, dk, L.nrec, s);
+    if (o_dtype == KDA_BF16) return dplr::launch_dk<float, bf>(q, k, v, a, b, o, p, dk, L.nrec, s);
+    return dplr::launch_dk<float, float>(q, k, v, a, b, o, p, dk, L.nrec, s);
 }
 
 }  // namespace kda

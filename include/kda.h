@@ -309,19 +309,27 @@ kda_status kda_varlen_bwd_workspace_size(int N, int T, int H, int dk, int dv, in
  *
  * (the pages write S_{t-1} (Diag(alpha_t) + a_t b_t^T) + v_t k_t^T for the
  * transposed d_v x d_k state).  With a_t = alpha_t * k_t, b_t = -beta_t k_t and
- * the key beta_t k_t it is the KDA layer.  fp32 arithmetic on CUDA cores; no
- * workspace.
+ * the key beta_t k_t it is the KDA layer.  fp32 arithmetic on CUDA cores.
  *
  *   q, k, a, b  [B, T, H, dk]  dtype;   v [B, T, H, dv]  dtype
  *   log_alpha   [B, T, H, dk]  fp32 (<= 0)
  *   initial_state / final_state [B, H, dk, dv] fp32 or NULL (final may alias initial)
  *   o           [B, T, H, dv]  o_dtype
+ *   workspace   device scratch of at least kda_dplr_fwd_workspace_size() bytes,
+ *               256-byte aligned, owned by the caller, not read across calls
+ *               (one record of chunk factors per (chunk, head)); NULL when
+ *               that size is 0.  Undersized or unaligned: KDA_ERR_INVALID_ARG.
  * d_k, d_v in {64, 128}, chunk 64; pointers 16-byte aligned.
  */
 kda_status kda_dplr_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
                         const float* log_alpha, const float* initial_state, void* o, float* final_state,
                         int B, int T, int H, int dk, int dv, int chunk,
-                        kda_dtype dtype, kda_dtype o_dtype, void* stream);
+                        kda_dtype dtype, kda_dtype o_dtype, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Bytes of workspace kda_dplr_fwd needs for these sizes (0 for empty input). */
+kda_status kda_dplr_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                                       size_t* bytes);
 
 /* The same over N packed variable-length sequences (layouts and boundary
  * rules of kda_varlen_fwd). */
@@ -329,7 +337,11 @@ kda_status kda_dplr_varlen_fwd(const void* q, const void* k, const void* v, cons
                                const float* log_alpha, const int32_t* cu_seqlens, int N,
                                const float* initial_state, void* o, float* final_state,
                                int T, int H, int dk, int dv, int chunk,
-                               kda_dtype dtype, kda_dtype o_dtype, void* stream);
+                               kda_dtype dtype, kda_dtype o_dtype, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+kda_status kda_dplr_varlen_fwd_workspace_size(int N, int T, int H, int dk, int dv, int chunk, kda_dtype dtype,
+                                              size_t* bytes);
 
 /*
  * Synchronises `stream` and reports (then clears) the current device's
