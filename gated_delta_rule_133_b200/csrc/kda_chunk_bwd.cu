@@ -53,14 +53,22 @@ constexpr int NW = 32;      // value columns per walk CTA
 constexpr int NV = 16;      // value columns per pass of the gradient kernel
 constexpr int NT = 256;     // threads per CTA
 
-// Factor record of one (chunk, head), in floats: Q~, K~, K~n, G [C][DK];
-// P, T, MA [C][C]; e^G_m, e^G_last, e^(G_last - G_m) [DK]; beta [C].
+// Factor record of one (chunk, head), in floats, laid out so that each walk
+// streams two contiguous parts (the channel vectors are stored twice):
+//   Q~, K~ [C][DK]; VEC;  P, T [C][C]; K~n [C][DK]; VEC again;  G [C][DK]; MA [C][C]
+// with VEC = e^G_m, e^G_last, e^(G_last - G_m) [DK] and beta [C].
+//   forward walk: part 0 = K~, VEC;          part 1 = T, K~n, VEC
+//   reverse walk: part 0 = P, T, K~n, VEC;   part 1 = Q~, K~, VEC
 template <int DK>
 struct Rec {
-    static constexpr int QM = 0, KM = QM + C * DK, KF = KM + C * DK, G = KF + C * DK;
-    static constexpr int P = G + C * DK, T = P + C * C, MA = T + C * C;
-    static constexpr int GM = MA + C * C, GAM = GM + DK, GLM = GAM + DK, BETA = GLM + DK;
-    static constexpr int FLOATS = (BETA + C + 63) & ~63;
+    static constexpr int VECN = 3 * DK + C;
+    static constexpr int QM = 0, KM = QM + C * DK, VEC = KM + C * DK;
+    static constexpr int GM = VEC, GAM = VEC + DK, GLM = VEC + 2 * DK, BETA = VEC + 3 * DK;
+    static constexpr int P = VEC + VECN, T = P + C * C, KF = T + C * C, VEC2 = KF + C * DK;
+    static constexpr int G = VEC2 + VECN, MA = G + C * DK;
+    static constexpr int FLOATS = (MA + C * C + 63) & ~63;
+    // vector offsets inside a VEC block
+    static constexpr int V_GM = 0, V_GAM = DK, V_GLM = 2 * DK, V_BETA = 3 * DK;
 };
 
 struct Params {
@@ -176,7 +184,8 @@ bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Pa
     if (tid < C) {
         const float b = tid < L ? p.beta[(size_t)(x.tok + tid) * H + h] : 0.f;
         sm.beta[tid] = b;
-        rec[R::BETA + tid] = b;
+        rec[R::VEC + R::V_BETA + tid] = b;
+        rec[R::VEC2 + R::V_BETA + tid] = b;
     }
     __syncthreads();
     if (tid < DK) {   // gate cumsum per channel (fp32, log space) and the factor split
@@ -188,9 +197,12 @@ bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Pa
             rec[R::G + r * DK + c] = acc;
         }
         const float Gm = sm.kf[(C / 2 - 1) * LDK + c];
-        rec[R::GM + c] = expf(Gm);
-        rec[R::GAM + c] = expf(acc);
-        rec[R::GLM + c] = expf(acc - Gm);
+        const float vg[3] = {expf(Gm), expf(acc), expf(acc - Gm)};
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+            rec[R::VEC + u * DK + c] = vg[u];
+            rec[R::VEC2 + u * DK + c] = vg[u];
+        }
         for (int r = 0; r < C; ++r) {
             const float e = fminf(fmaxf(sm.kf[r * LDK + c] - Gm, -80.f), 80.f);
             const float E = expf(e), F = expf(-e);
@@ -239,22 +251,24 @@ bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Pa
 
 // ================================================================ 2. forward walk
 
+// Shared memory of the forward walk: the two streamed record parts
+// (unpadded, as stored), the state slice, e^G_m S, V, Y and U.
 template <int DK>
 struct FwdSmem {
-    static constexpr int LDK = DK + 1, LDC = C + 1;
-    float Kh[C * LDK];    // e^G_m K~
-    float Kl[C * LDK];    // e^(G_last - G_m) K~n
-    float T[C * LDC];
+    using R = Rec<DK>;
+    float p0[C * DK + R::VECN];            // K~, VEC
+    float p1[C * C + C * DK + R::VECN];    // T, K~n, VEC
     float S[DK * NW];     // state slice entering the chunk
+    float Sm[DK * NW];    // e^G_m S
     float V[C * NW];
     float Y[C * NW];
     float U[C * NW];
-    float gm[DK];
-    float glm[DK];
-    float gam[DK];
-    float beta[C];
+    packed::Stream st;
 };
 
+// Per chunk: wait for part 0; X = K~ (e^G_m S), Y = beta (V - X); part 0 of
+// the next chunk is fetched; wait for part 1; U = T Y; S <- gamma S +
+// e^(G_last - G_m) (K~n^T U); part 1 of the next chunk is fetched.
 template <typename TIn, int DK>
 __global__ void __launch_bounds__(NT, 1)
 bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
@@ -262,8 +276,14 @@ bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
     extern __shared__ __align__(16) unsigned char smem_raw[];
     FwdSmem<DK>& sm = *reinterpret_cast<FwdSmem<DK>*>(smem_raw);
     using R = Rec<DK>;
-    constexpr int LDK = FwdSmem<DK>::LDK, LDC = FwdSmem<DK>::LDC;
     constexpr int TK = DK / 16;
+    constexpr int NVR = C * NW / NT;   // V elements per thread
+    constexpr uint32_t B0 = (C * DK + R::VECN) * 4, B1 = (C * C + C * DK + R::VECN) * 4;
+    const float* KM = sm.p0;
+    const float* vec = sm.p0 + C * DK;
+    const float* T = sm.p1;
+    const float* KF = sm.p1 + C * C;
+    const float* vec2 = KF + C * DK;
     const int DV = p.DV, H = p.H;
     const int nslice = DV / NW;
     const int slice = blockIdx.x % nslice;
@@ -274,51 +294,54 @@ bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
 
     const packed::Walk wk = packed::walk_of(layout_of(p), n, true);
     if (!wk.has_slots) return;   // nothing of this sequence is read again
-    const int tok0 = wk.tok0, len = wk.len;
-    const long long sbase = wk.sbase, rbase = wk.rbase;
-    const int nch = (len + C - 1) / C;
+    const int nch = (wk.len + C - 1) / C;
+    auto rec_of = [&](int ci) { return p.rec + ((size_t)(wk.rbase + ci) * H + h) * R::FLOATS; };
+    auto v_at = [&](int ci, int e) {
+        const int r = e / NW, j = e % NW;
+        return ci * C + r < wk.len ? Elem<TIn>::load(v + ((size_t)(wk.tok0 + ci * C + r) * H + h) * DV + col0 + j)
+                                   : 0.f;
+    };
 
+    packed::stream_init(sm.st);
+    if (tid == 0 && nch > 0) {
+        packed::stream_fetch(sm.st, 0, sm.p0, rec_of(0) + R::KM, B0);
+        packed::stream_fetch(sm.st, 1, sm.p1, rec_of(0) + R::T, B1);
+    }
     for (int e = tid; e < DK * NW; e += NT) {
         const int c = e / NW, j = e % NW;
         sm.S[e] = p.s0 ? p.s0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
     }
+    if (nch > 0)
+#pragma unroll
+        for (int i = 0; i < NVR; ++i) sm.V[tid + i * NT] = v_at(0, tid + i * NT);
     __syncthreads();
     for (int ci = 0; ci < nch; ++ci) {
-        const int L = min(C, len - ci * C), tok = tok0 + ci * C;
-        const size_t item = (size_t)(rbase + ci) * H + h;
-        const float* rec = p.rec + item * R::FLOATS;
-        float* st = p.states + ((sbase + ci) * H + h) * (size_t)DK * DV + col0;
+        const size_t item = (size_t)(wk.rbase + ci) * H + h;
+        float* st = p.states + ((wk.sbase + ci) * H + h) * (size_t)DK * DV + col0;
         for (int e = tid; e < DK * NW; e += NT) st[(e / NW) * DV + e % NW] = sm.S[e];
-        if (tid < DK) {
-            sm.gm[tid] = rec[R::GM + tid];
-            sm.glm[tid] = rec[R::GLM + tid];
-            sm.gam[tid] = rec[R::GAM + tid];
-        }
-        if (tid < C) sm.beta[tid] = rec[R::BETA + tid];
-        for (int e = tid; e < C * NW; e += NT) {
-            const int r = e / NW, j = e % NW;
-            sm.V[e] = r < L ? Elem<TIn>::load(v + ((size_t)(tok + r) * H + h) * DV + col0 + j) : 0.f;
-        }
+        if (!packed::stream_wait(sm.st, 0, ci)) goto drain;
+        for (int e = tid; e < DK * NW; e += NT) sm.Sm[e] = vec[R::V_GM + e / NW] * sm.S[e];
         __syncthreads();
-        stage<C, DK>(sm.Kh, LDK, rec + R::KM, sm.gm);
-        stage<C, DK>(sm.Kl, LDK, rec + R::KF, sm.glm);
-        stage<C, C>(sm.T, LDC, rec + R::T);
-        __syncthreads();
-        {   // X = Kh S, Y = beta (V - X)
+        {   // X = K~ Sm, Y = beta (V - X)
             float xx[4][2] = {};
-            mma_tile<4, 2>(xx, sm.Kh, LDK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
+            mma_tile<4, 2>(xx, KM, DK, 1, sm.Sm, NW, 1, DK, tm, 16, tn, 16);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int r = tm + 16 * i, e = r * NW + tn + 16 * j;
-                    sm.Y[e] = sm.beta[r] * (sm.V[e] - xx[i][j]);
+                    sm.Y[e] = vec[R::V_BETA + r] * (sm.V[e] - xx[i][j]);
                 }
         }
-        __syncthreads();
+        __syncthreads();   // part 0 is read
+        if (tid == 0 && ci + 1 < nch) packed::stream_fetch(sm.st, 0, sm.p0, rec_of(ci + 1) + R::KM, B0);
+        if (!packed::stream_wait(sm.st, 1, ci)) goto drain;
+        float vn[NVR];   // next chunk's V, in flight during the arithmetic below
+#pragma unroll
+        for (int i = 0; i < NVR; ++i) vn[i] = ci + 1 < nch ? v_at(ci + 1, tid + i * NT) : 0.f;
         {   // U = T Y
             float u[4][2] = {};
-            mma_tile<4, 2>(u, sm.T, LDC, 1, sm.Y, NW, 1, C, tm, 16, tn, 16);
+            mma_tile<4, 2>(u, T, C, 1, sm.Y, NW, 1, C, tm, 16, tn, 16);
             float* ug = p.U + item * (size_t)C * DV + col0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -330,43 +353,50 @@ bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
                 }
         }
         __syncthreads();
-        {   // S <- gamma S + Kl^T U
+        {   // S <- gamma S + e^(G_last - G_m) (K~n^T U)
             float ds[TK][2] = {};
-            mma_tile<TK, 2>(ds, sm.Kl, 1, LDK, sm.U, NW, 1, C, tm, 16, tn, 16);
+            mma_tile<TK, 2>(ds, KF, 1, DK, sm.U, NW, 1, C, tm, 16, tn, 16);
 #pragma unroll
             for (int i = 0; i < TK; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
-                    sm.S[e] = fmaf(sm.gam[c], sm.S[e], ds[i][j]);
+                    sm.S[e] = fmaf(vec2[R::V_GAM + c], sm.S[e], vec2[R::V_GLM + c] * ds[i][j]);
                 }
         }
+        __syncthreads();   // part 1, V and U are read
+        if (tid == 0 && ci + 1 < nch) packed::stream_fetch(sm.st, 1, sm.p1, rec_of(ci + 1) + R::T, B1);
+#pragma unroll
+        for (int i = 0; i < NVR; ++i) sm.V[tid + i * NT] = vn[i];
         __syncthreads();
     }
-    float* st = p.states + ((sbase + nch) * H + h) * (size_t)DK * DV + col0;
-    for (int e = tid; e < DK * NW; e += NT) st[(e / NW) * DV + e % NW] = sm.S[e];
+    {
+        float* st = p.states + ((wk.sbase + nch) * H + h) * (size_t)DK * DV + col0;
+        for (int e = tid; e < DK * NW; e += NT) st[(e / NW) * DV + e % NW] = sm.S[e];
+    }
+    return;
+drain:
+    packed::stream_drain(sm.st);
 }
 
 // ================================================================ 3. reverse walk
 
 template <int DK>
 struct RevSmem {
-    static constexpr int LDK = DK + 1, LDC = C + 1;
-    float Qh[C * LDK];    // e^G_m Q~
-    float Kh[C * LDK];    // e^G_m K~
-    float Kl[C * LDK];    // e^(G_last - G_m) K~n
-    float P[C * LDC];
-    float T[C * LDC];
+    using R = Rec<DK>;
+    float p0[2 * C * C + C * DK + R::VECN];   // P, T, K~n, VEC
+    float p1[2 * C * DK + R::VECN];           // Q~, K~, VEC
     float dS[DK * NW];    // gradient reaching the state after the chunk, then before it
+    float dSg[DK * NW];   // e^(G_last - G_m) dS'
     float dO[C * NW];
     float dU[C * NW];
-    float dY[C * NW];     // dX = -beta dY
-    float gm[DK];
-    float glm[DK];
-    float gam[DK];
-    float beta[C];
+    float dX[C * NW];     // -beta dY
+    packed::Stream st;
 };
 
+// Per chunk (last to first): wait for part 0; dU = P^T dO + K~n dSg, dY =
+// T^T dU (dv and dX); part 0 of the previous chunk is fetched; wait for part
+// 1; dS <- gamma dS' + e^G_m (Q~^T dO + K~^T dX); part 1 is fetched.
 template <int DK>
 __global__ void __launch_bounds__(NT, 1)
 bwd_reverse_kernel(const Params p)
@@ -374,8 +404,16 @@ bwd_reverse_kernel(const Params p)
     extern __shared__ __align__(16) unsigned char smem_raw[];
     RevSmem<DK>& sm = *reinterpret_cast<RevSmem<DK>*>(smem_raw);
     using R = Rec<DK>;
-    constexpr int LDK = RevSmem<DK>::LDK, LDC = RevSmem<DK>::LDC;
     constexpr int TK = DK / 16;
+    constexpr int NVR = C * NW / NT;
+    constexpr uint32_t B0 = (2 * C * C + C * DK + R::VECN) * 4, B1 = (2 * C * DK + R::VECN) * 4;
+    const float* P = sm.p0;
+    const float* T = sm.p0 + C * C;
+    const float* KF = sm.p0 + 2 * C * C;
+    const float* vec2 = KF + C * DK;
+    const float* QM = sm.p1;
+    const float* KM = sm.p1 + C * DK;
+    const float* vec = sm.p1 + 2 * C * DK;
     const int DV = p.DV, H = p.H;
     const int nslice = DV / NW;
     const int slice = blockIdx.x % nslice;
@@ -386,42 +424,38 @@ bwd_reverse_kernel(const Params p)
 
     // a skipped sequence was reported by the forward walk
     const packed::Walk wk = packed::walk_of(layout_of(p), n, false);
-    const int tok0 = wk.tok0, len = wk.len;
-    const long long rbase = wk.rbase;
-    const int nch = (len + C - 1) / C;
+    const int nch = (wk.len + C - 1) / C;
+    auto rec_of = [&](int ci) { return p.rec + ((size_t)(wk.rbase + ci) * H + h) * R::FLOATS; };
+    auto do_at = [&](int ci, int e) {
+        const int r = e / NW, j = e % NW;
+        return ci * C + r < wk.len ? p.dout[((size_t)(wk.tok0 + ci * C + r) * H + h) * DV + col0 + j] : 0.f;
+    };
 
+    packed::stream_init(sm.st);
+    if (tid == 0 && nch > 0) {
+        packed::stream_fetch(sm.st, 0, sm.p0, rec_of(nch - 1) + R::P, B0);
+        packed::stream_fetch(sm.st, 1, sm.p1, rec_of(nch - 1) + R::QM, B1);
+    }
     for (int e = tid; e < DK * NW; e += NT) {
         const int c = e / NW, j = e % NW;
         sm.dS[e] = p.dsT ? p.dsT[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
     }
+    if (nch > 0)
+#pragma unroll
+        for (int i = 0; i < NVR; ++i) sm.dO[tid + i * NT] = do_at(nch - 1, tid + i * NT);
     __syncthreads();
-    for (int ci = nch - 1; ci >= 0; --ci) {
-        const int L = min(C, len - ci * C), tok = tok0 + ci * C;
-        const size_t item = (size_t)(rbase + ci) * H + h;
-        const float* rec = p.rec + item * R::FLOATS;
+    for (int ci = nch - 1, k = 0; ci >= 0; --ci, ++k) {
+        const int L = min(C, wk.len - ci * C), tok = wk.tok0 + ci * C;
+        const size_t item = (size_t)(wk.rbase + ci) * H + h;
         float* dsn = p.dSn + item * (size_t)DK * DV + col0;
         for (int e = tid; e < DK * NW; e += NT) dsn[(e / NW) * DV + e % NW] = sm.dS[e];
-        if (tid < DK) {
-            sm.gm[tid] = rec[R::GM + tid];
-            sm.glm[tid] = rec[R::GLM + tid];
-            sm.gam[tid] = rec[R::GAM + tid];
-        }
-        if (tid < C) sm.beta[tid] = rec[R::BETA + tid];
-        for (int e = tid; e < C * NW; e += NT) {
-            const int r = e / NW, j = e % NW;
-            sm.dO[e] = r < L ? p.dout[((size_t)(tok + r) * H + h) * DV + col0 + j] : 0.f;
-        }
+        if (!packed::stream_wait(sm.st, 0, k)) goto drain;
+        for (int e = tid; e < DK * NW; e += NT) sm.dSg[e] = vec2[R::V_GLM + e / NW] * sm.dS[e];
         __syncthreads();
-        stage<C, DK>(sm.Qh, LDK, rec + R::QM, sm.gm);
-        stage<C, DK>(sm.Kh, LDK, rec + R::KM, sm.gm);
-        stage<C, DK>(sm.Kl, LDK, rec + R::KF, sm.glm);
-        stage<C, C>(sm.P, LDC, rec + R::P);
-        stage<C, C>(sm.T, LDC, rec + R::T);
-        __syncthreads();
-        {   // dU = P^T dO + Kl dS'
+        {   // dU = P^T dO + K~n dSg
             float du[4][2] = {};
-            mma_tile<4, 2>(du, sm.P, 1, LDC, sm.dO, NW, 1, C, tm, 16, tn, 16);
-            mma_tile<4, 2>(du, sm.Kl, LDK, 1, sm.dS, NW, 1, DK, tm, 16, tn, 16);
+            mma_tile<4, 2>(du, P, 1, C, sm.dO, NW, 1, C, tm, 16, tn, 16);
+            mma_tile<4, 2>(du, KF, DK, 1, sm.dSg, NW, 1, DK, tm, 16, tn, 16);
             float* g = p.dU + item * (size_t)C * DV + col0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -435,32 +469,41 @@ bwd_reverse_kernel(const Params p)
         __syncthreads();
         {   // dY = T^T dU; dv = beta dY; dX = -beta dY
             float dy[4][2] = {};
-            mma_tile<4, 2>(dy, sm.T, 1, LDC, sm.dU, NW, 1, C, tm, 16, tn, 16);
+            mma_tile<4, 2>(dy, T, 1, C, sm.dU, NW, 1, C, tm, 16, tn, 16);
             float* g = p.dY + item * (size_t)C * DV + col0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int r = tm + 16 * i, cc = tn + 16 * j;
-                    const float b = sm.beta[r];
+                    const float b = vec2[R::V_BETA + r];
                     g[(size_t)r * DV + cc] = dy[i][j];
-                    sm.dY[r * NW + cc] = -b * dy[i][j];
+                    sm.dX[r * NW + cc] = -b * dy[i][j];
                     if (r < L) p.dv[((size_t)(tok + r) * H + h) * DV + col0 + cc] = b * dy[i][j];
                 }
         }
-        __syncthreads();
-        {   // dS = diag(gamma) dS' + Qh^T dO + Kh^T dX
+        __syncthreads();   // part 0 is read
+        if (tid == 0 && ci > 0) packed::stream_fetch(sm.st, 0, sm.p0, rec_of(ci - 1) + R::P, B0);
+        if (!packed::stream_wait(sm.st, 1, k)) goto drain;
+        float dn[NVR];   // previous chunk's dO, in flight during the arithmetic below
+#pragma unroll
+        for (int i = 0; i < NVR; ++i) dn[i] = ci > 0 ? do_at(ci - 1, tid + i * NT) : 0.f;
+        {   // dS = gamma dS' + e^G_m (Q~^T dO + K~^T dX)
             float ds[TK][2] = {};
-            mma_tile<TK, 2>(ds, sm.Qh, 1, LDK, sm.dO, NW, 1, C, tm, 16, tn, 16);
-            mma_tile<TK, 2>(ds, sm.Kh, 1, LDK, sm.dY, NW, 1, C, tm, 16, tn, 16);
+            mma_tile<TK, 2>(ds, QM, 1, DK, sm.dO, NW, 1, C, tm, 16, tn, 16);
+            mma_tile<TK, 2>(ds, KM, 1, DK, sm.dX, NW, 1, C, tm, 16, tn, 16);
 #pragma unroll
             for (int i = 0; i < TK; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
-                    sm.dS[e] = fmaf(sm.gam[c], sm.dS[e], ds[i][j]);
+                    sm.dS[e] = fmaf(vec[R::V_GAM + c], sm.dS[e], vec[R::V_GM + c] * ds[i][j]);
                 }
         }
+        __syncthreads();   // part 1 and dO are read
+        if (tid == 0 && ci > 0) packed::stream_fetch(sm.st, 1, sm.p1, rec_of(ci - 1) + R::QM, B1);
+#pragma unroll
+        for (int i = 0; i < NVR; ++i) sm.dO[tid + i * NT] = dn[i];
         __syncthreads();
     }
     if (p.ds0)
@@ -468,6 +511,9 @@ bwd_reverse_kernel(const Params p)
             const int c = e / NW, j = e % NW;
             p.ds0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] = sm.dS[e];
         }
+    return;
+drain:
+    packed::stream_drain(sm.st);
 }
 
 // ================================================================ 4. gradients

@@ -39,14 +39,18 @@ constexpr int C = 64;
 constexpr int NW = 32;      // value columns per walk CTA
 constexpr int NT = 256;
 
-// Record of one (chunk, head), in floats: e^{Gx} a, e^G q, e^{G_last - G} b,
-// e^{G_last - G} k [C][DK]; (I - A_ab)^-1, A_ak, P_qb, P_qk [C][C]; e^{G_last} [DK].
+// Record of one (chunk, head), in floats, as two parts that the walk streams
+// separately: part 1 e^{Gx} a, e^G q [C][DK], (I - A_ab)^-1, A_ak [C][C];
+// part 2 e^{G_last - G} b, e^{G_last - G} k [C][DK], P_qb, P_qk [C][C],
+// e^{G_last} [DK].
 template <int DK>
 struct Rec {
-    static constexpr int AX = 0, QX = AX + C * DK, BL = QX + C * DK, KL = BL + C * DK;
-    static constexpr int TI = KL + C * DK, AAK = TI + C * C, PQB = AAK + C * C, PQK = PQB + C * C;
+    static constexpr int AX = 0, QX = AX + C * DK, TI = QX + C * DK, AAK = TI + C * C;
+    static constexpr int PART2 = AAK + C * C;
+    static constexpr int BL = PART2, KL = BL + C * DK, PQB = KL + C * DK, PQK = PQB + C * C;
     static constexpr int GAM = PQK + C * C;
     static constexpr int FLOATS = (GAM + DK + 63) & ~63;
+    static constexpr uint32_t PART1_BYTES = PART2 * 4u, PART2_BYTES = (GAM + DK - PART2) * 4u;
 };
 
 struct Params {
@@ -57,31 +61,6 @@ struct Params {
     packed::Layout lay;
     int DV;
 };
-
-// Copies a [ROWS][COLS] row-major block from global memory into shared
-// memory with row pitch ld; every load of a thread is issued before its first
-// store (src 16-byte aligned, read-only for the kernel's lifetime).
-template <int ROWS, int COLS>
-__device__ __forceinline__ void stage(float* dst, int ld, const float* src)
-{
-    constexpr int Q4 = COLS / 4, N = ROWS * Q4 / NT;
-    static_assert(ROWS * Q4 % NT == 0, "tile not a multiple of the CTA");
-    float4 x[N];
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-        const int e = threadIdx.x + i * NT;
-        x[i] = __ldg(reinterpret_cast<const float4*>(src + (size_t)(e / Q4) * COLS + 4 * (e % Q4)));
-    }
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-        const int e = threadIdx.x + i * NT;
-        float* d = dst + (e / Q4) * ld + 4 * (e % Q4);
-        d[0] = x[i].x;
-        d[1] = x[i].y;
-        d[2] = x[i].z;
-        d[3] = x[i].w;
-    }
-}
 
 // ================================================================ 1. factors
 
@@ -202,23 +181,22 @@ dplr_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
 
 // ================================================================ 2. walk
 
+// Shared memory of the walk: the two record parts (unpadded, as stored),
+// the state slice, V and W.
 template <int DK>
 struct WalkSmem {
-    static constexpr int LDK = DK + 1, LDC = C + 1;
-    float AX[C * LDK];
-    float QX[C * LDK];
-    float BL[C * LDK];
-    float KL[C * LDK];
-    float TI[C * LDC];
-    float AAK[C * LDC];
-    float PQB[C * LDC];
-    float PQK[C * LDC];
+    float part1[Rec<DK>::PART2];                       // AX, QX, TI, AAK
+    float part2[Rec<DK>::GAM + DK - Rec<DK>::PART2];   // BL, KL, PQB, PQK, e^{G_last}
     float S[DK * NW];     // state slice
     float V[C * NW];
     float W[C * NW];      // (e^{Gx} a) S + A_ak V, then U
-    float gam[DK];
+    packed::Stream st;
 };
 
+// Per chunk: wait for part 1; W = (e^{Gx} a) S + A_ak V and (e^G q) S;
+// U = (I - A_ab)^-1 W; part 1 of the next chunk is fetched; wait for part 2;
+// the output rows and the state update; part 2 of the next chunk is fetched.
+// Each part's copy overlaps the other part's arithmetic.
 template <typename TIn, typename TOut, int DK>
 __global__ void __launch_bounds__(NT, 1)
 dplr_walk_kernel(const TIn* __restrict__ v, TOut* __restrict__ o, const Params p)
@@ -226,8 +204,17 @@ dplr_walk_kernel(const TIn* __restrict__ v, TOut* __restrict__ o, const Params p
     extern __shared__ __align__(16) unsigned char smem_raw[];
     WalkSmem<DK>& sm = *reinterpret_cast<WalkSmem<DK>*>(smem_raw);
     using R = Rec<DK>;
-    constexpr int LDK = WalkSmem<DK>::LDK, LDC = WalkSmem<DK>::LDC;
     constexpr int TK = DK / 16;
+    constexpr int NVR = C * NW / NT;   // V elements per thread
+    const float* AX = sm.part1 + R::AX;
+    const float* QX = sm.part1 + R::QX;
+    const float* TI = sm.part1 + R::TI;
+    const float* AAK = sm.part1 + R::AAK;
+    const float* BL = sm.part2 + (R::BL - R::PART2);
+    const float* KL = sm.part2 + (R::KL - R::PART2);
+    const float* PQB = sm.part2 + (R::PQB - R::PART2);
+    const float* PQK = sm.part2 + (R::PQK - R::PART2);
+    const float* gam = sm.part2 + (R::GAM - R::PART2);
     const int DV = p.DV, H = p.lay.H;
     const int nslice = DV / NW;
     const int slice = blockIdx.x % nslice;
@@ -236,35 +223,34 @@ dplr_walk_kernel(const TIn* __restrict__ v, TOut* __restrict__ o, const Params p
     const int col0 = slice * NW;
     const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
     const packed::Walk wk = packed::walk_of(p.lay, n, true);   // a skipped sequence keeps its initial state
+    const int nch = (wk.len + C - 1) / C;
+    auto rec_of = [&](int ci) { return p.rec + ((size_t)(wk.rbase + ci) * H + h) * R::FLOATS; };
+    auto v_at = [&](int ci, int e) {   // element e of chunk ci's V slice (0 past the sequence)
+        const int r = e / NW, j = e % NW;
+        return ci * C + r < wk.len ? Elem<TIn>::load(v + ((size_t)(wk.tok0 + ci * C + r) * H + h) * DV + col0 + j)
+                                   : 0.f;
+    };
 
+    packed::stream_init(sm.st);
+    if (tid == 0 && nch > 0) {
+        packed::stream_fetch(sm.st, 0, sm.part1, rec_of(0), R::PART1_BYTES);
+        packed::stream_fetch(sm.st, 1, sm.part2, rec_of(0) + R::PART2, R::PART2_BYTES);
+    }
     for (int e = tid; e < DK * NW; e += NT) {
         const int c = e / NW, j = e % NW;
         sm.S[e] = p.s0 ? p.s0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
     }
-    const int nch = (wk.len + C - 1) / C;
+    if (nch > 0)
+#pragma unroll
+        for (int i = 0; i < NVR; ++i) sm.V[tid + i * NT] = v_at(0, tid + i * NT);
     for (int ci = 0; ci < nch; ++ci) {
         const int L = min(C, wk.len - ci * C), tok = wk.tok0 + ci * C;
-        const float* rec = p.rec + ((size_t)(wk.rbase + ci) * H + h) * R::FLOATS;
-        __syncthreads();   // the previous chunk has read every tile
-        stage<C, DK>(sm.AX, LDK, rec + R::AX);
-        stage<C, DK>(sm.QX, LDK, rec + R::QX);
-        stage<C, DK>(sm.BL, LDK, rec + R::BL);
-        stage<C, DK>(sm.KL, LDK, rec + R::KL);
-        stage<C, C>(sm.TI, LDC, rec + R::TI);
-        stage<C, C>(sm.AAK, LDC, rec + R::AAK);
-        stage<C, C>(sm.PQB, LDC, rec + R::PQB);
-        stage<C, C>(sm.PQK, LDC, rec + R::PQK);
-        if (tid < DK) sm.gam[tid] = rec[R::GAM + tid];
-        for (int e = tid; e < C * NW; e += NT) {
-            const int r = e / NW, j = e % NW;
-            sm.V[e] = r < L ? Elem<TIn>::load(v + ((size_t)(tok + r) * H + h) * DV + col0 + j) : 0.f;
-        }
-        __syncthreads();
+        if (!packed::stream_wait(sm.st, 0, ci)) goto drain;   // also orders S and V
         // W = (e^{Gx} a) S + A_ak V;  OQ = (e^G q) S
         float w[4][2] = {}, oq[4][2] = {};
-        mma_tile<4, 2>(w, sm.AX, LDK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
-        mma_tile<4, 2>(w, sm.AAK, LDC, 1, sm.V, NW, 1, C, tm, 16, tn, 16);
-        mma_tile<4, 2>(oq, sm.QX, LDK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
+        mma_tile<4, 2>(w, AX, DK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
+        mma_tile<4, 2>(w, AAK, C, 1, sm.V, NW, 1, C, tm, 16, tn, 16);
+        mma_tile<4, 2>(oq, QX, DK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -272,16 +258,20 @@ dplr_walk_kernel(const TIn* __restrict__ v, TOut* __restrict__ o, const Params p
         __syncthreads();
         // U = (I - A_ab)^-1 W
         float u[4][2] = {};
-        mma_tile<4, 2>(u, sm.TI, LDC, 1, sm.W, NW, 1, C, tm, 16, tn, 16);
-        __syncthreads();
+        mma_tile<4, 2>(u, TI, C, 1, sm.W, NW, 1, C, tm, 16, tn, 16);
+        __syncthreads();   // part 1 and W are read
+        if (tid == 0 && ci + 1 < nch) packed::stream_fetch(sm.st, 0, sm.part1, rec_of(ci + 1), R::PART1_BYTES);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 2; ++j) sm.W[(tm + 16 * i) * NW + tn + 16 * j] = u[i][j];
-        __syncthreads();
+        if (!packed::stream_wait(sm.st, 1, ci)) goto drain;   // also orders U
+        float vn[NVR];   // next chunk's V, in flight during the arithmetic below
+#pragma unroll
+        for (int i = 0; i < NVR; ++i) vn[i] = ci + 1 < nch ? v_at(ci + 1, tid + i * NT) : 0.f;
         // O = OQ + P_qb U + P_qk V -> rows < L
-        mma_tile<4, 2>(oq, sm.PQB, LDC, 1, sm.W, NW, 1, C, tm, 16, tn, 16);
-        mma_tile<4, 2>(oq, sm.PQK, LDC, 1, sm.V, NW, 1, C, tm, 16, tn, 16);
+        mma_tile<4, 2>(oq, PQB, C, 1, sm.W, NW, 1, C, tm, 16, tn, 16);
+        mma_tile<4, 2>(oq, PQK, C, 1, sm.V, NW, 1, C, tm, 16, tn, 16);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = tm + 16 * i;
@@ -291,16 +281,23 @@ dplr_walk_kernel(const TIn* __restrict__ v, TOut* __restrict__ o, const Params p
                     Elem<TOut>::store(o + ((size_t)(tok + r) * H + h) * DV + col0 + tn + 16 * j, oq[i][j]);
         }
         // S <- e^{G_last} S + (e^{G_last - G} b)^T U + (e^{G_last - G} k)^T V
-        float ds[TK][2] = {};
-        mma_tile<TK, 2>(ds, sm.BL, 1, LDK, sm.W, NW, 1, C, tm, 16, tn, 16);
-        mma_tile<TK, 2>(ds, sm.KL, 1, LDK, sm.V, NW, 1, C, tm, 16, tn, 16);
+        {
+            float ds[TK][2] = {};
+            mma_tile<TK, 2>(ds, BL, 1, DK, sm.W, NW, 1, C, tm, 16, tn, 16);
+            mma_tile<TK, 2>(ds, KL, 1, DK, sm.V, NW, 1, C, tm, 16, tn, 16);
 #pragma unroll
-        for (int i = 0; i < TK; ++i)
+            for (int i = 0; i < TK; ++i)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
-                sm.S[e] = fmaf(sm.gam[c], sm.S[e], ds[i][j]);
-            }
+                for (int j = 0; j < 2; ++j) {
+                    const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
+                    sm.S[e] = fmaf(gam[c], sm.S[e], ds[i][j]);
+                }
+        }
+        __syncthreads();   // part 2, V and U are read
+        if (tid == 0 && ci + 1 < nch)
+            packed::stream_fetch(sm.st, 1, sm.part2, rec_of(ci + 1) + R::PART2, R::PART2_BYTES);
+#pragma unroll
+        for (int i = 0; i < NVR; ++i) sm.V[tid + i * NT] = vn[i];
     }
     __syncthreads();
     if (p.sT)
@@ -308,6 +305,9 @@ dplr_walk_kernel(const TIn* __restrict__ v, TOut* __restrict__ o, const Params p
             const int c = e / NW, j = e % NW;
             p.sT[(((size_t)n * H + h) * DK + c) * DV + col0 + j] = sm.S[e];
         }
+    return;
+drain:
+    packed::stream_drain(sm.st);
 }
 
 // ================================================================ host side

@@ -10,6 +10,7 @@
 #pragma once
 
 #include "kda_common.cuh"
+#include "kda_sm100.cuh"
 
 namespace kda {
 
@@ -157,6 +158,70 @@ __device__ __forceinline__ Walk walk_of(const Layout& g, int n, bool report)
         w.sbase = (long long)n * (g.nch + 1);
     }
     return w;
+}
+
+// Record streaming: bulk copies of record parts into shared memory that
+// complete on an mbarrier (one phase per fetch), waited for with a bound.
+constexpr long long kWaitCycles = 1LL << 31;   // about 1 s at the B200 clock
+
+// One thread: copies `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) in pieces of at most 32 KB, all completing on `bar`.  The fence
+// orders this CTA's earlier generic accesses of dst before the async writes.
+__device__ __forceinline__ void fetch(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    sm100::fence_proxy_async();
+    sm100::mbar_expect_tx(bar, bytes);
+    for (uint32_t off = 0; off < bytes; off += 32768u)
+        sm100::bulk_load(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off,
+                         min(32768u, bytes - off), bar);
+}
+
+// Per-CTA state of up to two streamed parts.  issued[i] / done[i] count the
+// fetches of part i that were issued / seen complete by thread 0.
+struct Stream {
+    uint64_t bar[2];
+    int issued[2], done[2];
+    int abort;
+};
+
+__device__ __forceinline__ void stream_init(Stream& st)
+{
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&st.bar[0], 1);
+        sm100::mbar_init(&st.bar[1], 1);
+        st.issued[0] = st.issued[1] = st.done[0] = st.done[1] = 0;
+        st.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void stream_fetch(Stream& st, int i, void* dst, const void* src, uint32_t bytes)
+{
+    fetch(dst, src, bytes, &st.bar[i]);
+    ++st.issued[i];
+}
+
+// Every thread waits for fetch number `k` (0-based) of part i; returns false
+// for every thread of the CTA if any thread's wait ran out (status word set).
+__device__ __forceinline__ bool stream_wait(Stream& st, int i, int k)
+{
+    const bool ok = sm100::mbar_wait(&st.bar[i], (uint32_t)(k & 1), &st.abort, kWaitCycles);
+    if (threadIdx.x == 0 && ok) st.done[i] = k + 1;
+    return !__syncthreads_or(!ok);
+}
+
+// After a failed wait: thread 0 waits (bounded again) for the copies still in
+// flight, so that none lands in shared memory after the CTA has exited.
+__device__ __forceinline__ void stream_drain(Stream& st)
+{
+    if (threadIdx.x == 0) {
+        volatile int never = 0;
+        for (int i = 0; i < 2; ++i)
+            for (int k = st.done[i]; k < st.issued[i]; ++k)
+                if (!sm100::mbar_wait(&st.bar[i], (uint32_t)(k & 1), &never, kWaitCycles)) break;
+    }
+    __syncthreads();
 }
 
 }  // namespace packed
