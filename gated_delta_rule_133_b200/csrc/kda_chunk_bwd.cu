@@ -168,18 +168,11 @@ bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Pa
     const int tid = threadIdx.x, H = p.H, L = x.L, h = x.h;
     float* rec = p.rec + (size_t)blockIdx.x * R::FLOATS;
 
-    for (int e = tid; e < C * DK; e += NT) {
-        const int r = e / DK, c = e % DK;
-        float qv = 0.f, kv = 0.f, gv = 0.f;
-        if (r < L) {
-            const size_t off = ((size_t)(x.tok + r) * H + h) * DK + c;
-            qv = Elem<TIn>::load(q + off);
-            kv = Elem<TIn>::load(k + off);
-            gv = p.log_alpha[off];
-        }
-        sm.qm[r * LDK + c] = qv;
-        sm.km[r * LDK + c] = kv;
-        sm.kf[r * LDK + c] = gv;
+    {
+        const size_t row0 = ((size_t)x.tok * H + h) * DK, stride = (size_t)H * DK;
+        packed::load_rows<TIn, DK, NT>(sm.qm, LDK, q + row0, stride, L);
+        packed::load_rows<TIn, DK, NT>(sm.km, LDK, k + row0, stride, L);
+        packed::load_rows<float, DK, NT>(sm.kf, LDK, p.log_alpha + row0, stride, L);
     }
     if (tid < C) {
         const float b = tid < L ? p.beta[(size_t)(x.tok + tid) * H + h] : 0.f;
@@ -535,6 +528,7 @@ struct GradSmem {
     float U[C * NV];
     float dU[C * NV];
     float Y[C * NV];      // beta (V - X)
+    float dY[C * NV];
     float dX[C * NV];     // -beta dY
     float gm[DK];
     float glm[DK];
@@ -579,29 +573,61 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
     float aq[4][TK] = {}, ak[4][TK] = {}, an[4][TK] = {};
     float dp[4][4] = {}, dt[4][4] = {};
     float db1[4] = {0.f, 0.f, 0.f, 0.f};
-    float dgl[TK] = {};   // channel tm + 16 i, summed over this thread's columns
+    // pass loads: thread tid holds float4 number tid + i NT of each [DK][16]
+    // slice (channel (tid + i NT) / 4) and float4 number tid of each [C][16]
+    // slice (row tid / 4); all are issued before the first store
+    constexpr int NS = DK * NV / 4 / NT;              // float4 per thread of a [DK][16] slice
+    constexpr int EPV = 16 / (int)sizeof(TIn), VPR = NV / EPV;
+    static_assert(C * NV / 4 == NT, "one float4 of a [C][16] slice per thread");
+    float dgl[NS] = {};   // channel (tid + i NT) / 4, summed over this thread's columns
+    const int rr = tid / 4, c4 = 4 * (tid % 4);
+    const bool rin = rr < L;
+    const size_t rowg = ((size_t)(x.tok + rr) * H + h) * DV;
     for (int j0 = 0; j0 < DV; j0 += NV) {
-        __syncthreads();   // the previous pass has read its slices (first pass: the vectors are in place)
-        for (int e = tid; e < DK * NV; e += NT) {
-            const int c = e / NV, j = e % NV;
-            const size_t g = (size_t)c * DV + j0 + j;
-            sm.Sm[e] = sm.gm[c] * S0[g];
-            sm.dSg[e] = sm.glm[c] * dS1[g];
-        }
+        float4 s0[NS], d1[NS], s1[NS];
 #pragma unroll
-        for (int i = 0; i < TK; ++i) {   // thread (tm, tn): channel tm + 16 i, column tn
-            const size_t g = (size_t)(tm + 16 * i) * DV + j0 + tn;
-            dgl[i] = fmaf(dS1[g], S1[g], dgl[i]);
+        for (int i = 0; i < NS; ++i) {
+            const int e = tid + i * NT;
+            const size_t g = (size_t)(e / 4) * DV + j0 + 4 * (e % 4);
+            s0[i] = __ldg(reinterpret_cast<const float4*>(S0 + g));
+            d1[i] = __ldg(reinterpret_cast<const float4*>(dS1 + g));
+            s1[i] = __ldg(reinterpret_cast<const float4*>(S1 + g));
         }
-        for (int e = tid; e < C * NV; e += NT) {
-            const int r = e / NV, j = e % NV;
-            const size_t g = (size_t)r * DV + j0 + j;
-            const bool in = r < L;
-            sm.VX[e] = in ? Elem<TIn>::load(v + ((size_t)(x.tok + r) * H + h) * DV + j0 + j) : 0.f;
-            sm.dO[e] = in ? p.dout[((size_t)(x.tok + r) * H + h) * DV + j0 + j] : 0.f;
-            sm.U[e] = Ug[g];
-            sm.dU[e] = dUg[g];
-            sm.dX[e] = -sm.beta[r] * dYg[g];
+        const size_t g = (size_t)rr * DV + j0 + c4;
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 o4 = rin ? __ldg(reinterpret_cast<const float4*>(p.dout + rowg + j0 + c4)) : z4;
+        const float4 u4 = __ldg(reinterpret_cast<const float4*>(Ug + g));
+        const float4 du4 = __ldg(reinterpret_cast<const float4*>(dUg + g));
+        const float4 dy4 = __ldg(reinterpret_cast<const float4*>(dYg + g));
+        uint4 vv = make_uint4(0u, 0u, 0u, 0u);
+        const int vr = tid / VPR;
+        if (tid < C * VPR && vr < L)
+            vv = __ldg(reinterpret_cast<const uint4*>(v + ((size_t)(x.tok + vr) * H + h) * DV + j0 + (tid % VPR) * EPV));
+        __syncthreads();   // the previous pass has read its slices (first pass: the vectors are in place)
+#pragma unroll
+        for (int i = 0; i < NS; ++i) {
+            const int e = tid + i * NT, c = e / 4;
+            const float gmc = sm.gm[c], glc = sm.glm[c];
+            float* sm4 = sm.Sm + 4 * e;
+            float* dg4 = sm.dSg + 4 * e;
+            sm4[0] = gmc * s0[i].x; sm4[1] = gmc * s0[i].y; sm4[2] = gmc * s0[i].z; sm4[3] = gmc * s0[i].w;
+            dg4[0] = glc * d1[i].x; dg4[1] = glc * d1[i].y; dg4[2] = glc * d1[i].z; dg4[3] = glc * d1[i].w;
+            dgl[i] += d1[i].x * s1[i].x + d1[i].y * s1[i].y + d1[i].z * s1[i].z + d1[i].w * s1[i].w;
+        }
+        {
+            const int e = rr * NV + c4;
+            const float b = sm.beta[rr];
+            *reinterpret_cast<float4*>(sm.dO + e) = o4;
+            *reinterpret_cast<float4*>(sm.U + e) = u4;
+            *reinterpret_cast<float4*>(sm.dU + e) = du4;
+            *reinterpret_cast<float4*>(sm.dY + e) = dy4;
+            *reinterpret_cast<float4*>(sm.dX + e) = make_float4(-b * dy4.x, -b * dy4.y, -b * dy4.z, -b * dy4.w);
+            if (tid < C * VPR) {
+                const TIn* xv = reinterpret_cast<const TIn*>(&vv);
+                float* d = sm.VX + vr * NV + (tid % VPR) * EPV;
+#pragma unroll
+                for (int u = 0; u < EPV; ++u) d[u] = Elem<TIn>::load(xv + u);
+            }
         }
         __syncthreads();
         {   // X = K~ (e^G_m S); V - X; Y = beta (V - X); rowsum((V - X) dY)
@@ -613,7 +639,7 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
                 const float vx = sm.VX[e] - xx[i][0];
                 sm.VX[e] = vx;
                 sm.Y[e] = sm.beta[r] * vx;
-                db1[i] = fmaf(vx, dYg[(size_t)r * DV + j0 + tn], db1[i]);
+                db1[i] = fmaf(vx, sm.dY[e], db1[i]);
             }
         }
         __syncthreads();
@@ -638,9 +664,11 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
         if (tn == 0) sm.db[r] = b;
     }
 #pragma unroll
-    for (int i = 0; i < TK; ++i) {
-        const float g = sum16(dgl[i]);
-        if (tn == 0) sm.dgl[tm + 16 * i] = g;
+    for (int i = 0; i < NS; ++i) {   // the 4 threads of a channel are consecutive lanes
+        float g = dgl[i];
+        g += __shfl_xor_sync(0xffffffffu, g, 1);
+        g += __shfl_xor_sync(0xffffffffu, g, 2);
+        if ((tid & 3) == 0) sm.dgl[(tid + i * NT) / 4] = g;
     }
     __syncthreads();
     // a_q += dP K~n; a_n += dP^T Q~

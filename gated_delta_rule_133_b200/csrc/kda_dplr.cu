@@ -90,20 +90,12 @@ dplr_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
     float* rec = p.rec + (size_t)blockIdx.x * R::FLOATS;
 
     // rows >= L are zero: no key, no value, no decay
-    for (int e = tid; e < C * DK; e += NT) {
-        const int r = e / DK, c = e % DK;
-        float av = 0.f, bv = 0.f, kv = 0.f, qv = 0.f;
-        if (r < L) {
-            const size_t off = ((size_t)(x.tok + r) * H + h) * DK + c;
-            av = Elem<TIn>::load(a + off);
-            bv = Elem<TIn>::load(b + off);
-            kv = Elem<TIn>::load(k + off);
-            qv = Elem<TIn>::load(q + off);
-        }
-        sm.ax[r * LDK + c] = av;
-        sm.bf[r * LDK + c] = bv;
-        sm.kf[r * LDK + c] = kv;
-        sm.qx[r * LDK + c] = qv;
+    {
+        const size_t row0 = ((size_t)x.tok * H + h) * DK, stride = (size_t)H * DK;
+        packed::load_rows<TIn, DK, NT>(sm.ax, LDK, a + row0, stride, L);
+        packed::load_rows<TIn, DK, NT>(sm.bf, LDK, b + row0, stride, L);
+        packed::load_rows<TIn, DK, NT>(sm.kf, LDK, k + row0, stride, L);
+        packed::load_rows<TIn, DK, NT>(sm.qx, LDK, q + row0, stride, L);
     }
     __syncthreads();
     if (tid < DK) {   // gate cumsum per channel (fp32, log space), factors and the record's scaled rows

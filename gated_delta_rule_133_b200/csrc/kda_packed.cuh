@@ -160,6 +160,34 @@ __device__ __forceinline__ Walk walk_of(const Layout& g, int n, bool report)
     return w;
 }
 
+// Loads rows [0, L) of a [64][D] tile of TIn elements (row r at
+// src + r * stride elements, rows 16-byte aligned) into shared memory as
+// floats with row pitch ld; rows >= L become zero.  Every load of a thread is
+// issued before its first store.  NTHR threads take part.
+template <typename TIn, int D, int NTHR>
+__device__ __forceinline__ void load_rows(float* dst, int ld, const TIn* src, size_t stride, int L)
+{
+    constexpr int EPV = 16 / (int)sizeof(TIn);   // elements per 16-byte vector
+    constexpr int VPR = D / EPV;                 // vectors per row
+    constexpr int N = C * VPR / NTHR;            // vectors per thread
+    static_assert(C * VPR % NTHR == 0, "tile not a multiple of the CTA");
+    uint4 x[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int e = threadIdx.x + i * NTHR, r = e / VPR;
+        x[i] = r < L ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * stride + (e % VPR) * EPV))
+                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int e = threadIdx.x + i * NTHR;
+        float* d = dst + (e / VPR) * ld + (e % VPR) * EPV;
+        const TIn* xv = reinterpret_cast<const TIn*>(&x[i]);
+#pragma unroll
+        for (int u = 0; u < EPV; ++u) d[u] = Elem<TIn>::load(xv + u);
+    }
+}
+
 // Record streaming: bulk copies of record parts into shared memory that
 // complete on an mbarrier (one phase per fetch), waited for with a bound.
 constexpr long long kWaitCycles = 1LL << 31;   // about 1 s at the B200 clock
