@@ -513,7 +513,9 @@ drain:
 
 template <int DK>
 struct GradSmem {
-    static constexpr int LDK = DK + 1, LDC = C + 1;
+    // NVP: padded pitch of the [*][16] pass tiles, which the products also
+    // read down their columns
+    static constexpr int LDK = DK + 1, LDC = C + 1, NVP = NV + 1;
     float qm[C * LDK];    // Q~, then dG
     float km[C * LDK];    // K~
     float kf[C * LDK];    // K~n
@@ -521,15 +523,15 @@ struct GradSmem {
     float T[C * LDC];
     float D1[C * LDC];    // dP, then T^T dT
     float D2[C * LDC];    // dT, then dMA
-    float Sm[DK * NV];    // e^G_m S (value columns of this pass)
-    float dSg[DK * NV];   // e^(G_last - G_m) dS'
-    float VX[C * NV];     // V, then V - X
-    float dO[C * NV];
-    float U[C * NV];
-    float dU[C * NV];
-    float Y[C * NV];      // beta (V - X)
-    float dY[C * NV];
-    float dX[C * NV];     // -beta dY
+    float Sm[DK * NVP];    // e^G_m S (value columns of this pass)
+    float dSg[DK * NVP];   // e^(G_last - G_m) dS'
+    float VX[C * NVP];     // V, then V - X
+    float dO[C * NVP];
+    float U[C * NVP];
+    float dU[C * NVP];
+    float Y[C * NVP];      // beta (V - X)
+    float dY[C * NVP];
+    float dX[C * NVP];     // -beta dY
     float gm[DK];
     float glm[DK];
     float dgl[DK];        // rowsum(dS' S'): the last row's extra dG
@@ -544,7 +546,7 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
     extern __shared__ __align__(16) unsigned char smem_raw[];
     GradSmem<DK>& sm = *reinterpret_cast<GradSmem<DK>*>(smem_raw);
     using R = Rec<DK>;
-    constexpr int LDK = GradSmem<DK>::LDK, LDC = GradSmem<DK>::LDC;
+    constexpr int LDK = GradSmem<DK>::LDK, LDC = GradSmem<DK>::LDC, NVP = GradSmem<DK>::NVP;
     constexpr int TK = DK / 16;
     const packed::Pos x = packed::locate(layout_of(p), blockIdx.x);
     if (!x.ok) return;
@@ -608,23 +610,29 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
         for (int i = 0; i < NS; ++i) {
             const int e = tid + i * NT, c = e / 4;
             const float gmc = sm.gm[c], glc = sm.glm[c];
-            float* sm4 = sm.Sm + 4 * e;
-            float* dg4 = sm.dSg + 4 * e;
+            float* sm4 = sm.Sm + c * NVP + 4 * (e % 4);
+            float* dg4 = sm.dSg + c * NVP + 4 * (e % 4);
             sm4[0] = gmc * s0[i].x; sm4[1] = gmc * s0[i].y; sm4[2] = gmc * s0[i].z; sm4[3] = gmc * s0[i].w;
             dg4[0] = glc * d1[i].x; dg4[1] = glc * d1[i].y; dg4[2] = glc * d1[i].z; dg4[3] = glc * d1[i].w;
             dgl[i] += d1[i].x * s1[i].x + d1[i].y * s1[i].y + d1[i].z * s1[i].z + d1[i].w * s1[i].w;
         }
         {
-            const int e = rr * NV + c4;
+            const int e = rr * NVP + c4;
             const float b = sm.beta[rr];
-            *reinterpret_cast<float4*>(sm.dO + e) = o4;
-            *reinterpret_cast<float4*>(sm.U + e) = u4;
-            *reinterpret_cast<float4*>(sm.dU + e) = du4;
-            *reinterpret_cast<float4*>(sm.dY + e) = dy4;
-            *reinterpret_cast<float4*>(sm.dX + e) = make_float4(-b * dy4.x, -b * dy4.y, -b * dy4.z, -b * dy4.w);
+            auto put = [&](float* t, const float4& x4) {
+                t[e] = x4.x;
+                t[e + 1] = x4.y;
+                t[e + 2] = x4.z;
+                t[e + 3] = x4.w;
+            };
+            put(sm.dO, o4);
+            put(sm.U, u4);
+            put(sm.dU, du4);
+            put(sm.dY, dy4);
+            put(sm.dX, make_float4(-b * dy4.x, -b * dy4.y, -b * dy4.z, -b * dy4.w));
             if (tid < C * VPR) {
                 const TIn* xv = reinterpret_cast<const TIn*>(&vv);
-                float* d = sm.VX + vr * NV + (tid % VPR) * EPV;
+                float* d = sm.VX + vr * NVP + (tid % VPR) * EPV;
 #pragma unroll
                 for (int u = 0; u < EPV; ++u) d[u] = Elem<TIn>::load(xv + u);
             }
@@ -632,10 +640,10 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
         __syncthreads();
         {   // X = K~ (e^G_m S); V - X; Y = beta (V - X); rowsum((V - X) dY)
             float xx[4][1] = {};
-            mma_tile<4, 1>(xx, sm.km, LDK, 1, sm.Sm, NV, 1, DK, tm, 16, tn, 16);
+            mma_tile<4, 1>(xx, sm.km, LDK, 1, sm.Sm, NVP, 1, DK, tm, 16, tn, 16);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int r = tm + 16 * i, e = r * NV + tn;
+                const int r = tm + 16 * i, e = r * NVP + tn;
                 const float vx = sm.VX[e] - xx[i][0];
                 sm.VX[e] = vx;
                 sm.Y[e] = sm.beta[r] * vx;
@@ -644,11 +652,11 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
         }
         __syncthreads();
         // a_q += dO Sm^T, a_k += dX Sm^T, a_n += U dSg^T; dP += dO U^T, dT += dU Y^T
-        mma_tile<4, TK>(aq, sm.dO, NV, 1, sm.Sm, 1, NV, NV, tm, 16, tn, 16);
-        mma_tile<4, TK>(ak, sm.dX, NV, 1, sm.Sm, 1, NV, NV, tm, 16, tn, 16);
-        mma_tile<4, TK>(an, sm.U, NV, 1, sm.dSg, 1, NV, NV, tm, 16, tn, 16);
-        mma_tile<4, 4>(dp, sm.dO, NV, 1, sm.U, 1, NV, NV, tm, 16, tn, 16);
-        mma_tile<4, 4>(dt, sm.dU, NV, 1, sm.Y, 1, NV, NV, tm, 16, tn, 16);
+        mma_tile<4, TK>(aq, sm.dO, NVP, 1, sm.Sm, 1, NVP, NV, tm, 16, tn, 16);
+        mma_tile<4, TK>(ak, sm.dX, NVP, 1, sm.Sm, 1, NVP, NV, tm, 16, tn, 16);
+        mma_tile<4, TK>(an, sm.U, NVP, 1, sm.dSg, 1, NVP, NV, tm, 16, tn, 16);
+        mma_tile<4, 4>(dp, sm.dO, NVP, 1, sm.U, 1, NVP, NV, tm, 16, tn, 16);
+        mma_tile<4, 4>(dt, sm.dU, NVP, 1, sm.Y, 1, NVP, NV, tm, 16, tn, 16);
     }
     // dP (lower incl.) -> D1, dT -> D2; dgl and the first part of dbeta
 #pragma unroll
