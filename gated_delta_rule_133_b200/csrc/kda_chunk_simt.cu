@@ -37,7 +37,20 @@ constexpr int C = 64;       // chunk length
 constexpr int NV = 32;      // value columns per CTA
 constexpr int NT = 256;     // threads per CTA
 
+// (d0, d1) = (x0 * y0 + d0, x1 * y1 + d1) as one packed fp32x2 FMA; each
+// lane rounds exactly as fmaf does.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float x0, float x1, float y0, float y1)
+{
+    asm("{\n\t.reg .b64 xx, yy, dd;\n\t"
+        "mov.b64 xx, {%2, %3};\n\tmov.b64 yy, {%4, %5};\n\tmov.b64 dd, {%0, %1};\n\t"
+        "fma.rn.f32x2 dd, xx, yy, dd;\n\tmov.b64 {%0, %1}, dd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
+}
+
 // acc[i][j] += sum_kk A[(m0 + i*MS) * a_m + kk * a_k] * B[kk * b_k + (n0 + j*NS) * b_n]
+// The FMAs go in pairs (along j, else along i) as packed fp32x2 FMAs; every
+// element is accumulated in the same order and rounding as with fmaf.
 template <int TM, int TN>
 __device__ __forceinline__ void mma_tile(float (&acc)[TM][TN], const float* A, int a_m, int a_k,
                                          const float* B, int b_k, int b_n, int K, int m0, int MS,
@@ -50,10 +63,22 @@ __device__ __forceinline__ void mma_tile(float (&acc)[TM][TN], const float* A, i
         for (int i = 0; i < TM; ++i) a[i] = A[(m0 + i * MS) * a_m + kk * a_k];
 #pragma unroll
         for (int j = 0; j < TN; ++j) b[j] = B[kk * b_k + (n0 + j * NS) * b_n];
+        if constexpr (TN % 2 == 0) {
 #pragma unroll
-        for (int i = 0; i < TM; ++i)
+            for (int i = 0; i < TM; ++i)
 #pragma unroll
-            for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < TN; j += 2) fma2(acc[i][j], acc[i][j + 1], a[i], a[i], b[j], b[j + 1]);
+        } else if constexpr (TM % 2 == 0) {
+#pragma unroll
+            for (int i = 0; i < TM; i += 2)
+#pragma unroll
+                for (int j = 0; j < TN; ++j) fma2(acc[i][j], acc[i + 1][j], a[i], a[i + 1], b[j], b[j]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
     }
 }
 

@@ -179,3 +179,31 @@ def test_undersized_workspace_is_rejected_on_the_host():
     needv = _ws_size("kda_varlen_fwd_workspace_size", 3, T, H, 128, 128, 64, _lib.KDA_BF16, 0)
     v = (P, P, P, P, P, P, 3, None, P, None, T, H, 128, 128, 64, 1, 0)
     assert lib.kda_varlen_fwd(*v, W, needv - 1, None) == _lib.KDA_ERR_INVALID_ARG
+
+
+def test_backward_and_dplr_workspace_is_checked_on_the_host():
+    """The backward and the diagonal-plus-low-rank forward take a caller
+    workspace too: the size queries answer on the host, and a workspace that
+    is too small, missing or misaligned is refused before any launch."""
+    lib = _lib.load()
+    B, T, H = 1, 200, 2
+    W = 1 << 20   # a 256-byte aligned fake address
+    nb = _ws_size("kda_chunk_bwd_workspace_size", B, T, H, 128, 128, 64, _lib.KDA_BF16)
+    assert nb >= 4 * H * 64 * 128 * 4   # at least one record per (chunk, head)
+    assert _ws_size("kda_chunk_bwd_workspace_size", 0, T, H, 128, 128, 64, _lib.KDA_BF16) == 0
+    bwd = (P,) * 14 + (B, T, H, 128, 128, 64, 1)
+    assert lib.kda_chunk_bwd(*bwd, W, nb - 1, None) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_bwd(*bwd, None, nb, None) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_bwd(*bwd, W + 16, nb, None) == _lib.KDA_ERR_INVALID_ARG
+    nd = _ws_size("kda_dplr_fwd_workspace_size", B, T, H, 128, 128, 64, _lib.KDA_BF16)
+    assert nd >= 4 * H * 64 * 128 * 4
+    assert _ws_size("kda_dplr_fwd_workspace_size", B, 0, H, 128, 128, 64, _lib.KDA_BF16) == 0
+    dp = (P,) * 9 + (B, T, H, 128, 128, 64, 1, 0)
+    assert lib.kda_dplr_fwd(*dp, W, nd - 1, None) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_dplr_fwd(*dp, None, nd, None) == _lib.KDA_ERR_INVALID_ARG
+    ndv = _ws_size("kda_dplr_varlen_fwd_workspace_size", 3, T, H, 128, 128, 64, _lib.KDA_BF16)
+    assert ndv > 0
+    dv = (P,) * 7 + (3,) + (P,) * 3 + (T, H, 128, 128, 64, 1, 0)
+    assert lib.kda_dplr_varlen_fwd(*dv, W, ndv - 1, None) == _lib.KDA_ERR_INVALID_ARG
+    out = ctypes.c_size_t(0)
+    assert lib.kda_dplr_fwd_workspace_size(B, T, H, 96, 128, 64, 1, ctypes.byref(out)) == _lib.KDA_ERR_UNSUPPORTED

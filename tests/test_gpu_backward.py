@@ -115,3 +115,49 @@ def test_chunk_bwd_prefill_shape_sampled_heads():
         mine = [sl(t) for t in got[:3]] + [f64(got[3][n, :, h:h + 1]), sl(got[4]),
                                             f64(got[5][n:n + 1, h:h + 1])]
         _check(mine, ref)
+
+
+def test_varlen_bwd_boundaries_outside_the_tokens_are_skipped_and_reported():
+    """cu_seqlens whose last sequence runs past the token axis: that sequence
+    is skipped (zero gradients for its rows, dS_0 = dS_T), the others match
+    the oracle, and kda_check reports KDA_ERR_INVALID_ARG."""
+    lens = [100, 150, 50]
+    cu = cu_from_lengths(lens)
+    H, d, T = 2, 128, 300
+    t = draw_tokens(T, H, d, d, "bf16", -3.0, 340, "cpu", init_states=3, init_std=0.05)
+    g = torch.Generator().manual_seed(341)
+    do = torch.randn(T, H, d, generator=g)
+    dsT = torch.randn(3, H, d, d, generator=g)
+    dev = {n: (None if v is None else v.to(DEV)) for n, v in t.items()}
+    bad_cu = torch.tensor([0, 100, 250, 400], dtype=torch.int32, device=DEV)
+    got = kda.kda_varlen_bwd(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_alpha"], bad_cu,
+                             dev["initial_state"], do.to(DEV), dsT.to(DEV))
+    torch.cuda.synchronize()
+    with pytest.raises(kda.KdaError) as e:
+        kda.kda_check()
+    assert e.value.status == kda._lib.KDA_ERR_INVALID_ARG
+    n = 250
+    ref = backward.recurrence_backward(f64(t["q"])[:n], f64(t["k"])[:n], f64(t["v"])[:n], f64(t["beta"])[:n],
+                                       f64(t["log_alpha"])[:n], cu[:3], f64(t["initial_state"])[:2],
+                                       f64(do)[:n], f64(dsT)[:2])
+    _check([f64(x)[:n] for x in got[:5]] + [f64(got[5])[:2]], ref)
+    for x in (got[0], got[1], got[3], got[4]):
+        assert not x[n:].any()
+    assert torch.equal(got[5][2], dsT[2].to(DEV))
+
+
+def test_bwd_dirty_workspace_gives_identical_results():
+    """A caller workspace full of garbage gives bit-identical gradients."""
+    B, T, H, d = 2, 200, 2, 128
+    w = Workload("bwd", "dense", B, T, H, d, d, "bf16", -3.0, 0.05, seed=350)
+    x = {n: (None if v is None else v.to(DEV)) for n, v in make_inputs(w, "cpu").items()}
+    do = torch.randn(B, T, H, d, generator=torch.Generator().manual_seed(351)).to(DEV)
+    args = (x["q"], x["k"], x["v"], x["beta"], x["log_alpha"], x["initial_state"], do)
+    g1 = kda.kda_chunk_bwd(*args)
+    n = kda._lib.workspace_size("kda_chunk_bwd_workspace_size", B, T, H, d, d, 64, kda._lib.KDA_BF16)
+    ws = torch.full((n,), 0xFF, dtype=torch.uint8, device=DEV)
+    g2 = kda.kda_chunk_bwd(*args, workspace=ws)
+    torch.cuda.synchronize()
+    kda.kda_check()
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)

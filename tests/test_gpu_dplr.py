@@ -80,3 +80,44 @@ def test_dplr_varlen_matches_oracle():
                                    f64(x["initial_state"]))
     assert norm_max_err(f64(o), o_ref) <= TOL
     assert norm_max_err(f64(sN), s_ref) <= TOL
+
+
+def test_dplr_varlen_boundaries_outside_the_tokens_are_skipped_and_reported():
+    """cu_seqlens whose last sequence runs past the token axis: that sequence
+    is skipped (o rows untouched, final state = initial state), the others are
+    computed, and kda_check reports KDA_ERR_INVALID_ARG."""
+    lens = [100, 150, 50]
+    cu = cu_from_lengths(lens)
+    H, d, T = 2, 128, 300
+    x = draw_tokens(T, H, d, d, "bf16", -3.0, 530, "cpu", init_states=3, init_std=0.05)
+    a, b = _ab(T, H, d, "bf16", 531)
+    s0 = x["initial_state"].to(DEV)
+    o = torch.full((T, H, d), float("nan"), device=DEV)
+    bad_cu = torch.tensor([0, 100, 250, 400], dtype=torch.int32, device=DEV)
+    o, sN = kda.kda_dplr_varlen_fwd(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), a.to(DEV), b.to(DEV),
+                                    x["log_alpha"].to(DEV), bad_cu, s0, o=o)
+    torch.cuda.synchronize()
+    with pytest.raises(kda.KdaError) as e:
+        kda.kda_check()
+    assert e.value.status == kda._lib.KDA_ERR_INVALID_ARG
+    o_ref, s_ref = dplr.recurrence(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(a), f64(b), f64(x["log_alpha"]), cu,
+                                   f64(x["initial_state"]))
+    assert norm_max_err(f64(o[:250]), o_ref[:250]) <= TOL
+    assert norm_max_err(f64(sN[:2]), s_ref[:2]) <= TOL
+    assert torch.isnan(o[250:]).all()
+    assert torch.equal(sN[2], s0[2])
+
+
+def test_dplr_dirty_workspace_gives_identical_results():
+    """A caller workspace full of garbage gives bit-identical results."""
+    B, T, H, d = 2, 300, 2, 128
+    x = draw_tokens(B * T, H, d, d, "bf16", -3.0, 540, "cpu", init_states=B, init_std=0.05)
+    a, b = _ab(B * T, H, d, "bf16", 541)
+    r = lambda t: t.reshape(B, T, *t.shape[1:]).to(DEV)
+    args = (r(x["q"]), r(x["k"]), r(x["v"]), r(a), r(b), r(x["log_alpha"]), x["initial_state"].to(DEV))
+    o1, s1 = kda.kda_dplr_fwd(*args)
+    ws = torch.full((kda.dplr_fwd_workspace_size(B, T, H, d, d),), 0xFF, dtype=torch.uint8, device=DEV)
+    o2, s2 = kda.kda_dplr_fwd(*args, workspace=ws)
+    torch.cuda.synchronize()
+    kda.kda_check()
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
