@@ -88,6 +88,7 @@ struct Params {
     float* U;                // [record][H][C][DV]
     float* dU;
     float* dY;
+    float* VX;               // V - X of every chunk: [record][H][C][DV]
     float* dSn;              // gradient reaching the state after each chunk: [record][H][DK][DV]
     const int32_t* cu;
     const int32_t* choff;    // varlen: first record of each sequence, [nseq + 1]
@@ -146,17 +147,26 @@ __device__ __forceinline__ void stage(float* dst, int ld, const float* src, cons
 
 template <int DK>
 struct FacSmem {
+    // A and T take the place of q E and k E once the products have read
+    // them, so that two CTAs fit on an SM
     static constexpr int LDK = DK + 1, LDC = C + 1;
-    float qm[C * LDK];    // q, then q E
-    float km[C * LDK];    // k, then k E
+    union {
+        struct {
+            float qm[C * LDK];    // q, then q E
+            float km[C * LDK];    // k, then k E
+        };
+        struct {
+            float D[C * LDC];     // A = beta MA
+            float T[C * LDC];     // (I + A)^-1
+        };
+    };
     float kf[C * LDK];    // log alpha, then G, then k F
-    float D[C * LDC];     // A = beta MA
-    float T[C * LDC];     // (I + A)^-1
     float beta[C];
+    static_assert(LDC <= LDK, "A and T fit in the space of q E and k E");
 };
 
 template <typename TIn, int DK>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT, 2)
 bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Params p)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -215,6 +225,7 @@ bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Pa
         float pp[4][4] = {}, a[4][4] = {};
         mma_tile<4, 4>(pp, sm.qm, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
         mma_tile<4, 4>(a, sm.km, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
+        __syncthreads();   // q E and k E are read: A takes their place
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -315,15 +326,18 @@ bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
         if (!packed::stream_wait(sm.st, 0, ci)) goto drain;
         for (int e = tid; e < DK * NW; e += NT) sm.Sm[e] = vec[R::V_GM + e / NW] * sm.S[e];
         __syncthreads();
-        {   // X = K~ Sm, Y = beta (V - X)
+        {   // X = K~ Sm, Y = beta (V - X); V - X is kept for the gradient kernel
             float xx[4][2] = {};
             mma_tile<4, 2>(xx, KM, DK, 1, sm.Sm, NW, 1, DK, tm, 16, tn, 16);
+            float* vxg = p.VX + item * (size_t)C * DV + col0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int r = tm + 16 * i, e = r * NW + tn + 16 * j;
-                    sm.Y[e] = vec[R::V_BETA + r] * (sm.V[e] - xx[i][j]);
+                    const int r = tm + 16 * i, cc = tn + 16 * j, e = r * NW + cc;
+                    const float vx = sm.V[e] - xx[i][j];
+                    sm.Y[e] = vec[R::V_BETA + r] * vx;
+                    vxg[(size_t)r * DV + cc] = vx;
                 }
         }
         __syncthreads();   // part 0 is read
@@ -525,12 +539,10 @@ struct GradSmem {
     float D2[C * LDC];    // dT, then dMA
     float Sm[DK * NVP];    // e^G_m S (value columns of this pass)
     float dSg[DK * NVP];   // e^(G_last - G_m) dS'
-    float VX[C * NVP];     // V, then V - X
     float dO[C * NVP];
     float U[C * NVP];
     float dU[C * NVP];
     float Y[C * NVP];      // beta (V - X)
-    float dY[C * NVP];
     float dX[C * NVP];     // -beta dY
     float gm[DK];
     float glm[DK];
@@ -539,9 +551,9 @@ struct GradSmem {
     float db[C];
 };
 
-template <typename TIn, int DK>
+template <int DK>
 __global__ void __launch_bounds__(NT, 1)
-bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
+bwd_grad_kernel(const Params p)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     GradSmem<DK>& sm = *reinterpret_cast<GradSmem<DK>*>(smem_raw);
@@ -560,6 +572,7 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
     const float* Ug = p.U + item * (size_t)C * DV;
     const float* dUg = p.dU + item * (size_t)C * DV;
     const float* dYg = p.dY + item * (size_t)C * DV;
+    const float* VXg = p.VX + item * (size_t)C * DV;
 
     if (tid < DK) {
         sm.gm[tid] = rec[R::GM + tid];
@@ -574,12 +587,11 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
 
     float aq[4][TK] = {}, ak[4][TK] = {}, an[4][TK] = {};
     float dp[4][4] = {}, dt[4][4] = {};
-    float db1[4] = {0.f, 0.f, 0.f, 0.f};
+    float db1 = 0.f;      // rowsum((V - X) dY) of row tid / 4 over this thread's columns
     // pass loads: thread tid holds float4 number tid + i NT of each [DK][16]
     // slice (channel (tid + i NT) / 4) and float4 number tid of each [C][16]
     // slice (row tid / 4); all are issued before the first store
     constexpr int NS = DK * NV / 4 / NT;              // float4 per thread of a [DK][16] slice
-    constexpr int EPV = 16 / (int)sizeof(TIn), VPR = NV / EPV;
     static_assert(C * NV / 4 == NT, "one float4 of a [C][16] slice per thread");
     float dgl[NS] = {};   // channel (tid + i NT) / 4, summed over this thread's columns
     const int rr = tid / 4, c4 = 4 * (tid % 4);
@@ -601,10 +613,7 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
         const float4 u4 = __ldg(reinterpret_cast<const float4*>(Ug + g));
         const float4 du4 = __ldg(reinterpret_cast<const float4*>(dUg + g));
         const float4 dy4 = __ldg(reinterpret_cast<const float4*>(dYg + g));
-        uint4 vv = make_uint4(0u, 0u, 0u, 0u);
-        const int vr = tid / VPR;
-        if (tid < C * VPR && vr < L)
-            vv = __ldg(reinterpret_cast<const uint4*>(v + ((size_t)(x.tok + vr) * H + h) * DV + j0 + (tid % VPR) * EPV));
+        const float4 vx4 = __ldg(reinterpret_cast<const float4*>(VXg + g));
         __syncthreads();   // the previous pass has read its slices (first pass: the vectors are in place)
 #pragma unroll
         for (int i = 0; i < NS; ++i) {
@@ -628,27 +637,9 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
             put(sm.dO, o4);
             put(sm.U, u4);
             put(sm.dU, du4);
-            put(sm.dY, dy4);
             put(sm.dX, make_float4(-b * dy4.x, -b * dy4.y, -b * dy4.z, -b * dy4.w));
-            if (tid < C * VPR) {
-                const TIn* xv = reinterpret_cast<const TIn*>(&vv);
-                float* d = sm.VX + vr * NVP + (tid % VPR) * EPV;
-#pragma unroll
-                for (int u = 0; u < EPV; ++u) d[u] = Elem<TIn>::load(xv + u);
-            }
-        }
-        __syncthreads();
-        {   // X = K~ (e^G_m S); V - X; Y = beta (V - X); rowsum((V - X) dY)
-            float xx[4][1] = {};
-            mma_tile<4, 1>(xx, sm.km, LDK, 1, sm.Sm, NVP, 1, DK, tm, 16, tn, 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = tm + 16 * i, e = r * NVP + tn;
-                const float vx = sm.VX[e] - xx[i][0];
-                sm.VX[e] = vx;
-                sm.Y[e] = sm.beta[r] * vx;
-                db1[i] = fmaf(vx, sm.dY[e], db1[i]);
-            }
+            put(sm.Y, make_float4(b * vx4.x, b * vx4.y, b * vx4.z, b * vx4.w));
+            db1 += vx4.x * dy4.x + vx4.y * dy4.y + vx4.z * dy4.z + vx4.w * dy4.w;
         }
         __syncthreads();
         // a_q += dO Sm^T, a_k += dX Sm^T, a_n += U dSg^T; dP += dO U^T, dT += dU Y^T
@@ -668,8 +659,12 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
             sm.D1[r * LDC + s] = s <= r ? dp[i][j] : 0.f;
             sm.D2[r * LDC + s] = dt[i][j];
         }
-        const float b = sum16(db1[i]);
-        if (tn == 0) sm.db[r] = b;
+    }
+    {   // the 4 threads of a row are consecutive lanes
+        float b = db1;
+        b += __shfl_xor_sync(0xffffffffu, b, 1);
+        b += __shfl_xor_sync(0xffffffffu, b, 2);
+        if ((tid & 3) == 0) sm.db[tid / 4] = b;
     }
 #pragma unroll
     for (int i = 0; i < NS; ++i) {   // the 4 threads of a channel are consecutive lanes
@@ -751,7 +746,7 @@ bwd_grad_kernel(const TIn* __restrict__ v, const Params p)
 
 // Parts of a call's workspace (byte offsets).
 struct Ws {
-    size_t states, rec, U, dU, dY, dSn, choff, bytes;
+    size_t states, rec, U, dU, dY, VX, dSn, choff, bytes;
     long long nrec;   // records per head (an upper bound for packed batches)
 };
 
@@ -773,6 +768,8 @@ static Ws ws_layout(int nseq, int T, long long tokens, int H, int dk, int dv, bo
     w.dU = off;
     off += al1k((size_t)w.nrec * H * C * dv * 4);
     w.dY = off;
+    off += al1k((size_t)w.nrec * H * C * dv * 4);
+    w.VX = off;
     off += al1k((size_t)w.nrec * H * C * dv * 4);
     w.dSn = off;
     off += al1k((size_t)w.nrec * H * dk * dv * 4);
@@ -796,7 +793,7 @@ cudaError_t launch(const void* q, const void* k, const void* v, const Params& p,
     auto kf = bwd_factor_kernel<TIn, DK>;
     auto kw = bwd_forward_kernel<TIn, DK>;
     auto kr = bwd_reverse_kernel<DK>;
-    auto kg = bwd_grad_kernel<TIn, DK>;
+    auto kg = bwd_grad_kernel<DK>;
     cudaError_t err = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(FacSmem<DK>));
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(kw, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(FwdSmem<DK>));
@@ -818,7 +815,7 @@ cudaError_t launch(const void* q, const void* k, const void* v, const Params& p,
     kr<<<(unsigned)walk_ctas, NT, sizeof(RevSmem<DK>), stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (items > 0) {
-        kg<<<(unsigned)items, NT, sizeof(GradSmem<DK>), stream>>>(vv, p);
+        kg<<<(unsigned)items, NT, sizeof(GradSmem<DK>), stream>>>(p);
         err = cudaGetLastError();
     }
     return err;
@@ -857,6 +854,7 @@ cudaError_t chunk_bwd(const void* q, const void* k, const void* v, const float* 
     p.U = reinterpret_cast<float*>(w + L.U);
     p.dU = reinterpret_cast<float*>(w + L.dU);
     p.dY = reinterpret_cast<float*>(w + L.dY);
+    p.VX = reinterpret_cast<float*>(w + L.VX);
     p.dSn = reinterpret_cast<float*>(w + L.dSn);
     int32_t* choff = reinterpret_cast<int32_t*>(w + L.choff);
     p.cu = cu;
