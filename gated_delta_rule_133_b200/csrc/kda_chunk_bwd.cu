@@ -46,6 +46,8 @@ namespace kda {
 
 namespace bwd {
 
+using simt::mma_rk;
+using simt::mma_tk;
 using simt::mma_tile;
 
 constexpr int C = 64;       // chunk length
@@ -328,13 +330,13 @@ bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
         __syncthreads();
         {   // X = K~ Sm, Y = beta (V - X); V - X is kept for the gradient kernel
             float xx[4][2] = {};
-            mma_tile<4, 2>(xx, KM, DK, 1, sm.Sm, NW, 1, DK, tm, 16, tn, 16);
+            mma_rk<4, 2>(xx, KM, DK, sm.Sm, NW, DK, 4 * tm, 2 * tn);
             float* vxg = p.VX + item * (size_t)C * DV + col0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int r = tm + 16 * i, cc = tn + 16 * j, e = r * NW + cc;
+                    const int r = 4 * tm + i, cc = 2 * tn + j, e = r * NW + cc;
                     const float vx = sm.V[e] - xx[i][j];
                     sm.Y[e] = vec[R::V_BETA + r] * vx;
                     vxg[(size_t)r * DV + cc] = vx;
@@ -348,13 +350,13 @@ bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
         for (int i = 0; i < NVR; ++i) vn[i] = ci + 1 < nch ? v_at(ci + 1, tid + i * NT) : 0.f;
         {   // U = T Y
             float u[4][2] = {};
-            mma_tile<4, 2>(u, T, C, 1, sm.Y, NW, 1, C, tm, 16, tn, 16);
+            mma_rk<4, 2>(u, T, C, sm.Y, NW, C, 4 * tm, 2 * tn);
             float* ug = p.U + item * (size_t)C * DV + col0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int r = tm + 16 * i, cc = tn + 16 * j;
+                    const int r = 4 * tm + i, cc = 2 * tn + j;
                     sm.U[r * NW + cc] = u[i][j];
                     ug[(size_t)r * DV + cc] = u[i][j];
                 }
@@ -362,12 +364,12 @@ bwd_forward_kernel(const TIn* __restrict__ v, const Params p)
         __syncthreads();
         {   // S <- gamma S + e^(G_last - G_m) (K~n^T U)
             float ds[TK][2] = {};
-            mma_tile<TK, 2>(ds, KF, 1, DK, sm.U, NW, 1, C, tm, 16, tn, 16);
+            mma_tk<TK, 2>(ds, KF, DK, sm.U, NW, C, TK * tm, 2 * tn);
 #pragma unroll
             for (int i = 0; i < TK; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
+                    const int c = TK * tm + i, e = c * NW + 2 * tn + j;
                     sm.S[e] = fmaf(vec2[R::V_GAM + c], sm.S[e], vec2[R::V_GLM + c] * ds[i][j]);
                 }
         }
@@ -461,14 +463,14 @@ bwd_reverse_kernel(const Params p)
         __syncthreads();
         {   // dU = P^T dO + K~n dSg
             float du[4][2] = {};
-            mma_tile<4, 2>(du, P, 1, C, sm.dO, NW, 1, C, tm, 16, tn, 16);
-            mma_tile<4, 2>(du, KF, DK, 1, sm.dSg, NW, 1, DK, tm, 16, tn, 16);
+            mma_tk<4, 2>(du, P, C, sm.dO, NW, C, 4 * tm, 2 * tn);
+            mma_rk<4, 2>(du, KF, DK, sm.dSg, NW, DK, 4 * tm, 2 * tn);
             float* g = p.dU + item * (size_t)C * DV + col0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int r = tm + 16 * i, cc = tn + 16 * j;
+                    const int r = 4 * tm + i, cc = 2 * tn + j;
                     sm.dU[r * NW + cc] = du[i][j];
                     g[(size_t)r * DV + cc] = du[i][j];
                 }
@@ -476,13 +478,13 @@ bwd_reverse_kernel(const Params p)
         __syncthreads();
         {   // dY = T^T dU; dv = beta dY; dX = -beta dY
             float dy[4][2] = {};
-            mma_tile<4, 2>(dy, T, 1, C, sm.dU, NW, 1, C, tm, 16, tn, 16);
+            mma_tk<4, 2>(dy, T, C, sm.dU, NW, C, 4 * tm, 2 * tn);
             float* g = p.dY + item * (size_t)C * DV + col0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int r = tm + 16 * i, cc = tn + 16 * j;
+                    const int r = 4 * tm + i, cc = 2 * tn + j;
                     const float b = vec2[R::V_BETA + r];
                     g[(size_t)r * DV + cc] = dy[i][j];
                     sm.dX[r * NW + cc] = -b * dy[i][j];
@@ -497,13 +499,13 @@ bwd_reverse_kernel(const Params p)
         for (int i = 0; i < NVR; ++i) dn[i] = ci > 0 ? do_at(ci - 1, tid + i * NT) : 0.f;
         {   // dS = gamma dS' + e^G_m (Q~^T dO + K~^T dX)
             float ds[TK][2] = {};
-            mma_tile<TK, 2>(ds, QM, 1, DK, sm.dO, NW, 1, C, tm, 16, tn, 16);
-            mma_tile<TK, 2>(ds, KM, 1, DK, sm.dX, NW, 1, C, tm, 16, tn, 16);
+            mma_tk<TK, 2>(ds, QM, DK, sm.dO, NW, C, TK * tm, 2 * tn);
+            mma_tk<TK, 2>(ds, KM, DK, sm.dX, NW, C, TK * tm, 2 * tn);
 #pragma unroll
             for (int i = 0; i < TK; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
+                    const int c = TK * tm + i, e = c * NW + 2 * tn + j;
                     sm.dS[e] = fmaf(vec[R::V_GAM + c], sm.dS[e], vec[R::V_GM + c] * ds[i][j]);
                 }
         }

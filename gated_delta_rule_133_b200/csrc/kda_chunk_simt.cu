@@ -82,6 +82,77 @@ __device__ __forceinline__ void mma_tile(float (&acc)[TM][TN], const float* A, i
     }
 }
 
+// B row kk, columns n0 .. n0 + TN - 1 (contiguous, 8-byte aligned for TN = 2,
+// 16-byte aligned for TN = 4 or 8) into b.
+template <int TN>
+__device__ __forceinline__ void ld_row(float (&b)[TN], const float* p)
+{
+    static_assert(TN == 2 || TN % 4 == 0, "row segment of 2, 4 or 8 floats");
+    if constexpr (TN == 2) {
+        const float2 x = *reinterpret_cast<const float2*>(p);
+        b[0] = x.x;
+        b[1] = x.y;
+    } else {
+#pragma unroll
+        for (int j = 0; j < TN; j += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(p + j);
+            b[j] = x.x;
+            b[j + 1] = x.y;
+            b[j + 2] = x.z;
+            b[j + 3] = x.w;
+        }
+    }
+}
+
+// acc[i][j] += sum_kk A[(m0 + i) * lda + kk] * B[kk * ldb + n0 + j]: TM
+// consecutive rows and TN consecutive columns per thread, A rows read four K
+// values at a time.  K, lda and m0's row offsets are multiples of 4 (16-byte
+// aligned A rows); B rows as for ld_row.  Each element is accumulated in K
+// order with packed fp32x2 FMAs (the rounding of fmaf).
+template <int TM, int TN>
+__device__ __forceinline__ void mma_rk(float (&acc)[TM][TN], const float* A, int lda, const float* B, int ldb, int K,
+                                       int m0, int n0)
+{
+    static_assert(TN % 2 == 0, "columns in pairs");
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 4) {
+        float4 a[TM];
+#pragma unroll
+        for (int i = 0; i < TM; ++i) a[i] = *reinterpret_cast<const float4*>(A + (m0 + i) * lda + k0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float b[TN];
+            ld_row<TN>(b, B + (k0 + u) * ldb + n0);
+#pragma unroll
+            for (int i = 0; i < TM; ++i) {
+                const float av = u == 0 ? a[i].x : u == 1 ? a[i].y : u == 2 ? a[i].z : a[i].w;
+#pragma unroll
+                for (int j = 0; j < TN; j += 2) fma2(acc[i][j], acc[i][j + 1], av, av, b[j], b[j + 1]);
+            }
+        }
+    }
+}
+
+// acc[i][j] += sum_kk A[kk * lda + m0 + i] * B[kk * ldb + n0 + j]: the same
+// with A stored transposed (K rows of M), read TM values at a time (m0 and lda
+// multiples of 4).
+template <int TM, int TN>
+__device__ __forceinline__ void mma_tk(float (&acc)[TM][TN], const float* A, int lda, const float* B, int ldb, int K,
+                                       int m0, int n0)
+{
+    static_assert(TN % 2 == 0 && TM % 4 == 0, "columns in pairs, rows in fours");
+#pragma unroll 4
+    for (int kk = 0; kk < K; ++kk) {
+        float a[TM], b[TN];
+        ld_row<TM>(a, A + kk * lda + m0);
+        ld_row<TN>(b, B + kk * ldb + n0);
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TN; j += 2) fma2(acc[i][j], acc[i][j + 1], a[i], a[i], b[j], b[j + 1]);
+    }
+}
+
 template <int DK>
 struct Smem {
     static constexpr int LDK = DK + 1;   // padded row pitch of the [C][DK] tiles

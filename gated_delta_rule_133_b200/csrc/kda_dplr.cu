@@ -33,6 +33,8 @@ namespace kda {
 
 namespace dplr {
 
+using simt::mma_rk;
+using simt::mma_tk;
 using simt::mma_tile;
 
 constexpr int C = 64;
@@ -240,48 +242,48 @@ dplr_walk_kernel(const TIn* __restrict__ v, TOut* __restrict__ o, const Params p
         if (!packed::stream_wait(sm.st, 0, ci)) goto drain;   // also orders S and V
         // W = (e^{Gx} a) S + A_ak V;  OQ = (e^G q) S
         float w[4][2] = {}, oq[4][2] = {};
-        mma_tile<4, 2>(w, AX, DK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
-        mma_tile<4, 2>(w, AAK, C, 1, sm.V, NW, 1, C, tm, 16, tn, 16);
-        mma_tile<4, 2>(oq, QX, DK, 1, sm.S, NW, 1, DK, tm, 16, tn, 16);
+        mma_rk<4, 2>(w, AX, DK, sm.S, NW, DK, 4 * tm, 2 * tn);
+        mma_rk<4, 2>(w, AAK, C, sm.V, NW, C, 4 * tm, 2 * tn);
+        mma_rk<4, 2>(oq, QX, DK, sm.S, NW, DK, 4 * tm, 2 * tn);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) sm.W[(tm + 16 * i) * NW + tn + 16 * j] = w[i][j];
+            for (int j = 0; j < 2; ++j) sm.W[(4 * tm + i) * NW + 2 * tn + j] = w[i][j];
         __syncthreads();
         // U = (I - A_ab)^-1 W
         float u[4][2] = {};
-        mma_tile<4, 2>(u, TI, C, 1, sm.W, NW, 1, C, tm, 16, tn, 16);
+        mma_rk<4, 2>(u, TI, C, sm.W, NW, C, 4 * tm, 2 * tn);
         __syncthreads();   // part 1 and W are read
         if (tid == 0 && ci + 1 < nch) packed::stream_fetch(sm.st, 0, sm.part1, rec_of(ci + 1), R::PART1_BYTES);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) sm.W[(tm + 16 * i) * NW + tn + 16 * j] = u[i][j];
+            for (int j = 0; j < 2; ++j) sm.W[(4 * tm + i) * NW + 2 * tn + j] = u[i][j];
         if (!packed::stream_wait(sm.st, 1, ci)) goto drain;   // also orders U
         float vn[NVR];   // next chunk's V, in flight during the arithmetic below
 #pragma unroll
         for (int i = 0; i < NVR; ++i) vn[i] = ci + 1 < nch ? v_at(ci + 1, tid + i * NT) : 0.f;
         // O = OQ + P_qb U + P_qk V -> rows < L
-        mma_tile<4, 2>(oq, PQB, C, 1, sm.W, NW, 1, C, tm, 16, tn, 16);
-        mma_tile<4, 2>(oq, PQK, C, 1, sm.V, NW, 1, C, tm, 16, tn, 16);
+        mma_rk<4, 2>(oq, PQB, C, sm.W, NW, C, 4 * tm, 2 * tn);
+        mma_rk<4, 2>(oq, PQK, C, sm.V, NW, C, 4 * tm, 2 * tn);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int r = tm + 16 * i;
+            const int r = 4 * tm + i;
             if (r < L)
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
-                    Elem<TOut>::store(o + ((size_t)(tok + r) * H + h) * DV + col0 + tn + 16 * j, oq[i][j]);
+                    Elem<TOut>::store(o + ((size_t)(tok + r) * H + h) * DV + col0 + 2 * tn + j, oq[i][j]);
         }
         // S <- e^{G_last} S + (e^{G_last - G} b)^T U + (e^{G_last - G} k)^T V
         {
             float ds[TK][2] = {};
-            mma_tile<TK, 2>(ds, BL, 1, DK, sm.W, NW, 1, C, tm, 16, tn, 16);
-            mma_tile<TK, 2>(ds, KL, 1, DK, sm.V, NW, 1, C, tm, 16, tn, 16);
+            mma_tk<TK, 2>(ds, BL, DK, sm.W, NW, C, TK * tm, 2 * tn);
+            mma_tk<TK, 2>(ds, KL, DK, sm.V, NW, C, TK * tm, 2 * tn);
 #pragma unroll
             for (int i = 0; i < TK; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int c = tm + 16 * i, e = c * NW + tn + 16 * j;
+                    const int c = TK * tm + i, e = c * NW + 2 * tn + j;
                     sm.S[e] = fmaf(gam[c], sm.S[e], ds[i][j]);
                 }
         }
