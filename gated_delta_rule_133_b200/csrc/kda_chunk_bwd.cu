@@ -57,7 +57,7 @@ constexpr int NT = 256;     // threads per CTA
 
 // Factor record of one (chunk, head), in floats, laid out so that each walk
 // streams two contiguous parts (the channel vectors are stored twice):
-//   Q~, K~ [C][DK]; VEC;  P, T [C][C]; K~n [C][DK]; VEC again;  G [C][DK]; MA [C][C]
+//   Q~, K~ [C][DK]; VEC;  P, T [C][C]; K~n [C][DK]; VEC again;  G [C][DK]; MA, T^T [C][C]
 // with VEC = e^G_m, e^G_last, e^(G_last - G_m) [DK] and beta [C].
 //   forward walk: part 0 = K~, VEC;          part 1 = T, K~n, VEC
 //   reverse walk: part 0 = P, T, K~n, VEC;   part 1 = Q~, K~, VEC
@@ -67,8 +67,8 @@ struct Rec {
     static constexpr int QM = 0, KM = QM + C * DK, VEC = KM + C * DK;
     static constexpr int GM = VEC, GAM = VEC + DK, GLM = VEC + 2 * DK, BETA = VEC + 3 * DK;
     static constexpr int P = VEC + VECN, T = P + C * C, KF = T + C * C, VEC2 = KF + C * DK;
-    static constexpr int G = VEC2 + VECN, MA = G + C * DK;
-    static constexpr int FLOATS = (MA + C * C + 63) & ~63;
+    static constexpr int G = VEC2 + VECN, MA = G + C * DK, TT = MA + C * C;
+    static constexpr int FLOATS = (TT + C * C + 63) & ~63;
     // vector offsets inside a VEC block
     static constexpr int V_GM = 0, V_GAM = DK, V_GLM = 2 * DK, V_BETA = 3 * DK;
 };
@@ -252,7 +252,10 @@ bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Pa
         }
     }
     __syncthreads();
-    for (int e = tid; e < C * C; e += NT) rec[R::T + e] = sm.T[(e / C) * LDC + e % C];
+    for (int e = tid; e < C * C; e += NT) {
+        rec[R::T + e] = sm.T[(e / C) * LDC + e % C];
+        rec[R::TT + e] = sm.T[(e % C) * LDC + e / C];
+    }
 }
 
 // ================================================================ 2. forward walk
@@ -527,25 +530,28 @@ drain:
 
 // ================================================================ 4. gradients
 
+// Every operand tile is laid out so that the products read it along rows:
+// the record tiles unpadded, the pass tiles that serve as B operands
+// transposed ([16][*]).  A thread owns rows 4 tm .. 4 tm + 3 and a run of
+// consecutive columns of every accumulator.
 template <int DK>
 struct GradSmem {
-    // NVP: padded pitch of the [*][16] pass tiles, which the products also
-    // read down their columns
-    static constexpr int LDK = DK + 1, LDC = C + 1, NVP = NV + 1;
-    float qm[C * LDK];    // Q~, then dG
-    float km[C * LDK];    // K~
-    float kf[C * LDK];    // K~n
-    float MA[C * LDC];
-    float T[C * LDC];
-    float D1[C * LDC];    // dP, then T^T dT
-    float D2[C * LDC];    // dT, then dMA
-    float Sm[DK * NVP];    // e^G_m S (value columns of this pass)
-    float dSg[DK * NVP];   // e^(G_last - G_m) dS'
-    float dO[C * NVP];
-    float U[C * NVP];
-    float dU[C * NVP];
-    float Y[C * NVP];      // beta (V - X)
-    float dX[C * NVP];     // -beta dY
+    float qm[C * DK];     // Q~, then dG
+    float km[C * DK];     // K~
+    float kf[C * DK];     // K~n
+    float MA[C * C];
+    float T[C * C];
+    float TT[C * C];      // T^T
+    float D1[C * C];      // dP, then T^T dT
+    float D2[C * C];      // dT, then dMA
+    float dO[C * NV];     // pass tiles, [C][16]
+    float dX[C * NV];     // -beta dY
+    float U[C * NV];
+    float dU[C * NV];
+    float SmT[NV * DK];   // (e^G_m S)^T, [16][DK]
+    float dSgT[NV * DK];  // (e^(G_last - G_m) dS')^T
+    float UT[NV * C];     // U^T, [16][C]
+    float YT[NV * C];     // (beta (V - X))^T
     float gm[DK];
     float glm[DK];
     float dgl[DK];        // rowsum(dS' S'): the last row's extra dG
@@ -560,12 +566,12 @@ bwd_grad_kernel(const Params p)
     extern __shared__ __align__(16) unsigned char smem_raw[];
     GradSmem<DK>& sm = *reinterpret_cast<GradSmem<DK>*>(smem_raw);
     using R = Rec<DK>;
-    constexpr int LDK = GradSmem<DK>::LDK, LDC = GradSmem<DK>::LDC, NVP = GradSmem<DK>::NVP;
-    constexpr int TK = DK / 16;
+    constexpr int TK = DK / 16;   // accumulator columns per thread: TK tn .. TK tn + TK - 1
     const packed::Pos x = packed::locate(layout_of(p), blockIdx.x);
     if (!x.ok) return;
     const int tid = threadIdx.x, tn = tid % 16, tm = tid / 16;
     const int DV = p.DV, H = p.H, L = x.L, h = x.h;
+    const int m0 = 4 * tm, n0 = TK * tn, s0c = 4 * tn;
     const size_t item = blockIdx.x;
     const float* rec = p.rec + item * R::FLOATS;
     const float* S0 = p.states + ((size_t)x.slot * H + h) * (size_t)DK * DV;          // entering the chunk
@@ -581,11 +587,12 @@ bwd_grad_kernel(const Params p)
         sm.glm[tid] = rec[R::GLM + tid];
     }
     if (tid < C) sm.beta[tid] = rec[R::BETA + tid];
-    stage<C, DK>(sm.qm, LDK, rec + R::QM);
-    stage<C, DK>(sm.km, LDK, rec + R::KM);
-    stage<C, DK>(sm.kf, LDK, rec + R::KF);
-    stage<C, C>(sm.MA, LDC, rec + R::MA);
-    stage<C, C>(sm.T, LDC, rec + R::T);
+    stage<C, DK>(sm.qm, DK, rec + R::QM);
+    stage<C, DK>(sm.km, DK, rec + R::KM);
+    stage<C, DK>(sm.kf, DK, rec + R::KF);
+    stage<C, C>(sm.MA, C, rec + R::MA);
+    stage<C, C>(sm.T, C, rec + R::T);
+    stage<C, C>(sm.TT, C, rec + R::TT);
 
     float aq[4][TK] = {}, ak[4][TK] = {}, an[4][TK] = {};
     float dp[4][4] = {}, dt[4][4] = {};
@@ -600,12 +607,12 @@ bwd_grad_kernel(const Params p)
     const bool rin = rr < L;
     const size_t rowg = ((size_t)(x.tok + rr) * H + h) * DV;
     for (int j0 = 0; j0 < DV; j0 += NV) {
-        float4 s0[NS], d1[NS], s1[NS];
+        float4 sa[NS], d1[NS], s1[NS];
 #pragma unroll
         for (int i = 0; i < NS; ++i) {
             const int e = tid + i * NT;
             const size_t g = (size_t)(e / 4) * DV + j0 + 4 * (e % 4);
-            s0[i] = __ldg(reinterpret_cast<const float4*>(S0 + g));
+            sa[i] = __ldg(reinterpret_cast<const float4*>(S0 + g));
             d1[i] = __ldg(reinterpret_cast<const float4*>(dS1 + g));
             s1[i] = __ldg(reinterpret_cast<const float4*>(S1 + g));
         }
@@ -616,51 +623,58 @@ bwd_grad_kernel(const Params p)
         const float4 du4 = __ldg(reinterpret_cast<const float4*>(dUg + g));
         const float4 dy4 = __ldg(reinterpret_cast<const float4*>(dYg + g));
         const float4 vx4 = __ldg(reinterpret_cast<const float4*>(VXg + g));
-        __syncthreads();   // the previous pass has read its slices (first pass: the vectors are in place)
+        __syncthreads();   // the previous pass has read its tiles (first pass: the vectors are in place)
 #pragma unroll
         for (int i = 0; i < NS; ++i) {
-            const int e = tid + i * NT, c = e / 4;
+            const int e = tid + i * NT, c = e / 4, q = 4 * (e % 4);
             const float gmc = sm.gm[c], glc = sm.glm[c];
-            float* sm4 = sm.Sm + c * NVP + 4 * (e % 4);
-            float* dg4 = sm.dSg + c * NVP + 4 * (e % 4);
-            sm4[0] = gmc * s0[i].x; sm4[1] = gmc * s0[i].y; sm4[2] = gmc * s0[i].z; sm4[3] = gmc * s0[i].w;
-            dg4[0] = glc * d1[i].x; dg4[1] = glc * d1[i].y; dg4[2] = glc * d1[i].z; dg4[3] = glc * d1[i].w;
+            sm.SmT[(q + 0) * DK + c] = gmc * sa[i].x;
+            sm.SmT[(q + 1) * DK + c] = gmc * sa[i].y;
+            sm.SmT[(q + 2) * DK + c] = gmc * sa[i].z;
+            sm.SmT[(q + 3) * DK + c] = gmc * sa[i].w;
+            sm.dSgT[(q + 0) * DK + c] = glc * d1[i].x;
+            sm.dSgT[(q + 1) * DK + c] = glc * d1[i].y;
+            sm.dSgT[(q + 2) * DK + c] = glc * d1[i].z;
+            sm.dSgT[(q + 3) * DK + c] = glc * d1[i].w;
             dgl[i] += d1[i].x * s1[i].x + d1[i].y * s1[i].y + d1[i].z * s1[i].z + d1[i].w * s1[i].w;
         }
         {
-            const int e = rr * NVP + c4;
+            const int e = rr * NV + c4;
             const float b = sm.beta[rr];
-            auto put = [&](float* t, const float4& x4) {
-                t[e] = x4.x;
-                t[e + 1] = x4.y;
-                t[e + 2] = x4.z;
-                t[e + 3] = x4.w;
-            };
-            put(sm.dO, o4);
-            put(sm.U, u4);
-            put(sm.dU, du4);
-            put(sm.dX, make_float4(-b * dy4.x, -b * dy4.y, -b * dy4.z, -b * dy4.w));
-            put(sm.Y, make_float4(b * vx4.x, b * vx4.y, b * vx4.z, b * vx4.w));
+            *reinterpret_cast<float4*>(sm.dO + e) = o4;
+            *reinterpret_cast<float4*>(sm.U + e) = u4;
+            *reinterpret_cast<float4*>(sm.dU + e) = du4;
+            *reinterpret_cast<float4*>(sm.dX + e) = make_float4(-b * dy4.x, -b * dy4.y, -b * dy4.z, -b * dy4.w);
+            sm.UT[(c4 + 0) * C + rr] = u4.x;
+            sm.UT[(c4 + 1) * C + rr] = u4.y;
+            sm.UT[(c4 + 2) * C + rr] = u4.z;
+            sm.UT[(c4 + 3) * C + rr] = u4.w;
+            sm.YT[(c4 + 0) * C + rr] = b * vx4.x;
+            sm.YT[(c4 + 1) * C + rr] = b * vx4.y;
+            sm.YT[(c4 + 2) * C + rr] = b * vx4.z;
+            sm.YT[(c4 + 3) * C + rr] = b * vx4.w;
             db1 += vx4.x * dy4.x + vx4.y * dy4.y + vx4.z * dy4.z + vx4.w * dy4.w;
         }
         __syncthreads();
         // a_q += dO Sm^T, a_k += dX Sm^T, a_n += U dSg^T; dP += dO U^T, dT += dU Y^T
-        mma_tile<4, TK>(aq, sm.dO, NVP, 1, sm.Sm, 1, NVP, NV, tm, 16, tn, 16);
-        mma_tile<4, TK>(ak, sm.dX, NVP, 1, sm.Sm, 1, NVP, NV, tm, 16, tn, 16);
-        mma_tile<4, TK>(an, sm.U, NVP, 1, sm.dSg, 1, NVP, NV, tm, 16, tn, 16);
-        mma_tile<4, 4>(dp, sm.dO, NVP, 1, sm.U, 1, NVP, NV, tm, 16, tn, 16);
-        mma_tile<4, 4>(dt, sm.dU, NVP, 1, sm.Y, 1, NVP, NV, tm, 16, tn, 16);
+        mma_rk<4, TK>(aq, sm.dO, NV, sm.SmT, DK, NV, m0, n0);
+        mma_rk<4, TK>(ak, sm.dX, NV, sm.SmT, DK, NV, m0, n0);
+        mma_rk<4, TK>(an, sm.U, NV, sm.dSgT, DK, NV, m0, n0);
+        mma_rk<4, 4>(dp, sm.dO, NV, sm.UT, C, NV, m0, s0c);
+        mma_rk<4, 4>(dt, sm.dU, NV, sm.YT, C, NV, m0, s0c);
     }
     // dP (lower incl.) -> D1, dT -> D2; dgl and the first part of dbeta
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int r = tm + 16 * i;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int s = tn + 16 * j;
-            sm.D1[r * LDC + s] = s <= r ? dp[i][j] : 0.f;
-            sm.D2[r * LDC + s] = dt[i][j];
-        }
+        const int r = m0 + i;
+        float4 a4, b4;
+        a4.x = s0c + 0 <= r ? dp[i][0] : 0.f;
+        a4.y = s0c + 1 <= r ? dp[i][1] : 0.f;
+        a4.z = s0c + 2 <= r ? dp[i][2] : 0.f;
+        a4.w = s0c + 3 <= r ? dp[i][3] : 0.f;
+        b4 = make_float4(dt[i][0], dt[i][1], dt[i][2], dt[i][3]);
+        *reinterpret_cast<float4*>(sm.D1 + r * C + s0c) = a4;
+        *reinterpret_cast<float4*>(sm.D2 + r * C + s0c) = b4;
     }
     {   // the 4 threads of a row are consecutive lanes
         float b = db1;
@@ -676,59 +690,71 @@ bwd_grad_kernel(const Params p)
         if ((tid & 3) == 0) sm.dgl[(tid + i * NT) / 4] = g;
     }
     __syncthreads();
-    // a_q += dP K~n; a_n += dP^T Q~
-    mma_tile<4, TK>(aq, sm.D1, LDC, 1, sm.kf, LDK, 1, C, tm, 16, tn, 16);
-    mma_tile<4, TK>(an, sm.D1, 1, LDC, sm.qm, LDK, 1, C, tm, 16, tn, 16);
-    {   // T^T dT
+    // a_q += dP K~n; a_n += dP^T Q~; T^T dT
+    mma_rk<4, TK>(aq, sm.D1, C, sm.kf, DK, C, m0, n0);
+    mma_tk<4, TK>(an, sm.D1, C, sm.qm, DK, C, m0, n0);
+    {
         float z[4][4] = {};
-        mma_tile<4, 4>(z, sm.T, 1, LDC, sm.D2, LDC, 1, C, tm, 16, tn, 16);
-        __syncthreads();
+        mma_tk<4, 4>(z, sm.T, C, sm.D2, C, C, m0, s0c);
+        __syncthreads();   // dP and dT are read
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) sm.D1[(tm + 16 * i) * LDC + tn + 16 * j] = z[i][j];
+            *reinterpret_cast<float4*>(sm.D1 + (m0 + i) * C + s0c) = make_float4(z[i][0], z[i][1], z[i][2], z[i][3]);
     }
     __syncthreads();
     {   // dA = -strictly-lower((T^T dT) T^T); dbeta += rowsum(MA dA); dMA = beta dA -> D2
         float da[4][4] = {};
-        mma_tile<4, 4>(da, sm.D1, LDC, 1, sm.T, 1, LDC, C, tm, 16, tn, 16);
+        mma_rk<4, 4>(da, sm.D1, C, sm.TT, C, C, m0, s0c);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int r = tm + 16 * i;
-            float part = 0.f;
+            const int r = m0 + i;
+            const float4 ma = *reinterpret_cast<const float4*>(sm.MA + r * C + s0c);
+            float a[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int s = tn + 16 * j;
-                const float a = s < r ? -da[i][j] : 0.f;
-                part = fmaf(sm.MA[r * LDC + s], a, part);
-                sm.D2[r * LDC + s] = sm.beta[r] * a;
-            }
+            for (int j = 0; j < 4; ++j) a[j] = s0c + j < r ? -da[i][j] : 0.f;
+            const float part = ma.x * a[0] + ma.y * a[1] + ma.z * a[2] + ma.w * a[3];
+            const float br = sm.beta[r];
+            *reinterpret_cast<float4*>(sm.D2 + r * C + s0c) = make_float4(br * a[0], br * a[1], br * a[2], br * a[3]);
             const float b = sum16(part);
             if (tn == 0) sm.db[r] += b;
         }
     }
     __syncthreads();
     // a_k += dMA K~n; a_n += dMA^T K~
-    mma_tile<4, TK>(ak, sm.D2, LDC, 1, sm.kf, LDK, 1, C, tm, 16, tn, 16);
-    mma_tile<4, TK>(an, sm.D2, 1, LDC, sm.km, LDK, 1, C, tm, 16, tn, 16);
+    mma_rk<4, TK>(ak, sm.D2, C, sm.kf, DK, C, m0, n0);
+    mma_tk<4, TK>(an, sm.D2, C, sm.km, DK, C, m0, n0);
     // dG = Q~ a_q + K~ a_k - K~n a_n into qm (each thread rewrites only the
     // elements it reads; no product reads Q~ any more); dq = E a_q,
     // dk = E a_k + a_n / E
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int r = tm + 16 * i;
+        const int r = m0 + i;
+        float qv[TK], kv[TK], fv[TK];
+        simt::ld_row<TK>(qv, sm.qm + r * DK + n0);
+        simt::ld_row<TK>(kv, sm.km + r * DK + n0);
+        simt::ld_row<TK>(fv, sm.kf + r * DK + n0);
+        float g[TK];
 #pragma unroll
-        for (int j = 0; j < TK; ++j) {
-            const int c = tn + 16 * j;
-            const float g = sm.qm[r * LDK + c] * aq[i][j] + sm.km[r * LDK + c] * ak[i][j] -
-                            sm.kf[r * LDK + c] * an[i][j];
-            sm.qm[r * LDK + c] = g;
-            if (r < L) {
-                const float e = fminf(fmaxf(rec[R::G + r * DK + c] - rec[R::G + (C / 2 - 1) * DK + c], -80.f), 80.f);
-                const float E = expf(e);
-                const size_t off = ((size_t)(x.tok + r) * H + h) * DK + c;
-                p.dq[off] = E * aq[i][j];
-                p.dk[off] = E * ak[i][j] + an[i][j] / E;
+        for (int j = 0; j < TK; ++j) g[j] = qv[j] * aq[i][j] + kv[j] * ak[i][j] - fv[j] * an[i][j];
+#pragma unroll
+        for (int j = 0; j < TK; j += 4)
+            *reinterpret_cast<float4*>(sm.qm + r * DK + n0 + j) = make_float4(g[j], g[j + 1], g[j + 2], g[j + 3]);
+        if (r < L) {
+            float gr[TK], gmid[TK];
+            simt::ld_row<TK>(gr, rec + R::G + r * DK + n0);
+            simt::ld_row<TK>(gmid, rec + R::G + (C / 2 - 1) * DK + n0);
+            float dqv[TK], dkv[TK];
+#pragma unroll
+            for (int j = 0; j < TK; ++j) {
+                const float E = expf(fminf(fmaxf(gr[j] - gmid[j], -80.f), 80.f));
+                dqv[j] = E * aq[i][j];
+                dkv[j] = E * ak[i][j] + an[i][j] / E;
+            }
+            const size_t off = ((size_t)(x.tok + r) * H + h) * DK + n0;
+#pragma unroll
+            for (int j = 0; j < TK; j += 4) {
+                *reinterpret_cast<float4*>(p.dq + off + j) = make_float4(dqv[j], dqv[j + 1], dqv[j + 2], dqv[j + 3]);
+                *reinterpret_cast<float4*>(p.dk + off + j) = make_float4(dkv[j], dkv[j + 1], dkv[j + 2], dkv[j + 3]);
             }
         }
     }
@@ -737,7 +763,7 @@ bwd_grad_kernel(const Params p)
         const int c = tid;
         float acc = sm.dgl[c];
         for (int r = L - 1; r >= 0; --r) {
-            acc += sm.qm[r * LDK + c];
+            acc += sm.qm[r * DK + c];
             p.dla[((size_t)(x.tok + r) * H + h) * DK + c] = acc;
         }
     }
