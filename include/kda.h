@@ -256,11 +256,14 @@ kda_status kda_recurrent_step_mode(const void* q, const void* k, const void* v,
  * Chunkwise backward pass: gradients of L = sum(o * grad_o) + sum(S_T * grad_final_state)
  * through kda_chunk_fwd's computation ("Hybrid Linear Attention Architecture:
  * Making LLM Training and Inference More Efficient", section IV: backpropagation
- * reuses the chunked structure of the forward pass).  It recomputes the
- * forward (the states entering every chunk go to the workspace), then walks
- * the chunks in reverse carrying the state's gradient, with the per-chunk
- * adjoint of the UT transform and of the gate factors.  fp32 arithmetic on
- * CUDA cores throughout; the plain layer only (no KDA_MODE_* variants).
+ * reuses the chunked structure of the forward pass).  Per (chunk, head) it
+ * forms the chunk's factors once; a forward walk stores the state entering
+ * every chunk, a reverse walk carries the state's gradient; the products that
+ * sum over value columns and the adjoint of the UT transform and of the gate
+ * factors then run per (chunk, head).  Everything between the launches lives
+ * in the workspace (one record of factors, the states, U, dU, dY, V - X and
+ * the state gradients per chunk).  fp32 arithmetic on CUDA cores throughout;
+ * the plain layer only (no KDA_MODE_* variants).
  *
  *   q, k, v, beta, log_alpha, initial_state: as in kda_chunk_fwd (dtype bf16 or fp32)
  *   grad_o           [B, T, H, dv] fp32
@@ -270,7 +273,12 @@ kda_status kda_recurrent_step_mode(const void* q, const void* k, const void* v,
  *   grad_beta        [B, T, H]     fp32, written
  *   grad_log_alpha   [B, T, H, dk] fp32, written
  *   grad_initial_state [B, H, dk, dv] fp32, or NULL if not wanted
- *   workspace        at least kda_chunk_bwd_workspace_size() bytes, 256-byte aligned
+ *   workspace        at least kda_chunk_bwd_workspace_size() bytes, 256-byte aligned,
+ *                    owned by the caller, not read across calls.  Undersized,
+ *                    missing or unaligned: KDA_ERR_INVALID_ARG before any launch.
+ * Packed batches: a sequence whose token range leaves [0, T) is skipped (zero
+ * gradients for its rows except grad_v, which is not written; its initial
+ * state gradient is grad_final_state) and reported by the next kda_check().
  * All tensor pointers 16-byte aligned (beta, grad_beta: 4).  d_k, d_v in
  * {64, 128}, chunk 64.  The gradient buffers must not alias the inputs.
  */
