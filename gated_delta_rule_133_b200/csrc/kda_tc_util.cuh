@@ -1,6 +1,6 @@
-// Building blocks shared by the tensor-core chunk kernels: the UT-transform
-// inversion on CUDA cores, operand descriptors and layouts, sequence ordering
-// and the TMA tensor maps of the [tokens, H, d] inputs.
+// Building blocks of the tensor-core chunk kernels: operand descriptors and
+// layouts, the hardware reciprocal, and the TMA tensor maps of the
+// [tokens, H, d] inputs.
 #pragma once
 
 #include "kda_sm100.cuh"
@@ -21,7 +21,6 @@ namespace tcu {
 using namespace sm100;
 
 constexpr int C = 64;      // chunk length
-constexpr int LDA = 65;    // fp32 pitch of the UT-transform scratch
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* p)
 {
@@ -38,102 +37,6 @@ __device__ __forceinline__ float rcp_approx(float x)
     float y;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// T[k][j] of the unit lower-triangular T, kept transposed in the upper
-// triangle (diagonal included) of the UT scratch.
-__device__ __forceinline__ float Tget(const float* As, int k, int j) { return k >= j ? As[j * LDA + k] : 0.f; }
-
-// UT transform, run by the first 128 threads (named barrier 1; the other
-// warps are free meanwhile).  On entry As[r*LDA + s] (s < r) holds the
-// strictly lower A; on return As[j*LDA + s] (s >= j) holds T[s][j],
-// T = (I + A)^-1, with A left intact below the diagonal.  Diagonal 16x16
-// blocks by column-sweep forward substitution (one lane per column), then
-// T10 = -T11 A10 T00, T32 = -T33 A32 T22 (2x2 register tiles) and the
-// lower-left 32x32 block -T_BB A_BA T_AA (2x4 register tiles).
-__device__ __forceinline__ void ut_transform(float* As, float* X)
-{
-    const int tid = threadIdx.x;
-    if (tid < 64) {
-        const int b0 = 16 * (tid >> 4), j = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-        for (int s = 0; s < 15; ++s) {
-            const float xs = x[s];
-#pragma unroll
-            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-As[(b0 + r) * LDA + b0 + s], xs, x[r]);
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r)
-            if (r >= j) As[(b0 + j) * LDA + b0 + r] = x[r];
-    }
-    bar_sync(1, 128);
-    {
-        const int blk = tid >> 6, tile = tid & 63, i0 = (tile >> 3) * 2, j0 = (tile & 7) * 2;
-        const int rb = blk ? 48 : 16, cb = blk ? 32 : 0;
-        float a[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float u0 = As[(rb + i0) * LDA + cb + k], u1 = As[(rb + i0 + 1) * LDA + cb + k];
-            const float t0 = Tget(As, cb + k, cb + j0), t1 = Tget(As, cb + k, cb + j0 + 1);
-            a[0][0] = fmaf(u0, t0, a[0][0]); a[0][1] = fmaf(u0, t1, a[0][1]);
-            a[1][0] = fmaf(u1, t0, a[1][0]); a[1][1] = fmaf(u1, t1, a[1][1]);
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < 2; ++v) X[(blk * 16 + i0 + u) * 33 + j0 + v] = a[u][v];
-        bar_sync(1, 128);
-        float t[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float w0 = Tget(As, rb + i0, rb + k), w1 = Tget(As, rb + i0 + 1, rb + k);
-            const float x0 = X[(blk * 16 + k) * 33 + j0], x1 = X[(blk * 16 + k) * 33 + j0 + 1];
-            t[0][0] = fmaf(w0, x0, t[0][0]); t[0][1] = fmaf(w0, x1, t[0][1]);
-            t[1][0] = fmaf(w1, x0, t[1][0]); t[1][1] = fmaf(w1, x1, t[1][1]);
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < 2; ++v) As[(cb + j0 + v) * LDA + rb + i0 + u] = -t[u][v];
-    }
-    bar_sync(1, 128);
-    {
-        const int i0 = (tid >> 3) * 2, j0 = (tid & 7) * 4;
-        float a[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-            const float u0 = As[(32 + i0) * LDA + k], u1 = As[(32 + i0 + 1) * LDA + k];
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const float tv = Tget(As, k, j0 + v);
-                a[0][v] = fmaf(u0, tv, a[0][v]);
-                a[1][v] = fmaf(u1, tv, a[1][v]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < 4; ++v) X[(i0 + u) * 33 + j0 + v] = a[u][v];
-        bar_sync(1, 128);
-        float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-            const float w0 = Tget(As, 32 + i0, 32 + k), w1 = Tget(As, 32 + i0 + 1, 32 + k);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const float xv = X[k * 33 + j0 + v];
-                t[0][v] = fmaf(w0, xv, t[0][v]);
-                t[1][v] = fmaf(w1, xv, t[1][v]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < 4; ++v) As[(j0 + v) * LDA + 32 + i0 + u] = -t[u][v];
-    }
 }
 
 // K-major SW128 operand descriptor for MMA k-step kk (32 bytes of K per step:

@@ -161,3 +161,25 @@ def test_bwd_dirty_workspace_gives_identical_results():
     kda.kda_check()
     for a, b in zip(g1, g2):
         assert torch.equal(a, b)
+
+
+def test_varlen_bwd_many_packed_sequences():
+    """Several hundred packed sequences, lengths 0, 1, 63, 64 and 65 among them."""
+    rng = np.random.default_rng(360)
+    lens = [int(x) for x in rng.integers(0, 150, size=300)]
+    for i, L in enumerate((0, 1, 63, 64, 65, 128, 129)):
+        lens[(i * 41) % len(lens)] = L
+    cu = cu_from_lengths(lens)
+    H, d = 2, 64
+    t = draw_tokens(int(cu[-1]), H, d, d, "bf16", -3.0, 361, "cpu", init_states=len(lens), init_std=0.05)
+    g = torch.Generator().manual_seed(362)
+    do = torch.randn(int(cu[-1]), H, d, generator=g)
+    dsT = torch.randn(len(lens), H, d, d, generator=g)
+    dev = {n: (None if v is None else v.to(DEV)) for n, v in t.items()}
+    got = kda.kda_varlen_bwd(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_alpha"],
+                             torch.from_numpy(cu).to(DEV), dev["initial_state"], do.to(DEV), dsT.to(DEV))
+    torch.cuda.synchronize()
+    kda.kda_check()
+    ref = backward.recurrence_backward(f64(t["q"]), f64(t["k"]), f64(t["v"]), f64(t["beta"]), f64(t["log_alpha"]),
+                                       cu, f64(t["initial_state"]), f64(do), f64(dsT))
+    _check([f64(x) for x in got], ref)

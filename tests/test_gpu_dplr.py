@@ -121,3 +121,38 @@ def test_dplr_dirty_workspace_gives_identical_results():
     torch.cuda.synchronize()
     kda.kda_check()
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_dplr_bf16_output_is_the_rounded_fp32_output():
+    """o_dtype=bf16 stores exactly the fp32 result rounded to nearest even."""
+    B, T, H, d = 1, 200, 2, 128
+    x = draw_tokens(B * T, H, d, d, "bf16", -3.0, 550, "cpu", init_states=B, init_std=0.05)
+    a, b = _ab(B * T, H, d, "bf16", 551)
+    r = lambda t: t.reshape(B, T, *t.shape[1:]).to(DEV)
+    args = (r(x["q"]), r(x["k"]), r(x["v"]), r(a), r(b), r(x["log_alpha"]), x["initial_state"].to(DEV))
+    o32, s32 = kda.kda_dplr_fwd(*args)
+    o16, s16 = kda.kda_dplr_fwd(*args, o_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    kda.kda_check()
+    assert o16.dtype == torch.bfloat16 and torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(s16, s32)
+
+
+def test_dplr_many_packed_sequences():
+    """Several hundred packed sequences, lengths 0, 1, 63, 64 and 65 among them."""
+    rng = np.random.default_rng(560)
+    lens = [int(x) for x in rng.integers(0, 150, size=300)]
+    for i, L in enumerate((0, 1, 63, 64, 65, 128, 129)):
+        lens[(i * 41) % len(lens)] = L
+    cu = cu_from_lengths(lens)
+    H, d = 2, 64
+    x = draw_tokens(int(cu[-1]), H, d, d, "bf16", -3.0, 561, "cpu", init_states=len(lens), init_std=0.05)
+    a, b = _ab(int(cu[-1]), H, d, "bf16", 562)
+    o, sN = kda.kda_dplr_varlen_fwd(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), a.to(DEV), b.to(DEV),
+                                    x["log_alpha"].to(DEV), torch.from_numpy(cu).to(DEV), x["initial_state"].to(DEV))
+    torch.cuda.synchronize()
+    kda.kda_check()
+    o_ref, s_ref = dplr.recurrence(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(a), f64(b), f64(x["log_alpha"]), cu,
+                                   f64(x["initial_state"]))
+    assert norm_max_err(f64(o), o_ref) <= TOL
+    assert norm_max_err(f64(sN), s_ref) <= TOL
