@@ -12,7 +12,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkda.so")
 
-KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_WARN_DOMAIN = range(6)
 KDA_F32, KDA_BF16 = 0, 1
 KDA_MODE_HEAD_GATE, KDA_MODE_NO_ERASE, KDA_MODE_NORM_QK, KDA_MODE_GATE_LOGITS = 1, 2, 4, 8
 KDA_MODE_CUDA_CORES = 16

@@ -408,6 +408,7 @@ kda_status kda_check(void* stream)
         return KDA_ERR_CUDA;
     if (word & kda::KDA_DEV_ERR_TIMEOUT) return KDA_ERR_TIMEOUT;
     if (word & kda::KDA_DEV_ERR_BAD_INPUT) return KDA_ERR_INVALID_ARG;
+    if (word & kda::KDA_DEV_WARN_DOMAIN) return KDA_WARN_DOMAIN;
     return KDA_OK;
 }
 
@@ -426,6 +427,8 @@ const char* kda_status_string(kda_status status)
     case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: size or type not implemented";
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA runtime call or kernel launch failed";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a device-side bounded wait ran out";
+    case KDA_WARN_DOMAIN:
+        return "KDA_WARN_DOMAIN: a chunk's gate decay left the mid-chunk factorisation range (results inexact)";
     }
     return "KDA_ERR_UNKNOWN";
 }

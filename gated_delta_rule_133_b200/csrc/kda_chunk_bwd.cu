@@ -202,6 +202,7 @@ bwd_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const Pa
             rec[R::G + r * DK + c] = acc;
         }
         const float Gm = sm.kf[(C / 2 - 1) * LDK + c];
+        check_domain(sm.kf[c], Gm, acc);
         const float vg[3] = {expf(Gm), expf(acc), expf(acc - Gm)};
 #pragma unroll
         for (int u = 0; u < 3; ++u) {

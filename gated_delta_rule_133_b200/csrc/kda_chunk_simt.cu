@@ -134,13 +134,13 @@ __device__ __forceinline__ void mma_rk(float (&acc)[TM][TN], const float* A, int
 }
 
 // acc[i][j] += sum_kk A[kk * lda + m0 + i] * B[kk * ldb + n0 + j]: the same
-// with A stored transposed (K rows of M), read TM values at a time (m0 and lda
-// multiples of 4).
+// with A stored transposed (K rows of M), read TM values at a time (TM = 2, 4
+// or 8; A's row segments aligned as for ld_row).
 template <int TM, int TN>
 __device__ __forceinline__ void mma_tk(float (&acc)[TM][TN], const float* A, int lda, const float* B, int ldb, int K,
                                        int m0, int n0)
 {
-    static_assert(TN % 2 == 0 && TM % 4 == 0, "columns in pairs, rows in fours");
+    static_assert(TN % 2 == 0 && (TM == 2 || TM % 4 == 0), "columns in pairs, rows in pairs or fours");
 #pragma unroll 4
     for (int kk = 0; kk < K; ++kk) {
         float a[TM], b[TN];
@@ -260,6 +260,7 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
             for (int r = 0; r < C; ++r) { acc += sm.kf[r * LDK + c]; sm.kf[r * LDK + c] = acc; }
             const float Gm = sm.kf[(C / 2 - 1) * LDK + c];
             const float Gl = acc;
+            check_domain(sm.kf[c], Gm, Gl);
             sm.gm[c] = expf(Gm);
             sm.gam[c] = expf(Gl);
             sm.glm[c] = expf(Gl - Gm);

@@ -290,6 +290,7 @@ __device__ __forceinline__ void cumsum384(float* gs, const Vec& v, int L, int t,
         }
     }
     bar_sync(2, 384);
+    if (part == 0 && ch < DK) check_domain(gs[ch], v.gml[ch], gs[(C - 1) * DK + ch]);
 }
 
 // Gate cumsum of one gate per (token, head), by 384 threads (named barrier 2):
@@ -331,6 +332,7 @@ __device__ __forceinline__ void cumsum_head384(float* gs, const Vec& v, int L, i
         v.gm[t] = expf(Gm);
         v.glm[t] = expf(Gl - Gm);
         v.egl[t] = expf(Gl);
+        if (t == 0) check_domain(gs[0], Gm, Gl);
     }
     bar_sync(2, 384);
 }

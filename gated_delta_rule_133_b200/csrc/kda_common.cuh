@@ -13,13 +13,22 @@ namespace kda {
 // Per-device status word (the library is one translation unit, so this is its
 // only definition).  Kernels set bits here when a bounded wait gives up or
 // when device-resident arguments (sequence boundaries) fall outside the
-// buffers they index, in which case the affected sequence is skipped;
+// buffers they index, in which case the affected sequence is skipped, or
+// when a chunk's gate decay leaves the range of the mid-chunk factorisation;
 // kda_check() reads and clears it.
-enum : unsigned { KDA_DEV_ERR_TIMEOUT = 1u, KDA_DEV_ERR_BAD_INPUT = 2u };
+enum : unsigned { KDA_DEV_ERR_TIMEOUT = 1u, KDA_DEV_ERR_BAD_INPUT = 2u, KDA_DEV_WARN_DOMAIN = 4u };
 __device__ unsigned g_status = 0;
 
 __device__ __forceinline__ void flag_timeout() { atomicOr(&g_status, KDA_DEV_ERR_TIMEOUT); }
 __device__ __forceinline__ void flag_bad_input() { atomicOr(&g_status, KDA_DEV_ERR_BAD_INPUT); }
+
+// Factors exp(G - G_m) of a chunk are clamped at exp(+-80); G is monotone
+// (log alpha <= 0), so for one channel the extremes are the first row, G_0,
+// and the last, G_last.  Flags the chunk when either lies outside the clamp.
+__device__ __forceinline__ void check_domain(float g0, float gm, float glast)
+{
+    if (g0 - gm > 80.f || gm - glast > 80.f) atomicOr(&g_status, KDA_DEV_WARN_DOMAIN);
+}
 
 // Element access for the two supported q/k/v/o element types.
 template <typename T> struct Elem;

@@ -75,6 +75,9 @@ struct FacSmem {
     float qx[C * LDK];    // q e^{G - G_m}
     float M[C * LDC];     // A_ab
     float T[C * LDC];     // (I - A_ab)^-1
+    float part[NT];       // per-part gate sums of the cumsum
+    float gmid[DK];       // G of the middle row
+    float glast[DK];      // G of the last row
 };
 
 template <typename TIn, int DK>
@@ -100,20 +103,39 @@ dplr_factor_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
         packed::load_rows<TIn, DK, NT>(sm.qx, LDK, q + row0, stride, L);
     }
     __syncthreads();
-    if (tid < DK) {   // gate cumsum per channel (fp32, log space), factors and the record's scaled rows
-        const int c = tid;
-        float G[C];
+    {   // gate cumsum per channel (fp32, log space), factors and the record's
+        // scaled rows: thread (part, c) takes rows [part RP, (part + 1) RP) of
+        // channel c; the part sums are added in part order
+        constexpr int NP = NT / DK, RP = C / NP;
+        const int c = tid % DK, part = tid / DK, r0 = part * RP;
+        float G[RP];
         float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < C; ++r) {
-            acc += r < L ? p.log_alpha[((size_t)(x.tok + r) * H + h) * DK + c] : 0.f;
-            G[r] = acc;
+        for (int rr = 0; rr < RP; ++rr) {
+            acc += r0 + rr < L ? p.log_alpha[((size_t)(x.tok + r0 + rr) * H + h) * DK + c] : 0.f;
+            G[rr] = acc;
         }
-        const float Gm = G[C / 2 - 1], Gl = G[C - 1];
-        rec[R::GAM + c] = expf(Gl);
+        sm.part[tid] = acc;
+        __syncthreads();
+        float off = 0.f;   // G of the row before this part
+        for (int q2 = 0; q2 < part; ++q2) off += sm.part[q2 * DK + c];
 #pragma unroll
-        for (int r = 0; r < C; ++r) {
-            const float g = G[r], gx = r ? G[r - 1] : 0.f;
+        for (int rr = 0; rr < RP; ++rr) G[rr] += off;
+#pragma unroll
+        for (int rr = 0; rr < RP; ++rr) {
+            if (r0 + rr == C / 2 - 1) sm.gmid[c] = G[rr];
+            if (r0 + rr == C - 1) sm.glast[c] = G[rr];
+        }
+        __syncthreads();
+        const float Gm = sm.gmid[c], Gl = sm.glast[c];
+        if (part == 0) {
+            rec[R::GAM + c] = expf(Gl);
+            check_domain(G[0], Gm, Gl);
+        }
+#pragma unroll
+        for (int rr = 0; rr < RP; ++rr) {
+            const int r = r0 + rr;
+            const float g = G[rr], gx = rr ? G[rr - 1] : off;
             const float f = expf(fminf(Gm - g, 80.f));
             const float av = sm.ax[r * LDK + c], bv = sm.bf[r * LDK + c], kv = sm.kf[r * LDK + c];
             const float qv = sm.qx[r * LDK + c];

@@ -45,7 +45,9 @@
  *    factored around the chunk's middle token; that requires the decay of any
  *    32 consecutive tokens of one channel to stay below about 80 nats
  *    (average alpha above ~0.08).  Stronger gates lose accuracy in the
- *    intra-chunk terms (results stay finite).  The tensor-core path rounds
+ *    intra-chunk terms (results stay finite); the chunk kernels detect it per
+ *    (chunk, channel) and kda_check() then reports KDA_WARN_DOMAIN.  The
+ *    decode step has no such limit.  The tensor-core path rounds
  *    its operands to fp16: entries of e^G q, e^G k, the state, beta (v - k S)
  *    and of the intra-chunk inverse (I + A)^-1 must stay below 65504 in
  *    magnitude.  With keys of norm at most 1 and beta <= 1 the inverse's
@@ -66,7 +68,9 @@ typedef enum {
     KDA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size          */
     KDA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (d, chunk, dtype)  */
     KDA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed         */
-    KDA_ERR_TIMEOUT = 4       /* a device-side bounded wait ran out           */
+    KDA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out           */
+    KDA_WARN_DOMAIN = 5       /* a chunk's gate decay left the factorisation
+                                 range: results are finite but inexact      */
 } kda_status;
 
 typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
@@ -356,7 +360,9 @@ kda_status kda_dplr_varlen_fwd_workspace_size(int N, int T, int H, int dk, int d
  * status word: KDA_ERR_TIMEOUT if a device-side bounded wait ran out since the
  * last check, KDA_ERR_INVALID_ARG if a kernel found device-resident sequence
  * boundaries (cu_seqlens) outside the token range and skipped that sequence,
- * KDA_ERR_CUDA if the stream reports an error, else KDA_OK.
+ * KDA_WARN_DOMAIN if a chunk kernel met a gate outside the numerical domain
+ * (see "Numerical domain" above), KDA_ERR_CUDA if the stream reports an error,
+ * else KDA_OK (in that order of precedence).
  */
 kda_status kda_check(void* stream);
 

@@ -27,8 +27,9 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_status_strings_and_version():
-    for st in range(5):
+    for st in range(6):
         assert _lib.status_string(st).startswith("KDA_")
+    assert "WARN_DOMAIN" in _lib.status_string(_lib.KDA_WARN_DOMAIN)
     assert "UNKNOWN" in _lib.status_string(99)
     assert _lib.load().kda_version() >= 100
 
