@@ -16,12 +16,20 @@
 //   O      = (exp(G) * Q) S + Tril_incl(P) V',   P[r,s] = sum_c q_rc k_sc exp(G_rc - G_sc)
 //   S     <- Diag(gamma) S + (exp(G_last - G) * K)^T V'
 //
-// Relative decays exp(G_r - G_s) are factored around the chunk's middle row m
-// ("segmenting intra-chunk cumulative gates"): E = exp(G - G_m) on the row
-// side and F = exp(G_m - G) on the column side, so every factor is bounded
-// by the decay of 32 tokens instead of a whole chunk.  Then
-// exp(G) = exp(G_m) E and exp(G_last - G) = exp(G_last - G_m) F, and the
-// per-channel factors exp(G_m), exp(G_last - G_m) are folded into the state.
+// The intra-chunk decays exp(G_r - G_s) of P and A are split so that no
+// factor overflows ("segmenting intra-chunk cumulative gates"):
+//  - when every channel decays at most 80 nats from the chunk's first row to
+//    its middle row m and from m to its last row, at m: e^(G_r - G_m) on the
+//    row side, e^(G_m - G_s) on the column side, each at most e^80;
+//  - otherwise by 16-row blocks (the sub-block references of the chunk
+//    algorithm): row block I against the columns s < 16 I at row 16 I,
+//    e^(G_r - G_16I) e^(G_16I - G_s), both factors at most 1 and each at least
+//    the product, and the diagonal 16 x 16 blocks with e^(G_r - G_s) per
+//    element.  These factors use the fast exponential __expf (CUDA documents
+//    its error as 2 + floor(1.173 |x|) ulp: below 6e-6 relative for the
+//    |x| < 88 whose results are not flushed to zero).
+// The state-side operands q e^G, k e^G and k e^(G_last - G) have factors at
+// most 1.  So this path has no limit on the gates' strength.
 //
 // One CTA (256 threads) per (sequence, head, 32-column slice of d_v); the
 // columns of S evolve independently because the transition acts on the d_k
@@ -36,6 +44,7 @@ namespace simt {
 constexpr int C = 64;       // chunk length
 constexpr int NV = 32;      // value columns per CTA
 constexpr int NT = 256;     // threads per CTA
+constexpr float kMidRange = 80.f;   // largest decay (nats) the middle-row split takes
 
 // (d0, d1) = (x0 * y0 + d0, x1 * y1 + d1) as one packed fp32x2 FMA; each
 // lane rounds exactly as fmaf does.
@@ -157,67 +166,128 @@ template <int DK>
 struct Smem {
     static constexpr int LDK = DK + 1;   // padded row pitch of the [C][DK] tiles
     static constexpr int LDC = C + 1;    // padded pitch of the [C][C] tiles
-    float qm[C * LDK];    // q * E
-    float km[C * LDK];    // k * E
-    float kf[C * LDK];    // cumulative gate G, then k * F
+    static constexpr int LDX = DK + 4;   // pitch of the 16-row blocks' operands (16-byte rows)
+    static constexpr int XROWS = 56;     // 32 row-block operand rows + up to 24 column rows
+    float qm[C * LDK];    // q * E (segmented chunks: q e^G)
+    float km[C * LDK];    // k * E (segmented chunks: k e^G)
+    float kf[C * LDK];    // cumulative gate G, then k * F (segmented chunks: k e^(G_last - G))
     float A[C * LDC];
     float P[C * LDC];
-    float T[C * LDC];
-    float S[DK * NV];     // state slice, fp32, carried across chunks
+    float T[C * LDC];     // T, and with Sm the operands of the 16-row blocks (free until the UT transform)
     float Sm[DK * NV];    // exp(G_m) * S for the current chunk
+    float S[DK * NV];     // state slice, fp32, carried across chunks
     float V[C * NV];      // values, then Y = beta (V - X)
     float Vp[C * NV];     // V' = T Y
-    float gm[DK];         // exp(G_m)
+    float gm[DK];         // exp(G_m) (segmented chunks: 1)
     float gam[DK];        // exp(G_last)
-    float glm[DK];        // exp(G_last - G_m)
+    float glm[DK];        // exp(G_last - G_m) (segmented chunks: 1)
+    float gl[DK];         // G_last
     float beta[C];
 };
 
-template <typename TIn, typename TOut, int DK>
-__global__ void __launch_bounds__(NT)
-chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
-                      const TIn* __restrict__ v, const float* __restrict__ beta,
-                      const float* __restrict__ log_alpha, const float* s0, TOut* __restrict__ o,
-                      float* sT, const int32_t* __restrict__ cu, int nseq, int T, long long tokens, int H, int DV,
-                      int mode)
+// P, A of a chunk outside the middle-row split's range, by 16-row blocks, on
+// the raw q, k and the cumulative gates G in qm, km, kf; then the state-side
+// operands q e^G, k e^G and k e^(G_last - G) in their place, gm = glm = 1 and
+// Sm = S.  Row block I against the columns s < r0 = 16 I: the decay split at
+// row r0, the block operands in T and Sm (X rows 0..15 = q e^(G - G_r0), 16..31
+// = k e^(G - G_r0) of rows r0 .. r0 + 15; 32.. = k e^(G_r0 - G) of up to 24
+// columns at a time).  Diagonal 16 x 16 blocks with e^(G_r - G_s) per element.
+static_assert(offsetof(Smem<128>, Sm) == offsetof(Smem<128>, T) + sizeof(float) * C * Smem<128>::LDC &&
+              Smem<128>::XROWS * Smem<128>::LDX <= C * Smem<128>::LDC + 128 * NV &&
+              Smem<64>::XROWS * Smem<64>::LDX <= C * Smem<64>::LDC + 64 * NV,
+              "the 16-row blocks' operands fit in T and Sm");
+
+template <int DK>
+__device__ __forceinline__ void segmented_pa(Smem<DK>& sm, int tid, bool erase)
+{
+    constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC, LDX = Smem<DK>::LDX;
+    float* X = sm.T;
+    for (int e = tid; e < C * C; e += NT) {
+        sm.P[(e / C) * LDC + e % C] = 0.f;
+        sm.A[(e / C) * LDC + e % C] = 0.f;
+    }
+    for (int I = 1; I < C / 16; ++I) {
+        const int r0 = 16 * I;
+        for (int e = tid; e < 32 * DK; e += NT) {
+            const int row = e / DK, c = e % DK, r = r0 + (row & 15);
+            const float f = __expf(sm.kf[r * LDK + c] - sm.kf[r0 * LDK + c]);
+            X[row * LDX + c] = (row < 16 ? sm.qm[r * LDK + c] : sm.km[r * LDK + c]) * f;
+        }
+        for (int s0 = 0; s0 < r0; s0 += 24) {
+            const int ns = min(24, r0 - s0);
+            for (int e = tid; e < ns * DK; e += NT) {
+                const int sr = s0 + e / DK, c = e % DK;
+                X[(32 + e / DK) * LDX + c] = sm.km[sr * LDK + c] * __expf(sm.kf[r0 * LDK + c] - sm.kf[sr * LDK + c]);
+            }
+            __syncthreads();
+            for (int ix = tid; ix < 16 * ns; ix += NT) {
+                const int r = ix / ns, j = ix % ns;
+                const float4* xq = reinterpret_cast<const float4*>(X + r * LDX);
+                const float4* xk = reinterpret_cast<const float4*>(X + (16 + r) * LDX);
+                const float4* xc = reinterpret_cast<const float4*>(X + (32 + j) * LDX);
+                float p = 0.f, a = 0.f;
+#pragma unroll 4
+                for (int c4 = 0; c4 < DK / 4; ++c4) {
+                    const float4 u = xq[c4], w = xk[c4], z = xc[c4];
+                    p = fmaf(u.x, z.x, p); p = fmaf(u.y, z.y, p); p = fmaf(u.z, z.z, p); p = fmaf(u.w, z.w, p);
+                    a = fmaf(w.x, z.x, a); a = fmaf(w.y, z.y, a); a = fmaf(w.z, z.z, a); a = fmaf(w.w, z.w, a);
+                }
+                sm.P[(r0 + r) * LDC + s0 + j] = p;
+                sm.A[(r0 + r) * LDC + s0 + j] = erase ? sm.beta[r0 + r] * a : 0.f;
+            }
+            __syncthreads();
+        }
+    }
+    for (int ix = tid; ix < (C / 16) * 136; ix += NT) {
+        int t = ix % 136, r = 0;
+        while (t > r) {   // (r, t): t-th entry of the lower-inclusive 16 x 16 triangle, row-major
+            t -= r + 1;
+            ++r;
+        }
+        const int R = 16 * (ix / 136) + r, Sc = R - r + t;
+        float p = 0.f, a = 0.f;
+        for (int c = 0; c < DK; ++c) {
+            const float kd = sm.km[Sc * LDK + c] * __expf(sm.kf[R * LDK + c] - sm.kf[Sc * LDK + c]);
+            p = fmaf(sm.qm[R * LDK + c], kd, p);
+            a = fmaf(sm.km[R * LDK + c], kd, a);
+        }
+        sm.P[R * LDC + Sc] = p;
+        sm.A[R * LDC + Sc] = (erase && t < r) ? sm.beta[R] * a : 0.f;
+    }
+    __syncthreads();
+    for (int e = tid; e < C * DK; e += NT) {
+        const int r = e / DK, c = e % DK;
+        const float g = sm.kf[r * LDK + c], kv = sm.km[r * LDK + c], eg = __expf(g);
+        sm.qm[r * LDK + c] *= eg;
+        sm.km[r * LDK + c] = kv * eg;
+        sm.kf[r * LDK + c] = kv * __expf(sm.gl[c] - g);
+    }
+    for (int e = tid; e < DK * NV; e += NT) sm.Sm[e] = sm.S[e];
+    if (tid < DK) {
+        sm.gm[tid] = 1.f;
+        sm.glm[tid] = 1.f;
+    }
+    __syncthreads();
+}
+
+// The chunk loop of one CTA from token t_begin of its sequence.  SEG = false:
+// every chunk takes the middle-row split, and the loop returns the offset of
+// the first chunk that the split cannot take (len if none) with that chunk's
+// state untouched; SEG = true: chunks outside its range are segmented by
+// 16-row blocks.  Two functions, so that the common loop is compiled alone.
+template <bool SEG, typename TIn, typename TOut, int DK>
+__device__ __noinline__ int chunk_loop(Smem<DK>& sm, const TIn* __restrict__ q, const TIn* __restrict__ k,
+                                       const TIn* __restrict__ v, const float* __restrict__ beta,
+                                       const float* __restrict__ log_alpha, TOut* __restrict__ o, int tok0,
+                                       int len, int t_begin, int H, int h, int DV, int col0, int mode)
 {
     const bool head_gate = (mode & KDA_MODE_HEAD_GATE) != 0;   // log_alpha [tokens, H]
     const bool erase = (mode & KDA_MODE_NO_ERASE) == 0;
     const bool logits = (mode & KDA_MODE_GATE_LOGITS) != 0;
     const bool norm_qk = (mode & KDA_MODE_NORM_QK) != 0;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    Smem<DK>& sm = *reinterpret_cast<Smem<DK>*>(smem_raw);
     constexpr int LDK = Smem<DK>::LDK, LDC = Smem<DK>::LDC;
-
-    const int nslice = DV / NV;
-    const int slice = blockIdx.x % nslice;
-    const int h = (blockIdx.x / nslice) % H;
-    const int rank = blockIdx.x / (nslice * H);
-    int n, tok0, len;
-    if (cu) {   // packed sequences in their own order; a range outside the token axis is skipped
-        n = rank;
-        tok0 = cu[n];
-        len = max(0, cu[n + 1] - tok0);
-        if (tok0 < 0 || (long long)tok0 + len > tokens) {   // no tokens read; final state = initial
-            if (threadIdx.x == 0) flag_bad_input();
-            tok0 = 0;
-            len = 0;
-        }
-    } else {
-        n = rank;
-        tok0 = n * T;
-        len = T;
-    }
-    const int col0 = slice * NV;
     const int tid = threadIdx.x;
-
-    // initial state slice
-    for (int e = tid; e < DK * NV; e += NT) {
-        const int c = e / NV, j = e % NV;
-        sm.S[e] = s0 ? s0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
-    }
-
-    for (int t0 = 0; t0 < len; t0 += C) {
+    for (int t0 = t_begin; t0 < len; t0 += C) {
         const int L = min(C, len - t0);
         __syncthreads();
         // ---- load the chunk (rows >= L are zero: no key, no value, no decay)
@@ -253,47 +323,61 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
             __syncthreads();
         }
 
-        // ---- gate cumsum per channel (fp32, log space) and the factor split
+        // ---- gate cumsum per channel (fp32, log space); does the chunk fit the middle-row split?
+        bool seg = false;
         if (tid < DK) {
             const int c = tid;
             float acc = 0.f;
             for (int r = 0; r < C; ++r) { acc += sm.kf[r * LDK + c]; sm.kf[r * LDK + c] = acc; }
             const float Gm = sm.kf[(C / 2 - 1) * LDK + c];
             const float Gl = acc;
-            check_domain(sm.kf[c], Gm, Gl);
             sm.gm[c] = expf(Gm);
             sm.gam[c] = expf(Gl);
             sm.glm[c] = expf(Gl - Gm);
-            for (int r = 0; r < C; ++r) {
-                const float G = sm.kf[r * LDK + c];
-                const float Er = expf(fminf(G - Gm, 80.f));
-                const float Fr = expf(fminf(Gm - G, 80.f));
-                sm.qm[r * LDK + c] *= Er;
-                const float kk = sm.km[r * LDK + c];
-                sm.km[r * LDK + c] = kk * Er;
-                sm.kf[r * LDK + c] = kk * Fr;
-            }
+            sm.gl[c] = Gl;
+            seg = sm.kf[c] - Gm > kMidRange || Gm - Gl > kMidRange;
         }
-        __syncthreads();
+        seg = __syncthreads_or(seg);
 
-        // ---- P = (q E)(k F)^T (lower incl.), A = beta (k E)(k F)^T (strictly lower)
-        {
-            const int tn = tid % 16, tm = tid / 16;
-            float p[4][4] = {}, a[4][4] = {};
-            mma_tile<4, 4>(p, sm.qm, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
-            mma_tile<4, 4>(a, sm.km, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int r = tm + 16 * i, s = tn + 16 * j;
-                    sm.P[r * LDC + s] = s <= r ? p[i][j] : 0.f;
-                    sm.A[r * LDC + s] = (erase && s < r) ? sm.beta[r] * a[i][j] : 0.f;
+        if (SEG && seg) {
+            segmented_pa<DK>(sm, tid, erase);
+        } else {
+            if (seg) return t0;   // first chunk the middle-row split cannot take
+            // ---- the factor split at the middle row m: E = e^(G - G_m), F = e^(G_m - G)
+            if (tid < DK) {
+                const int c = tid;
+                const float Gm = sm.kf[(C / 2 - 1) * LDK + c];
+                for (int r = 0; r < C; ++r) {
+                    const float G = sm.kf[r * LDK + c];
+                    const float Er = expf(fminf(G - Gm, 80.f));
+                    const float Fr = expf(fminf(Gm - G, 80.f));
+                    sm.qm[r * LDK + c] *= Er;
+                    const float kk = sm.km[r * LDK + c];
+                    sm.km[r * LDK + c] = kk * Er;
+                    sm.kf[r * LDK + c] = kk * Fr;
                 }
-            // Sm = exp(G_m) * S  (state rows scaled per key channel)
-            for (int e = tid; e < DK * NV; e += NT) sm.Sm[e] = sm.gm[e / NV] * sm.S[e];
+            }
+            __syncthreads();
+
+            // ---- P = (q E)(k F)^T (lower incl.), A = beta (k E)(k F)^T (strictly lower)
+            {
+                const int tn = tid % 16, tm = tid / 16;
+                float p[4][4] = {}, a[4][4] = {};
+                mma_tile<4, 4>(p, sm.qm, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
+                mma_tile<4, 4>(a, sm.km, LDK, 1, sm.kf, 1, LDK, DK, tm, 16, tn, 16);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int r = tm + 16 * i, s = tn + 16 * j;
+                        sm.P[r * LDC + s] = s <= r ? p[i][j] : 0.f;
+                        sm.A[r * LDC + s] = (erase && s < r) ? sm.beta[r] * a[i][j] : 0.f;
+                    }
+                // Sm = exp(G_m) * S  (state rows scaled per key channel)
+                for (int e = tid; e < DK * NV; e += NT) sm.Sm[e] = sm.gm[e / NV] * sm.S[e];
+            }
+            __syncthreads();
         }
-        __syncthreads();
 
         // ---- UT transform T = (I + A)^-1 by forward substitution: column j of T
         // depends only on column j of earlier rows; 4 lanes share one column.
@@ -368,6 +452,50 @@ chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
             }
         }
     }
+    return len;
+}
+
+template <typename TIn, typename TOut, int DK>
+__global__ void __launch_bounds__(NT)
+chunk_fwd_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                      const TIn* __restrict__ v, const float* __restrict__ beta,
+                      const float* __restrict__ log_alpha, const float* s0, TOut* __restrict__ o,
+                      float* sT, const int32_t* __restrict__ cu, int nseq, int T, long long tokens, int H, int DV,
+                      int mode)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    Smem<DK>& sm = *reinterpret_cast<Smem<DK>*>(smem_raw);
+
+    const int nslice = DV / NV;
+    const int slice = blockIdx.x % nslice;
+    const int h = (blockIdx.x / nslice) % H;
+    const int rank = blockIdx.x / (nslice * H);
+    int n, tok0, len;
+    if (cu) {   // packed sequences in their own order; a range outside the token axis is skipped
+        n = rank;
+        tok0 = cu[n];
+        len = max(0, cu[n + 1] - tok0);
+        if (tok0 < 0 || (long long)tok0 + len > tokens) {   // no tokens read; final state = initial
+            if (threadIdx.x == 0) flag_bad_input();
+            tok0 = 0;
+            len = 0;
+        }
+    } else {
+        n = rank;
+        tok0 = n * T;
+        len = T;
+    }
+    const int col0 = slice * NV;
+    const int tid = threadIdx.x;
+
+    // initial state slice
+    for (int e = tid; e < DK * NV; e += NT) {
+        const int c = e / NV, j = e % NV;
+        sm.S[e] = s0 ? s0[(((size_t)n * H + h) * DK + c) * DV + col0 + j] : 0.f;
+    }
+
+    const int t_seg = chunk_loop<false>(sm, q, k, v, beta, log_alpha, o, tok0, len, 0, H, h, DV, col0, mode);
+    if (t_seg < len) chunk_loop<true>(sm, q, k, v, beta, log_alpha, o, tok0, len, t_seg, H, h, DV, col0, mode);
     __syncthreads();
     if (sT)
         for (int e = tid; e < DK * NV; e += NT) {

@@ -41,13 +41,16 @@
  *    by kda_check().
  *  - Supported: d_k, d_v in {64, 128}, chunk == 64.  Other sizes return
  *    KDA_ERR_UNSUPPORTED.  No C++ exception crosses this interface.
- *  - Numerical domain: inside one 64-token chunk the per-channel decay is
- *    factored around the chunk's middle token; that requires the decay of any
- *    32 consecutive tokens of one channel to stay below about 80 nats
- *    (average alpha above ~0.08).  Stronger gates lose accuracy in the
- *    intra-chunk terms (results stay finite); the chunk kernels detect it per
- *    (chunk, channel) and kda_check() then reports KDA_WARN_DOMAIN.  The
- *    decode step has no such limit.  The tensor-core path rounds
+ *  - Numerical domain: the tensor-core chunk forward, the backward and the
+ *    DPLR forward factor the per-channel decay inside one 64-token chunk
+ *    around the chunk's middle token; that requires the decay of any 32
+ *    consecutive tokens of one channel to stay below about 80 nats (average
+ *    alpha above ~0.08).  Stronger gates lose accuracy in the intra-chunk
+ *    terms (results stay finite); those kernels detect it per (chunk,
+ *    channel) and kda_check() then reports KDA_WARN_DOMAIN.  The CUDA-core
+ *    chunk forward (fp32 inputs, or KDA_MODE_CUDA_CORES) splits the decay
+ *    by 16-token blocks with every factor at most 1 and has no such limit;
+ *    neither has the decode step.  The tensor-core path rounds
  *    its operands to fp16: entries of e^G q, e^G k, the state, beta (v - k S)
  *    and of the intra-chunk inverse (I + A)^-1 must stay below 65504 in
  *    magnitude.  With keys of norm at most 1 and beta <= 1 the inverse's

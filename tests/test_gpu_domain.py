@@ -1,12 +1,14 @@
 """GPU: gates at and past the edge of the chunk kernels' numerical domain.
 
-The chunk kernels factor the decay inside a 64-token chunk around its middle
-row, with the factors clamped at exp(+-80).  A chunk whose gates decay a
-channel by more than 80 nats between its first or last row and the middle is
-outside the domain: the kernels then flag the chunk, kda_check() reports
-KDA_WARN_DOMAIN, and the results stay finite but lose accuracy.  Inside the
-domain nothing is reported and the usual bars hold.  The decode step has no
-such limit.
+The tensor-core chunk forward, the backward and the DPLR forward factor the
+decay inside a 64-token chunk around its middle row, with the factors clamped
+at exp(+-80).  A chunk whose gates decay a channel by more than 80 nats
+between its first or last row and the middle is outside their domain: the
+kernels then flag the chunk, kda_check() reports KDA_WARN_DOMAIN, and the
+results stay finite but lose accuracy.  Inside the domain nothing is reported
+and the usual bars hold.  The CUDA-core chunk forward splits the decay by
+16-row blocks with every factor at most 1, and the decode step needs no
+factors: neither has a limit.
 
 Gates here are a constant log alpha = -s on every channel, so the decay from
 the first row to the middle row (31 tokens) is 31 s nats.
@@ -39,9 +41,10 @@ def _oracle(x):
                              flat(x["log_alpha"]), np.array([0, T]), f64(x["initial_state"]))
 
 
-def _run_fwd(x):
+def _run_fwd(x, cuda_cores=False):
     g = {n: (None if t is None else t.to(DEV)) for n, t in x.items()}
-    o, sT = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"])
+    o, sT = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["log_alpha"], g["initial_state"],
+                              cuda_cores=cuda_cores)
     torch.cuda.synchronize()
     return o, sT
 
@@ -56,12 +59,12 @@ def test_inside_the_domain_nothing_is_reported(dtype, tol):
     assert norm_max_err(f64(sT), s_ref) <= tol
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 @pytest.mark.parametrize("s", [2.7, 4.0, 8.0])
-def test_past_the_domain_is_reported_and_finite(dtype, s):
-    """31 s > 80 nats: KDA_WARN_DOMAIN, finite outputs; the error against the
-    oracle is recorded in the assertion message of the finiteness check."""
-    x = _inputs(s, dtype)
+def test_past_the_domain_is_reported_and_finite(s):
+    """Tensor-core path, 31 s > 80 nats: KDA_WARN_DOMAIN, finite outputs; the
+    error against the oracle is recorded in the assertion message of the
+    finiteness check."""
+    x = _inputs(s, "bf16")
     o, sT = _run_fwd(x)
     with pytest.raises(kda.KdaError) as e:
         kda.kda_check()
@@ -70,6 +73,38 @@ def test_past_the_domain_is_reported_and_finite(dtype, s):
     o_ref, s_ref = _oracle(x)
     err = norm_max_err(f64(o).reshape(o_ref.shape), o_ref)
     assert torch.isfinite(o).all() and torch.isfinite(sT).all(), f"s = {s}: error {err:.3e}"
+
+
+@pytest.mark.parametrize("dtype,tol", [("fp32", 1e-4), ("bf16", 1e-4)])
+@pytest.mark.parametrize("s", [2.7, 8.0, 30.0])
+def test_cuda_core_path_has_no_domain_limit(dtype, tol, s):
+    """The 16-row segmentation of the CUDA-core kernel keeps every factor at
+    most 1: gates far past the tensor-core path's edge are as exact as weak
+    ones, with nothing reported (bf16 inputs through KDA_MODE_CUDA_CORES are
+    computed in fp32 too)."""
+    x = _inputs(s, dtype, T=200)
+    o, sT = _run_fwd(x, cuda_cores=True)
+    kda.kda_check()
+    o_ref, s_ref = _oracle(x)
+    assert norm_max_err(f64(o).reshape(o_ref.shape), o_ref) <= tol
+    assert norm_max_err(f64(sT), s_ref) <= tol
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_cuda_core_path_mixed_chunks(dtype):
+    """One sequence whose odd chunks decay 8 nats per token and whose even
+    chunks carry the recipe's gates: the CUDA-core kernel takes the middle-row
+    split for some chunks and the 16-row segmentation for the others, with one
+    state carried across; both stay within the fp32 bar."""
+    w = Workload("domain", "dense", 1, 300, 2, 128, 128, dtype, -3.0, 0.05, seed=702)
+    x = make_inputs(w, "cpu")
+    strong = (torch.arange(300) // 64) % 2 == 1
+    x["log_alpha"][:, strong] = -8.0
+    o, sT = _run_fwd(x, cuda_cores=True)
+    kda.kda_check()
+    o_ref, s_ref = _oracle(x)
+    assert norm_max_err(f64(o).reshape(o_ref.shape), o_ref) <= 1e-4
+    assert norm_max_err(f64(sT), s_ref) <= 1e-4
 
 
 def test_backward_and_dplr_report_the_domain_too():
