@@ -858,6 +858,9 @@ struct ScanParams {
     long long timeout_cycles;
     const unsigned* ready;   // cooperative schedule: wait for ready[record] before loading it
     int no_erase;            // KDA_MODE_NO_ERASE: Y = beta V (no X term)
+    int items;               // scan kernel: (sequence, head, value slice) items over its CTAs
+    int* next_item;          // packed batches: items past the first gridDim.x are claimed from this
+                             // counter (zero before the launch); else strided over the CTAs
 };
 
 // Shared memory of the scan kernel: two 72 KB slots, each holding one record
@@ -940,9 +943,10 @@ __device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost,
     }
 }
 
-// One CTA per (sequence, head, NV value columns).  Thread (lane lt < d_k,
+// One (sequence, head, NV value columns) item at a time: items bid0,
+// bid0 + bid_step, ... (or claimed from p.next_item).  Thread (lane lt < d_k,
 // warpgroup wg) keeps S[lt][16 wg .. 16 wg + 16) of the state in registers.
-// Per chunk c (slot c % 2):
+// Per chunk c (slot c % 2, c counted over all of the CTA's items):
 //   S <- diag(e^G_last(c-1)) S + W(c-1)      W = Z Y of the chunk before, from TMEM
 //   S operand (fp16) -> smem;  MMA [O ; X] = [Qh ; Kh] S  -> TMEM buffer c % 2
 //   Y = diag(beta) (V - X) -> smem (lanes 64..127), while lanes 0..63 store
@@ -954,7 +958,7 @@ __device__ __forceinline__ void store_o_tile(uint32_t t_acc, unsigned char* ost,
 // one thread complete in issue order).
 template <typename TO, int DK, int VK>
 __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensorMap& tmo, const ScanParams& p,
-                                          int bid)
+                                          int bid0, int bid_step, int n_items)
 {
     const bool no_erase = VK == kVarNoErase || (VK == kVarAny && p.no_erase);   // layer variant
     using PL = ScanPlan<DK>;
@@ -977,44 +981,7 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
     const int lt = tid & 127;
     const int wg = tid >> 7;
     const int nslice = p.DV / NV;
-    const int slice = bid % nslice;
-    const int h = (bid / nslice) % p.H;
-    const int rank = bid / (nslice * p.H);
     const int H = p.H, DV = p.DV;
-    int n, tok0, len;
-    long long j0;
-    if (p.cu) {
-        n = p.order[rank];
-        tok0 = p.cu[n];
-        len = max(0, p.cu[n + 1] - tok0);
-        j0 = p.choff[n];
-    } else {
-        n = rank;
-        tok0 = n * p.T;
-        len = p.T;
-        j0 = (long long)n * p.rs - p.rc0;
-    }
-    const int col0 = slice * NV;
-    int nchunks = (len + C - 1) / C;
-    if ((long long)tok0 + len > p.tokens || tok0 < 0) {
-        if (tid == 0 && p.c_begin == 0) flag_bad_input();
-        nchunks = 0;
-        len = 0;
-    }
-    // this launch's part of the sequence: chunks [c_begin, c_end)
-    if (p.c_begin > 0 && p.c_begin >= nchunks) return;   // ended in an earlier launch; its state is final
-    {
-        const int lo = min(p.c_begin, nchunks), hi = min(p.c_end, nchunks);
-        tok0 += lo * C;
-        len = max(0, len - lo * C);
-        j0 += lo;
-        nchunks = max(0, hi - lo);
-    }
-    if (nchunks > 0 && (j0 < 0 || j0 + nchunks > p.max_chunks)) {   // records outside the buffer
-        if (tid == 0) flag_bad_input();
-        nchunks = 0;
-        len = 0;
-    }
     const float* s_src = p.s_in;
 
     if (tid == 0) {
@@ -1040,31 +1007,30 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
     constexpr uint32_t kBytesA = R::Z + C * NV * 2;     // [Qh ; Kh] tile + V tile
     constexpr uint32_t kBytesB = R::BYTES - R::Z;       // Z, PT, e^G_last, beta
 
+    // items bid0, bid0 + bid_step, ... (one (sequence, head, value slice) each):
+    // the barriers and TMEM carry over, their phases counted across items
+    int gbase = 0;                     // chunks this CTA ran before the current item
+    int xbase = 0;                     // mb_x completions before the current item
+    int slice = 0, h = 0, n = 0, tok0 = 0, len = 0, col0 = 0, nchunks = 0;
+    long long j0 = 0;
+
     auto rec_of = [&](int cc) { return p.rec + ((size_t)(j0 + cc) * H + h) * R::BYTES; };
+    // chunk cc of the current item is chunk gbase + cc of this CTA: its slot
+    // and the parities of the slot's barriers follow that count
     auto issue_a = [&](int cc) {
-        unsigned char* slot = sm + (cc & 1) * PL::SLOT;
+        const int sl = (gbase + cc) & 1;
+        unsigned char* slot = sm + sl * PL::SLOT;
         if (p.ready && !wait_ready(p.ready + (size_t)(j0 + cc) * H + h, abort_flag, p.timeout_cycles)) return;
-        mbar_expect_tx(mb_a + (cc & 1), kBytesA);
-        bulk_load(slot, rec_of(cc), R::Z, mb_a + (cc & 1));
-        tma_load_3d(slot + PL::VOFF, &tmv, mb_a + (cc & 1), col0, h, tok0 + cc * C);
+        mbar_expect_tx(mb_a + sl, kBytesA);
+        bulk_load(slot, rec_of(cc), R::Z, mb_a + sl);
+        tma_load_3d(slot + PL::VOFF, &tmv, mb_a + sl, col0, h, tok0 + cc * C);
     };
     auto issue_b = [&](int cc) {
-        unsigned char* slot = sm + (cc & 1) * PL::SLOT;
-        mbar_expect_tx(mb_b + (cc & 1), kBytesB);
-        bulk_load(slot + R::Z, rec_of(cc) + R::Z, kBytesB, mb_b + (cc & 1));
+        const int sl = (gbase + cc) & 1;
+        unsigned char* slot = sm + sl * PL::SLOT;
+        mbar_expect_tx(mb_b + sl, kBytesB);
+        bulk_load(slot + R::Z, rec_of(cc) + R::Z, kBytesB, mb_b + sl);
     };
-
-    // state rows of this thread
-    float S[16];
-    {
-        const bool own = lt < DK && s_src;
-        const float* src = own ? s_src + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg : nullptr;
-#pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-            const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-            S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
-        }
-    }
 
     // thread 0 issues the MMAs; thread kIssuer every copy (record refills, V
     // tiles, output stores)
@@ -1073,150 +1039,223 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
     unsigned pend = 0;                 // bits: 0-1 mb_a[slot], 2-3 mb_b[slot], 4 mb_x, 5 mb_w
     uint32_t apar = 0u, bpar = 0u;     // bit i: phase parity of the pending load of slot i
     int xph = 0, wph = 0;              // commits issued to mb_x / mb_w
-    int c = 0;
-    if (issuer)
-        for (int cc = 0; cc < 2 && cc < nchunks; ++cc) {
-            issue_a(cc);
-            issue_b(cc);
+    // packed batches: thread 0 claims the item after the current one when the
+    // current one starts (the atomic's latency overlaps the item) and hands it
+    // to the CTA after it
+    int* const claim_sh = reinterpret_cast<int*>(tmem_slot + 2);
+    int claimed = 0;
+    auto advance = [&](int cur) {   // by every thread, after an item
+        if (!p.next_item) return cur + bid_step;
+        if (tid == 0) *claim_sh = claimed;
+        __syncthreads();
+        const int nb = *claim_sh;
+        __syncthreads();   // every thread has read the claim before thread 0 writes the next
+        return nb;
+    };
+    for (int bid = bid0; bid < n_items; bid = advance(bid)) {
+        if (p.next_item && tid == 0) claimed = bid_step + atomicAdd(p.next_item, 1);
+        slice = bid % nslice;
+        h = (bid / nslice) % p.H;
+        const int rank = bid / (nslice * p.H);
+        if (p.cu) {
+            n = p.order[rank];
+            tok0 = p.cu[n];
+            len = max(0, p.cu[n + 1] - tok0);
+            j0 = p.choff[n];
+        } else {
+            n = rank;
+            tok0 = n * p.T;
+            len = p.T;
+            j0 = (long long)n * p.rs - p.rc0;
         }
-    for (int cc = 0; cc < 2 && cc < nchunks; ++cc) pend |= (1u | 4u) << cc;
+        col0 = slice * NV;
+        nchunks = (len + C - 1) / C;
+        if ((long long)tok0 + len > p.tokens || tok0 < 0) {
+            if (tid == 0 && p.c_begin == 0) flag_bad_input();
+            nchunks = 0;
+            len = 0;
+        }
+        // this launch's part of the sequence: chunks [c_begin, c_end)
+        if (p.c_begin > 0 && p.c_begin >= nchunks) continue;   // ended in an earlier launch; its state is final
+        {
+            const int lo = min(p.c_begin, nchunks), hi = min(p.c_end, nchunks);
+            tok0 += lo * C;
+            len = max(0, len - lo * C);
+            j0 += lo;
+            nchunks = max(0, hi - lo);
+        }
+        if (nchunks > 0 && (j0 < 0 || j0 + nchunks > p.max_chunks)) {   // records outside the buffer
+            if (tid == 0) flag_bad_input();
+            nchunks = 0;
+            len = 0;
+        }
+        // state rows of this thread
+        float S[16];
+        {
+            const bool own = lt < DK && s_src;
+            const float* src = own ? s_src + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg : nullptr;
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                const float4 v4 = own ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
+            }
+        }
 
-    float eglp = 1.f;                  // e^G_last of the previous chunk, key channel lt
-    int Lprev = 0;
-    for (c = 0; c < nchunks; ++c) {
-        const int b = c & 1;
-        unsigned char* slot = sm + b * PL::SLOT;
-        const uint32_t t_XO = tmem + 64 * b;
-        const int L = min(C, len - c * C);
-        KDA_PHASE(0);
+        int c = 0;
+        if (issuer)
+            for (int cc = 0; cc < 2 && cc < nchunks; ++cc) {
+                issue_a(cc);
+                issue_b(cc);
+            }
+        for (int cc = 0; cc < 2 && cc < nchunks; ++cc) {
+            const int sl = (gbase + cc) & 1;
+            const uint32_t par = (uint32_t)(((gbase + cc) >> 1) & 1);
+            pend |= (1u | 4u) << sl;
+            apar = (apar & ~(1u << sl)) | (par << sl);
+            bpar = (bpar & ~(1u << sl)) | (par << sl);
+        }
 
-        // ---- state of chunk c - 1, then its fp16 operand (row = value column)
-        if (c > 0) {
-            KDA_WAIT_OR_EXIT(mb_w, 32u, (c - 1) & 1);
+        float eglp = 1.f;                  // e^G_last of the previous chunk, key channel lt
+        int Lprev = 0;
+        for (c = 0; c < nchunks; ++c) {
+            const int g = gbase + c;   // this CTA's chunk count
+            const int b = g & 1;
+            unsigned char* slot = sm + b * PL::SLOT;
+            const uint32_t t_XO = tmem + 64 * b;
+            const int L = min(C, len - c * C);
+            KDA_PHASE(0);
+
+            // ---- state of chunk c - 1, then its fp16 operand (row = value column)
+            if (c > 0) {
+                KDA_WAIT_OR_EXIT(mb_w, 32u, (g - 1) & 1);
+                tc_fence_after();
+                float w[16];
+                tmem_ld16(t_W + lane_off + q_off, w);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
+            }
+            if (lt < DK) st_row_h16(Sop, lt, 16 * wg, DK, S);
+            fence_proxy_async();
+            tc_fence_before();
+            KDA_WAIT_OR_EXIT(mb_a + b, 1u << b, (apar >> b) & 1u);
+            KDA_PHASE(1);
+
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)    // [O ; X] = [Qh ; Kh] S
+                    umma_f16(t_XO, kdesc(slot + R::QK, kk, 128 * 128), mn_desc(Sop, kk, DK), kI, kk > 0);
+                umma_commit(mb_x);
+            }
+            ++xph;
+            pend |= 16u;
+            KDA_WAIT_OR_EXIT(mb_x, 16u, (xbase + c) & 1);
+            tc_fence_after();
+            // chunk c - 1's PT Y has completed as well: refill the other slot's
+            // second part with chunk c + 1
+            if (c >= 1 && c + 1 < nchunks) {
+                if (issuer) {
+                    fence_proxy_async();
+                    issue_b(c + 1);
+                }
+                pend |= 4u << (b ^ 1);
+                bpar = (bpar & ~(1u << (b ^ 1))) | ((uint32_t)(((g + 1) >> 1) & 1) << (b ^ 1));
+            }
+            KDA_WAIT_OR_EXIT(mb_b + b, 4u << b, (bpar >> b) & 1u);
+            KDA_PHASE(2);
+
+            // ---- Y = beta (V - X) (lanes 64..127) | o rows of chunk c - 1 (lanes 0..63)
+            {
+                const float* egl = reinterpret_cast<const float*>(slot + R::EGL);
+                const float* beta = reinterpret_cast<const float*>(slot + R::BETA);
+                eglp = lt < DK ? egl[lt] : 1.f;
+                if (lt >= C) {
+                    const int s = lt - C;
+                    float x16[16];
+                    tmem_ld16(t_XO + lane_off + q_off, x16);
+                    tmem_wait_ld();
+                    const float bs = beta[s];
+                    const unsigned char* vt = slot + PL::VOFF;
+                    uint4 vr[2];
+                    vr[0] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg, C));
+                    vr[1] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg + 8, C));
+                    float y[16];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const float2 f2 = __bfloat1622float2(v2[w]);
+                            const int jj = 8 * u + 2 * w;
+                            y[jj] = bs * (f2.x - (no_erase ? 0.f : x16[jj]));
+                            y[jj + 1] = bs * (f2.y - (no_erase ? 0.f : x16[jj + 1]));
+                        }
+                    }
+                    st_row_h16(Yb, s, 16 * wg, C, y);
+                } else if (c > 0) {
+                    const int tk = tok0 + (c - 1) * C;
+                    store_o_tile<TO>(tmem + 64 * (b ^ 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
+                                     ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            __syncthreads();
+            KDA_PHASE(3);
+            if (issuer && c + 2 < nchunks) {            // X MMA done, V consumed: refill part one
+                fence_proxy_async();
+                issue_a(c + 2);
+            }
+
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)     // W = Z Y
+                    umma_f16(t_W, kdesc(slot + R::Z, kk, DK * 128), mn_desc(Yb, kk, C), kI, kk > 0);
+                umma_commit(mb_w);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)     // O += PT Y  (rows 64..127: discarded)
+                    umma_f16(t_XO, kdesc(slot + R::PT, kk, C * 128), mn_desc(Yb, kk, C), kI, 1);
+            }
+            ++wph;
+            pend |= 32u;
+            if (c + 2 < nchunks) {
+                pend |= 1u << b;
+                apar = (apar & ~(1u << b)) | ((uint32_t)(((g + 2) >> 1) & 1) << b);
+            }
+            Lprev = L;
+            KDA_PHASE(4);
+        }
+
+        if (nchunks > 0) {
+            // W and O of the last chunk: one more commit covers every MMA issued
+            if (tid == 0) umma_commit(mb_x);
+            ++xph;
+            pend |= 16u;
+            KDA_WAIT_OR_EXIT(mb_x, 16u, (xbase + nchunks) & 1);
+            pend &= ~32u;
             tc_fence_after();
             float w[16];
             tmem_ld16(t_W + lane_off + q_off, w);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
-        }
-        if (lt < DK) st_row_h16(Sop, lt, 16 * wg, DK, S);
-        fence_proxy_async();
-        tc_fence_before();
-        KDA_WAIT_OR_EXIT(mb_a + b, 1u << b, (apar >> b) & 1u);
-        KDA_PHASE(1);
-
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)    // [O ; X] = [Qh ; Kh] S
-                umma_f16(t_XO, kdesc(slot + R::QK, kk, 128 * 128), mn_desc(Sop, kk, DK), kI, kk > 0);
-            umma_commit(mb_x);
-        }
-        ++xph;
-        pend |= 16u;
-        KDA_WAIT_OR_EXIT(mb_x, 16u, c & 1);
-        tc_fence_after();
-        // chunk c - 1's PT Y has completed as well: refill the other slot's
-        // second part with chunk c + 1
-        if (c >= 1 && c + 1 < nchunks) {
-            if (issuer) {
-                fence_proxy_async();
-                issue_b(c + 1);
-            }
-            pend |= 4u << (b ^ 1);
-            bpar = (bpar & ~(1u << (b ^ 1))) | ((uint32_t)(((c + 1) >> 1) & 1) << (b ^ 1));
-        }
-        KDA_WAIT_OR_EXIT(mb_b + b, 4u << b, (bpar >> b) & 1u);
-        KDA_PHASE(2);
-
-        // ---- Y = beta (V - X) (lanes 64..127) | o rows of chunk c - 1 (lanes 0..63)
-        {
-            const float* egl = reinterpret_cast<const float*>(slot + R::EGL);
-            const float* beta = reinterpret_cast<const float*>(slot + R::BETA);
-            eglp = lt < DK ? egl[lt] : 1.f;
-            if (lt >= C) {
-                const int s = lt - C;
-                float x16[16];
-                tmem_ld16(t_XO + lane_off + q_off, x16);
-                tmem_wait_ld();
-                const float bs = beta[s];
-                const unsigned char* vt = slot + PL::VOFF;
-                uint4 vr[2];
-                vr[0] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg, C));
-                vr[1] = *reinterpret_cast<const uint4*>(vt + swh_off(s, 16 * wg + 8, C));
-                float y[16];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const float2 f2 = __bfloat1622float2(v2[w]);
-                        const int jj = 8 * u + 2 * w;
-                        y[jj] = bs * (f2.x - (no_erase ? 0.f : x16[jj]));
-                        y[jj + 1] = bs * (f2.y - (no_erase ? 0.f : x16[jj + 1]));
-                    }
-                }
-                st_row_h16(Yb, s, 16 * wg, C, y);
-            } else if (c > 0) {
-                const int tk = tok0 + (c - 1) * C;
-                store_o_tile<TO>(tmem + 64 * (b ^ 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
+            if (lt < C) {
+                const int tk = tok0 + (nchunks - 1) * C;
+                store_o_tile<TO>(tmem + 64 * ((gbase + nchunks - 1) & 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
                                  ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
             }
         }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        KDA_PHASE(3);
-        if (issuer && c + 2 < nchunks) {            // X MMA done, V consumed: refill part one
-            fence_proxy_async();
-            issue_a(c + 2);
+        if (p.s_out && lt < DK) {
+            float* dst = p.s_out + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg;
+#pragma unroll
+            for (int j = 0; j < 16; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
 
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)     // W = Z Y
-                umma_f16(t_W, kdesc(slot + R::Z, kk, DK * 128), mn_desc(Yb, kk, C), kI, kk > 0);
-            umma_commit(mb_w);
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)     // O += PT Y  (rows 64..127: discarded)
-                umma_f16(t_XO, kdesc(slot + R::PT, kk, C * 128), mn_desc(Yb, kk, C), kI, 1);
-        }
-        ++wph;
-        pend |= 32u;
-        if (c + 2 < nchunks) {
-            pend |= 1u << b;
-            apar = (apar & ~(1u << b)) | ((uint32_t)(((c + 2) >> 1) & 1) << b);
-        }
-        Lprev = L;
-        KDA_PHASE(4);
-    }
-
-    if (nchunks > 0) {
-        // W and O of the last chunk: one more commit covers every MMA issued
-        if (tid == 0) umma_commit(mb_x);
-        ++xph;
-        pend |= 16u;
-        KDA_WAIT_OR_EXIT(mb_x, 16u, nchunks & 1);
-        pend &= ~32u;
-        tc_fence_after();
-        float w[16];
-        tmem_ld16(t_W + lane_off + q_off, w);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) S[j] = fmaf(eglp, S[j], w[j]);
-        if (lt < C) {
-            const int tk = tok0 + (nchunks - 1) * C;
-            store_o_tile<TO>(tmem + 64 * ((nchunks - 1) & 1) + lane_off + q_off, Ost, &tmo, p.o, tk, h, col0,
-                             ((size_t)tk * H + h) * DV + col0, (size_t)H * DV, Lprev, lt, wg, issuer);
-        }
-    }
-    if (p.s_out && lt < DK) {
-        float* dst = p.s_out + (((size_t)n * H + h) * DK + lt) * DV + col0 + 16 * wg;
-#pragma unroll
-        for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        gbase += nchunks;
+        xbase += nchunks > 0 ? nchunks + 1 : 0;
     }
 
 finish:
@@ -1257,7 +1296,7 @@ __global__ void __launch_bounds__(NT, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
                   const ScanParams p)
 {
-    scan_body<TO, DK, VK>(tmv, tmo, p, blockIdx.x);
+    scan_body<TO, DK, VK>(tmv, tmo, p, blockIdx.x, gridDim.x, p.items);
 }
 
 // Cooperative schedule: CTAs [0, n_scan) scan, the others prep; the scan
@@ -1270,7 +1309,8 @@ chunk_coop_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                   const __grid_constant__ CUtensorMap tmo, const PrepParams pp, const ScanParams sp, int n_scan)
 {
     // the scan of a per-head-gate call is the plain layer's
-    if ((int)blockIdx.x < n_scan) scan_body<TO, DK, VK == kVarHeadGate ? kVarPlain : VK>(tmv, tmo, sp, blockIdx.x);
+    if ((int)blockIdx.x < n_scan)
+        scan_body<TO, DK, VK == kVarHeadGate ? kVarPlain : VK>(tmv, tmo, sp, blockIdx.x, n_scan, n_scan);
     else prep_body<DK, VK>(tmq, tmk, tmg, pp, blockIdx.x - n_scan, gridDim.x - n_scan);
 }
 
@@ -1297,8 +1337,10 @@ constexpr int kIndexThreads = 1024;
 constexpr int kSmemKeys = 16384;
 
 __global__ void __launch_bounds__(kIndexThreads)
-varlen_index_kernel(const int32_t* cu, int nseq, int32_t* choff, int32_t* order, unsigned long long* gkeys)
+varlen_index_kernel(const int32_t* cu, int nseq, int32_t* choff, int32_t* order, unsigned long long* gkeys,
+                    int* work)
 {
+    if (threadIdx.x == 0) *work = 0;
     __shared__ int warp_tot[32];
     extern __shared__ unsigned long long skeys[];
     const int tid = threadIdx.x;
@@ -1414,7 +1456,7 @@ constexpr int kMaxBlocks = 8;
 
 // Offsets (bytes) of the parts of a call's workspace.
 struct WsLayout {
-    size_t choff, order, keys, carry, flags, rec, bytes;
+    size_t choff, order, work, keys, carry, flags, rec, bytes;
     long long max_chunks;
 };
 
@@ -1432,6 +1474,8 @@ static WsLayout ws_layout(int nseq, int T, long long tokens, int H, int dv, bool
     off += varlen ? align1k(((size_t)nseq + 1) * 4) : 0;
     w.order = off;
     off += varlen ? align1k((size_t)nseq * 4) : 0;
+    w.work = off;                                          // the packed scan's next-item counter
+    off += varlen ? 1024 : 0;
     w.keys = off;
     off += (varlen && npad > kSmemKeys) ? align1k((size_t)npad * 8) : 0;
     w.carry = off;                                         // state between blocks when no final state is kept
@@ -1518,7 +1562,8 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         err = cudaFuncSetAttribute(varlen_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 8);
         if (err == cudaSuccess) {
             varlen_index_kernel<<<1, kIndexThreads, smem, stream>>>(cu, nseq, choff, order,
-                                                                    reinterpret_cast<unsigned long long*>(ws + L.keys));
+                                                                    reinterpret_cast<unsigned long long*>(ws + L.keys),
+                                                                    reinterpret_cast<int*>(ws + L.work));
             err = cudaGetLastError();
         }
         if (err != cudaSuccess) {
@@ -1584,7 +1629,12 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         sp.s_in = b == 0 ? s0 : carry;
         sp.s_out = (b == nblocks - 1) ? sT : carry;
         if (scan_ctas <= 0) return cudaSuccess;
-        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
+        // one CTA per item; beyond 4 items per SM, one persistent CTA per SM
+        // takes items in rank order (packed batches: claimed from a counter)
+        const long long grid = scan_ctas > 4LL * nsm ? nsm : scan_ctas;
+        sp.items = (int)scan_ctas;
+        sp.next_item = (cu && grid < scan_ctas) ? reinterpret_cast<int*>(ws + L.work) : nullptr;
+        sk<<<(unsigned)grid, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
         return cudaGetLastError();
     };
 
@@ -1764,7 +1814,11 @@ static cudaError_t run_noalloc(const void* q, const void* k, const void* v, cons
         sp.s_in = b == 0 ? s0 : carry;
         sp.s_out = b == nblocks - 1 ? sT : carry;
         if (scan_ctas <= 0) return cudaSuccess;
-        sk<<<(unsigned)scan_ctas, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
+        // one CTA per item; beyond 4 items per SM, one persistent CTA per SM
+        // takes every gridDim.x-th item
+        const long long grid = scan_ctas > 4LL * nsm ? nsm : scan_ctas;
+        sp.items = (int)scan_ctas;
+        sk<<<(unsigned)grid, NT, ScanPlan<DK>::BYTES, stream>>>(tv, to, sp);
         return cudaGetLastError();
     };
 

@@ -101,3 +101,25 @@ def test_cooperative_schedule_bit_identical(B, T, H, d):
     o3, s3 = _call_coop(g, output_final_state=False, o_dtype=torch.bfloat16)
     o4, _ = _call(g, 1, output_final_state=False, o_dtype=torch.bfloat16)
     assert s3 is None and torch.equal(o3, o4)
+
+
+@pytest.mark.parametrize("d,H", [(128, 32), (64, 64)])
+def test_persistent_scan_matches_one_cta_per_item(d, H):
+    """A dense batch of more than four scan items per SM (B = 10: 640 items of
+    64 value columns) runs prep then scan, with one
+    persistent scan CTA per SM taking every gridDim.x-th item: each sequence's
+    results are bit-identical to the same sequence alone (a one-launch
+    schedule with one scan CTA per item); one pair of heads is checked
+    against the oracle."""
+    x, g = _inputs(10, 130, H, d, seed=910)
+    o, sT = _call(g, 0)
+    for b in (0, 3, 9):
+        one = {k: (None if v is None else v[b:b + 1].contiguous()) for k, v in g.items()}
+        o1, s1 = _call(one, 0)
+        assert torch.equal(o[b:b + 1], o1) and torch.equal(sT[b:b + 1], s1)
+    b, hs = 9, [0, H - 1]
+    flat = lambda t: f64(t[b, :, hs])
+    o_ref, s_ref = oracle.recurrence(flat(x["q"]), flat(x["k"]), flat(x["v"]), f64(x["beta"][b, :, hs]),
+                                     flat(x["log_alpha"]), np.array([0, 130]), f64(x["initial_state"][b:b + 1, hs]))
+    assert norm_max_err(f64(o[b, :, hs]), o_ref) <= TOL_BF16
+    assert norm_max_err(f64(sT[b:b + 1, hs]), s_ref) <= TOL_BF16
