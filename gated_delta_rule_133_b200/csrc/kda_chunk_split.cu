@@ -1089,6 +1089,33 @@ __device__ __forceinline__ void scan_body(const CUtensorMap& tmv, const CUtensor
             nchunks = 0;
             len = 0;
         }
+        // records written earlier (not the cooperative hand-off): the first
+        // two records and V tiles of item bid + bid_step, which some CTA takes
+        // about one round of items later, into L2 (the address loads overlap
+        // this item's first copies)
+        if (!p.ready && tid == 64 && bid + bid_step < n_items) {
+            const int nb = bid + bid_step;
+            const int sl2 = nb % nslice, h2 = (nb / nslice) % p.H, r2 = nb / (nslice * p.H);
+            int tk2, ln2;
+            long long jj2;
+            if (p.cu) {
+                const int n2 = p.order[r2];
+                tk2 = p.cu[n2];
+                ln2 = max(0, p.cu[n2 + 1] - tk2);
+                jj2 = p.choff[n2];
+            } else {
+                tk2 = r2 * p.T;
+                ln2 = p.T;
+                jj2 = (long long)r2 * p.rs - p.rc0;
+            }
+            const int lo2 = min(p.c_begin, (ln2 + C - 1) / C);
+            const int nc2 = min(2, max(0, min(p.c_end, (ln2 + C - 1) / C) - lo2));
+            if (tk2 >= 0 && (long long)tk2 + ln2 <= p.tokens && jj2 + lo2 >= 0 && jj2 + lo2 + nc2 <= p.max_chunks)
+                for (int cc = 0; cc < nc2; ++cc) {
+                    bulk_prefetch_l2(p.rec + ((size_t)(jj2 + lo2 + cc) * H + h2) * R::BYTES, (uint32_t)R::BYTES);
+                    tma_prefetch_3d(&tmv, sl2 * NV, h2, tk2 + (lo2 + cc) * C);
+                }
+        }
         // state rows of this thread
         float S[16];
         {
